@@ -1,0 +1,201 @@
+"""Python access to the plain C oracle (``fps_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and bench.py's
+CPU-baseline / reference legs may import this package; the CUDA library and
+its binding never do.  The oracle is built with gcc, ``-O2 -ffp-contract=off``
+and no fast-math, so every float32 operation is rounded on its own.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fps_oracle.c")
+_LIB = os.path.join(_HERE, "libfps_oracle.so")
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fexcess-precision=standard",
+          "-fPIC", "-shared"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library next to its source; return its path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def bind(path: str):
+    """Load an oracle shared library at ``path`` and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.fpso_dist.restype = ctypes.c_float
+    lib.fpso_dist.argtypes = [P, P]
+    lib.fpso_fps.argtypes = [P, P, I, I, P, P, P]
+    lib.fpso_assign.argtypes = [P, P, I, P, P, I, P]
+    lib.fpso_knn.argtypes = [P, P, I, P, P, I, I, P]
+    lib.fpso_lloyd.argtypes = [P, P, I, I, P, I, I, I, P, P]
+    lib.fpso_pool_voronoi.argtypes = [P, I, P, I, I, P, P, P]
+    lib.fpso_pool_knn.argtypes = [P, I, I, I, I, P, P, P]
+    lib.fpso_tokenize.argtypes = [P, P, I, P, I, P, I, I, I, I, I, P, P, P, P, P, P]
+    for f in (lib.fpso_fps, lib.fpso_assign, lib.fpso_knn, lib.fpso_lloyd,
+              lib.fpso_pool_voronoi, lib.fpso_pool_knn, lib.fpso_tokenize):
+        f.restype = I
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = bind(build())
+    return _lib
+
+
+class use_library:
+    """Context manager: route the wrappers below through another oracle build
+    (the mutation tests compile altered copies of the oracle to check that the
+    pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self._saved = _lib
+        _lib = bind(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self._saved
+        return False
+
+
+def _f32(a, shape_tail=None):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    if shape_tail is not None:
+        a = a.reshape((-1,) + tuple(shape_tail))
+    return a
+
+
+def _i64(a):
+    return np.ascontiguousarray(a, dtype=np.int64)
+
+
+def _i32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments")
+
+
+def dist(p, c) -> np.float32:
+    """The float32 squared 4D distance the oracle uses."""
+    p = _f32(p).reshape(4)
+    c = _f32(c).reshape(4)
+    return np.float32(_load().fpso_dist(_p(p), _p(c)))
+
+
+def fps(coords, offsets, K: int, start_local=None, with_sel_dist: bool = False):
+    coords, offsets = _f32(coords, (4,)), _i64(offsets)
+    B = offsets.shape[0] - 1
+    start_local = _i32(start_local)
+    idx = np.empty((B, K), np.int32)
+    sd = np.empty((B, K), np.float32) if with_sel_dist else None
+    _check(_load().fpso_fps(_p(coords), _p(offsets), B, K, _p(start_local), _p(idx), _p(sd)), "fps")
+    return (idx, sd) if with_sel_dist else idx
+
+
+def assign(coords, offsets, centroids, K: int, valid=None):
+    coords, offsets = _f32(coords, (4,)), _i64(offsets)
+    B = offsets.shape[0] - 1
+    centroids = _f32(centroids).reshape(B, K, 4)
+    tok = np.empty(coords.shape[0], np.int32)
+    _check(_load().fpso_assign(_p(coords), _p(offsets), B, _p(centroids), _p(_i32(valid)), K, _p(tok)),
+           "assign")
+    return tok
+
+
+def knn(coords, offsets, centroids, K: int, k: int, valid=None):
+    coords, offsets = _f32(coords, (4,)), _i64(offsets)
+    B = offsets.shape[0] - 1
+    centroids = _f32(centroids).reshape(B, K, 4)
+    out = np.empty((B, K, k), np.int32)
+    _check(_load().fpso_knn(_p(coords), _p(offsets), B, _p(centroids), _p(_i32(valid)), K, k, _p(out)),
+           "knn")
+    return out
+
+
+def lloyd(coords, feats, offsets, K: int, iters: int, centroids, token_id, charge_col: int = -1):
+    coords, offsets = _f32(coords, (4,)), _i64(offsets)
+    B = offsets.shape[0] - 1
+    feats = _f32(feats)
+    F = feats.shape[1] if feats.ndim == 2 else 0
+    c = _f32(centroids).reshape(B, K, 4).copy()
+    t = _i32(token_id).copy()
+    _check(_load().fpso_lloyd(_p(coords), _p(feats), F, charge_col, _p(offsets), B, K, iters, _p(c), _p(t)),
+           "lloyd")
+    return c, t
+
+
+def pool_voronoi(feats, offsets, K: int, token_id):
+    feats, offsets = _f32(feats), _i64(offsets)
+    B = offsets.shape[0] - 1
+    F = feats.shape[1]
+    pooled = np.empty((B, K, F), np.float32)
+    counts = np.empty((B, K), np.int32)
+    _check(_load().fpso_pool_voronoi(_p(feats), F, _p(offsets), B, K, _p(_i32(token_id)), _p(pooled),
+                                     _p(counts)), "pool_voronoi")
+    return pooled, counts
+
+
+def pool_knn(feats, knn_idx):
+    feats = _f32(feats)
+    knn_idx = _i32(knn_idx)
+    B, K, k = knn_idx.shape
+    F = feats.shape[1]
+    pooled = np.empty((B, K, F), np.float32)
+    counts = np.empty((B, K), np.int32)
+    _check(_load().fpso_pool_knn(_p(feats), F, B, K, k, _p(knn_idx), _p(pooled), _p(counts)), "pool_knn")
+    return pooled, counts
+
+
+def tokenize(coords, feats, offsets, K: int, assign_mode: int = 0, k: int = 0, lloyd_iters: int = 0,
+             charge_col: int = -1, start_local=None) -> dict:
+    """The whole tokenizer on one packed batch; returns a dict of numpy outputs."""
+    coords, feats, offsets = _f32(coords, (4,)), _f32(feats), _i64(offsets)
+    B = offsets.shape[0] - 1
+    P = coords.shape[0]
+    F = feats.shape[1]
+    out = {
+        "centroid_idx": np.empty((B, K), np.int32),
+        "token_id": np.empty(P, np.int32),
+        "knn_idx": np.empty((B, K, max(k, 1)), np.int32) if assign_mode == 1 else None,
+        "centroids": np.empty((B, K, 4), np.float32),
+        "pooled": np.empty((B, K, F), np.float32),
+        "counts": np.empty((B, K), np.int32),
+    }
+    rc = _load().fpso_tokenize(_p(coords), _p(feats), F, _p(offsets), B, _p(_i32(start_local)), K,
+                               assign_mode, k, lloyd_iters, charge_col, _p(out["centroid_idx"]),
+                               _p(out["token_id"]), _p(out["knn_idx"]), _p(out["centroids"]),
+                               _p(out["pooled"]), _p(out["counts"]))
+    _check(rc, "tokenize")
+    return out
+
+
+def tokenize_batch(batch) -> dict:
+    """``tokenize`` on a ``workloads.Batch``."""
+    return tokenize(batch.coords, batch.feats, batch.offsets, batch.K, batch.assign_mode, batch.k,
+                    batch.lloyd_iters, batch.charge_col, batch.start_local)

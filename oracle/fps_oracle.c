@@ -1,0 +1,365 @@
+/*
+ * CPU oracle for the batched 4D farthest-point-sampling tokenizer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * CPU-baseline / reference legs of bench.py may load or run this file.  It
+ * shares no code, header or constant with the CUDA library and never calls it.
+ *
+ * What it computes (plain loops, one event after another, no blocking):
+ *
+ *   Neptune README, "How it works", step 1 (Tokenization): farthest-point
+ *   sampling of each event down to at most num_patches (K) centroids, then
+ *   per-token pooling by nearest-centroid (Voronoi) assignment or by a kNN
+ *   gather, with optional charge-weighted Lloyd refinement of the centroids.
+ *
+ *   graphnet PR #923 "Add Neptune point-transformer backbone", "What is
+ *   added": FPSTokenizer keeps one token per pulse for small events;
+ *   components/fps.py names farthest_point_sampling(_with_assign/_with_knn)
+ *   and nearest_assign.  Review thread on the FPS `precision` argument: both
+ *   backends always compute in float32.  Review thread on the no-charge case:
+ *   unit charge when there is no charge column.
+ *
+ * Readings where the pages are silent (each one also listed in the design doc):
+ *   - distance d(i,c) = ((dx*dx + dy*dy) + dz*dz) + dt*dt in float32, each
+ *     operation rounded to nearest, no fused multiply-add (build with
+ *     -ffp-contract=off), raw (x,y,z,t), t unscaled;
+ *   - first centroid = start_local[b] (default 0, the event's first point);
+ *   - next centroid = the unselected point with the largest running minimum
+ *     distance, lowest index on ties (so with only duplicates left it is the
+ *     lowest-index unselected point and indices stay distinct);
+ *   - events with N <= K pass through: token j is point j;
+ *   - Voronoi label = nearest centroid, lowest slot on ties;
+ *   - kNN row = the k points with smallest (d, index), ascending, -1 padded;
+ *     a passthrough token's row is [its own point, -1, ...];
+ *   - pooling = plain mean of all F feature columns plus a count;
+ *   - Lloyd: c_j = sum(q_i p_i) / sum(q_i) over the cell of j (q = charge
+ *     column, or 1), the old c_j kept when the cell is empty or the weight is
+ *     <= 0; every iteration re-assigns; no Lloyd on passthrough events;
+ *   - sums (pool, Lloyd) accumulate in float64 and round once to float32.
+ *
+ * Return values: 0 on success, -1 on an argument error.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Squared 4D distance with the fixed operation order (see header comment). */
+float fpso_dist(const float *p, const float *c)
+{
+    float dx = p[0] - c[0];
+    float dy = p[1] - c[1];
+    float dz = p[2] - c[2];
+    float dt = p[3] - c[3];
+    float s = dx * dx + dy * dy;
+    s = s + dz * dz;
+    s = s + dt * dt;
+    return s;
+}
+
+static int bad_offsets(const int64_t *offsets, int B)
+{
+    if (B < 0 || offsets == NULL) return 1;
+    if (B > 0 && offsets[0] != 0) return 1;
+    for (int b = 0; b < B; ++b)
+        if (offsets[b + 1] < offsets[b]) return 1;
+    return 0;
+}
+
+/*
+ * Farthest point sampling (the greedy farthest-point recurrence).
+ * centroid_idx [B,K]: global packed indices, -1 padded.
+ * sel_dist [B,K] (optional): for slot s >= 1 the running minimum distance the
+ * s-th centroid had when it was chosen; slot 0 and passthrough slots get -1.
+ */
+int fpso_fps(const float *coords, const int64_t *offsets, int B, int K,
+             const int32_t *start_local, int32_t *centroid_idx, float *sel_dist)
+{
+    if (K < 1 || bad_offsets(offsets, B)) return -1;
+    for (int64_t e = 0; e < (int64_t)B * K; ++e) {
+        centroid_idx[e] = -1;
+        if (sel_dist) sel_dist[e] = -1.0f;
+    }
+    for (int b = 0; b < B; ++b) {
+        int64_t off = offsets[b];
+        int64_t n = offsets[b + 1] - off;
+        int32_t *out = centroid_idx + (int64_t)b * K;
+        if (n == 0) continue;
+        if (n <= K) {
+            for (int64_t j = 0; j < n; ++j) out[j] = (int32_t)(off + j);
+            continue;
+        }
+        int64_t c = start_local ? start_local[b] : 0;
+        if (c < 0 || c >= n) return -1;
+        float *dist = (float *)malloc(sizeof(float) * n);
+        unsigned char *chosen = (unsigned char *)calloc(n, 1);
+        for (int64_t i = 0; i < n; ++i) dist[i] = INFINITY;
+        for (int s = 0; s < K; ++s) {
+            out[s] = (int32_t)(off + c);
+            chosen[c] = 1;
+            if (s == K - 1) break;
+            const float *pc = coords + 4 * (off + c);
+            for (int64_t i = 0; i < n; ++i) {
+                float d = fpso_dist(coords + 4 * (off + i), pc);
+                if (d < dist[i]) dist[i] = d;
+            }
+            int64_t best = -1;
+            for (int64_t i = 0; i < n; ++i) {
+                if (chosen[i]) continue;
+                if (best < 0 || dist[i] > dist[best]) best = i;
+            }
+            if (sel_dist) sel_dist[(int64_t)b * K + s + 1] = dist[best];
+            c = best;
+        }
+        free(dist);
+        free(chosen);
+    }
+    return 0;
+}
+
+/* valid tokens of event b: valid[b] if given, else min(N, K). */
+static int64_t n_valid(const int32_t *valid, int b, int64_t n, int K)
+{
+    if (valid) return valid[b];
+    return n < K ? n : K;
+}
+
+/*
+ * Nearest-centroid (Voronoi) assignment: token_id[i] = argmin_j d(p_i, c_j)
+ * over the event's valid centroid rows, lowest slot on ties; -1 when the
+ * event has no valid centroid.
+ */
+int fpso_assign(const float *coords, const int64_t *offsets, int B,
+                const float *centroids, const int32_t *valid, int K, int32_t *token_id)
+{
+    if (K < 1 || bad_offsets(offsets, B)) return -1;
+    for (int b = 0; b < B; ++b) {
+        int64_t off = offsets[b], n = offsets[b + 1] - off;
+        int64_t nv = n_valid(valid, b, n, K);
+        if (nv < 0 || nv > K) return -1;
+        const float *cb = centroids + (int64_t)b * K * 4;
+        for (int64_t i = 0; i < n; ++i) {
+            const float *p = coords + 4 * (off + i);
+            int32_t lab = -1;
+            float best = 0.0f;
+            for (int64_t j = 0; j < nv; ++j) {
+                float d = fpso_dist(p, cb + 4 * j);
+                if (lab < 0 || d < best) {
+                    best = d;
+                    lab = (int32_t)j;
+                }
+            }
+            token_id[off + i] = lab;
+        }
+    }
+    return 0;
+}
+
+typedef struct {
+    float d;
+    int64_t i;
+} dkey;
+
+static int dkey_cmp(const void *a, const void *b)
+{
+    const dkey *x = (const dkey *)a, *y = (const dkey *)b;
+    if (x->d < y->d) return -1;
+    if (x->d > y->d) return 1;
+    return (x->i > y->i) - (x->i < y->i);
+}
+
+/*
+ * kNN gather: for each valid centroid row j of event b, the k points of the
+ * event with the smallest (d(p_i, c_j), i), ascending, as global indices;
+ * -1 padded when the event has fewer than k points; invalid rows all -1.
+ */
+int fpso_knn(const float *coords, const int64_t *offsets, int B, const float *centroids,
+             const int32_t *valid, int K, int k, int32_t *knn_idx)
+{
+    if (K < 1 || k < 1 || bad_offsets(offsets, B)) return -1;
+    for (int64_t e = 0; e < (int64_t)B * K * k; ++e) knn_idx[e] = -1;
+    for (int b = 0; b < B; ++b) {
+        int64_t off = offsets[b], n = offsets[b + 1] - off;
+        int64_t nv = n_valid(valid, b, n, K);
+        if (nv < 0 || nv > K) return -1;
+        if (n == 0) continue;
+        dkey *keys = (dkey *)malloc(sizeof(dkey) * n);
+        for (int64_t j = 0; j < nv; ++j) {
+            const float *c = centroids + ((int64_t)b * K + j) * 4;
+            for (int64_t i = 0; i < n; ++i) {
+                keys[i].d = fpso_dist(coords + 4 * (off + i), c);
+                keys[i].i = i;
+            }
+            qsort(keys, (size_t)n, sizeof(dkey), dkey_cmp);
+            int32_t *row = knn_idx + ((int64_t)b * K + j) * k;
+            for (int64_t r = 0; r < k && r < n; ++r) row[r] = (int32_t)(off + keys[r].i);
+        }
+        free(keys);
+    }
+    return 0;
+}
+
+/*
+ * Charge-weighted Lloyd refinement of events with N > K (all K rows valid).
+ * Each iteration: W_j = sum q_i, S_j = sum q_i p_i over the points labelled j
+ * (float64, point order), c_j = float(S_j / W_j) when W_j > 0, else c_j kept;
+ * then every point is re-assigned to its nearest centroid.
+ */
+int fpso_lloyd(const float *coords, const float *feats, int F, int charge_col,
+               const int64_t *offsets, int B, int K, int iters,
+               float *centroids, int32_t *token_id)
+{
+    if (K < 1 || iters < 0 || charge_col >= F || bad_offsets(offsets, B)) return -1;
+    double *W = (double *)malloc(sizeof(double) * K);
+    double *S = (double *)malloc(sizeof(double) * K * 4);
+    for (int b = 0; b < B; ++b) {
+        int64_t off = offsets[b], n = offsets[b + 1] - off;
+        if (n <= K) continue;
+        float *cb = centroids + (int64_t)b * K * 4;
+        for (int it = 0; it < iters; ++it) {
+            for (int j = 0; j < K; ++j) {
+                W[j] = 0.0;
+                for (int a = 0; a < 4; ++a) S[4 * j + a] = 0.0;
+            }
+            for (int64_t i = 0; i < n; ++i) {
+                int32_t j = token_id[off + i];
+                if (j < 0 || j >= K) {
+                    free(W);
+                    free(S);
+                    return -1;
+                }
+                double q = charge_col < 0 ? 1.0 : (double)feats[(off + i) * F + charge_col];
+                W[j] += q;
+                for (int a = 0; a < 4; ++a) S[4 * j + a] += q * (double)coords[4 * (off + i) + a];
+            }
+            for (int j = 0; j < K; ++j)
+                if (W[j] > 0.0)
+                    for (int a = 0; a < 4; ++a) cb[4 * j + a] = (float)(S[4 * j + a] / W[j]);
+            for (int64_t i = 0; i < n; ++i) {
+                const float *p = coords + 4 * (off + i);
+                int32_t lab = 0;
+                float best = fpso_dist(p, cb);
+                for (int j = 1; j < K; ++j) {
+                    float d = fpso_dist(p, cb + 4 * j);
+                    if (d < best) {
+                        best = d;
+                        lab = j;
+                    }
+                }
+                token_id[off + i] = lab;
+            }
+        }
+    }
+    free(W);
+    free(S);
+    return 0;
+}
+
+/* Voronoi mean-pool: pooled[b,j,:] = mean of features over points labelled j. */
+int fpso_pool_voronoi(const float *feats, int F, const int64_t *offsets, int B, int K,
+                      const int32_t *token_id, float *pooled, int32_t *counts)
+{
+    if (K < 1 || F < 1 || bad_offsets(offsets, B)) return -1;
+    double *sum = (double *)malloc(sizeof(double) * (size_t)K * F);
+    int64_t *cnt = (int64_t *)malloc(sizeof(int64_t) * K);
+    for (int b = 0; b < B; ++b) {
+        int64_t off = offsets[b], n = offsets[b + 1] - off;
+        for (int64_t e = 0; e < (int64_t)K * F; ++e) sum[e] = 0.0;
+        for (int j = 0; j < K; ++j) cnt[j] = 0;
+        for (int64_t i = 0; i < n; ++i) {
+            int32_t j = token_id[off + i];
+            if (j < 0) continue;
+            if (j >= K) {
+                free(sum);
+                free(cnt);
+                return -1;
+            }
+            cnt[j] += 1;
+            for (int f = 0; f < F; ++f) sum[(int64_t)j * F + f] += (double)feats[(off + i) * F + f];
+        }
+        for (int j = 0; j < K; ++j) {
+            counts[(int64_t)b * K + j] = (int32_t)cnt[j];
+            for (int f = 0; f < F; ++f)
+                pooled[((int64_t)b * K + j) * F + f] =
+                    cnt[j] ? (float)(sum[(int64_t)j * F + f] / (double)cnt[j]) : 0.0f;
+        }
+    }
+    free(sum);
+    free(cnt);
+    return 0;
+}
+
+/* kNN mean-pool: pooled[b,j,:] = mean of features over the valid row entries. */
+int fpso_pool_knn(const float *feats, int F, int B, int K, int k, const int32_t *knn_idx,
+                  float *pooled, int32_t *counts)
+{
+    if (K < 1 || F < 1 || k < 1 || B < 0) return -1;
+    double *sum = (double *)malloc(sizeof(double) * F);
+    for (int64_t r = 0; r < (int64_t)B * K; ++r) {
+        const int32_t *row = knn_idx + r * k;
+        int64_t cnt = 0;
+        for (int f = 0; f < F; ++f) sum[f] = 0.0;
+        for (int e = 0; e < k; ++e) {
+            if (row[e] < 0) continue;
+            cnt += 1;
+            for (int f = 0; f < F; ++f) sum[f] += (double)feats[(int64_t)row[e] * F + f];
+        }
+        counts[r] = (int32_t)cnt;
+        for (int f = 0; f < F; ++f) pooled[r * F + f] = cnt ? (float)(sum[f] / (double)cnt) : 0.0f;
+    }
+    free(sum);
+    return 0;
+}
+
+/*
+ * The whole tokenizer: FPS (or passthrough) -> centroids -> Voronoi labels ->
+ * Lloyd (events with N > K) -> Voronoi mean-pool, or kNN gather around the
+ * final centroids and kNN mean-pool.  token_id may be NULL in kNN mode;
+ * knn_idx is ignored in Voronoi mode.
+ */
+int fpso_tokenize(const float *coords, const float *feats, int F, const int64_t *offsets, int B,
+                  const int32_t *start_local, int K, int assign_mode, int k, int lloyd_iters,
+                  int charge_col, int32_t *centroid_idx, int32_t *token_id, int32_t *knn_idx,
+                  float *centroids, float *pooled, int32_t *counts)
+{
+    if (K < 1 || F < 1 || (assign_mode != 0 && assign_mode != 1) || lloyd_iters < 0 ||
+        charge_col >= F || bad_offsets(offsets, B))
+        return -1;
+    if (assign_mode == 1 && (k < 1 || knn_idx == NULL)) return -1;
+    if (assign_mode == 0 && token_id == NULL) return -1;
+    int64_t P = B > 0 ? offsets[B] : 0;
+    int rc = fpso_fps(coords, offsets, B, K, start_local, centroid_idx, NULL);
+    if (rc) return rc;
+    for (int64_t r = 0; r < (int64_t)B * K; ++r)
+        for (int a = 0; a < 4; ++a)
+            centroids[4 * r + a] = centroid_idx[r] >= 0 ? coords[4 * (int64_t)centroid_idx[r] + a] : 0.0f;
+    int32_t *lab = (int32_t *)malloc(sizeof(int32_t) * (P > 0 ? P : 1));
+    rc = fpso_assign(coords, offsets, B, centroids, NULL, K, lab);
+    /* passthrough events: token j is point j */
+    for (int b = 0; b < B && rc == 0; ++b) {
+        int64_t off = offsets[b], n = offsets[b + 1] - off;
+        if (n <= K)
+            for (int64_t i = 0; i < n; ++i) lab[off + i] = (int32_t)i;
+    }
+    if (rc == 0 && lloyd_iters > 0)
+        rc = fpso_lloyd(coords, feats, F, charge_col, offsets, B, K, lloyd_iters, centroids, lab);
+    if (rc == 0 && token_id)
+        memcpy(token_id, lab, sizeof(int32_t) * (size_t)P);
+    if (rc == 0 && assign_mode == 0) {
+        rc = fpso_pool_voronoi(feats, F, offsets, B, K, lab, pooled, counts);
+    } else if (rc == 0) {
+        rc = fpso_knn(coords, offsets, B, centroids, NULL, K, k, knn_idx);
+        for (int b = 0; b < B && rc == 0; ++b) {
+            int64_t off = offsets[b], n = offsets[b + 1] - off;
+            if (n > K) continue;
+            for (int64_t j = 0; j < n; ++j) {
+                int32_t *row = knn_idx + ((int64_t)b * K + j) * k;
+                row[0] = (int32_t)(off + j);
+                for (int e = 1; e < k; ++e) row[e] = -1;
+            }
+        }
+        if (rc == 0) rc = fpso_pool_knn(feats, F, B, K, k, knn_idx, pooled, counts);
+    }
+    free(lab);
+    return rc;
+}

@@ -1,0 +1,378 @@
+"""Pins for the CPU oracle: hand-worked fixtures, brute force, closed forms, invariants.
+
+None of these compare the oracle with itself or with the CUDA path.  The
+``pin_*`` functions are also re-run against deliberately broken copies of the
+oracle (``test_oracle_mutations.py``) to show each plausible slip is caught.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import bruteforce as bf
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def read_fps_fixture(name):
+    coords, meta, mode = [], {}, None
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, *rest = line.split()
+            if key == "coords":
+                mode = "coords"
+                continue
+            if key in ("N", "K", "start", "expected", "sel_dist"):
+                mode = None
+                meta[key] = rest
+                continue
+            if mode == "coords":
+                coords.append([float(v) for v in line.split()])
+    return (np.array(coords, np.float32), int(meta["K"][0]), int(meta["start"][0]),
+            np.array([int(v) for v in meta["expected"]]), np.array([float(v) for v in meta["sel_dist"]],
+                                                                    np.float32))
+
+
+FPS_FIXTURES = ["fps_collinear9.txt", "fps_hypercube16.txt", "fps_duplicates.txt"]
+
+
+# ---------------------------------------------------------------- distance
+
+def pin_dist_golden():
+    rows = np.loadtxt(os.path.join(GOLDEN, "dist_order.txt"), dtype=np.float64, comments="#")
+    for r in rows:
+        got = oracle.dist(r[0:4], r[4:8])
+        assert got == np.float32(r[8]), (r, got)
+        assert oracle.dist(r[4:8], r[0:4]) == got  # a-b = -(b-a) exactly
+
+
+def pin_dist_error_bound():
+    rng = np.random.default_rng(11)
+    for _ in range(2000):
+        p = (rng.standard_normal(4) * rng.choice([1e-3, 1.0, 100.0, 5000.0], 4)).astype(np.float32)
+        c = (rng.standard_normal(4) * rng.choice([1e-3, 1.0, 100.0, 5000.0], 4)).astype(np.float32)
+        exact = float(np.sum((p.astype(np.float64) - c.astype(np.float64)) ** 2))
+        got = float(oracle.dist(p, c))
+        # 4 subtractions, 4 products, 3 sums: relative error below 8 units of 2^-24
+        assert abs(got - exact) <= 8 * 2.0 ** -24 * exact + 1e-30, (p, c, got, exact)
+
+
+def test_dist_golden():
+    pin_dist_golden()
+
+
+def test_dist_error_bound():
+    pin_dist_error_bound()
+
+
+# ---------------------------------------------------------------- FPS
+
+def pin_fps_fixtures():
+    for name in FPS_FIXTURES:
+        pts, K, start, expected, seld = read_fps_fixture(name)
+        idx, sd = oracle.fps(pts, [0, len(pts)], K, start_local=[start], with_sel_dist=True)
+        assert idx[0].tolist() == expected.tolist(), (name, idx[0])
+        assert np.array_equal(sd[0], seld), (name, sd[0])
+
+
+def _tiny_batches():
+    for seed in range(60):
+        rng = np.random.default_rng(1000 + seed)
+        K = int(rng.integers(1, 17))
+        sizes = rng.integers(0, 65, int(rng.integers(1, 6)))
+        kw = {}
+        if seed % 3 == 1:
+            kw["dup_frac"] = 0.4
+        if seed % 3 == 2:
+            kw["grid"] = 50.0
+        b = workloads.random_batch(seed, sizes, K, **kw)
+        starts = np.array([rng.integers(0, max(int(n), 1)) for n in sizes], np.int32)
+        yield b, K, starts
+
+
+def pin_fps_bruteforce():
+    for b, K, starts in _tiny_batches():
+        got = oracle.fps(b.coords, b.offsets, K, start_local=starts)
+        want = bf.fps(b.coords, b.offsets, K, start_local=starts)
+        assert np.array_equal(got, want), (b.sizes(), K)
+
+
+def pin_fps_invariants():
+    for b, K, starts in _tiny_batches():
+        idx, sd = oracle.fps(b.coords, b.offsets, K, start_local=starts, with_sel_dist=True)
+        for e in range(b.B):
+            o0, o1 = b.offsets[e], b.offsets[e + 1]
+            n = o1 - o0
+            row = idx[e]
+            valid = row[row >= 0]
+            assert len(valid) == min(n, K)
+            assert np.all(row[len(valid):] == -1)
+            assert len(set(valid.tolist())) == len(valid)  # distinct
+            assert np.all((valid >= o0) & (valid < o1))  # inside the event
+            if n <= K:
+                assert np.array_equal(valid, np.arange(o0, o1))  # one token per pulse
+            else:
+                assert valid[0] == o0 + starts[e]
+                s = sd[e, 1:]
+                assert np.all(np.diff(s) <= 0)  # selection distance never grows
+
+
+def test_fps_fixtures():
+    pin_fps_fixtures()
+
+
+def test_fps_bruteforce():
+    pin_fps_bruteforce()
+
+
+def test_fps_invariants():
+    pin_fps_invariants()
+
+
+def test_fps_time_shift_invariance():
+    # t on a 2^-8 ns grid, |t| < 2^15 before and after the shift: every shifted
+    # value is exact in f32, so each difference (and distance) is unchanged.
+    rng = np.random.default_rng(5)
+    sizes = [300, 129, 1000]
+    b = workloads.random_batch(5, sizes, 64)
+    t = np.round(rng.uniform(0, 2 ** 14, b.P) * 256) / 256
+    b.coords[:, 3] = t.astype(np.float32)
+    base = oracle.fps(b.coords, b.offsets, 64)
+    for shift in (1024.0, -8192.25, 12345.5):
+        c2 = b.coords.copy()
+        c2[:, 3] = (t + shift).astype(np.float32)
+        assert np.array_equal((c2[:, 3].astype(np.float64) - shift), t)  # shift exact
+        assert np.array_equal(oracle.fps(c2, b.offsets, 64), base)
+
+
+def test_fps_edge_cases():
+    pts = np.random.default_rng(0).standard_normal((10, 4)).astype(np.float32)
+    # empty batch, empty event, N=1, N=K, N=K+1, K=1
+    assert oracle.fps(np.zeros((0, 4)), [0], 4).shape == (0, 4)
+    idx = oracle.fps(pts[:0], [0, 0], 4)
+    assert idx.tolist() == [[-1, -1, -1, -1]]
+    assert oracle.fps(pts[:1], [0, 1], 4).tolist() == [[0, -1, -1, -1]]
+    assert oracle.fps(pts[:4], [0, 4], 4).tolist() == [[0, 1, 2, 3]]
+    row = oracle.fps(pts[:5], [0, 5], 4)[0]
+    assert row[0] == 0 and len(set(row.tolist())) == 4
+    assert oracle.fps(pts, [0, 10], 1, start_local=[7]).tolist() == [[7]]
+    with pytest.raises(ValueError):
+        oracle.fps(pts, [0, 10], 4, start_local=[10])
+    with pytest.raises(ValueError):
+        oracle.fps(pts, [0, 6, 5], 4)
+
+
+# ---------------------------------------------------------------- assign
+
+def _centroids(b, idx):
+    return np.where(idx[..., None] >= 0, b.coords[np.maximum(idx, 0)], 0).astype(np.float32)
+
+
+def pin_assign_bruteforce():
+    for b, K, starts in _tiny_batches():
+        idx = bf.fps(b.coords, b.offsets, K, start_local=starts)
+        cents = _centroids(b, idx)
+        valid = np.minimum(b.sizes(), K).astype(np.int32)
+        got = oracle.assign(b.coords, b.offsets, cents, K, valid=valid)
+        want = bf.assign(b.coords, b.offsets, cents, valid)
+        assert np.array_equal(got, want)
+
+
+def test_assign_bruteforce():
+    pin_assign_bruteforce()
+
+
+def test_assign_invariants():
+    b = workloads.make_workload("c0")
+    idx = oracle.fps(b.coords, b.offsets, b.K)
+    cents = _centroids(b, idx)
+    tok = oracle.assign(b.coords, b.offsets, cents, b.K)
+    for e in range(b.B):
+        o0, o1 = b.offsets[e], b.offsets[e + 1]
+        # every centroid lands in its own cell (c0 has no duplicate points)
+        assert np.array_equal(tok[idx[e]], np.arange(b.K))
+        counts = np.bincount(tok[o0:o1], minlength=b.K)
+        assert counts.sum() == o1 - o0
+        # the label's distance is the minimum over all centroids
+        D = bf.pair_dist(b.coords[o0:o1], cents[e])
+        assert np.array_equal(D[np.arange(o1 - o0), tok[o0:o1]], D.min(1))
+
+
+# ---------------------------------------------------------------- kNN
+
+def pin_knn_bruteforce():
+    for b, K, starts in _tiny_batches():
+        idx = bf.fps(b.coords, b.offsets, K, start_local=starts)
+        cents = _centroids(b, idx)
+        valid = np.minimum(b.sizes(), K).astype(np.int32)
+        for k in (1, 3, 8):
+            got = oracle.knn(b.coords, b.offsets, cents, K, k, valid=valid)
+            want = bf.knn(b.coords, b.offsets, cents, valid, k)
+            assert np.array_equal(got, want)
+
+
+def test_knn_bruteforce():
+    pin_knn_bruteforce()
+
+
+def test_knn_row0_is_centroid():
+    b = workloads.make_workload("c0")
+    idx = oracle.fps(b.coords, b.offsets, b.K)
+    got = oracle.knn(b.coords, b.offsets, _centroids(b, idx), b.K, 5)
+    assert np.array_equal(got[:, :, 0], idx)
+
+
+# ---------------------------------------------------------------- pool
+
+def pin_pool_bruteforce():
+    for b, K, starts in _tiny_batches():
+        idx = bf.fps(b.coords, b.offsets, K, start_local=starts)
+        cents = _centroids(b, idx)
+        valid = np.minimum(b.sizes(), K).astype(np.int32)
+        tok = bf.assign(b.coords, b.offsets, cents, valid)
+        pooled, counts = oracle.pool_voronoi(b.feats, b.offsets, K, tok)
+        wp, wc = bf.pool_voronoi(b.feats, b.offsets, K, tok)
+        assert np.array_equal(counts, wc)
+        np.testing.assert_allclose(pooled, wp, rtol=1e-6, atol=1e-7)
+
+
+def test_pool_bruteforce():
+    pin_pool_bruteforce()
+
+
+def test_pool_closed_forms():
+    rng = np.random.default_rng(3)
+    offsets = np.array([0, 50, 50, 130])
+    tok = np.concatenate([rng.integers(0, 4, 50), rng.integers(0, 4, 80)]).astype(np.int32)
+    # constant features pool to the constant
+    f = np.full((130, 3), 2.5, np.float32)
+    pooled, counts = oracle.pool_voronoi(f, offsets, 4, tok)
+    assert np.all(pooled[counts > 0] == 2.5) and np.all(pooled[counts == 0] == 0)
+    assert counts[0].sum() == 50 and counts[1].sum() == 0 and counts[2].sum() == 80
+    # one-hot of a 2-valued feature pools to the fraction of each value
+    v = rng.integers(0, 2, 130)
+    f = np.stack([v == 0, v == 1], 1).astype(np.float32)
+    pooled, counts = oracle.pool_voronoi(f, offsets, 4, tok)
+    for e, (o0, o1) in enumerate([(0, 50), (50, 50), (50, 130)]):
+        for j in range(4):
+            m = tok[o0:o1] == j
+            if m.any():
+                assert pooled[e, j, 1] == np.float32(v[o0:o1][m].sum() / m.sum())
+    # kNN pool: counts are the number of valid entries
+    knn_idx = np.array([[[0, 1, -1], [2, -1, -1]]], np.int32)
+    f = np.arange(12, dtype=np.float32).reshape(4, 3)
+    pooled, counts = oracle.pool_knn(f, knn_idx)
+    assert counts.tolist() == [[2, 1]]
+    assert pooled[0, 0].tolist() == [1.5, 2.5, 3.5] and pooled[0, 1].tolist() == [6, 7, 8]
+
+
+# ---------------------------------------------------------------- Lloyd
+
+def pin_lloyd_closed_form():
+    rng = np.random.default_rng(7)
+    n, K = 40, 3
+    pts = (rng.standard_normal((n, 4)) * [100, 100, 100, 1000]).astype(np.float32)
+    q = rng.lognormal(0, 1, n).astype(np.float32)
+    feats = np.stack([q, rng.standard_normal(n).astype(np.float32)], 1)
+    lab = rng.integers(0, K, n).astype(np.int32)
+    cents = pts[[0, 1, 2]].copy()
+    got_c, got_t = oracle.lloyd(pts, feats, [0, n], K, 1, cents[None], lab, charge_col=0)
+    want_c = bf.lloyd_update(pts, q, lab, cents)
+    np.testing.assert_allclose(got_c[0], want_c, rtol=2e-7, atol=0)
+    # the re-assignment is the all-pairs nearest centroid of the new centroids
+    assert np.array_equal(got_t, bf.assign(pts, [0, n], got_c, [K]))
+    # unit charge (charge_col = -1) gives the plain mean of each cell
+    got_c, _ = oracle.lloyd(pts, feats, [0, n], K, 1, cents[None], lab, charge_col=-1)
+    for j in range(K):
+        np.testing.assert_allclose(got_c[0, j], pts[lab == j].astype(np.float64).mean(0), rtol=2e-7)
+
+
+def test_lloyd_closed_form():
+    pin_lloyd_closed_form()
+
+
+def test_lloyd_keeps_empty_and_nonpositive_cells():
+    rng = np.random.default_rng(8)
+    n, K = 12, 4
+    pts = rng.standard_normal((n, 4)).astype(np.float32)
+    q = np.ones(n, np.float32)
+    q[lab_neg := np.arange(4, 8)] = -1.0  # cell 1 has weight -4
+    lab = np.array([0] * 4 + [1] * 4 + [2] * 4, np.int32)  # cell 3 empty
+    cents = (np.arange(16, dtype=np.float32).reshape(4, 4) * 10)
+    got_c, _ = oracle.lloyd(pts, q[:, None], [0, n], K, 1, cents[None], lab, charge_col=0)
+    assert np.array_equal(got_c[0, 1], cents[1]) and np.array_equal(got_c[0, 3], cents[3])
+    assert not np.array_equal(got_c[0, 0], cents[0])
+    del lab_neg
+
+
+def test_lloyd_objective_nonincreasing():
+    b = workloads.random_batch(21, [600, 900], 16, charge_col=0)
+    idx = oracle.fps(b.coords, b.offsets, 16)
+    cents = _centroids(b, idx)
+    tok = oracle.assign(b.coords, b.offsets, cents, 16)
+    q = b.feats[:, 0].astype(np.float64)
+
+    def objective(c, t):
+        e = np.repeat(np.arange(b.B), b.sizes())
+        diff = b.coords.astype(np.float64) - c[e, t].astype(np.float64)
+        return float(np.sum(q * np.sum(diff * diff, 1)))
+
+    prev = objective(cents, tok)
+    for _ in range(5):
+        cents, tok = oracle.lloyd(b.coords, b.feats, b.offsets, 16, 1, cents, tok, charge_col=0)
+        cur = objective(cents, tok)
+        assert cur <= prev * (1 + 1e-6)
+        prev = cur
+
+
+def test_lloyd_skips_passthrough_events():
+    b = workloads.random_batch(4, [10, 40], 16)
+    idx = oracle.fps(b.coords, b.offsets, 16)
+    cents = _centroids(b, idx)
+    tok = oracle.assign(b.coords, b.offsets, cents, 16)
+    c2, t2 = oracle.lloyd(b.coords, b.feats, b.offsets, 16, 2, cents, tok)
+    assert np.array_equal(c2[0], cents[0]) and np.array_equal(t2[:10], tok[:10])
+
+
+# ---------------------------------------------------------------- whole tokenizer
+
+def test_tokenize_composition():
+    for mode, k, iters in ((0, 0, 0), (1, 4, 0), (0, 0, 2), (1, 6, 1)):
+        b = workloads.random_batch(30 + mode, [0, 5, 16, 17, 90, 200], 16, assign_mode=mode, k=k,
+                                   lloyd_iters=iters, charge_col=0)
+        out = oracle.tokenize_batch(b)
+        idx = bf.fps(b.coords, b.offsets, 16)
+        assert np.array_equal(out["centroid_idx"], idx)
+        valid = np.minimum(b.sizes(), 16)
+        tok = out["token_id"]
+        for e in range(b.B):
+            o0, o1 = b.offsets[e], b.offsets[e + 1]
+            n = o1 - o0
+            assert np.all(out["centroids"][e, valid[e]:] == 0)
+            if n <= 16:  # passthrough: token j is point j, pooled = own features
+                assert np.array_equal(tok[o0:o1], np.arange(n))
+                assert np.array_equal(out["pooled"][e, :n], b.feats[o0:o1])
+                assert np.all(out["counts"][e, :n] == 1) and np.all(out["counts"][e, n:] == 0)
+                if mode == 1:
+                    assert np.array_equal(out["knn_idx"][e, :n, 0], np.arange(o0, o1))
+                    assert np.all(out["knn_idx"][e, :n, 1:] == -1)
+        big = b.sizes() > 16
+        if iters == 0:
+            assert np.array_equal(out["centroids"][big], b.coords[idx[big]])
+        want_tok = bf.assign(b.coords, b.offsets, out["centroids"], valid)
+        m = np.repeat(big, b.sizes())
+        assert np.array_equal(tok[m], want_tok[m])
+        if mode == 0:
+            assert out["counts"].sum() == b.P
+            wp, wc = bf.pool_voronoi(b.feats, b.offsets, 16, tok)
+            assert np.array_equal(out["counts"], wc)
+            np.testing.assert_allclose(out["pooled"], wp, rtol=1e-6, atol=1e-7)
+        else:
+            want = bf.knn(b.coords, b.offsets, out["centroids"], valid, k)
+            assert np.array_equal(out["knn_idx"][big], want[big])
+            assert np.all(out["counts"][big] == min(k, 17))
