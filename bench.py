@@ -1,0 +1,488 @@
+#!/usr/bin/env python
+"""Benchmark of the batched 4D FPS tokenizer on B200.
+
+One step = one ``fps_tokenize`` call over one batch (binning, passthrough, FPS
+fused with the Voronoi labels, Lloyd if configured, kNN or Voronoi pooling),
+inputs resident in HBM.  The default workload is the 64-event track batch
+(N ~ lognormal(median 300, sigma 1), K = 128, Voronoi assign + mean-pool).
+
+Prints one JSON line (rank 0).  ``value`` is events/s over all GPUs; the
+per-kernel roofline uses CUDA events recorded by the library around each
+internal stage in the timed region.  ``--impl reference`` times the CPU
+oracle instead, on the host cores.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       (N > 1: launch under torch.distributed.run, one process per GPU).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+FP32_OPS_PER_EVAL = 11  # 4 sub + 4 mul + 3 add
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+SM_MAX_MHZ_NOMINAL = 1965.0
+STAGES = ["bin+passthrough", "fps_warp", "fps_cta", "fps_cluster", "lloyd", "knn+pool", "voronoi_pool"]
+STAGE_KERNELS = {0: "k_bin+k_passthrough", 1: "k_fps_warp", 2: "k_fps_block<1>", 3: "k_fps_block<16>",
+                 4: "k_lloyd_sums+k_lloyd_step", 5: "k_knn", 6: "k_pool_voronoi"}
+METRIC = "FPS+assign events/s (K=128)"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c1", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--K", type=int, default=None, help="override K (c4 sweep)")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ workload
+
+def global_batch(name, n_gpus, K=None):
+    """The workload at n_gpus times its batch size (weak scaling)."""
+    kw = {}
+    if K is not None:
+        kw["K"] = K
+    base = workloads.make_workload(name, **kw)
+    if n_gpus == 1:
+        return base
+    kw2 = dict(kw)
+    if name != "c0":
+        kw2["B"] = base.B * n_gpus
+    return workloads.make_workload(name, **kw2)
+
+
+def event_cost(sizes, K):
+    return np.where(sizes > K, sizes.astype(np.float64) * K, sizes.astype(np.float64) * 0.01 + 1.0)
+
+
+def partition_events(sizes, K, world):
+    """Longest-processing-time split of events over ranks by N*K cost."""
+    cost = event_cost(np.asarray(sizes), K)
+    order = np.argsort(-cost, kind="stable")
+    load = np.zeros(world)
+    parts = [[] for _ in range(world)]
+    for e in order:
+        r = int(np.argmin(load))
+        parts[r].append(int(e))
+        load[r] += cost[e]
+    return [np.array(sorted(p), dtype=np.int64) for p in parts]
+
+
+def shard(batch, events):
+    sizes = batch.sizes()
+    cs, fs = [], []
+    for e in events:
+        o0, o1 = batch.offsets[e], batch.offsets[e + 1]
+        cs.append(batch.coords[o0:o1])
+        fs.append(batch.feats[o0:o1])
+    off = np.zeros(len(events) + 1, np.int64)
+    np.cumsum(sizes[events], out=off[1:])
+    return workloads.Batch(np.ascontiguousarray(np.concatenate(cs)) if cs else batch.coords[:0],
+                           np.ascontiguousarray(np.concatenate(fs)) if fs else batch.feats[:0], off, batch.K,
+                           batch.assign_mode, batch.k, batch.lloyd_iters, batch.charge_col, None, batch.name)
+
+
+def algorithmic(batch):
+    """Distance evaluations and bytes of one step (the design doc accounting)."""
+    sizes = batch.sizes()
+    K, F = batch.K, batch.F
+    fpsev = sizes[sizes > K]
+    evals = int((fpsev * K).sum()) * (1 + batch.lloyd_iters)
+    if batch.assign_mode == 1:
+        evals += int((fpsev * K).sum())
+    P, B = batch.P, batch.B
+    byts = 16 * P + 4 * F * P + 4 * P + 8 * (B + 1) + B * K * (4 + 16 + 4 * F + 4)
+    if batch.assign_mode == 1:
+        byts += B * K * batch.k * 4
+    return evals, byts
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, enabled=True):
+        self.gpu = gpu_index
+        self.proc = None
+        self.enabled = enabled
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                     "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        if not getattr(self, "lines", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ profiles (ncu traffic)
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("fps_kernels.cu", "common.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "farthest_point_sampling_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_stage, workload):
+    """DRAM bytes per launch recorded in a committed ncu summary, if it was
+    taken from the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    pat = re.compile(r"^\|\s*(\S+)\s*\|\s*(\S+)\s*\|\s*([0-9.]+)\s*\|\s*([0-9a-f]{16})\s*\|")
+    with open(path) as fh:
+        for ln in fh:
+            m = pat.match(ln)
+            if m and m.group(1) == STAGE_KERNELS[kernel_stage] and m.group(2) == workload and m.group(4) == want:
+                return float(m.group(3))
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_rate(batch, seconds):
+    import oracle
+
+    oracle.build()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.tokenize_batch(batch)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return batch.B * reps / el, reps, el
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    batch = global_batch(args.workload, 1, args.K)
+    import oracle
+
+    oracle.build()
+    for _ in range(args.warmup):
+        oracle.tokenize_batch(batch)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.tokenize_batch(batch)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = batch.B * args.steps / total
+    evals, _ = algorithmic(batch)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "events/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded generator)", "config": config_of(batch, args, l2="n/a (host)"),
+        "gevals_per_s": evals * args.steps / total / 1e9,
+        "cpu_baseline": {"value": value, "unit": "events/s", "cores": 1, "kind": "oracle",
+                         "sample": f"the full batch ({batch.B} events) per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": "events/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(batch, args, l2):
+    return {"workload": batch.name, "events_per_gpu": batch.B, "points_per_gpu": batch.P, "K": batch.K,
+            "assign_mode": "knn" if batch.assign_mode == 1 else "voronoi", "k": batch.k,
+            "lloyd_iters": batch.lloyd_iters, "parallelism": f"dp{args.gpus} (events sharded, no collective)",
+            "l2": l2}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import farthest_point_sampling_b200 as fps
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    full = global_batch(args.workload, world, args.K)
+    if world > 1:
+        parts = partition_events(full.sizes(), full.K, world)
+        batch = shard(full, parts[rank])
+    else:
+        batch = full
+    fps.build()
+    fps.load_library()
+
+    coords = torch.from_numpy(batch.coords).to(dev)
+    feats = torch.from_numpy(batch.feats).to(dev)
+    offsets = torch.from_numpy(batch.offsets).to(dev)
+    hint = int(batch.sizes().max()) if batch.B else 0
+    kw = dict(K=batch.K, assign_mode=batch.assign_mode, k=max(batch.k, 1), lloyd_iters=batch.lloyd_iters,
+              charge_col=batch.charge_col, max_event_hint=hint)
+    out = fps.fps_tokenize(coords, feats, offsets, check_device=True, **kw)
+    ws = torch.empty(0, dtype=torch.uint8, device=dev)
+    lib = fps.load_library()
+    import ctypes
+
+    opts = fps.Options(**{k: v for k, v in kw.items()})
+    ws = torch.empty(lib.fps_workspace_bytes(batch.P, batch.B, batch.F, ctypes.byref(opts.c)), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fps.fps_tokenize(coords, feats, offsets, workspace=ws, out=out, **kw)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))] for _ in range(K)]
+    for evs in stage_ev:  # materialise the handles the library records into
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = fps.launch_count()
+    wall0 = time.perf_counter()
+    with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as clocks:
+        for i in range(K):
+            flush.zero_()
+            fps.set_stage_events(stage_ev[i])
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        fps.set_stage_events(None)
+        torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    launches = fps.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    events_all = full.B
+    ms_per_step = total_ms / K
+    value = events_all / (ms_per_step / 1e3)
+    evals, _ = algorithmic(full)
+
+    # per-stage device time (recorded by the library inside the timed steps)
+    stage_ms = {}
+    for s in range(len(STAGES)):
+        ts = []
+        for evs in stage_ev:
+            try:
+                ts.append(evs[2 * s].elapsed_time(evs[2 * s + 1]))
+            except RuntimeError:
+                break
+        if len(ts) == K:
+            stage_ms[s] = float(np.mean(ts))
+    # stages that did not run in this workload keep their warm-up recordings: drop them
+    sizes = batch.sizes()
+    sched = np.array([lib.fps_schedule_for(int(n), batch.K, -1) for n in sizes])
+    ran = {0, 6 if batch.assign_mode == 0 else 5}
+    ran |= {1 + s for s in (0, 1, 2) if (sched == s).any()}
+    if batch.lloyd_iters:
+        ran.add(4)
+    stage_ms = {s: v for s, v in stage_ms.items() if s in ran}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "events/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded generator shaped like the pages' events)",
+        "config": config_of(batch, args, l2="flushed between steps (256 MiB write outside the timed events)"),
+        "gevals_per_s": evals / (ms_per_step / 1e3) / 1e9,
+        "gpu_launches": int(launches),
+        "stage_ms": {STAGES[s]: round(v, 5) for s, v in sorted(stage_ms.items())},
+        "wall_s_timed_region": wall,
+    }
+
+    if rank == 0:
+        # roofline of the dominant kernel (FP32 issue bound for the FPS kernels)
+        dom = max(stage_ms, key=stage_ms.get)
+        t_dom = stage_ms[dom] / 1e3
+        peak = SM_COUNT * FP32_LANES_PER_SM * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
+        if dom in (1, 2, 3):
+            ev = int(sum(int(n) * batch.K for n, s in zip(sizes, sched) if s == dom - 1))
+            achieved = ev * FP32_OPS_PER_EVAL / t_dom / 1e12
+            roof = {"bound": "alu", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 1965 MHz (non-FMA float32 ops)",
+                    "algorithmic": f"{ev} point-centroid evals x {FP32_OPS_PER_EVAL} FP32 ops per launch",
+                    "traffic": recorded_traffic(dom, args.workload)}
+        else:
+            _, byts = algorithmic(batch)
+            import json as _j
+
+            peaks = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+                os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+            hbm = float(peaks.get("hbm_gbs", 6650.0))
+            achieved = byts / t_dom / 1e9
+            roof = {"bound": "hbm", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": hbm,
+                    "unit": "GB/s", "frac": achieved / hbm, "traffic": recorded_traffic(dom, args.workload)}
+        roof["microbench_fp32_tflops"] = microbench_fp32(dev)
+        result["roofline"] = roof
+        result["clocks"] = clocks.summary()
+        result["e2e"] = e2e(fps, batch, kw, dev, args.e2e_steps)
+        if world == 1 and not args.no_cpu_baseline:
+            rate, reps, el = cpu_oracle_rate(batch, args.cpu_seconds)
+            result["cpu_baseline"] = {"value": rate, "unit": "events/s", "cores": 1, "kind": "oracle",
+                                      "sample": f"the full batch ({batch.B} events) x {reps} passes, {el:.1f} s"}
+        print(json.dumps(result))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def microbench_fp32(dev):
+    """Best measured non-FMA FP32 op rate (TFLOP/s) of scalar and f32x2 chains."""
+    import ctypes
+
+    import torch
+
+    import farthest_point_sampling_b200 as fps
+
+    lib = ctypes.CDLL(fps.build_microbench())
+    lib.fpstok_microbench_fp32.restype = ctypes.c_double
+    lib.fpstok_microbench_fp32.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    blocks = torch.cuda.get_device_properties(dev).multi_processor_count * 8
+    out = torch.empty(blocks, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    best = {}
+    for packed in (0, 1):
+        rates = []
+        for _ in range(4):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ops = lib.fpstok_microbench_fp32(packed, blocks, 256, 4096, ctypes.c_void_p(out.data_ptr()),
+                                             ctypes.c_void_p(a.cuda_event), ctypes.c_void_p(b.cuda_event),
+                                             ctypes.c_void_p(stream.cuda_stream))
+            torch.cuda.synchronize(dev)
+            rates.append(ops / (a.elapsed_time(b) / 1e3) / 1e12)
+        best["f32x2" if packed else "scalar"] = max(rates)
+    return best
+
+
+def e2e(fps, batch, kw, dev, steps):
+    """Same metric through the host-pointer C entry point (H2D + compute + D2H)."""
+    import torch
+
+    c = torch.from_numpy(batch.coords).pin_memory()
+    f = torch.from_numpy(batch.feats).pin_memory()
+    o = torch.from_numpy(batch.offsets)
+    kw2 = {k: v for k, v in kw.items() if k not in ("max_event_hint",)}
+    out = fps.fps_tokenize_host(c, f, o, device=dev, **kw2)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        fps.fps_tokenize_host(c, f, o, device=dev, out=out, **kw2)
+    tot = 0.0
+    for _ in range(steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fps.fps_tokenize_host(c, f, o, device=dev, out=out, synchronize=False, **kw2)
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    h2d = batch.coords.nbytes + batch.feats.nbytes + batch.offsets.nbytes
+    d2h = sum(v.numel() * v.element_size() for v in out.values())
+    return {"value": batch.B * steps / (tot / 1e3), "unit": "events/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / steps}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

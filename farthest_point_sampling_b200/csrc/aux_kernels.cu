@@ -1,0 +1,642 @@
+// Binning, passthrough, pooling, Lloyd refinement, nearest-centroid assignment
+// and the kNN gather of the fpstok tokenizer.
+//
+// Per-token pooling ("pools the pulses of each token", graphnet PR #923 "Add
+// Neptune point-transformer backbone", Summary), small events kept at one
+// token per pulse (same page, "What is added", FPSTokenizer), nearest-centroid
+// assignment and the kNN gather (components/fps.py nearest_assign and
+// farthest_point_sampling_with_knn, same list), and charge-weighted Lloyd
+// refinement (Neptune README, "How it works", step 1).
+//
+// Float sums (pool means, Lloyd weighted means) accumulate in float64 in any
+// order, first per CTA in shared memory and then, for events spread over
+// several CTAs, in global memory; they are rounded once to float32.  Every
+// term is an exact float64 (a float32, or the product of two float32), so the
+// result differs from a sequential float64 sum only by float64 rounding,
+// far below the float32 rounding of the final mean.
+#include "common.cuh"
+#include "internal.h"
+
+namespace fpstok {
+
+// ------------------------------------------------------------------ binning
+
+__global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
+                                               int K, const int32_t* __restrict__ start_local,
+                                               int force, int chunk_all, Workspace ws) {
+  __shared__ int cnt[8];
+  if (threadIdx.x < 8) cnt[threadIdx.x] = 0;
+  if (threadIdx.x == 0) {
+    ws.hdr->status = 0;
+    ws.hdr->detail = 0;
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t o0 = offsets[b], o1 = offsets[b + 1];
+    int cls;
+    int64_t n = 0;
+    if (o0 < 0 || o1 < o0 || o1 > P) {
+      record_error(ws.hdr, kDevBadOffsets);
+      cls = kClsSkip;
+    } else {
+      if ((b == 0 && o0 != 0) || (b == B - 1 && o1 != P)) record_error(ws.hdr, kDevBadOffsets);
+      n = o1 - o0;
+      cls = n == 0 ? kClsEmpty : (n <= K ? kClsPass : kClsFps);
+      if (cls == kClsFps) {
+        const int s = start_local ? start_local[b] : 0;
+        if (s < 0 || s >= n) {
+          record_error(ws.hdr, kDevBadStart);
+          cls = kClsSkip;
+        } else if (n > kClusterCap) {
+          record_error(ws.hdr, kDevTooLarge);
+          cls = kClsSkip;
+        }
+      }
+    }
+    ws.cls[b] = cls;
+    int fslot = -1, pslot = -1;
+    if (cls == kClsFps) {
+      int sched = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : 2);
+      if (force > sched) sched = force > 2 ? 2 : force;
+      int* list = sched == 0 ? ws.list_warp : (sched == 1 ? ws.list_cta : ws.list_cluster);
+      list[atomicAdd(&cnt[sched], 1)] = b;
+      fslot = atomicAdd(&cnt[kListFps], 1);
+    }
+    if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
+      const int nch = (int)((n + kChunk - 1) / kChunk);
+      const int base = atomicAdd(&cnt[kListChunks], nch);
+      for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
+      if (nch > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
+    }
+    ws.fps_slot[b] = fslot;
+    ws.pool_slot[b] = pslot;
+  }
+  __syncthreads();
+  if (threadIdx.x < 8) ws.hdr->n_items[threadIdx.x] = cnt[threadIdx.x];
+}
+
+cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s) {
+  count_launch();
+  k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
+                           ws);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ passthrough
+
+// Events with N <= K keep one token per pulse; empty and skipped events get
+// empty rows; FPS events get their global accumulators cleared.
+__global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, int lloyd_on) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int K = pb.K, F = pb.F, k = pb.k;
+  for (int b = gw; b < pb.B; b += nw) {
+    const int cls = ws.cls[b];
+    if (cls == kClsFps) {
+      const int ps = ws.pool_slot[b];
+      if (ps >= 0) {
+        for (int e = lane; e < K * F; e += 32) ws.pool_acc[(int64_t)ps * K * F + e] = 0.0;
+        for (int e = lane; e < K; e += 32) ws.pool_cnt[(int64_t)ps * K + e] = 0;
+        if (lane == 0) ws.pool_ticket[ps] = 0;
+      }
+      const int fs = ws.fps_slot[b];
+      if (lloyd_on && fs >= 0) {
+        for (int e = lane; e < K * 5; e += 32) {
+          ws.lloyd[0][(int64_t)fs * K * 5 + e] = 0.0;
+          ws.lloyd[1][(int64_t)fs * K * 5 + e] = 0.0;
+        }
+      }
+      continue;
+    }
+    int64_t off = 0;
+    int n = 0;
+    if (cls == kClsPass) {
+      off = pb.offsets[b];
+      n = (int)(pb.offsets[b + 1] - off);
+    }
+    const float* cf = reinterpret_cast<const float*>(pb.coords);
+    float* outc = reinterpret_cast<float*>(pb.centroids) + (int64_t)b * K * 4;
+    for (int e = lane; e < K * 4; e += 32) outc[e] = e < n * 4 ? cf[off * 4 + e] : 0.f;
+    float* outp = pb.pooled + (int64_t)b * K * F;
+    for (int e = lane; e < K * F; e += 32) outp[e] = e < n * F ? pb.feats[off * F + e] : 0.f;
+    for (int j = lane; j < K; j += 32) {
+      pb.centroid_idx[(int64_t)b * K + j] = j < n ? (int32_t)(off + j) : -1;
+      pb.counts[(int64_t)b * K + j] = j < n ? 1 : 0;
+    }
+    if (pb.token_id)
+      for (int j = lane; j < n; j += 32) pb.token_id[off + j] = j;
+    if (pb.knn_idx) {
+      int32_t* outk = pb.knn_idx + (int64_t)b * K * k;
+      for (int e = lane; e < K * k; e += 32) {
+        const int j = e / k, r = e - j * k;
+        outk[e] = (r == 0 && j < n) ? (int32_t)(off + j) : -1;
+      }
+    }
+  }
+}
+
+cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  int blocks = (pb.B + 7) / 8;
+  const int cap = di.sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  count_launch();
+  k_passthrough<<<blocks, 256, 0, s>>>(pb, ws, pb.lloyd_iters > 0 ? 1 : 0);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ Voronoi pool
+
+// One CTA per (event, chunk) item: shared-memory float64 sums per token, then
+// either the final means (single-chunk event) or global float64 accumulation
+// with the last-arriving CTA of the event producing the means.
+__global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ feats, int F,
+                                                      const int64_t* __restrict__ offsets, int K,
+                                                      const int32_t* __restrict__ labels,
+                                                      float* __restrict__ pooled,
+                                                      int32_t* __restrict__ counts, Workspace ws) {
+  extern __shared__ double smem_d[];
+  double* s_sum = smem_d;                                 // [K*F]
+  int* s_cnt = reinterpret_cast<int*>(s_sum + K * F);     // [K]
+  __shared__ int s_last;
+  const int nitems = ws.hdr->n_items[kListChunks];
+  const int KF = K * F;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int2 it = ws.chunks[item];
+    const int b = it.x;
+    const int64_t off = offsets[b];
+    const int n = (int)(offsets[b + 1] - off);
+    const int i0 = it.y * kChunk;
+    const int i1 = min(n, i0 + kChunk);
+    const int nch = (n + kChunk - 1) / kChunk;
+    for (int e = threadIdx.x; e < KF; e += blockDim.x) s_sum[e] = 0.0;
+    for (int e = threadIdx.x; e < K; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    const int64_t e0 = (off + i0) * F, e1 = (off + i1) * F;
+    for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+      const int64_t i = e / F;
+      const int f = (int)(e - i * F);
+      const int j = labels[i];
+      if (j < 0) continue;
+      if (j >= K) {
+        record_error(ws.hdr, kDevBadToken);
+        continue;
+      }
+      if (f == 0) atomicAdd(&s_cnt[j], 1);
+      atomicAdd(&s_sum[j * F + f], (double)feats[e]);
+    }
+    __syncthreads();
+    if (nch == 1) {
+      for (int e = threadIdx.x; e < KF; e += blockDim.x) {
+        const int c = s_cnt[e / F];
+        pooled[(int64_t)b * KF + e] = c ? (float)(s_sum[e] / (double)c) : 0.f;
+      }
+      for (int j = threadIdx.x; j < K; j += blockDim.x) counts[(int64_t)b * K + j] = s_cnt[j];
+    } else {
+      const int ps = ws.pool_slot[b];
+      double* acc = ws.pool_acc + (int64_t)ps * KF;
+      int* cnt = ws.pool_cnt + (int64_t)ps * K;
+      for (int e = threadIdx.x; e < KF; e += blockDim.x)
+        if (s_sum[e] != 0.0) atomicAdd(&acc[e], s_sum[e]);
+      for (int j = threadIdx.x; j < K; j += blockDim.x)
+        if (s_cnt[j]) atomicAdd(&cnt[j], s_cnt[j]);
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) s_last = atomicAdd(&ws.pool_ticket[ps], 1) == nch - 1;
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        for (int e = threadIdx.x; e < KF; e += blockDim.x) {
+          const int c = __ldcg(&cnt[e / F]);
+          pooled[(int64_t)b * KF + e] = c ? (float)(__ldcg(&acc[e]) / (double)c) : 0.f;
+        }
+        for (int j = threadIdx.x; j < K; j += blockDim.x) counts[(int64_t)b * K + j] = __ldcg(&cnt[j]);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+static size_t pool_smem(int K, int F) { return (size_t)K * F * sizeof(double) + (size_t)K * sizeof(int); }
+
+cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
+                                const int32_t* labels, float* pooled, int32_t* counts,
+                                const Workspace& ws, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  const size_t sm = pool_smem(K, F);
+  count_launch();
+  k_pool_voronoi<<<di.sm_count * 4, 256, sm, s>>>(feats, F, offsets, K, labels, pooled, counts, ws);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ nearest centroid
+
+// Centroids of one event in shared memory, broadcast into packed pairs.
+__device__ __forceinline__ void load_cents(const float4* __restrict__ c, int nv, Cent2* s) {
+  for (int j = threadIdx.x; j < nv; j += blockDim.x) s[j] = cent2(c[j]);
+}
+
+// Nearest of the first nv shared-memory centroids for points [i0, i1) of an
+// event (thread-strided, two points per packed evaluation); strict '<' over
+// increasing slots keeps the lowest slot on ties.  Calls emit(i, label) once
+// per point.
+template <int PAIRS, typename Emit>
+__device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int i0, int i1,
+                                             const Cent2* __restrict__ cs, int nv, Emit emit) {
+  const int T = blockDim.x;
+  for (int base = i0; base < i1; base += 2 * PAIRS * T) {
+    uint64_t X[PAIRS], Y[PAIRS], Z[PAIRS], W[PAIRS];
+    float best[2 * PAIRS];
+    int lab[2 * PAIRS];
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+      if (ia < i1) a = ldg4(pts + ia);
+      if (ib < i1) c = ldg4(pts + ib);
+      X[p] = pack2(a.x, c.x);
+      Y[p] = pack2(a.y, c.y);
+      Z[p] = pack2(a.z, c.z);
+      W[p] = pack2(a.w, c.w);
+      best[2 * p] = best[2 * p + 1] = __int_as_float(0x7f800000);
+      lab[2 * p] = lab[2 * p + 1] = -1;
+    }
+    for (int j = 0; j < nv; ++j) {
+      const Cent2 C = cs[j];
+#pragma unroll
+      for (int p = 0; p < PAIRS; ++p) {
+        const uint64_t d = dist2(X[p], Y[p], Z[p], W[p], C);
+        relax(lo2(d), best[2 * p], lab[2 * p], j);
+        relax(hi2(d), best[2 * p + 1], lab[2 * p + 1], j);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
+      if (ia < i1) emit(ia, nv > 0 ? (lab[2 * p] < 0 ? 0 : lab[2 * p]) : -1);
+      if (ib < i1) emit(ib, nv > 0 ? (lab[2 * p + 1] < 0 ? 0 : lab[2 * p + 1]) : -1);
+    }
+  }
+}
+
+constexpr int kAssignPairs = 4;
+
+// Standalone nearest-centroid assignment over (event, chunk) items.
+__global__ void __launch_bounds__(256) k_assign(const float4* __restrict__ coords,
+                                                const int64_t* __restrict__ offsets, int K,
+                                                const float4* __restrict__ centroids,
+                                                const int32_t* __restrict__ valid,
+                                                int32_t* __restrict__ token_id, Workspace ws) {
+  extern __shared__ Cent2 s_cent[];
+  const int nitems = ws.hdr->n_items[kListChunks];
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int2 it = ws.chunks[item];
+    const int b = it.x;
+    const int64_t off = offsets[b];
+    const int n = (int)(offsets[b + 1] - off);
+    int nv = valid ? valid[b] : min(n, K);
+    if (nv < 0 || nv > K) {
+      record_error(ws.hdr, kDevBadToken);
+      nv = 0;
+    }
+    load_cents(centroids + (int64_t)b * K, nv, s_cent);
+    __syncthreads();
+    const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
+    int32_t* out = token_id + off;
+    nearest_pass<kAssignPairs>(coords + off, i0, i1, s_cent, nv, [&](int i, int l) { out[i] = l; });
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ Lloyd
+
+// Adds (q, q*x, q*y, q*z, q*t) of point i (event-local) to token j's shared sums.
+__device__ __forceinline__ void lloyd_accum(double* s, const float4* pts, const float* fe, int F,
+                                            int charge_col, int i, int j) {
+  const float4 p = ldg4(pts + i);
+  const double q = charge_col < 0 ? 1.0 : (double)fe[(int64_t)i * F + charge_col];
+  atomicAdd(&s[j * 5 + 0], q);
+  atomicAdd(&s[j * 5 + 1], q * (double)p.x);
+  atomicAdd(&s[j * 5 + 2], q * (double)p.y);
+  atomicAdd(&s[j * 5 + 3], q * (double)p.z);
+  atomicAdd(&s[j * 5 + 4], q * (double)p.w);
+}
+
+__device__ __forceinline__ void flush_sums(const double* s, double* g, int n) {
+  for (int e = threadIdx.x; e < n; e += blockDim.x)
+    if (s[e] != 0.0) atomicAdd(&g[e], s[e]);
+}
+
+// Cell sums of the current labels.
+__global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ coords,
+                                                    const float* __restrict__ feats, int F,
+                                                    int charge_col, const int64_t* __restrict__ offsets,
+                                                    int K, const int32_t* __restrict__ labels,
+                                                    Workspace ws, double* __restrict__ out) {
+  extern __shared__ double s_sum[];  // [K*5]
+  const int nitems = ws.hdr->n_items[kListChunks];
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int2 it = ws.chunks[item];
+    const int b = it.x;
+    const int fs = ws.fps_slot[b];
+    if (fs < 0) continue;  // uniform across the CTA
+    const int64_t off = offsets[b];
+    const int n = (int)(offsets[b + 1] - off);
+    for (int e = threadIdx.x; e < K * 5; e += blockDim.x) s_sum[e] = 0.0;
+    __syncthreads();
+    const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+      const int j = labels[off + i];
+      if (j < 0 || j >= K) {
+        record_error(ws.hdr, kDevBadToken);
+        continue;
+      }
+      lloyd_accum(s_sum, coords + off, feats ? feats + off * F : nullptr, F, charge_col, i, j);
+    }
+    __syncthreads();
+    flush_sums(s_sum, out + (int64_t)fs * K * 5, K * 5);
+    __syncthreads();
+  }
+}
+
+// One Lloyd iteration: centroids from the sums `in`, re-assign the chunk and
+// (unless last) accumulate the next sums into `next`; clears `clear`.
+__global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict__ coords,
+                                                    const float* __restrict__ feats, int F,
+                                                    int charge_col, const int64_t* __restrict__ offsets,
+                                                    int K, int32_t* __restrict__ labels,
+                                                    float4* __restrict__ centroids, Workspace ws,
+                                                    const double* __restrict__ in, double* __restrict__ next,
+                                                    double* __restrict__ clear, int64_t clear_n) {
+  extern __shared__ double smem_l[];
+  double* s_sum = smem_l;                                  // [K*5]
+  Cent2* s_cent = reinterpret_cast<Cent2*>(s_sum + K * 5);  // [K]
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < clear_n;
+       e += (int64_t)gridDim.x * blockDim.x)
+    clear[e] = 0.0;
+  const int nitems = ws.hdr->n_items[kListChunks];
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int2 it = ws.chunks[item];
+    const int b = it.x;
+    const int fs = ws.fps_slot[b];
+    if (fs < 0) continue;
+    const int64_t off = offsets[b];
+    const int n = (int)(offsets[b + 1] - off);
+    const double* sb = in + (int64_t)fs * K * 5;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const double W = __ldcg(&sb[j * 5]);
+      float4 c = centroids[(int64_t)b * K + j];
+      if (W > 0.0) {
+        c.x = (float)(__ldcg(&sb[j * 5 + 1]) / W);
+        c.y = (float)(__ldcg(&sb[j * 5 + 2]) / W);
+        c.z = (float)(__ldcg(&sb[j * 5 + 3]) / W);
+        c.w = (float)(__ldcg(&sb[j * 5 + 4]) / W);
+      }
+      s_cent[j] = cent2(c);
+      if (it.y == 0) centroids[(int64_t)b * K + j] = c;
+    }
+    if (next)
+      for (int e = threadIdx.x; e < K * 5; e += blockDim.x) s_sum[e] = 0.0;
+    __syncthreads();
+    const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
+    int32_t* lab = labels + off;
+    const float4* pts = coords + off;
+    const float* fe = feats ? feats + off * F : nullptr;
+    nearest_pass<kAssignPairs>(pts, i0, i1, s_cent, K, [&](int i, int l) {
+      lab[i] = l;
+      if (next) lloyd_accum(s_sum, pts, fe, F, charge_col, i, l);
+    });
+    __syncthreads();
+    if (next) flush_sums(s_sum, next + (int64_t)fs * K * 5, K * 5);
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  const int K = pb.K;
+  const int grid = di.sm_count * 4;
+  const size_t sm_sums = (size_t)K * 5 * sizeof(double);
+  const size_t sm_step = sm_sums + (size_t)K * sizeof(Cent2);
+  cudaError_t e;
+  const float* feats = pb.charge_col >= 0 ? pb.feats : nullptr;
+  count_launch();
+  k_lloyd_sums<<<grid, 256, sm_sums, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels,
+                                          ws, ws.lloyd[0]);
+  if ((e = cudaGetLastError())) return e;
+  // iteration t reads buffer t%3, accumulates into (t+1)%3 unless it is the
+  // last one, and clears (t+2)%3 when iteration t+1 will accumulate into it
+  const int64_t per = (int64_t)K * 5;
+  for (int t = 0; t < pb.lloyd_iters; ++t) {
+    const bool last = t == pb.lloyd_iters - 1;
+    double* clear = (t + 1 < pb.lloyd_iters - 1) ? ws.lloyd[(t + 2) % 3] : nullptr;
+    count_launch();
+    k_lloyd_step<<<grid, 256, sm_step, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K,
+                                            labels, pb.centroids, ws, ws.lloyd[t % 3],
+                                            last ? nullptr : ws.lloyd[(t + 1) % 3], clear,
+                                            clear ? (int64_t)ws.fps_slots * per : 0);
+    if ((e = cudaGetLastError())) return e;
+  }
+  return cudaSuccess;
+}
+
+// Shared-memory limits of the auxiliary kernels, set once per device for the
+// largest K and F the ABI accepts.
+cudaError_t prepare_aux_kernels() {
+  cudaError_t e;
+  const int pool_max = (int)pool_smem(256, 64);
+  const int sums_max = 256 * 5 * (int)sizeof(double);
+  const int step_max = sums_max + 256 * (int)sizeof(Cent2);
+  if ((e = cudaFuncSetAttribute(k_pool_voronoi, cudaFuncAttributeMaxDynamicSharedMemorySize, pool_max)))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, sums_max)))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize, step_max)))
+    return e;
+  return cudaSuccess;
+}
+
+// ------------------------------------------------------------------ kNN
+
+// Mean of the features of the valid entries of one kNN row (warp-cooperative;
+// each lane contributes the entries it holds).  Lane 0 writes the results.
+template <int KPL>
+__device__ __forceinline__ void knn_row_pool(const float* __restrict__ feats, int F, const int* gidx,
+                                             float* __restrict__ pooled_row, int32_t* count_out) {
+  const int lane = threadIdx.x & 31;
+  int c = 0;
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) c += gidx[q] >= 0;
+  c = __reduce_add_sync(kFull, c);
+  for (int f = 0; f < F; ++f) {
+    double s = 0.0;
+#pragma unroll
+    for (int q = 0; q < KPL; ++q)
+      if (gidx[q] >= 0) s += (double)feats[(int64_t)gidx[q] * F + f];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+    if (lane == 0) pooled_row[f] = c ? (float)(s / (double)c) : 0.f;
+  }
+  if (lane == 0) *count_out = c;
+}
+
+// One warp per (event, centroid) row: the k smallest (d, index) keys of the
+// event, kept sorted across the warp (element e at lane e % 32, slot e / 32).
+template <int KPL>
+__global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
+                                             const int64_t* __restrict__ offsets, int B,
+                                             const float4* __restrict__ centroids,
+                                             const int32_t* __restrict__ valid, int K, int k,
+                                             int32_t* __restrict__ knn_idx,
+                                             const float* __restrict__ feats, int F,
+                                             float* __restrict__ pooled, int32_t* __restrict__ counts,
+                                             const int* __restrict__ cls, WsHeader* hdr) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int64_t rows = (int64_t)B * K;
+  const int kq = (k - 1) >> 5, kl = (k - 1) & 31;
+  for (int64_t r = gw; r < rows; r += nw) {
+    const int b = (int)(r / K), j = (int)(r - (int64_t)b * K);
+    if (cls && cls[b] != kClsFps) continue;
+    const int64_t o0 = offsets[b], o1 = offsets[b + 1];
+    int n = 0, nv = 0;
+    if (o0 >= 0 && o1 >= o0) {
+      n = (int)(o1 - o0);
+      nv = valid ? valid[b] : min(n, K);
+      if (nv < 0 || nv > K) {
+        if (lane == 0) record_error(hdr, kDevBadToken);
+        nv = 0;
+      }
+    } else if (lane == 0) {
+      record_error(hdr, kDevBadOffsets);
+    }
+    uint64_t L[KPL];
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) L[q] = ~0ull;
+    if (j < nv) {
+      const float4 c = centroids[r];
+      const float4* pts = coords + o0;
+      uint64_t thr = ~0ull;
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        uint64_t key = ~0ull;
+        if (i < n) key = ((uint64_t)__float_as_uint(dist1(ldg4(pts + i), c)) << 32) | (uint32_t)i;
+        unsigned mask = __ballot_sync(kFull, key < thr);
+        while (mask) {
+          const int src = __ffs(mask) - 1;
+          mask &= mask - 1;
+          const uint64_t v = __shfl_sync(kFull, key, src);
+          if (v >= thr) continue;
+          int pos = 0;
+#pragma unroll
+          for (int q = 0; q < KPL; ++q) pos += __popc(__ballot_sync(kFull, L[q] < v));
+#pragma unroll
+          for (int q = KPL - 1; q >= 0; --q) {
+            uint64_t up = __shfl_up_sync(kFull, L[q], 1);
+            if (q > 0) {
+              const uint64_t carry = __shfl_sync(kFull, L[q - 1], 31);
+              if (lane == 0) up = carry;
+            }
+            const int e = q * 32 + lane;
+            if (e > pos) L[q] = up;
+            else if (e == pos) L[q] = v;
+          }
+          uint64_t t = 0;
+#pragma unroll
+          for (int q = 0; q < KPL; ++q)
+            if (q == kq) t = L[q];
+          thr = __shfl_sync(kFull, t, kl);
+        }
+      }
+    }
+    int gidx[KPL];
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) {
+      const int e = q * 32 + lane;
+      gidx[q] = (e < k && L[q] != ~0ull) ? (int)(o0 + (int64_t)(uint32_t)L[q]) : -1;
+      if (e < k) knn_idx[r * k + e] = gidx[q];
+    }
+    if (pooled) knn_row_pool<KPL>(feats, F, gidx, pooled + r * F, counts + r);
+  }
+}
+
+cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
+                       const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, const float* feats,
+                       int F, float* pooled, int32_t* counts, const int* cls, WsHeader* hdr,
+                       cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  const int64_t rows = (int64_t)B * K;
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = (int64_t)di.sm_count * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  count_launch();
+  if (k <= 32)
+    k_knn<1><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
+                                         feats, F, pooled, counts, cls, hdr);
+  else if (k <= 64)
+    k_knn<2><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
+                                         feats, F, pooled, counts, cls, hdr);
+  else
+    k_knn<4><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
+                                         feats, F, pooled, counts, cls, hdr);
+  return cudaGetLastError();
+}
+
+// Standalone kNN pooling over given rows.
+template <int KPL>
+__global__ void __launch_bounds__(256) k_pool_knn(const float* __restrict__ feats, int F, int64_t rows,
+                                                  int k, const int32_t* __restrict__ knn_idx, int64_t P,
+                                                  float* __restrict__ pooled, int32_t* __restrict__ counts,
+                                                  WsHeader* hdr) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = gw; r < rows; r += nw) {
+    int gidx[KPL];
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) {
+      const int e = q * 32 + lane;
+      int v = e < k ? knn_idx[r * k + e] : -1;
+      if (v >= P) {
+        record_error(hdr, kDevBadToken);
+        v = -1;
+      }
+      gidx[q] = v;
+    }
+    knn_row_pool<KPL>(feats, F, gidx, pooled + r * F, counts + r);
+  }
+}
+
+cudaError_t launch_pool_knn(const float* feats, int F, int B, int K, int k, const int32_t* knn_idx,
+                            int64_t P, float* pooled, int32_t* counts, WsHeader* hdr, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  const int64_t rows = (int64_t)B * K;
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = (int64_t)di.sm_count * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  count_launch();
+  if (k <= 32)
+    k_pool_knn<1><<<(int)blocks, 256, 0, s>>>(feats, F, rows, k, knn_idx, P, pooled, counts, hdr);
+  else if (k <= 64)
+    k_pool_knn<2><<<(int)blocks, 256, 0, s>>>(feats, F, rows, k, knn_idx, P, pooled, counts, hdr);
+  else
+    k_pool_knn<4><<<(int)blocks, 256, 0, s>>>(feats, F, rows, k, knn_idx, P, pooled, counts, hdr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const float4* centroids,
+                          const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,
+                          cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  const size_t sm = (size_t)K * sizeof(Cent2);
+  count_launch();
+  k_assign<<<di.sm_count * 4, 256, sm, s>>>(coords, offsets, K, centroids, valid_tokens, token_id, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace fpstok

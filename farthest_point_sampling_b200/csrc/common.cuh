@@ -1,0 +1,120 @@
+// Device-side building blocks shared by the fpstok kernels (sm_100a only).
+//
+// The squared distance follows the tokenizer's fixed float32 contract:
+// d(i, c) = ((dx*dx + dy*dy) + dz*dz) + dt*dt, every operation rounded to
+// nearest-even and never fused (4D (x, y, z, t) points: graphnet PR #923 "Add
+// Neptune point-transformer backbone", Summary; float32 only: same page,
+// review thread on the FPS `precision` argument).  Two points are evaluated
+// at once with the packed f32x2 instructions of sm_100a: each lane of a pair
+// is an ordinary IEEE round-to-nearest float32 operation, so the result is
+// bit-identical to the scalar formula while using half the issue slots.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "fpstok kernels are written for sm_100a (B200) only"
+#endif
+
+namespace fpstok {
+
+constexpr int kWarp = 32;
+constexpr unsigned kFull = 0xffffffffu;
+// Running-minimum value of a slot that holds no point: negative, so it never
+// wins the arg-max (whose keys are the bit patterns of non-negative floats).
+constexpr float kEmptySlot = -1.0f;
+
+// Device status codes (match FPS_DEV_* in fpstok.h).
+constexpr int kDevBadOffsets = 1;
+constexpr int kDevBadStart = 2;
+constexpr int kDevBadToken = 3;
+constexpr int kDevTooLarge = 4;
+
+// Workspace header: status word, detail word, then counters.
+struct WsHeader {
+  int status;
+  int detail;
+  int n_items[14];  // per work list
+};
+
+__device__ __forceinline__ void record_error(WsHeader* h, int code) {
+  atomicCAS(&h->status, 0, code);
+}
+
+// ---------------------------------------------------------------- packed f32x2
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// A centroid broadcast into both halves of four packed registers.
+struct Cent2 {
+  uint64_t x, y, z, t;
+};
+__device__ __forceinline__ Cent2 cent2(float4 c) {
+  return Cent2{pack2(c.x, c.x), pack2(c.y, c.y), pack2(c.z, c.z), pack2(c.w, c.w)};
+}
+
+// Distances of two points (packed component-wise) to one centroid.
+__device__ __forceinline__ uint64_t dist2(uint64_t X, uint64_t Y, uint64_t Z, uint64_t T,
+                                          const Cent2& c) {
+  uint64_t dx = sub2(X, c.x);
+  uint64_t dy = sub2(Y, c.y);
+  uint64_t dz = sub2(Z, c.z);
+  uint64_t dt = sub2(T, c.t);
+  uint64_t s = add2(mul2(dx, dx), mul2(dy, dy));
+  s = add2(s, mul2(dz, dz));
+  s = add2(s, mul2(dt, dt));
+  return s;
+}
+
+// Scalar form of the same distance.
+__device__ __forceinline__ float dist1(float4 p, float4 c) {
+  float dx = __fsub_rn(p.x, c.x);
+  float dy = __fsub_rn(p.y, c.y);
+  float dz = __fsub_rn(p.z, c.z);
+  float dt = __fsub_rn(p.w, c.w);
+  float s = __fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy));
+  s = __fadd_rn(s, __fmul_rn(dz, dz));
+  s = __fadd_rn(s, __fmul_rn(dt, dt));
+  return s;
+}
+
+// Running-min / label update of one slot: strict '<' so that, over slots
+// visited in increasing order, the lowest slot wins ties.
+__device__ __forceinline__ void relax(float d, float& dist, int& lab, int s) {
+  lab = d < dist ? s : lab;
+  dist = fminf(dist, d);
+}
+
+__device__ __forceinline__ int fkey(float v) { return __float_as_int(v); }
+
+// Warp arg-max of (key, idx): the largest key, then the smallest idx among
+// the lanes holding it.  Both results are warp-uniform.
+__device__ __forceinline__ void warp_argmax(int key, unsigned idx, int& mkey, unsigned& midx) {
+  mkey = __reduce_max_sync(kFull, key);
+  midx = __reduce_min_sync(kFull, key == mkey ? idx : 0xffffffffu);
+}
+
+__device__ __forceinline__ float4 ldg4(const float4* p) { return __ldg(p); }
+
+}  // namespace fpstok

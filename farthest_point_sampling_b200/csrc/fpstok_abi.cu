@@ -1,0 +1,449 @@
+// C ABI of the fpstok tokenizer (declared in include/fpstok.h): argument
+// checks, workspace carving and the launch sequence.  No allocation, no
+// synchronisation (except fps_device_status, which exists to read back).
+#include <atomic>
+#include <cstring>
+
+#include "../../include/fpstok.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace fpstok {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static void* g_stage_events[16];
+static int g_n_stage_events = 0;
+
+void stage_mark(int stage, int end, cudaStream_t s) {
+  const int e = 2 * stage + end;
+  if (e < g_n_stage_events && g_stage_events[e])
+    cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_stage_events[e]), s);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t n) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align256(off + n * sizeof(T));
+    return p;
+  }
+};
+
+// Lays out the workspace; with base == nullptr only computes the size.
+static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, bool labels) {
+  Carver c{static_cast<char*>(base)};
+  Workspace w = {};
+  const int64_t nb = B > 0 ? B : 1;
+  const int64_t chunks = nb + P / kChunk + 1;
+  const int64_t pool_slots = P / kChunk + 1;
+  int64_t fps_slots = P / (K + 1) + 1;
+  if (fps_slots > nb) fps_slots = nb;
+  w.hdr = c.take<WsHeader>(1);
+  w.list_warp = c.take<int>(nb);
+  w.list_cta = c.take<int>(nb);
+  w.list_cluster = c.take<int>(nb);
+  w.chunks = c.take<int2>(chunks);
+  w.cls = c.take<int>(nb);
+  w.fps_slot = c.take<int>(nb);
+  w.pool_slot = c.take<int>(nb);
+  w.pool_acc = c.take<double>(pool_slots * K * (F > 0 ? F : 1));
+  w.pool_cnt = c.take<int>(pool_slots * K);
+  w.pool_ticket = c.take<int>(pool_slots);
+  for (int i = 0; i < 3; ++i) w.lloyd[i] = lloyd ? c.take<double>(fps_slots * K * 5) : nullptr;
+  w.labels = labels ? c.take<int>(P > 0 ? P : 1) : nullptr;
+  w.fps_slots = (int)fps_slots;
+  w.pool_slots = (int)pool_slots;
+  w.bytes = c.off;
+  return w;
+}
+
+static int from_cuda(cudaError_t e) { return e == cudaSuccess ? FPS_OK : FPS_ERR_CUDA; }
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static int check_common(int64_t P, int B, const int64_t* offsets) {
+  if (B < 0 || P < 0) return FPS_ERR_ARG;
+  if (P >= ((int64_t)1 << 31)) return FPS_ERR_TOO_LARGE;
+  if (B > 0 && offsets == nullptr) return FPS_ERR_ARG;
+  return FPS_OK;
+}
+
+static int check_opts(const fps_opts* o, int F) {
+  if (!o) return FPS_ERR_ARG;
+  if (o->K < 1) return FPS_ERR_ARG;
+  if (o->K > FPS_MAX_K) return FPS_ERR_TOO_LARGE;
+  if (o->assign_mode != FPS_ASSIGN_VORONOI && o->assign_mode != FPS_ASSIGN_KNN) return FPS_ERR_ARG;
+  if (o->assign_mode == FPS_ASSIGN_KNN) {
+    if (o->k < 1) return FPS_ERR_ARG;
+    if (o->k > o->K || o->k > FPS_MAX_KNN) return FPS_ERR_TOO_LARGE;
+  }
+  if (o->lloyd_iters < 0) return FPS_ERR_ARG;
+  if (F < 1) return FPS_ERR_ARG;
+  if (F > FPS_MAX_F) return FPS_ERR_TOO_LARGE;
+  if (o->charge_col < -1 || o->charge_col >= F) return FPS_ERR_ARG;
+  if (o->force_schedule < -1 || o->force_schedule > 2) return FPS_ERR_ARG;
+  if (o->max_event_hint < 0) return FPS_ERR_ARG;
+  if (o->max_event_hint > kClusterCap) return FPS_ERR_TOO_LARGE;
+  return FPS_OK;
+}
+
+static bool needs_labels(const fps_opts* o, const int32_t* token_id) {
+  return o->assign_mode == FPS_ASSIGN_KNN && o->lloyd_iters > 0 && token_id == nullptr;
+}
+
+static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s) {
+  Problem pb = pb0;
+  int32_t* labels = pb.token_id ? pb.token_id : ws.labels;
+  pb.token_id = labels;  // FPS writes the Voronoi labels here (may be null in plain kNN mode)
+  cudaError_t e;
+  stage_mark(0, 0, s);
+  if ((e = launch_bin(pb, ws, 0, s))) return from_cuda(e);
+  Problem pt = pb;
+  pt.token_id = pb0.token_id;
+  pt.knn_idx = pb.assign_mode == FPS_ASSIGN_KNN ? pb.knn_idx : nullptr;
+  if ((e = launch_passthrough(pt, ws, s))) return from_cuda(e);
+  stage_mark(0, 1, s);
+  if ((e = launch_fps(pb, ws, s, stage_mark))) return from_cuda(e);
+  if (pb.lloyd_iters > 0) {
+    stage_mark(4, 0, s);
+    if ((e = launch_lloyd(pb, ws, labels, s))) return from_cuda(e);
+    stage_mark(4, 1, s);
+  }
+  if (pb.assign_mode == FPS_ASSIGN_KNN) {
+    stage_mark(5, 0, s);
+    if ((e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx,
+                        pb.feats, pb.F, pb.pooled, pb.counts, ws.cls, ws.hdr, s)))
+      return from_cuda(e);
+    stage_mark(5, 1, s);
+  } else {
+    stage_mark(6, 0, s);
+    if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.K, labels, pb.pooled, pb.counts, ws, s)))
+      return from_cuda(e);
+    stage_mark(6, 1, s);
+  }
+  return FPS_OK;
+}
+
+}  // namespace fpstok
+
+using namespace fpstok;
+
+extern "C" {
+
+int64_t fps_max_event_points(void) { return kClusterCap; }
+
+int fps_schedule_for(int64_t n, int K, int force_schedule) {
+  if (n > kClusterCap) return -2;
+  if (n <= 0 || n <= K) return -1;
+  int sched = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : 2);
+  if (force_schedule > sched) sched = force_schedule > 2 ? 2 : force_schedule;
+  return sched;
+}
+
+size_t fps_workspace_bytes(int64_t P, int B, int F, const fps_opts* opts) {
+  if (!opts || P < 0 || B < 0 || opts->K < 1) return 0;
+  const bool lab = opts->assign_mode == FPS_ASSIGN_KNN && opts->lloyd_iters > 0;
+  return carve(nullptr, P, B, opts->K, F, opts->lloyd_iters > 0, lab).bytes;
+}
+
+int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* offsets, int B, int64_t P,
+                 const int32_t* start_local, const fps_opts* opts, int32_t* centroid_idx, int32_t* token_id,
+                 int32_t* knn_idx, float* centroids, float* pooled, int32_t* counts, void* workspace,
+                 size_t workspace_bytes, fps_stream_t stream) {
+  int rc = check_common(P, B, offsets);
+  if (rc) return rc;
+  if ((rc = check_opts(opts, F))) return rc;
+  if (B == 0) return FPS_OK;
+  if (!centroid_idx || !centroids || !pooled || !counts) return FPS_ERR_ARG;
+  if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id) return FPS_ERR_ARG;
+  if (opts->assign_mode == FPS_ASSIGN_KNN && !knn_idx) return FPS_ERR_ARG;
+  if (P > 0 && (!coords || !feats)) return FPS_ERR_ARG;
+  if (!aligned(coords, 16) || !aligned(centroids, 16)) return FPS_ERR_ARG;
+  const bool lab = needs_labels(opts, token_id);
+  const Workspace need = carve(nullptr, P, B, opts->K, F, opts->lloyd_iters > 0, lab);
+  if (!workspace || workspace_bytes < need.bytes || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  const Workspace ws = carve(workspace, P, B, opts->K, F, opts->lloyd_iters > 0, lab);
+  Problem pb = {reinterpret_cast<const float4*>(coords), feats, F, offsets, B, P, start_local,
+                opts->K, opts->assign_mode, opts->k, opts->lloyd_iters, opts->charge_col,
+                opts->force_schedule, opts->max_event_hint, centroid_idx, token_id,
+                opts->assign_mode == FPS_ASSIGN_KNN ? knn_idx : nullptr,
+                reinterpret_cast<float4*>(centroids), pooled, counts};
+  return run_tokenize(pb, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Host-pointer variant: staging layout after the regular workspace.
+struct HostStage {
+  size_t coords, feats, offsets, start, cidx, tok, knn, cents, pooled, counts, total;
+};
+
+static HostStage host_stage(size_t base, int64_t P, int B, int F, const fps_opts* o, bool has_start) {
+  HostStage h;
+  size_t off = align256(base);
+  auto take = [&](size_t n) {
+    const size_t at = off;
+    off = align256(off + n);
+    return at;
+  };
+  const int K = o->K;
+  const int k = o->assign_mode == FPS_ASSIGN_KNN ? o->k : 0;
+  h.coords = take((size_t)P * 16);
+  h.feats = take((size_t)P * F * 4);
+  h.offsets = take((size_t)(B + 1) * 8);
+  h.start = take(has_start ? (size_t)B * 4 : 0);
+  h.cidx = take((size_t)B * K * 4);
+  h.tok = take((size_t)P * 4);
+  h.knn = take((size_t)B * K * k * 4);
+  h.cents = take((size_t)B * K * 16);
+  h.pooled = take((size_t)B * K * F * 4);
+  h.counts = take((size_t)B * K * 4);
+  h.total = off;
+  return h;
+}
+
+size_t fps_host_workspace_bytes(int64_t P, int B, int F, const fps_opts* opts) {
+  const size_t base = fps_workspace_bytes(P, B, F, opts);
+  if (!base) return 0;
+  return host_stage(base, P, B, F, opts, true).total;
+}
+
+int fps_tokenize_host(const float* coords, const float* feats, int F, const int64_t* offsets, int B,
+                      int64_t P, const int32_t* start_local, const fps_opts* opts, int32_t* centroid_idx,
+                      int32_t* token_id, int32_t* knn_idx, float* centroids, float* pooled, int32_t* counts,
+                      void* workspace, size_t workspace_bytes, fps_stream_t stream) {
+  int rc = check_common(P, B, offsets);
+  if (rc) return rc;
+  if ((rc = check_opts(opts, F))) return rc;
+  if (B == 0) return FPS_OK;
+  if (!centroid_idx || !centroids || !pooled || !counts) return FPS_ERR_ARG;
+  if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id) return FPS_ERR_ARG;
+  if (opts->assign_mode == FPS_ASSIGN_KNN && !knn_idx) return FPS_ERR_ARG;
+  if (P > 0 && (!coords || !feats)) return FPS_ERR_ARG;
+  const size_t base = fps_workspace_bytes(P, B, F, opts);
+  const HostStage h = host_stage(base, P, B, F, opts, start_local != nullptr);
+  if (!workspace || workspace_bytes < h.total || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  char* w = static_cast<char*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int K = opts->K;
+  const int k = opts->assign_mode == FPS_ASSIGN_KNN ? opts->k : 0;
+  auto h2d = [&](size_t at, const void* src, size_t n) {
+    return n ? cudaMemcpyAsync(w + at, src, n, cudaMemcpyHostToDevice, s) : cudaSuccess;
+  };
+  auto d2h = [&](void* dst, size_t at, size_t n) {
+    return (n && dst) ? cudaMemcpyAsync(dst, w + at, n, cudaMemcpyDeviceToHost, s) : cudaSuccess;
+  };
+  cudaError_t e;
+  if ((e = h2d(h.coords, coords, (size_t)P * 16)) || (e = h2d(h.feats, feats, (size_t)P * F * 4)) ||
+      (e = h2d(h.offsets, offsets, (size_t)(B + 1) * 8)) ||
+      (e = h2d(h.start, start_local, start_local ? (size_t)B * 4 : 0)))
+    return from_cuda(e);
+  rc = fps_tokenize(reinterpret_cast<const float*>(w + h.coords), reinterpret_cast<const float*>(w + h.feats),
+                    F, reinterpret_cast<const int64_t*>(w + h.offsets), B, P,
+                    start_local ? reinterpret_cast<const int32_t*>(w + h.start) : nullptr, opts,
+                    reinterpret_cast<int32_t*>(w + h.cidx), token_id ? reinterpret_cast<int32_t*>(w + h.tok) : nullptr,
+                    k ? reinterpret_cast<int32_t*>(w + h.knn) : nullptr, reinterpret_cast<float*>(w + h.cents),
+                    reinterpret_cast<float*>(w + h.pooled), reinterpret_cast<int32_t*>(w + h.counts), workspace,
+                    base, stream);
+  if (rc) return rc;
+  if ((e = d2h(centroid_idx, h.cidx, (size_t)B * K * 4)) || (e = d2h(token_id, h.tok, (size_t)P * 4)) ||
+      (e = d2h(k ? knn_idx : nullptr, h.knn, (size_t)B * K * k * 4)) ||
+      (e = d2h(centroids, h.cents, (size_t)B * K * 16)) || (e = d2h(pooled, h.pooled, (size_t)B * K * F * 4)) ||
+      (e = d2h(counts, h.counts, (size_t)B * K * 4)))
+    return from_cuda(e);
+  return FPS_OK;
+}
+
+size_t fps_assign_workspace_bytes(int64_t P, int B) { return carve(nullptr, P, B, 1, 1, false, false).bytes; }
+
+int fps_assign(const float* coords, const int64_t* offsets, int B, int64_t P, const float* centroids,
+               const int32_t* valid_tokens, int K, int32_t* token_id, void* workspace, size_t workspace_bytes,
+               fps_stream_t stream) {
+  int rc = check_common(P, B, offsets);
+  if (rc) return rc;
+  if (K < 1) return FPS_ERR_ARG;
+  if (K > FPS_MAX_K) return FPS_ERR_TOO_LARGE;
+  if (B == 0 || P == 0) return FPS_OK;
+  if (!coords || !centroids || !token_id) return FPS_ERR_ARG;
+  if (!aligned(coords, 16) || !aligned(centroids, 16)) return FPS_ERR_ARG;
+  const size_t need = fps_assign_workspace_bytes(P, B);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  const Workspace ws = carve(workspace, P, B, 1, 1, false, false);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // every non-empty event becomes (event, chunk) items: K here only splits classes
+  Problem pb = {};
+  pb.offsets = offsets;
+  pb.B = B;
+  pb.P = P;
+  pb.K = K;
+  pb.force_schedule = -1;
+  cudaError_t e;
+  if ((e = launch_bin(pb, ws, 1, s))) return from_cuda(e);
+  return from_cuda(launch_assign(reinterpret_cast<const float4*>(coords), offsets,
+                                 reinterpret_cast<const float4*>(centroids), valid_tokens, K, token_id, ws, s));
+}
+
+size_t fps_knn_workspace_bytes(int64_t P, int B) {
+  (void)P;
+  (void)B;
+  return align256(sizeof(WsHeader));
+}
+
+int fps_knn(const float* coords, const int64_t* offsets, int B, int64_t P, const float* centroids,
+            const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, void* workspace, size_t workspace_bytes,
+            fps_stream_t stream) {
+  int rc = check_common(P, B, offsets);
+  if (rc) return rc;
+  if (K < 1 || k < 1) return FPS_ERR_ARG;
+  if (K > FPS_MAX_K || k > FPS_MAX_KNN) return FPS_ERR_TOO_LARGE;
+  if (B == 0) return FPS_OK;
+  if (!centroids || !knn_idx || (P > 0 && !coords)) return FPS_ERR_ARG;
+  if (!aligned(coords, 16) || !aligned(centroids, 16)) return FPS_ERR_ARG;
+  if (!workspace || workspace_bytes < fps_knn_workspace_bytes(P, B) || !aligned(workspace, 256))
+    return FPS_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+  return from_cuda(launch_knn(reinterpret_cast<const float4*>(coords), offsets, B,
+                              reinterpret_cast<const float4*>(centroids), valid_tokens, K, k, knn_idx, nullptr,
+                              0, nullptr, nullptr, nullptr, hdr, s));
+}
+
+size_t lloyd_workspace_bytes(int64_t P, int B, int K) {
+  if (K < 1) return 0;
+  return carve(nullptr, P, B, K, 1, true, false).bytes;
+}
+
+int lloyd_refine(const float* coords, const float* feats, int F, int charge_col, const int64_t* offsets, int B,
+                 int64_t P, int K, int iters, float* centroids, int32_t* token_id, void* workspace,
+                 size_t workspace_bytes, fps_stream_t stream) {
+  int rc = check_common(P, B, offsets);
+  if (rc) return rc;
+  if (K < 1 || iters < 0 || charge_col < -1) return FPS_ERR_ARG;
+  if (K > FPS_MAX_K) return FPS_ERR_TOO_LARGE;
+  if (charge_col >= 0 && (F < 1 || charge_col >= F || !feats)) return FPS_ERR_ARG;
+  if (B == 0 || P == 0 || iters == 0) return FPS_OK;
+  if (!coords || !centroids || !token_id) return FPS_ERR_ARG;
+  if (!aligned(coords, 16) || !aligned(centroids, 16)) return FPS_ERR_ARG;
+  const size_t need = lloyd_workspace_bytes(P, B, K);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  const Workspace ws = carve(workspace, P, B, K, 1, true, false);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Problem pb = {};
+  pb.coords = reinterpret_cast<const float4*>(coords);
+  pb.feats = feats;
+  pb.F = F;
+  pb.offsets = offsets;
+  pb.B = B;
+  pb.P = P;
+  pb.K = K;
+  pb.lloyd_iters = iters;
+  pb.charge_col = charge_col;
+  pb.force_schedule = -1;
+  pb.centroids = reinterpret_cast<float4*>(centroids);
+  cudaError_t e;
+  stage_mark(4, 0, s);
+  if ((e = launch_bin(pb, ws, 0, s))) return from_cuda(e);
+  const size_t zbytes = (size_t)ws.fps_slots * K * 5 * sizeof(double);
+  if ((e = cudaMemsetAsync(ws.lloyd[0], 0, zbytes, s)) || (e = cudaMemsetAsync(ws.lloyd[1], 0, zbytes, s)))
+    return from_cuda(e);
+  if ((e = launch_lloyd(pb, ws, token_id, s))) return from_cuda(e);
+  stage_mark(4, 1, s);
+  return FPS_OK;
+}
+
+size_t segment_pool_workspace_bytes(int64_t P, int B, int K, int F) {
+  if (K < 1 || F < 1) return 0;
+  return carve(nullptr, P, B, K, F, false, false).bytes;
+}
+
+int segment_pool(const float* feats, int F, const int64_t* offsets, int B, int64_t P, int K, int mode,
+                 const int32_t* token_id, const int32_t* knn_idx, int k, float* pooled, int32_t* counts,
+                 void* workspace, size_t workspace_bytes, fps_stream_t stream) {
+  if (B < 0 || P < 0) return FPS_ERR_ARG;
+  if (P >= ((int64_t)1 << 31)) return FPS_ERR_TOO_LARGE;
+  if (K < 1 || F < 1) return FPS_ERR_ARG;
+  if (K > FPS_MAX_K || F > FPS_MAX_F) return FPS_ERR_TOO_LARGE;
+  if (mode != FPS_ASSIGN_VORONOI && mode != FPS_ASSIGN_KNN) return FPS_ERR_ARG;
+  if (B == 0) return FPS_OK;
+  if (!pooled || !counts || (P > 0 && !feats)) return FPS_ERR_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (mode == FPS_ASSIGN_KNN) {
+    if (k < 1) return FPS_ERR_ARG;
+    if (k > FPS_MAX_KNN) return FPS_ERR_TOO_LARGE;
+    if (!knn_idx) return FPS_ERR_ARG;
+    if (!workspace || workspace_bytes < align256(sizeof(WsHeader)) || !aligned(workspace, 256))
+      return FPS_ERR_WORKSPACE;
+    WsHeader* hdr = static_cast<WsHeader*>(workspace);
+    if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+    return from_cuda(launch_pool_knn(feats, F, B, K, k, knn_idx, P, pooled, counts, hdr, s));
+  }
+  if (!offsets || (P > 0 && !token_id)) return FPS_ERR_ARG;
+  const size_t need = segment_pool_workspace_bytes(P, B, K, F);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  const Workspace ws = carve(workspace, P, B, K, F, false, false);
+  Problem pb = {};
+  pb.offsets = offsets;
+  pb.B = B;
+  pb.P = P;
+  pb.K = K;
+  pb.F = F;
+  pb.force_schedule = -1;
+  // empty rows first (events without points), then pooled rows of every event
+  if ((e = cudaMemsetAsync(pooled, 0, (size_t)B * K * F * sizeof(float), s)) ||
+      (e = cudaMemsetAsync(counts, 0, (size_t)B * K * sizeof(int32_t), s)))
+    return from_cuda(e);
+  if ((e = launch_bin(pb, ws, 1, s))) return from_cuda(e);
+  if ((e = cudaMemsetAsync(ws.pool_acc, 0, (size_t)ws.pool_slots * K * F * sizeof(double), s)) ||
+      (e = cudaMemsetAsync(ws.pool_cnt, 0, (size_t)ws.pool_slots * K * sizeof(int), s)) ||
+      (e = cudaMemsetAsync(ws.pool_ticket, 0, (size_t)ws.pool_slots * sizeof(int), s)))
+    return from_cuda(e);
+  return from_cuda(launch_pool_voronoi(feats, F, offsets, K, token_id, pooled, counts, ws, s));
+}
+
+int fps_device_status(void* workspace, fps_stream_t stream, int* detail) {
+  if (!workspace) return FPS_ERR_ARG;
+  WsHeader h;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(WsHeader), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return FPS_ERR_CUDA;
+  if (detail) *detail = h.status;
+  if (h.status == 0) return FPS_OK;
+  const int zero[2] = {0, 0};
+  cudaMemcpyAsync(workspace, zero, sizeof(zero), cudaMemcpyHostToDevice, s);
+  cudaStreamSynchronize(s);
+  return FPS_ERR_DEVICE;
+}
+
+const char* fps_status_string(int status) {
+  switch (status) {
+    case FPS_OK: return "ok";
+    case FPS_ERR_ARG: return "invalid argument";
+    case FPS_ERR_TOO_LARGE: return "size above a library limit";
+    case FPS_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case FPS_ERR_CUDA: return "CUDA launch or copy failed";
+    case FPS_ERR_DEVICE: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+uint64_t fps_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void fps_set_stage_events(void* const* events, int n_events) {
+  if (!events || n_events <= 0) {
+    g_n_stage_events = 0;
+    return;
+  }
+  if (n_events > 16) n_events = 16;
+  for (int i = 0; i < n_events; ++i) g_stage_events[i] = events[i];
+  g_n_stage_events = n_events;
+}
+
+}  // extern "C"

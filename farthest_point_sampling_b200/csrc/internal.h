@@ -1,0 +1,101 @@
+// Internal host-side interfaces between the C ABI and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fpstok {
+
+// Event classes written by the binning kernel.
+enum EventClass : int { kClsSkip = 0, kClsEmpty = 1, kClsPass = 2, kClsFps = 3 };
+
+// Work lists (indices into WsHeader::n_items).
+enum ListId : int {
+  kListWarp = 0,
+  kListCta = 1,
+  kListCluster = 2,
+  kListChunks = 3,     // (event, chunk) items of FPS events
+  kListPoolSlots = 4,  // events that need global pooling accumulators
+  kListFps = 5,        // number of FPS events (Lloyd slots)
+};
+
+// Schedule capacities (points per event).
+constexpr int kWarpPPL = 14;                  // points per lane, warp schedule
+constexpr int kWarpCap = 32 * kWarpPPL;       // 448
+constexpr int kBlockThreads = 512;            // CTA / cluster schedules
+constexpr int kBlockPairs = 12;               // point pairs per thread (shared memory)
+constexpr int kCtaCap = kBlockThreads * 2 * kBlockPairs;  // 12288
+constexpr int kMaxCluster = 16;
+constexpr int kClusterCap = kMaxCluster * kCtaCap;        // 196608
+constexpr int kChunk = 2048;                  // points per pooling / Lloyd work item
+
+struct Workspace {
+  struct WsHeader* hdr;
+  int* list_warp;
+  int* list_cta;
+  int* list_cluster;
+  int2* chunks;     // (event, chunk)
+  int* cls;         // EventClass per event
+  int* fps_slot;    // compact index of FPS events, -1 otherwise
+  int* pool_slot;   // compact index of multi-chunk FPS events, -1 otherwise
+  double* pool_acc; // [pool slots][K][F]
+  int* pool_cnt;    // [pool slots][K]
+  int* pool_ticket; // [pool slots]
+  double* lloyd[3]; // 3 x [fps slots][K][5]
+  int* labels;      // [P] internal Voronoi labels (kNN mode with Lloyd)
+  int fps_slots;    // capacity of the Lloyd slot range
+  int pool_slots;   // capacity of the pooling slot range
+  size_t bytes;
+};
+
+struct Problem {
+  const float4* coords;
+  const float* feats;
+  int F;
+  const int64_t* offsets;
+  int B;
+  int64_t P;
+  const int32_t* start_local;
+  int K, assign_mode, k, lloyd_iters, charge_col, force_schedule, max_event_hint;
+  int32_t* centroid_idx;
+  int32_t* token_id;
+  int32_t* knn_idx;
+  float4* centroids;
+  float* pooled;
+  int32_t* counts;
+};
+
+// Kernel launchers (return the cudaError_t of the launch).
+cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s);
+cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s);
+typedef void (*StageMark)(int stage, int end, cudaStream_t s);
+void stage_mark(int stage, int end, cudaStream_t s);
+cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, StageMark mark);
+cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s);
+cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
+                                const int32_t* labels, float* pooled, int32_t* counts,
+                                const Workspace& ws, cudaStream_t s);
+cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
+                       const int32_t* valid_tokens, int K, int k, int32_t* knn_idx,
+                       const float* feats, int F, float* pooled, int32_t* counts, const int* cls,
+                       struct WsHeader* hdr, cudaStream_t s);
+cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const float4* centroids,
+                          const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,
+                          cudaStream_t s);
+cudaError_t launch_pool_knn(const float* feats, int F, int B, int K, int k, const int32_t* knn_idx,
+                            int64_t P, float* pooled, int32_t* counts, struct WsHeader* hdr,
+                            cudaStream_t s);
+
+// Device properties cached per device.
+struct DeviceInfo {
+  int sm_count;
+  int warp_blocks_per_sm;
+  int cluster_max_active;  // clusters of kMaxCluster CTAs of the cluster kernel
+  bool ready;
+};
+const DeviceInfo& device_info();  // prepares the current device on first use
+cudaError_t prepare_aux_kernels();   // shared-memory attributes of the auxiliary kernels
+
+void count_launch(int n = 1);
+
+}  // namespace fpstok

@@ -1,0 +1,225 @@
+/*
+ * fpstok: batched 4D farthest-point-sampling tokenizer on B200 (sm_100a).
+ *
+ * What the library computes follows the Neptune tokenizer as the pages state it:
+ *   - Neptune README, "How it works", step 1 (Tokenization): farthest-point
+ *     sampling down to num_patches (K) centroids, then per-token pooling by
+ *     nearest-centroid (Voronoi) assignment or a k-NN gather
+ *     (assign_mode="knn", k_neighbors), with optional charge-weighted Lloyd
+ *     refinement of the centroids (lloyd_iters).
+ *   - graphnet PR #923 "Add Neptune point-transformer backbone", "What is
+ *     added": FPSTokenizer keeps one token per pulse for small events;
+ *     components/fps.py provides farthest_point_sampling, the _with_assign and
+ *     _with_knn variants, and nearest_assign.  Review thread on the FPS
+ *     `precision` argument: computation is float32 only.  Review thread on
+ *     the no-charge case: unit charge when no charge column is given.
+ *   - Neptune README, "Usage": coords [N, 4] = (x, y, z, t) with time in the
+ *     fourth column, features [N, F], per-point event ids.
+ *
+ * Exact semantics (readings where the pages are silent):
+ *   d(i, c) = ((dx*dx + dy*dy) + dz*dz) + dt*dt in float32, each operation
+ *   rounded to nearest-even, never fused; first centroid = start_local[b]
+ *   (default 0); each next centroid = the unselected point with the largest
+ *   running minimum distance, lowest index on ties (when every unselected
+ *   point is at distance 0, the lowest-index unselected point); Voronoi label
+ *   = nearest centroid, lowest slot on ties; kNN row = the k points with the
+ *   smallest (d, index), ascending, -1 padded; pooling = arithmetic mean of
+ *   every feature column plus a count; Lloyd: c_j = sum(q p) / sum(q) over
+ *   the cell (q = features[:, charge_col] or 1), c_j kept when the cell is
+ *   empty or its weight <= 0, then re-assign; sums accumulate in float64 and
+ *   round once to float32.  Indices, labels and kNN ids are exact; pooled
+ *   values and Lloyd centroids agree with a sequential float64 sum to well
+ *   within 1e-5 relative (1e-6 absolute floor).
+ *
+ * Layout (all row-major, packed by event):
+ *   coords   float32 [P, 4], 16-byte aligned; event b is rows
+ *            offsets[b] .. offsets[b+1]-1.
+ *   feats    float32 [P, F], F >= 1.
+ *   offsets  int64 [B + 1], offsets[0] = 0, non-decreasing, offsets[B] = P.
+ *
+ * Outputs per event b with N = offsets[b+1] - offsets[b] points:
+ *   N == 0      : no tokens; rows are -1 (indices) or 0 (floats, counts).
+ *   N <= K      : passthrough, token j is point j (j < N): centroid_idx =
+ *                 offsets[b] + j, token_id = local index, kNN row =
+ *                 [point, -1, ...], pooled = that point's features, count 1.
+ *   N  > K      : K tokens from FPS; Lloyd applies only to these events.
+ *   centroid_idx int32 [B, K]  global packed indices of the FPS points, -1 pad.
+ *   token_id     int32 [P]     local token slot 0..K-1 of every point.
+ *   knn_idx      int32 [B,K,k] global packed indices, -1 pad.
+ *   centroids    float32 [B,K,4] centroid positions (Lloyd-refined if any).
+ *   pooled       float32 [B,K,F], counts int32 [B, K].
+ *
+ * Ownership and execution: every pointer is a caller-owned buffer; the
+ * library never allocates, frees or synchronises.  Unless stated otherwise
+ * pointers are DEVICE pointers and all work is enqueued on `stream`.  Scratch
+ * space is the caller's `workspace` (device, 256-byte aligned) of at least the
+ * size the matching *_workspace_bytes() call returns.
+ *
+ * Errors: every call returns FPS_OK or an FPS_ERR_* code.  Argument errors
+ * are found on the host before anything is launched.  Problems only visible
+ * on the device (inconsistent offsets, a start index outside its event, a
+ * token id outside 0..K-1) make the kernels skip the offending event and
+ * record a code in the workspace; fps_device_status() reads it back (this
+ * one call synchronises the stream).
+ */
+#ifndef FPSTOK_H
+#define FPSTOK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fps_stream_t; /* same type as cudaStream_t */
+
+enum {
+    FPS_OK = 0,
+    FPS_ERR_ARG = 1,        /* null pointer, bad size, bad mode, misaligned */
+    FPS_ERR_TOO_LARGE = 2,  /* K > FPS_MAX_K, k > K or > FPS_MAX_KNN, P >= 2^31,
+                               an event above FPS_MAX_EVENT points, F > FPS_MAX_F */
+    FPS_ERR_WORKSPACE = 3,  /* workspace missing, too small or misaligned */
+    FPS_ERR_CUDA = 4,       /* a CUDA launch or copy failed */
+    FPS_ERR_DEVICE = 5      /* a device-side check failed (fps_device_status) */
+};
+
+#define FPS_MAX_K 256
+#define FPS_MAX_KNN 128
+#define FPS_MAX_F 64
+
+/* assign_mode */
+#define FPS_ASSIGN_VORONOI 0
+#define FPS_ASSIGN_KNN 1
+
+/* force_schedule: -1 picks by event size; 0 warp, 1 CTA, 2 cluster means "use
+ * at least this schedule" (events too large for it move up). */
+typedef struct fps_opts {
+    int K;             /* maximum tokens per event, 1..FPS_MAX_K */
+    int assign_mode;   /* FPS_ASSIGN_VORONOI or FPS_ASSIGN_KNN */
+    int k;             /* kNN size, 1..min(K, FPS_MAX_KNN); ignored for Voronoi */
+    int lloyd_iters;   /* >= 0 */
+    int charge_col;    /* feature column used as Lloyd weight; -1 = unit weight */
+    int force_schedule;
+    int max_event_hint;/* upper bound on the largest event's N, 0 = unknown */
+} fps_opts;
+
+/* Largest event (points) the FPS schedules accept. */
+int64_t fps_max_event_points(void);
+
+/* Workspace bytes fps_tokenize needs for P points, B events and these options. */
+size_t fps_workspace_bytes(int64_t P, int B, int F, const fps_opts *opts);
+
+/*
+ * The whole tokenizer: FPS (fused with the Voronoi labels) -> optional Lloyd
+ * -> Voronoi mean-pool, or kNN gather around the final centroids and kNN
+ * mean-pool.  start_local: int32 [B] local start index per event, or NULL for
+ * 0.  token_id is required for Voronoi and optional (NULL) for kNN, where it
+ * receives the Voronoi labels when given.  knn_idx is required for kNN and
+ * ignored for Voronoi.  feats is required (F >= 1).
+ */
+int fps_tokenize(const float *coords, const float *feats, int F, const int64_t *offsets, int B,
+                 int64_t P, const int32_t *start_local, const fps_opts *opts,
+                 int32_t *centroid_idx, int32_t *token_id, int32_t *knn_idx, float *centroids,
+                 float *pooled, int32_t *counts, void *workspace, size_t workspace_bytes,
+                 fps_stream_t stream);
+
+/*
+ * Same as fps_tokenize but every input and output pointer is a HOST pointer
+ * (page-locked memory gives asynchronous copies).  The inputs are staged into
+ * the device workspace, the tokenizer runs there and the outputs are copied
+ * back, all on `stream`; the results are valid once the stream is
+ * synchronised.  Workspace size: fps_host_workspace_bytes().
+ */
+size_t fps_host_workspace_bytes(int64_t P, int B, int F, const fps_opts *opts);
+int fps_tokenize_host(const float *coords, const float *feats, int F, const int64_t *offsets,
+                      int B, int64_t P, const int32_t *start_local, const fps_opts *opts,
+                      int32_t *centroid_idx, int32_t *token_id, int32_t *knn_idx,
+                      float *centroids, float *pooled, int32_t *counts, void *workspace,
+                      size_t workspace_bytes, fps_stream_t stream);
+
+/*
+ * Nearest-centroid assignment (components/fps.py nearest_assign):
+ * token_id[i] = argmin over the event's first valid_tokens[b] centroid rows of
+ * d(p_i, c_j), lowest slot on ties; -1 when the event has no valid row.
+ * centroids float32 [B, K, 4]; valid_tokens int32 [B] or NULL for min(N, K).
+ */
+size_t fps_assign_workspace_bytes(int64_t P, int B);
+int fps_assign(const float *coords, const int64_t *offsets, int B, int64_t P,
+               const float *centroids, const int32_t *valid_tokens, int K, int32_t *token_id,
+               void *workspace, size_t workspace_bytes, fps_stream_t stream);
+
+/*
+ * kNN gather: for every valid centroid row j of event b, the k points of the
+ * event with the smallest (d(p_i, c_j), i), ascending, as global indices,
+ * -1 padded when the event has fewer than k points; invalid rows are all -1.
+ */
+size_t fps_knn_workspace_bytes(int64_t P, int B);
+int fps_knn(const float *coords, const int64_t *offsets, int B, int64_t P,
+            const float *centroids, const int32_t *valid_tokens, int K, int k,
+            int32_t *knn_idx, void *workspace, size_t workspace_bytes, fps_stream_t stream);
+
+/*
+ * Charge-weighted Lloyd refinement (README "How it works", step 1) of the
+ * events with N > K: `iters` times, every centroid moves to the weighted mean
+ * of its cell (q = feats[:, charge_col], or 1 when charge_col = -1; kept when
+ * the cell is empty or its weight <= 0) and every point is re-assigned.
+ * centroids [B,K,4] and token_id [P] are read and updated in place; events
+ * with N <= K are left untouched.  feats may be NULL when charge_col = -1.
+ */
+size_t lloyd_workspace_bytes(int64_t P, int B, int K);
+int lloyd_refine(const float *coords, const float *feats, int F, int charge_col,
+                 const int64_t *offsets, int B, int64_t P, int K, int iters, float *centroids,
+                 int32_t *token_id, void *workspace, size_t workspace_bytes, fps_stream_t stream);
+
+/*
+ * Per-token mean-pool ("pools the pulses of each token", graphnet PR #923,
+ * Summary).  mode FPS_ASSIGN_VORONOI: pooled[b,j,:] = mean of feats over the
+ * points of event b with token_id == j (token_id -1 = unassigned, skipped).
+ * mode FPS_ASSIGN_KNN: pooled[b,j,:] = mean of feats over the non-negative
+ * entries of knn_idx[b,j,:] (k entries per row; `offsets` may be NULL).
+ * Empty tokens give 0 and count 0.
+ */
+size_t segment_pool_workspace_bytes(int64_t P, int B, int K, int F);
+int segment_pool(const float *feats, int F, const int64_t *offsets, int B, int64_t P, int K,
+                 int mode, const int32_t *token_id, const int32_t *knn_idx, int k,
+                 float *pooled, int32_t *counts, void *workspace, size_t workspace_bytes,
+                 fps_stream_t stream);
+
+/* Reads (and clears) the device-side status word in `workspace`; synchronises
+ * `stream`.  Returns FPS_OK or FPS_ERR_DEVICE; *detail (optional) receives the
+ * recorded reason (see FPS_DEV_* below). */
+int fps_device_status(void *workspace, fps_stream_t stream, int *detail);
+
+#define FPS_DEV_BAD_OFFSETS 1
+#define FPS_DEV_BAD_START 2
+#define FPS_DEV_BAD_TOKEN 3
+#define FPS_DEV_TOO_LARGE 4
+
+/* Human-readable name of a status code. */
+const char *fps_status_string(int status);
+
+/* Number of kernels this library has launched in this process (a counter
+ * for measurement; it is not reset). */
+uint64_t fps_launch_count(void);
+
+/*
+ * Measurement hook: when `events` is non-NULL the next calls record
+ * events[2*s] before and events[2*s+1] after internal stage s on the
+ * launching stream.  Stages: 0 binning + passthrough, 1 FPS warp schedule,
+ * 2 FPS CTA schedule, 3 FPS cluster schedule, 4 Lloyd, 5 kNN gather + pool,
+ * 6 Voronoi pool.  A stage that does not run records nothing.  The events
+ * are cudaEvent_t handles the caller created; at most 16 are used.  Pass
+ * NULL to turn it off.  Not thread-safe: meant for benchmarks.
+ */
+void fps_set_stage_events(void *const *events, int n_events);
+
+/* Schedule fps_tokenize gives an event of n points: -1 none (n <= K, or n = 0),
+ * 0 warp, 1 CTA, 2 cluster; -2 if n exceeds fps_max_event_points(). */
+int fps_schedule_for(int64_t n, int K, int force_schedule);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FPSTOK_H */
