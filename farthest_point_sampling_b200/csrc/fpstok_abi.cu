@@ -161,7 +161,7 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
   if ((rc = check_opts(opts, F))) return rc;
   if (B == 0) return FPS_OK;
   if (!centroid_idx || !centroids || !pooled || !counts) return FPS_ERR_ARG;
-  if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id) return FPS_ERR_ARG;
+  if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id && P > 0) return FPS_ERR_ARG;
   if (opts->assign_mode == FPS_ASSIGN_KNN && !knn_idx) return FPS_ERR_ARG;
   if (P > 0 && (!coords || !feats)) return FPS_ERR_ARG;
   if (!aligned(coords, 16) || !aligned(centroids, 16)) return FPS_ERR_ARG;
@@ -221,7 +221,7 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
   if ((rc = check_opts(opts, F))) return rc;
   if (B == 0) return FPS_OK;
   if (!centroid_idx || !centroids || !pooled || !counts) return FPS_ERR_ARG;
-  if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id) return FPS_ERR_ARG;
+  if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id && P > 0) return FPS_ERR_ARG;
   if (opts->assign_mode == FPS_ASSIGN_KNN && !knn_idx) return FPS_ERR_ARG;
   if (P > 0 && (!coords || !feats)) return FPS_ERR_ARG;
   const size_t base = fps_workspace_bytes(P, B, F, opts);
