@@ -139,6 +139,26 @@ int fps_tokenize_host(const float *coords, const float *feats, int F, const int6
                       size_t workspace_bytes, fps_stream_t stream);
 
 /*
+ * fps_tokenize for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this exists for callers embedded in a host program
+ * that owns all device memory and may not call cudaMalloc or an allocating
+ * library routine, or that cannot accept the synchronisation cudaMalloc can
+ * cause.  Same arguments and results as fps_tokenize, without the workspace:
+ * the scratch is a file-scope device array of FPS_STATIC_SCRATCH_BYTES
+ * (8 MiB) that every GPU loading the library holds until the process exits.
+ * Returns FPS_ERR_TOO_LARGE when the batch needs more scratch than that
+ * (fps_workspace_bytes() tells how much it needs).  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress); make it
+ * before any stream capture.  All calls share the array: calls whose work
+ * overlaps on the GPU race.  It allocates and frees nothing.
+ */
+#define FPS_STATIC_SCRATCH_BYTES (8u << 20)
+int fps_tokenize_static(const float *coords, const float *feats, int F, const int64_t *offsets,
+                        int B, int64_t P, const int32_t *start_local, const fps_opts *opts,
+                        int32_t *centroid_idx, int32_t *token_id, int32_t *knn_idx,
+                        float *centroids, float *pooled, int32_t *counts, fps_stream_t stream);
+
+/*
  * Nearest-centroid assignment (components/fps.py nearest_assign):
  * token_id[i] = argmin over the event's first valid_tokens[b] centroid rows of
  * d(p_i, c_j), lowest slot on ties; -1 when the event has no valid row.
