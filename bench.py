@@ -37,10 +37,13 @@ import workloads  # noqa: E402
 FP32_OPS_PER_EVAL = 11  # 4 sub + 4 mul + 3 add
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
+FP32_OPS_PER_LANE_CLK = 2  # packed f32x2 add/sub/mul: two float32 operations per lane per clock
 SM_MAX_MHZ_NOMINAL = 1965.0
-STAGES = ["bin+passthrough", "fps_warp", "fps_cta", "fps_cluster", "lloyd", "knn+pool", "voronoi_pool"]
-STAGE_KERNELS = {0: "k_bin+k_passthrough", 1: "k_fps_warp", 2: "k_fps_block<1>", 3: "k_fps_block<16>",
-                 4: "k_lloyd_sums+k_lloyd_step", 5: "k_knn", 6: "k_pool_voronoi"}
+STAGES = ["bin+passthrough", "fps_warp", "fps_cta", "fps_cta_smem", "fps_cluster", "lloyd", "knn+pool",
+          "voronoi_pool"]
+STAGE_KERNELS = {0: "k_bin+k_passthrough", 1: "k_fps_warp", 2: "k_fps_cta", 3: "k_fps_block<1>",
+                 4: "k_fps_block<16>", 5: "k_lloyd_sums+k_lloyd_step", 6: "k_knn", 7: "k_pool_voronoi"}
+FPS_STAGES = (1, 2, 3, 4)
 METRIC = "FPS+assign events/s (K=128)"
 
 
@@ -56,6 +59,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-microbench", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls only")
     return ap.parse_args()
 
 
@@ -298,19 +304,32 @@ def main():
     kw = dict(K=batch.K, assign_mode=batch.assign_mode, k=max(batch.k, 1), lloyd_iters=batch.lloyd_iters,
               charge_col=batch.charge_col, max_event_hint=hint)
     out = fps.fps_tokenize(coords, feats, offsets, check_device=True, **kw)
-    ws = torch.empty(0, dtype=torch.uint8, device=dev)
     lib = fps.load_library()
     import ctypes
 
-    opts = fps.Options(**{k: v for k, v in kw.items()})
+    opts = fps.Options(**kw)
     ws = torch.empty(lib.fps_workspace_bytes(batch.P, batch.B, batch.F, ctypes.byref(opts.c)), dtype=torch.uint8,
                      device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    vp = ctypes.c_void_p
 
-    def step():
-        fps.fps_tokenize(coords, feats, offsets, workspace=ws, out=out, **kw)
+    def make_call(strm):
+        """One fps_tokenize call with every argument prebuilt (no Python checks)."""
+        args = (vp(coords.data_ptr()), vp(feats.data_ptr()), batch.F, vp(offsets.data_ptr()), batch.B, batch.P,
+                None, ctypes.byref(opts.c), vp(out["centroid_idx"].data_ptr()), vp(out["token_id"].data_ptr()),
+                vp(out["knn_idx"].data_ptr()) if "knn_idx" in out else None, vp(out["centroids"].data_ptr()),
+                vp(out["pooled"].data_ptr()), vp(out["counts"].data_ptr()), vp(ws.data_ptr()), ws.numel(),
+                vp(strm.cuda_stream))
+        fn = lib.fps_tokenize
 
+        def call():
+            rc = fn(*args)
+            if rc:
+                raise fps.FpsError(rc, "fps_tokenize")
+        return call
+
+    step = make_call(stream)
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -323,6 +342,7 @@ def main():
     for evs in stage_ev:  # materialise the handles the library records into
         for e in evs:
             e.record(stream)
+    stage_arr = [(vp * len(evs))(*[vp(e.cuda_event) for e in evs]) for evs in stage_ev]
     torch.cuda.synchronize(dev)
 
     if world > 1:
@@ -333,25 +353,52 @@ def main():
     with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as clocks:
         for i in range(K):
             flush.zero_()
-            fps.set_stage_events(stage_ev[i])
+            lib.fps_set_stage_events(stage_arr[i], len(STAGES) * 2)
             starts[i].record(stream)
             step()
             ends[i].record(stream)
-        fps.set_stage_events(None)
+        lib.fps_set_stage_events(None, 0)
         torch.cuda.synchronize(dev)
-    wall = time.perf_counter() - wall0
-    launches = fps.launch_count() - launches0
+        wall = time.perf_counter() - wall0
+        launches = fps.launch_count() - launches0
+        launches_per_step = launches / K
+        eager_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / K
+
+        # the same step replayed from a CUDA graph (launch overhead removed)
+        graph_ms = None
+        if not args.no_graph:
+            g = torch.cuda.CUDAGraph()
+            cap_stream = torch.cuda.Stream(dev)
+            cap_stream.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap_stream):
+                make_call(cap_stream)()
+            torch.cuda.synchronize(dev)
+            for _ in range(args.warmup):
+                flush.zero_()
+                g.replay()
+            torch.cuda.synchronize(dev)
+            if world > 1:
+                dist.barrier()
+            gs = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+            ge = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+            for i in range(K):
+                flush.zero_()
+                gs[i].record(stream)
+                g.replay()
+                ge[i].record(stream)
+            torch.cuda.synchronize(dev)
+            graph_ms = sum(a.elapsed_time(b) for a, b in zip(gs, ge)) / K
+            del g
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
 
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    best_ms = graph_ms if graph_ms is not None else eager_ms
+    t = torch.tensor([best_ms, eager_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    ms_per_step, eager_ms = float(t[0].item()), float(t[1].item())
     events_all = full.B
-    ms_per_step = total_ms / K
     value = events_all / (ms_per_step / 1e3)
     evals, _ = algorithmic(full)
 
@@ -369,10 +416,10 @@ def main():
     # stages that did not run in this workload keep their warm-up recordings: drop them
     sizes = batch.sizes()
     sched = np.array([lib.fps_schedule_for(int(n), batch.K, -1) for n in sizes])
-    ran = {0, 6 if batch.assign_mode == 0 else 5}
-    ran |= {1 + s for s in (0, 1, 2) if (sched == s).any()}
+    ran = {0, 7 if batch.assign_mode == 0 else 6}
+    ran |= {1 + s for s in (0, 1, 2, 3) if (sched == s).any()}
     if batch.lloyd_iters:
-        ran.add(4)
+        ran.add(5)
     stage_ms = {s: v for s, v in stage_ms.items() if s in ran}
 
     result = {
@@ -381,7 +428,10 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded generator shaped like the pages' events)",
         "config": config_of(batch, args, l2="flushed between steps (256 MiB write outside the timed events)"),
         "gevals_per_s": evals / (ms_per_step / 1e3) / 1e9,
-        "gpu_launches": int(launches),
+        "gpu_launches": int(round(launches_per_step * K)),
+        "timing": {"graph_replay_ms_per_step": graph_ms, "eager_ms_per_step": eager_ms,
+                   "value_from": "graph replay" if graph_ms is not None else "eager calls",
+                   "kernels_per_step": launches_per_step},
         "stage_ms": {STAGES[s]: round(v, 5) for s, v in sorted(stage_ms.items())},
         "wall_s_timed_region": wall,
     }
@@ -390,13 +440,13 @@ def main():
         # roofline of the dominant kernel (FP32 issue bound for the FPS kernels)
         dom = max(stage_ms, key=stage_ms.get)
         t_dom = stage_ms[dom] / 1e3
-        peak = SM_COUNT * FP32_LANES_PER_SM * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
-        if dom in (1, 2, 3):
+        peak = SM_COUNT * FP32_LANES_PER_SM * FP32_OPS_PER_LANE_CLK * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
+        if dom in FPS_STAGES:
             ev = int(sum(int(n) * batch.K for n, s in zip(sizes, sched) if s == dom - 1))
             achieved = ev * FP32_OPS_PER_EVAL / t_dom / 1e12
             roof = {"bound": "alu", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 1965 MHz (non-FMA float32 ops)",
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 (f32x2) x 1965 MHz, non-FMA float32 ops",
                     "algorithmic": f"{ev} point-centroid evals x {FP32_OPS_PER_EVAL} FP32 ops per launch",
                     "traffic": recorded_traffic(dom, args.workload)}
         else:
@@ -409,10 +459,12 @@ def main():
             achieved = byts / t_dom / 1e9
             roof = {"bound": "hbm", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": hbm,
                     "unit": "GB/s", "frac": achieved / hbm, "traffic": recorded_traffic(dom, args.workload)}
-        roof["microbench_fp32_tflops"] = microbench_fp32(dev)
+        if not args.no_microbench:
+            roof["microbench_fp32_tflops"] = microbench_fp32(dev)
         result["roofline"] = roof
         result["clocks"] = clocks.summary()
-        result["e2e"] = e2e(fps, batch, kw, dev, args.e2e_steps)
+        if not args.no_e2e:
+            result["e2e"] = e2e(fps, batch, kw, dev, args.e2e_steps)
         if world == 1 and not args.no_cpu_baseline:
             rate, reps, el = cpu_oracle_rate(batch, args.cpu_seconds)
             result["cpu_baseline"] = {"value": rate, "unit": "events/s", "cores": 1, "kind": "oracle",

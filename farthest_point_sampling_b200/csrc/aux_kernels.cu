@@ -24,8 +24,8 @@ namespace fpstok {
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
                                                int force, int chunk_all, Workspace ws) {
-  __shared__ int cnt[8];
-  if (threadIdx.x < 8) cnt[threadIdx.x] = 0;
+  __shared__ int cnt[kNumLists];
+  if (threadIdx.x < kNumLists) cnt[threadIdx.x] = 0;
   if (threadIdx.x == 0) {
     ws.hdr->status = 0;
     ws.hdr->detail = 0;
@@ -56,9 +56,10 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     ws.cls[b] = cls;
     int fslot = -1, pslot = -1;
     if (cls == kClsFps) {
-      int sched = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : 2);
-      if (force > sched) sched = force > 2 ? 2 : force;
-      int* list = sched == 0 ? ws.list_warp : (sched == 1 ? ws.list_cta : ws.list_cluster);
+      int sched = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : 3));
+      if (force > sched) sched = force > 3 ? 3 : force;
+      int* list = sched == 0 ? ws.list_warp
+                             : (sched == 1 ? ws.list_cta : (sched == 2 ? ws.list_cta_smem : ws.list_cluster));
       list[atomicAdd(&cnt[sched], 1)] = b;
       fslot = atomicAdd(&cnt[kListFps], 1);
     }
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     ws.pool_slot[b] = pslot;
   }
   __syncthreads();
-  if (threadIdx.x < 8) ws.hdr->n_items[threadIdx.x] = cnt[threadIdx.x];
+  if (threadIdx.x < kNumLists) ws.hdr->n_items[threadIdx.x] = cnt[threadIdx.x];
 }
 
 cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s) {
@@ -85,24 +86,23 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
 // ------------------------------------------------------------------ passthrough
 
 // Events with N <= K keep one token per pulse; empty and skipped events get
-// empty rows; FPS events get their global accumulators cleared.
+// empty rows; FPS events get their global accumulators cleared.  One CTA per
+// event (grid-stride), copies unrolled so that loads overlap.
 __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, int lloyd_on) {
-  const int lane = threadIdx.x & 31;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
   const int K = pb.K, F = pb.F, k = pb.k;
-  for (int b = gw; b < pb.B; b += nw) {
+  const int T = blockDim.x;
+  for (int b = blockIdx.x; b < pb.B; b += gridDim.x) {
     const int cls = ws.cls[b];
     if (cls == kClsFps) {
       const int ps = ws.pool_slot[b];
       if (ps >= 0) {
-        for (int e = lane; e < K * F; e += 32) ws.pool_acc[(int64_t)ps * K * F + e] = 0.0;
-        for (int e = lane; e < K; e += 32) ws.pool_cnt[(int64_t)ps * K + e] = 0;
-        if (lane == 0) ws.pool_ticket[ps] = 0;
+        for (int e = threadIdx.x; e < K * F; e += T) ws.pool_acc[(int64_t)ps * K * F + e] = 0.0;
+        for (int e = threadIdx.x; e < K; e += T) ws.pool_cnt[(int64_t)ps * K + e] = 0;
+        if (threadIdx.x == 0) ws.pool_ticket[ps] = 0;
       }
       const int fs = ws.fps_slot[b];
       if (lloyd_on && fs >= 0) {
-        for (int e = lane; e < K * 5; e += 32) {
+        for (int e = threadIdx.x; e < K * 5; e += T) {
           ws.lloyd[0][(int64_t)fs * K * 5 + e] = 0.0;
           ws.lloyd[1][(int64_t)fs * K * 5 + e] = 0.0;
         }
@@ -117,18 +117,20 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
     }
     const float* cf = reinterpret_cast<const float*>(pb.coords);
     float* outc = reinterpret_cast<float*>(pb.centroids) + (int64_t)b * K * 4;
-    for (int e = lane; e < K * 4; e += 32) outc[e] = e < n * 4 ? cf[off * 4 + e] : 0.f;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < K * 4; e += T) outc[e] = e < n * 4 ? cf[off * 4 + e] : 0.f;
     float* outp = pb.pooled + (int64_t)b * K * F;
-    for (int e = lane; e < K * F; e += 32) outp[e] = e < n * F ? pb.feats[off * F + e] : 0.f;
-    for (int j = lane; j < K; j += 32) {
+#pragma unroll 4
+    for (int e = threadIdx.x; e < K * F; e += T) outp[e] = e < n * F ? pb.feats[off * F + e] : 0.f;
+    for (int j = threadIdx.x; j < K; j += T) {
       pb.centroid_idx[(int64_t)b * K + j] = j < n ? (int32_t)(off + j) : -1;
       pb.counts[(int64_t)b * K + j] = j < n ? 1 : 0;
     }
     if (pb.token_id)
-      for (int j = lane; j < n; j += 32) pb.token_id[off + j] = j;
+      for (int j = threadIdx.x; j < n; j += T) pb.token_id[off + j] = j;
     if (pb.knn_idx) {
       int32_t* outk = pb.knn_idx + (int64_t)b * K * k;
-      for (int e = lane; e < K * k; e += 32) {
+      for (int e = threadIdx.x; e < K * k; e += T) {
         const int j = e / k, r = e - j * k;
         outk[e] = (r == 0 && j < n) ? (int32_t)(off + j) : -1;
       }
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
 
 cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s) {
   const DeviceInfo& di = device_info();
-  int blocks = (pb.B + 7) / 8;
+  int blocks = pb.B;
   const int cap = di.sm_count * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
@@ -174,18 +176,34 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
     for (int e = threadIdx.x; e < KF; e += blockDim.x) s_sum[e] = 0.0;
     for (int e = threadIdx.x; e < K; e += blockDim.x) s_cnt[e] = 0;
     __syncthreads();
+    // element-major over the chunk's features, 8 loads in flight per thread
     const int64_t e0 = (off + i0) * F, e1 = (off + i1) * F;
-    for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
-      const int64_t i = e / F;
-      const int f = (int)(e - i * F);
-      const int j = labels[i];
-      if (j < 0) continue;
-      if (j >= K) {
-        record_error(ws.hdr, kDevBadToken);
-        continue;
+    constexpr int R = 8;
+    for (int64_t base = e0 + threadIdx.x; base < e1; base += (int64_t)R * blockDim.x) {
+      float v[R];
+      int lab[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t e = base + (int64_t)r * blockDim.x;
+        lab[r] = -1;
+        if (e < e1) {
+          v[r] = feats[e];
+          lab[r] = labels[e / F];
+        }
       }
-      if (f == 0) atomicAdd(&s_cnt[j], 1);
-      atomicAdd(&s_sum[j * F + f], (double)feats[e]);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t e = base + (int64_t)r * blockDim.x;
+        const int j = lab[r];
+        if (e >= e1 || j < 0) continue;
+        if (j >= K) {
+          record_error(ws.hdr, kDevBadToken);
+          continue;
+        }
+        const int f = (int)(e - (e / F) * F);
+        if (f == 0) atomicAdd(&s_cnt[j], 1);
+        atomicAdd(&s_sum[j * F + f], (double)v[r]);
+      }
     }
     __syncthreads();
     if (nch == 1) {
@@ -240,8 +258,8 @@ __device__ __forceinline__ void load_cents(const float4* __restrict__ c, int nv,
 
 // Nearest of the first nv shared-memory centroids for points [i0, i1) of an
 // event (thread-strided, two points per packed evaluation); strict '<' over
-// increasing slots keeps the lowest slot on ties.  Calls emit(i, label) once
-// per point.
+// increasing slots keeps the lowest slot on ties.  Calls emit(i, label, p)
+// once per point p.
 template <int PAIRS, typename Emit>
 __device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int i0, int i1,
                                              const Cent2* __restrict__ cs, int nv, Emit emit) {
@@ -250,12 +268,17 @@ __device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int
     uint64_t X[PAIRS], Y[PAIRS], Z[PAIRS], W[PAIRS];
     float best[2 * PAIRS];
     int lab[2 * PAIRS];
+    float4 pa[PAIRS], pc[PAIRS];
 #pragma unroll
     for (int p = 0; p < PAIRS; ++p) {
       const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-      if (ia < i1) a = ldg4(pts + ia);
-      if (ib < i1) c = ldg4(pts + ib);
+      pa[p] = pc[p] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ia < i1) pa[p] = ldg4(pts + ia);
+      if (ib < i1) pc[p] = ldg4(pts + ib);
+    }
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      const float4 a = pa[p], c = pc[p];
       X[p] = pack2(a.x, c.x);
       Y[p] = pack2(a.y, c.y);
       Z[p] = pack2(a.z, c.z);
@@ -275,8 +298,8 @@ __device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int
 #pragma unroll
     for (int p = 0; p < PAIRS; ++p) {
       const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
-      if (ia < i1) emit(ia, nv > 0 ? (lab[2 * p] < 0 ? 0 : lab[2 * p]) : -1);
-      if (ib < i1) emit(ib, nv > 0 ? (lab[2 * p + 1] < 0 ? 0 : lab[2 * p + 1]) : -1);
+      if (ia < i1) emit(ia, nv > 0 ? (lab[2 * p] < 0 ? 0 : lab[2 * p]) : -1, pa[p]);
+      if (ib < i1) emit(ib, nv > 0 ? (lab[2 * p + 1] < 0 ? 0 : lab[2 * p + 1]) : -1, pc[p]);
     }
   }
 }
@@ -305,23 +328,24 @@ __global__ void __launch_bounds__(256) k_assign(const float4* __restrict__ coord
     __syncthreads();
     const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
     int32_t* out = token_id + off;
-    nearest_pass<kAssignPairs>(coords + off, i0, i1, s_cent, nv, [&](int i, int l) { out[i] = l; });
+    nearest_pass<kAssignPairs>(coords + off, i0, i1, s_cent, nv, [&](int i, int l, float4) { out[i] = l; });
     __syncthreads();
   }
 }
 
 // ------------------------------------------------------------------ Lloyd
 
-// Adds (q, q*x, q*y, q*z, q*t) of point i (event-local) to token j's shared sums.
-__device__ __forceinline__ void lloyd_accum(double* s, const float4* pts, const float* fe, int F,
-                                            int charge_col, int i, int j) {
-  const float4 p = ldg4(pts + i);
-  const double q = charge_col < 0 ? 1.0 : (double)fe[(int64_t)i * F + charge_col];
+// Adds (q, q*x, q*y, q*z, q*t) of point p to token j's shared sums.
+__device__ __forceinline__ void lloyd_accum(double* s, float4 p, double q, int j) {
   atomicAdd(&s[j * 5 + 0], q);
   atomicAdd(&s[j * 5 + 1], q * (double)p.x);
   atomicAdd(&s[j * 5 + 2], q * (double)p.y);
   atomicAdd(&s[j * 5 + 3], q * (double)p.z);
   atomicAdd(&s[j * 5 + 4], q * (double)p.w);
+}
+
+__device__ __forceinline__ double charge_of(const float* fe, int F, int charge_col, int i) {
+  return charge_col < 0 ? 1.0 : (double)__ldg(fe + (int64_t)i * F + charge_col);
 }
 
 __device__ __forceinline__ void flush_sums(const double* s, double* g, int n) {
@@ -347,13 +371,32 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
     for (int e = threadIdx.x; e < K * 5; e += blockDim.x) s_sum[e] = 0.0;
     __syncthreads();
     const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
-    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-      const int j = labels[off + i];
-      if (j < 0 || j >= K) {
-        record_error(ws.hdr, kDevBadToken);
-        continue;
+    const float4* pts = coords + off;
+    const float* fe = feats ? feats + off * F : nullptr;
+    constexpr int R = 4;
+    for (int base = i0 + threadIdx.x; base < i1; base += R * blockDim.x) {
+      int lab[R];
+      float4 pp[R];
+      double q[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = base + r * blockDim.x;
+        lab[r] = -2;
+        if (i < i1) {
+          lab[r] = labels[off + i];
+          pp[r] = ldg4(pts + i);
+          q[r] = charge_of(fe, F, charge_col, i);
+        }
       }
-      lloyd_accum(s_sum, coords + off, feats ? feats + off * F : nullptr, F, charge_col, i, j);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (lab[r] == -2) continue;
+        if (lab[r] < 0 || lab[r] >= K) {
+          record_error(ws.hdr, kDevBadToken);
+          continue;
+        }
+        lloyd_accum(s_sum, pp[r], q[r], lab[r]);
+      }
     }
     __syncthreads();
     flush_sums(s_sum, out + (int64_t)fs * K * 5, K * 5);
@@ -404,9 +447,9 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
     int32_t* lab = labels + off;
     const float4* pts = coords + off;
     const float* fe = feats ? feats + off * F : nullptr;
-    nearest_pass<kAssignPairs>(pts, i0, i1, s_cent, K, [&](int i, int l) {
+    nearest_pass<kAssignPairs>(pts, i0, i1, s_cent, K, [&](int i, int l, float4 p) {
       lab[i] = l;
-      if (next) lloyd_accum(s_sum, pts, fe, F, charge_col, i, l);
+      if (next) lloyd_accum(s_sum, p, charge_of(fe, F, charge_col, i), l);
     });
     __syncthreads();
     if (next) flush_sums(s_sum, next + (int64_t)fs * K * 5, K * 5);
@@ -520,35 +563,45 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
       const float4 c = centroids[r];
       const float4* pts = coords + o0;
       uint64_t thr = ~0ull;
-      for (int base = 0; base < n; base += 32) {
-        const int i = base + lane;
-        uint64_t key = ~0ull;
-        if (i < n) key = ((uint64_t)__float_as_uint(dist1(ldg4(pts + i), c)) << 32) | (uint32_t)i;
-        unsigned mask = __ballot_sync(kFull, key < thr);
-        while (mask) {
-          const int src = __ffs(mask) - 1;
-          mask &= mask - 1;
-          const uint64_t v = __shfl_sync(kFull, key, src);
-          if (v >= thr) continue;
-          int pos = 0;
+      constexpr int U = 4;  // 32-point chunks loaded per iteration
+      for (int base = 0; base < n; base += 32 * U) {
+        float4 pt[U];
 #pragma unroll
-          for (int q = 0; q < KPL; ++q) pos += __popc(__ballot_sync(kFull, L[q] < v));
+        for (int u = 0; u < U; ++u) {
+          const int i = base + u * 32 + lane;
+          pt[u] = i < n ? ldg4(pts + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-          for (int q = KPL - 1; q >= 0; --q) {
-            uint64_t up = __shfl_up_sync(kFull, L[q], 1);
-            if (q > 0) {
-              const uint64_t carry = __shfl_sync(kFull, L[q - 1], 31);
-              if (lane == 0) up = carry;
+        for (int u = 0; u < U; ++u) {
+          const int i = base + u * 32 + lane;
+          const uint64_t key =
+              i < n ? (((uint64_t)__float_as_uint(dist1(pt[u], c)) << 32) | (uint32_t)i) : ~0ull;
+          unsigned mask = __ballot_sync(kFull, key < thr);
+          while (mask) {
+            const int src = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const uint64_t v = __shfl_sync(kFull, key, src);
+            if (v >= thr) continue;
+            int pos = 0;
+#pragma unroll
+            for (int q = 0; q < KPL; ++q) pos += __popc(__ballot_sync(kFull, L[q] < v));
+#pragma unroll
+            for (int q = KPL - 1; q >= 0; --q) {
+              uint64_t up = __shfl_up_sync(kFull, L[q], 1);
+              if (q > 0) {
+                const uint64_t carry = __shfl_sync(kFull, L[q - 1], 31);
+                if (lane == 0) up = carry;
+              }
+              const int e = q * 32 + lane;
+              if (e > pos) L[q] = up;
+              else if (e == pos) L[q] = v;
             }
-            const int e = q * 32 + lane;
-            if (e > pos) L[q] = up;
-            else if (e == pos) L[q] = v;
-          }
-          uint64_t t = 0;
+            uint64_t t = 0;
 #pragma unroll
-          for (int q = 0; q < KPL; ++q)
-            if (q == kq) t = L[q];
-          thr = __shfl_sync(kFull, t, kl);
+            for (int q = 0; q < KPL; ++q)
+              if (q == kq) t = L[q];
+            thr = __shfl_sync(kFull, t, kl);
+          }
         }
       }
     }

@@ -108,6 +108,32 @@ __device__ __forceinline__ void relax(float d, float& dist, int& lab, int s) {
 
 __device__ __forceinline__ int fkey(float v) { return __float_as_int(v); }
 
+// Three-input float32 maximum (sm_100): one instruction for two new values.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Centroid position stored with every component duplicated, so that two
+// 128-bit shared-memory loads give the four packed registers of Cent2.
+struct DupPoint {
+  uint4 xy;  // (x, x, y, y)
+  uint4 zt;  // (z, z, t, t)
+};
+__device__ __forceinline__ DupPoint dup_point(float4 a) {
+  return DupPoint{make_uint4(__float_as_uint(a.x), __float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(a.y)),
+                  make_uint4(__float_as_uint(a.z), __float_as_uint(a.z), __float_as_uint(a.w), __float_as_uint(a.w))};
+}
+__device__ __forceinline__ Cent2 cent2_dup(const DupPoint& p) {
+  return Cent2{(uint64_t)p.xy.x | ((uint64_t)p.xy.y << 32), (uint64_t)p.xy.z | ((uint64_t)p.xy.w << 32),
+               (uint64_t)p.zt.x | ((uint64_t)p.zt.y << 32), (uint64_t)p.zt.z | ((uint64_t)p.zt.w << 32)};
+}
+__device__ __forceinline__ float4 dup_to_float4(const DupPoint& p) {
+  return make_float4(__uint_as_float(p.xy.x), __uint_as_float(p.xy.z), __uint_as_float(p.zt.x),
+                     __uint_as_float(p.zt.z));
+}
+
 // Warp arg-max of (key, idx): the largest key, then the smallest idx among
 // the lanes holding it.  Both results are warp-uniform.
 __device__ __forceinline__ void warp_argmax(int key, unsigned idx, int& mkey, unsigned& midx) {

@@ -1,4 +1,4 @@
-// Farthest point sampling fused with the Voronoi labels, three schedules.
+// Farthest point sampling fused with the Voronoi labels, four schedules.
 //
 // Tokenization per the Neptune README ("How it works", step 1): farthest-point
 // sampling of every event down to K centroids with nearest-centroid (Voronoi)
@@ -17,18 +17,25 @@
 // keeps the earliest slot, label_i equals the nearest centroid with the
 // lowest slot on ties, i.e. the plain Voronoi assignment.
 //
-// Schedules (chosen per event by the binning kernel):
-//   warp    N <= 448     one warp per event, points held in registers
-//                        (lane l owns points l + 32 j), shuffle-free
-//                        arg-max with two redux.sync per step.
-//   CTA     N <= 12288   one 512-thread CTA per event, points in shared
-//                        memory as packed f32x2 pairs, distances and labels
-//                        in registers, one barrier per step.
-//   cluster N <= 196608  a 16-CTA thread-block cluster per event; every warp
-//                        posts its candidate (key, index, position) into every
-//                        CTA's shared memory over DSMEM, one barrier.cluster
-//                        per step, then each warp reduces the posted entries.
+// Schedules (chosen per event by the binning kernel; all run concurrently,
+// the three block schedules on helper streams forked from the caller's):
+//   warp      N <= 448      one warp per event; points in registers (lane l
+//                           owns points l + 32 j); arg-max with two redux.sync.
+//   CTA       N <= 2560     one 128-thread CTA per event; points in registers;
+//                           warp results exchanged through shared memory,
+//                           one barrier per step.
+//   CTA-smem  N <= 12288    one 256-thread CTA per event; points in shared
+//                           memory as packed f32x2 pairs; distances and labels
+//                           in registers.
+//   cluster   N <= 196608   a 16-CTA thread-block cluster per event (same
+//                           layout); every warp posts its candidate into every
+//                           CTA's shared memory over DSMEM; one
+//                           barrier.cluster per step.
+// Every step touches exactly the occupied point pairs: the unrolled per-pair
+// code is entered through a switch on the pair count (no per-pair guards).
 #include <cooperative_groups.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -37,19 +44,38 @@ namespace cg = cooperative_groups;
 
 namespace fpstok {
 
+// Runs BODY(p) for p = np-1 down to 0 (np <= 24): the switch enters the
+// unrolled sequence at the right place.  BODY(p) is compiled only for
+// p < kMaxPairs, a constexpr in the calling scope.
+#define FPS_CASE(p, BODY) \
+  case (p) + 1:           \
+    if constexpr ((p) < kMaxPairs) { BODY(p) } [[fallthrough]];
+#define FPS_FALL(np, BODY)                                                                                   \
+  switch (np) {                                                                                              \
+    FPS_CASE(23, BODY) FPS_CASE(22, BODY) FPS_CASE(21, BODY) FPS_CASE(20, BODY) FPS_CASE(19, BODY)          \
+    FPS_CASE(18, BODY) FPS_CASE(17, BODY) FPS_CASE(16, BODY) FPS_CASE(15, BODY) FPS_CASE(14, BODY)          \
+    FPS_CASE(13, BODY) FPS_CASE(12, BODY) FPS_CASE(11, BODY) FPS_CASE(10, BODY) FPS_CASE(9, BODY)           \
+    FPS_CASE(8, BODY) FPS_CASE(7, BODY) FPS_CASE(6, BODY) FPS_CASE(5, BODY) FPS_CASE(4, BODY)               \
+    FPS_CASE(3, BODY) FPS_CASE(2, BODY) FPS_CASE(1, BODY) FPS_CASE(0, BODY) default : break;                \
+  }
+
+__device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xffffffffu : ((1u << n) - 1u); }
+
 // ------------------------------------------------------------------ warp
 
-template <int PPL>
+template <int NP>
 __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ coords,
-                                                  const int64_t* __restrict__ offsets,
-                                                  const int32_t* __restrict__ start_local,
-                                                  const int* __restrict__ list, WsHeader* hdr, int K,
-                                                  int32_t* __restrict__ centroid_idx,
-                                                  int32_t* __restrict__ token_id,
-                                                  float4* __restrict__ centroids) {
-  static_assert(PPL % 2 == 0 && PPL <= 32, "points per lane must be even and <= 32");
-  constexpr int NP = PPL / 2;
+                                                     const int64_t* __restrict__ offsets,
+                                                     const int32_t* __restrict__ start_local,
+                                                     const int* __restrict__ list, WsHeader* hdr, int K,
+                                                     int32_t* __restrict__ centroid_idx,
+                                                     int32_t* __restrict__ token_id,
+                                                     float4* __restrict__ centroids) {
+  constexpr int kMaxPairs = NP;
+  static_assert(2 * NP <= 32, "selected-slot mask is 32 bits");
+  extern __shared__ DupPoint s_dup_all[];
   const int lane = threadIdx.x & 31;
+  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NP);  // this warp's event copy
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int count = hdr->n_items[kListWarp];
@@ -58,20 +84,22 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
     const int b = list[w];
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    const int npairs = (((n + 31) >> 5) + 1) >> 1;
+    const int npairs = (n + 63) >> 6;
     const float4* pts = coords + off;
 
     uint64_t X[NP], Y[NP], Z[NP], T[NP];
-    float dist[PPL];
-    int lab[PPL];
-    unsigned taken = 0;  // bit j: slot j is selected or holds no point
+    float dist[2 * NP];
+    int lab[2 * NP];
+    unsigned taken = 0;  // bit j: slot j (point 32 j + lane) is selected or empty
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      const int i0 = (2 * p) * 32 + lane, i1 = i0 + 32;
+      const int i0 = 64 * p + lane, i1 = i0 + 32;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
       if (p < npairs) {
         if (i0 < n) a = ldg4(pts + i0);
         if (i1 < n) c = ldg4(pts + i1);
+        if (i0 < n) s_dup[i0] = dup_point(a);
+        if (i1 < n) s_dup[i1] = dup_point(c);
       }
       X[p] = pack2(a.x, c.x);
       Y[p] = pack2(a.y, c.y);
@@ -84,57 +112,184 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
       if (i0 >= n) taken |= 1u << (2 * p);
       if (i1 >= n) taken |= 1u << (2 * p + 1);
     }
+    __syncwarp();
 
     int c = start_local ? start_local[b] : 0;
-    float4 cc = ldg4(pts + c);
     for (int s = 0; s < K; ++s) {
+      const DupPoint cp = s_dup[c];
       if (lane == 0) {
         centroid_idx[(int64_t)b * K + s] = (int32_t)(off + c);
-        centroids[(int64_t)b * K + s] = cc;
+        centroids[(int64_t)b * K + s] = dup_to_float4(cp);
       }
       if ((c & 31) == lane) taken |= 1u << (c >> 5);
-      const Cent2 C = cent2(cc);
-      float m = kEmptySlot;
-#pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        if (p < npairs) {
-          const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);
-          relax(lo2(d), dist[2 * p], lab[2 * p], s);
-          relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
-          m = fmaxf(m, fmaxf(dist[2 * p], dist[2 * p + 1]));
-        }
-      }
+      const Cent2 C = cent2_dup(cp);
+      float m0 = kEmptySlot, m1 = kEmptySlot;
+#define W_UPD(p)                                                  \
+  {                                                               \
+    const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);          \
+    relax(lo2(d), dist[2 * (p)], lab[2 * (p)], s);                \
+    relax(hi2(d), dist[2 * (p) + 1], lab[2 * (p) + 1], s);        \
+    if ((p) & 1)                                                  \
+      m1 = max3f(m1, dist[2 * (p)], dist[2 * (p) + 1]);           \
+    else                                                          \
+      m0 = max3f(m0, dist[2 * (p)], dist[2 * (p) + 1]);           \
+  }
+      FPS_FALL(npairs, W_UPD)
+#undef W_UPD
       if (s == K - 1) break;
-      const int key = fkey(m);
+      const int key = fkey(fmaxf(m0, m1));
       const int M = __reduce_max_sync(kFull, key);
       unsigned cand = 0xffffffffu;
       if (key == M) {
-#pragma unroll
-        for (int j = PPL - 1; j >= 0; --j)
-          if (fkey(dist[j]) == M) cand = (unsigned)(j * 32 + lane);
+#define W_SCAN(p)                                                                         \
+  {                                                                                       \
+    if (fkey(dist[2 * (p) + 1]) == M) cand = (unsigned)((2 * (p) + 1) * 32 + lane);       \
+    if (fkey(dist[2 * (p)]) == M) cand = (unsigned)((2 * (p)) * 32 + lane);               \
+  }
+        FPS_FALL(npairs, W_SCAN)
+#undef W_SCAN
       }
       unsigned idx = __reduce_min_sync(kFull, cand);
       if (M == 0) {  // only duplicates of chosen points remain
-        const unsigned free_slots = ~taken & ((PPL == 32) ? 0xffffffffu : ((1u << PPL) - 1u));
+        const unsigned free_slots = ~taken & low_bits(2 * npairs);
         cand = free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu;
         idx = __reduce_min_sync(kFull, cand);
       }
       c = (int)idx;
-      cc = ldg4(pts + c);
     }
     if (token_id) {
 #pragma unroll
-      for (int j = 0; j < PPL; ++j) {
+      for (int j = 0; j < 2 * NP; ++j) {
         const int i = j * 32 + lane;
         if (i < n) token_id[off + i] = lab[j];
       }
     }
+    __syncwarp();  // the next event overwrites this warp's copy
   }
 }
 
-// ------------------------------------------------------------------ CTA / cluster
+// ------------------------------------------------------------------ CTA, points in registers
 
-template <int CL, int NT, int PSP>
+template <int PR>
+__global__ void __launch_bounds__(128, 1) k_fps_cta(const float4* __restrict__ coords,
+                                                    const int64_t* __restrict__ offsets,
+                                                    const int32_t* __restrict__ start_local,
+                                                    const int* __restrict__ list, WsHeader* hdr, int K,
+                                                    int32_t* __restrict__ centroid_idx,
+                                                    int32_t* __restrict__ token_id,
+                                                    float4* __restrict__ centroids) {
+  constexpr int kMaxPairs = PR;
+  constexpr int NT = 128, NW = 4;
+  static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
+  extern __shared__ DupPoint s_dup[];  // [256 * PR] event copy for centroid look-up
+  __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int count = hdr->n_items[kListCta];
+  int round = 0;
+
+  auto exchange = [&](int wkey, unsigned widx, int& M, unsigned& idx) {
+    if (lane == 0) xk[(round & 1) * NW + warp] = make_int2(wkey, (int)widx);
+    __syncthreads();
+    const int2 v = lane < NW ? xk[(round & 1) * NW + lane] : make_int2(-0x7fffffff - 1, -1);
+    warp_argmax(v.x, (unsigned)v.y, M, idx);
+    ++round;
+  };
+
+  for (int item = blockIdx.x; item < count; item += gridDim.x) {
+    const int b = list[item];
+    const int64_t off = offsets[b];
+    const int n = (int)(offsets[b + 1] - off);
+    const int npairs = (n + 2 * NT - 1) / (2 * NT);
+    const float4* pts = coords + off;
+
+    uint64_t X[PR], Y[PR], Z[PR], T[PR];
+    float dist[2 * PR];
+    int lab[2 * PR];
+    unsigned taken = 0;  // bit j: slot j (point NT j + tid) is selected or empty
+#pragma unroll
+    for (int p = 0; p < PR; ++p) {
+      const int i0 = 2 * NT * p + tid, i1 = i0 + NT;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+      if (p < npairs) {
+        if (i0 < n) a = ldg4(pts + i0);
+        if (i1 < n) c = ldg4(pts + i1);
+        if (i0 < n) s_dup[i0] = dup_point(a);
+        if (i1 < n) s_dup[i1] = dup_point(c);
+      }
+      X[p] = pack2(a.x, c.x);
+      Y[p] = pack2(a.y, c.y);
+      Z[p] = pack2(a.z, c.z);
+      T[p] = pack2(a.w, c.w);
+      dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+      dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+      lab[2 * p] = 0;
+      lab[2 * p + 1] = 0;
+      if (i0 >= n) taken |= 1u << (2 * p);
+      if (i1 >= n) taken |= 1u << (2 * p + 1);
+    }
+    __syncthreads();
+
+    int c = start_local ? start_local[b] : 0;
+    for (int s = 0; s < K; ++s) {
+      const DupPoint cp = s_dup[c];
+      if (tid == 0) {
+        centroid_idx[(int64_t)b * K + s] = (int32_t)(off + c);
+        centroids[(int64_t)b * K + s] = dup_to_float4(cp);
+      }
+      if (c % NT == tid) taken |= 1u << (c / NT);
+      const Cent2 C = cent2_dup(cp);
+      float m0 = kEmptySlot, m1 = kEmptySlot;
+#define C_UPD(p)                                                  \
+  {                                                               \
+    const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);          \
+    relax(lo2(d), dist[2 * (p)], lab[2 * (p)], s);                \
+    relax(hi2(d), dist[2 * (p) + 1], lab[2 * (p) + 1], s);        \
+    if ((p) & 1)                                                  \
+      m1 = max3f(m1, dist[2 * (p)], dist[2 * (p) + 1]);           \
+    else                                                          \
+      m0 = max3f(m0, dist[2 * (p)], dist[2 * (p) + 1]);           \
+  }
+      FPS_FALL(npairs, C_UPD)
+#undef C_UPD
+      if (s == K - 1) break;
+      const int key = fkey(fmaxf(m0, m1));
+      const int wM = __reduce_max_sync(kFull, key);
+      unsigned cand = 0xffffffffu;
+      if (key == wM) {
+#define C_SCAN(p)                                                                      \
+  {                                                                                    \
+    if (fkey(dist[2 * (p) + 1]) == wM) cand = (unsigned)((2 * (p) + 1) * NT + tid);    \
+    if (fkey(dist[2 * (p)]) == wM) cand = (unsigned)((2 * (p)) * NT + tid);            \
+  }
+        FPS_FALL(npairs, C_SCAN)
+#undef C_SCAN
+      }
+      const unsigned widx = __reduce_min_sync(kFull, cand);
+      int M;
+      unsigned idx;
+      exchange(wM, widx, M, idx);
+      if (M == 0) {  // only duplicates of chosen points remain
+        const unsigned free_slots = ~taken & low_bits(2 * npairs);
+        const unsigned mine = free_slots ? (unsigned)((__ffs(free_slots) - 1) * NT + tid) : 0xffffffffu;
+        const unsigned wmin = __reduce_min_sync(kFull, mine);
+        exchange(wmin != 0xffffffffu ? 1 : 0, wmin, M, idx);
+      }
+      c = (int)idx;
+    }
+    if (token_id) {
+#pragma unroll
+      for (int j = 0; j < 2 * PR; ++j) {
+        const int i = j * NT + tid;
+        if (i < n) token_id[off + i] = lab[j];
+      }
+    }
+    __syncthreads();  // the next event overwrites the shared copy
+  }
+}
+
+// ------------------------------------------------------------------ CTA / cluster, points in shared memory
+
+template <int CL, int NT, int PS>
 __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ coords,
                                                      const int64_t* __restrict__ offsets,
                                                      const int32_t* __restrict__ start_local,
@@ -143,13 +298,14 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
                                                      float4* __restrict__ centroids) {
-  static_assert(2 * PSP <= 32, "selected-slot mask is 32 bits");
+  constexpr int kMaxPairs = PS;
+  static_assert(2 * PS <= 64, "selected-slot mask is 64 bits");
   constexpr int NW = NT / 32;
   constexpr int E = CL * NW;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  ulonglong2* sXY = reinterpret_cast<ulonglong2*>(smem_raw);  // [PSP][NT] packed (x, y)
-  ulonglong2* sZT = sXY + PSP * NT;                           // [PSP][NT] packed (z, t)
-  int2* xkey = reinterpret_cast<int2*>(sZT + PSP * NT);       // [2][E] (key, index)
+  ulonglong2* sXY = reinterpret_cast<ulonglong2*>(smem_raw);  // [PS][NT] packed (x, y)
+  ulonglong2* sZT = sXY + PS * NT;                            // [PS][NT] packed (z, t)
+  int2* xkey = reinterpret_cast<int2*>(sZT + PS * NT);        // [2][E] (key, index)
   float4* xpos = reinterpret_cast<float4*>(xkey + 2 * E);     // [2][E] candidate position
 
   const int tid = threadIdx.x;
@@ -230,11 +386,11 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     const int npairs = (n + 2 * G - 1) / (2 * G);
     const float4* pts = coords + off;
 
-    float dist[2 * PSP];
-    int lab[2 * PSP];
-    unsigned taken = 0;
+    float dist[2 * PS];
+    int lab[2 * PS];
+    unsigned long long taken = 0;
 #pragma unroll
-    for (int p = 0; p < PSP; ++p) {
+    for (int p = 0; p < PS; ++p) {
       const int i0 = g + G * (2 * p), i1 = i0 + G;
       if (p < npairs) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
@@ -247,8 +403,8 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
       dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
       lab[2 * p] = 0;
       lab[2 * p + 1] = 0;
-      if (i0 >= n) taken |= 1u << (2 * p);
-      if (i1 >= n) taken |= 1u << (2 * p + 1);
+      if (i0 >= n) taken |= 1ull << (2 * p);
+      if (i1 >= n) taken |= 1ull << (2 * p + 1);
     }
 
     int c = start_local ? start_local[b] : 0;
@@ -258,32 +414,38 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
         centroid_idx[(int64_t)b * K + s] = (int32_t)(off + c);
         centroids[(int64_t)b * K + s] = cc;
       }
-      if (c % G == g) taken |= 1u << (c / G);
+      if (c % G == g) taken |= 1ull << (c / G);
       const Cent2 C = cent2(cc);
-      float m = kEmptySlot;
-#pragma unroll
-      for (int p = 0; p < PSP; ++p) {
-        if (p < npairs) {
-          const ulonglong2 xy = sXY[p * NT + tid];
-          const ulonglong2 zt = sZT[p * NT + tid];
-          const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C);
-          relax(lo2(d), dist[2 * p], lab[2 * p], s);
-          relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
-          m = fmaxf(m, fmaxf(dist[2 * p], dist[2 * p + 1]));
-        }
-      }
+      float m0 = kEmptySlot, m1 = kEmptySlot;
+#define B_UPD(p)                                                   \
+  {                                                                \
+    const ulonglong2 xy = sXY[(p) * NT + tid];                     \
+    const ulonglong2 zt = sZT[(p) * NT + tid];                     \
+    const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C);           \
+    relax(lo2(d), dist[2 * (p)], lab[2 * (p)], s);                 \
+    relax(hi2(d), dist[2 * (p) + 1], lab[2 * (p) + 1], s);         \
+    if ((p) & 1)                                                   \
+      m1 = max3f(m1, dist[2 * (p)], dist[2 * (p) + 1]);            \
+    else                                                           \
+      m0 = max3f(m0, dist[2 * (p)], dist[2 * (p) + 1]);            \
+  }
+      FPS_FALL(npairs, B_UPD)
+#undef B_UPD
       if (s == K - 1) break;
 
-      const int key = fkey(m);
-      int wM;
-      unsigned wcand = 0xffffffffu, widx;
-      wM = __reduce_max_sync(kFull, key);
+      const int key = fkey(fmaxf(m0, m1));
+      const int wM = __reduce_max_sync(kFull, key);
+      unsigned wcand = 0xffffffffu;
       if (key == wM) {
-#pragma unroll
-        for (int j = 2 * PSP - 1; j >= 0; --j)
-          if (fkey(dist[j]) == wM) wcand = (unsigned)(g + G * j);
+#define B_SCAN(p)                                                                     \
+  {                                                                                   \
+    if (fkey(dist[2 * (p) + 1]) == wM) wcand = (unsigned)(g + G * (2 * (p) + 1));     \
+    if (fkey(dist[2 * (p)]) == wM) wcand = (unsigned)(g + G * (2 * (p)));             \
+  }
+        FPS_FALL(npairs, B_SCAN)
+#undef B_SCAN
       }
-      widx = __reduce_min_sync(kFull, wcand);
+      const unsigned widx = __reduce_min_sync(kFull, wcand);
       float4 wpos = make_float4(0.f, 0.f, 0.f, 0.f);
       if (wM >= 0) wpos = local_pos(widx);
       post(wM, widx, wpos);
@@ -292,12 +454,11 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
       unsigned idx;
       gather(M, idx, cc);
       if (M == 0) {  // only duplicates of chosen points remain
-        const unsigned free_slots = ~taken & ((2 * PSP == 32) ? 0xffffffffu : ((1u << (2 * PSP)) - 1u));
+        const int nslots = 2 * npairs;
+        const unsigned long long mask = nslots >= 64 ? ~0ull : ((1ull << nslots) - 1ull);
+        const unsigned long long free_slots = ~taken & mask;
         unsigned cand = 0xffffffffu;
-        if (free_slots) {
-          const int j = __ffs(free_slots) - 1;
-          if (j < 2 * npairs) cand = (unsigned)(g + G * j);
-        }
+        if (free_slots) cand = (unsigned)(g + G * (__ffsll((long long)free_slots) - 1));
         const unsigned wmin = __reduce_min_sync(kFull, cand);
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
         if (wmin != 0xffffffffu) p = local_pos(wmin);
@@ -310,7 +471,7 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     }
     if (token_id) {
 #pragma unroll
-      for (int j = 0; j < 2 * PSP; ++j) {
+      for (int j = 0; j < 2 * PS; ++j) {
         const int i = g + G * j;
         if (j < 2 * npairs && i < n) token_id[off + i] = lab[j];
       }
@@ -318,6 +479,15 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
   }
   if constexpr (CL > 1) cg::this_cluster().sync();  // no CTA leaves while peers may post into it
 }
+
+#undef FPS_FALL
+#undef FPS_CASE
+
+// ------------------------------------------------------------------ launch
+
+constexpr int kWarpBlock = 128;
+constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(DupPoint);
+constexpr size_t kCtaSmem = (size_t)2 * 128 * kCtaPairs * sizeof(DupPoint);
 
 template <int CL>
 constexpr size_t block_smem_bytes() {
@@ -357,16 +527,26 @@ static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  const int* list = list_id == kListCta ? ws.list_cta : ws.list_cluster;
+  const int* list = list_id == kListCtaSmem ? ws.list_cta_smem : ws.list_cluster;
   count_launch();
   return cudaLaunchKernelEx(&cfg, k_fps_block<CL, kBlockThreads, kBlockPairs>, pb.coords,
                             pb.offsets, pb.start_local, list, ws.hdr, list_id, pb.K, pb.centroid_idx,
                             pb.token_id, pb.centroids);
 }
 
+// Per-device state: occupancy figures and the helper streams / events that
+// let the four schedules run concurrently.
+struct DeviceCtx {
+  DeviceInfo info;
+  cudaStream_t helper[3];
+  cudaEvent_t fork, join[3];
+  std::mutex launch_mu;
+  bool prepared;
+};
+
 constexpr int kMaxDevices = 64;
-static bool g_prepared[kMaxDevices];
-static DeviceInfo g_info[kMaxDevices];
+static DeviceCtx g_ctx[kMaxDevices];
+static std::mutex g_prepare_mu;
 
 static int current_device() {
   int dev = 0;
@@ -374,13 +554,23 @@ static int current_device() {
   return dev;
 }
 
-// One-time set-up per device: kernel attributes and occupancy figures.
+// One-time set-up per device: kernel attributes, occupancy figures, helper
+// streams and fork/join events.
 static cudaError_t prepare(int dev) {
-  if (g_prepared[dev]) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(g_prepare_mu);
+  DeviceCtx& ctx = g_ctx[dev];
+  if (ctx.prepared) return cudaSuccess;
   DeviceInfo info = {};
   cudaError_t e = cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&info.warp_blocks_per_sm, k_fps_warp<kWarpPPL>, 128, 0);
+  if ((e = cudaFuncSetAttribute(k_fps_warp<kWarpPairs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kWarpSmem)))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_fps_cta<kCtaPairs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kCtaSmem)))
+    return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&info.warp_blocks_per_sm, k_fps_warp<kWarpPairs>,
+                                                    kWarpBlock, kWarpSmem);
   if (e != cudaSuccess) return e;
   if ((e = prepare_block_kernel<1>()) != cudaSuccess) return e;
   if ((e = prepare_block_kernel<kMaxCluster>()) != cudaSuccess) return e;
@@ -399,9 +589,14 @@ static cudaError_t prepare(int dev) {
                                      k_fps_block<kMaxCluster, kBlockThreads, kBlockPairs>, &cfg);
   if (e != cudaSuccess) return e;
   if ((e = prepare_aux_kernels()) != cudaSuccess) return e;
+  for (int i = 0; i < 3; ++i) {
+    if ((e = cudaStreamCreateWithFlags(&ctx.helper[i], cudaStreamNonBlocking))) return e;
+    if ((e = cudaEventCreateWithFlags(&ctx.join[i], cudaEventDisableTiming))) return e;
+  }
+  if ((e = cudaEventCreateWithFlags(&ctx.fork, cudaEventDisableTiming))) return e;
   info.ready = true;
-  g_info[dev] = info;
-  g_prepared[dev] = true;
+  ctx.info = info;
+  ctx.prepared = true;
   return cudaSuccess;
 }
 
@@ -410,40 +605,63 @@ static const DeviceInfo g_none = {};
 const DeviceInfo& device_info() {
   const int dev = current_device();
   if (dev < 0 || prepare(dev) != cudaSuccess) return g_none;
-  return g_info[dev];
+  return g_ctx[dev].info;
 }
 
 cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, StageMark mark) {
-  const DeviceInfo& di = device_info();
-  if (!di.ready) return cudaErrorInitializationError;
-  cudaError_t e;
-  // Launch a schedule unless the size hint rules out every event it could get.
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  cudaError_t e = prepare(dev);
+  if (e != cudaSuccess) return e;
+  DeviceCtx& ctx = g_ctx[dev];
+  const DeviceInfo& di = ctx.info;
+  // Launch a schedule unless the size hint rules out every event it could get:
+  // schedule q receives events above `lower[q]` (or above K when forced).
   const int hint = pb.max_event_hint;
   const int f = pb.force_schedule;
-  const bool any_warp = f <= 0 && (hint == 0 || hint > pb.K);
-  const bool any_cta = f <= 1 && (hint == 0 || hint > (f >= 1 ? pb.K : kWarpCap));
-  const bool any_cluster = hint == 0 || hint > (f >= 2 ? pb.K : kCtaCap);
-  if (any_warp) {
+  const int lower[4] = {pb.K, kWarpCap, kCtaCap, kCtaSmemCap};
+  bool run[4];
+  for (int q = 0; q < 4; ++q) {
+    const int lo = f >= q ? pb.K : lower[q];
+    run[q] = (q == 3 || f <= q) && (hint == 0 || hint > lo);
+  }
+
+  std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
+  const bool forked = run[1] || run[2] || run[3];
+  if (forked && (e = cudaEventRecord(ctx.fork, s))) return e;
+  for (int h = 0; h < 3; ++h) {
+    if (!run[h + 1]) continue;
+    cudaStream_t hs = ctx.helper[h];
+    if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
+    mark(2 + h, 0, hs);
+    if (h == 0) {
+      count_launch();
+      k_fps_cta<kCtaPairs><<<di.sm_count, 128, kCtaSmem, hs>>>(pb.coords, pb.offsets, pb.start_local, ws.list_cta,
+                                                               ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
+                                                               pb.centroids);
+      e = cudaGetLastError();
+    } else if (h == 1) {
+      e = launch_block<1>(pb, ws, kListCtaSmem, di.sm_count, hs);
+    } else {
+      const int groups = di.cluster_max_active > 0 ? di.cluster_max_active : 1;
+      e = launch_block<kMaxCluster>(pb, ws, kListCluster, groups, hs);
+    }
+    if (e != cudaSuccess) return e;
+    mark(2 + h, 1, hs);
+    if ((e = cudaEventRecord(ctx.join[h], hs))) return e;
+  }
+  if (run[0]) {
     const int blocks = di.sm_count * (di.warp_blocks_per_sm > 0 ? di.warp_blocks_per_sm : 1);
     mark(1, 0, s);
     count_launch();
-    k_fps_warp<kWarpPPL><<<blocks, 128, 0, s>>>(pb.coords, pb.offsets, pb.start_local, ws.list_warp,
-                                                ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-                                                pb.centroids);
+    k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, s>>>(pb.coords, pb.offsets, pb.start_local,
+                                                                 ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
+                                                                 pb.token_id, pb.centroids);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1, 1, s);
   }
-  if (any_cta) {
-    mark(2, 0, s);
-    if ((e = launch_block<1>(pb, ws, kListCta, di.sm_count, s)) != cudaSuccess) return e;
-    mark(2, 1, s);
-  }
-  if (any_cluster) {
-    const int groups = di.cluster_max_active > 0 ? di.cluster_max_active : 1;
-    mark(3, 0, s);
-    if ((e = launch_block<kMaxCluster>(pb, ws, kListCluster, groups, s)) != cudaSuccess) return e;
-    mark(3, 1, s);
-  }
+  for (int h = 0; h < 3; ++h)
+    if (run[h + 1] && (e = cudaStreamWaitEvent(s, ctx.join[h], 0))) return e;
   return cudaSuccess;
 }
 

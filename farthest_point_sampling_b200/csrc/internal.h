@@ -13,26 +13,31 @@ enum EventClass : int { kClsSkip = 0, kClsEmpty = 1, kClsPass = 2, kClsFps = 3 }
 enum ListId : int {
   kListWarp = 0,
   kListCta = 1,
-  kListCluster = 2,
-  kListChunks = 3,     // (event, chunk) items of FPS events
-  kListPoolSlots = 4,  // events that need global pooling accumulators
-  kListFps = 5,        // number of FPS events (Lloyd slots)
+  kListCtaSmem = 2,
+  kListCluster = 3,
+  kListChunks = 4,     // (event, chunk) items of FPS events
+  kListPoolSlots = 5,  // events that need global pooling accumulators
+  kListFps = 6,        // number of FPS events (Lloyd slots)
+  kNumLists = 7,
 };
 
 // Schedule capacities (points per event).
-constexpr int kWarpPPL = 14;                  // points per lane, warp schedule
-constexpr int kWarpCap = 32 * kWarpPPL;       // 448
-constexpr int kBlockThreads = 512;            // CTA / cluster schedules
-constexpr int kBlockPairs = 12;               // point pairs per thread (shared memory)
-constexpr int kCtaCap = kBlockThreads * 2 * kBlockPairs;  // 12288
+constexpr int kWarpPairs = 7;                          // point pairs per lane, warp schedule
+constexpr int kWarpCap = 64 * kWarpPairs;              // 448
+constexpr int kCtaPairs = 10;                          // pairs per thread, 128-thread CTA
+constexpr int kCtaCap = 256 * kCtaPairs;               // 2560
+constexpr int kBlockThreads = 256;                     // shared-memory CTA / cluster schedules
+constexpr int kBlockPairs = 24;                        // pairs per thread in shared memory
+constexpr int kCtaSmemCap = kBlockThreads * 2 * kBlockPairs;  // 12288
 constexpr int kMaxCluster = 16;
-constexpr int kClusterCap = kMaxCluster * kCtaCap;        // 196608
-constexpr int kChunk = 2048;                  // points per pooling / Lloyd work item
+constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
+constexpr int kChunk = 1024;                           // points per pooling / Lloyd work item
 
 struct Workspace {
   struct WsHeader* hdr;
   int* list_warp;
   int* list_cta;
+  int* list_cta_smem;
   int* list_cluster;
   int2* chunks;     // (event, chunk)
   int* cls;         // EventClass per event

@@ -45,8 +45,8 @@ def test_c1_host_offsets_hint():
 
 # ------------------------------------------------------------- sizes, tiles, ragged tails
 
-EDGE_SIZES = [0, 1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 447, 448, 449, 1000, 4095,
-              12287, 12288, 12289, 30001]
+EDGE_SIZES = [0, 1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 447, 448, 449, 1000, 2559, 2560,
+              2561, 4095, 12287, 12288, 12289, 30001]
 
 
 @pytest.mark.parametrize("K", [1, 2, 16, 128, 256])
@@ -70,9 +70,9 @@ def test_ties_and_duplicates(kind):
     compare(b, run_gpu(b))
 
 
-@pytest.mark.parametrize("force", [0, 1, 2])
+@pytest.mark.parametrize("force", [0, 1, 2, 3])
 def test_forced_schedules_agree(force):
-    sizes = [129, 300, 448, 449, 2000, 12288, 12289, 40000]
+    sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000]
     b = workloads.random_batch(11, sizes, 128, dup_frac=0.05)
     ora = oracle.tokenize_batch(b)
     compare(b, run_gpu(b, force_schedule=force), ora)
@@ -236,3 +236,26 @@ def test_no_host_sync_and_launch_count():
     n = fps.launch_count() - before
     assert 3 <= n <= 8, n
     torch.cuda.synchronize()
+
+
+def test_cuda_graph_capture_and_replay():
+    """One fps_tokenize call captured into a CUDA graph (the internal helper
+    streams join the capture) and replayed on new inputs of the same shape."""
+    dev = torch.device("cuda")
+    b1 = workloads.make_workload("c1")
+    b2 = workloads.random_batch(77, b1.sizes(), b1.K)  # same shapes, other values
+    c, f, o, _ = to_dev(b1)
+    out = fps.fps_tokenize(c, f, o, K=b1.K)  # first call on the device happens before capture
+    ws = torch.empty(1 << 22, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        fps.fps_tokenize(c, f, o, K=b1.K, workspace=ws, out=out)
+    for b in (b1, b2):
+        c.copy_(torch.from_numpy(b.coords))
+        f.copy_(torch.from_numpy(b.feats))
+        g.replay()
+        torch.cuda.synchronize()
+        compare(b, {k: v.cpu().numpy() for k, v in out.items()})
