@@ -21,50 +21,101 @@ namespace fpstok {
 
 // ------------------------------------------------------------------ binning
 
+// Size buckets of the counting sort that orders each schedule's list by
+// decreasing event size (bucket = n >> shift; shift keeps cap >> shift < 256).
+constexpr int kBins = 256;
+__device__ __forceinline__ int sched_shift(int q) {
+  return q == 0 ? 1 : (q == 1 ? 4 : (q == 2 ? 6 : (q == 3 ? 9 : 10)));
+}
+
+// One CTA: classifies every event, builds the per-schedule work lists sorted
+// by decreasing size (longest chains first), the (event, chunk) items of FPS
+// events, and the accumulator slots; resets the status word and the cursors.
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
-                                               int force, int chunk_all, Workspace ws) {
+                                               int force, int chunk_all, int latency_events, Workspace ws) {
   __shared__ int cnt[kNumLists];
+  __shared__ int hist[kNumSchedules][kBins];
+  __shared__ int n_fps;
+  for (int i = threadIdx.x; i < kNumSchedules * kBins; i += blockDim.x) (&hist[0][0])[i] = 0;
   if (threadIdx.x < kNumLists) cnt[threadIdx.x] = 0;
+  if (threadIdx.x < 8) ws.hdr->next_item[threadIdx.x] = 0;
   if (threadIdx.x == 0) {
     ws.hdr->status = 0;
     ws.hdr->detail = 0;
+    n_fps = 0;
   }
   __syncthreads();
+  // pass 1: classify and count FPS events
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int64_t o0 = offsets[b], o1 = offsets[b + 1];
     int cls;
-    int64_t n = 0;
     if (o0 < 0 || o1 < o0 || o1 > P) {
       record_error(ws.hdr, kDevBadOffsets);
       cls = kClsSkip;
     } else {
       if ((b == 0 && o0 != 0) || (b == B - 1 && o1 != P)) record_error(ws.hdr, kDevBadOffsets);
-      n = o1 - o0;
+      const int64_t n = o1 - o0;
       cls = n == 0 ? kClsEmpty : (n <= K ? kClsPass : kClsFps);
       if (cls == kClsFps) {
-        const int s = start_local ? start_local[b] : 0;
-        if (s < 0 || s >= n) {
+        const int st = start_local ? start_local[b] : 0;
+        if (st < 0 || st >= n) {
           record_error(ws.hdr, kDevBadStart);
           cls = kClsSkip;
         } else if (n > kClusterCap) {
           record_error(ws.hdr, kDevTooLarge);
           cls = kClsSkip;
+        } else {
+          atomicAdd(&n_fps, 1);
         }
       }
     }
     ws.cls[b] = cls;
+  }
+  __syncthreads();
+  const bool few = n_fps <= latency_events;
+  auto schedule_of = [&](int n) {
+    int q = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : (n <= kCluster8Cap ? 3 : 4)));
+    if (q == 0 && few) q = 1;  // few events: lower latency per step on a whole CTA
+    if (force > q) q = force > 4 ? 4 : force;
+    return q;
+  };
+  // pass 2: size histogram per schedule
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    if (ws.cls[b] != kClsFps) continue;
+    const int n = (int)(offsets[b + 1] - offsets[b]);
+    const int q = schedule_of(n);
+    atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1);
+  }
+  __syncthreads();
+  // exclusive scan from the largest bucket down: list position of each bucket
+  if (threadIdx.x < kNumSchedules) {
+    const int q = threadIdx.x;
+    int run = 0;
+    for (int i = kBins - 1; i >= 0; --i) {
+      const int h = hist[q][i];
+      hist[q][i] = run;
+      run += h;
+    }
+    cnt[q] = run;
+  }
+  __syncthreads();
+  // pass 3: scatter into the sorted lists; chunks and accumulator slots
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int cls = ws.cls[b];
     int fslot = -1, pslot = -1;
+    int n = 0;
+    if (cls == kClsFps || cls == kClsPass) n = (int)(offsets[b + 1] - offsets[b]);
     if (cls == kClsFps) {
-      int sched = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : 3));
-      if (force > sched) sched = force > 3 ? 3 : force;
-      int* list = sched == 0 ? ws.list_warp
-                             : (sched == 1 ? ws.list_cta : (sched == 2 ? ws.list_cta_smem : ws.list_cluster));
-      list[atomicAdd(&cnt[sched], 1)] = b;
+      const int q = schedule_of(n);
+      int* list = q == 0 ? ws.list_warp
+                         : (q == 1 ? ws.list_cta
+                                   : (q == 2 ? ws.list_cta_smem : (q == 3 ? ws.list_cluster8 : ws.list_cluster16)));
+      list[atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1)] = b;
       fslot = atomicAdd(&cnt[kListFps], 1);
     }
     if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
-      const int nch = (int)((n + kChunk - 1) / kChunk);
+      const int nch = (n + kChunk - 1) / kChunk;
       const int base = atomicAdd(&cnt[kListChunks], nch);
       for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
       if (nch > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
@@ -77,9 +128,10 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
 }
 
 cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
   count_launch();
   k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
-                           ws);
+                           kLatencyEventsPerSm * di.sm_count, ws);
   return cudaGetLastError();
 }
 
@@ -268,17 +320,12 @@ __device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int
     uint64_t X[PAIRS], Y[PAIRS], Z[PAIRS], W[PAIRS];
     float best[2 * PAIRS];
     int lab[2 * PAIRS];
-    float4 pa[PAIRS], pc[PAIRS];
 #pragma unroll
     for (int p = 0; p < PAIRS; ++p) {
       const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
-      pa[p] = pc[p] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ia < i1) pa[p] = ldg4(pts + ia);
-      if (ib < i1) pc[p] = ldg4(pts + ib);
-    }
-#pragma unroll
-    for (int p = 0; p < PAIRS; ++p) {
-      const float4 a = pa[p], c = pc[p];
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+      if (ia < i1) a = ldg4(pts + ia);
+      if (ib < i1) c = ldg4(pts + ib);
       X[p] = pack2(a.x, c.x);
       Y[p] = pack2(a.y, c.y);
       Z[p] = pack2(a.z, c.z);
@@ -298,8 +345,12 @@ __device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int
 #pragma unroll
     for (int p = 0; p < PAIRS; ++p) {
       const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
-      if (ia < i1) emit(ia, nv > 0 ? (lab[2 * p] < 0 ? 0 : lab[2 * p]) : -1, pa[p]);
-      if (ib < i1) emit(ib, nv > 0 ? (lab[2 * p + 1] < 0 ? 0 : lab[2 * p + 1]) : -1, pc[p]);
+      if (ia < i1)
+        emit(ia, nv > 0 ? (lab[2 * p] < 0 ? 0 : lab[2 * p]) : -1,
+             make_float4(lo2(X[p]), lo2(Y[p]), lo2(Z[p]), lo2(W[p])));
+      if (ib < i1)
+        emit(ib, nv > 0 ? (lab[2 * p + 1] < 0 ? 0 : lab[2 * p + 1]) : -1,
+             make_float4(hi2(X[p]), hi2(Y[p]), hi2(Z[p]), hi2(W[p])));
     }
   }
 }

@@ -31,11 +31,14 @@ constexpr int kDevBadStart = 2;
 constexpr int kDevBadToken = 3;
 constexpr int kDevTooLarge = 4;
 
-// Workspace header: status word, detail word, then counters.
+// Workspace header: status word, detail word, work-list sizes and the
+// cursors the persistent kernels take items from (all reset by the binning
+// kernel at the start of every call).
 struct WsHeader {
   int status;
   int detail;
   int n_items[14];  // per work list
+  int next_item[8];  // per schedule: next unclaimed item
 };
 
 __device__ __forceinline__ void record_error(WsHeader* h, int code) {

@@ -1,4 +1,4 @@
-// Farthest point sampling fused with the Voronoi labels, four schedules.
+// Farthest point sampling fused with the Voronoi labels, five schedules.
 //
 // Tokenization per the Neptune README ("How it works", step 1): farthest-point
 // sampling of every event down to K centroids with nearest-centroid (Voronoi)
@@ -17,22 +17,22 @@
 // keeps the earliest slot, label_i equals the nearest centroid with the
 // lowest slot on ties, i.e. the plain Voronoi assignment.
 //
-// Schedules (chosen per event by the binning kernel; all run concurrently,
-// the three block schedules on helper streams forked from the caller's):
-//   warp      N <= 448      one warp per event; points in registers (lane l
-//                           owns points l + 32 j); arg-max with two redux.sync.
-//   CTA       N <= 2560     one 128-thread CTA per event; points in registers;
-//                           warp results exchanged through shared memory,
-//                           one barrier per step.
-//   CTA-smem  N <= 12288    one 256-thread CTA per event; points in shared
-//                           memory as packed f32x2 pairs; distances and labels
-//                           in registers.
-//   cluster   N <= 196608   a 16-CTA thread-block cluster per event (same
-//                           layout); every warp posts its candidate into every
-//                           CTA's shared memory over DSMEM; one
-//                           barrier.cluster per step.
-// Every step touches exactly the occupied point pairs: the unrolled per-pair
-// code is entered through a switch on the pair count (no per-pair guards).
+// Schedules (chosen per event by the binning kernel; they run concurrently,
+// the block schedules on helper streams forked from the caller's stream):
+//   warp        N <= 448     one warp per event, points in registers (lane l
+//                            owns points l + 32 j); arg-max by two redux.sync.
+//   CTA         N <= 2560    one 256-thread CTA per event, points in
+//                            registers; warp winners exchanged through shared
+//                            memory, one barrier per step.  Also takes the
+//                            warp-class events when there are few events.
+//   CTA-smem    N <= 12288   one 256-thread CTA per event, points in shared
+//                            memory as packed f32x2 pairs.
+//   cluster-8   N <= 98304   an 8-CTA cluster per event (same layout); every
+//   cluster-16  N <= 196608  warp posts its winner into every CTA's shared
+//                            memory over DSMEM; one barrier.cluster per step.
+// Each event runs a step loop compiled for its exact number of point pairs
+// (one dispatch per event), and work items are claimed from a counter in
+// decreasing size order so that the longest chains start first.
 #include <cooperative_groups.h>
 
 #include <mutex>
@@ -44,26 +44,89 @@ namespace cg = cooperative_groups;
 
 namespace fpstok {
 
-// Runs BODY(p) for p = np-1 down to 0 (np <= 24): the switch enters the
-// unrolled sequence at the right place.  BODY(p) is compiled only for
-// p < kMaxPairs, a constexpr in the calling scope.
-#define FPS_CASE(p, BODY) \
-  case (p) + 1:           \
-    if constexpr ((p) < kMaxPairs) { BODY(p) } [[fallthrough]];
-#define FPS_FALL(np, BODY)                                                                                   \
-  switch (np) {                                                                                              \
-    FPS_CASE(23, BODY) FPS_CASE(22, BODY) FPS_CASE(21, BODY) FPS_CASE(20, BODY) FPS_CASE(19, BODY)          \
-    FPS_CASE(18, BODY) FPS_CASE(17, BODY) FPS_CASE(16, BODY) FPS_CASE(15, BODY) FPS_CASE(14, BODY)          \
-    FPS_CASE(13, BODY) FPS_CASE(12, BODY) FPS_CASE(11, BODY) FPS_CASE(10, BODY) FPS_CASE(9, BODY)           \
-    FPS_CASE(8, BODY) FPS_CASE(7, BODY) FPS_CASE(6, BODY) FPS_CASE(5, BODY) FPS_CASE(4, BODY)               \
-    FPS_CASE(3, BODY) FPS_CASE(2, BODY) FPS_CASE(1, BODY) FPS_CASE(0, BODY) default : break;                \
-  }
-
 __device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xffffffffu : ((1u << n) - 1u); }
 
-// ------------------------------------------------------------------ warp
+// Dispatches CALL(N) for the compile-time N that equals the runtime np
+// (N <= kMaxPairs).
+#define FPS_CASE(N, CALL) \
+  case N:                 \
+    if constexpr ((N) <= kMaxPairs) { CALL(N); } break;
+#define FPS_DISPATCH_7(np, CALL) \
+  switch (np) { FPS_CASE(1, CALL) FPS_CASE(2, CALL) FPS_CASE(3, CALL) FPS_CASE(4, CALL) FPS_CASE(5, CALL) \
+                FPS_CASE(6, CALL) FPS_CASE(7, CALL) default : break; }
 
+// One FPS event on one warp, NP point pairs per lane.
 template <int NP>
+__device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
+                                           int lane, DupPoint* s_dup, int32_t* __restrict__ cidx,
+                                           float4* __restrict__ cpos, int32_t* __restrict__ tok) {
+  uint64_t X[NP], Y[NP], Z[NP], T[NP];
+  float dist[2 * NP];
+  int lab[2 * NP];
+  unsigned taken = 0;  // bit j: slot j (point 32 j + lane) is selected or empty
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int i0 = 64 * p + lane, i1 = i0 + 32;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (i0 < n) a = ldg4(pts + i0);
+    if (i1 < n) b = ldg4(pts + i1);
+    if (i0 < n) s_dup[i0] = dup_point(a);
+    if (i1 < n) s_dup[i1] = dup_point(b);
+    X[p] = pack2(a.x, b.x);
+    Y[p] = pack2(a.y, b.y);
+    Z[p] = pack2(a.z, b.z);
+    T[p] = pack2(a.w, b.w);
+    dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+    dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+    lab[2 * p] = 0;
+    lab[2 * p + 1] = 0;
+    if (i0 >= n) taken |= 1u << (2 * p);
+    if (i1 >= n) taken |= 1u << (2 * p + 1);
+  }
+  __syncwarp();
+  for (int s = 0; s < K; ++s) {
+    const DupPoint cp = s_dup[c];
+    if (lane == 0) {
+      cidx[s] = (int32_t)(off + c);
+      cpos[s] = dup_to_float4(cp);
+    }
+    if ((c & 31) == lane) taken |= 1u << (c >> 5);
+    const Cent2 C = cent2_dup(cp);
+    float m0 = kEmptySlot, m1 = kEmptySlot;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);
+      relax(lo2(d), dist[2 * p], lab[2 * p], s);
+      relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
+      if (p & 1)
+        m1 = max3f(m1, dist[2 * p], dist[2 * p + 1]);
+      else
+        m0 = max3f(m0, dist[2 * p], dist[2 * p + 1]);
+    }
+    if (s == K - 1) break;
+    const int M = __reduce_max_sync(kFull, fkey(fmaxf(m0, m1)));
+    unsigned cand = 0xffffffffu;  // lowest slot of this lane holding the maximum
+#pragma unroll
+    for (int j = 2 * NP - 1; j >= 0; --j) cand = fkey(dist[j]) == M ? (unsigned)(j * 32 + lane) : cand;
+    unsigned idx = __reduce_min_sync(kFull, cand);
+    if (M == 0) {  // only duplicates of chosen points remain
+      const unsigned free_slots = ~taken & low_bits(2 * NP);
+      cand = free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu;
+      idx = __reduce_min_sync(kFull, cand);
+    }
+    c = (int)idx;
+  }
+  if (tok) {
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < n) tok[i] = lab[j];
+    }
+  }
+  __syncwarp();  // the next event overwrites this warp's copy
+}
+
+template <int NPMAX>
 __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ coords,
                                                      const int64_t* __restrict__ offsets,
                                                      const int32_t* __restrict__ start_local,
@@ -71,122 +134,73 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
                                                      float4* __restrict__ centroids) {
-  constexpr int kMaxPairs = NP;
-  static_assert(2 * NP <= 32, "selected-slot mask is 32 bits");
+  constexpr int kMaxPairs = NPMAX;
+  static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
   extern __shared__ DupPoint s_dup_all[];
   const int lane = threadIdx.x & 31;
-  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NP);  // this warp's event copy
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
+  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
   const int count = hdr->n_items[kListWarp];
-
-  for (int w = gw; w < count; w += nw) {
+  for (;;) {
+    int w = 0;
+    if (lane == 0) w = atomicAdd(&hdr->next_item[kListWarp], 1);
+    w = __shfl_sync(kFull, w, 0);
+    if (w >= count) break;
     const int b = list[w];
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    const int npairs = (n + 63) >> 6;
-    const float4* pts = coords + off;
-
-    uint64_t X[NP], Y[NP], Z[NP], T[NP];
-    float dist[2 * NP];
-    int lab[2 * NP];
-    unsigned taken = 0;  // bit j: slot j (point 32 j + lane) is selected or empty
-#pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      const int i0 = 64 * p + lane, i1 = i0 + 32;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-      if (p < npairs) {
-        if (i0 < n) a = ldg4(pts + i0);
-        if (i1 < n) c = ldg4(pts + i1);
-        if (i0 < n) s_dup[i0] = dup_point(a);
-        if (i1 < n) s_dup[i1] = dup_point(c);
-      }
-      X[p] = pack2(a.x, c.x);
-      Y[p] = pack2(a.y, c.y);
-      Z[p] = pack2(a.z, c.z);
-      T[p] = pack2(a.w, c.w);
-      dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-      dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-      lab[2 * p] = 0;
-      lab[2 * p + 1] = 0;
-      if (i0 >= n) taken |= 1u << (2 * p);
-      if (i1 >= n) taken |= 1u << (2 * p + 1);
-    }
-    __syncwarp();
-
-    int c = start_local ? start_local[b] : 0;
-    for (int s = 0; s < K; ++s) {
-      const DupPoint cp = s_dup[c];
-      if (lane == 0) {
-        centroid_idx[(int64_t)b * K + s] = (int32_t)(off + c);
-        centroids[(int64_t)b * K + s] = dup_to_float4(cp);
-      }
-      if ((c & 31) == lane) taken |= 1u << (c >> 5);
-      const Cent2 C = cent2_dup(cp);
-      float m0 = kEmptySlot, m1 = kEmptySlot;
-#define W_UPD(p)                                                  \
-  {                                                               \
-    const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);          \
-    relax(lo2(d), dist[2 * (p)], lab[2 * (p)], s);                \
-    relax(hi2(d), dist[2 * (p) + 1], lab[2 * (p) + 1], s);        \
-    if ((p) & 1)                                                  \
-      m1 = max3f(m1, dist[2 * (p)], dist[2 * (p) + 1]);           \
-    else                                                          \
-      m0 = max3f(m0, dist[2 * (p)], dist[2 * (p) + 1]);           \
-  }
-      FPS_FALL(npairs, W_UPD)
-#undef W_UPD
-      if (s == K - 1) break;
-      const int key = fkey(fmaxf(m0, m1));
-      const int M = __reduce_max_sync(kFull, key);
-      unsigned cand = 0xffffffffu;
-      if (key == M) {
-#define W_SCAN(p)                                                                         \
-  {                                                                                       \
-    if (fkey(dist[2 * (p) + 1]) == M) cand = (unsigned)((2 * (p) + 1) * 32 + lane);       \
-    if (fkey(dist[2 * (p)]) == M) cand = (unsigned)((2 * (p)) * 32 + lane);               \
-  }
-        FPS_FALL(npairs, W_SCAN)
-#undef W_SCAN
-      }
-      unsigned idx = __reduce_min_sync(kFull, cand);
-      if (M == 0) {  // only duplicates of chosen points remain
-        const unsigned free_slots = ~taken & low_bits(2 * npairs);
-        cand = free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu;
-        idx = __reduce_min_sync(kFull, cand);
-      }
-      c = (int)idx;
-    }
-    if (token_id) {
-#pragma unroll
-      for (int j = 0; j < 2 * NP; ++j) {
-        const int i = j * 32 + lane;
-        if (i < n) token_id[off + i] = lab[j];
-      }
-    }
-    __syncwarp();  // the next event overwrites this warp's copy
+    const int c0 = start_local ? start_local[b] : 0;
+    int32_t* tok = token_id ? token_id + off : nullptr;
+#define WARP_CALL(N)                                                                                   \
+  warp_event<N>(coords + off, n, c0, K, off, lane, s_dup, centroid_idx + (int64_t)b * K,               \
+                centroids + (int64_t)b * K, tok)
+    FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
+#undef WARP_CALL
   }
 }
 
 // ------------------------------------------------------------------ CTA, points in registers
 
-template <int PR>
-__global__ void __launch_bounds__(128, 1) k_fps_cta(const float4* __restrict__ coords,
-                                                    const int64_t* __restrict__ offsets,
-                                                    const int32_t* __restrict__ start_local,
-                                                    const int* __restrict__ list, WsHeader* hdr, int K,
-                                                    int32_t* __restrict__ centroid_idx,
-                                                    int32_t* __restrict__ token_id,
-                                                    float4* __restrict__ centroids) {
-  constexpr int kMaxPairs = PR;
-  constexpr int NT = 128, NW = 4;
-  static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
-  extern __shared__ DupPoint s_dup[];  // [256 * PR] event copy for centroid look-up
-  __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int count = hdr->n_items[kListCta];
-  int round = 0;
+// Claims the next item of `list_id` for the whole CTA (thread 0 draws, the
+// others read it after the barrier).
+__device__ __forceinline__ int claim_cta(WsHeader* hdr, int list_id, int* slot) {
+  __syncthreads();
+  if (threadIdx.x == 0) *slot = atomicAdd(&hdr->next_item[list_id], 1);
+  __syncthreads();
+  return *slot;
+}
 
+template <int NP, int NT>
+__device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
+                                          DupPoint* s_dup, int2* xk, int& round, int32_t* __restrict__ cidx,
+                                          float4* __restrict__ cpos, int32_t* __restrict__ tok) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t X[NP], Y[NP], Z[NP], T[NP];
+  float dist[2 * NP];
+  int lab[2 * NP];
+  unsigned taken = 0;  // bit j: slot j (point NT j + tid) is selected or empty
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int i0 = 2 * NT * p + tid, i1 = i0 + NT;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (i0 < n) a = ldg4(pts + i0);
+    if (i1 < n) b = ldg4(pts + i1);
+    if (i0 < n) s_dup[i0] = dup_point(a);
+    if (i1 < n) s_dup[i1] = dup_point(b);
+    X[p] = pack2(a.x, b.x);
+    Y[p] = pack2(a.y, b.y);
+    Z[p] = pack2(a.z, b.z);
+    T[p] = pack2(a.w, b.w);
+    dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+    dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+    lab[2 * p] = 0;
+    lab[2 * p + 1] = 0;
+    if (i0 >= n) taken |= 1u << (2 * p);
+    if (i1 >= n) taken |= 1u << (2 * p + 1);
+  }
+  __syncthreads();
+
+  // one exchange round: every warp posts (key, index), all warps reduce them
   auto exchange = [&](int wkey, unsigned widx, int& M, unsigned& idx) {
     if (lane == 0) xk[(round & 1) * NW + warp] = make_int2(wkey, (int)widx);
     __syncthreads();
@@ -195,134 +209,102 @@ __global__ void __launch_bounds__(128, 1) k_fps_cta(const float4* __restrict__ c
     ++round;
   };
 
-  for (int item = blockIdx.x; item < count; item += gridDim.x) {
+  for (int s = 0; s < K; ++s) {
+    const DupPoint cp = s_dup[c];
+    if (tid == 0) {
+      cidx[s] = (int32_t)(off + c);
+      cpos[s] = dup_to_float4(cp);
+    }
+    if (c % NT == tid) taken |= 1u << (c / NT);
+    const Cent2 C = cent2_dup(cp);
+    float m0 = kEmptySlot, m1 = kEmptySlot;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);
+      relax(lo2(d), dist[2 * p], lab[2 * p], s);
+      relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
+      if (p & 1)
+        m1 = max3f(m1, dist[2 * p], dist[2 * p + 1]);
+      else
+        m0 = max3f(m0, dist[2 * p], dist[2 * p + 1]);
+    }
+    if (s == K - 1) break;
+    const int wM = __reduce_max_sync(kFull, fkey(fmaxf(m0, m1)));
+    unsigned cand = 0xffffffffu;
+#pragma unroll
+    for (int j = 2 * NP - 1; j >= 0; --j) cand = fkey(dist[j]) == wM ? (unsigned)(j * NT + tid) : cand;
+    const unsigned widx = __reduce_min_sync(kFull, cand);
+    int M;
+    unsigned idx;
+    exchange(wM, widx, M, idx);
+    if (M == 0) {  // only duplicates of chosen points remain
+      const unsigned free_slots = ~taken & low_bits(2 * NP);
+      const unsigned mine = free_slots ? (unsigned)((__ffs(free_slots) - 1) * NT + tid) : 0xffffffffu;
+      const unsigned wmin = __reduce_min_sync(kFull, mine);
+      exchange(wmin != 0xffffffffu ? 1 : 0, wmin, M, idx);
+    }
+    c = (int)idx;
+  }
+  if (tok) {
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = j * NT + tid;
+      if (i < n) tok[i] = lab[j];
+    }
+  }
+}
+
+template <int PR>
+__global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __restrict__ coords,
+                                                            const int64_t* __restrict__ offsets,
+                                                            const int32_t* __restrict__ start_local,
+                                                            const int* __restrict__ list, WsHeader* hdr, int K,
+                                                            int32_t* __restrict__ centroid_idx,
+                                                            int32_t* __restrict__ token_id,
+                                                            float4* __restrict__ centroids) {
+  constexpr int kMaxPairs = PR;
+  constexpr int NT = kCtaThreads, NW = NT / 32;
+  static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
+  extern __shared__ DupPoint s_dup[];  // [2 * NT * PR] event copy for centroid look-up
+  __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
+  __shared__ int s_item;
+  const int count = hdr->n_items[kListCta];
+  int round = 0;
+  for (;;) {
+    const int item = claim_cta(hdr, kListCta, &s_item);
+    if (item >= count) break;
     const int b = list[item];
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    const int npairs = (n + 2 * NT - 1) / (2 * NT);
-    const float4* pts = coords + off;
-
-    uint64_t X[PR], Y[PR], Z[PR], T[PR];
-    float dist[2 * PR];
-    int lab[2 * PR];
-    unsigned taken = 0;  // bit j: slot j (point NT j + tid) is selected or empty
-#pragma unroll
-    for (int p = 0; p < PR; ++p) {
-      const int i0 = 2 * NT * p + tid, i1 = i0 + NT;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-      if (p < npairs) {
-        if (i0 < n) a = ldg4(pts + i0);
-        if (i1 < n) c = ldg4(pts + i1);
-        if (i0 < n) s_dup[i0] = dup_point(a);
-        if (i1 < n) s_dup[i1] = dup_point(c);
-      }
-      X[p] = pack2(a.x, c.x);
-      Y[p] = pack2(a.y, c.y);
-      Z[p] = pack2(a.z, c.z);
-      T[p] = pack2(a.w, c.w);
-      dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-      dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-      lab[2 * p] = 0;
-      lab[2 * p + 1] = 0;
-      if (i0 >= n) taken |= 1u << (2 * p);
-      if (i1 >= n) taken |= 1u << (2 * p + 1);
-    }
-    __syncthreads();
-
-    int c = start_local ? start_local[b] : 0;
-    for (int s = 0; s < K; ++s) {
-      const DupPoint cp = s_dup[c];
-      if (tid == 0) {
-        centroid_idx[(int64_t)b * K + s] = (int32_t)(off + c);
-        centroids[(int64_t)b * K + s] = dup_to_float4(cp);
-      }
-      if (c % NT == tid) taken |= 1u << (c / NT);
-      const Cent2 C = cent2_dup(cp);
-      float m0 = kEmptySlot, m1 = kEmptySlot;
-#define C_UPD(p)                                                  \
-  {                                                               \
-    const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);          \
-    relax(lo2(d), dist[2 * (p)], lab[2 * (p)], s);                \
-    relax(hi2(d), dist[2 * (p) + 1], lab[2 * (p) + 1], s);        \
-    if ((p) & 1)                                                  \
-      m1 = max3f(m1, dist[2 * (p)], dist[2 * (p) + 1]);           \
-    else                                                          \
-      m0 = max3f(m0, dist[2 * (p)], dist[2 * (p) + 1]);           \
-  }
-      FPS_FALL(npairs, C_UPD)
-#undef C_UPD
-      if (s == K - 1) break;
-      const int key = fkey(fmaxf(m0, m1));
-      const int wM = __reduce_max_sync(kFull, key);
-      unsigned cand = 0xffffffffu;
-      if (key == wM) {
-#define C_SCAN(p)                                                                      \
-  {                                                                                    \
-    if (fkey(dist[2 * (p) + 1]) == wM) cand = (unsigned)((2 * (p) + 1) * NT + tid);    \
-    if (fkey(dist[2 * (p)]) == wM) cand = (unsigned)((2 * (p)) * NT + tid);            \
-  }
-        FPS_FALL(npairs, C_SCAN)
-#undef C_SCAN
-      }
-      const unsigned widx = __reduce_min_sync(kFull, cand);
-      int M;
-      unsigned idx;
-      exchange(wM, widx, M, idx);
-      if (M == 0) {  // only duplicates of chosen points remain
-        const unsigned free_slots = ~taken & low_bits(2 * npairs);
-        const unsigned mine = free_slots ? (unsigned)((__ffs(free_slots) - 1) * NT + tid) : 0xffffffffu;
-        const unsigned wmin = __reduce_min_sync(kFull, mine);
-        exchange(wmin != 0xffffffffu ? 1 : 0, wmin, M, idx);
-      }
-      c = (int)idx;
-    }
-    if (token_id) {
-#pragma unroll
-      for (int j = 0; j < 2 * PR; ++j) {
-        const int i = j * NT + tid;
-        if (i < n) token_id[off + i] = lab[j];
-      }
-    }
-    __syncthreads();  // the next event overwrites the shared copy
+    const int c0 = start_local ? start_local[b] : 0;
+    int32_t* tok = token_id ? token_id + off : nullptr;
+#define CTA_CALL(N)                                                                                     \
+  cta_event<N, NT>(coords + off, n, c0, K, off, s_dup, xk, round, centroid_idx + (int64_t)b * K,        \
+                   centroids + (int64_t)b * K, tok)
+    FPS_DISPATCH_7((n + 2 * NT - 1) / (2 * NT), CTA_CALL)
+#undef CTA_CALL
   }
 }
 
 // ------------------------------------------------------------------ CTA / cluster, points in shared memory
 
-template <int CL, int NT, int PS>
-__global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ coords,
-                                                     const int64_t* __restrict__ offsets,
-                                                     const int32_t* __restrict__ start_local,
-                                                     const int* __restrict__ list, WsHeader* hdr,
-                                                     int list_id, int K,
-                                                     int32_t* __restrict__ centroid_idx,
-                                                     int32_t* __restrict__ token_id,
-                                                     float4* __restrict__ centroids) {
-  constexpr int kMaxPairs = PS;
-  static_assert(2 * PS <= 64, "selected-slot mask is 64 bits");
+template <int CL, int NT>
+struct BlockShared {
+  static constexpr int NW = NT / 32;
+  static constexpr int E = CL * NW;  // posted entries per exchange round
+};
+
+template <int NP, int CL, int NT>
+__device__ __forceinline__ void block_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
+                                            int rank, ulonglong2* sXY, ulonglong2* sZT, int2* xkey, float4* xpos,
+                                            int& round, int32_t* __restrict__ cidx, float4* __restrict__ cpos,
+                                            int32_t* __restrict__ tok) {
   constexpr int NW = NT / 32;
   constexpr int E = CL * NW;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  ulonglong2* sXY = reinterpret_cast<ulonglong2*>(smem_raw);  // [PS][NT] packed (x, y)
-  ulonglong2* sZT = sXY + PS * NT;                            // [PS][NT] packed (z, t)
-  int2* xkey = reinterpret_cast<int2*>(sZT + PS * NT);        // [2][E] (key, index)
-  float4* xpos = reinterpret_cast<float4*>(xkey + 2 * E);     // [2][E] candidate position
-
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  int rank = 0;
-  if constexpr (CL > 1) {
-    rank = (int)cg::this_cluster().block_rank();
-    cg::this_cluster().sync();  // every CTA of the cluster is running before DSMEM use
-  }
-  const int G = CL * NT;
+  constexpr int G = CL * NT;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = rank * NT + tid;
-  const int nclusters = gridDim.x / CL;
-  const int count = hdr->n_items[list_id];
-  int round = 0;
 
-  // Posts (key, idx, pos) of this warp into slot [round&1][rank*NW+warp] of every CTA.
   auto post = [&](int key, unsigned idx, float4 pos) {
     const int slot = (round & 1) * E + rank * NW + warp;
     if constexpr (CL > 1) {
@@ -347,7 +329,6 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
       __syncthreads();
     }
   };
-  // Reduces the posted entries of this round: largest key, then smallest index.
   auto gather = [&](int& M, unsigned& idx, float4& pos) {
     const int base = (round & 1) * E;
     int bk = -0x7fffffff - 1;
@@ -368,7 +349,6 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     pos = xpos[base + e];
     ++round;
   };
-  // Position of a point this CTA holds, from its shared-memory pair.
   auto local_pos = [&](unsigned idx) {
     const int gi = (int)(idx % (unsigned)G);
     const int j = (int)(idx / (unsigned)G);
@@ -379,140 +359,193 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
                    : make_float4(lo2(xy.x), lo2(xy.y), lo2(zt.x), lo2(zt.y));
   };
 
-  for (int item = blockIdx.x / CL; item < count; item += nclusters) {
+  float dist[2 * NP];
+  int lab[2 * NP];
+  unsigned long long taken = 0;
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int i0 = g + G * (2 * p), i1 = i0 + G;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (i0 < n) a = ldg4(pts + i0);
+    if (i1 < n) b = ldg4(pts + i1);
+    sXY[p * NT + tid] = make_ulonglong2(pack2(a.x, b.x), pack2(a.y, b.y));
+    sZT[p * NT + tid] = make_ulonglong2(pack2(a.z, b.z), pack2(a.w, b.w));
+    dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+    dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
+    lab[2 * p] = 0;
+    lab[2 * p + 1] = 0;
+    if (i0 >= n) taken |= 1ull << (2 * p);
+    if (i1 >= n) taken |= 1ull << (2 * p + 1);
+  }
+
+  float4 cc = ldg4(pts + c);
+  for (int s = 0; s < K; ++s) {
+    if (rank == 0 && tid == 0) {
+      cidx[s] = (int32_t)(off + c);
+      cpos[s] = cc;
+    }
+    if (c % G == g) taken |= 1ull << (c / G);
+    const Cent2 C = cent2(cc);
+    float m0 = kEmptySlot, m1 = kEmptySlot;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const ulonglong2 xy = sXY[p * NT + tid];
+      const ulonglong2 zt = sZT[p * NT + tid];
+      const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C);
+      relax(lo2(d), dist[2 * p], lab[2 * p], s);
+      relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
+      if (p & 1)
+        m1 = max3f(m1, dist[2 * p], dist[2 * p + 1]);
+      else
+        m0 = max3f(m0, dist[2 * p], dist[2 * p + 1]);
+    }
+    if (s == K - 1) break;
+    const int wM = __reduce_max_sync(kFull, fkey(fmaxf(m0, m1)));
+    unsigned wcand = 0xffffffffu;
+#pragma unroll
+    for (int j = 2 * NP - 1; j >= 0; --j) wcand = fkey(dist[j]) == wM ? (unsigned)(g + G * j) : wcand;
+    const unsigned widx = __reduce_min_sync(kFull, wcand);
+    float4 wpos = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (wM >= 0) wpos = local_pos(widx);
+    post(wM, widx, wpos);
+    barrier();
+    int M;
+    unsigned idx;
+    gather(M, idx, cc);
+    if (M == 0) {  // only duplicates of chosen points remain
+      const unsigned long long mask = 2 * NP >= 64 ? ~0ull : ((1ull << (2 * NP)) - 1ull);
+      const unsigned long long free_slots = ~taken & mask;
+      unsigned cand = 0xffffffffu;
+      if (free_slots) cand = (unsigned)(g + G * (__ffsll((long long)free_slots) - 1));
+      const unsigned wmin = __reduce_min_sync(kFull, cand);
+      float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (wmin != 0xffffffffu) p = local_pos(wmin);
+      // keys: 1 for a real candidate, 0 for none; ties resolve to the lowest index
+      post(wmin != 0xffffffffu ? 1 : 0, wmin, p);
+      barrier();
+      gather(M, idx, cc);
+    }
+    c = (int)idx;
+  }
+  if (tok) {
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = g + G * j;
+      if (i < n) tok[i] = lab[j];
+    }
+  }
+}
+
+// Pair counts compiled for the shared-memory schedules; an event uses the
+// smallest one that covers it (extra pairs hold no points).
+#define FPS_BLOCK_BUCKETS(np, CALL)                                                                     \
+  if ((np) <= 2) { CALL(2); } else if ((np) <= 4) { CALL(4); } else if ((np) <= 6) { CALL(6); }          \
+  else if ((np) <= 8) { CALL(8); } else if ((np) <= 10) { CALL(10); } else if ((np) <= 12) { CALL(12); } \
+  else if ((np) <= 14) { CALL(14); } else if ((np) <= 16) { CALL(16); } else if ((np) <= 18) { CALL(18); } \
+  else if ((np) <= 20) { CALL(20); } else if ((np) <= 22) { CALL(22); } else { CALL(24); }
+
+template <int CL, int NT, int PS>
+__global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ coords,
+                                                     const int64_t* __restrict__ offsets,
+                                                     const int32_t* __restrict__ start_local,
+                                                     const int* __restrict__ list, WsHeader* hdr,
+                                                     int list_id, int K,
+                                                     int32_t* __restrict__ centroid_idx,
+                                                     int32_t* __restrict__ token_id,
+                                                     float4* __restrict__ centroids) {
+  static_assert(2 * PS <= 64, "selected-slot mask is 64 bits");
+  constexpr int E = BlockShared<CL, NT>::E;
+  constexpr int G = CL * NT;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ulonglong2* sXY = reinterpret_cast<ulonglong2*>(smem_raw);  // [PS][NT] packed (x, y)
+  ulonglong2* sZT = sXY + PS * NT;                            // [PS][NT] packed (z, t)
+  int2* xkey = reinterpret_cast<int2*>(sZT + PS * NT);        // [2][E] (key, index)
+  float4* xpos = reinterpret_cast<float4*>(xkey + 2 * E);     // [2][E] candidate position
+  __shared__ int s_item;
+
+  int rank = 0;
+  if constexpr (CL > 1) {
+    rank = (int)cg::this_cluster().block_rank();
+    cg::this_cluster().sync();  // every CTA of the cluster is running before DSMEM use
+  }
+  const int count = hdr->n_items[list_id];
+  int round = 0;
+  for (;;) {
+    // the cluster's first CTA claims an item and hands it to the others
+    if constexpr (CL > 1) {
+      if (rank == 0 && threadIdx.x == 0) {
+        const int it = atomicAdd(&hdr->next_item[list_id], 1);
+        cg::cluster_group cl = cg::this_cluster();
+        for (int r = 0; r < CL; ++r) *cl.map_shared_rank(&s_item, r) = it;
+      }
+      cg::this_cluster().sync();
+    } else {
+      __syncthreads();
+      if (threadIdx.x == 0) s_item = atomicAdd(&hdr->next_item[list_id], 1);
+      __syncthreads();
+    }
+    const int item = s_item;
+    if (item >= count) break;
     const int b = list[item];
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    const int npairs = (n + 2 * G - 1) / (2 * G);
-    const float4* pts = coords + off;
-
-    float dist[2 * PS];
-    int lab[2 * PS];
-    unsigned long long taken = 0;
-#pragma unroll
-    for (int p = 0; p < PS; ++p) {
-      const int i0 = g + G * (2 * p), i1 = i0 + G;
-      if (p < npairs) {
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-        if (i0 < n) a = ldg4(pts + i0);
-        if (i1 < n) c = ldg4(pts + i1);
-        sXY[p * NT + tid] = make_ulonglong2(pack2(a.x, c.x), pack2(a.y, c.y));
-        sZT[p * NT + tid] = make_ulonglong2(pack2(a.z, c.z), pack2(a.w, c.w));
-      }
-      dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-      dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-      lab[2 * p] = 0;
-      lab[2 * p + 1] = 0;
-      if (i0 >= n) taken |= 1ull << (2 * p);
-      if (i1 >= n) taken |= 1ull << (2 * p + 1);
-    }
-
-    int c = start_local ? start_local[b] : 0;
-    float4 cc = ldg4(pts + c);
-    for (int s = 0; s < K; ++s) {
-      if (rank == 0 && tid == 0) {
-        centroid_idx[(int64_t)b * K + s] = (int32_t)(off + c);
-        centroids[(int64_t)b * K + s] = cc;
-      }
-      if (c % G == g) taken |= 1ull << (c / G);
-      const Cent2 C = cent2(cc);
-      float m0 = kEmptySlot, m1 = kEmptySlot;
-#define B_UPD(p)                                                   \
-  {                                                                \
-    const ulonglong2 xy = sXY[(p) * NT + tid];                     \
-    const ulonglong2 zt = sZT[(p) * NT + tid];                     \
-    const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C);           \
-    relax(lo2(d), dist[2 * (p)], lab[2 * (p)], s);                 \
-    relax(hi2(d), dist[2 * (p) + 1], lab[2 * (p) + 1], s);         \
-    if ((p) & 1)                                                   \
-      m1 = max3f(m1, dist[2 * (p)], dist[2 * (p) + 1]);            \
-    else                                                           \
-      m0 = max3f(m0, dist[2 * (p)], dist[2 * (p) + 1]);            \
-  }
-      FPS_FALL(npairs, B_UPD)
-#undef B_UPD
-      if (s == K - 1) break;
-
-      const int key = fkey(fmaxf(m0, m1));
-      const int wM = __reduce_max_sync(kFull, key);
-      unsigned wcand = 0xffffffffu;
-      if (key == wM) {
-#define B_SCAN(p)                                                                     \
-  {                                                                                   \
-    if (fkey(dist[2 * (p) + 1]) == wM) wcand = (unsigned)(g + G * (2 * (p) + 1));     \
-    if (fkey(dist[2 * (p)]) == wM) wcand = (unsigned)(g + G * (2 * (p)));             \
-  }
-        FPS_FALL(npairs, B_SCAN)
-#undef B_SCAN
-      }
-      const unsigned widx = __reduce_min_sync(kFull, wcand);
-      float4 wpos = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (wM >= 0) wpos = local_pos(widx);
-      post(wM, widx, wpos);
-      barrier();
-      int M;
-      unsigned idx;
-      gather(M, idx, cc);
-      if (M == 0) {  // only duplicates of chosen points remain
-        const int nslots = 2 * npairs;
-        const unsigned long long mask = nslots >= 64 ? ~0ull : ((1ull << nslots) - 1ull);
-        const unsigned long long free_slots = ~taken & mask;
-        unsigned cand = 0xffffffffu;
-        if (free_slots) cand = (unsigned)(g + G * (__ffsll((long long)free_slots) - 1));
-        const unsigned wmin = __reduce_min_sync(kFull, cand);
-        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (wmin != 0xffffffffu) p = local_pos(wmin);
-        // keys: 1 for a real candidate, 0 for none; ties resolve to the lowest index
-        post(wmin != 0xffffffffu ? 1 : 0, wmin, p);
-        barrier();
-        gather(M, idx, cc);
-      }
-      c = (int)idx;
-    }
-    if (token_id) {
-#pragma unroll
-      for (int j = 0; j < 2 * PS; ++j) {
-        const int i = g + G * j;
-        if (j < 2 * npairs && i < n) token_id[off + i] = lab[j];
-      }
-    }
+    const int c0 = start_local ? start_local[b] : 0;
+    int32_t* tok = token_id ? token_id + off : nullptr;
+    const int np = (n + 2 * G - 1) / (2 * G);
+#define BLOCK_CALL(N)                                                                                   \
+  block_event<N, CL, NT>(coords + off, n, c0, K, off, rank, sXY, sZT, xkey, xpos, round,                \
+                         centroid_idx + (int64_t)b * K, centroids + (int64_t)b * K, tok)
+    FPS_BLOCK_BUCKETS(np, BLOCK_CALL)
+#undef BLOCK_CALL
+    if constexpr (CL > 1) cg::this_cluster().sync();  // s_item is rewritten for the next claim
   }
   if constexpr (CL > 1) cg::this_cluster().sync();  // no CTA leaves while peers may post into it
 }
 
-#undef FPS_FALL
+#undef FPS_BLOCK_BUCKETS
+#undef FPS_DISPATCH_7
 #undef FPS_CASE
 
 // ------------------------------------------------------------------ launch
 
 constexpr int kWarpBlock = 128;
 constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(DupPoint);
-constexpr size_t kCtaSmem = (size_t)2 * 128 * kCtaPairs * sizeof(DupPoint);
+constexpr size_t kCtaSmem = (size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint);
 
 template <int CL>
 constexpr size_t block_smem_bytes() {
   return (size_t)2 * kBlockPairs * kBlockThreads * sizeof(ulonglong2) +
-         (size_t)2 * CL * (kBlockThreads / 32) * (sizeof(int2) + sizeof(float4));
+         (size_t)2 * BlockShared<CL, kBlockThreads>::E * (sizeof(int2) + sizeof(float4));
 }
 
 template <int CL>
-static cudaError_t prepare_block_kernel() {
+static cudaError_t prepare_block_kernel(int* max_active_clusters) {
   auto kern = k_fps_block<CL, kBlockThreads, kBlockPairs>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)block_smem_bytes<CL>());
   if (e != cudaSuccess) return e;
-  if (CL > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  if (CL > 8 && (e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)))
+    return e;
+  if (CL == 1) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL);
+  cfg.blockDim = dim3(kBlockThreads);
+  cfg.dynamicSmemBytes = block_smem_bytes<CL>();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaOccupancyMaxActiveClusters(max_active_clusters, kern, &cfg);
 }
 
 template <int CL>
-static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list_id, int n_groups,
-                                cudaStream_t s) {
+static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list_id, const int* list,
+                                int n_groups, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_groups * CL);
+  cfg.gridDim = dim3((n_groups > 0 ? n_groups : 1) * CL);
   cfg.blockDim = dim3(kBlockThreads);
   cfg.dynamicSmemBytes = block_smem_bytes<CL>();
   cfg.stream = s;
@@ -527,19 +560,19 @@ static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  const int* list = list_id == kListCtaSmem ? ws.list_cta_smem : ws.list_cluster;
   count_launch();
-  return cudaLaunchKernelEx(&cfg, k_fps_block<CL, kBlockThreads, kBlockPairs>, pb.coords,
-                            pb.offsets, pb.start_local, list, ws.hdr, list_id, pb.K, pb.centroid_idx,
-                            pb.token_id, pb.centroids);
+  return cudaLaunchKernelEx(&cfg, k_fps_block<CL, kBlockThreads, kBlockPairs>, pb.coords, pb.offsets,
+                            pb.start_local, list, ws.hdr, list_id, pb.K, pb.centroid_idx, pb.token_id,
+                            pb.centroids);
 }
 
 // Per-device state: occupancy figures and the helper streams / events that
-// let the four schedules run concurrently.
+// let the schedules run concurrently.
+constexpr int kHelpers = kNumSchedules - 1;
 struct DeviceCtx {
   DeviceInfo info;
-  cudaStream_t helper[3];
-  cudaEvent_t fork, join[3];
+  cudaStream_t helper[kHelpers];
+  cudaEvent_t fork, join[kHelpers];
   std::mutex launch_mu;
   bool prepared;
 };
@@ -572,24 +605,12 @@ static cudaError_t prepare(int dev) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&info.warp_blocks_per_sm, k_fps_warp<kWarpPairs>,
                                                     kWarpBlock, kWarpSmem);
   if (e != cudaSuccess) return e;
-  if ((e = prepare_block_kernel<1>()) != cudaSuccess) return e;
-  if ((e = prepare_block_kernel<kMaxCluster>()) != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kMaxCluster);
-  cfg.blockDim = dim3(kBlockThreads);
-  cfg.dynamicSmemBytes = block_smem_bytes<kMaxCluster>();
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kMaxCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaOccupancyMaxActiveClusters(&info.cluster_max_active,
-                                     k_fps_block<kMaxCluster, kBlockThreads, kBlockPairs>, &cfg);
-  if (e != cudaSuccess) return e;
+  int unused = 0;
+  if ((e = prepare_block_kernel<1>(&unused)) != cudaSuccess) return e;
+  if ((e = prepare_block_kernel<8>(&info.cluster8_max_active)) != cudaSuccess) return e;
+  if ((e = prepare_block_kernel<16>(&info.cluster16_max_active)) != cudaSuccess) return e;
   if ((e = prepare_aux_kernels()) != cudaSuccess) return e;
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < kHelpers; ++i) {
     if ((e = cudaStreamCreateWithFlags(&ctx.helper[i], cudaStreamNonBlocking))) return e;
     if ((e = cudaEventCreateWithFlags(&ctx.join[i], cudaEventDisableTiming))) return e;
   }
@@ -615,40 +636,50 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
   if (e != cudaSuccess) return e;
   DeviceCtx& ctx = g_ctx[dev];
   const DeviceInfo& di = ctx.info;
-  // Launch a schedule unless the size hint rules out every event it could get:
-  // schedule q receives events above `lower[q]` (or above K when forced).
+  // Launch a schedule unless the size hint rules out every event it could
+  // get: schedule q receives events above lower[q] (above K when forced; the
+  // CTA schedule also takes small events when there are few of them).
   const int hint = pb.max_event_hint;
   const int f = pb.force_schedule;
-  const int lower[4] = {pb.K, kWarpCap, kCtaCap, kCtaSmemCap};
-  bool run[4];
-  for (int q = 0; q < 4; ++q) {
+  const bool maybe_few = pb.B <= kLatencyEventsPerSm * di.sm_count;  // small events may move to the CTA
+  const int lower[kNumSchedules] = {pb.K, maybe_few ? pb.K : kWarpCap, kCtaCap, kCtaSmemCap, kCluster8Cap};
+  bool run[kNumSchedules];
+  for (int q = 0; q < kNumSchedules; ++q) {
     const int lo = f >= q ? pb.K : lower[q];
-    run[q] = (q == 3 || f <= q) && (hint == 0 || hint > lo);
+    const bool allowed = f < 0 || q == kNumSchedules - 1 || f <= q;
+    run[q] = allowed && (hint == 0 || hint > lo);
   }
 
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
-  const bool forked = run[1] || run[2] || run[3];
+  bool forked = false;
+  for (int q = 1; q < kNumSchedules; ++q) forked |= run[q];
   if (forked && (e = cudaEventRecord(ctx.fork, s))) return e;
-  for (int h = 0; h < 3; ++h) {
-    if (!run[h + 1]) continue;
-    cudaStream_t hs = ctx.helper[h];
+  for (int q = 1; q < kNumSchedules; ++q) {
+    if (!run[q]) continue;
+    cudaStream_t hs = ctx.helper[q - 1];
     if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
-    mark(2 + h, 0, hs);
-    if (h == 0) {
-      count_launch();
-      k_fps_cta<kCtaPairs><<<di.sm_count, 128, kCtaSmem, hs>>>(pb.coords, pb.offsets, pb.start_local, ws.list_cta,
-                                                               ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-                                                               pb.centroids);
-      e = cudaGetLastError();
-    } else if (h == 1) {
-      e = launch_block<1>(pb, ws, kListCtaSmem, di.sm_count, hs);
-    } else {
-      const int groups = di.cluster_max_active > 0 ? di.cluster_max_active : 1;
-      e = launch_block<kMaxCluster>(pb, ws, kListCluster, groups, hs);
+    mark(1 + q, 0, hs);
+    switch (q) {
+      case 1:
+        count_launch();
+        k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
+            pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
+            pb.centroids);
+        e = cudaGetLastError();
+        break;
+      case 2:
+        e = launch_block<1>(pb, ws, kListCtaSmem, ws.list_cta_smem, di.sm_count, hs);
+        break;
+      case 3:
+        e = launch_block<8>(pb, ws, kListCluster8, ws.list_cluster8, di.cluster8_max_active, hs);
+        break;
+      default:
+        e = launch_block<16>(pb, ws, kListCluster16, ws.list_cluster16, di.cluster16_max_active, hs);
+        break;
     }
     if (e != cudaSuccess) return e;
-    mark(2 + h, 1, hs);
-    if ((e = cudaEventRecord(ctx.join[h], hs))) return e;
+    mark(1 + q, 1, hs);
+    if ((e = cudaEventRecord(ctx.join[q - 1], hs))) return e;
   }
   if (run[0]) {
     const int blocks = di.sm_count * (di.warp_blocks_per_sm > 0 ? di.warp_blocks_per_sm : 1);
@@ -660,8 +691,8 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1, 1, s);
   }
-  for (int h = 0; h < 3; ++h)
-    if (run[h + 1] && (e = cudaStreamWaitEvent(s, ctx.join[h], 0))) return e;
+  for (int q = 1; q < kNumSchedules; ++q)
+    if (run[q] && (e = cudaStreamWaitEvent(s, ctx.join[q - 1], 0))) return e;
   return cudaSuccess;
 }
 

@@ -13,7 +13,7 @@ namespace fpstok {
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
-static void* g_stage_events[16];
+static void* g_stage_events[32];
 static int g_n_stage_events = 0;
 
 void stage_mark(int stage, int end, cudaStream_t s) {
@@ -48,7 +48,8 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   w.list_warp = c.take<int>(nb);
   w.list_cta = c.take<int>(nb);
   w.list_cta_smem = c.take<int>(nb);
-  w.list_cluster = c.take<int>(nb);
+  w.list_cluster8 = c.take<int>(nb);
+  w.list_cluster16 = c.take<int>(nb);
   w.chunks = c.take<int2>(chunks);
   w.cls = c.take<int>(nb);
   w.fps_slot = c.take<int>(nb);
@@ -88,7 +89,7 @@ static int check_opts(const fps_opts* o, int F) {
   if (F < 1) return FPS_ERR_ARG;
   if (F > FPS_MAX_F) return FPS_ERR_TOO_LARGE;
   if (o->charge_col < -1 || o->charge_col >= F) return FPS_ERR_ARG;
-  if (o->force_schedule < -1 || o->force_schedule > 3) return FPS_ERR_ARG;
+  if (o->force_schedule < -1 || o->force_schedule > 4) return FPS_ERR_ARG;
   if (o->max_event_hint < 0) return FPS_ERR_ARG;
   if (o->max_event_hint > kClusterCap) return FPS_ERR_TOO_LARGE;
   return FPS_OK;
@@ -112,21 +113,21 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
   stage_mark(0, 1, s);
   if ((e = launch_fps(pb, ws, s, stage_mark))) return from_cuda(e);
   if (pb.lloyd_iters > 0) {
-    stage_mark(5, 0, s);
+    stage_mark(6, 0, s);
     if ((e = launch_lloyd(pb, ws, labels, s))) return from_cuda(e);
-    stage_mark(5, 1, s);
+    stage_mark(6, 1, s);
   }
   if (pb.assign_mode == FPS_ASSIGN_KNN) {
-    stage_mark(6, 0, s);
+    stage_mark(7, 0, s);
     if ((e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx,
                         pb.feats, pb.F, pb.pooled, pb.counts, ws.cls, ws.hdr, s)))
       return from_cuda(e);
-    stage_mark(6, 1, s);
+    stage_mark(7, 1, s);
   } else {
-    stage_mark(7, 0, s);
+    stage_mark(8, 0, s);
     if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.K, labels, pb.pooled, pb.counts, ws, s)))
       return from_cuda(e);
-    stage_mark(7, 1, s);
+    stage_mark(8, 1, s);
   }
   return FPS_OK;
 }
@@ -142,9 +143,9 @@ int64_t fps_max_event_points(void) { return kClusterCap; }
 int fps_schedule_for(int64_t n, int K, int force_schedule) {
   if (n > kClusterCap) return -2;
   if (n <= 0 || n <= K) return -1;
-  int sched = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : 3));
-  if (force_schedule > sched) sched = force_schedule > 3 ? 3 : force_schedule;
-  return sched;
+  int q = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : (n <= kCluster8Cap ? 3 : 4)));
+  if (force_schedule > q) q = force_schedule > 4 ? 4 : force_schedule;
+  return q;
 }
 
 size_t fps_workspace_bytes(int64_t P, int B, int F, const fps_opts* opts) {
@@ -348,13 +349,13 @@ int lloyd_refine(const float* coords, const float* feats, int F, int charge_col,
   pb.force_schedule = -1;
   pb.centroids = reinterpret_cast<float4*>(centroids);
   cudaError_t e;
-  stage_mark(5, 0, s);
+  stage_mark(6, 0, s);
   if ((e = launch_bin(pb, ws, 0, s))) return from_cuda(e);
   const size_t zbytes = (size_t)ws.fps_slots * K * 5 * sizeof(double);
   if ((e = cudaMemsetAsync(ws.lloyd[0], 0, zbytes, s)) || (e = cudaMemsetAsync(ws.lloyd[1], 0, zbytes, s)))
     return from_cuda(e);
   if ((e = launch_lloyd(pb, ws, token_id, s))) return from_cuda(e);
-  stage_mark(5, 1, s);
+  stage_mark(6, 1, s);
   return FPS_OK;
 }
 
@@ -442,7 +443,7 @@ void fps_set_stage_events(void* const* events, int n_events) {
     g_n_stage_events = 0;
     return;
   }
-  if (n_events > 16) n_events = 16;
+  if (n_events > 32) n_events = 32;
   for (int i = 0; i < n_events; ++i) g_stage_events[i] = events[i];
   g_n_stage_events = n_events;
 }

@@ -14,31 +14,39 @@ enum ListId : int {
   kListWarp = 0,
   kListCta = 1,
   kListCtaSmem = 2,
-  kListCluster = 3,
-  kListChunks = 4,     // (event, chunk) items of FPS events
-  kListPoolSlots = 5,  // events that need global pooling accumulators
-  kListFps = 6,        // number of FPS events (Lloyd slots)
-  kNumLists = 7,
+  kListCluster8 = 3,
+  kListCluster16 = 4,
+  kListChunks = 5,     // (event, chunk) items of FPS events
+  kListPoolSlots = 6,  // events that need global pooling accumulators
+  kListFps = 7,        // number of FPS events (Lloyd slots)
+  kNumLists = 8,
 };
+constexpr int kNumSchedules = 5;  // warp, CTA, CTA-smem, 8-CTA cluster, 16-CTA cluster
 
 // Schedule capacities (points per event).
 constexpr int kWarpPairs = 7;                          // point pairs per lane, warp schedule
 constexpr int kWarpCap = 64 * kWarpPairs;              // 448
-constexpr int kCtaPairs = 10;                          // pairs per thread, 128-thread CTA
-constexpr int kCtaCap = 256 * kCtaPairs;               // 2560
+constexpr int kCtaThreads = 256;                       // register-resident CTA schedule
+constexpr int kCtaPairs = 5;                           // pairs per thread
+constexpr int kCtaCap = 2 * kCtaThreads * kCtaPairs;   // 2560
 constexpr int kBlockThreads = 256;                     // shared-memory CTA / cluster schedules
 constexpr int kBlockPairs = 24;                        // pairs per thread in shared memory
 constexpr int kCtaSmemCap = kBlockThreads * 2 * kBlockPairs;  // 12288
+constexpr int kCluster8Cap = 8 * kCtaSmemCap;                 // 98304
 constexpr int kMaxCluster = 16;
 constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
-constexpr int kChunk = 1024;                           // points per pooling / Lloyd work item
+constexpr int kChunk = 2048;                           // points per pooling / Lloyd work item
+// With at most this many FPS events per SM, events of the warp class run on
+// the CTA schedule instead (lower latency per step when the GPU is not full).
+constexpr int kLatencyEventsPerSm = 1;
 
 struct Workspace {
   struct WsHeader* hdr;
   int* list_warp;
   int* list_cta;
   int* list_cta_smem;
-  int* list_cluster;
+  int* list_cluster8;
+  int* list_cluster16;
   int2* chunks;     // (event, chunk)
   int* cls;         // EventClass per event
   int* fps_slot;    // compact index of FPS events, -1 otherwise
@@ -95,7 +103,8 @@ cudaError_t launch_pool_knn(const float* feats, int F, int B, int K, int k, cons
 struct DeviceInfo {
   int sm_count;
   int warp_blocks_per_sm;
-  int cluster_max_active;  // clusters of kMaxCluster CTAs of the cluster kernel
+  int cluster8_max_active;   // co-resident 8-CTA clusters of the shared-memory kernel
+  int cluster16_max_active;  // co-resident 16-CTA clusters
   bool ready;
 };
 const DeviceInfo& device_info();  // prepares the current device on first use

@@ -94,8 +94,8 @@ enum {
 
 /* force_schedule: -1 picks by event size; 0 warp (N <= 448), 1 CTA with points
  * in registers (N <= 2560), 2 CTA with points in shared memory (N <= 12288),
- * 3 16-CTA cluster (N <= 196608) means "use at least this schedule" (events
- * too large for it move up). */
+ * 3 8-CTA cluster (N <= 98304), 4 16-CTA cluster (N <= 196608) means "use at
+ * least this schedule" (events too large for it move up). */
 typedef struct fps_opts {
     int K;             /* maximum tokens per event, 1..FPS_MAX_K */
     int assign_mode;   /* FPS_ASSIGN_VORONOI or FPS_ASSIGN_KNN */
@@ -231,16 +231,17 @@ uint64_t fps_launch_count(void);
  * launching stream (the block schedules run on internal helper streams forked
  * from it; their events are recorded there).  Stages: 0 binning +
  * passthrough, 1 FPS warp schedule, 2 FPS CTA schedule, 3 FPS CTA
- * shared-memory schedule, 4 FPS cluster schedule, 5 Lloyd, 6 kNN gather +
- * pool, 7 Voronoi pool.  A stage that does not run records nothing.  The events
- * are cudaEvent_t handles the caller created; at most 16 are used.  Pass
- * NULL to turn it off.  Not thread-safe: meant for benchmarks.
+ * shared-memory schedule, 4 FPS 8-CTA cluster, 5 FPS 16-CTA cluster, 6 Lloyd,
+ * 7 kNN gather + pool, 8 Voronoi pool.  A stage that does not run records
+ * nothing.  The events are cudaEvent_t handles the caller created; at most 32
+ * are used.  Pass NULL to turn it off.  Not thread-safe: meant for benchmarks.
  */
 void fps_set_stage_events(void *const *events, int n_events);
 
 /* Schedule fps_tokenize gives an event of n points: -1 none (n <= K, or n = 0),
- * 0 warp, 1 CTA, 2 CTA shared-memory, 3 cluster; -2 if n exceeds
- * fps_max_event_points(). */
+ * 0 warp, 1 CTA, 2 CTA shared-memory, 3 8-CTA cluster, 4 16-CTA cluster; -2
+ * if n exceeds fps_max_event_points().  When a batch has at most one FPS event
+ * per SM, events of class 0 run on schedule 1 instead. */
 int fps_schedule_for(int64_t n, int K, int force_schedule);
 
 #ifdef __cplusplus

@@ -68,7 +68,7 @@ def test_host_side_argument_errors():
     assert _tok(lib, O(K=16), F=65) == _lib.FPS_ERR_TOO_LARGE
     assert _tok(lib, O(K=16), P=1 << 31) == _lib.FPS_ERR_TOO_LARGE
     assert _tok(lib, O(K=16), B=-1) == _lib.FPS_ERR_ARG
-    assert _tok(lib, O(K=16, force_schedule=4)) == _lib.FPS_ERR_ARG
+    assert _tok(lib, O(K=16, force_schedule=5)) == _lib.FPS_ERR_ARG
     assert _tok(lib, O(K=16), coords=8) == _lib.FPS_ERR_ARG  # misaligned float4 rows
     assert _tok(lib, O(K=16), tok=0) == _lib.FPS_ERR_ARG  # Voronoi needs token_id
     assert _tok(lib, O(K=16, assign_mode="knn", k=4), knn=0) == _lib.FPS_ERR_ARG

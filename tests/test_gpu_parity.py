@@ -46,7 +46,7 @@ def test_c1_host_offsets_hint():
 # ------------------------------------------------------------- sizes, tiles, ragged tails
 
 EDGE_SIZES = [0, 1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 447, 448, 449, 1000, 2559, 2560,
-              2561, 4095, 12287, 12288, 12289, 30001]
+              2561, 4095, 12287, 12288, 12289, 30001, 98305]
 
 
 @pytest.mark.parametrize("K", [1, 2, 16, 128, 256])
@@ -70,9 +70,9 @@ def test_ties_and_duplicates(kind):
     compare(b, run_gpu(b))
 
 
-@pytest.mark.parametrize("force", [0, 1, 2, 3])
+@pytest.mark.parametrize("force", [0, 1, 2, 3, 4])
 def test_forced_schedules_agree(force):
-    sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000]
+    sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000, 98304, 98305]
     b = workloads.random_batch(11, sizes, 128, dup_frac=0.05)
     ora = oracle.tokenize_batch(b)
     compare(b, run_gpu(b, force_schedule=force), ora)
@@ -222,6 +222,12 @@ def test_dtype_is_not_converted():
         fps.fps_tokenize(c.half(), f, o, K=16)
 
 
+def test_many_small_events_use_the_warp_schedule():
+    # more FPS events than SMs: the warp schedule, in decreasing size order
+    b = workloads.random_batch(70, np.random.default_rng(70).integers(129, 449, 700), 128)
+    compare(b, run_gpu(b))
+
+
 def test_no_host_sync_and_launch_count():
     b = workloads.make_workload("c1")
     c, f, o, _ = to_dev(b)
@@ -234,7 +240,7 @@ def test_no_host_sync_and_launch_count():
     finally:
         torch.cuda.set_sync_debug_mode("default")
     n = fps.launch_count() - before
-    assert 3 <= n <= 8, n
+    assert 3 <= n <= 10, n
     torch.cuda.synchronize()
 
 
