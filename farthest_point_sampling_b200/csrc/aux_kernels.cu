@@ -356,6 +356,7 @@ __device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int
 }
 
 constexpr int kAssignPairs = 4;
+constexpr int kLloydPairs = 2;
 
 // Standalone nearest-centroid assignment over (event, chunk) items.
 __global__ void __launch_bounds__(256) k_assign(const float4* __restrict__ coords,
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
     int32_t* lab = labels + off;
     const float4* pts = coords + off;
     const float* fe = feats ? feats + off * F : nullptr;
-    nearest_pass<kAssignPairs>(pts, i0, i1, s_cent, K, [&](int i, int l, float4 p) {
+    nearest_pass<kLloydPairs>(pts, i0, i1, s_cent, K, [&](int i, int l, float4 p) {
       lab[i] = l;
       if (next) lloyd_accum(s_sum, p, charge_of(fe, F, charge_col, i), l);
     });
