@@ -8,12 +8,14 @@
 // farthest_point_sampling_with_knn, same list), and charge-weighted Lloyd
 // refinement (Neptune README, "How it works", step 1).
 //
-// Float sums (pool means, Lloyd weighted means) accumulate in float64 in any
-// order, first per CTA in shared memory and then, for events spread over
-// several CTAs, in global memory; they are rounded once to float32.  Every
-// term is an exact float64 (a float32, or the product of two float32), so the
-// result differs from a sequential float64 sum only by float64 rounding,
-// far below the float32 rounding of the final mean.
+// Float sums (pool means, Lloyd weighted means) accumulate in float64 and are
+// rounded once to float32.  A CTA sorts the points of its chunk by token
+// (a counting sort in shared memory), then one thread per (token, value) adds
+// that token's points; events spread over several chunks combine their chunk
+// sums with float64 atomics in global memory.  Every term is an exact float64
+// (a float32, or the product of two float32), so the result differs from a
+// sequential float64 sum only by float64 rounding, far below the float32
+// rounding of the final mean.
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,7 +35,8 @@ __device__ __forceinline__ int sched_shift(int q) {
 // events, and the accumulator slots; resets the status word and the cursors.
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
-                                               int force, int chunk_all, int latency_events, Workspace ws) {
+                                               int force, int chunk_all, int fused_pool, int latency_events,
+                                               Workspace ws) {
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps;
@@ -114,10 +117,15 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
       list[atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1)] = b;
       fslot = atomicAdd(&cnt[kListFps], 1);
     }
+    const int nch = (n + kChunk - 1) / kChunk;
     if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
-      const int nch = (n + kChunk - 1) / kChunk;
       const int base = atomicAdd(&cnt[kListChunks], nch);
       for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
+    }
+    // events the pool kernel handles (the others are pooled by their FPS kernel)
+    if ((cls == kClsFps && !(fused_pool && schedule_of(n) <= 1)) || (chunk_all && cls == kClsPass)) {
+      const int base = atomicAdd(&cnt[kListPoolChunks], nch);
+      for (int c = 0; c < nch; ++c) ws.pool_chunks[base + c] = make_int2(b, c);
       if (nch > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
     }
     ws.fps_slot[b] = fslot;
@@ -131,7 +139,7 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
   const DeviceInfo& di = device_info();
   count_launch();
   k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
-                           kLatencyEventsPerSm * di.sm_count, ws);
+                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, ws);
   return cudaGetLastError();
 }
 
@@ -191,9 +199,8 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
 }
 
 cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s) {
-  const DeviceInfo& di = device_info();
   int blocks = pb.B;
-  const int cap = di.sm_count * 8;
+  const int cap = 65535;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   count_launch();
@@ -203,101 +210,95 @@ cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStrea
 
 // ------------------------------------------------------------------ Voronoi pool
 
-// One CTA per (event, chunk) item: shared-memory float64 sums per token, then
-// either the final means (single-chunk event) or global float64 accumulation
-// with the last-arriving CTA of the event producing the means.
+// Shared-memory layout of one chunk's counting sort.
+struct SortSmem {
+  int* lab;    // [kChunk]
+  int* perm;   // [kChunk]
+  int* cnt;    // [256]
+  int* start;  // [256]
+  int* cur;    // [256]
+};
+__device__ __forceinline__ SortSmem sort_smem(int* base) {
+  return SortSmem{base, base + kChunk, base + 2 * kChunk, base + 2 * kChunk + 256, base + 2 * kChunk + 512};
+}
+constexpr size_t kSortSmemBytes = (size_t)(2 * kChunk + 3 * 256) * sizeof(int);
+
+__device__ __forceinline__ void cta_sync() { __syncthreads(); }
+
+// One CTA per (event, chunk) item: counting sort of the chunk's points by
+// token, float64 sums per (token, feature), then the means (single-chunk
+// event) or float64 accumulation in global memory with the last-arriving CTA
+// of the event producing the means.
 __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ feats, int F,
                                                       const int64_t* __restrict__ offsets, int K,
                                                       const int32_t* __restrict__ labels,
                                                       float* __restrict__ pooled,
                                                       int32_t* __restrict__ counts, Workspace ws) {
-  extern __shared__ double smem_d[];
-  double* s_sum = smem_d;                                 // [K*F]
-  int* s_cnt = reinterpret_cast<int*>(s_sum + K * F);     // [K]
+  extern __shared__ int smem_i[];
+  const SortSmem sm = sort_smem(smem_i);
   __shared__ int s_last;
-  const int nitems = ws.hdr->n_items[kListChunks];
+  const int nitems = ws.hdr->n_items[kListPoolChunks];
   const int KF = K * F;
+  const int T = blockDim.x, tid = threadIdx.x;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int2 it = ws.chunks[item];
+    const int2 it = ws.pool_chunks[item];
     const int b = it.x;
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
     const int i0 = it.y * kChunk;
-    const int i1 = min(n, i0 + kChunk);
+    const int npts = min(n, i0 + kChunk) - i0;
     const int nch = (n + kChunk - 1) / kChunk;
-    for (int e = threadIdx.x; e < KF; e += blockDim.x) s_sum[e] = 0.0;
-    for (int e = threadIdx.x; e < K; e += blockDim.x) s_cnt[e] = 0;
-    __syncthreads();
-    // element-major over the chunk's features, 8 loads in flight per thread
-    const int64_t e0 = (off + i0) * F, e1 = (off + i1) * F;
-    constexpr int R = 8;
-    for (int64_t base = e0 + threadIdx.x; base < e1; base += (int64_t)R * blockDim.x) {
-      float v[R];
-      int lab[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int64_t e = base + (int64_t)r * blockDim.x;
-        lab[r] = -1;
-        if (e < e1) {
-          v[r] = feats[e];
-          lab[r] = labels[e / F];
-        }
+#pragma unroll 8
+    for (int i = tid; i < npts; i += T) {
+      int l = labels[off + i0 + i];
+      if (l >= K) {
+        record_error(ws.hdr, kDevBadToken);
+        l = -1;
       }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int64_t e = base + (int64_t)r * blockDim.x;
-        const int j = lab[r];
-        if (e >= e1 || j < 0) continue;
-        if (j >= K) {
-          record_error(ws.hdr, kDevBadToken);
-          continue;
-        }
-        const int f = (int)(e - (e / F) * F);
-        if (f == 0) atomicAdd(&s_cnt[j], 1);
-        atomicAdd(&s_sum[j * F + f], (double)v[r]);
-      }
+      sm.lab[i] = l;
     }
-    __syncthreads();
+    label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, tid, T, cta_sync);
+    const float* fe = feats + (off + i0) * F;
+    auto val = [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); };
     if (nch == 1) {
-      for (int e = threadIdx.x; e < KF; e += blockDim.x) {
-        const int c = s_cnt[e / F];
-        pooled[(int64_t)b * KF + e] = c ? (float)(s_sum[e] / (double)c) : 0.f;
-      }
-      for (int j = threadIdx.x; j < K; j += blockDim.x) counts[(int64_t)b * K + j] = s_cnt[j];
+      float* prow = pooled + (int64_t)b * KF;
+      int32_t* crow = counts + (int64_t)b * K;
+      token_sums(sm.cnt, sm.start, sm.perm, K, F, tid, T, val, [&](int j, int f, double sum, int c) {
+        prow[j * F + f] = c ? (float)(sum / (double)c) : 0.f;
+        if (f == 0) crow[j] = c;
+      });
     } else {
       const int ps = ws.pool_slot[b];
       double* acc = ws.pool_acc + (int64_t)ps * KF;
       int* cnt = ws.pool_cnt + (int64_t)ps * K;
-      for (int e = threadIdx.x; e < KF; e += blockDim.x)
-        if (s_sum[e] != 0.0) atomicAdd(&acc[e], s_sum[e]);
-      for (int j = threadIdx.x; j < K; j += blockDim.x)
-        if (s_cnt[j]) atomicAdd(&cnt[j], s_cnt[j]);
+      token_sums(sm.cnt, sm.start, sm.perm, K, F, tid, T, val, [&](int j, int f, double sum, int c) {
+        if (c == 0) return;
+        atomicAdd(&acc[j * F + f], sum);
+        if (f == 0) atomicAdd(&cnt[j], c);
+      });
       __threadfence();
       __syncthreads();
-      if (threadIdx.x == 0) s_last = atomicAdd(&ws.pool_ticket[ps], 1) == nch - 1;
+      if (tid == 0) s_last = atomicAdd(&ws.pool_ticket[ps], 1) == nch - 1;
       __syncthreads();
       if (s_last) {
         __threadfence();
-        for (int e = threadIdx.x; e < KF; e += blockDim.x) {
+        for (int e = tid; e < KF; e += T) {
           const int c = __ldcg(&cnt[e / F]);
           pooled[(int64_t)b * KF + e] = c ? (float)(__ldcg(&acc[e]) / (double)c) : 0.f;
         }
-        for (int j = threadIdx.x; j < K; j += blockDim.x) counts[(int64_t)b * K + j] = __ldcg(&cnt[j]);
+        for (int j = tid; j < K; j += T) counts[(int64_t)b * K + j] = __ldcg(&cnt[j]);
       }
     }
     __syncthreads();
   }
 }
 
-static size_t pool_smem(int K, int F) { return (size_t)K * F * sizeof(double) + (size_t)K * sizeof(int); }
-
 cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,
                                 const Workspace& ws, cudaStream_t s) {
   const DeviceInfo& di = device_info();
-  const size_t sm = pool_smem(K, F);
   count_launch();
-  k_pool_voronoi<<<di.sm_count * 4, 256, sm, s>>>(feats, F, offsets, K, labels, pooled, counts, ws);
+  k_pool_voronoi<<<di.sm_count * 4, 256, kSortSmemBytes, s>>>(feats, F, offsets, K, labels, pooled, counts, ws);
   return cudaGetLastError();
 }
 
@@ -387,23 +388,29 @@ __global__ void __launch_bounds__(256) k_assign(const float4* __restrict__ coord
 
 // ------------------------------------------------------------------ Lloyd
 
-// Adds (q, q*x, q*y, q*z, q*t) of point p to token j's shared sums.
-__device__ __forceinline__ void lloyd_accum(double* s, float4 p, double q, int j) {
-  atomicAdd(&s[j * 5 + 0], q);
-  atomicAdd(&s[j * 5 + 1], q * (double)p.x);
-  atomicAdd(&s[j * 5 + 2], q * (double)p.y);
-  atomicAdd(&s[j * 5 + 3], q * (double)p.z);
-  atomicAdd(&s[j * 5 + 4], q * (double)p.w);
+__device__ __forceinline__ float charge_of(const float* fe, int F, int charge_col, int i) {
+  return charge_col < 0 ? 1.0f : __ldg(fe + (int64_t)i * F + charge_col);
 }
 
-__device__ __forceinline__ double charge_of(const float* fe, int F, int charge_col, int i) {
-  return charge_col < 0 ? 1.0 : (double)__ldg(fe + (int64_t)i * F + charge_col);
+// Lloyd sums of one chunk whose labels, points and charges are in shared
+// memory: W_j = sum q and S_j = sum q p per token, added to `out` (float64,
+// [K][5], global).
+__device__ __forceinline__ void lloyd_chunk_sums(const SortSmem& sm, const float4* s_p, const float* s_q, int npts,
+                                                 int K, double* out) {
+  label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, (int)threadIdx.x, (int)blockDim.x, cta_sync);
+  auto val = [&](int i, int v) {
+    const double q = (double)s_q[i];
+    if (v == 0) return q;
+    const float4 p = s_p[i];
+    return q * (double)(v == 1 ? p.x : (v == 2 ? p.y : (v == 3 ? p.z : p.w)));
+  };
+  token_sums(sm.cnt, sm.start, sm.perm, K, 5, (int)threadIdx.x, (int)blockDim.x, val,
+             [&](int j, int v, double sum, int c) {
+               if (c) atomicAdd(&out[j * 5 + v], sum);
+             });
 }
 
-__device__ __forceinline__ void flush_sums(const double* s, double* g, int n) {
-  for (int e = threadIdx.x; e < n; e += blockDim.x)
-    if (s[e] != 0.0) atomicAdd(&g[e], s[e]);
-}
+constexpr size_t kLloydSmemBytes = kSortSmemBytes + (size_t)kChunk * (sizeof(float4) + sizeof(float));
 
 // Cell sums of the current labels.
 __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ coords,
@@ -411,7 +418,10 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
                                                     int charge_col, const int64_t* __restrict__ offsets,
                                                     int K, const int32_t* __restrict__ labels,
                                                     Workspace ws, double* __restrict__ out) {
-  extern __shared__ double s_sum[];  // [K*5]
+  extern __shared__ int smem_i[];
+  const SortSmem sm = sort_smem(smem_i);
+  float4* s_p = reinterpret_cast<float4*>(smem_i + 2 * kChunk + 3 * 256);
+  float* s_q = reinterpret_cast<float*>(s_p + kChunk);
   const int nitems = ws.hdr->n_items[kListChunks];
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
     const int2 it = ws.chunks[item];
@@ -420,38 +430,21 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
     if (fs < 0) continue;  // uniform across the CTA
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    for (int e = threadIdx.x; e < K * 5; e += blockDim.x) s_sum[e] = 0.0;
-    __syncthreads();
-    const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
-    const float4* pts = coords + off;
-    const float* fe = feats ? feats + off * F : nullptr;
-    constexpr int R = 4;
-    for (int base = i0 + threadIdx.x; base < i1; base += R * blockDim.x) {
-      int lab[R];
-      float4 pp[R];
-      double q[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = base + r * blockDim.x;
-        lab[r] = -2;
-        if (i < i1) {
-          lab[r] = labels[off + i];
-          pp[r] = ldg4(pts + i);
-          q[r] = charge_of(fe, F, charge_col, i);
-        }
+    const int i0 = it.y * kChunk, npts = min(n, i0 + kChunk) - i0;
+    const float4* pts = coords + off + i0;
+    const float* fe = feats ? feats + (off + i0) * F : nullptr;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < npts; i += blockDim.x) {
+      int l = labels[off + i0 + i];
+      if ((unsigned)l >= (unsigned)K) {
+        record_error(ws.hdr, kDevBadToken);
+        l = -1;
       }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (lab[r] == -2) continue;
-        if (lab[r] < 0 || lab[r] >= K) {
-          record_error(ws.hdr, kDevBadToken);
-          continue;
-        }
-        lloyd_accum(s_sum, pp[r], q[r], lab[r]);
-      }
+      sm.lab[i] = l;
+      s_p[i] = ldg4(pts + i);
+      s_q[i] = charge_of(fe, F, charge_col, i);
     }
-    __syncthreads();
-    flush_sums(s_sum, out + (int64_t)fs * K * 5, K * 5);
+    lloyd_chunk_sums(sm, s_p, s_q, npts, K, out + (int64_t)fs * K * 5);
     __syncthreads();
   }
 }
@@ -459,15 +452,17 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
 // One Lloyd iteration: centroids from the sums `in`, re-assign the chunk and
 // (unless last) accumulate the next sums into `next`; clears `clear`.
 __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict__ coords,
-                                                    const float* __restrict__ feats, int F,
-                                                    int charge_col, const int64_t* __restrict__ offsets,
-                                                    int K, int32_t* __restrict__ labels,
-                                                    float4* __restrict__ centroids, Workspace ws,
-                                                    const double* __restrict__ in, double* __restrict__ next,
-                                                    double* __restrict__ clear, int64_t clear_n) {
-  extern __shared__ double smem_l[];
-  double* s_sum = smem_l;                                  // [K*5]
-  Cent2* s_cent = reinterpret_cast<Cent2*>(s_sum + K * 5);  // [K]
+                                                       const float* __restrict__ feats, int F,
+                                                       int charge_col, const int64_t* __restrict__ offsets,
+                                                       int K, int32_t* __restrict__ labels,
+                                                       float4* __restrict__ centroids, Workspace ws,
+                                                       const double* __restrict__ in, double* __restrict__ next,
+                                                       double* __restrict__ clear, int64_t clear_n) {
+  extern __shared__ int smem_i[];
+  const SortSmem sm = sort_smem(smem_i);
+  float4* s_p = reinterpret_cast<float4*>(smem_i + 2 * kChunk + 3 * 256);
+  float* s_q = reinterpret_cast<float*>(s_p + kChunk);
+  Cent2* s_cent = reinterpret_cast<Cent2*>(s_q + kChunk);  // [K]
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < clear_n;
        e += (int64_t)gridDim.x * blockDim.x)
     clear[e] = 0.0;
@@ -492,8 +487,6 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
       s_cent[j] = cent2(c);
       if (it.y == 0) centroids[(int64_t)b * K + j] = c;
     }
-    if (next)
-      for (int e = threadIdx.x; e < K * 5; e += blockDim.x) s_sum[e] = 0.0;
     __syncthreads();
     const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
     int32_t* lab = labels + off;
@@ -501,10 +494,16 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
     const float* fe = feats ? feats + off * F : nullptr;
     nearest_pass<kLloydPairs>(pts, i0, i1, s_cent, K, [&](int i, int l, float4 p) {
       lab[i] = l;
-      if (next) lloyd_accum(s_sum, p, charge_of(fe, F, charge_col, i), l);
+      if (next) {
+        sm.lab[i - i0] = l;
+        s_p[i - i0] = p;
+        s_q[i - i0] = charge_of(fe, F, charge_col, i);
+      }
     });
-    __syncthreads();
-    if (next) flush_sums(s_sum, next + (int64_t)fs * K * 5, K * 5);
+    if (next) {
+      __syncthreads();
+      lloyd_chunk_sums(sm, s_p, s_q, i1 - i0, K, next + (int64_t)fs * K * 5);
+    }
     __syncthreads();
   }
 }
@@ -513,8 +512,8 @@ cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels
   const DeviceInfo& di = device_info();
   const int K = pb.K;
   const int grid = di.sm_count * 4;
-  const size_t sm_sums = (size_t)K * 5 * sizeof(double);
-  const size_t sm_step = sm_sums + (size_t)K * sizeof(Cent2);
+  const size_t sm_sums = kLloydSmemBytes;
+  const size_t sm_step = kLloydSmemBytes + (size_t)K * sizeof(Cent2);
   cudaError_t e;
   const float* feats = pb.charge_col >= 0 ? pb.feats : nullptr;
   count_launch();
@@ -541,12 +540,8 @@ cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels
 // largest K and F the ABI accepts.
 cudaError_t prepare_aux_kernels() {
   cudaError_t e;
-  const int pool_max = (int)pool_smem(256, 64);
-  const int sums_max = 256 * 5 * (int)sizeof(double);
-  const int step_max = sums_max + 256 * (int)sizeof(Cent2);
-  if ((e = cudaFuncSetAttribute(k_pool_voronoi, cudaFuncAttributeMaxDynamicSharedMemorySize, pool_max)))
-    return e;
-  if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, sums_max)))
+  const int step_max = (int)(kLloydSmemBytes + 256 * sizeof(Cent2));
+  if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLloydSmemBytes)))
     return e;
   if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize, step_max)))
     return e;

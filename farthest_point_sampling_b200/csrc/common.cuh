@@ -146,4 +146,80 @@ __device__ __forceinline__ void warp_argmax(int key, unsigned idx, int& mkey, un
 
 __device__ __forceinline__ float4 ldg4(const float4* p) { return __ldg(p); }
 
+// ---------------------------------------------------------------- per-token sums
+
+// Counting sort of npts labelled points by a group of threads (a warp or a
+// CTA; `rank` / `size` are this thread's index in it and its size, `sync` its
+// barrier): cnt[j] = number of points labelled j, start[j] = exclusive prefix
+// sum, perm[start[j] .. start[j] + cnt[j]) = the local indices of those
+// points.  Labels outside [0, K) are left out.  K <= 256.  All arrays are in
+// shared memory; cur[K] is scratch.
+template <typename Sync>
+__device__ __forceinline__ void label_sort(const int* lab, int npts, int K, int* cnt, int* start, int* cur,
+                                           int* perm, int rank, int size, Sync sync) {
+  for (int j = rank; j < K; j += size) cnt[j] = 0;
+  sync();
+  for (int i = rank; i < npts; i += size) {
+    const int l = lab[i];
+    if ((unsigned)l < (unsigned)K) atomicAdd(&cnt[l], 1);
+  }
+  sync();
+  if (rank < 32) {  // exclusive scan by the group's first warp, 8 entries per lane
+    int local[8];
+    int sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = rank * 8 + q;
+      local[q] = j < K ? cnt[j] : 0;
+      sum += local[q];
+    }
+    int x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, o);
+      if (rank >= o) x += y;
+    }
+    int run = x - sum;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = rank * 8 + q;
+      if (j < K) {
+        start[j] = run;
+        cur[j] = run;
+      }
+      run += local[q];
+    }
+  }
+  sync();
+  for (int i = rank; i < npts; i += size) {
+    const int l = lab[i];
+    if ((unsigned)l < (unsigned)K) perm[atomicAdd(&cur[l], 1)] = i;
+  }
+  sync();
+}
+
+// For every (token j, value v) pair (v < V) handled by this thread of the
+// group: the float64 sum of val(i, v) over the points i sorted to token j,
+// then out(j, v, sum, count).  Loads of four points are issued together.
+template <typename Val, typename Out>
+__device__ __forceinline__ void token_sums(const int* cnt, const int* start, const int* perm, int K, int V,
+                                           int rank, int size, Val val, Out out) {
+  for (int e = rank; e < K * V; e += size) {
+    const int j = e / V, v = e - j * V;
+    const int c = cnt[j];
+    const int* pj = perm + start[j];
+    double s = 0.0;
+    int t = 0;
+    for (; t + 4 <= c; t += 4) {
+      const double a0 = val(pj[t], v), a1 = val(pj[t + 1], v), a2 = val(pj[t + 2], v), a3 = val(pj[t + 3], v);
+      s += a0;
+      s += a1;
+      s += a2;
+      s += a3;
+    }
+    for (; t < c; ++t) s += val(pj[t], v);
+    out(j, v, s, c);
+  }
+}
+
 }  // namespace fpstok

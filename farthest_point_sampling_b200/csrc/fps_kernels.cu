@@ -56,10 +56,41 @@ __device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xfffffff
                 FPS_CASE(6, CALL) FPS_CASE(7, CALL) default : break; }
 
 // One FPS event on one warp, NP point pairs per lane.
+// Token means of an event whose labels sit in registers, pooled in place
+// (no Lloyd follows): a counting sort by token in the group's shared scratch
+// (labels[n], perm[n], cnt/start/cur[256] ints, n <= nmax), then float64 sums
+// per (token, feature) in point-index-sorted-by-token order.
+struct PoolOut {
+  const float* feats;  // null: no pooling in the FPS kernel
+  int F;
+  float* pooled;
+  int32_t* counts;
+};
+
+template <typename Sync>
+__device__ __forceinline__ void pool_event(int* scratch, int nmax, int n, int K, int64_t b, int64_t off,
+                                           const PoolOut& po, int rank, int size, Sync sync) {
+  int* s_lab = scratch;
+  int* perm = scratch + nmax;
+  int* cnt = perm + nmax;
+  label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, rank, size, sync);
+  const int F = po.F;
+  const float* fe = po.feats + off * F;
+  float* prow = po.pooled + b * K * F;
+  int32_t* crow = po.counts + b * K;
+  token_sums(cnt, cnt + 256, perm, K, F, rank, size,
+             [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); },
+             [&](int j, int f, double sum, int c) {
+               prow[j * F + f] = c ? (float)(sum / (double)c) : 0.f;
+               if (f == 0) crow[j] = c;
+             });
+}
+
 template <int NP>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                            int lane, DupPoint* s_dup, int32_t* __restrict__ cidx,
-                                           float4* __restrict__ cpos, int32_t* __restrict__ tok) {
+                                           float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
+                                           const PoolOut& po, int nmax) {
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -123,6 +154,17 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       if (i < n) tok[i] = lab[j];
     }
   }
+  if (po.feats) {
+    __syncwarp();  // the event copy is done with; its space becomes the sort scratch
+    int* scratch = reinterpret_cast<int*>(s_dup);
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < n) scratch[i] = lab[j];
+    }
+    __syncwarp();
+    pool_event(scratch, nmax, n, K, b, off, po, lane, 32, [] { __syncwarp(); });
+  }
   __syncwarp();  // the next event overwrites this warp's copy
 }
 
@@ -133,9 +175,11 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
                                                      const int* __restrict__ list, WsHeader* hdr, int K,
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
-                                                     float4* __restrict__ centroids) {
+                                                     float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
+  static_assert(2 * 64 * NPMAX + 3 * 256 <= 64 * NPMAX * (int)(sizeof(DupPoint) / sizeof(int)),
+                "pooling scratch fits in the warp's event copy");
   extern __shared__ DupPoint s_dup_all[];
   const int lane = threadIdx.x & 31;
   DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
@@ -152,7 +196,7 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define WARP_CALL(N)                                                                                   \
   warp_event<N>(coords + off, n, c0, K, off, lane, s_dup, centroid_idx + (int64_t)b * K,               \
-                centroids + (int64_t)b * K, tok)
+                centroids + (int64_t)b * K, tok, b, po, 64 * NPMAX)
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
   }
@@ -172,7 +216,8 @@ __device__ __forceinline__ int claim_cta(WsHeader* hdr, int list_id, int* slot) 
 template <int NP, int NT>
 __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                           DupPoint* s_dup, int2* xk, int& round, int32_t* __restrict__ cidx,
-                                          float4* __restrict__ cpos, int32_t* __restrict__ tok) {
+                                          float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
+                                          const PoolOut& po, int nmax) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
@@ -252,6 +297,17 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       if (i < n) tok[i] = lab[j];
     }
   }
+  if (po.feats) {
+    __syncthreads();  // the event copy is done with; its space becomes the sort scratch
+    int* scratch = reinterpret_cast<int*>(s_dup);
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = j * NT + tid;
+      if (i < n) scratch[i] = lab[j];
+    }
+    __syncthreads();
+    pool_event(scratch, nmax, n, K, b, off, po, tid, NT, [] { __syncthreads(); });
+  }
 }
 
 template <int PR>
@@ -261,9 +317,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
                                                             const int* __restrict__ list, WsHeader* hdr, int K,
                                                             int32_t* __restrict__ centroid_idx,
                                                             int32_t* __restrict__ token_id,
-                                                            float4* __restrict__ centroids) {
+                                                            float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = PR;
   constexpr int NT = kCtaThreads, NW = NT / 32;
+  static_assert(2 * 2 * NT * PR + 3 * 256 <= 2 * NT * PR * (int)(sizeof(DupPoint) / sizeof(int)),
+                "pooling scratch fits in the event copy");
   static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
   extern __shared__ DupPoint s_dup[];  // [2 * NT * PR] event copy for centroid look-up
   __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
@@ -280,7 +338,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define CTA_CALL(N)                                                                                     \
   cta_event<N, NT>(coords + off, n, c0, K, off, s_dup, xk, round, centroid_idx + (int64_t)b * K,        \
-                   centroids + (int64_t)b * K, tok)
+                   centroids + (int64_t)b * K, tok, b, po, 2 * NT * PR)
     FPS_DISPATCH_7((n + 2 * NT - 1) / (2 * NT), CTA_CALL)
 #undef CTA_CALL
   }
@@ -650,6 +708,8 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     run[q] = allowed && (hint == 0 || hint > lo);
   }
 
+  const PoolOut po = pb.fused_pool ? PoolOut{pb.feats, pb.F, pb.pooled, pb.counts} : PoolOut{nullptr, 0, nullptr, nullptr};
+
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
   bool forked = false;
   for (int q = 1; q < kNumSchedules; ++q) forked |= run[q];
@@ -664,7 +724,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
         count_launch();
         k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
             pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-            pb.centroids);
+            pb.centroids, po);
         e = cudaGetLastError();
         break;
       case 2:
@@ -687,7 +747,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     count_launch();
     k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, s>>>(pb.coords, pb.offsets, pb.start_local,
                                                                  ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                 pb.token_id, pb.centroids);
+                                                                 pb.token_id, pb.centroids, po);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1, 1, s);
   }

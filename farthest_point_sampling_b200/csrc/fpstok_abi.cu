@@ -51,6 +51,7 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   w.list_cluster8 = c.take<int>(nb);
   w.list_cluster16 = c.take<int>(nb);
   w.chunks = c.take<int2>(chunks);
+  w.pool_chunks = c.take<int2>(chunks);
   w.cls = c.take<int>(nb);
   w.fps_slot = c.take<int>(nb);
   w.pool_slot = c.take<int>(nb);
@@ -175,7 +176,8 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
                 opts->K, opts->assign_mode, opts->k, opts->lloyd_iters, opts->charge_col,
                 opts->force_schedule, opts->max_event_hint, centroid_idx, token_id,
                 opts->assign_mode == FPS_ASSIGN_KNN ? knn_idx : nullptr,
-                reinterpret_cast<float4*>(centroids), pooled, counts};
+                reinterpret_cast<float4*>(centroids), pooled, counts,
+                opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0};
   return run_tokenize(pb, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 

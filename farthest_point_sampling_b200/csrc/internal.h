@@ -16,10 +16,11 @@ enum ListId : int {
   kListCtaSmem = 2,
   kListCluster8 = 3,
   kListCluster16 = 4,
-  kListChunks = 5,     // (event, chunk) items of FPS events
-  kListPoolSlots = 6,  // events that need global pooling accumulators
-  kListFps = 7,        // number of FPS events (Lloyd slots)
-  kNumLists = 8,
+  kListChunks = 5,      // (event, chunk) items of FPS events (Lloyd, assignment)
+  kListPoolSlots = 6,   // events that need global pooling accumulators
+  kListFps = 7,         // number of FPS events (Lloyd slots)
+  kListPoolChunks = 8,  // (event, chunk) items pooled by k_pool_voronoi
+  kNumLists = 9,
 };
 constexpr int kNumSchedules = 5;  // warp, CTA, CTA-smem, 8-CTA cluster, 16-CTA cluster
 
@@ -47,7 +48,8 @@ struct Workspace {
   int* list_cta_smem;
   int* list_cluster8;
   int* list_cluster16;
-  int2* chunks;     // (event, chunk)
+  int2* chunks;     // (event, chunk) items of FPS events
+  int2* pool_chunks; // (event, chunk) items of events pooled by the pool kernel
   int* cls;         // EventClass per event
   int* fps_slot;    // compact index of FPS events, -1 otherwise
   int* pool_slot;   // compact index of multi-chunk FPS events, -1 otherwise
@@ -76,6 +78,7 @@ struct Problem {
   float4* centroids;
   float* pooled;
   int32_t* counts;
+  int fused_pool;  // FPS kernels of the warp / CTA schedules also pool their events
 };
 
 // Kernel launchers (return the cudaError_t of the launch).
