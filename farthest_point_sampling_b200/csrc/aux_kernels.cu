@@ -26,6 +26,7 @@ namespace fpstok {
 // Size buckets of the counting sort that orders each schedule's list by
 // decreasing event size (bucket = n >> shift; shift keeps cap >> shift < 256).
 constexpr int kBins = 256;
+constexpr int kBinCache = 8192;  // events whose size the binning kernel keeps in shared memory
 __device__ __forceinline__ int sched_shift(int q) {
   return q == 0 ? 1 : (q == 1 ? 4 : (q == 2 ? 6 : (q == 3 ? 9 : 10)));
 }
@@ -40,6 +41,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps;
+  __shared__ int s_n[kBinCache];  // event sizes (cls in the sign: -1 - cls for non-FPS events)
   for (int i = threadIdx.x; i < kNumSchedules * kBins; i += blockDim.x) (&hist[0][0])[i] = 0;
   if (threadIdx.x < kNumLists) cnt[threadIdx.x] = 0;
   if (threadIdx.x < 8) ws.hdr->next_item[threadIdx.x] = 0;
@@ -49,31 +51,50 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     n_fps = 0;
   }
   __syncthreads();
-  // pass 1: classify and count FPS events
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const int64_t o0 = offsets[b], o1 = offsets[b + 1];
-    int cls;
-    if (o0 < 0 || o1 < o0 || o1 > P) {
-      record_error(ws.hdr, kDevBadOffsets);
-      cls = kClsSkip;
-    } else {
-      if ((b == 0 && o0 != 0) || (b == B - 1 && o1 != P)) record_error(ws.hdr, kDevBadOffsets);
-      const int64_t n = o1 - o0;
-      cls = n == 0 ? kClsEmpty : (n <= K ? kClsPass : kClsFps);
-      if (cls == kClsFps) {
-        const int st = start_local ? start_local[b] : 0;
-        if (st < 0 || st >= n) {
-          record_error(ws.hdr, kDevBadStart);
-          cls = kClsSkip;
-        } else if (n > kClusterCap) {
-          record_error(ws.hdr, kDevTooLarge);
-          cls = kClsSkip;
-        } else {
-          atomicAdd(&n_fps, 1);
-        }
+  // pass 1: classify and count FPS events (four events per thread in flight)
+  constexpr int U = 4;
+  for (int b0 = threadIdx.x; b0 < B; b0 += U * blockDim.x) {
+    int64_t o0[U], o1[U];
+    int st[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int b = b0 + u * blockDim.x;
+      o0[u] = o1[u] = 0;
+      st[u] = 0;
+      if (b < B) {
+        o0[u] = offsets[b];
+        o1[u] = offsets[b + 1];
+        if (start_local) st[u] = start_local[b];
       }
     }
-    ws.cls[b] = cls;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int b = b0 + u * blockDim.x;
+      if (b >= B) continue;
+      int cls;
+      int64_t n = 0;
+      if (o0[u] < 0 || o1[u] < o0[u] || o1[u] > P) {
+        record_error(ws.hdr, kDevBadOffsets);
+        cls = kClsSkip;
+      } else {
+        if ((b == 0 && o0[u] != 0) || (b == B - 1 && o1[u] != P)) record_error(ws.hdr, kDevBadOffsets);
+        n = o1[u] - o0[u];
+        cls = n == 0 ? kClsEmpty : (n <= K ? kClsPass : kClsFps);
+        if (cls == kClsFps) {
+          if (st[u] < 0 || st[u] >= n) {
+            record_error(ws.hdr, kDevBadStart);
+            cls = kClsSkip;
+          } else if (n > kClusterCap) {
+            record_error(ws.hdr, kDevTooLarge);
+            cls = kClsSkip;
+          } else {
+            atomicAdd(&n_fps, 1);
+          }
+        }
+      }
+      ws.cls[b] = cls;
+      if (b < kBinCache) s_n[b] = cls == kClsFps || cls == kClsPass ? (int)n : -1;
+    }
   }
   __syncthreads();
   const bool few = n_fps <= latency_events;
@@ -83,10 +104,11 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     if (force > q) q = force > 4 ? 4 : force;
     return q;
   };
+  auto size_of = [&](int b) { return b < kBinCache ? s_n[b] : (int)(offsets[b + 1] - offsets[b]); };
   // pass 2: size histogram per schedule
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     if (ws.cls[b] != kClsFps) continue;
-    const int n = (int)(offsets[b + 1] - offsets[b]);
+    const int n = size_of(b);
     const int q = schedule_of(n);
     atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1);
   }
@@ -108,7 +130,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     const int cls = ws.cls[b];
     int fslot = -1, pslot = -1;
     int n = 0;
-    if (cls == kClsFps || cls == kClsPass) n = (int)(offsets[b + 1] - offsets[b]);
+    if (cls == kClsFps || cls == kClsPass) n = size_of(b);
     if (cls == kClsFps) {
       const int q = schedule_of(n);
       int* list = q == 0 ? ws.list_warp
@@ -123,7 +145,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
       for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
     }
     // events the pool kernel handles (the others are pooled by their FPS kernel)
-    if ((cls == kClsFps && !(fused_pool && schedule_of(n) <= 1)) || (chunk_all && cls == kClsPass)) {
+    if ((cls == kClsFps && !((fused_pool >> schedule_of(n)) & 1)) || (chunk_all && cls == kClsPass)) {
       const int base = atomicAdd(&cnt[kListPoolChunks], nch);
       for (int c = 0; c < nch; ++c) ws.pool_chunks[base + c] = make_int2(b, c);
       if (nch > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);

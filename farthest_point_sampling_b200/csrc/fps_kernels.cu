@@ -46,6 +46,22 @@ namespace fpstok {
 
 __device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xffffffffu : ((1u << n) - 1u); }
 
+// Shared memory of one warp of the warp schedule and of a CTA of the
+// register CTA schedule: the event copy during FPS, then (pooling in place)
+// the sort scratch and the staged feature rows of at most kFuse*MaxF floats.
+constexpr size_t pool_region_bytes(int nmax, int max_f) {
+  return (size_t)(2 * nmax + 3 * 256) * sizeof(int) + (size_t)nmax * max_f * sizeof(float);
+}
+constexpr size_t cmax(size_t a, size_t b) { return a > b ? a : b; }
+constexpr size_t kWarpRegionBytes =
+    (cmax((size_t)64 * kWarpPairs * sizeof(DupPoint), pool_region_bytes(64 * kWarpPairs, kFuseWarpMaxF)) + 15) &
+    ~(size_t)15;
+constexpr size_t kCtaRegionBytes =
+    (cmax((size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint), pool_region_bytes(2 * kCtaThreads * kCtaPairs,
+                                                                                    kFuseCtaMaxF)) +
+     15) &
+    ~(size_t)15;
+
 // Dispatches CALL(N) for the compile-time N that equals the runtime np
 // (N <= kMaxPairs).
 #define FPS_CASE(N, CALL) \
@@ -57,9 +73,10 @@ __device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xfffffff
 
 // One FPS event on one warp, NP point pairs per lane.
 // Token means of an event whose labels sit in registers, pooled in place
-// (no Lloyd follows): a counting sort by token in the group's shared scratch
-// (labels[n], perm[n], cnt/start/cur[256] ints, n <= nmax), then float64 sums
-// per (token, feature) in point-index-sorted-by-token order.
+// (no Lloyd follows): the event's feature rows are staged in the group's
+// shared scratch (labels[nmax], perm[nmax], cnt/start/cur[256] ints, then
+// the rows), the points are counting-sorted by token, and one thread per
+// (token, feature) adds its token's rows in float64.
 struct PoolOut {
   const float* feats;  // null: no pooling in the FPS kernel
   int F;
@@ -73,17 +90,20 @@ __device__ __forceinline__ void pool_event(int* scratch, int nmax, int n, int K,
   int* s_lab = scratch;
   int* perm = scratch + nmax;
   int* cnt = perm + nmax;
-  label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, rank, size, sync);
+  float* s_feat = reinterpret_cast<float*>(cnt + 768);  // [n * F] staged feature rows
   const int F = po.F;
   const float* fe = po.feats + off * F;
+#pragma unroll 4
+  for (int e = rank; e < n * F; e += size) s_feat[e] = __ldg(fe + e);
+  label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, rank, size, sync);
   float* prow = po.pooled + b * K * F;
   int32_t* crow = po.counts + b * K;
-  token_sums(cnt, cnt + 256, perm, K, F, rank, size,
-             [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); },
+  token_sums(cnt, cnt + 256, perm, K, F, rank, size, [&](int i, int f) { return (double)s_feat[i * F + f]; },
              [&](int j, int f, double sum, int c) {
                prow[j * F + f] = c ? (float)(sum / (double)c) : 0.f;
                if (f == 0) crow[j] = c;
              });
+  sync();
 }
 
 template <int NP>
@@ -178,11 +198,10 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
                                                      float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
-  static_assert(2 * 64 * NPMAX + 3 * 256 <= 64 * NPMAX * (int)(sizeof(DupPoint) / sizeof(int)),
-                "pooling scratch fits in the warp's event copy");
+  static_assert(64 * NPMAX * sizeof(DupPoint) <= kWarpRegionBytes, "event copy fits in the warp's region");
   extern __shared__ DupPoint s_dup_all[];
   const int lane = threadIdx.x & 31;
-  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
+  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (kWarpRegionBytes / sizeof(DupPoint));  // this warp's region
   const int count = hdr->n_items[kListWarp];
   for (;;) {
     int w = 0;
@@ -320,8 +339,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
                                                             float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = PR;
   constexpr int NT = kCtaThreads, NW = NT / 32;
-  static_assert(2 * 2 * NT * PR + 3 * 256 <= 2 * NT * PR * (int)(sizeof(DupPoint) / sizeof(int)),
-                "pooling scratch fits in the event copy");
+  static_assert(2 * NT * PR * sizeof(DupPoint) <= kCtaRegionBytes, "event copy fits in the region");
   static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
   extern __shared__ DupPoint s_dup[];  // [2 * NT * PR] event copy for centroid look-up
   __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
@@ -567,8 +585,8 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
 // ------------------------------------------------------------------ launch
 
 constexpr int kWarpBlock = 128;
-constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(DupPoint);
-constexpr size_t kCtaSmem = (size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint);
+constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * kWarpRegionBytes;
+constexpr size_t kCtaSmem = kCtaRegionBytes;
 
 template <int CL>
 constexpr size_t block_smem_bytes() {
@@ -708,7 +726,10 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     run[q] = allowed && (hint == 0 || hint > lo);
   }
 
-  const PoolOut po = pb.fused_pool ? PoolOut{pb.feats, pb.F, pb.pooled, pb.counts} : PoolOut{nullptr, 0, nullptr, nullptr};
+  const PoolOut none = {nullptr, 0, nullptr, nullptr};
+  const PoolOut pool = {pb.feats, pb.F, pb.pooled, pb.counts};
+  const PoolOut po_warp = (pb.fused_pool & 1) ? pool : none;
+  const PoolOut po_cta = (pb.fused_pool & 2) ? pool : none;
 
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
   bool forked = false;
@@ -724,7 +745,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
         count_launch();
         k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
             pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-            pb.centroids, po);
+            pb.centroids, po_cta);
         e = cudaGetLastError();
         break;
       case 2:
@@ -747,7 +768,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     count_launch();
     k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, s>>>(pb.coords, pb.offsets, pb.start_local,
                                                                  ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                 pb.token_id, pb.centroids, po);
+                                                                 pb.token_id, pb.centroids, po_warp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1, 1, s);
   }

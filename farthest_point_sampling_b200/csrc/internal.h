@@ -37,6 +37,8 @@ constexpr int kCluster8Cap = 8 * kCtaSmemCap;                 // 98304
 constexpr int kMaxCluster = 16;
 constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
 constexpr int kChunk = 2048;                           // points per pooling / Lloyd work item
+constexpr int kFuseWarpMaxF = 6;  // the warp schedule pools its events in place when F <= this
+constexpr int kFuseCtaMaxF = 7;   // the register CTA schedule likewise
 // With at most this many FPS events per SM, events of the warp class run on
 // the CTA schedule instead (lower latency per step when the GPU is not full).
 constexpr int kLatencyEventsPerSm = 1;
@@ -78,7 +80,7 @@ struct Problem {
   float4* centroids;
   float* pooled;
   int32_t* counts;
-  int fused_pool;  // FPS kernels of the warp / CTA schedules also pool their events
+  int fused_pool;  // bit 0 / bit 1: the warp / register-CTA FPS kernels also pool their events
 };
 
 // Kernel launchers (return the cudaError_t of the launch).
