@@ -36,8 +36,7 @@ __device__ __forceinline__ int sched_shift(int q) {
 // events, and the accumulator slots; resets the status word and the cursors.
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
-                                               int force, int chunk_all, int fused_pool, int latency_events,
-                                               Workspace ws) {
+                                               int force, int chunk_all, int latency_events, Workspace ws) {
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps;
@@ -144,8 +143,8 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
       const int base = atomicAdd(&cnt[kListChunks], nch);
       for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
     }
-    // events the pool kernel handles (the others are pooled by their FPS kernel)
-    if ((cls == kClsFps && !((fused_pool >> schedule_of(n)) & 1)) || (chunk_all && cls == kClsPass)) {
+    // events the pool kernel handles (passthrough events are written directly)
+    if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
       const int base = atomicAdd(&cnt[kListPoolChunks], nch);
       for (int c = 0; c < nch; ++c) ws.pool_chunks[base + c] = make_int2(b, c);
       if (nch > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
@@ -161,7 +160,7 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
   const DeviceInfo& di = device_info();
   count_launch();
   k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
-                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, ws);
+                           kLatencyEventsPerSm * di.sm_count, ws);
   return cudaGetLastError();
 }
 
@@ -234,23 +233,39 @@ cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStrea
 
 // Shared-memory layout of one chunk's counting sort.
 struct SortSmem {
-  int* lab;    // [kChunk]
-  int* perm;   // [kChunk]
+  int* lab;    // [kChunk] token of every point
+  int* perm;   // [kChunk] point of every sorted position
+  int* slab;   // [kChunk] token of every sorted position
   int* cnt;    // [256]
   int* start;  // [256]
   int* cur;    // [256]
 };
 __device__ __forceinline__ SortSmem sort_smem(int* base) {
-  return SortSmem{base, base + kChunk, base + 2 * kChunk, base + 2 * kChunk + 256, base + 2 * kChunk + 512};
+  return SortSmem{base, base + kChunk, base + 2 * kChunk, base + 3 * kChunk, base + 3 * kChunk + 256,
+                  base + 3 * kChunk + 512};
 }
-constexpr size_t kSortSmemBytes = (size_t)(2 * kChunk + 3 * 256) * sizeof(int);
+constexpr size_t kSortSmemBytes = (size_t)(3 * kChunk + 3 * 256) * sizeof(int);
 
 __device__ __forceinline__ void cta_sync() { __syncthreads(); }
 
+// Sorts the chunk by token and adds up V values per token into acc[K * V]
+// (shared float64, zeroed here): balanced over the CTA.
+template <typename Val>
+__device__ __forceinline__ void chunk_token_sums(const SortSmem& sm, int npts, int K, int V, double* acc, Val val) {
+  const int tid = threadIdx.x, T = blockDim.x;
+  for (int e = tid; e < K * V; e += T) acc[e] = 0.0;
+  label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, sm.slab, tid, T, cta_sync);
+  int nsorted = 0;
+  if (K > 0) nsorted = sm.start[K - 1] + sm.cnt[K - 1];
+  for (int v0 = 0; v0 < V; v0 += 8)
+    segment_sums(sm.perm, sm.slab, nsorted, min(8, V - v0), v0, V, acc, tid, T, val);
+  __syncthreads();
+}
+
 // One CTA per (event, chunk) item: counting sort of the chunk's points by
-// token, float64 sums per (token, feature), then the means (single-chunk
-// event) or float64 accumulation in global memory with the last-arriving CTA
-// of the event producing the means.
+// token, balanced float64 sums per (token, feature), then the means
+// (single-chunk event) or float64 accumulation in global memory with the
+// last-arriving CTA of the event producing the means.
 __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ feats, int F,
                                                       const int64_t* __restrict__ offsets, int K,
                                                       const int32_t* __restrict__ labels,
@@ -258,6 +273,7 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
                                                       int32_t* __restrict__ counts, Workspace ws) {
   extern __shared__ int smem_i[];
   const SortSmem sm = sort_smem(smem_i);
+  double* acc = reinterpret_cast<double*>(smem_i + 3 * kChunk + 3 * 256);  // [K * F]
   __shared__ int s_last;
   const int nitems = ws.hdr->n_items[kListPoolChunks];
   const int KF = K * F;
@@ -279,25 +295,22 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
       }
       sm.lab[i] = l;
     }
-    label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, tid, T, cta_sync);
     const float* fe = feats + (off + i0) * F;
-    auto val = [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); };
+    chunk_token_sums(sm, npts, K, F, acc, [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); });
     if (nch == 1) {
-      float* prow = pooled + (int64_t)b * KF;
-      int32_t* crow = counts + (int64_t)b * K;
-      token_sums(sm.cnt, sm.start, sm.perm, K, F, tid, T, val, [&](int j, int f, double sum, int c) {
-        prow[j * F + f] = c ? (float)(sum / (double)c) : 0.f;
-        if (f == 0) crow[j] = c;
-      });
+      for (int e = tid; e < KF; e += T) {
+        const int c = sm.cnt[e / F];
+        pooled[(int64_t)b * KF + e] = c ? (float)(acc[e] / (double)c) : 0.f;
+      }
+      for (int j = tid; j < K; j += T) counts[(int64_t)b * K + j] = sm.cnt[j];
     } else {
       const int ps = ws.pool_slot[b];
-      double* acc = ws.pool_acc + (int64_t)ps * KF;
-      int* cnt = ws.pool_cnt + (int64_t)ps * K;
-      token_sums(sm.cnt, sm.start, sm.perm, K, F, tid, T, val, [&](int j, int f, double sum, int c) {
-        if (c == 0) return;
-        atomicAdd(&acc[j * F + f], sum);
-        if (f == 0) atomicAdd(&cnt[j], c);
-      });
+      double* gacc = ws.pool_acc + (int64_t)ps * KF;
+      int* gcnt = ws.pool_cnt + (int64_t)ps * K;
+      for (int e = tid; e < KF; e += T)
+        if (sm.cnt[e / F]) atomicAdd(&gacc[e], acc[e]);
+      for (int j = tid; j < K; j += T)
+        if (sm.cnt[j]) atomicAdd(&gcnt[j], sm.cnt[j]);
       __threadfence();
       __syncthreads();
       if (tid == 0) s_last = atomicAdd(&ws.pool_ticket[ps], 1) == nch - 1;
@@ -305,22 +318,25 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
       if (s_last) {
         __threadfence();
         for (int e = tid; e < KF; e += T) {
-          const int c = __ldcg(&cnt[e / F]);
-          pooled[(int64_t)b * KF + e] = c ? (float)(__ldcg(&acc[e]) / (double)c) : 0.f;
+          const int c = __ldcg(&gcnt[e / F]);
+          pooled[(int64_t)b * KF + e] = c ? (float)(__ldcg(&gacc[e]) / (double)c) : 0.f;
         }
-        for (int j = tid; j < K; j += T) counts[(int64_t)b * K + j] = __ldcg(&cnt[j]);
+        for (int j = tid; j < K; j += T) counts[(int64_t)b * K + j] = __ldcg(&gcnt[j]);
       }
     }
     __syncthreads();
   }
 }
 
+static size_t pool_smem_bytes(int K, int F) { return kSortSmemBytes + (size_t)K * F * sizeof(double); }
+
 cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,
                                 const Workspace& ws, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   count_launch();
-  k_pool_voronoi<<<di.sm_count * 4, 256, kSortSmemBytes, s>>>(feats, F, offsets, K, labels, pooled, counts, ws);
+  k_pool_voronoi<<<di.sm_count * 6, 256, pool_smem_bytes(K, F), s>>>(feats, F, offsets, K, labels, pooled, counts,
+                                                                     ws);
   return cudaGetLastError();
 }
 
@@ -418,21 +434,19 @@ __device__ __forceinline__ float charge_of(const float* fe, int F, int charge_co
 // memory: W_j = sum q and S_j = sum q p per token, added to `out` (float64,
 // [K][5], global).
 __device__ __forceinline__ void lloyd_chunk_sums(const SortSmem& sm, const float4* s_p, const float* s_q, int npts,
-                                                 int K, double* out) {
-  label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, (int)threadIdx.x, (int)blockDim.x, cta_sync);
-  auto val = [&](int i, int v) {
+                                                 int K, double* acc, double* out) {
+  chunk_token_sums(sm, npts, K, 5, acc, [&](int i, int v) {
     const double q = (double)s_q[i];
     if (v == 0) return q;
     const float4 p = s_p[i];
     return q * (double)(v == 1 ? p.x : (v == 2 ? p.y : (v == 3 ? p.z : p.w)));
-  };
-  token_sums(sm.cnt, sm.start, sm.perm, K, 5, (int)threadIdx.x, (int)blockDim.x, val,
-             [&](int j, int v, double sum, int c) {
-               if (c) atomicAdd(&out[j * 5 + v], sum);
-             });
+  });
+  for (int e = threadIdx.x; e < K * 5; e += blockDim.x)
+    if (sm.cnt[e / 5]) atomicAdd(&out[e], acc[e]);
 }
 
-constexpr size_t kLloydSmemBytes = kSortSmemBytes + (size_t)kChunk * (sizeof(float4) + sizeof(float));
+constexpr size_t kLloydSmemBytes =
+    kSortSmemBytes + (size_t)kChunk * (sizeof(float4) + sizeof(float)) + 256 * 5 * sizeof(double);
 
 // Cell sums of the current labels.
 __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ coords,
@@ -442,8 +456,9 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
                                                     Workspace ws, double* __restrict__ out) {
   extern __shared__ int smem_i[];
   const SortSmem sm = sort_smem(smem_i);
-  float4* s_p = reinterpret_cast<float4*>(smem_i + 2 * kChunk + 3 * 256);
+  float4* s_p = reinterpret_cast<float4*>(smem_i + 3 * kChunk + 3 * 256);
   float* s_q = reinterpret_cast<float*>(s_p + kChunk);
+  double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]
   const int nitems = ws.hdr->n_items[kListChunks];
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
     const int2 it = ws.chunks[item];
@@ -466,7 +481,7 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
       s_p[i] = ldg4(pts + i);
       s_q[i] = charge_of(fe, F, charge_col, i);
     }
-    lloyd_chunk_sums(sm, s_p, s_q, npts, K, out + (int64_t)fs * K * 5);
+    lloyd_chunk_sums(sm, s_p, s_q, npts, K, acc, out + (int64_t)fs * K * 5);
     __syncthreads();
   }
 }
@@ -482,9 +497,10 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
                                                        double* __restrict__ clear, int64_t clear_n) {
   extern __shared__ int smem_i[];
   const SortSmem sm = sort_smem(smem_i);
-  float4* s_p = reinterpret_cast<float4*>(smem_i + 2 * kChunk + 3 * 256);
+  float4* s_p = reinterpret_cast<float4*>(smem_i + 3 * kChunk + 3 * 256);
   float* s_q = reinterpret_cast<float*>(s_p + kChunk);
-  Cent2* s_cent = reinterpret_cast<Cent2*>(s_q + kChunk);  // [K]
+  double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]
+  Cent2* s_cent = reinterpret_cast<Cent2*>(acc + 256 * 5);  // [K]
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < clear_n;
        e += (int64_t)gridDim.x * blockDim.x)
     clear[e] = 0.0;
@@ -524,7 +540,7 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
     });
     if (next) {
       __syncthreads();
-      lloyd_chunk_sums(sm, s_p, s_q, i1 - i0, K, next + (int64_t)fs * K * 5);
+      lloyd_chunk_sums(sm, s_p, s_q, i1 - i0, K, acc, next + (int64_t)fs * K * 5);
     }
     __syncthreads();
   }
@@ -566,6 +582,9 @@ cudaError_t prepare_aux_kernels() {
   if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLloydSmemBytes)))
     return e;
   if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize, step_max)))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_pool_voronoi, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)pool_smem_bytes(256, 64))))
     return e;
   return cudaSuccess;
 }

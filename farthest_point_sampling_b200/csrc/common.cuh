@@ -152,11 +152,12 @@ __device__ __forceinline__ float4 ldg4(const float4* p) { return __ldg(p); }
 // CTA; `rank` / `size` are this thread's index in it and its size, `sync` its
 // barrier): cnt[j] = number of points labelled j, start[j] = exclusive prefix
 // sum, perm[start[j] .. start[j] + cnt[j]) = the local indices of those
-// points.  Labels outside [0, K) are left out.  K <= 256.  All arrays are in
-// shared memory; cur[K] is scratch.
+// points and slab[] the token of every sorted position.  Labels outside
+// [0, K) are left out (the sorted range then ends before npts).  K <= 256.
+// All arrays are in shared memory; cur[K] is scratch.
 template <typename Sync>
 __device__ __forceinline__ void label_sort(const int* lab, int npts, int K, int* cnt, int* start, int* cur,
-                                           int* perm, int rank, int size, Sync sync) {
+                                           int* perm, int* slab, int rank, int size, Sync sync) {
   for (int j = rank; j < K; j += size) cnt[j] = 0;
   sync();
   for (int i = rank; i < npts; i += size) {
@@ -193,33 +194,49 @@ __device__ __forceinline__ void label_sort(const int* lab, int npts, int K, int*
   sync();
   for (int i = rank; i < npts; i += size) {
     const int l = lab[i];
-    if ((unsigned)l < (unsigned)K) perm[atomicAdd(&cur[l], 1)] = i;
+    if ((unsigned)l < (unsigned)K) {
+      const int pos = atomicAdd(&cur[l], 1);
+      perm[pos] = i;
+      slab[pos] = l;
+    }
   }
   sync();
 }
 
-// For every (token j, value v) pair (v < V) handled by this thread of the
-// group: the float64 sum of val(i, v) over the points i sorted to token j,
-// then out(j, v, sum, count).  Loads of four points are issued together.
-template <typename Val, typename Out>
-__device__ __forceinline__ void token_sums(const int* cnt, const int* start, const int* perm, int K, int V,
-                                           int rank, int size, Val val, Out out) {
-  for (int e = rank; e < K * V; e += size) {
-    const int j = e / V, v = e - j * V;
-    const int c = cnt[j];
-    const int* pj = perm + start[j];
-    double s = 0.0;
-    int t = 0;
-    for (; t + 4 <= c; t += 4) {
-      const double a0 = val(pj[t], v), a1 = val(pj[t + 1], v), a2 = val(pj[t + 2], v), a3 = val(pj[t + 3], v);
-      s += a0;
-      s += a1;
-      s += a2;
-      s += a3;
+// Per-token float64 sums over the first nsorted positions of a counting
+// sort, balanced over the group: every thread takes an equal run of sorted
+// positions, adds val(i, v) for v < V along it and flushes its partial sums
+// into acc[token * V + v] (shared memory, zeroed beforehand) whenever the
+// token changes and at the end of its run.  V <= 8 per call.
+template <typename Val>
+__device__ __forceinline__ void segment_sums(const int* perm, const int* slab, int nsorted, int V, int v0,
+                                             int ldacc, double* acc, int rank, int size, Val val) {
+  const int per = (nsorted + size - 1) / size;
+  const int p0 = rank * per, p1 = min(nsorted, p0 + per);
+  if (p0 >= p1) return;
+  double s[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) s[v] = 0.0;
+  int cur = slab[p0];
+  for (int q = p0; q < p1; ++q) {
+    const int i = perm[q];
+    const int l = slab[q];
+    if (l != cur) {
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        if (v < V) {
+          atomicAdd(&acc[cur * ldacc + v0 + v], s[v]);
+          s[v] = 0.0;
+        }
+      cur = l;
     }
-    for (; t < c; ++t) s += val(pj[t], v);
-    out(j, v, s, c);
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      if (v < V) s[v] += val(i, v0 + v);
   }
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    if (v < V) atomicAdd(&acc[cur * ldacc + v0 + v], s[v]);
 }
 
 }  // namespace fpstok

@@ -46,22 +46,6 @@ namespace fpstok {
 
 __device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xffffffffu : ((1u << n) - 1u); }
 
-// Shared memory of one warp of the warp schedule and of a CTA of the
-// register CTA schedule: the event copy during FPS, then (pooling in place)
-// the sort scratch and the staged feature rows of at most kFuse*MaxF floats.
-constexpr size_t pool_region_bytes(int nmax, int max_f) {
-  return (size_t)(2 * nmax + 3 * 256) * sizeof(int) + (size_t)nmax * max_f * sizeof(float);
-}
-constexpr size_t cmax(size_t a, size_t b) { return a > b ? a : b; }
-constexpr size_t kWarpRegionBytes =
-    (cmax((size_t)64 * kWarpPairs * sizeof(DupPoint), pool_region_bytes(64 * kWarpPairs, kFuseWarpMaxF)) + 15) &
-    ~(size_t)15;
-constexpr size_t kCtaRegionBytes =
-    (cmax((size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint), pool_region_bytes(2 * kCtaThreads * kCtaPairs,
-                                                                                    kFuseCtaMaxF)) +
-     15) &
-    ~(size_t)15;
-
 // Dispatches CALL(N) for the compile-time N that equals the runtime np
 // (N <= kMaxPairs).
 #define FPS_CASE(N, CALL) \
@@ -72,45 +56,10 @@ constexpr size_t kCtaRegionBytes =
                 FPS_CASE(6, CALL) FPS_CASE(7, CALL) default : break; }
 
 // One FPS event on one warp, NP point pairs per lane.
-// Token means of an event whose labels sit in registers, pooled in place
-// (no Lloyd follows): the event's feature rows are staged in the group's
-// shared scratch (labels[nmax], perm[nmax], cnt/start/cur[256] ints, then
-// the rows), the points are counting-sorted by token, and one thread per
-// (token, feature) adds its token's rows in float64.
-struct PoolOut {
-  const float* feats;  // null: no pooling in the FPS kernel
-  int F;
-  float* pooled;
-  int32_t* counts;
-};
-
-template <typename Sync>
-__device__ __forceinline__ void pool_event(int* scratch, int nmax, int n, int K, int64_t b, int64_t off,
-                                           const PoolOut& po, int rank, int size, Sync sync) {
-  int* s_lab = scratch;
-  int* perm = scratch + nmax;
-  int* cnt = perm + nmax;
-  float* s_feat = reinterpret_cast<float*>(cnt + 768);  // [n * F] staged feature rows
-  const int F = po.F;
-  const float* fe = po.feats + off * F;
-#pragma unroll 4
-  for (int e = rank; e < n * F; e += size) s_feat[e] = __ldg(fe + e);
-  label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, rank, size, sync);
-  float* prow = po.pooled + b * K * F;
-  int32_t* crow = po.counts + b * K;
-  token_sums(cnt, cnt + 256, perm, K, F, rank, size, [&](int i, int f) { return (double)s_feat[i * F + f]; },
-             [&](int j, int f, double sum, int c) {
-               prow[j * F + f] = c ? (float)(sum / (double)c) : 0.f;
-               if (f == 0) crow[j] = c;
-             });
-  sync();
-}
-
 template <int NP>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                            int lane, DupPoint* s_dup, int32_t* __restrict__ cidx,
-                                           float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
-                                           const PoolOut& po, int nmax) {
+                                           float4* __restrict__ cpos, int32_t* __restrict__ tok) {
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -174,17 +123,6 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       if (i < n) tok[i] = lab[j];
     }
   }
-  if (po.feats) {
-    __syncwarp();  // the event copy is done with; its space becomes the sort scratch
-    int* scratch = reinterpret_cast<int*>(s_dup);
-#pragma unroll
-    for (int j = 0; j < 2 * NP; ++j) {
-      const int i = j * 32 + lane;
-      if (i < n) scratch[i] = lab[j];
-    }
-    __syncwarp();
-    pool_event(scratch, nmax, n, K, b, off, po, lane, 32, [] { __syncwarp(); });
-  }
   __syncwarp();  // the next event overwrites this warp's copy
 }
 
@@ -195,13 +133,12 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
                                                      const int* __restrict__ list, WsHeader* hdr, int K,
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
-                                                     float4* __restrict__ centroids, PoolOut po) {
+                                                     float4* __restrict__ centroids) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
-  static_assert(64 * NPMAX * sizeof(DupPoint) <= kWarpRegionBytes, "event copy fits in the warp's region");
   extern __shared__ DupPoint s_dup_all[];
   const int lane = threadIdx.x & 31;
-  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (kWarpRegionBytes / sizeof(DupPoint));  // this warp's region
+  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
   const int count = hdr->n_items[kListWarp];
   for (;;) {
     int w = 0;
@@ -215,7 +152,7 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define WARP_CALL(N)                                                                                   \
   warp_event<N>(coords + off, n, c0, K, off, lane, s_dup, centroid_idx + (int64_t)b * K,               \
-                centroids + (int64_t)b * K, tok, b, po, 64 * NPMAX)
+                centroids + (int64_t)b * K, tok)
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
   }
@@ -235,8 +172,7 @@ __device__ __forceinline__ int claim_cta(WsHeader* hdr, int list_id, int* slot) 
 template <int NP, int NT>
 __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                           DupPoint* s_dup, int2* xk, int& round, int32_t* __restrict__ cidx,
-                                          float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
-                                          const PoolOut& po, int nmax) {
+                                          float4* __restrict__ cpos, int32_t* __restrict__ tok) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
@@ -316,17 +252,6 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       if (i < n) tok[i] = lab[j];
     }
   }
-  if (po.feats) {
-    __syncthreads();  // the event copy is done with; its space becomes the sort scratch
-    int* scratch = reinterpret_cast<int*>(s_dup);
-#pragma unroll
-    for (int j = 0; j < 2 * NP; ++j) {
-      const int i = j * NT + tid;
-      if (i < n) scratch[i] = lab[j];
-    }
-    __syncthreads();
-    pool_event(scratch, nmax, n, K, b, off, po, tid, NT, [] { __syncthreads(); });
-  }
 }
 
 template <int PR>
@@ -336,10 +261,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
                                                             const int* __restrict__ list, WsHeader* hdr, int K,
                                                             int32_t* __restrict__ centroid_idx,
                                                             int32_t* __restrict__ token_id,
-                                                            float4* __restrict__ centroids, PoolOut po) {
+                                                            float4* __restrict__ centroids) {
   constexpr int kMaxPairs = PR;
   constexpr int NT = kCtaThreads, NW = NT / 32;
-  static_assert(2 * NT * PR * sizeof(DupPoint) <= kCtaRegionBytes, "event copy fits in the region");
   static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
   extern __shared__ DupPoint s_dup[];  // [2 * NT * PR] event copy for centroid look-up
   __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
@@ -356,7 +280,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define CTA_CALL(N)                                                                                     \
   cta_event<N, NT>(coords + off, n, c0, K, off, s_dup, xk, round, centroid_idx + (int64_t)b * K,        \
-                   centroids + (int64_t)b * K, tok, b, po, 2 * NT * PR)
+                   centroids + (int64_t)b * K, tok)
     FPS_DISPATCH_7((n + 2 * NT - 1) / (2 * NT), CTA_CALL)
 #undef CTA_CALL
   }
@@ -585,8 +509,8 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
 // ------------------------------------------------------------------ launch
 
 constexpr int kWarpBlock = 128;
-constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * kWarpRegionBytes;
-constexpr size_t kCtaSmem = kCtaRegionBytes;
+constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(DupPoint);
+constexpr size_t kCtaSmem = (size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint);
 
 template <int CL>
 constexpr size_t block_smem_bytes() {
@@ -726,10 +650,6 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     run[q] = allowed && (hint == 0 || hint > lo);
   }
 
-  const PoolOut none = {nullptr, 0, nullptr, nullptr};
-  const PoolOut pool = {pb.feats, pb.F, pb.pooled, pb.counts};
-  const PoolOut po_warp = (pb.fused_pool & 1) ? pool : none;
-  const PoolOut po_cta = (pb.fused_pool & 2) ? pool : none;
 
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
   bool forked = false;
@@ -745,7 +665,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
         count_launch();
         k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
             pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-            pb.centroids, po_cta);
+            pb.centroids);
         e = cudaGetLastError();
         break;
       case 2:
@@ -768,7 +688,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     count_launch();
     k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, s>>>(pb.coords, pb.offsets, pb.start_local,
                                                                  ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                 pb.token_id, pb.centroids, po_warp);
+                                                                 pb.token_id, pb.centroids);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1, 1, s);
   }

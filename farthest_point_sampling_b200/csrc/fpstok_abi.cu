@@ -176,10 +176,7 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
                 opts->K, opts->assign_mode, opts->k, opts->lloyd_iters, opts->charge_col,
                 opts->force_schedule, opts->max_event_hint, centroid_idx, token_id,
                 opts->assign_mode == FPS_ASSIGN_KNN ? knn_idx : nullptr,
-                reinterpret_cast<float4*>(centroids), pooled, counts,
-                opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0
-                    ? (F <= kFuseWarpMaxF ? 1 : 0) | (F <= kFuseCtaMaxF ? 2 : 0)
-                    : 0};
+                reinterpret_cast<float4*>(centroids), pooled, counts};
   return run_tokenize(pb, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 

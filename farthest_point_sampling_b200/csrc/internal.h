@@ -19,7 +19,7 @@ enum ListId : int {
   kListChunks = 5,      // (event, chunk) items of FPS events (Lloyd, assignment)
   kListPoolSlots = 6,   // events that need global pooling accumulators
   kListFps = 7,         // number of FPS events (Lloyd slots)
-  kListPoolChunks = 8,  // (event, chunk) items pooled by k_pool_voronoi
+  kListPoolChunks = 8,  // (event, chunk) items of the events k_pool_voronoi pools
   kNumLists = 9,
 };
 constexpr int kNumSchedules = 5;  // warp, CTA, CTA-smem, 8-CTA cluster, 16-CTA cluster
@@ -37,8 +37,6 @@ constexpr int kCluster8Cap = 8 * kCtaSmemCap;                 // 98304
 constexpr int kMaxCluster = 16;
 constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
 constexpr int kChunk = 2048;                           // points per pooling / Lloyd work item
-constexpr int kFuseWarpMaxF = 6;  // the warp schedule pools its events in place when F <= this
-constexpr int kFuseCtaMaxF = 7;   // the register CTA schedule likewise
 // With at most this many FPS events per SM, events of the warp class run on
 // the CTA schedule instead (lower latency per step when the GPU is not full).
 constexpr int kLatencyEventsPerSm = 1;
@@ -80,7 +78,6 @@ struct Problem {
   float4* centroids;
   float* pooled;
   int32_t* counts;
-  int fused_pool;  // bit 0 / bit 1: the warp / register-CTA FPS kernels also pool their events
 };
 
 // Kernel launchers (return the cudaError_t of the launch).
