@@ -248,6 +248,8 @@ constexpr size_t kSortSmemBytes = (size_t)(3 * kChunk + 3 * 256) * sizeof(int);
 
 __device__ __forceinline__ void cta_sync() { __syncthreads(); }
 
+constexpr int kStageMaxF = 8;  // the pool kernel stages feature rows in shared memory up to this F
+
 // Sorts the chunk by token and adds up V values per token into acc[K * V]
 // (shared float64, zeroed here): balanced over the CTA.
 template <typename Val>
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
   extern __shared__ int smem_i[];
   const SortSmem sm = sort_smem(smem_i);
   double* acc = reinterpret_cast<double*>(smem_i + 3 * kChunk + 3 * 256);  // [K * F]
+  float* s_feat = reinterpret_cast<float*>(acc + K * F);                    // [kChunk * F] when F <= kStageMaxF
   __shared__ int s_last;
   const int nitems = ws.hdr->n_items[kListPoolChunks];
   const int KF = K * F;
@@ -296,7 +299,13 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
       sm.lab[i] = l;
     }
     const float* fe = feats + (off + i0) * F;
-    chunk_token_sums(sm, npts, K, F, acc, [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); });
+    if (F <= kStageMaxF) {  // stage the chunk's rows with coalesced loads, then sum from shared memory
+#pragma unroll 8
+      for (int e = tid; e < npts * F; e += T) s_feat[e] = __ldg(fe + e);
+      chunk_token_sums(sm, npts, K, F, acc, [&](int i, int f) { return (double)s_feat[i * F + f]; });
+    } else {
+      chunk_token_sums(sm, npts, K, F, acc, [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); });
+    }
     if (nch == 1) {
       for (int e = tid; e < KF; e += T) {
         const int c = sm.cnt[e / F];
@@ -328,7 +337,10 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
   }
 }
 
-static size_t pool_smem_bytes(int K, int F) { return kSortSmemBytes + (size_t)K * F * sizeof(double); }
+static size_t pool_smem_bytes(int K, int F) {
+  return kSortSmemBytes + (size_t)K * F * sizeof(double) +
+         (F <= kStageMaxF ? (size_t)kChunk * F * sizeof(float) : 0);
+}
 
 cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,
@@ -583,8 +595,10 @@ cudaError_t prepare_aux_kernels() {
     return e;
   if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize, step_max)))
     return e;
-  if ((e = cudaFuncSetAttribute(k_pool_voronoi, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)pool_smem_bytes(256, 64))))
+  const size_t pool_max = pool_smem_bytes(256, 64) > pool_smem_bytes(256, kStageMaxF)
+                              ? pool_smem_bytes(256, 64)
+                              : pool_smem_bytes(256, kStageMaxF);
+  if ((e = cudaFuncSetAttribute(k_pool_voronoi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pool_max)))
     return e;
   return cudaSuccess;
 }

@@ -46,7 +46,7 @@ def test_c1_host_offsets_hint():
 # ------------------------------------------------------------- sizes, tiles, ragged tails
 
 EDGE_SIZES = [0, 1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 447, 448, 449, 1000, 2559, 2560,
-              2561, 4095, 12287, 12288, 12289, 30001, 98305]
+              2561, 3071, 3072, 3073, 4095, 12287, 12288, 12289, 30001, 98305]
 
 
 @pytest.mark.parametrize("K", [1, 2, 16, 128, 256])
@@ -72,7 +72,7 @@ def test_ties_and_duplicates(kind):
 
 @pytest.mark.parametrize("force", [0, 1, 2, 3, 4])
 def test_forced_schedules_agree(force):
-    sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000, 98304, 98305]
+    sizes = [129, 300, 448, 449, 2000, 3072, 3073, 12288, 12289, 40000, 98304, 98305]
     b = workloads.random_batch(11, sizes, 128, dup_frac=0.05)
     ora = oracle.tokenize_batch(b)
     compare(b, run_gpu(b, force_schedule=force), ora)
