@@ -138,16 +138,15 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
       list[atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1)] = b;
       fslot = atomicAdd(&cnt[kListFps], 1);
     }
-    const int nch = (n + kChunk - 1) / kChunk;
     if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
+      const int nch = (n + kChunk - 1) / kChunk;
       const int base = atomicAdd(&cnt[kListChunks], nch);
       for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
-    }
-    // events the pool kernel handles (passthrough events are written directly)
-    if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
-      const int base = atomicAdd(&cnt[kListPoolChunks], nch);
-      for (int c = 0; c < nch; ++c) ws.pool_chunks[base + c] = make_int2(b, c);
-      if (nch > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
+      // pooling items (passthrough events of fps_tokenize are written directly)
+      const int npc = (n + kPoolChunk - 1) / kPoolChunk;
+      const int pbase = atomicAdd(&cnt[kListPoolChunks], npc);
+      for (int c = 0; c < npc; ++c) ws.pool_chunks[pbase + c] = make_int2(b, c);
+      if (npc > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
     }
     ws.fps_slot[b] = fslot;
     ws.pool_slot[b] = pslot;
@@ -240,11 +239,11 @@ struct SortSmem {
   int* start;  // [256]
   int* cur;    // [256]
 };
-__device__ __forceinline__ SortSmem sort_smem(int* base) {
-  return SortSmem{base, base + kChunk, base + 2 * kChunk, base + 3 * kChunk, base + 3 * kChunk + 256,
-                  base + 3 * kChunk + 512};
+__device__ __forceinline__ SortSmem sort_smem(int* base, int chunk) {
+  return SortSmem{base, base + chunk, base + 2 * chunk, base + 3 * chunk, base + 3 * chunk + 256,
+                  base + 3 * chunk + 512};
 }
-constexpr size_t kSortSmemBytes = (size_t)(3 * kChunk + 3 * 256) * sizeof(int);
+constexpr size_t sort_smem_bytes(int chunk) { return (size_t)(3 * chunk + 3 * 256) * sizeof(int); }
 
 __device__ __forceinline__ void cta_sync() { __syncthreads(); }
 
@@ -274,9 +273,9 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
                                                       float* __restrict__ pooled,
                                                       int32_t* __restrict__ counts, Workspace ws) {
   extern __shared__ int smem_i[];
-  const SortSmem sm = sort_smem(smem_i);
-  double* acc = reinterpret_cast<double*>(smem_i + 3 * kChunk + 3 * 256);  // [K * F]
-  float* s_feat = reinterpret_cast<float*>(acc + K * F);                    // [kChunk * F] when F <= kStageMaxF
+  const SortSmem sm = sort_smem(smem_i, kPoolChunk);
+  double* acc = reinterpret_cast<double*>(smem_i + 3 * kPoolChunk + 3 * 256);  // [K * F]
+  float* s_feat = reinterpret_cast<float*>(acc + K * F);  // [kPoolChunk * F] when F <= kStageMaxF
   __shared__ int s_last;
   const int nitems = ws.hdr->n_items[kListPoolChunks];
   const int KF = K * F;
@@ -286,10 +285,10 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
     const int b = it.x;
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    const int i0 = it.y * kChunk;
-    const int npts = min(n, i0 + kChunk) - i0;
-    const int nch = (n + kChunk - 1) / kChunk;
-#pragma unroll 8
+    const int i0 = it.y * kPoolChunk;
+    const int npts = min(n, i0 + kPoolChunk) - i0;
+    const int nch = (n + kPoolChunk - 1) / kPoolChunk;
+#pragma unroll 2
     for (int i = tid; i < npts; i += T) {
       int l = labels[off + i0 + i];
       if (l >= K) {
@@ -338,8 +337,8 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
 }
 
 static size_t pool_smem_bytes(int K, int F) {
-  return kSortSmemBytes + (size_t)K * F * sizeof(double) +
-         (F <= kStageMaxF ? (size_t)kChunk * F * sizeof(float) : 0);
+  return sort_smem_bytes(kPoolChunk) + (size_t)K * F * sizeof(double) +
+         (F <= kStageMaxF ? (size_t)kPoolChunk * F * sizeof(float) : 0);
 }
 
 cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
@@ -347,7 +346,7 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
                                 const Workspace& ws, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   count_launch();
-  k_pool_voronoi<<<di.sm_count * 6, 256, pool_smem_bytes(K, F), s>>>(feats, F, offsets, K, labels, pooled, counts,
+  k_pool_voronoi<<<di.sm_count * 8, 256, pool_smem_bytes(K, F), s>>>(feats, F, offsets, K, labels, pooled, counts,
                                                                      ws);
   return cudaGetLastError();
 }
@@ -458,7 +457,7 @@ __device__ __forceinline__ void lloyd_chunk_sums(const SortSmem& sm, const float
 }
 
 constexpr size_t kLloydSmemBytes =
-    kSortSmemBytes + (size_t)kChunk * (sizeof(float4) + sizeof(float)) + 256 * 5 * sizeof(double);
+    sort_smem_bytes(kChunk) + (size_t)kChunk * (sizeof(float4) + sizeof(float)) + 256 * 5 * sizeof(double);
 
 // Cell sums of the current labels.
 __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ coords,
@@ -467,7 +466,7 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
                                                     int K, const int32_t* __restrict__ labels,
                                                     Workspace ws, double* __restrict__ out) {
   extern __shared__ int smem_i[];
-  const SortSmem sm = sort_smem(smem_i);
+  const SortSmem sm = sort_smem(smem_i, kChunk);
   float4* s_p = reinterpret_cast<float4*>(smem_i + 3 * kChunk + 3 * 256);
   float* s_q = reinterpret_cast<float*>(s_p + kChunk);
   double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]
@@ -508,7 +507,7 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
                                                        const double* __restrict__ in, double* __restrict__ next,
                                                        double* __restrict__ clear, int64_t clear_n) {
   extern __shared__ int smem_i[];
-  const SortSmem sm = sort_smem(smem_i);
+  const SortSmem sm = sort_smem(smem_i, kChunk);
   float4* s_p = reinterpret_cast<float4*>(smem_i + 3 * kChunk + 3 * 256);
   float* s_q = reinterpret_cast<float*>(s_p + kChunk);
   double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]

@@ -21,7 +21,7 @@
 // the block schedules on helper streams forked from the caller's stream):
 //   warp        N <= 448     one warp per event, points in registers (lane l
 //                            owns points l + 32 j); arg-max by two redux.sync.
-//   CTA         N <= 3072    one 512-thread CTA per event, points in
+//   CTA         N <= 2560    one 256-thread CTA per event, points in
 //                            registers; warp winners exchanged through shared
 //                            memory, one barrier per step.  Also takes the
 //                            warp-class events when there are few events.

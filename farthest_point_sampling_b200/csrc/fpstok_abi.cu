@@ -41,7 +41,8 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   Workspace w = {};
   const int64_t nb = B > 0 ? B : 1;
   const int64_t chunks = nb + P / kChunk + 1;
-  const int64_t pool_slots = P / kChunk + 1;
+  const int64_t pool_chunks = nb + P / kPoolChunk + 1;
+  const int64_t pool_slots = P / kPoolChunk + 1;
   int64_t fps_slots = P / (K + 1) + 1;
   if (fps_slots > nb) fps_slots = nb;
   w.hdr = c.take<WsHeader>(1);
@@ -51,7 +52,7 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   w.list_cluster8 = c.take<int>(nb);
   w.list_cluster16 = c.take<int>(nb);
   w.chunks = c.take<int2>(chunks);
-  w.pool_chunks = c.take<int2>(chunks);
+  w.pool_chunks = c.take<int2>(pool_chunks);
   w.cls = c.take<int>(nb);
   w.fps_slot = c.take<int>(nb);
   w.pool_slot = c.take<int>(nb);

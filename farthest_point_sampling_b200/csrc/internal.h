@@ -27,16 +27,17 @@ constexpr int kNumSchedules = 5;  // warp, CTA, CTA-smem, 8-CTA cluster, 16-CTA 
 // Schedule capacities (points per event).
 constexpr int kWarpPairs = 7;                          // point pairs per lane, warp schedule
 constexpr int kWarpCap = 64 * kWarpPairs;              // 448
-constexpr int kCtaThreads = 512;                       // register-resident CTA schedule
-constexpr int kCtaPairs = 3;                           // pairs per thread
-constexpr int kCtaCap = 2 * kCtaThreads * kCtaPairs;   // 3072
+constexpr int kCtaThreads = 256;                       // register-resident CTA schedule
+constexpr int kCtaPairs = 5;                           // pairs per thread
+constexpr int kCtaCap = 2 * kCtaThreads * kCtaPairs;   // 2560
 constexpr int kBlockThreads = 256;                     // shared-memory CTA / cluster schedules
 constexpr int kBlockPairs = 24;                        // pairs per thread in shared memory
 constexpr int kCtaSmemCap = kBlockThreads * 2 * kBlockPairs;  // 12288
 constexpr int kCluster8Cap = 8 * kCtaSmemCap;                 // 98304
 constexpr int kMaxCluster = 16;
 constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
-constexpr int kChunk = 2048;                           // points per pooling / Lloyd work item
+constexpr int kChunk = 2048;                           // points per Lloyd / assignment work item
+constexpr int kPoolChunk = 512;                        // points per pooling work item
 // With at most this many FPS events per SM, events of the warp class run on
 // the CTA schedule instead (lower latency per step when the GPU is not full).
 constexpr int kLatencyEventsPerSm = 1;

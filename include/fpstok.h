@@ -93,7 +93,7 @@ enum {
 #define FPS_ASSIGN_KNN 1
 
 /* force_schedule: -1 picks by event size; 0 warp (N <= 448), 1 CTA with points
- * in registers (N <= 3072), 2 CTA with points in shared memory (N <= 12288),
+ * in registers (N <= 2560), 2 CTA with points in shared memory (N <= 12288),
  * 3 8-CTA cluster (N <= 98304), 4 16-CTA cluster (N <= 196608) means "use at
  * least this schedule" (events too large for it move up). */
 typedef struct fps_opts {

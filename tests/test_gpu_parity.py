@@ -72,7 +72,7 @@ def test_ties_and_duplicates(kind):
 
 @pytest.mark.parametrize("force", [0, 1, 2, 3, 4])
 def test_forced_schedules_agree(force):
-    sizes = [129, 300, 448, 449, 2000, 3072, 3073, 12288, 12289, 40000, 98304, 98305]
+    sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000, 98304, 98305]
     b = workloads.random_batch(11, sizes, 128, dup_frac=0.05)
     ora = oracle.tokenize_batch(b)
     compare(b, run_gpu(b, force_schedule=force), ora)
@@ -164,7 +164,7 @@ def test_standalone_knn():
 
 
 def test_standalone_pool():
-    b = workloads.random_batch(52, [0, 10, 100, 2047, 2048, 2049, 9000], 32, F=5)
+    b = workloads.random_batch(52, [0, 10, 100, 511, 512, 513, 2047, 2048, 2049, 9000], 32, F=5)
     c, f, o, ora, cent = _fps_state(b)
     tok = torch.from_numpy(ora["token_id"]).cuda()
     pooled, counts = fps.segment_pool(f, o, 32, token_id=tok)
