@@ -112,16 +112,30 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1);
   }
   __syncthreads();
-  // exclusive scan from the largest bucket down: list position of each bucket
-  if (threadIdx.x < kNumSchedules) {
-    const int q = threadIdx.x;
-    int run = 0;
-    for (int i = kBins - 1; i >= 0; --i) {
-      const int h = hist[q][i];
-      hist[q][i] = run;
-      run += h;
+  // exclusive scan from the largest bucket down (one warp per schedule, 8
+  // buckets per lane): list position of each bucket
+  if (threadIdx.x < 32 * kNumSchedules) {
+    const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int v[kBins / 32];
+    int sum = 0;
+#pragma unroll
+    for (int r = 0; r < kBins / 32; ++r) {
+      v[r] = hist[q][kBins - 1 - (lane * (kBins / 32) + r)];
+      sum += v[r];
     }
-    cnt[q] = run;
+    int x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += y;
+    }
+    int run = x - sum;
+#pragma unroll
+    for (int r = 0; r < kBins / 32; ++r) {
+      hist[q][kBins - 1 - (lane * (kBins / 32) + r)] = run;
+      run += v[r];
+    }
+    if (lane == 31) cnt[q] = run;
   }
   __syncthreads();
   // pass 3: scatter into the sorted lists; chunks and accumulator slots
@@ -166,23 +180,25 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
 // ------------------------------------------------------------------ passthrough
 
 // Events with N <= K keep one token per pulse; empty and skipped events get
-// empty rows; FPS events get their global accumulators cleared.  One CTA per
-// event (grid-stride), copies unrolled so that loads overlap.
+// empty rows; FPS events get their global accumulators cleared.  One warp per
+// event, copies unrolled so that loads overlap.
 __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, int lloyd_on) {
   const int K = pb.K, F = pb.F, k = pb.k;
-  const int T = blockDim.x;
-  for (int b = blockIdx.x; b < pb.B; b += gridDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int b = gw; b < pb.B; b += nw) {
     const int cls = ws.cls[b];
     if (cls == kClsFps) {
       const int ps = ws.pool_slot[b];
       if (ps >= 0) {
-        for (int e = threadIdx.x; e < K * F; e += T) ws.pool_acc[(int64_t)ps * K * F + e] = 0.0;
-        for (int e = threadIdx.x; e < K; e += T) ws.pool_cnt[(int64_t)ps * K + e] = 0;
-        if (threadIdx.x == 0) ws.pool_ticket[ps] = 0;
+        for (int e = lane; e < K * F; e += 32) ws.pool_acc[(int64_t)ps * K * F + e] = 0.0;
+        for (int e = lane; e < K; e += 32) ws.pool_cnt[(int64_t)ps * K + e] = 0;
+        if (lane == 0) ws.pool_ticket[ps] = 0;
       }
       const int fs = ws.fps_slot[b];
       if (lloyd_on && fs >= 0) {
-        for (int e = threadIdx.x; e < K * 5; e += T) {
+        for (int e = lane; e < K * 5; e += 32) {
           ws.lloyd[0][(int64_t)fs * K * 5 + e] = 0.0;
           ws.lloyd[1][(int64_t)fs * K * 5 + e] = 0.0;
         }
@@ -195,33 +211,36 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
       off = pb.offsets[b];
       n = (int)(pb.offsets[b + 1] - off);
     }
-    const float* cf = reinterpret_cast<const float*>(pb.coords);
+    const float* cf = reinterpret_cast<const float*>(pb.coords) + off * 4;
     float* outc = reinterpret_cast<float*>(pb.centroids) + (int64_t)b * K * 4;
-#pragma unroll 4
-    for (int e = threadIdx.x; e < K * 4; e += T) outc[e] = e < n * 4 ? cf[off * 4 + e] : 0.f;
+    const int nc = n * 4;
+#pragma unroll 8
+    for (int e = lane; e < K * 4; e += 32) outc[e] = e < nc ? cf[e] : 0.f;
+    const float* fe = pb.feats + off * F;
     float* outp = pb.pooled + (int64_t)b * K * F;
+    const int nf = n * F;
+#pragma unroll 8
+    for (int e = lane; e < K * F; e += 32) outp[e] = e < nf ? fe[e] : 0.f;
+    int32_t* ci = pb.centroid_idx + (int64_t)b * K;
+    int32_t* co = pb.counts + (int64_t)b * K;
 #pragma unroll 4
-    for (int e = threadIdx.x; e < K * F; e += T) outp[e] = e < n * F ? pb.feats[off * F + e] : 0.f;
-    for (int j = threadIdx.x; j < K; j += T) {
-      pb.centroid_idx[(int64_t)b * K + j] = j < n ? (int32_t)(off + j) : -1;
-      pb.counts[(int64_t)b * K + j] = j < n ? 1 : 0;
+    for (int j = lane; j < K; j += 32) {
+      ci[j] = j < n ? (int32_t)(off + j) : -1;
+      co[j] = j < n ? 1 : 0;
     }
     if (pb.token_id)
-      for (int j = threadIdx.x; j < n; j += T) pb.token_id[off + j] = j;
+      for (int j = lane; j < n; j += 32) pb.token_id[off + j] = j;
     if (pb.knn_idx) {
       int32_t* outk = pb.knn_idx + (int64_t)b * K * k;
-      for (int e = threadIdx.x; e < K * k; e += T) {
-        const int j = e / k, r = e - j * k;
-        outk[e] = (r == 0 && j < n) ? (int32_t)(off + j) : -1;
-      }
+      for (int j = 0; j < K; ++j)
+        for (int r = lane; r < k; r += 32) outk[j * k + r] = (r == 0 && j < n) ? (int32_t)(off + j) : -1;
     }
   }
 }
 
 cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s) {
-  int blocks = pb.B;
-  const int cap = 65535;
-  if (blocks > cap) blocks = cap;
+  int blocks = (pb.B + 7) / 8;
+  if (blocks > 65535) blocks = 65535;
   if (blocks < 1) blocks = 1;
   count_launch();
   k_passthrough<<<blocks, 256, 0, s>>>(pb, ws, pb.lloyd_iters > 0 ? 1 : 0);
@@ -264,9 +283,13 @@ __device__ __forceinline__ void chunk_token_sums(const SortSmem& sm, int npts, i
 }
 
 // One CTA per (event, chunk) item: counting sort of the chunk's points by
-// token, balanced float64 sums per (token, feature), then the means
-// (single-chunk event) or float64 accumulation in global memory with the
-// last-arriving CTA of the event producing the means.
+// token, float64 sums per (token, feature) -- one thread per token when no
+// token holds more than kDenseToken points of the chunk, else the balanced
+// segmented sums -- then the means (single-chunk event) or float64
+// accumulation in global memory with the last-arriving CTA of the event
+// producing the means.  Thread j < K owns token j's outputs.
+constexpr int kDenseToken = 32;
+
 __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ feats, int F,
                                                       const int64_t* __restrict__ offsets, int K,
                                                       const int32_t* __restrict__ labels,
@@ -278,7 +301,6 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
   float* s_feat = reinterpret_cast<float*>(acc + K * F);  // [kPoolChunk * F] when F <= kStageMaxF
   __shared__ int s_last;
   const int nitems = ws.hdr->n_items[kListPoolChunks];
-  const int KF = K * F;
   const int T = blockDim.x, tid = threadIdx.x;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
     const int2 it = ws.pool_chunks[item];
@@ -288,6 +310,8 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
     const int i0 = it.y * kPoolChunk;
     const int npts = min(n, i0 + kPoolChunk) - i0;
     const int nch = (n + kPoolChunk - 1) / kPoolChunk;
+    const bool staged = F <= kStageMaxF;
+    const float* fe = feats + (off + i0) * F;
 #pragma unroll 2
     for (int i = tid; i < npts; i += T) {
       int l = labels[off + i0 + i];
@@ -297,39 +321,62 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
       }
       sm.lab[i] = l;
     }
-    const float* fe = feats + (off + i0) * F;
-    if (F <= kStageMaxF) {  // stage the chunk's rows with coalesced loads, then sum from shared memory
-#pragma unroll 8
+    if (staged) {
+#pragma unroll 4
       for (int e = tid; e < npts * F; e += T) s_feat[e] = __ldg(fe + e);
-      chunk_token_sums(sm, npts, K, F, acc, [&](int i, int f) { return (double)s_feat[i * F + f]; });
-    } else {
-      chunk_token_sums(sm, npts, K, F, acc, [&](int i, int f) { return (double)__ldg(fe + (int64_t)i * F + f); });
     }
-    if (nch == 1) {
-      for (int e = tid; e < KF; e += T) {
-        const int c = sm.cnt[e / F];
-        pooled[(int64_t)b * KF + e] = c ? (float)(acc[e] / (double)c) : 0.f;
+    label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, sm.slab, tid, T, cta_sync);
+    auto val = [&](int i, int f) { return staged ? (double)s_feat[i * F + f] : (double)__ldg(fe + (int64_t)i * F + f); };
+    const int cj = tid < K ? sm.cnt[tid] : 0;
+    const bool dense = __syncthreads_or(cj > kDenseToken);
+    if (dense) {  // balanced over the CTA, flushed into acc
+      for (int e = tid; e < K * F; e += T) acc[e] = 0.0;
+      __syncthreads();
+      const int nsorted = sm.start[K - 1] + sm.cnt[K - 1];
+      for (int v0 = 0; v0 < F; v0 += 8)
+        segment_sums(sm.perm, sm.slab, nsorted, min(8, F - v0), v0, F, acc, tid, T, val);
+    } else if (tid < K) {  // one thread per token: its (short) run, in sorted order
+      const int* pj = sm.perm + sm.start[tid];
+      for (int f0 = 0; f0 < F; f0 += 8) {
+        double s8[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) s8[v] = 0.0;
+        for (int t = 0; t < cj; ++t) {
+          const int i = pj[t];
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            if (f0 + v < F) s8[v] += val(i, f0 + v);
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          if (f0 + v < F) acc[tid * F + f0 + v] = s8[v];
       }
-      for (int j = tid; j < K; j += T) counts[(int64_t)b * K + j] = sm.cnt[j];
+    }
+    __syncthreads();
+    if (nch == 1) {
+      if (tid < K) {
+        float* prow = pooled + ((int64_t)b * K + tid) * F;
+        for (int f = 0; f < F; ++f) prow[f] = cj ? (float)(acc[tid * F + f] / (double)cj) : 0.f;
+        counts[(int64_t)b * K + tid] = cj;
+      }
     } else {
       const int ps = ws.pool_slot[b];
-      double* gacc = ws.pool_acc + (int64_t)ps * KF;
+      double* gacc = ws.pool_acc + (int64_t)ps * K * F;
       int* gcnt = ws.pool_cnt + (int64_t)ps * K;
-      for (int e = tid; e < KF; e += T)
-        if (sm.cnt[e / F]) atomicAdd(&gacc[e], acc[e]);
-      for (int j = tid; j < K; j += T)
-        if (sm.cnt[j]) atomicAdd(&gcnt[j], sm.cnt[j]);
+      if (tid < K && cj) {
+        for (int f = 0; f < F; ++f) atomicAdd(&gacc[tid * F + f], acc[tid * F + f]);
+        atomicAdd(&gcnt[tid], cj);
+      }
       __threadfence();
       __syncthreads();
       if (tid == 0) s_last = atomicAdd(&ws.pool_ticket[ps], 1) == nch - 1;
       __syncthreads();
-      if (s_last) {
+      if (s_last && tid < K) {
         __threadfence();
-        for (int e = tid; e < KF; e += T) {
-          const int c = __ldcg(&gcnt[e / F]);
-          pooled[(int64_t)b * KF + e] = c ? (float)(__ldcg(&gacc[e]) / (double)c) : 0.f;
-        }
-        for (int j = tid; j < K; j += T) counts[(int64_t)b * K + j] = __ldcg(&gcnt[j]);
+        const int c = __ldcg(&gcnt[tid]);
+        float* prow = pooled + ((int64_t)b * K + tid) * F;
+        for (int f = 0; f < F; ++f) prow[f] = c ? (float)(__ldcg(&gacc[tid * F + f]) / (double)c) : 0.f;
+        counts[(int64_t)b * K + tid] = c;
       }
     }
     __syncthreads();
