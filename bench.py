@@ -39,11 +39,11 @@ SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 FP32_OPS_PER_LANE_CLK = 2  # packed f32x2 add/sub/mul: two float32 operations per lane per clock
 SM_MAX_MHZ_NOMINAL = 1965.0
-STAGES = ["bin+passthrough", "fps_warp", "fps_cta", "fps_cta_smem", "fps_cluster8", "fps_cluster16", "lloyd",
-          "knn+pool", "voronoi_pool"]
-STAGE_KERNELS = {0: "k_bin+k_passthrough", 1: "k_fps_warp", 2: "k_fps_cta", 3: "k_fps_block<1>",
+STAGES = ["bin", "fps_warp", "fps_cta", "fps_cta_smem", "fps_cluster8", "fps_cluster16", "lloyd",
+          "knn+pool", "voronoi_pool", "passthrough"]
+STAGE_KERNELS = {0: "k_bin", 1: "k_fps_warp", 2: "k_fps_cta", 3: "k_fps_block<1>",
                  4: "k_fps_block<8>", 5: "k_fps_block<16>", 6: "k_lloyd_sums+k_lloyd_step", 7: "k_knn",
-                 8: "k_pool_voronoi"}
+                 8: "k_pool_voronoi", 9: "k_passthrough"}
 FPS_STAGES = (1, 2, 3, 4, 5)
 METRIC = "FPS+assign events/s (K=128)"
 
@@ -419,7 +419,7 @@ def main():
     sched = np.array([lib.fps_schedule_for(int(n), batch.K, -1) for n in sizes])
     if (sched >= 0).sum() <= SM_COUNT:  # few events: the warp class runs on the CTA schedule
         sched = np.where(sched == 0, 1, sched)
-    ran = {0, 8 if batch.assign_mode == 0 else 7}
+    ran = {0, 9, 8 if batch.assign_mode == 0 else 7}
     ran |= {1 + s for s in (0, 1, 2, 3, 4) if (sched == s).any()}
     if batch.lloyd_iters:
         ran.add(6)

@@ -36,7 +36,8 @@ __device__ __forceinline__ int sched_shift(int q) {
 // events, and the accumulator slots; resets the status word and the cursors.
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
-                                               int force, int chunk_all, int latency_events, Workspace ws) {
+                                               int force, int chunk_all, int fused_pool, int latency_events,
+                                               Workspace ws) {
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps;
@@ -156,7 +157,13 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
       const int nch = (n + kChunk - 1) / kChunk;
       const int base = atomicAdd(&cnt[kListChunks], nch);
       for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
-      // pooling items (passthrough events of fps_tokenize are written directly)
+      // pooling items (passthrough events of fps_tokenize are written directly;
+      // events of schedules that pool in place are left out)
+      if (cls == kClsFps && ((fused_pool >> schedule_of(n)) & 1)) {
+        ws.fps_slot[b] = fslot;
+        ws.pool_slot[b] = -1;
+        continue;
+      }
       const int npc = (n + kPoolChunk - 1) / kPoolChunk;
       const int pbase = atomicAdd(&cnt[kListPoolChunks], npc);
       for (int c = 0; c < npc; ++c) ws.pool_chunks[pbase + c] = make_int2(b, c);
@@ -173,7 +180,7 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
   const DeviceInfo& di = device_info();
   count_launch();
   k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
-                           kLatencyEventsPerSm * di.sm_count, ws);
+                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, ws);
   return cudaGetLastError();
 }
 
@@ -230,10 +237,13 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
     }
     if (pb.token_id)
       for (int j = lane; j < n; j += 32) pb.token_id[off + j] = j;
-    if (pb.knn_idx) {
+    if (pb.knn_idx) {  // row j = [point j, -1, ...]; one row per lane at a time
       int32_t* outk = pb.knn_idx + (int64_t)b * K * k;
-      for (int j = 0; j < K; ++j)
-        for (int r = lane; r < k; r += 32) outk[j * k + r] = (r == 0 && j < n) ? (int32_t)(off + j) : -1;
+      for (int j = lane; j < K; j += 32) {
+        int32_t* row = outk + (int64_t)j * k;
+        row[0] = j < n ? (int32_t)(off + j) : -1;
+        for (int r = 1; r < k; ++r) row[r] = -1;
+      }
     }
   }
 }

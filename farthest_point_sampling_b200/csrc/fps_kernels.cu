@@ -55,11 +55,21 @@ __device__ __forceinline__ unsigned low_bits(int n) { return n >= 32 ? 0xfffffff
   switch (np) { FPS_CASE(1, CALL) FPS_CASE(2, CALL) FPS_CASE(3, CALL) FPS_CASE(4, CALL) FPS_CASE(5, CALL) \
                 FPS_CASE(6, CALL) FPS_CASE(7, CALL) default : break; }
 
+// Where an FPS kernel writes the token means of the events it pools itself
+// (no Lloyd follows): feats == nullptr means the pool kernel does it.
+struct PoolOut {
+  const float* feats;
+  int F;
+  float* pooled;
+  int32_t* counts;
+};
+
 // One FPS event on one warp, NP point pairs per lane.
 template <int NP>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                            int lane, DupPoint* s_dup, int32_t* __restrict__ cidx,
-                                           float4* __restrict__ cpos, int32_t* __restrict__ tok) {
+                                           float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
+                                           const PoolOut& po) {
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -123,6 +133,39 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       if (i < n) tok[i] = lab[j];
     }
   }
+  if (po.feats) {  // token means: float64 shared sums over the event copy's space
+    const int F = po.F;
+    __syncwarp();
+    double* acc = reinterpret_cast<double*>(s_dup);  // [K * F]
+    int* cnt = reinterpret_cast<int*>(acc + K * F);   // [K]
+    for (int e = lane; e < K * F; e += 32) acc[e] = 0.0;
+    for (int j = lane; j < K; j += 32) cnt[j] = 0;
+    __syncwarp();
+    const float* fe = po.feats + off * F;
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {  // slot j: 32 consecutive rows, one per lane
+      const int i = j * 32 + lane;
+      if (i >= n) continue;
+      const int l = lab[j];
+      atomicAdd(&cnt[l], 1);
+      const float* row = fe + (int64_t)i * F;
+      for (int f0 = 0; f0 < F; f0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int f = 0; f < 8; ++f) v[f] = f0 + f < F ? __ldg(row + f0 + f) : 0.f;
+#pragma unroll
+        for (int f = 0; f < 8; ++f)
+          if (f0 + f < F) atomicAdd(&acc[l * F + f0 + f], (double)v[f]);
+      }
+    }
+    __syncwarp();
+    for (int j = lane; j < K; j += 32) {
+      const int c = cnt[j];
+      float* prow = po.pooled + (b * K + j) * F;
+      for (int f = 0; f < F; ++f) prow[f] = c ? (float)(acc[j * F + f] / (double)c) : 0.f;
+      po.counts[b * K + j] = c;
+    }
+  }
   __syncwarp();  // the next event overwrites this warp's copy
 }
 
@@ -133,7 +176,7 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
                                                      const int* __restrict__ list, WsHeader* hdr, int K,
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
-                                                     float4* __restrict__ centroids) {
+                                                     float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
   extern __shared__ DupPoint s_dup_all[];
@@ -152,7 +195,7 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define WARP_CALL(N)                                                                                   \
   warp_event<N>(coords + off, n, c0, K, off, lane, s_dup, centroid_idx + (int64_t)b * K,               \
-                centroids + (int64_t)b * K, tok)
+                centroids + (int64_t)b * K, tok, b, po)
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
   }
@@ -169,10 +212,11 @@ __device__ __forceinline__ int claim_cta(WsHeader* hdr, int list_id, int* slot) 
   return *slot;
 }
 
-template <int NP, int NT>
+template <int NP, int NT, int kMaxPairsCta>
 __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                           DupPoint* s_dup, int2* xk, int& round, int32_t* __restrict__ cidx,
-                                          float4* __restrict__ cpos, int32_t* __restrict__ tok) {
+                                          float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
+                                          const PoolOut& po) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
@@ -252,6 +296,37 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       if (i < n) tok[i] = lab[j];
     }
   }
+  if (po.feats) {  // token means: sort by token, balanced float64 sums over the event copy's space
+    constexpr int NMAX = 2 * NT * kMaxPairsCta;
+    const int F = po.F;
+    __syncthreads();
+    int* s_lab = reinterpret_cast<int*>(s_dup);
+    int* perm = s_lab + NMAX;
+    int* slab = perm + NMAX;
+    int* cnt = slab + NMAX;  // cnt, start, cur: 3 x 256
+    float* s_feat = reinterpret_cast<float*>(cnt + 768);        // [n * F]
+    double* acc = reinterpret_cast<double*>(s_feat + NMAX * F);  // [K * F]
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = j * NT + tid;
+      if (i < n) s_lab[i] = lab[j];
+    }
+    const float* fe = po.feats + off * F;
+#pragma unroll 4
+    for (int e = tid; e < n * F; e += NT) s_feat[e] = __ldg(fe + e);
+    for (int e = tid; e < K * F; e += NT) acc[e] = 0.0;
+    label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, slab, tid, NT, [] { __syncthreads(); });
+    for (int v0 = 0; v0 < F; v0 += 8)
+      segment_sums(perm, slab, n, min(8, F - v0), v0, F, acc, tid, NT,
+                   [&](int i, int f) { return (double)s_feat[i * F + f]; });
+    __syncthreads();
+    for (int j = tid; j < K; j += NT) {
+      const int c = cnt[j];
+      float* prow = po.pooled + (b * K + j) * F;
+      for (int f = 0; f < F; ++f) prow[f] = c ? (float)(acc[j * F + f] / (double)c) : 0.f;
+      po.counts[b * K + j] = c;
+    }
+  }
 }
 
 template <int PR>
@@ -261,7 +336,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
                                                             const int* __restrict__ list, WsHeader* hdr, int K,
                                                             int32_t* __restrict__ centroid_idx,
                                                             int32_t* __restrict__ token_id,
-                                                            float4* __restrict__ centroids) {
+                                                            float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = PR;
   constexpr int NT = kCtaThreads, NW = NT / 32;
   static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
@@ -279,8 +354,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
     const int c0 = start_local ? start_local[b] : 0;
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define CTA_CALL(N)                                                                                     \
-  cta_event<N, NT>(coords + off, n, c0, K, off, s_dup, xk, round, centroid_idx + (int64_t)b * K,        \
-                   centroids + (int64_t)b * K, tok)
+  cta_event<N, NT, PR>(coords + off, n, c0, K, off, s_dup, xk, round, centroid_idx + (int64_t)b * K,    \
+                       centroids + (int64_t)b * K, tok, b, po)
     FPS_DISPATCH_7((n + 2 * NT - 1) / (2 * NT), CTA_CALL)
 #undef CTA_CALL
   }
@@ -510,7 +585,11 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
 
 constexpr int kWarpBlock = 128;
 constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(DupPoint);
-constexpr size_t kCtaSmem = (size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint);
+constexpr size_t kCtaSmem = kCtaSmemBytes;
+static_assert((size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint) <= kCtaSmem, "event copy fits");
+
+size_t warp_region_bytes() { return (size_t)64 * kWarpPairs * sizeof(DupPoint); }
+size_t cta_region_bytes() { return kCtaSmem; }
 
 template <int CL>
 constexpr size_t block_smem_bytes() {
@@ -568,7 +647,7 @@ static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list
 
 // Per-device state: occupancy figures and the helper streams / events that
 // let the schedules run concurrently.
-constexpr int kHelpers = kNumSchedules - 1;
+constexpr int kHelpers = kNumSchedules;  // four block schedules and the passthrough kernel
 struct DeviceCtx {
   DeviceInfo info;
   cudaStream_t helper[kHelpers];
@@ -629,7 +708,7 @@ const DeviceInfo& device_info() {
   return g_ctx[dev].info;
 }
 
-cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, StageMark mark) {
+cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws, cudaStream_t s, StageMark mark) {
   const int dev = current_device();
   if (dev < 0) return cudaErrorInvalidDevice;
   cudaError_t e = prepare(dev);
@@ -651,10 +730,21 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
   }
 
 
+  const PoolOut none = {nullptr, 0, nullptr, nullptr};
+  const PoolOut pool = {pb.feats, pb.F, pb.pooled, pb.counts};
+  const PoolOut po_warp = (pb.fused_pool & 1) ? pool : none;
+  const PoolOut po_cta = (pb.fused_pool & 2) ? pool : none;
+
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
-  bool forked = false;
-  for (int q = 1; q < kNumSchedules; ++q) forked |= run[q];
-  if (forked && (e = cudaEventRecord(ctx.fork, s))) return e;
+  if ((e = cudaEventRecord(ctx.fork, s))) return e;
+  {  // passthrough rows and accumulator clearing overlap the FPS kernels
+    cudaStream_t hs = ctx.helper[kHelpers - 1];
+    if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
+    mark(kStagePassthrough, 0, hs);
+    if ((e = launch_passthrough(pt, ws, hs))) return e;
+    mark(kStagePassthrough, 1, hs);
+    if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;
+  }
   for (int q = 1; q < kNumSchedules; ++q) {
     if (!run[q]) continue;
     cudaStream_t hs = ctx.helper[q - 1];
@@ -665,7 +755,7 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
         count_launch();
         k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
             pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-            pb.centroids);
+            pb.centroids, po_cta);
         e = cudaGetLastError();
         break;
       case 2:
@@ -688,13 +778,13 @@ cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, S
     count_launch();
     k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, s>>>(pb.coords, pb.offsets, pb.start_local,
                                                                  ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                 pb.token_id, pb.centroids);
+                                                                 pb.token_id, pb.centroids, po_warp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1, 1, s);
   }
   for (int q = 1; q < kNumSchedules; ++q)
     if (run[q] && (e = cudaStreamWaitEvent(s, ctx.join[q - 1], 0))) return e;
-  return cudaSuccess;
+  return cudaStreamWaitEvent(s, ctx.join[kHelpers - 1], 0);
 }
 
 }  // namespace fpstok

@@ -108,12 +108,11 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
   cudaError_t e;
   stage_mark(0, 0, s);
   if ((e = launch_bin(pb, ws, 0, s))) return from_cuda(e);
+  stage_mark(0, 1, s);
   Problem pt = pb;
   pt.token_id = pb0.token_id;
   pt.knn_idx = pb.assign_mode == FPS_ASSIGN_KNN ? pb.knn_idx : nullptr;
-  if ((e = launch_passthrough(pt, ws, s))) return from_cuda(e);
-  stage_mark(0, 1, s);
-  if ((e = launch_fps(pb, ws, s, stage_mark))) return from_cuda(e);
+  if ((e = launch_fps(pb, pt, ws, s, stage_mark))) return from_cuda(e);
   if (pb.lloyd_iters > 0) {
     stage_mark(6, 0, s);
     if ((e = launch_lloyd(pb, ws, labels, s))) return from_cuda(e);
@@ -126,10 +125,16 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
       return from_cuda(e);
     stage_mark(7, 1, s);
   } else {
-    stage_mark(8, 0, s);
-    if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.K, labels, pb.pooled, pb.counts, ws, s)))
-      return from_cuda(e);
-    stage_mark(8, 1, s);
+    // with a size hint, a batch whose events all fit the schedules that pool
+    // in place needs no pool kernel
+    const bool none_left = pb.max_event_hint > 0 && pb.max_event_hint <= kCtaCap && pb.force_schedule <= 1 &&
+                           (pb.fused_pool & 3) == 3;
+    if (!none_left) {
+      stage_mark(8, 0, s);
+      if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.K, labels, pb.pooled, pb.counts, ws, s)))
+        return from_cuda(e);
+      stage_mark(8, 1, s);
+    }
   }
   return FPS_OK;
 }
@@ -177,7 +182,14 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
                 opts->K, opts->assign_mode, opts->k, opts->lloyd_iters, opts->charge_col,
                 opts->force_schedule, opts->max_event_hint, centroid_idx, token_id,
                 opts->assign_mode == FPS_ASSIGN_KNN ? knn_idx : nullptr,
-                reinterpret_cast<float4*>(centroids), pooled, counts};
+                reinterpret_cast<float4*>(centroids), pooled, counts, 0};
+  if (opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0) {
+    const size_t K = (size_t)opts->K, Fz = (size_t)F;
+    if (K * Fz * sizeof(double) + K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
+    if ((size_t)(3 * kCtaCap + 768) * sizeof(int) + (size_t)kCtaCap * Fz * sizeof(float) +
+            K * Fz * sizeof(double) <= cta_region_bytes())
+      pb.fused_pool |= 2;
+  }
   return run_tokenize(pb, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 

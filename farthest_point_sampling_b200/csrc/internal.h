@@ -23,6 +23,7 @@ enum ListId : int {
   kNumLists = 9,
 };
 constexpr int kNumSchedules = 5;  // warp, CTA, CTA-smem, 8-CTA cluster, 16-CTA cluster
+constexpr int kStagePassthrough = 9;  // stage id of the passthrough kernel (helper stream)
 
 // Schedule capacities (points per event).
 constexpr int kWarpPairs = 7;                          // point pairs per lane, warp schedule
@@ -30,6 +31,7 @@ constexpr int kWarpCap = 64 * kWarpPairs;              // 448
 constexpr int kCtaThreads = 256;                       // register-resident CTA schedule
 constexpr int kCtaPairs = 5;                           // pairs per thread
 constexpr int kCtaCap = 2 * kCtaThreads * kCtaPairs;   // 2560
+constexpr size_t kCtaSmemBytes = 104 * 1024;           // register-CTA shared memory (event copy / pooling)
 constexpr int kBlockThreads = 256;                     // shared-memory CTA / cluster schedules
 constexpr int kBlockPairs = 24;                        // pairs per thread in shared memory
 constexpr int kCtaSmemCap = kBlockThreads * 2 * kBlockPairs;  // 12288
@@ -79,6 +81,7 @@ struct Problem {
   float4* centroids;
   float* pooled;
   int32_t* counts;
+  int fused_pool;  // bit 0 / bit 1: the warp / register-CTA FPS kernels pool their own events
 };
 
 // Kernel launchers (return the cudaError_t of the launch).
@@ -86,7 +89,13 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
 cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s);
 typedef void (*StageMark)(int stage, int end, cudaStream_t s);
 void stage_mark(int stage, int end, cudaStream_t s);
-cudaError_t launch_fps(const Problem& pb, const Workspace& ws, cudaStream_t s, StageMark mark);
+// FPS schedules plus the passthrough kernel (`pt`), all concurrent after the
+// binning kernel; returns once the work is enqueued and joined into `s`.
+cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws, cudaStream_t s, StageMark mark);
+// Bytes of shared memory of the warp-schedule event copy (per warp) and of
+// the register-CTA schedule (per CTA): fused pooling must fit into them.
+size_t warp_region_bytes();
+size_t cta_region_bytes();
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s);
 cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,

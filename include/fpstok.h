@@ -229,11 +229,11 @@ uint64_t fps_launch_count(void);
  * Measurement hook: when `events` is non-NULL the next calls record
  * events[2*s] before and events[2*s+1] after internal stage s on the
  * launching stream (the block schedules run on internal helper streams forked
- * from it; their events are recorded there).  Stages: 0 binning +
- * passthrough, 1 FPS warp schedule, 2 FPS CTA schedule, 3 FPS CTA
- * shared-memory schedule, 4 FPS 8-CTA cluster, 5 FPS 16-CTA cluster, 6 Lloyd,
- * 7 kNN gather + pool, 8 Voronoi pool.  A stage that does not run records
- * nothing.  The events are cudaEvent_t handles the caller created; at most 32
+ * from it; their events are recorded there).  Stages: 0 binning, 1 FPS warp
+ * schedule, 2 FPS CTA schedule, 3 FPS CTA shared-memory schedule, 4 FPS 8-CTA
+ * cluster, 5 FPS 16-CTA cluster, 6 Lloyd, 7 kNN gather + pool, 8 Voronoi pool
+ * (events not pooled by their FPS kernel), 9 passthrough.  A stage that does
+ * not run records nothing.  The events are cudaEvent_t handles the caller created; at most 32
  * are used.  Pass NULL to turn it off.  Not thread-safe: meant for benchmarks.
  */
 void fps_set_stage_events(void *const *events, int n_events);
