@@ -64,12 +64,27 @@ struct PoolOut {
   int32_t* counts;
 };
 
+// Asks L2 to fetch the event's feature rows [lo, lo + bytes) while the FPS
+// loop runs, so that the pooling at its end reads them from L2.  The range
+// is shrunk inward to 16-byte boundaries (it never leaves the rows) and
+// split into 16 KiB bulk prefetches, one per calling `part` < nparts.
+__device__ __forceinline__ void prefetch_rows_l2(const float* lo, size_t bytes, int part, int nparts) {
+  uintptr_t a = (reinterpret_cast<uintptr_t>(lo) + 15) & ~(uintptr_t)15;
+  const uintptr_t end = (reinterpret_cast<uintptr_t>(lo) + bytes) & ~(uintptr_t)15;
+  constexpr uintptr_t kPiece = 16384;
+  for (uintptr_t p = a + (uintptr_t)part * kPiece; p < end; p += (uintptr_t)nparts * kPiece) {
+    const uint32_t len = (uint32_t)((end - p) < kPiece ? (end - p) : kPiece);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(len) : "memory");
+  }
+}
+
 // One FPS event on one warp, NP point pairs per lane.
 template <int NP>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                            int lane, DupPoint* s_dup, int32_t* __restrict__ cidx,
                                            float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
                                            const PoolOut& po) {
+  if (po.feats && lane < 4) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), lane, 4);
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -219,6 +234,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
                                           const PoolOut& po) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (po.feats && tid < 32) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), tid, 32);
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -312,7 +328,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       if (i < n) s_lab[i] = lab[j];
     }
     const float* fe = po.feats + off * F;
-#pragma unroll 4
+#pragma unroll 16
     for (int e = tid; e < n * F; e += NT) s_feat[e] = __ldg(fe + e);
     for (int e = tid; e < K * F; e += NT) acc[e] = 0.0;
     label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, slab, tid, NT, [] { __syncthreads(); });
@@ -647,7 +663,7 @@ static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list
 
 // Per-device state: occupancy figures and the helper streams / events that
 // let the schedules run concurrently.
-constexpr int kHelpers = kNumSchedules;  // four block schedules and the passthrough kernel
+constexpr int kHelpers = kNumSchedules + 1;  // one per schedule (high priority) and the passthrough kernel
 struct DeviceCtx {
   DeviceInfo info;
   cudaStream_t helper[kHelpers];
@@ -689,8 +705,13 @@ static cudaError_t prepare(int dev) {
   if ((e = prepare_block_kernel<8>(&info.cluster8_max_active)) != cudaSuccess) return e;
   if ((e = prepare_block_kernel<16>(&info.cluster16_max_active)) != cudaSuccess) return e;
   if ((e = prepare_aux_kernels()) != cudaSuccess) return e;
+  // FPS schedules (the critical path) on the highest priority, the passthrough
+  // kernel (which only has to finish before pooling) on the lowest
+  int least = 0, greatest = 0;
+  if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest))) return e;
   for (int i = 0; i < kHelpers; ++i) {
-    if ((e = cudaStreamCreateWithFlags(&ctx.helper[i], cudaStreamNonBlocking))) return e;
+    const int prio = i == kHelpers - 1 ? least : greatest;
+    if ((e = cudaStreamCreateWithPriority(&ctx.helper[i], cudaStreamNonBlocking, prio))) return e;
     if ((e = cudaEventCreateWithFlags(&ctx.join[i], cudaEventDisableTiming))) return e;
   }
   if ((e = cudaEventCreateWithFlags(&ctx.fork, cudaEventDisableTiming))) return e;
@@ -737,20 +758,21 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
 
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
   if ((e = cudaEventRecord(ctx.fork, s))) return e;
-  {  // passthrough rows and accumulator clearing overlap the FPS kernels
-    cudaStream_t hs = ctx.helper[kHelpers - 1];
-    if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
-    mark(kStagePassthrough, 0, hs);
-    if ((e = launch_passthrough(pt, ws, hs))) return e;
-    mark(kStagePassthrough, 1, hs);
-    if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;
-  }
-  for (int q = 1; q < kNumSchedules; ++q) {
+  for (int q = 0; q < kNumSchedules; ++q) {
     if (!run[q]) continue;
-    cudaStream_t hs = ctx.helper[q - 1];
+    cudaStream_t hs = ctx.helper[q];
     if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
     mark(1 + q, 0, hs);
     switch (q) {
+      case 0: {
+        const int blocks = di.sm_count * (di.warp_blocks_per_sm > 0 ? di.warp_blocks_per_sm : 1);
+        count_launch();
+        k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, hs>>>(pb.coords, pb.offsets, pb.start_local,
+                                                                      ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
+                                                                      pb.token_id, pb.centroids, po_warp);
+        e = cudaGetLastError();
+        break;
+      }
       case 1:
         count_launch();
         k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
@@ -770,20 +792,18 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     }
     if (e != cudaSuccess) return e;
     mark(1 + q, 1, hs);
-    if ((e = cudaEventRecord(ctx.join[q - 1], hs))) return e;
+    if ((e = cudaEventRecord(ctx.join[q], hs))) return e;
   }
-  if (run[0]) {
-    const int blocks = di.sm_count * (di.warp_blocks_per_sm > 0 ? di.warp_blocks_per_sm : 1);
-    mark(1, 0, s);
-    count_launch();
-    k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, s>>>(pb.coords, pb.offsets, pb.start_local,
-                                                                 ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                 pb.token_id, pb.centroids, po_warp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    mark(1, 1, s);
+  {  // passthrough rows and accumulator clearing overlap the FPS kernels (enqueued last, lowest priority)
+    cudaStream_t hs = ctx.helper[kHelpers - 1];
+    if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
+    mark(kStagePassthrough, 0, hs);
+    if ((e = launch_passthrough(pt, ws, hs))) return e;
+    mark(kStagePassthrough, 1, hs);
+    if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;
   }
-  for (int q = 1; q < kNumSchedules; ++q)
-    if (run[q] && (e = cudaStreamWaitEvent(s, ctx.join[q - 1], 0))) return e;
+  for (int q = 0; q < kNumSchedules; ++q)
+    if (run[q] && (e = cudaStreamWaitEvent(s, ctx.join[q], 0))) return e;
   return cudaStreamWaitEvent(s, ctx.join[kHelpers - 1], 0);
 }
 
