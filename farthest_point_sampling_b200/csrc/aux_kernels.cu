@@ -287,8 +287,7 @@ __device__ __forceinline__ void chunk_token_sums(const SortSmem& sm, int npts, i
   label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, sm.slab, tid, T, cta_sync);
   int nsorted = 0;
   if (K > 0) nsorted = sm.start[K - 1] + sm.cnt[K - 1];
-  for (int v0 = 0; v0 < V; v0 += 8)
-    segment_sums(sm.perm, sm.slab, nsorted, min(8, V - v0), v0, V, acc, tid, T, val);
+  segment_sums(sm.perm, sm.slab, nsorted, V, 0, V, acc, tid, T, val);
   __syncthreads();
 }
 
@@ -343,8 +342,7 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
       for (int e = tid; e < K * F; e += T) acc[e] = 0.0;
       __syncthreads();
       const int nsorted = sm.start[K - 1] + sm.cnt[K - 1];
-      for (int v0 = 0; v0 < F; v0 += 8)
-        segment_sums(sm.perm, sm.slab, nsorted, min(8, F - v0), v0, F, acc, tid, T, val);
+      segment_sums(sm.perm, sm.slab, nsorted, F, 0, F, acc, tid, T, val);
     } else if (tid < K) {  // one thread per token: its (short) run, in sorted order
       const int* pj = sm.perm + sm.start[tid];
       for (int f0 = 0; f0 < F; f0 += 8) {

@@ -204,39 +204,38 @@ __device__ __forceinline__ void label_sort(const int* lab, int npts, int K, int*
 }
 
 // Per-token float64 sums over the first nsorted positions of a counting
-// sort, balanced over the group: every thread takes an equal run of sorted
-// positions, adds val(i, v) for v < V along it and flushes its partial sums
-// into acc[token * V + v] (shared memory, zeroed beforehand) whenever the
-// token changes and at the end of its run.  V <= 8 per call.
+// sort: each warp of the group takes tiles of 32 consecutive sorted
+// positions, forms a segmented inclusive scan of val(i, v) over the lanes of
+// each token with shuffles, and the last lane of every token in the tile adds
+// the tile's partial sum into acc[token * ldacc + v] (shared memory, zeroed
+// beforehand).  A token therefore gets one atomic per tile it spans, not one
+// per point.  The group size is a multiple of 32; v runs over [v0, v0 + V).
 template <typename Val>
 __device__ __forceinline__ void segment_sums(const int* perm, const int* slab, int nsorted, int V, int v0,
                                              int ldacc, double* acc, int rank, int size, Val val) {
-  const int per = (nsorted + size - 1) / size;
-  const int p0 = rank * per, p1 = min(nsorted, p0 + per);
-  if (p0 >= p1) return;
-  double s[8];
+  const int lane = rank & 31, warp = rank >> 5, nwarps = size >> 5;
+  for (int tile = warp * 32; tile < nsorted; tile += nwarps * 32) {
+    const int q = tile + lane;
+    const bool valid = q < nsorted;
+    const int tok = valid ? slab[q] : -1 - lane;  // empty lanes form singleton segments
+    const int i = valid ? perm[q] : 0;
+    const bool last = valid && (lane == 31 || __shfl_down_sync(kFull, tok, 1) != tok);
+    bool same[5];
 #pragma unroll
-  for (int v = 0; v < 8; ++v) s[v] = 0.0;
-  int cur = slab[p0];
-  for (int q = p0; q < p1; ++q) {
-    const int i = perm[q];
-    const int l = slab[q];
-    if (l != cur) {
-#pragma unroll
-      for (int v = 0; v < 8; ++v)
-        if (v < V) {
-          atomicAdd(&acc[cur * ldacc + v0 + v], s[v]);
-          s[v] = 0.0;
-        }
-      cur = l;
+    for (int k = 0; k < 5; ++k) {
+      const int o = 1 << k;
+      same[k] = lane >= o && __shfl_up_sync(kFull, tok, o) == tok;
     }
+    for (int v = 0; v < V; ++v) {
+      double x = valid ? val(i, v0 + v) : 0.0;
 #pragma unroll
-    for (int v = 0; v < 8; ++v)
-      if (v < V) s[v] += val(i, v0 + v);
+      for (int k = 0; k < 5; ++k) {
+        const double y = __shfl_up_sync(kFull, x, 1 << k);
+        if (same[k]) x += y;
+      }
+      if (last) atomicAdd(&acc[tok * ldacc + v0 + v], x);
+    }
   }
-#pragma unroll
-  for (int v = 0; v < 8; ++v)
-    if (v < V) atomicAdd(&acc[cur * ldacc + v0 + v], s[v]);
 }
 
 }  // namespace fpstok

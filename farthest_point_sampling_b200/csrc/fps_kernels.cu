@@ -332,9 +332,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     for (int e = tid; e < n * F; e += NT) s_feat[e] = __ldg(fe + e);
     for (int e = tid; e < K * F; e += NT) acc[e] = 0.0;
     label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, slab, tid, NT, [] { __syncthreads(); });
-    for (int v0 = 0; v0 < F; v0 += 8)
-      segment_sums(perm, slab, n, min(8, F - v0), v0, F, acc, tid, NT,
-                   [&](int i, int f) { return (double)s_feat[i * F + f]; });
+    segment_sums(perm, slab, n, F, 0, F, acc, tid, NT, [&](int i, int f) { return (double)s_feat[i * F + f]; });
     __syncthreads();
     for (int j = tid; j < K; j += NT) {
       const int c = cnt[j];
