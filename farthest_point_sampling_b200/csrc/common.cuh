@@ -219,12 +219,15 @@ __device__ __forceinline__ void segment_sums(const int* perm, const int* slab, i
     const bool valid = q < nsorted;
     const int tok = valid ? slab[q] : -1 - lane;  // empty lanes form singleton segments
     const int i = valid ? perm[q] : 0;
-    const bool last = valid && (lane == 31 || __shfl_down_sync(kFull, tok, 1) != tok);
+    // every lane takes part in every shuffle: none sits behind a short-circuit
+    const int next_tok = __shfl_down_sync(kFull, tok, 1);
+    const bool last = valid && (lane == 31 || next_tok != tok);
     bool same[5];
 #pragma unroll
     for (int k = 0; k < 5; ++k) {
       const int o = 1 << k;
-      same[k] = lane >= o && __shfl_up_sync(kFull, tok, o) == tok;
+      const int up_tok = __shfl_up_sync(kFull, tok, o);
+      same[k] = lane >= o && up_tok == tok;
     }
     for (int v = 0; v < V; ++v) {
       double x = valid ? val(i, v0 + v) : 0.0;
