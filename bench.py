@@ -37,7 +37,7 @@ import workloads  # noqa: E402
 FP32_OPS_PER_EVAL = 11  # 4 sub + 4 mul + 3 add
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
-FP32_OPS_PER_LANE_CLK = 2  # packed f32x2 add/sub/mul: two float32 operations per lane per clock
+FP32_OPS_PER_LANE_CLK = 1  # nominal fallback only: one non-FMA float32 op per lane per clock
 SM_MAX_MHZ_NOMINAL = 1965.0
 STAGES = ["bin", "fps_warp", "fps_cta", "fps_cta_smem", "fps_cluster8", "fps_cluster16", "lloyd",
           "knn+pool", "voronoi_pool", "passthrough"]
@@ -443,13 +443,19 @@ def main():
         # roofline of the dominant kernel (FP32 issue bound for the FPS kernels)
         dom = max(stage_ms, key=stage_ms.get)
         t_dom = stage_ms[dom] / 1e3
-        peak = SM_COUNT * FP32_LANES_PER_SM * FP32_OPS_PER_LANE_CLK * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
+        mb = None if args.no_microbench else microbench_fp32(dev)
+        if mb and mb.get("non_fma_peak"):
+            peak = mb["non_fma_peak"]
+            peak_source = "measured in this run: best non-FMA FP32 chain rate (microbench, see microbench_fp32_tflops)"
+        else:
+            peak = SM_COUNT * FP32_LANES_PER_SM * FP32_OPS_PER_LANE_CLK * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
+            peak_source = "derived: 148 SMs x 128 FP32 lanes x 1 op x 1965 MHz (non-FMA float32 ops)"
         if dom in FPS_STAGES:
             ev = int(sum(int(n) * batch.K for n, s in zip(sizes, sched) if s == dom - 1))
             achieved = ev * FP32_OPS_PER_EVAL / t_dom / 1e12
             roof = {"bound": "alu", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 (f32x2) x 1965 MHz, non-FMA float32 ops",
+                    "peak_source": peak_source,
                     "algorithmic": f"{ev} point-centroid evals x {FP32_OPS_PER_EVAL} FP32 ops per launch",
                     "traffic": recorded_traffic(dom, args.workload)}
         else:
@@ -462,8 +468,8 @@ def main():
             achieved = byts / t_dom / 1e9
             roof = {"bound": "hbm", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": hbm,
                     "unit": "GB/s", "frac": achieved / hbm, "traffic": recorded_traffic(dom, args.workload)}
-        if not args.no_microbench:
-            roof["microbench_fp32_tflops"] = microbench_fp32(dev)
+        if mb:
+            roof["microbench_fp32_tflops"] = mb
         result["roofline"] = roof
         result["clocks"] = clocks.summary()
         if not args.no_e2e:
@@ -479,8 +485,16 @@ def main():
     return 0
 
 
+MICROBENCH_MODES = {0: "scalar_fmul_fadd", 1: "f32x2_add", 2: "f32x2_mul", 3: "f32x2_fma", 4: "f32x2_distance"}
+
+
 def microbench_fp32(dev):
-    """Best measured non-FMA FP32 op rate (TFLOP/s) of scalar and f32x2 chains."""
+    """Measured FP32 rates (TFLOP/s, an FMA counted as two) of the microbenchmark modes.
+
+    The non-FMA peak is the best of the scalar and the separate packed add and
+    multiply chains; "f32x2_distance" is the rate of the distance exactly as
+    the FPS kernels compute it.
+    """
     import ctypes
 
     import torch
@@ -495,20 +509,23 @@ def microbench_fp32(dev):
     out = torch.empty(blocks, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     best = {}
-    for packed in (0, 1):
+    for mode, name in MICROBENCH_MODES.items():
         rates = []
         for _ in range(4):
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+            a.record(stream)  # creates the underlying events
             b.record(stream)
             torch.cuda.synchronize(dev)
-            ops = lib.fpstok_microbench_fp32(packed, blocks, 256, 4096, ctypes.c_void_p(out.data_ptr()),
+            ops = lib.fpstok_microbench_fp32(mode, blocks, 256, 2048, ctypes.c_void_p(out.data_ptr()),
                                              ctypes.c_void_p(a.cuda_event), ctypes.c_void_p(b.cuda_event),
                                              ctypes.c_void_p(stream.cuda_stream))
             torch.cuda.synchronize(dev)
-            rates.append(ops / (a.elapsed_time(b) / 1e3) / 1e12)
-        best["f32x2" if packed else "scalar"] = max(rates)
+            if ops > 0:
+                rates.append(ops / (a.elapsed_time(b) / 1e3) / 1e12)
+        best[name] = max(rates) if rates else None
+    vals = [best[k] for k in ("scalar_fmul_fadd", "f32x2_add", "f32x2_mul") if best.get(k)]
+    best["non_fma_peak"] = max(vals) if vals else None
     return best
 
 

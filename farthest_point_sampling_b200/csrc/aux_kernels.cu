@@ -287,7 +287,8 @@ __device__ __forceinline__ void chunk_token_sums(const SortSmem& sm, int npts, i
   label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, sm.slab, tid, T, cta_sync);
   int nsorted = 0;
   if (K > 0) nsorted = sm.start[K - 1] + sm.cnt[K - 1];
-  segment_sums(sm.perm, sm.slab, nsorted, V, 0, V, acc, tid, T, val);
+  for (int v0 = 0; v0 < V; v0 += 8)
+    segment_sums(sm.perm, sm.slab, nsorted, min(8, V - v0), v0, V, acc, tid, T, val);
   __syncthreads();
 }
 
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
       for (int e = tid; e < K * F; e += T) acc[e] = 0.0;
       __syncthreads();
       const int nsorted = sm.start[K - 1] + sm.cnt[K - 1];
-      segment_sums(sm.perm, sm.slab, nsorted, F, 0, F, acc, tid, T, val);
+      segment_sums_scan(sm.perm, sm.slab, nsorted, F, 0, F, acc, tid, T, val);
     } else if (tid < K) {  // one thread per token: its (short) run, in sorted order
       const int* pj = sm.perm + sm.start[tid];
       for (int f0 = 0; f0 < F; f0 += 8) {
@@ -408,68 +409,107 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
 
 // ------------------------------------------------------------------ nearest centroid
 
-// Centroids of one event in shared memory, broadcast into packed pairs.
-__device__ __forceinline__ void load_cents(const float4* __restrict__ c, int nv, Cent2* s) {
-  for (int j = threadIdx.x; j < nv; j += blockDim.x) s[j] = cent2(c[j]);
+// Centroid slots padded to a whole number of pairs; the pad holds +inf
+// coordinates, whose distance to any finite point is +inf.
+__host__ __device__ constexpr int pad_pairs(int nv) { return (nv + 1) & ~1; }
+
+__device__ __forceinline__ void load_cents_padded(const float4* __restrict__ c, int nv, Cent2* s) {
+  const float inf = __int_as_float(0x7f800000);
+  for (int j = threadIdx.x; j < pad_pairs(nv); j += blockDim.x)
+    s[j] = cent2(j < nv ? c[j] : make_float4(inf, inf, inf, inf));
 }
 
-// Nearest of the first nv shared-memory centroids for points [i0, i1) of an
-// event (thread-strided, two points per packed evaluation); strict '<' over
-// increasing slots keeps the lowest slot on ties.  Calls emit(i, label, p)
-// once per point p.
-template <int PAIRS, typename Emit>
-__device__ __forceinline__ void nearest_pass(const float4* __restrict__ pts, int i0, int i1,
-                                             const Cent2* __restrict__ cs, int nv, Emit emit) {
-  const int T = blockDim.x;
-  for (int base = i0; base < i1; base += 2 * PAIRS * T) {
-    uint64_t X[PAIRS], Y[PAIRS], Z[PAIRS], W[PAIRS];
-    float best[2 * PAIRS];
-    int lab[2 * PAIRS];
+// Nearest centroid of this thread's 2 PR points (PR packed pairs) among the
+// centroid pairs cs[0 .. 2 ng) (pads +inf).  The loop keeps, per point, the
+// smallest distance and the pair g of centroids holding it: one three-input
+// minimum, one compare and one select per point and pair of centroids, the
+// strict '<' keeping the earliest pair on ties.  The slot inside the winning
+// pair is then 2 g when the recomputed distance to centroid 2 g equals the
+// minimum, else 2 g + 1.  Both passes evaluate the same float32 distance, so
+// the result is exactly the lowest-slot nearest centroid.
+template <int PR>
+__device__ __forceinline__ void nearest_pairs(const uint64_t (&X)[PR], const uint64_t (&Y)[PR],
+                                              const uint64_t (&Z)[PR], const uint64_t (&W)[PR],
+                                              const Cent2* __restrict__ cs, int ng, int (&lab)[2 * PR]) {
+  const uint64_t z2 = opaque_zero2();
+  float best[2 * PR];
 #pragma unroll
-    for (int p = 0; p < PAIRS; ++p) {
-      const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
+  for (int r = 0; r < 2 * PR; ++r) {
+    best[r] = __int_as_float(0x7f800000);
+    lab[r] = 0;
+  }
+#pragma unroll 1
+  for (int g = 0; g < ng; ++g) {
+    const Cent2 A = cs[2 * g], B = cs[2 * g + 1];
+#pragma unroll
+    for (int p = 0; p < PR; ++p) {
+      const uint64_t da = dist2(X[p], Y[p], Z[p], W[p], A, z2);
+      const uint64_t db = dist2(X[p], Y[p], Z[p], W[p], B, z2);
+      const float m0 = min3f(best[2 * p], lo2(da), lo2(db));
+      const float m1 = min3f(best[2 * p + 1], hi2(da), hi2(db));
+      lab[2 * p] = m0 < best[2 * p] ? g : lab[2 * p];
+      lab[2 * p + 1] = m1 < best[2 * p + 1] ? g : lab[2 * p + 1];
+      best[2 * p] = m0;
+      best[2 * p + 1] = m1;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2 * PR; ++r) {
+    const int p = r >> 1;
+    const float4 q = (r & 1) ? make_float4(hi2(X[p]), hi2(Y[p]), hi2(Z[p]), hi2(W[p]))
+                             : make_float4(lo2(X[p]), lo2(Y[p]), lo2(Z[p]), lo2(W[p]));
+    const Cent2 c = cs[2 * lab[r]];
+    const float d = dist1(q, make_float4(lo2(c.x), lo2(c.y), lo2(c.z), lo2(c.t)));
+    lab[r] = 2 * lab[r] + (d == best[r] ? 0 : 1);
+  }
+}
+
+// Nearest centroid of the chunk points tid + r T (r < 2 PR NPASS) of
+// `pts` (npts valid), in NPASS passes of PR pairs; emit(li, label) is called
+// for every valid local point li at the end of its pass.
+template <int PR, int NPASS, int T, typename Emit>
+__device__ __forceinline__ void chunk_nearest(const float4* __restrict__ pts, int npts,
+                                              const Cent2* __restrict__ cs, int ng, Emit emit) {
+  const int tid = threadIdx.x;
+#pragma unroll 1
+  for (int q = 0; q < NPASS; ++q) {
+    uint64_t X[PR], Y[PR], Z[PR], W[PR];
+#pragma unroll
+    for (int p = 0; p < PR; ++p) {
+      const int ia = tid + (2 * PR * q + 2 * p) * T, ib = ia + T;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-      if (ia < i1) a = ldg4(pts + ia);
-      if (ib < i1) c = ldg4(pts + ib);
+      if (ia < npts) a = ldg4(pts + ia);
+      if (ib < npts) c = ldg4(pts + ib);
       X[p] = pack2(a.x, c.x);
       Y[p] = pack2(a.y, c.y);
       Z[p] = pack2(a.z, c.z);
       W[p] = pack2(a.w, c.w);
-      best[2 * p] = best[2 * p + 1] = __int_as_float(0x7f800000);
-      lab[2 * p] = lab[2 * p + 1] = -1;
     }
-    for (int j = 0; j < nv; ++j) {
-      const Cent2 C = cs[j];
+    int l[2 * PR];
+    nearest_pairs<PR>(X, Y, Z, W, cs, ng, l);
 #pragma unroll
-      for (int p = 0; p < PAIRS; ++p) {
-        const uint64_t d = dist2(X[p], Y[p], Z[p], W[p], C);
-        relax(lo2(d), best[2 * p], lab[2 * p], j);
-        relax(hi2(d), best[2 * p + 1], lab[2 * p + 1], j);
-      }
-    }
-#pragma unroll
-    for (int p = 0; p < PAIRS; ++p) {
-      const int ia = base + threadIdx.x + (2 * p) * T, ib = ia + T;
-      if (ia < i1)
-        emit(ia, nv > 0 ? (lab[2 * p] < 0 ? 0 : lab[2 * p]) : -1,
-             make_float4(lo2(X[p]), lo2(Y[p]), lo2(Z[p]), lo2(W[p])));
-      if (ib < i1)
-        emit(ib, nv > 0 ? (lab[2 * p + 1] < 0 ? 0 : lab[2 * p + 1]) : -1,
-             make_float4(hi2(X[p]), hi2(Y[p]), hi2(Z[p]), hi2(W[p])));
+    for (int r = 0; r < 2 * PR; ++r) {
+      const int li = tid + (2 * PR * q + r) * T;
+      if (li < npts) emit(li, l[r]);
     }
   }
 }
 
-constexpr int kAssignPairs = 4;
-constexpr int kLloydPairs = 2;
+constexpr int kNearestPairs = 2;  // pairs per pass: with two centroids in flight, 8 distance chains
+constexpr int kNearestPasses = kChunk / (2 * kNearestPairs * 256);
+static_assert(kNearestPasses * 2 * kNearestPairs * 256 == kChunk, "whole passes per chunk");
 
 // Standalone nearest-centroid assignment over (event, chunk) items.
-__global__ void __launch_bounds__(256) k_assign(const float4* __restrict__ coords,
-                                                const int64_t* __restrict__ offsets, int K,
-                                                const float4* __restrict__ centroids,
-                                                const int32_t* __restrict__ valid,
-                                                int32_t* __restrict__ token_id, Workspace ws) {
-  extern __shared__ Cent2 s_cent[];
+constexpr int kAssignThreads = 256;
+
+__global__ void __launch_bounds__(kAssignThreads, 3) k_assign(const float4* __restrict__ coords,
+                                                           const int64_t* __restrict__ offsets, int K,
+                                                           const float4* __restrict__ centroids,
+                                                           const int32_t* __restrict__ valid,
+                                                           int32_t* __restrict__ token_id, Workspace ws) {
+  constexpr int T = kAssignThreads;
+  extern __shared__ Cent2 s_cent[];  // [pad_pairs(K)]
+  const int tid = threadIdx.x;
   const int nitems = ws.hdr->n_items[kListChunks];
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
     const int2 it = ws.chunks[item];
@@ -481,11 +521,12 @@ __global__ void __launch_bounds__(256) k_assign(const float4* __restrict__ coord
       record_error(ws.hdr, kDevBadToken);
       nv = 0;
     }
-    load_cents(centroids + (int64_t)b * K, nv, s_cent);
+    load_cents_padded(centroids + (int64_t)b * K, nv, s_cent);
     __syncthreads();
-    const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
-    int32_t* out = token_id + off;
-    nearest_pass<kAssignPairs>(coords + off, i0, i1, s_cent, nv, [&](int i, int l, float4) { out[i] = l; });
+    const int i0 = it.y * kChunk, npts = min(n, i0 + kChunk) - i0;
+    int32_t* out = token_id + off + i0;
+    chunk_nearest<kNearestPairs, kNearestPasses, T>(coords + off + i0, npts, s_cent, pad_pairs(nv) / 2,
+                                                    [&](int li, int l) { out[li] = nv > 0 ? l : -1; });
     __syncthreads();
   }
 }
@@ -552,34 +593,53 @@ __global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ c
   }
 }
 
-// One Lloyd iteration: centroids from the sums `in`, re-assign the chunk and
-// (unless last) accumulate the next sums into `next`; clears `clear`.
-__global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict__ coords,
-                                                       const float* __restrict__ feats, int F,
-                                                       int charge_col, const int64_t* __restrict__ offsets,
-                                                       int K, int32_t* __restrict__ labels,
-                                                       float4* __restrict__ centroids, Workspace ws,
-                                                       const double* __restrict__ in, double* __restrict__ next,
-                                                       double* __restrict__ clear, int64_t clear_n) {
+// One Lloyd iteration per (event, chunk) item: the centroids from the cell
+// sums `in` (an empty cell or a zero weight keeps its centroid), the nearest
+// of them for the chunk's points (eight per thread, in two passes) and,
+// unless this is the last iteration (next == nullptr), the chunk's cell sums
+// of the new labels added into `next`.  Also clears `clear`, which the
+// following iteration accumulates into.
+constexpr int kLloydThreads = 256;
+constexpr int kLloydPts = kChunk / kLloydThreads;  // points per thread
+static_assert(kLloydPts == 2 * kNearestPairs * kNearestPasses, "chunk_nearest covers the chunk");
+
+static size_t lloyd_step_smem_bytes(int K) {
+  return (size_t)(2 * kChunk + 3 * 256) * sizeof(int) + (size_t)kChunk * (sizeof(float4) + sizeof(float)) +
+         (size_t)K * 5 * sizeof(double) + (size_t)pad_pairs(K) * sizeof(Cent2);
+}
+
+__global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* __restrict__ coords,
+                                                                 const float* __restrict__ feats, int F,
+                                                                 int charge_col,
+                                                                 const int64_t* __restrict__ offsets, int K,
+                                                                 int32_t* __restrict__ labels,
+                                                                 float4* __restrict__ centroids, Workspace ws,
+                                                                 const double* __restrict__ in,
+                                                                 double* __restrict__ next,
+                                                                 double* __restrict__ clear, int64_t clear_n) {
+  constexpr int T = kLloydThreads;
   extern __shared__ int smem_i[];
-  const SortSmem sm = sort_smem(smem_i, kChunk);
-  float4* s_p = reinterpret_cast<float4*>(smem_i + 3 * kChunk + 3 * 256);
-  float* s_q = reinterpret_cast<float*>(s_p + kChunk);
+  int* perm = smem_i;              // [kChunk]
+  int* slab = perm + kChunk;       // [kChunk]
+  int* cnt = slab + kChunk;        // [256]
+  int* start = cnt + 256;          // [256]
+  int* cur = start + 256;          // [256]
+  float4* s_p = reinterpret_cast<float4*>(cur + 256);  // [kChunk]
+  float* s_q = reinterpret_cast<float*>(s_p + kChunk);  // [kChunk]
   double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]
-  Cent2* s_cent = reinterpret_cast<Cent2*>(acc + 256 * 5);  // [K]
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < clear_n;
-       e += (int64_t)gridDim.x * blockDim.x)
-    clear[e] = 0.0;
+  Cent2* s_cent = reinterpret_cast<Cent2*>(acc + K * 5);  // [K]
+  const int tid = threadIdx.x;
+  for (int64_t e = (int64_t)blockIdx.x * T + tid; e < clear_n; e += (int64_t)gridDim.x * T) clear[e] = 0.0;
   const int nitems = ws.hdr->n_items[kListChunks];
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
     const int2 it = ws.chunks[item];
     const int b = it.x;
     const int fs = ws.fps_slot[b];
-    if (fs < 0) continue;
+    if (fs < 0) continue;  // uniform across the CTA
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
     const double* sb = in + (int64_t)fs * K * 5;
-    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+    for (int j = tid; j < K; j += T) {
       const double W = __ldcg(&sb[j * 5]);
       float4 c = centroids[(int64_t)b * K + j];
       if (W > 0.0) {
@@ -589,52 +649,81 @@ __global__ void __launch_bounds__(256, 2) k_lloyd_step(const float4* __restrict_
         c.w = (float)(__ldcg(&sb[j * 5 + 4]) / W);
       }
       s_cent[j] = cent2(c);
-      if (it.y == 0) centroids[(int64_t)b * K + j] = c;
+      if (it.y == 0) centroids[(int64_t)b * K + j] = c;  // every chunk computes the same values
+    }
+    if (tid == 0 && (K & 1)) {
+      const float inf = __int_as_float(0x7f800000);
+      s_cent[K] = cent2(make_float4(inf, inf, inf, inf));
+    }
+    if (next) {
+      for (int j = tid; j < K; j += T) cnt[j] = 0;
+      for (int e = tid; e < K * 5; e += T) acc[e] = 0.0;
     }
     __syncthreads();
-    const int i0 = it.y * kChunk, i1 = min(n, i0 + kChunk);
-    int32_t* lab = labels + off;
-    const float4* pts = coords + off;
-    const float* fe = feats ? feats + off * F : nullptr;
-    nearest_pass<kLloydPairs>(pts, i0, i1, s_cent, K, [&](int i, int l, float4 p) {
-      lab[i] = l;
+    const int i0 = it.y * kChunk, npts = min(n, i0 + kChunk) - i0;
+    const float4* pts = coords + off + i0;
+    int32_t* lab_out = labels + off + i0;
+    const float* fe = feats ? feats + (off + i0) * F : nullptr;
+    chunk_nearest<kNearestPairs, kNearestPasses, T>(pts, npts, s_cent, pad_pairs(K) / 2, [&](int li, int l) {
+      lab_out[li] = l;
       if (next) {
-        sm.lab[i - i0] = l;
-        s_p[i - i0] = p;
-        s_q[i - i0] = charge_of(fe, F, charge_col, i);
+        s_p[li] = ldg4(pts + li);  // read a moment ago: a cache hit
+        s_q[li] = charge_of(fe, F, charge_col, li);
+        atomicAdd(&cnt[l], 1);
       }
     });
-    if (next) {
+    if (next) {  // counting sort by label (this thread's own labels, read back), then the cell sums
       __syncthreads();
-      lloyd_chunk_sums(sm, s_p, s_q, i1 - i0, K, acc, next + (int64_t)fs * K * 5);
+      if (tid < 32) count_scan(cnt, start, cur, K, tid);
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < kLloydPts; ++r) {
+        const int li = tid + r * T;
+        if (li < npts) {
+          const int l = lab_out[li];
+          const int pos = atomicAdd(&cur[l], 1);
+          perm[pos] = li;
+          slab[pos] = l;
+        }
+      }
+      __syncthreads();
+      segment_sums(perm, slab, npts, 5, 0, 5, acc, tid, T, [&](int i, int v) {
+        const double q = (double)s_q[i];
+        if (v == 0) return q;
+        const float4 p = s_p[i];
+        return q * (double)(v == 1 ? p.x : (v == 2 ? p.y : (v == 3 ? p.z : p.w)));
+      });
+      __syncthreads();
+      double* out = next + (int64_t)fs * K * 5;
+      for (int e = tid; e < K * 5; e += T)
+        if (cnt[e / 5]) atomicAdd(&out[e], acc[e]);
     }
     __syncthreads();
   }
 }
 
+// Lloyd refinement: cell sums of the incoming labels into buffer 0, then
+// iteration t updates from buffer t % 3, accumulates the next sums into
+// (t + 1) % 3 unless it is the last one, and clears (t + 2) % 3 when
+// iteration t + 1 will accumulate into it (buffers 0 and 1 start zeroed).
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   const int K = pb.K;
-  const int grid = di.sm_count * 4;
-  const size_t sm_sums = kLloydSmemBytes;
-  const size_t sm_step = kLloydSmemBytes + (size_t)K * sizeof(Cent2);
-  cudaError_t e;
   const float* feats = pb.charge_col >= 0 ? pb.feats : nullptr;
-  count_launch();
-  k_lloyd_sums<<<grid, 256, sm_sums, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels,
-                                          ws, ws.lloyd[0]);
-  if ((e = cudaGetLastError())) return e;
-  // iteration t reads buffer t%3, accumulates into (t+1)%3 unless it is the
-  // last one, and clears (t+2)%3 when iteration t+1 will accumulate into it
   const int64_t per = (int64_t)K * 5;
+  cudaError_t e;
+  count_launch();
+  k_lloyd_sums<<<di.sm_count * 2, 256, kLloydSmemBytes, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets,
+                                                             K, labels, ws, ws.lloyd[0]);
+  if ((e = cudaGetLastError())) return e;
+  const size_t sm_step = lloyd_step_smem_bytes(K);
   for (int t = 0; t < pb.lloyd_iters; ++t) {
     const bool last = t == pb.lloyd_iters - 1;
     double* clear = (t + 1 < pb.lloyd_iters - 1) ? ws.lloyd[(t + 2) % 3] : nullptr;
     count_launch();
-    k_lloyd_step<<<grid, 256, sm_step, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K,
-                                            labels, pb.centroids, ws, ws.lloyd[t % 3],
-                                            last ? nullptr : ws.lloyd[(t + 1) % 3], clear,
-                                            clear ? (int64_t)ws.fps_slots * per : 0);
+    k_lloyd_step<<<di.sm_count * 3, kLloydThreads, sm_step, s>>>(
+        pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels, pb.centroids, ws, ws.lloyd[t % 3],
+        last ? nullptr : ws.lloyd[(t + 1) % 3], clear, clear ? (int64_t)ws.fps_slots * per : 0);
     if ((e = cudaGetLastError())) return e;
   }
   return cudaSuccess;
@@ -644,10 +733,10 @@ cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels
 // largest K and F the ABI accepts.
 cudaError_t prepare_aux_kernels() {
   cudaError_t e;
-  const int step_max = (int)(kLloydSmemBytes + 256 * sizeof(Cent2));
   if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLloydSmemBytes)))
     return e;
-  if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize, step_max)))
+  if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)lloyd_step_smem_bytes(256))))
     return e;
   const size_t pool_max = pool_smem_bytes(256, 64) > pool_smem_bytes(256, kStageMaxF)
                               ? pool_smem_bytes(256, 64)
@@ -681,6 +770,59 @@ __device__ __forceinline__ void knn_row_pool(const float* __restrict__ feats, in
   if (lane == 0) *count_out = c;
 }
 
+// Compare-exchange of a bitonic network step across the warp: the lane
+// keeps the smaller key when it is the lower lane of an ascending pair (or
+// the upper lane of a descending one), else the larger.
+__device__ __forceinline__ uint64_t cmpx64(uint64_t v, int lane, int stride, bool ascending) {
+  const uint64_t o = __shfl_xor_sync(kFull, v, stride);
+  const bool keep_min = ((lane & stride) == 0) == ascending;
+  const bool o_less = o < v;
+  return keep_min == o_less ? o : v;
+}
+
+// Ascending bitonic sort of one 64-bit key per lane (lane e ends with the
+// e-th smallest).
+__device__ __forceinline__ uint64_t warp_sort64(uint64_t v, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) v = cmpx64(v, lane, stride, (lane & size) == 0);
+  return v;
+}
+
+// The 32 smallest keys of two ascending warp lists, ascending: the
+// element-wise minimum of one list and the other reversed is a bitonic
+// sequence holding them, which one half-cleaner cascade sorts.
+__device__ __forceinline__ uint64_t warp_merge64(uint64_t a, uint64_t b, int lane) {
+  const uint64_t r = __shfl_sync(kFull, b, 31 - lane);
+  uint64_t v = a < r ? a : r;
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) v = cmpx64(v, lane, stride, true);
+  return v;
+}
+
+// A 32-point chunk with more passing keys than this is sorted and merged
+// into the list at once; fewer are inserted one by one.
+constexpr int kKnnInsertMax = 4;
+
+// Row order of the kNN kernel inside fps_tokenize: the FPS events of the
+// binning kernel's schedule lists, largest schedule first (each list is
+// sorted by decreasing size), so that the longest rows start first.
+struct KnnOrder {
+  const int* list[kNumSchedules];  // list[q] = the list of schedule kNumSchedules - 1 - q
+  int on;
+};
+
+__device__ __forceinline__ int ordered_event(const WsHeader* hdr, const KnnOrder& o, int e) {
+#pragma unroll
+  for (int q = 0; q < kNumSchedules; ++q) {
+    const int nq = hdr->n_items[kNumSchedules - 1 - q];
+    if (e < nq) return o.list[q][e];
+    e -= nq;
+  }
+  return -1;
+}
+
 // One warp per (event, centroid) row: the k smallest (d, index) keys of the
 // event, kept sorted across the warp (element e at lane e % 32, slot e / 32).
 template <int KPL>
@@ -691,15 +833,22 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
                                              int32_t* __restrict__ knn_idx,
                                              const float* __restrict__ feats, int F,
                                              float* __restrict__ pooled, int32_t* __restrict__ counts,
-                                             const int* __restrict__ cls, WsHeader* hdr) {
+                                             KnnOrder ord, WsHeader* hdr) {
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int64_t rows = (int64_t)B * K;
+  int n_ev = B;
+  if (ord.on) {
+    n_ev = 0;
+#pragma unroll
+    for (int q = 0; q < kNumSchedules; ++q) n_ev += hdr->n_items[q];
+  }
+  const int64_t rows = (int64_t)n_ev * K;
   const int kq = (k - 1) >> 5, kl = (k - 1) & 31;
   for (int64_t r = gw; r < rows; r += nw) {
-    const int b = (int)(r / K), j = (int)(r - (int64_t)b * K);
-    if (cls && cls[b] != kClsFps) continue;
+    const int e = (int)(r / K), j = (int)(r - (int64_t)e * K);
+    const int b = ord.on ? ordered_event(hdr, ord, e) : e;
+    const int64_t orow = (int64_t)b * K + j;  // output row
     const int64_t o0 = offsets[b], o1 = offsets[b + 1];
     int n = 0, nv = 0;
     if (o0 >= 0 && o1 >= o0) {
@@ -716,7 +865,7 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
 #pragma unroll
     for (int q = 0; q < KPL; ++q) L[q] = ~0ull;
     if (j < nv) {
-      const float4 c = centroids[r];
+      const float4 c = centroids[orow];
       const float4* pts = coords + o0;
       uint64_t thr = ~0ull;
       constexpr int U = 4;  // 32-point chunks loaded per iteration
@@ -733,6 +882,13 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
           const uint64_t key =
               i < n ? (((uint64_t)__float_as_uint(dist1(pt[u], c)) << 32) | (uint32_t)i) : ~0ull;
           unsigned mask = __ballot_sync(kFull, key < thr);
+          if constexpr (KPL == 1) {
+            if (__popc(mask) > kKnnInsertMax) {  // many candidates: sort them and merge
+              L[0] = warp_merge64(L[0], warp_sort64(key < thr ? key : ~0ull, lane), lane);
+              thr = __shfl_sync(kFull, L[0], kl);
+              mask = 0;
+            }
+          }
           while (mask) {
             const int src = __ffs(mask) - 1;
             mask &= mask - 1;
@@ -748,9 +904,9 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
                 const uint64_t carry = __shfl_sync(kFull, L[q - 1], 31);
                 if (lane == 0) up = carry;
               }
-              const int e = q * 32 + lane;
-              if (e > pos) L[q] = up;
-              else if (e == pos) L[q] = v;
+              const int e2 = q * 32 + lane;
+              if (e2 > pos) L[q] = up;
+              else if (e2 == pos) L[q] = v;
             }
             uint64_t t = 0;
 #pragma unroll
@@ -764,17 +920,17 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
     int gidx[KPL];
 #pragma unroll
     for (int q = 0; q < KPL; ++q) {
-      const int e = q * 32 + lane;
-      gidx[q] = (e < k && L[q] != ~0ull) ? (int)(o0 + (int64_t)(uint32_t)L[q]) : -1;
-      if (e < k) knn_idx[r * k + e] = gidx[q];
+      const int e2 = q * 32 + lane;
+      gidx[q] = (e2 < k && L[q] != ~0ull) ? (int)(o0 + (int64_t)(uint32_t)L[q]) : -1;
+      if (e2 < k) knn_idx[orow * k + e2] = gidx[q];
     }
-    if (pooled) knn_row_pool<KPL>(feats, F, gidx, pooled + r * F, counts + r);
+    if (pooled) knn_row_pool<KPL>(feats, F, gidx, pooled + orow * F, counts + orow);
   }
 }
 
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
                        const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, const float* feats,
-                       int F, float* pooled, int32_t* counts, const int* cls, WsHeader* hdr,
+                       int F, float* pooled, int32_t* counts, const Workspace* ws, WsHeader* hdr,
                        cudaStream_t s) {
   const DeviceInfo& di = device_info();
   const int64_t rows = (int64_t)B * K;
@@ -782,16 +938,25 @@ cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, cons
   const int64_t cap = (int64_t)di.sm_count * 16;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
+  KnnOrder ord{};
+  if (ws) {
+    ord.on = 1;
+    ord.list[0] = ws->list_cluster16;
+    ord.list[1] = ws->list_cluster8;
+    ord.list[2] = ws->list_cta_smem;
+    ord.list[3] = ws->list_cta;
+    ord.list[4] = ws->list_warp;
+  }
   count_launch();
   if (k <= 32)
     k_knn<1><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
-                                         feats, F, pooled, counts, cls, hdr);
+                                         feats, F, pooled, counts, ord, hdr);
   else if (k <= 64)
     k_knn<2><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
-                                         feats, F, pooled, counts, cls, hdr);
+                                         feats, F, pooled, counts, ord, hdr);
   else
     k_knn<4><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
-                                         feats, F, pooled, counts, cls, hdr);
+                                         feats, F, pooled, counts, ord, hdr);
   return cudaGetLastError();
 }
 
@@ -842,7 +1007,7 @@ cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const fl
                           const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,
                           cudaStream_t s) {
   const DeviceInfo& di = device_info();
-  const size_t sm = (size_t)K * sizeof(Cent2);
+  const size_t sm = (size_t)pad_pairs(K) * sizeof(Cent2);
   count_launch();
   k_assign<<<di.sm_count * 4, 256, sm, s>>>(coords, offsets, K, centroids, valid_tokens, token_id, ws);
   return cudaGetLastError();

@@ -77,16 +77,35 @@ __device__ __forceinline__ Cent2 cent2(float4 c) {
   return Cent2{pack2(c.x, c.x), pack2(c.y, c.y), pack2(c.z, c.z), pack2(c.w, c.w)};
 }
 
-// Distances of two points (packed component-wise) to one centroid.
+// A packed zero the compiler cannot prove to be zero: a volatile load of a
+// device variable that is never written.  ptxas merges a packed multiply
+// that feeds a packed add into one fused multiply-add even with contraction
+// disabled (-fmad=false, .rn), which rounds d*d + s once instead of twice.
+// The squares are therefore formed as fma(d, d, z) with this runtime zero:
+// d*d + 0 rounds exactly like d*d, and an FMA whose addend is an unknown
+// register is not merged with the add that follows.
+static __device__ uint64_t g_opaque_zero2;
+__device__ __forceinline__ uint64_t opaque_zero2() { return *reinterpret_cast<volatile uint64_t*>(&g_opaque_zero2); }
+
+// d * d of both lanes, rounded once each (z: opaque_zero2()).
+__device__ __forceinline__ uint64_t sq2(uint64_t d, uint64_t z) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %1, %2;" : "=l"(r) : "l"(d), "l"(z));
+  return r;
+}
+
+// Distances of two points (packed component-wise) to one centroid:
+// ((dx*dx + dy*dy) + dz*dz) + dt*dt per lane, every operation rounded to
+// nearest on its own (z: opaque_zero2()).
 __device__ __forceinline__ uint64_t dist2(uint64_t X, uint64_t Y, uint64_t Z, uint64_t T,
-                                          const Cent2& c) {
+                                          const Cent2& c, uint64_t z) {
   uint64_t dx = sub2(X, c.x);
   uint64_t dy = sub2(Y, c.y);
   uint64_t dz = sub2(Z, c.z);
   uint64_t dt = sub2(T, c.t);
-  uint64_t s = add2(mul2(dx, dx), mul2(dy, dy));
-  s = add2(s, mul2(dz, dz));
-  s = add2(s, mul2(dt, dt));
+  uint64_t s = add2(sq2(dx, z), sq2(dy, z));
+  s = add2(s, sq2(dz, z));
+  s = add2(s, sq2(dt, z));
   return s;
 }
 
@@ -115,6 +134,13 @@ __device__ __forceinline__ int fkey(float v) { return __float_as_int(v); }
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Three-input float32 minimum (sm_100).
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
@@ -148,6 +174,35 @@ __device__ __forceinline__ float4 ldg4(const float4* p) { return __ldg(p); }
 
 // ---------------------------------------------------------------- per-token sums
 
+// Exclusive prefix sum of cnt[0 .. K) into start[] and cur[] by one warp
+// (lane = rank < 32), 8 entries per lane; K <= 256.
+__device__ __forceinline__ void count_scan(const int* cnt, int* start, int* cur, int K, int lane) {
+  int local[8];
+  int sum = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int j = lane * 8 + q;
+    local[q] = j < K ? cnt[j] : 0;
+    sum += local[q];
+  }
+  int x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  int run = x - sum;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int j = lane * 8 + q;
+    if (j < K) {
+      start[j] = run;
+      cur[j] = run;
+    }
+    run += local[q];
+  }
+}
+
 // Counting sort of npts labelled points by a group of threads (a warp or a
 // CTA; `rank` / `size` are this thread's index in it and its size, `sync` its
 // barrier): cnt[j] = number of points labelled j, start[j] = exclusive prefix
@@ -165,32 +220,7 @@ __device__ __forceinline__ void label_sort(const int* lab, int npts, int K, int*
     if ((unsigned)l < (unsigned)K) atomicAdd(&cnt[l], 1);
   }
   sync();
-  if (rank < 32) {  // exclusive scan by the group's first warp, 8 entries per lane
-    int local[8];
-    int sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int j = rank * 8 + q;
-      local[q] = j < K ? cnt[j] : 0;
-      sum += local[q];
-    }
-    int x = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, x, o);
-      if (rank >= o) x += y;
-    }
-    int run = x - sum;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int j = rank * 8 + q;
-      if (j < K) {
-        start[j] = run;
-        cur[j] = run;
-      }
-      run += local[q];
-    }
-  }
+  if (rank < 32) count_scan(cnt, start, cur, K, rank);
   sync();
   for (int i = rank; i < npts; i += size) {
     const int l = lab[i];
@@ -204,14 +234,50 @@ __device__ __forceinline__ void label_sort(const int* lab, int npts, int K, int*
 }
 
 // Per-token float64 sums over the first nsorted positions of a counting
-// sort: each warp of the group takes tiles of 32 consecutive sorted
+// sort, balanced over the group: every thread takes an equal run of sorted
+// positions, adds val(i, v) for v < V along it and flushes its partial sums
+// into acc[token * V + v] (shared memory, zeroed beforehand) whenever the
+// token changes and at the end of its run.  V <= 8 per call.
+template <typename Val>
+__device__ __forceinline__ void segment_sums(const int* perm, const int* slab, int nsorted, int V, int v0,
+                                             int ldacc, double* acc, int rank, int size, Val val) {
+  const int per = (nsorted + size - 1) / size;
+  const int p0 = rank * per, p1 = min(nsorted, p0 + per);
+  if (p0 >= p1) return;
+  double s[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) s[v] = 0.0;
+  int cur = slab[p0];
+  for (int q = p0; q < p1; ++q) {
+    const int i = perm[q];
+    const int l = slab[q];
+    if (l != cur) {
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        if (v < V) {
+          atomicAdd(&acc[cur * ldacc + v0 + v], s[v]);
+          s[v] = 0.0;
+        }
+      cur = l;
+    }
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      if (v < V) s[v] += val(i, v0 + v);
+  }
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    if (v < V) atomicAdd(&acc[cur * ldacc + v0 + v], s[v]);
+}
+
+// Per-token float64 sums, warp-tile form (for cheap val() reads such as
+// staged shared memory): each warp of the group takes tiles of 32 consecutive sorted
 // positions, forms a segmented inclusive scan of val(i, v) over the lanes of
 // each token with shuffles, and the last lane of every token in the tile adds
 // the tile's partial sum into acc[token * ldacc + v] (shared memory, zeroed
 // beforehand).  A token therefore gets one atomic per tile it spans, not one
 // per point.  The group size is a multiple of 32; v runs over [v0, v0 + V).
 template <typename Val>
-__device__ __forceinline__ void segment_sums(const int* perm, const int* slab, int nsorted, int V, int v0,
+__device__ __forceinline__ void segment_sums_scan(const int* perm, const int* slab, int nsorted, int V, int v0,
                                              int ldacc, double* acc, int rank, int size, Val val) {
   const int lane = rank & 31, warp = rank >> 5, nwarps = size >> 5;
   for (int tile = warp * 32; tile < nsorted; tile += nwarps * 32) {

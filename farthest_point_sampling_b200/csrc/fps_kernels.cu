@@ -81,10 +81,11 @@ __device__ __forceinline__ void prefetch_rows_l2(const float* lo, size_t bytes, 
 // One FPS event on one warp, NP point pairs per lane.
 template <int NP>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
-                                           int lane, DupPoint* s_dup, int32_t* __restrict__ cidx,
+                                           int lane, float4* s_pts, int32_t* __restrict__ cidx,
                                            float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
                                            const PoolOut& po) {
   if (po.feats && lane < 4) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), lane, 4);
+  const uint64_t z2 = opaque_zero2();
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -95,8 +96,8 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (i0 < n) a = ldg4(pts + i0);
     if (i1 < n) b = ldg4(pts + i1);
-    if (i0 < n) s_dup[i0] = dup_point(a);
-    if (i1 < n) s_dup[i1] = dup_point(b);
+    if (i0 < n) s_pts[i0] = a;
+    if (i1 < n) s_pts[i1] = b;
     X[p] = pack2(a.x, b.x);
     Y[p] = pack2(a.y, b.y);
     Z[p] = pack2(a.z, b.z);
@@ -110,17 +111,17 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
   }
   __syncwarp();
   for (int s = 0; s < K; ++s) {
-    const DupPoint cp = s_dup[c];
+    const float4 cp = s_pts[c];
     if (lane == 0) {
       cidx[s] = (int32_t)(off + c);
-      cpos[s] = dup_to_float4(cp);
+      cpos[s] = cp;
     }
     if ((c & 31) == lane) taken |= 1u << (c >> 5);
-    const Cent2 C = cent2_dup(cp);
+    const Cent2 C = cent2(cp);
     float m0 = kEmptySlot, m1 = kEmptySlot;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);
+      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
       relax(lo2(d), dist[2 * p], lab[2 * p], s);
       relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
       if (p & 1)
@@ -151,7 +152,7 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
   if (po.feats) {  // token means: float64 shared sums over the event copy's space
     const int F = po.F;
     __syncwarp();
-    double* acc = reinterpret_cast<double*>(s_dup);  // [K * F]
+    double* acc = reinterpret_cast<double*>(s_pts);  // [K * F]
     int* cnt = reinterpret_cast<int*>(acc + K * F);   // [K]
     for (int e = lane; e < K * F; e += 32) acc[e] = 0.0;
     for (int j = lane; j < K; j += 32) cnt[j] = 0;
@@ -185,7 +186,7 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
 }
 
 template <int NPMAX>
-__global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ coords,
+__global__ void __launch_bounds__(128, 4) k_fps_warp(const float4* __restrict__ coords,
                                                      const int64_t* __restrict__ offsets,
                                                      const int32_t* __restrict__ start_local,
                                                      const int* __restrict__ list, WsHeader* hdr, int K,
@@ -194,9 +195,9 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
                                                      float4* __restrict__ centroids, PoolOut po) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
-  extern __shared__ DupPoint s_dup_all[];
+  extern __shared__ float4 s_pts_all[];
   const int lane = threadIdx.x & 31;
-  DupPoint* s_dup = s_dup_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
+  float4* s_pts = s_pts_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
   const int count = hdr->n_items[kListWarp];
   for (;;) {
     int w = 0;
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(128, 3) k_fps_warp(const float4* __restrict__ 
     const int c0 = start_local ? start_local[b] : 0;
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define WARP_CALL(N)                                                                                   \
-  warp_event<N>(coords + off, n, c0, K, off, lane, s_dup, centroid_idx + (int64_t)b * K,               \
+  warp_event<N>(coords + off, n, c0, K, off, lane, s_pts, centroid_idx + (int64_t)b * K,               \
                 centroids + (int64_t)b * K, tok, b, po)
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
@@ -235,6 +236,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (po.feats && tid < 32) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), tid, 32);
+  const uint64_t z2 = opaque_zero2();
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
@@ -280,7 +282,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     float m0 = kEmptySlot, m1 = kEmptySlot;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C);
+      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
       relax(lo2(d), dist[2 * p], lab[2 * p], s);
       relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
       if (p & 1)
@@ -332,7 +334,9 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     for (int e = tid; e < n * F; e += NT) s_feat[e] = __ldg(fe + e);
     for (int e = tid; e < K * F; e += NT) acc[e] = 0.0;
     label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, slab, tid, NT, [] { __syncthreads(); });
-    segment_sums(perm, slab, n, F, 0, F, acc, tid, NT, [&](int i, int f) { return (double)s_feat[i * F + f]; });
+    for (int v0 = 0; v0 < F; v0 += 8)
+      segment_sums(perm, slab, n, min(8, F - v0), v0, F, acc, tid, NT,
+                   [&](int i, int f) { return (double)s_feat[i * F + f]; });
     __syncthreads();
     for (int j = tid; j < K; j += NT) {
       const int c = cnt[j];
@@ -448,6 +452,7 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
                    : make_float4(lo2(xy.x), lo2(xy.y), lo2(zt.x), lo2(zt.y));
   };
 
+  const uint64_t z2 = opaque_zero2();
   float dist[2 * NP];
   int lab[2 * NP];
   unsigned long long taken = 0;
@@ -480,7 +485,7 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
     for (int p = 0; p < NP; ++p) {
       const ulonglong2 xy = sXY[p * NT + tid];
       const ulonglong2 zt = sZT[p * NT + tid];
-      const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C);
+      const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C, z2);
       relax(lo2(d), dist[2 * p], lab[2 * p], s);
       relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
       if (p & 1)
@@ -598,11 +603,11 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
 // ------------------------------------------------------------------ launch
 
 constexpr int kWarpBlock = 128;
-constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(DupPoint);
+constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(float4);
 constexpr size_t kCtaSmem = kCtaSmemBytes;
 static_assert((size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint) <= kCtaSmem, "event copy fits");
 
-size_t warp_region_bytes() { return (size_t)64 * kWarpPairs * sizeof(DupPoint); }
+size_t warp_region_bytes() { return (size_t)64 * kWarpPairs * sizeof(float4); }
 size_t cta_region_bytes() { return kCtaSmem; }
 
 template <int CL>

@@ -121,7 +121,7 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
   if (pb.assign_mode == FPS_ASSIGN_KNN) {
     stage_mark(7, 0, s);
     if ((e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx,
-                        pb.feats, pb.F, pb.pooled, pb.counts, ws.cls, ws.hdr, s)))
+                        pb.feats, pb.F, pb.pooled, pb.counts, &ws, ws.hdr, s)))
       return from_cuda(e);
     stage_mark(7, 1, s);
   } else {

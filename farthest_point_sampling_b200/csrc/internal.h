@@ -59,7 +59,7 @@ struct Workspace {
   double* pool_acc; // [pool slots][K][F]
   int* pool_cnt;    // [pool slots][K]
   int* pool_ticket; // [pool slots]
-  double* lloyd[3]; // 3 x [fps slots][K][5]
+  double* lloyd[3]; // 3 x [fps slots][K][5] cell sums (W, S_x, S_y, S_z, S_t)
   int* labels;      // [P] internal Voronoi labels (kNN mode with Lloyd)
   int fps_slots;    // capacity of the Lloyd slot range
   int pool_slots;   // capacity of the pooling slot range
@@ -102,7 +102,7 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
                                 const Workspace& ws, cudaStream_t s);
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
                        const int32_t* valid_tokens, int K, int k, int32_t* knn_idx,
-                       const float* feats, int F, float* pooled, int32_t* counts, const int* cls,
+                       const float* feats, int F, float* pooled, int32_t* counts, const Workspace* ws,
                        struct WsHeader* hdr, cudaStream_t s);
 cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const float4* centroids,
                           const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,

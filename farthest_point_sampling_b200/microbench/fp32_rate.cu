@@ -1,11 +1,18 @@
-// In-run FP32 issue-rate microbenchmark for the roofline of the FPS kernels.
+// In-run FP32 rate microbenchmark for the roofline of the FPS kernels.
 //
-// The FPS distance is made of separate (unfused) float32 adds and multiplies,
-// so its ceiling is the rate of non-FMA FP32 operations.  Two kernels measure
-// it on every SM: independent chains of scalar FADD/FMUL, and of the packed
-// f32x2 forms (two float32 operations per instruction).  Each thread keeps 8
-// independent chains so latency is hidden; the result is stored only when an
-// impossible value appears, which keeps the compiler from removing the work.
+// The FPS distance ((dx*dx + dy*dy) + dz*dz) + dt*dt is made of separately
+// rounded float32 subtracts, multiplies and adds, so its ceiling is the rate
+// of non-FMA FP32 operations.  Each mode runs independent dependency chains
+// (8 per thread, so latency is hidden) on every SM:
+//   0  scalar FMUL + FADD (round-to-nearest intrinsics, never fused)
+//   1  packed f32x2 adds only
+//   2  packed f32x2 multiplies only
+//   3  packed f32x2 fused multiply-adds with a register addend (2 ops each)
+//   4  the packed distance exactly as the FPS kernels compute it (squares as
+//      FMAs with a runtime zero addend, see common.cuh), 11 ops per lane
+// A packed multiply feeding a packed add is merged into one FMA by ptxas, so
+// modes 1 and 2 keep the two operations in separate chains.  The result is
+// stored only when an impossible value appears, which keeps the work alive.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -21,6 +28,23 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   asm volatile("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm volatile("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm volatile("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ uint64_t g_zero2;  // never written: a zero the compiler cannot see
+
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ uint64_t splat(float v) { return pk(v, v); }
 
 __global__ void k_scalar(float* out, int iters, float seed) {
   float a[8];
@@ -40,19 +64,34 @@ __global__ void k_scalar(float* out, int iters, float seed) {
   if (s == -1.2345f) out[blockIdx.x] = s;
 }
 
+template <int MODE>
 __global__ void k_packed(float* out, int iters, float seed) {
   uint64_t a[8];
   const float base = seed + (float)threadIdx.x;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    a[i] = (uint64_t)__float_as_uint(base + i) | ((uint64_t)__float_as_uint(base - i) << 32);
-  const uint64_t m = (uint64_t)__float_as_uint(0.999999f) * 0x100000001ull;
-  const uint64_t c = (uint64_t)__float_as_uint(1e-7f) * 0x100000001ull;
+  for (int i = 0; i < 8; ++i) a[i] = pk(base + i, base - i);
+  const uint64_t m = splat(0.999999f), c = splat(1e-7f);
+  const uint64_t z = *reinterpret_cast<volatile uint64_t*>(&g_zero2);
+  const uint64_t cx = splat(0.5f), cy = splat(-0.25f), cz = splat(0.125f), ct = splat(2.0f);
+  uint64_t Y = splat(base * 0.5f), Z = splat(base * 0.25f), T = splat(base * 0.125f);
   for (int it = 0; it < iters; ++it) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      a[i] = mul2(a[i], m);
-      a[i] = add2(a[i], c);
+      if (MODE == 1) {
+        a[i] = add2(a[i], c);
+        a[i] = add2(a[i], m);
+      } else if (MODE == 2) {
+        a[i] = mul2(a[i], m);
+        a[i] = mul2(a[i], m);
+      } else if (MODE == 3) {
+        a[i] = fma2(a[i], m, c);
+        a[i] = fma2(a[i], m, c);
+      } else {  // the distance, fed back into its x input
+        const uint64_t dx = sub2(a[i], cx), dy = sub2(Y, cy), dz = sub2(Z, cz), dt = sub2(T, ct);
+        uint64_t s = add2(fma2(dx, dx, z), fma2(dy, dy, z));
+        s = add2(s, fma2(dz, dz, z));
+        a[i] = add2(s, fma2(dt, dt, z));
+      }
     }
   }
   float s = 0.f;
@@ -65,22 +104,31 @@ __global__ void k_packed(float* out, int iters, float seed) {
 
 extern "C" {
 
-// Runs one kernel (packed != 0: f32x2) over `blocks` x `threads` threads for
+// Runs mode `mode` (0..4, see above) over `blocks` x `threads` threads for
 // `iters` iterations on `stream` between the caller's two events; returns
-// the number of float32 operations it performs, or -1 on a launch error.
-// `out` is a device buffer of at least `blocks` floats.
-double fpstok_microbench_fp32(int packed, int blocks, int threads, int iters, float* out, void* start_event,
+// the number of float32 operations it performs (an FMA counts as two), or
+// -1 on a bad mode or a launch error.  `out`: at least `blocks` floats.
+double fpstok_microbench_fp32(int mode, int blocks, int threads, int iters, float* out, void* start_event,
                               void* stop_event, void* stream) {
+  if (mode < 0 || mode > 4) return -1.0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaEventRecord(reinterpret_cast<cudaEvent_t>(start_event), s);
-  if (packed)
-    k_packed<<<blocks, threads, 0, s>>>(out, iters, 1.0f);
-  else
-    k_scalar<<<blocks, threads, 0, s>>>(out, iters, 1.0f);
+  switch (mode) {
+    case 0: k_scalar<<<blocks, threads, 0, s>>>(out, iters, 1.0f); break;
+    case 1: k_packed<1><<<blocks, threads, 0, s>>>(out, iters, 1.0f); break;
+    case 2: k_packed<2><<<blocks, threads, 0, s>>>(out, iters, 1.0f); break;
+    case 3: k_packed<3><<<blocks, threads, 0, s>>>(out, iters, 1.0f); break;
+    default: k_packed<4><<<blocks, threads, 0, s>>>(out, iters, 1.0f); break;
+  }
   cudaEventRecord(reinterpret_cast<cudaEvent_t>(stop_event), s);
   if (cudaGetLastError() != cudaSuccess) return -1.0;
-  // 8 chains x (1 mul + 1 add) per iteration; f32x2 does two lanes each
-  return (double)blocks * threads * (double)iters * 16.0 * (packed ? 2.0 : 1.0);
+  const double lanes = (double)blocks * threads * (double)iters * 8.0;  // chain links
+  switch (mode) {
+    case 0: return lanes * 2.0;        // one FMUL + one FADD
+    case 1: case 2: return lanes * 4.0;  // two packed ops, two lanes each
+    case 3: return lanes * 8.0;        // two packed FMAs, two lanes, two ops
+    default: return lanes * 22.0;      // 11 ops per lane, two lanes
+  }
 }
 
 }
