@@ -31,13 +31,59 @@ __device__ __forceinline__ int sched_shift(int q) {
   return q == 0 ? 1 : (q == 1 ? 4 : (q == 2 ? 6 : (q == 3 ? 9 : 10)));
 }
 
+// Reserves v consecutive entries of the shared counter *ctr for every lane
+// of the warp (all lanes call it; v may be 0) with one atomic per warp;
+// returns the lane's first entry.
+__device__ __forceinline__ int warp_reserve(int* ctr, int v) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  const int total = __shfl_sync(kFull, x, 31);
+  int base = 0;
+  if (lane == 31 && total > 0) base = atomicAdd(ctr, total);
+  base = __shfl_sync(kFull, base, 31);
+  return base + x - v;
+}
+
+// Exclusive prefix sum of v over the CTA and (in `total`) the CTA's sum;
+// tmp: 32 ints of shared memory.  Every thread of the CTA must call it.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* tmp, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, w, o);
+      if (lane >= o) w += y;
+    }
+    tmp[lane] = w;  // inclusive over the warps
+  }
+  __syncthreads();
+  const int before = warp > 0 ? tmp[warp - 1] : 0;
+  total = tmp[nw - 1];
+  __syncthreads();  // tmp may be reused
+  return before + x - v;
+}
+
 // One CTA: classifies every event, builds the per-schedule work lists sorted
 // by decreasing size (longest chains first), the (event, chunk) items of FPS
 // events, and the accumulator slots; resets the status word and the cursors.
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
                                                int force, int chunk_all, int fused_pool, int latency_events,
-                                               Workspace ws) {
+                                               int need_passes, Workspace ws) {
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps;
@@ -139,39 +185,59 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     if (lane == 31) cnt[q] = run;
   }
   __syncthreads();
-  // pass 3: scatter into the sorted lists; chunks and accumulator slots
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const int cls = ws.cls[b];
-    int fslot = -1, pslot = -1;
+  // pass 3: scatter into the sorted lists; pooling items and accumulator
+  // slots.  The loop is warp-uniform so that the shared counters are bumped
+  // once per warp (warp_reserve) rather than once per event.
+  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+    const int b = b0 + threadIdx.x;
+    const int cls = b < B ? ws.cls[b] : kClsSkip;
     int n = 0;
     if (cls == kClsFps || cls == kClsPass) n = size_of(b);
+    const int q = cls == kClsFps ? schedule_of(n) : 0;
     if (cls == kClsFps) {
-      const int q = schedule_of(n);
       int* list = q == 0 ? ws.list_warp
                          : (q == 1 ? ws.list_cta
                                    : (q == 2 ? ws.list_cta_smem : (q == 3 ? ws.list_cluster8 : ws.list_cluster16)));
       list[atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1)] = b;
-      fslot = atomicAdd(&cnt[kListFps], 1);
     }
-    if (cls == kClsFps || (chunk_all && cls == kClsPass)) {
-      const int nch = (n + kChunk - 1) / kChunk;
-      const int base = atomicAdd(&cnt[kListChunks], nch);
-      for (int c = 0; c < nch; ++c) ws.chunks[base + c] = make_int2(b, c);
-      // pooling items (passthrough events of fps_tokenize are written directly;
-      // events of schedules that pool in place are left out)
-      if (cls == kClsFps && ((fused_pool >> schedule_of(n)) & 1)) {
-        ws.fps_slot[b] = fslot;
-        ws.pool_slot[b] = -1;
-        continue;
-      }
-      const int npc = (n + kPoolChunk - 1) / kPoolChunk;
-      const int pbase = atomicAdd(&cnt[kListPoolChunks], npc);
-      for (int c = 0; c < npc; ++c) ws.pool_chunks[pbase + c] = make_int2(b, c);
-      if (npc > 1) pslot = atomicAdd(&cnt[kListPoolSlots], 1);
+    const int fslot = warp_reserve(&cnt[kListFps], cls == kClsFps ? 1 : 0);
+    // pooling items (passthrough events of fps_tokenize are written directly;
+    // events of schedules that pool in place are left out)
+    const bool pooled_here = (cls == kClsFps && !((fused_pool >> q) & 1)) || (chunk_all && cls == kClsPass);
+    const int npc = pooled_here ? (n + kPoolChunk - 1) / kPoolChunk : 0;
+    const int pbase = warp_reserve(&cnt[kListPoolChunks], npc);
+    for (int c = 0; c < npc; ++c) ws.pool_chunks[pbase + c] = make_int2(b, c);
+    const int pslot = warp_reserve(&cnt[kListPoolSlots], npc > 1 ? min(kPoolReplicas, npc) : 0);
+    const int pev = warp_reserve(&cnt[kListPoolEvents], npc > 1 ? 1 : 0);
+    if (npc > 1) ws.pool_event[pev] = b;
+    if (b < B) {
+      ws.fps_slot[b] = cls == kClsFps ? fslot : -1;
+      ws.pool_slot[b] = npc > 1 ? pslot : -1;
     }
-    ws.fps_slot[b] = fslot;
-    ws.pool_slot[b] = pslot;
   }
+
+  __syncthreads();
+  // pass 4 (need_passes): the nearest-centroid passes of the chunked events (FPS events,
+  // and the passthrough ones with chunk_all) in batch order: event b with n_b
+  // points contributes passes (b, 0), (b, kPass), ... -- ceil(n_b / kPass)
+  // of them, consecutive -- so that a CTA given a contiguous range of passes
+  // mostly stays on one event.
+  __shared__ int s_tmp[32];
+  int carry = 0;
+  for (int b0 = 0; need_passes && b0 < B; b0 += blockDim.x) {
+    const int b = b0 + threadIdx.x;
+    int n = 0;
+    if (b < B) {
+      const int cls = ws.cls[b];
+      if (cls == kClsFps || (chunk_all && cls == kClsPass)) n = size_of(b);
+    }
+    const int np = (n + kPass - 1) / kPass;
+    int tot;
+    const int base = carry + cta_exclusive_scan(np, s_tmp, tot);
+    for (int j = 0; j < np; ++j) ws.passes[base + j] = make_int2(b, j * kPass);
+    carry += tot;
+  }
+  if (threadIdx.x == 0) cnt[kListChunks] = carry;
   __syncthreads();
   if (threadIdx.x < kNumLists) ws.hdr->n_items[threadIdx.x] = cnt[threadIdx.x];
 }
@@ -179,8 +245,9 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
 cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   count_launch();
+  const int need_passes = chunk_all || pb.lloyd_iters > 0;
   k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
-                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, ws);
+                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, need_passes, ws);
   return cudaGetLastError();
 }
 
@@ -197,12 +264,6 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
   for (int b = gw; b < pb.B; b += nw) {
     const int cls = ws.cls[b];
     if (cls == kClsFps) {
-      const int ps = ws.pool_slot[b];
-      if (ps >= 0) {
-        for (int e = lane; e < K * F; e += 32) ws.pool_acc[(int64_t)ps * K * F + e] = 0.0;
-        for (int e = lane; e < K; e += 32) ws.pool_cnt[(int64_t)ps * K + e] = 0;
-        if (lane == 0) ws.pool_ticket[ps] = 0;
-      }
       const int fs = ws.fps_slot[b];
       if (lloyd_on && fs >= 0) {
         for (int e = lane; e < K * 5; e += 32) {
@@ -261,9 +322,9 @@ cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStrea
 
 // Shared-memory layout of one chunk's counting sort.
 struct SortSmem {
-  int* lab;    // [kChunk] token of every point
-  int* perm;   // [kChunk] point of every sorted position
-  int* slab;   // [kChunk] token of every sorted position
+  int* lab;    // [chunk] token of every point
+  int* perm;   // [chunk] point of every sorted position
+  int* slab;   // [chunk] token of every sorted position
   int* cnt;    // [256]
   int* start;  // [256]
   int* cur;    // [256]
@@ -277,20 +338,6 @@ constexpr size_t sort_smem_bytes(int chunk) { return (size_t)(3 * chunk + 3 * 25
 __device__ __forceinline__ void cta_sync() { __syncthreads(); }
 
 constexpr int kStageMaxF = 8;  // the pool kernel stages feature rows in shared memory up to this F
-
-// Sorts the chunk by token and adds up V values per token into acc[K * V]
-// (shared float64, zeroed here): balanced over the CTA.
-template <typename Val>
-__device__ __forceinline__ void chunk_token_sums(const SortSmem& sm, int npts, int K, int V, double* acc, Val val) {
-  const int tid = threadIdx.x, T = blockDim.x;
-  for (int e = tid; e < K * V; e += T) acc[e] = 0.0;
-  label_sort(sm.lab, npts, K, sm.cnt, sm.start, sm.cur, sm.perm, sm.slab, tid, T, cta_sync);
-  int nsorted = 0;
-  if (K > 0) nsorted = sm.start[K - 1] + sm.cnt[K - 1];
-  for (int v0 = 0; v0 < V; v0 += 8)
-    segment_sums(sm.perm, sm.slab, nsorted, min(8, V - v0), v0, V, acc, tid, T, val);
-  __syncthreads();
-}
 
 // One CTA per (event, chunk) item: counting sort of the chunk's points by
 // token, float64 sums per (token, feature) -- one thread per token when no
@@ -309,7 +356,6 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
   const SortSmem sm = sort_smem(smem_i, kPoolChunk);
   double* acc = reinterpret_cast<double*>(smem_i + 3 * kPoolChunk + 3 * 256);  // [K * F]
   float* s_feat = reinterpret_cast<float*>(acc + K * F);  // [kPoolChunk * F] when F <= kStageMaxF
-  __shared__ int s_last;
   const int nitems = ws.hdr->n_items[kListPoolChunks];
   const int T = blockDim.x, tid = threadIdx.x;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
@@ -369,27 +415,62 @@ __global__ void __launch_bounds__(256) k_pool_voronoi(const float* __restrict__ 
         counts[(int64_t)b * K + tid] = cj;
       }
     } else {
-      const int ps = ws.pool_slot[b];
+      // chunk c adds into replica c % nrep: fewer updates per address
+      const int ps = ws.pool_slot[b] + it.y % min(kPoolReplicas, nch);
       double* gacc = ws.pool_acc + (int64_t)ps * K * F;
       int* gcnt = ws.pool_cnt + (int64_t)ps * K;
-      if (tid < K && cj) {
+      if (tid < K && cj) {  // reductions only; k_pool_finalize forms the means
         for (int f = 0; f < F; ++f) atomicAdd(&gacc[tid * F + f], acc[tid * F + f]);
         atomicAdd(&gcnt[tid], cj);
-      }
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) s_last = atomicAdd(&ws.pool_ticket[ps], 1) == nch - 1;
-      __syncthreads();
-      if (s_last && tid < K) {
-        __threadfence();
-        const int c = __ldcg(&gcnt[tid]);
-        float* prow = pooled + ((int64_t)b * K + tid) * F;
-        for (int f = 0; f < F; ++f) prow[f] = c ? (float)(__ldcg(&gacc[tid * F + f]) / (double)c) : 0.f;
-        counts[(int64_t)b * K + tid] = c;
       }
     }
     __syncthreads();
   }
+}
+
+// Means of the events pooled over several chunks, from the float64 sums and
+// counts of their accumulator replicas in global memory: one thread per
+// (event, token), the replica loads of a value issued together.
+__global__ void __launch_bounds__(256) k_pool_finalize(const int64_t* __restrict__ offsets,
+                                                       float* __restrict__ pooled, int32_t* __restrict__ counts,
+                                                       int K, int F, Workspace ws) {
+  const int64_t total = (int64_t)ws.hdr->n_items[kListPoolEvents] * K;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    const int e = (int)(t / K), j = (int)(t - (int64_t)e * K);
+    const int b = ws.pool_event[e];
+    const int ps = ws.pool_slot[b];
+    const int n = (int)(offsets[b + 1] - offsets[b]);
+    const int nrep = min(kPoolReplicas, (n + kPoolChunk - 1) / kPoolChunk);
+    int c = 0;
+#pragma unroll
+    for (int r = 0; r < kPoolReplicas; ++r)
+      if (r < nrep) c += ws.pool_cnt[(int64_t)(ps + r) * K + j];
+    float* prow = pooled + ((int64_t)b * K + j) * F;
+    for (int f = 0; f < F; ++f) {
+      double sum = 0.0;
+#pragma unroll
+      for (int r = 0; r < kPoolReplicas; ++r)
+        if (r < nrep) sum += ws.pool_acc[((int64_t)(ps + r) * K + j) * F + f];
+      prow[f] = c ? (float)(sum / (double)c) : 0.f;
+    }
+    counts[(int64_t)b * K + j] = c;
+  }
+}
+
+// Clears the pooling accumulator slots the binning kernel handed out.
+__global__ void __launch_bounds__(256) k_pool_clear(int K, int F, Workspace ws) {
+  const int64_t ns = ws.hdr->n_items[kListPoolSlots];
+  const int64_t na = ns * K * F, nc = ns * K;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < na; e += stride) ws.pool_acc[e] = 0.0;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < nc; e += stride) ws.pool_cnt[e] = 0;
+}
+
+cudaError_t launch_pool_clear(const Problem& pb, const Workspace& ws, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  count_launch();
+  k_pool_clear<<<di.sm_count * 2, 256, 0, s>>>(pb.K, pb.F, ws);
+  return cudaGetLastError();
 }
 
 static size_t pool_smem_bytes(int K, int F) {
@@ -397,13 +478,17 @@ static size_t pool_smem_bytes(int K, int F) {
          (F <= kStageMaxF ? (size_t)kPoolChunk * F * sizeof(float) : 0);
 }
 
-cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
+cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int B, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,
                                 const Workspace& ws, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   count_launch();
   k_pool_voronoi<<<di.sm_count * 8, 256, pool_smem_bytes(K, F), s>>>(feats, F, offsets, K, labels, pooled, counts,
                                                                      ws);
+  cudaError_t e = cudaGetLastError();
+  if (e) return e;
+  count_launch();
+  k_pool_finalize<<<di.sm_count * 2, 256, 0, s>>>(offsets, pooled, counts, K, F, ws);
   return cudaGetLastError();
 }
 
@@ -495,39 +580,53 @@ __device__ __forceinline__ void chunk_nearest(const float4* __restrict__ pts, in
   }
 }
 
-constexpr int kNearestPairs = 2;  // pairs per pass: with two centroids in flight, 8 distance chains
-constexpr int kNearestPasses = kChunk / (2 * kNearestPairs * 256);
-static_assert(kNearestPasses * 2 * kNearestPairs * 256 == kChunk, "whole passes per chunk");
+constexpr int kNearestPairs = 2;  // pairs per thread: with two centroids in flight, 8 distance chains
+static_assert(2 * kNearestPairs * 256 == kPass, "one nearest pass covers kPass points with 256 threads");
 
-// Standalone nearest-centroid assignment over (event, chunk) items.
+// The Lloyd and assignment kernels run the pass list: CTA g takes the
+// contiguous range of ceil(Q / grid) passes starting at g ceil(Q / grid)
+// (Q passes in all), so that every CTA does the same number of equal-cost
+// passes and moves to a new event only where the list does.
+__device__ __forceinline__ void pass_range(const Workspace& ws, int& q0, int& q1) {
+  const int Q = ws.hdr->n_items[kListChunks];
+  const int per = (Q + gridDim.x - 1) / gridDim.x;
+  q0 = min(Q, blockIdx.x * per);
+  q1 = min(Q, q0 + per);
+}
+
+// Standalone nearest-centroid assignment.
 constexpr int kAssignThreads = 256;
 
 __global__ void __launch_bounds__(kAssignThreads, 3) k_assign(const float4* __restrict__ coords,
-                                                           const int64_t* __restrict__ offsets, int K,
-                                                           const float4* __restrict__ centroids,
-                                                           const int32_t* __restrict__ valid,
-                                                           int32_t* __restrict__ token_id, Workspace ws) {
+                                                              const int64_t* __restrict__ offsets, int K,
+                                                              const float4* __restrict__ centroids,
+                                                              const int32_t* __restrict__ valid,
+                                                              int32_t* __restrict__ token_id, Workspace ws) {
   constexpr int T = kAssignThreads;
   extern __shared__ Cent2 s_cent[];  // [pad_pairs(K)]
-  const int tid = threadIdx.x;
-  const int nitems = ws.hdr->n_items[kListChunks];
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int2 it = ws.chunks[item];
-    const int b = it.x;
+  int q0, q1;
+  pass_range(ws, q0, q1);
+  int cur = -1, nv = 0;
+  for (int q = q0; q < q1; ++q) {
+    const int2 it = ws.passes[q];
+    const int b = it.x, i0 = it.y;
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
-    int nv = valid ? valid[b] : min(n, K);
-    if (nv < 0 || nv > K) {
-      record_error(ws.hdr, kDevBadToken);
-      nv = 0;
+    if (b != cur) {  // uniform: every thread reads the same pass
+      __syncthreads();
+      nv = valid ? valid[b] : min(n, K);
+      if (nv < 0 || nv > K) {
+        record_error(ws.hdr, kDevBadToken);
+        nv = 0;
+      }
+      load_cents_padded(centroids + (int64_t)b * K, nv, s_cent);
+      __syncthreads();
+      cur = b;
     }
-    load_cents_padded(centroids + (int64_t)b * K, nv, s_cent);
-    __syncthreads();
-    const int i0 = it.y * kChunk, npts = min(n, i0 + kChunk) - i0;
     int32_t* out = token_id + off + i0;
-    chunk_nearest<kNearestPairs, kNearestPasses, T>(coords + off + i0, npts, s_cent, pad_pairs(nv) / 2,
-                                                    [&](int li, int l) { out[li] = nv > 0 ? l : -1; });
-    __syncthreads();
+    const int v = nv;
+    chunk_nearest<kNearestPairs, 1, T>(coords + off + i0, min(n - i0, kPass), s_cent, pad_pairs(nv) / 2,
+                                       [&](int li, int l) { out[li] = v > 0 ? l : -1; });
   }
 }
 
@@ -537,77 +636,131 @@ __device__ __forceinline__ float charge_of(const float* fe, int F, int charge_co
   return charge_col < 0 ? 1.0f : __ldg(fe + (int64_t)i * F + charge_col);
 }
 
-// Lloyd sums of one chunk whose labels, points and charges are in shared
-// memory: W_j = sum q and S_j = sum q p per token, added to `out` (float64,
-// [K][5], global).
-__device__ __forceinline__ void lloyd_chunk_sums(const SortSmem& sm, const float4* s_p, const float* s_q, int npts,
-                                                 int K, double* acc, double* out) {
-  chunk_token_sums(sm, npts, K, 5, acc, [&](int i, int v) {
-    const double q = (double)s_q[i];
-    if (v == 0) return q;
-    const float4 p = s_p[i];
-    return q * (double)(v == 1 ? p.x : (v == 2 ? p.y : (v == 3 ? p.z : p.w)));
-  });
-  for (int e = threadIdx.x; e < K * 5; e += blockDim.x)
-    if (sm.cnt[e / 5]) atomicAdd(&out[e], acc[e]);
+constexpr int kLloydThreads = 256;
+constexpr int kLloydPts = kPass / kLloydThreads;  // points per thread
+static_assert(kLloydPts == 2 * kNearestPairs, "chunk_nearest covers a pass");
+
+// Shared memory of the cell-sum kernel: the counting sort of one piece by
+// label, its points and charges, and the per-token sums.
+struct LloydSmem {
+  int* perm;     // [kPass]
+  int* slab;     // [kPass]
+  int* cnt;      // [256]
+  int* start;    // [256]
+  int* cur;      // [256]
+  float4* s_p;   // [kPass]
+  float* s_q;    // [kPass]
+  double* acc;   // [K * 5]
+};
+static size_t lloyd_smem_bytes(int K) {
+  return (size_t)(2 * kPass + 3 * 256) * sizeof(int) + (size_t)kPass * (sizeof(float4) + sizeof(float)) +
+         (size_t)K * 5 * sizeof(double);
+}
+__device__ __forceinline__ LloydSmem lloyd_smem(char* base) {
+  LloydSmem m;
+  m.perm = reinterpret_cast<int*>(base);
+  m.slab = m.perm + kPass;
+  m.cnt = m.slab + kPass;
+  m.start = m.cnt + 256;
+  m.cur = m.start + 256;
+  m.s_p = reinterpret_cast<float4*>(m.cur + 256);
+  m.s_q = reinterpret_cast<float*>(m.s_p + kPass);
+  m.acc = reinterpret_cast<double*>(m.s_q + kPass);
+  return m;
 }
 
-constexpr size_t kLloydSmemBytes =
-    sort_smem_bytes(kChunk) + (size_t)kChunk * (sizeof(float4) + sizeof(float)) + 256 * 5 * sizeof(double);
+// Cell sums W_j = sum q and S_j = sum q p (float64) of one piece -- points
+// tid + r T, r < kLloydPts, of `pts`, labels `lab`, charges from `fe` --
+// added into out[K][5]: all loads issued first, a counting sort by label in
+// shared memory, balanced per-token sums, one float64 reduction per value of
+// every non-empty cell.  Labels outside [0, K) are reported and left out.
+__device__ __forceinline__ void lloyd_piece_sums(const float4* __restrict__ pts, const float* __restrict__ fe,
+                                        int F, int charge_col, const int32_t* lab, int npts, int K,
+                                                 const LloydSmem& sm, double* __restrict__ out, WsHeader* hdr) {
+  constexpr int T = kLloydThreads;
+  const int tid = threadIdx.x;
+  for (int j = tid; j < K; j += T) sm.cnt[j] = 0;
+  for (int e = tid; e < K * 5; e += T) sm.acc[e] = 0.0;
+  __syncthreads();
+  int l[kLloydPts];
+  float4 p[kLloydPts];
+  float q[kLloydPts];
+#pragma unroll
+  for (int r = 0; r < kLloydPts; ++r) {
+    const int li = tid + r * T;
+    l[r] = -1;
+    if (li < npts) {
+      l[r] = lab[li];
+      p[r] = ldg4(pts + li);
+      q[r] = charge_of(fe, F, charge_col, li);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kLloydPts; ++r) {
+    const int li = tid + r * T;
+    if (li < npts) {
+      if ((unsigned)l[r] >= (unsigned)K) {
+        record_error(hdr, kDevBadToken);
+        l[r] = -1;
+        continue;
+      }
+      sm.s_p[li] = p[r];
+      sm.s_q[li] = q[r];
+      atomicAdd(&sm.cnt[l[r]], 1);
+    }
+  }
+  __syncthreads();
+  if (tid < 32) count_scan(sm.cnt, sm.start, sm.cur, K, tid);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kLloydPts; ++r) {
+    if (l[r] >= 0) {
+      const int pos = atomicAdd(&sm.cur[l[r]], 1);
+      sm.perm[pos] = tid + r * T;
+      sm.slab[pos] = l[r];
+    }
+  }
+  __syncthreads();
+  const int nsorted = sm.start[K - 1] + sm.cnt[K - 1];
+  segment_sums(sm.perm, sm.slab, nsorted, 5, 0, 5, sm.acc, tid, T, [&](int i, int v) {
+    const double qq = (double)sm.s_q[i];
+    if (v == 0) return qq;
+    const float4 pp = sm.s_p[i];
+    return qq * (double)(v == 1 ? pp.x : (v == 2 ? pp.y : (v == 3 ? pp.z : pp.w)));
+  });
+  __syncthreads();
+  for (int e = tid; e < K * 5; e += T)
+    if (sm.cnt[e / 5]) atomicAdd(&out[e], sm.acc[e]);
+}
 
 // Cell sums of the current labels.
-__global__ void __launch_bounds__(256) k_lloyd_sums(const float4* __restrict__ coords,
-                                                    const float* __restrict__ feats, int F,
-                                                    int charge_col, const int64_t* __restrict__ offsets,
-                                                    int K, const int32_t* __restrict__ labels,
-                                                    Workspace ws, double* __restrict__ out) {
-  extern __shared__ int smem_i[];
-  const SortSmem sm = sort_smem(smem_i, kChunk);
-  float4* s_p = reinterpret_cast<float4*>(smem_i + 3 * kChunk + 3 * 256);
-  float* s_q = reinterpret_cast<float*>(s_p + kChunk);
-  double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]
-  const int nitems = ws.hdr->n_items[kListChunks];
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int2 it = ws.chunks[item];
-    const int b = it.x;
+__global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_sums(const float4* __restrict__ coords,
+                                                                 const float* __restrict__ feats, int F,
+                                                                 int charge_col,
+                                                                 const int64_t* __restrict__ offsets, int K,
+                                                                 const int32_t* __restrict__ labels,
+                                                                 Workspace ws, double* __restrict__ out) {
+  extern __shared__ __align__(16) char smem_c[];
+  const LloydSmem sm = lloyd_smem(smem_c);
+  int q0, q1;
+  pass_range(ws, q0, q1);
+  for (int q = q0; q < q1; ++q) {
+    const int2 it = ws.passes[q];
+    const int b = it.x, i0 = it.y;
     const int fs = ws.fps_slot[b];
     if (fs < 0) continue;  // uniform across the CTA
-    const int64_t off = offsets[b];
-    const int n = (int)(offsets[b + 1] - off);
-    const int i0 = it.y * kChunk, npts = min(n, i0 + kChunk) - i0;
-    const float4* pts = coords + off + i0;
-    const float* fe = feats ? feats + (off + i0) * F : nullptr;
-#pragma unroll 4
-    for (int i = threadIdx.x; i < npts; i += blockDim.x) {
-      int l = labels[off + i0 + i];
-      if ((unsigned)l >= (unsigned)K) {
-        record_error(ws.hdr, kDevBadToken);
-        l = -1;
-      }
-      sm.lab[i] = l;
-      s_p[i] = ldg4(pts + i);
-      s_q[i] = charge_of(fe, F, charge_col, i);
-    }
-    lloyd_chunk_sums(sm, s_p, s_q, npts, K, acc, out + (int64_t)fs * K * 5);
+    const int64_t off = offsets[b] + i0;
+    const int npts = min((int)(offsets[b + 1] - offsets[b]) - i0, kPass);
+    lloyd_piece_sums(coords + off, feats ? feats + off * F : nullptr, F, charge_col, labels + off, npts, K, sm,
+                     out + (int64_t)fs * K * 5, ws.hdr);
     __syncthreads();
   }
 }
 
-// One Lloyd iteration per (event, chunk) item: the centroids from the cell
-// sums `in` (an empty cell or a zero weight keeps its centroid), the nearest
-// of them for the chunk's points (eight per thread, in two passes) and,
-// unless this is the last iteration (next == nullptr), the chunk's cell sums
-// of the new labels added into `next`.  Also clears `clear`, which the
-// following iteration accumulates into.
-constexpr int kLloydThreads = 256;
-constexpr int kLloydPts = kChunk / kLloydThreads;  // points per thread
-static_assert(kLloydPts == 2 * kNearestPairs * kNearestPasses, "chunk_nearest covers the chunk");
-
-static size_t lloyd_step_smem_bytes(int K) {
-  return (size_t)(2 * kChunk + 3 * 256) * sizeof(int) + (size_t)kChunk * (sizeof(float4) + sizeof(float)) +
-         (size_t)K * 5 * sizeof(double) + (size_t)pad_pairs(K) * sizeof(Cent2);
-}
-
+// One Lloyd update and re-assignment: the centroids from the cell sums `in`
+// (an empty cell or a zero weight keeps its centroid), then the nearest of
+// them for every point of the piece.  Also clears `clear`, the buffer that
+// the next k_lloyd_sums accumulates into.
 __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* __restrict__ coords,
                                                                  const float* __restrict__ feats, int F,
                                                                  int charge_col,
@@ -615,116 +768,78 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* _
                                                                  int32_t* __restrict__ labels,
                                                                  float4* __restrict__ centroids, Workspace ws,
                                                                  const double* __restrict__ in,
-                                                                 double* __restrict__ next,
                                                                  double* __restrict__ clear, int64_t clear_n) {
   constexpr int T = kLloydThreads;
-  extern __shared__ int smem_i[];
-  int* perm = smem_i;              // [kChunk]
-  int* slab = perm + kChunk;       // [kChunk]
-  int* cnt = slab + kChunk;        // [256]
-  int* start = cnt + 256;          // [256]
-  int* cur = start + 256;          // [256]
-  float4* s_p = reinterpret_cast<float4*>(cur + 256);  // [kChunk]
-  float* s_q = reinterpret_cast<float*>(s_p + kChunk);  // [kChunk]
-  double* acc = reinterpret_cast<double*>(s_q + kChunk);  // [K * 5]
-  Cent2* s_cent = reinterpret_cast<Cent2*>(acc + K * 5);  // [K]
+  extern __shared__ Cent2 s_cent[];  // [pad_pairs(K)]
   const int tid = threadIdx.x;
   for (int64_t e = (int64_t)blockIdx.x * T + tid; e < clear_n; e += (int64_t)gridDim.x * T) clear[e] = 0.0;
-  const int nitems = ws.hdr->n_items[kListChunks];
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int2 it = ws.chunks[item];
-    const int b = it.x;
+  int q0, q1;
+  pass_range(ws, q0, q1);
+  int cur = -1;
+  for (int q = q0; q < q1; ++q) {
+    const int2 it = ws.passes[q];
+    const int b = it.x, i0 = it.y;
     const int fs = ws.fps_slot[b];
     if (fs < 0) continue;  // uniform across the CTA
-    const int64_t off = offsets[b];
-    const int n = (int)(offsets[b + 1] - off);
-    const double* sb = in + (int64_t)fs * K * 5;
-    for (int j = tid; j < K; j += T) {
-      const double W = __ldcg(&sb[j * 5]);
-      float4 c = centroids[(int64_t)b * K + j];
-      if (W > 0.0) {
-        c.x = (float)(__ldcg(&sb[j * 5 + 1]) / W);
-        c.y = (float)(__ldcg(&sb[j * 5 + 2]) / W);
-        c.z = (float)(__ldcg(&sb[j * 5 + 3]) / W);
-        c.w = (float)(__ldcg(&sb[j * 5 + 4]) / W);
-      }
-      s_cent[j] = cent2(c);
-      if (it.y == 0) centroids[(int64_t)b * K + j] = c;  // every chunk computes the same values
-    }
-    if (tid == 0 && (K & 1)) {
-      const float inf = __int_as_float(0x7f800000);
-      s_cent[K] = cent2(make_float4(inf, inf, inf, inf));
-    }
-    if (next) {
-      for (int j = tid; j < K; j += T) cnt[j] = 0;
-      for (int e = tid; e < K * 5; e += T) acc[e] = 0.0;
-    }
-    __syncthreads();
-    const int i0 = it.y * kChunk, npts = min(n, i0 + kChunk) - i0;
-    const float4* pts = coords + off + i0;
-    int32_t* lab_out = labels + off + i0;
-    const float* fe = feats ? feats + (off + i0) * F : nullptr;
-    chunk_nearest<kNearestPairs, kNearestPasses, T>(pts, npts, s_cent, pad_pairs(K) / 2, [&](int li, int l) {
-      lab_out[li] = l;
-      if (next) {
-        s_p[li] = ldg4(pts + li);  // read a moment ago: a cache hit
-        s_q[li] = charge_of(fe, F, charge_col, li);
-        atomicAdd(&cnt[l], 1);
-      }
-    });
-    if (next) {  // counting sort by label (this thread's own labels, read back), then the cell sums
+    if (b != cur) {  // the event's updated centroids
       __syncthreads();
-      if (tid < 32) count_scan(cnt, start, cur, K, tid);
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < kLloydPts; ++r) {
-        const int li = tid + r * T;
-        if (li < npts) {
-          const int l = lab_out[li];
-          const int pos = atomicAdd(&cur[l], 1);
-          perm[pos] = li;
-          slab[pos] = l;
+      const double* sb = in + (int64_t)fs * K * 5;
+      const bool writer = i0 == 0;  // the event's first pass writes them back (all passes compute the same)
+      for (int j = tid; j < K; j += T) {
+        const double W = __ldcg(&sb[j * 5]);
+        float4 c = centroids[(int64_t)b * K + j];
+        if (W > 0.0) {
+          c.x = (float)(__ldcg(&sb[j * 5 + 1]) / W);
+          c.y = (float)(__ldcg(&sb[j * 5 + 2]) / W);
+          c.z = (float)(__ldcg(&sb[j * 5 + 3]) / W);
+          c.w = (float)(__ldcg(&sb[j * 5 + 4]) / W);
         }
+        s_cent[j] = cent2(c);
+        if (writer) centroids[(int64_t)b * K + j] = c;
+      }
+      if (tid == 0 && (K & 1)) {
+        const float inf = __int_as_float(0x7f800000);
+        s_cent[K] = cent2(make_float4(inf, inf, inf, inf));
       }
       __syncthreads();
-      segment_sums(perm, slab, npts, 5, 0, 5, acc, tid, T, [&](int i, int v) {
-        const double q = (double)s_q[i];
-        if (v == 0) return q;
-        const float4 p = s_p[i];
-        return q * (double)(v == 1 ? p.x : (v == 2 ? p.y : (v == 3 ? p.z : p.w)));
-      });
-      __syncthreads();
-      double* out = next + (int64_t)fs * K * 5;
-      for (int e = tid; e < K * 5; e += T)
-        if (cnt[e / 5]) atomicAdd(&out[e], acc[e]);
+      cur = b;
     }
-    __syncthreads();
+    const int64_t off = offsets[b] + i0;
+    const int npts = min((int)(offsets[b + 1] - offsets[b]) - i0, kPass);
+    int32_t* lab_out = labels + off;
+    chunk_nearest<kNearestPairs, 1, T>(coords + off, npts, s_cent, pad_pairs(K) / 2,
+                                       [&](int li, int l) { lab_out[li] = l; });
   }
 }
 
-// Lloyd refinement: cell sums of the incoming labels into buffer 0, then
-// iteration t updates from buffer t % 3, accumulates the next sums into
-// (t + 1) % 3 unless it is the last one, and clears (t + 2) % 3 when
-// iteration t + 1 will accumulate into it (buffers 0 and 1 start zeroed).
+// Lloyd refinement: cell sums of the incoming labels into buffer 0; then
+// iteration t updates and re-assigns from buffer t % 2 and, unless it is the
+// last one, k_lloyd_sums adds the new labels' cell sums into buffer
+// (t + 1) % 2, which iteration t clears first (from t = 1 on; buffers 0 and
+// 1 start zeroed).
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   const int K = pb.K;
   const float* feats = pb.charge_col >= 0 ? pb.feats : nullptr;
   const int64_t per = (int64_t)K * 5;
+  const int grid = di.sm_count * kPassCtasPerSm;
+  auto sums = [&](double* out) {
+    count_launch();
+    k_lloyd_sums<<<grid, kLloydThreads, lloyd_smem_bytes(K), s>>>(pb.coords, feats, pb.F, pb.charge_col,
+                                                                         pb.offsets, K, labels, ws, out);
+    return cudaGetLastError();
+  };
   cudaError_t e;
-  count_launch();
-  k_lloyd_sums<<<di.sm_count * 2, 256, kLloydSmemBytes, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets,
-                                                             K, labels, ws, ws.lloyd[0]);
-  if ((e = cudaGetLastError())) return e;
-  const size_t sm_step = lloyd_step_smem_bytes(K);
+  if ((e = sums(ws.lloyd[0]))) return e;
   for (int t = 0; t < pb.lloyd_iters; ++t) {
     const bool last = t == pb.lloyd_iters - 1;
-    double* clear = (t + 1 < pb.lloyd_iters - 1) ? ws.lloyd[(t + 2) % 3] : nullptr;
+    double* clear = (t >= 1 && !last) ? ws.lloyd[(t + 1) % 2] : nullptr;
     count_launch();
-    k_lloyd_step<<<di.sm_count * 3, kLloydThreads, sm_step, s>>>(
-        pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels, pb.centroids, ws, ws.lloyd[t % 3],
-        last ? nullptr : ws.lloyd[(t + 1) % 3], clear, clear ? (int64_t)ws.fps_slots * per : 0);
+    k_lloyd_step<<<grid, kLloydThreads, (size_t)pad_pairs(K) * sizeof(Cent2), s>>>(
+        pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels, pb.centroids, ws, ws.lloyd[t % 2], clear,
+        clear ? (int64_t)ws.fps_slots * per : 0);
     if ((e = cudaGetLastError())) return e;
+    if (!last && (e = sums(ws.lloyd[(t + 1) % 2]))) return e;
   }
   return cudaSuccess;
 }
@@ -733,11 +848,10 @@ cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels
 // largest K and F the ABI accepts.
 cudaError_t prepare_aux_kernels() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLloydSmemBytes)))
+  if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)lloyd_smem_bytes(256))))
     return e;
-  if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)lloyd_step_smem_bytes(256))))
-    return e;
+
   const size_t pool_max = pool_smem_bytes(256, 64) > pool_smem_bytes(256, kStageMaxF)
                               ? pool_smem_bytes(256, 64)
                               : pool_smem_bytes(256, kStageMaxF);
@@ -1009,7 +1123,8 @@ cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const fl
   const DeviceInfo& di = device_info();
   const size_t sm = (size_t)pad_pairs(K) * sizeof(Cent2);
   count_launch();
-  k_assign<<<di.sm_count * 4, 256, sm, s>>>(coords, offsets, K, centroids, valid_tokens, token_id, ws);
+  k_assign<<<di.sm_count * kPassCtasPerSm, kAssignThreads, sm, s>>>(coords, offsets, K, centroids, valid_tokens,
+                                                                token_id, ws);
   return cudaGetLastError();
 }
 

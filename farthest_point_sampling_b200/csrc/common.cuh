@@ -70,7 +70,7 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 }
 
 // A centroid broadcast into both halves of four packed registers.
-struct Cent2 {
+struct __align__(16) Cent2 {
   uint64_t x, y, z, t;
 };
 __device__ __forceinline__ Cent2 cent2(float4 c) {

@@ -395,51 +395,62 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
   constexpr int NW = NT / 32;
   constexpr int E = CL * NW;
   constexpr int G = CL * NT;
+  static_assert(CL > 1 || E <= 32, "one warp reads the CTA's warp winners");
+  static_assert(CL == 1 || (CL <= 32 && 2 * CL <= 2 * E - NW), "posts and warp winners do not overlap");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = rank * NT + tid;
 
-  auto post = [&](int key, unsigned idx, float4 pos) {
-    const int slot = (round & 1) * E + rank * NW + warp;
+  // One exchange of (key, index, position) candidates: the event's winner --
+  // largest key, then lowest index -- in M, idx, pos on every thread.
+  // Clusters: the CTA's warp winners meet in shared memory, warp 0 posts the
+  // CTA winner into every CTA of the cluster over DSMEM and arrives on the
+  // cluster barrier with release semantics (the other warps, having written
+  // nothing remote, arrive relaxed), and every warp reads the CL posts after
+  // the acquiring wait.  Posts alternate between two buffers (round & 1): a
+  // CTA cannot post twice ahead of a peer that is still reading.
+  auto exchange = [&](int key, unsigned idx_in, float4 pos_in, int& M, unsigned& idx, float4& pos) {
     if constexpr (CL > 1) {
-      if (lane < CL) {
-        cg::cluster_group cl = cg::this_cluster();
-        int2* rk = cl.map_shared_rank(xkey, lane);
-        float4* rp = cl.map_shared_rank(xpos, lane);
-        rk[slot] = make_int2(key, (int)idx);
-        rp[slot] = pos;
-      }
-    } else {
+      int2* lkey = xkey + 2 * E - NW;  // warp winners (the buffers' tail, unused by the posts)
+      float4* lpos = xpos + 2 * E - NW;
+      const int slot = (round & 1) * CL;
       if (lane == 0) {
-        xkey[slot] = make_int2(key, (int)idx);
-        xpos[slot] = pos;
+        lkey[warp] = make_int2(key, (int)idx_in);
+        lpos[warp] = pos_in;
       }
-    }
-  };
-  auto barrier = [&]() {
-    if constexpr (CL > 1) {
-      cg::this_cluster().sync();
-    } else {
       __syncthreads();
-    }
-  };
-  auto gather = [&](int& M, unsigned& idx, float4& pos) {
-    const int base = (round & 1) * E;
-    int bk = -0x7fffffff - 1;
-    unsigned bi = 0xffffffffu;
-    int be = 0;
-#pragma unroll
-    for (int e = lane; e < E; e += 32) {
-      const int2 v = xkey[base + e];
-      if (v.x > bk || (v.x == bk && (unsigned)v.y < bi)) {
-        bk = v.x;
-        bi = (unsigned)v.y;
-        be = e;
+      if (warp == 0) {
+        const int2 v = lane < NW ? lkey[lane] : make_int2(-0x7fffffff - 1, -1);
+        int cM;
+        unsigned cI;
+        warp_argmax(v.x, (unsigned)v.y, cM, cI);
+        const unsigned who = __ballot_sync(kFull, lane < NW && v.x == cM && (unsigned)v.y == cI);
+        const float4 cp = lpos[__ffs(who) - 1];
+        if (lane < CL) {
+          cg::cluster_group cl = cg::this_cluster();
+          *cl.map_shared_rank(xkey + slot + rank, lane) = make_int2(cM, (int)cI);
+          *cl.map_shared_rank(xpos + slot + rank, lane) = cp;
+        }
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+      } else {
+        asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
       }
+      asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+      const int2 v = lane < CL ? xkey[slot + lane] : make_int2(-0x7fffffff - 1, -1);
+      warp_argmax(v.x, (unsigned)v.y, M, idx);
+      const unsigned who = __ballot_sync(kFull, lane < CL && v.x == M && (unsigned)v.y == idx);
+      pos = xpos[slot + __ffs(who) - 1];
+    } else {
+      const int base = (round & 1) * E;
+      if (lane == 0) {
+        xkey[base + warp] = make_int2(key, (int)idx_in);
+        xpos[base + warp] = pos_in;
+      }
+      __syncthreads();
+      const int2 v = lane < E ? xkey[base + lane] : make_int2(-0x7fffffff - 1, -1);
+      warp_argmax(v.x, (unsigned)v.y, M, idx);
+      const unsigned who = __ballot_sync(kFull, lane < E && v.x == M && (unsigned)v.y == idx);
+      pos = xpos[base + __ffs(who) - 1];
     }
-    warp_argmax(bk, bi, M, idx);
-    const unsigned who = __ballot_sync(kFull, bk == M && bi == idx);
-    const int e = __shfl_sync(kFull, be, __ffs(who) - 1);
-    pos = xpos[base + e];
     ++round;
   };
   auto local_pos = [&](unsigned idx) {
@@ -501,11 +512,9 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
     const unsigned widx = __reduce_min_sync(kFull, wcand);
     float4 wpos = make_float4(0.f, 0.f, 0.f, 0.f);
     if (wM >= 0) wpos = local_pos(widx);
-    post(wM, widx, wpos);
-    barrier();
     int M;
     unsigned idx;
-    gather(M, idx, cc);
+    exchange(wM, widx, wpos, M, idx, cc);
     if (M == 0) {  // only duplicates of chosen points remain
       const unsigned long long mask = 2 * NP >= 64 ? ~0ull : ((1ull << (2 * NP)) - 1ull);
       const unsigned long long free_slots = ~taken & mask;
@@ -515,9 +524,7 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
       float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
       if (wmin != 0xffffffffu) p = local_pos(wmin);
       // keys: 1 for a real candidate, 0 for none; ties resolve to the lowest index
-      post(wmin != 0xffffffffu ? 1 : 0, wmin, p);
-      barrier();
-      gather(M, idx, cc);
+      exchange(wmin != 0xffffffffu ? 1 : 0, wmin, p, M, idx, cc);
     }
     c = (int)idx;
   }
@@ -801,6 +808,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     cudaStream_t hs = ctx.helper[kHelpers - 1];
     if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
     mark(kStagePassthrough, 0, hs);
+    if (pb.assign_mode == 0 && (e = launch_pool_clear(pb, ws, hs))) return e;  // Voronoi mode: the pool kernel may run
     if ((e = launch_passthrough(pt, ws, hs))) return e;
     mark(kStagePassthrough, 1, hs);
     if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;

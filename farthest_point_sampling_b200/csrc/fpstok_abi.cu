@@ -40,9 +40,11 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   Carver c{static_cast<char*>(base)};
   Workspace w = {};
   const int64_t nb = B > 0 ? B : 1;
-  const int64_t chunks = nb + P / kChunk + 1;
+  const int64_t passes = nb + P / kPass + 1;
   const int64_t pool_chunks = nb + P / kPoolChunk + 1;
-  const int64_t pool_slots = P / kPoolChunk + 1;
+  // an event pooled in c > 1 chunks takes min(kPoolReplicas, c) slots: at most
+  // ceil(n / kPoolChunk) <= n / kPoolChunk + 1 with n > kPoolChunk
+  const int64_t pool_slots = 2 * (P / kPoolChunk) + 1;
   int64_t fps_slots = P / (K + 1) + 1;
   if (fps_slots > nb) fps_slots = nb;
   w.hdr = c.take<WsHeader>(1);
@@ -51,15 +53,15 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   w.list_cta_smem = c.take<int>(nb);
   w.list_cluster8 = c.take<int>(nb);
   w.list_cluster16 = c.take<int>(nb);
-  w.chunks = c.take<int2>(chunks);
+  w.passes = c.take<int2>(passes);
   w.pool_chunks = c.take<int2>(pool_chunks);
   w.cls = c.take<int>(nb);
   w.fps_slot = c.take<int>(nb);
   w.pool_slot = c.take<int>(nb);
+  w.pool_event = c.take<int>(nb);
   w.pool_acc = c.take<double>(pool_slots * K * (F > 0 ? F : 1));
   w.pool_cnt = c.take<int>(pool_slots * K);
-  w.pool_ticket = c.take<int>(pool_slots);
-  for (int i = 0; i < 3; ++i) w.lloyd[i] = lloyd ? c.take<double>(fps_slots * K * 5) : nullptr;
+  for (int i = 0; i < 2; ++i) w.lloyd[i] = lloyd ? c.take<double>(fps_slots * K * 5) : nullptr;
   w.labels = labels ? c.take<int>(P > 0 ? P : 1) : nullptr;
   w.fps_slots = (int)fps_slots;
   w.pool_slots = (int)pool_slots;
@@ -131,7 +133,7 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
                            (pb.fused_pool & 3) == 3;
     if (!none_left) {
       stage_mark(8, 0, s);
-      if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.K, labels, pb.pooled, pb.counts, ws, s)))
+      if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.B, pb.K, labels, pb.pooled, pb.counts, ws, s)))
         return from_cuda(e);
       stage_mark(8, 1, s);
     }
@@ -417,10 +419,9 @@ int segment_pool(const float* feats, int F, const int64_t* offsets, int B, int64
     return from_cuda(e);
   if ((e = launch_bin(pb, ws, 1, s))) return from_cuda(e);
   if ((e = cudaMemsetAsync(ws.pool_acc, 0, (size_t)ws.pool_slots * K * F * sizeof(double), s)) ||
-      (e = cudaMemsetAsync(ws.pool_cnt, 0, (size_t)ws.pool_slots * K * sizeof(int), s)) ||
-      (e = cudaMemsetAsync(ws.pool_ticket, 0, (size_t)ws.pool_slots * sizeof(int), s)))
+      (e = cudaMemsetAsync(ws.pool_cnt, 0, (size_t)ws.pool_slots * K * sizeof(int), s)))
     return from_cuda(e);
-  return from_cuda(launch_pool_voronoi(feats, F, offsets, K, token_id, pooled, counts, ws, s));
+  return from_cuda(launch_pool_voronoi(feats, F, offsets, B, K, token_id, pooled, counts, ws, s));
 }
 
 int fps_device_status(void* workspace, fps_stream_t stream, int* detail) {

@@ -16,11 +16,12 @@ enum ListId : int {
   kListCtaSmem = 2,
   kListCluster8 = 3,
   kListCluster16 = 4,
-  kListChunks = 5,      // (event, chunk) items of FPS events (Lloyd, assignment)
-  kListPoolSlots = 6,   // events that need global pooling accumulators
+  kListChunks = 5,      // nearest-centroid passes over FPS events (Lloyd, assignment)
+  kListPoolSlots = 6,   // global pooling accumulator slots in use
   kListFps = 7,         // number of FPS events (Lloyd slots)
   kListPoolChunks = 8,  // (event, chunk) items of the events k_pool_voronoi pools
-  kNumLists = 9,
+  kListPoolEvents = 9,  // events pooled in several chunks (k_pool_finalize)
+  kNumLists = 10,
 };
 constexpr int kNumSchedules = 5;  // warp, CTA, CTA-smem, 8-CTA cluster, 16-CTA cluster
 constexpr int kStagePassthrough = 9;  // stage id of the passthrough kernel (helper stream)
@@ -38,8 +39,10 @@ constexpr int kCtaSmemCap = kBlockThreads * 2 * kBlockPairs;  // 12288
 constexpr int kCluster8Cap = 8 * kCtaSmemCap;                 // 98304
 constexpr int kMaxCluster = 16;
 constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
-constexpr int kChunk = 2048;                           // points per Lloyd / assignment work item
+constexpr int kPass = 1024;                            // points per Lloyd / assignment pass (256 threads x 4)
+constexpr int kPassCtasPerSm = 3;                      // resident CTAs per SM of the pass kernels
 constexpr int kPoolChunk = 512;                        // points per pooling work item
+constexpr int kPoolReplicas = 16;                      // accumulator copies per event pooled in several chunks
 // With at most this many FPS events per SM, events of the warp class run on
 // the CTA schedule instead (lower latency per step when the GPU is not full).
 constexpr int kLatencyEventsPerSm = 1;
@@ -51,15 +54,15 @@ struct Workspace {
   int* list_cta_smem;
   int* list_cluster8;
   int* list_cluster16;
-  int2* chunks;     // (event, chunk) items of FPS events
+  int2* passes;     // (event, first point) of every nearest-centroid pass, in batch order
   int2* pool_chunks; // (event, chunk) items of events pooled by the pool kernel
   int* cls;         // EventClass per event
   int* fps_slot;    // compact index of FPS events, -1 otherwise
-  int* pool_slot;   // compact index of multi-chunk FPS events, -1 otherwise
+  int* pool_slot;   // first accumulator slot of events pooled in several chunks, -1 otherwise
+  int* pool_event;  // [events] the events pooled in several chunks
   double* pool_acc; // [pool slots][K][F]
   int* pool_cnt;    // [pool slots][K]
-  int* pool_ticket; // [pool slots]
-  double* lloyd[3]; // 3 x [fps slots][K][5] cell sums (W, S_x, S_y, S_z, S_t)
+  double* lloyd[2]; // 2 x [fps slots][K][5] cell sums (W, S_x, S_y, S_z, S_t)
   int* labels;      // [P] internal Voronoi labels (kNN mode with Lloyd)
   int fps_slots;    // capacity of the Lloyd slot range
   int pool_slots;   // capacity of the pooling slot range
@@ -86,6 +89,7 @@ struct Problem {
 
 // Kernel launchers (return the cudaError_t of the launch).
 cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s);
+cudaError_t launch_pool_clear(const Problem& pb, const Workspace& ws, cudaStream_t s);
 cudaError_t launch_passthrough(const Problem& pb, const Workspace& ws, cudaStream_t s);
 typedef void (*StageMark)(int stage, int end, cudaStream_t s);
 void stage_mark(int stage, int end, cudaStream_t s);
@@ -97,7 +101,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
 size_t warp_region_bytes();
 size_t cta_region_bytes();
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s);
-cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int K,
+cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int B, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,
                                 const Workspace& ws, cudaStream_t s);
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
