@@ -30,6 +30,7 @@ constexpr int kDevBadOffsets = 1;
 constexpr int kDevBadStart = 2;
 constexpr int kDevBadToken = 3;
 constexpr int kDevTooLarge = 4;
+constexpr int kDevExchangeTimeout = 5;
 
 // Workspace header: status word, detail word, work-list sizes and the
 // cursors the persistent kernels take items from (all reset by the binning

@@ -381,6 +381,55 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
 
 // ------------------------------------------------------------------ CTA / cluster, points in shared memory
 
+// DSMEM exchange primitives of the cluster schedules: stores into a peer's
+// shared memory that signal the peer's mbarrier with their byte count, and a
+// bounded wait on the local mbarrier.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void st_async_v4(uint32_t addr, int a, int b, int c, int d, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t addr, int a, int b, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(addr), "r"(a),
+               "r"(b), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// try_wait already suspends in hardware between polls; this many polls is
+// far beyond any real exchange (microseconds), and ends a wait that a fault
+// elsewhere would otherwise leave spinning.
+constexpr int kExchangeSpinLimit = 1 << 20;
+
+// Slot of one posted candidate: (key, index, x, y) and (z, t).
+struct __align__(16) ExSlot {
+  int4 a;
+  int2 b;
+  int2 pad;
+};
+constexpr uint32_t kExSlotBytes = 24;  // bytes each post carries (16 + 8)
+
 template <int CL, int NT>
 struct BlockShared {
   static constexpr int NW = NT / 32;
@@ -390,7 +439,8 @@ struct BlockShared {
 template <int NP, int CL, int NT>
 __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                             int rank, ulonglong2* sXY, ulonglong2* sZT, int2* xkey, float4* xpos,
-                                            int& round, int32_t* __restrict__ cidx, float4* __restrict__ cpos,
+                                            ExSlot* xslot, uint64_t* xbar, WsHeader* hdr, int& round,
+                                            int32_t* __restrict__ cidx, float4* __restrict__ cpos,
                                             int32_t* __restrict__ tok) {
   constexpr int NW = NT / 32;
   constexpr int E = CL * NW;
@@ -402,17 +452,24 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
 
   // One exchange of (key, index, position) candidates: the event's winner --
   // largest key, then lowest index -- in M, idx, pos on every thread.
-  // Clusters: the CTA's warp winners meet in shared memory, warp 0 posts the
-  // CTA winner into every CTA of the cluster over DSMEM and arrives on the
-  // cluster barrier with release semantics (the other warps, having written
-  // nothing remote, arrive relaxed), and every warp reads the CL posts after
-  // the acquiring wait.  Posts alternate between two buffers (round & 1): a
-  // CTA cannot post twice ahead of a peer that is still reading.
+  // Clusters: the CTA's warp winners meet in shared memory; warp 0 sends the
+  // CTA winner into slot `rank` of every CTA with st.async, which signals the
+  // receiving CTA's mbarrier with its bytes; every thread waits (bounded) on
+  // its own mbarrier for the CL posts and reads them.  No cluster barrier and
+  // no release fence.  Rounds alternate between two slot sets and mbarriers
+  // (round & 1; phase parity (round >> 1) & 1): a CTA cannot post round r + 2
+  // before every peer has posted round r + 1, which each does after reading
+  // round r.  Posts arriving before the local arm are counted in the same
+  // phase (it cannot complete before the local arrival).
   auto exchange = [&](int key, unsigned idx_in, float4 pos_in, int& M, unsigned& idx, float4& pos) {
     if constexpr (CL > 1) {
-      int2* lkey = xkey + 2 * E - NW;  // warp winners (the buffers' tail, unused by the posts)
+      int2* lkey = xkey + 2 * E - NW;  // warp winners
       float4* lpos = xpos + 2 * E - NW;
-      const int slot = (round & 1) * CL;
+      const int p = round & 1;
+      const uint32_t parity = (uint32_t)(round >> 1) & 1u;
+      ExSlot* slots = xslot + p * CL;
+      const uint32_t bar = smem_addr(&xbar[p]);
+      if (tid == 0) mbar_arrive_expect(bar, CL * kExSlotBytes);  // this round: CL posts
       if (lane == 0) {
         lkey[warp] = make_int2(key, (int)idx_in);
         lpos[warp] = pos_in;
@@ -425,20 +482,25 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
         warp_argmax(v.x, (unsigned)v.y, cM, cI);
         const unsigned who = __ballot_sync(kFull, lane < NW && v.x == cM && (unsigned)v.y == cI);
         const float4 cp = lpos[__ffs(who) - 1];
-        if (lane < CL) {
-          cg::cluster_group cl = cg::this_cluster();
-          *cl.map_shared_rank(xkey + slot + rank, lane) = make_int2(cM, (int)cI);
-          *cl.map_shared_rank(xpos + slot + rank, lane) = cp;
+        if (lane < CL) {  // the CTA winner into slot `rank` of every CTA, signalling its barrier
+          const uint32_t ra = peer_addr(smem_addr(&slots[rank]), lane);
+          const uint32_t rb = peer_addr(bar, lane);
+          st_async_v4(ra, cM, (int)cI, __float_as_int(cp.x), __float_as_int(cp.y), rb);
+          st_async_v2(ra + 16, __float_as_int(cp.z), __float_as_int(cp.w), rb);
         }
-        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-      } else {
-        asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
       }
-      asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-      const int2 v = lane < CL ? xkey[slot + lane] : make_int2(-0x7fffffff - 1, -1);
+      bool ok = false;
+      for (int it = 0; it < kExchangeSpinLimit && !ok; ++it) ok = mbar_try_wait(bar, parity);
+      if (!ok && tid == 0) record_error(hdr, kDevExchangeTimeout);  // carry on: control flow stays uniform
+      int2 v = make_int2(-0x7fffffff - 1, -1);
+      if (lane < CL) {
+        const int4 a = slots[lane].a;
+        v = make_int2(a.x, a.y);
+      }
       warp_argmax(v.x, (unsigned)v.y, M, idx);
       const unsigned who = __ballot_sync(kFull, lane < CL && v.x == M && (unsigned)v.y == idx);
-      pos = xpos[slot + __ffs(who) - 1];
+      const ExSlot& w = slots[__ffs(who) - 1];
+      pos = make_float4(__int_as_float(w.a.z), __int_as_float(w.a.w), __int_as_float(w.b.x), __int_as_float(w.b.y));
     } else {
       const int base = (round & 1) * E;
       if (lane == 0) {
@@ -562,12 +624,19 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
   ulonglong2* sZT = sXY + PS * NT;                            // [PS][NT] packed (z, t)
   int2* xkey = reinterpret_cast<int2*>(sZT + PS * NT);        // [2][E] (key, index)
   float4* xpos = reinterpret_cast<float4*>(xkey + 2 * E);     // [2][E] candidate position
+  ExSlot* xslot = reinterpret_cast<ExSlot*>(xpos + 2 * E);    // [2][CL] posted CTA winners
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(xslot + 2 * CL);  // [2] exchange mbarriers
   __shared__ int s_item;
 
   int rank = 0;
   if constexpr (CL > 1) {
     rank = (int)cg::this_cluster().block_rank();
-    cg::this_cluster().sync();  // every CTA of the cluster is running before DSMEM use
+    if (threadIdx.x == 0) {
+      mbar_init(smem_addr(&xbar[0]), 1);
+      mbar_init(smem_addr(&xbar[1]), 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    cg::this_cluster().sync();  // every CTA is running, its barriers initialised, before DSMEM use
   }
   const int count = hdr->n_items[list_id];
   int round = 0;
@@ -594,7 +663,7 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     int32_t* tok = token_id ? token_id + off : nullptr;
     const int np = (n + 2 * G - 1) / (2 * G);
 #define BLOCK_CALL(N)                                                                                   \
-  block_event<N, CL, NT>(coords + off, n, c0, K, off, rank, sXY, sZT, xkey, xpos, round,                \
+  block_event<N, CL, NT>(coords + off, n, c0, K, off, rank, sXY, sZT, xkey, xpos, xslot, xbar, hdr, round, \
                          centroid_idx + (int64_t)b * K, centroids + (int64_t)b * K, tok)
     FPS_BLOCK_BUCKETS(np, BLOCK_CALL)
 #undef BLOCK_CALL
@@ -620,7 +689,8 @@ size_t cta_region_bytes() { return kCtaSmem; }
 template <int CL>
 constexpr size_t block_smem_bytes() {
   return (size_t)2 * kBlockPairs * kBlockThreads * sizeof(ulonglong2) +
-         (size_t)2 * BlockShared<CL, kBlockThreads>::E * (sizeof(int2) + sizeof(float4));
+         (size_t)2 * BlockShared<CL, kBlockThreads>::E * (sizeof(int2) + sizeof(float4)) +
+         (size_t)2 * CL * sizeof(ExSlot) + 2 * sizeof(uint64_t);
 }
 
 template <int CL>

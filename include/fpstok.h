@@ -217,6 +217,9 @@ int fps_device_status(void *workspace, fps_stream_t stream, int *detail);
 #define FPS_DEV_BAD_START 2
 #define FPS_DEV_BAD_TOKEN 3
 #define FPS_DEV_TOO_LARGE 4
+/* A cluster FPS kernel gave up waiting for its peers' candidates (a bounded
+ * wait ran out); that launch's results are not valid. */
+#define FPS_DEV_EXCHANGE_TIMEOUT 5
 
 /* Human-readable name of a status code. */
 const char *fps_status_string(int status);
