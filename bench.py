@@ -419,6 +419,8 @@ def main():
     sched = np.array([lib.fps_schedule_for(int(n), batch.K, -1) for n in sizes])
     if (sched >= 0).sum() <= SM_COUNT:  # few events: the warp class runs on the CTA schedule
         sched = np.where(sched == 0, 1, sched)
+    if (sched == 2).sum() <= SM_COUNT // 8:  # few mid-size events: 8-CTA clusters
+        sched = np.where(sched == 2, 3, sched)
     ran = {0, 9, 8 if batch.assign_mode == 0 else 7}
     ran |= {1 + s for s in (0, 1, 2, 3, 4) if (sched == s).any()}
     if batch.lloyd_iters:

@@ -83,10 +83,10 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* tmp, int& total) {
 __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
                                                int force, int chunk_all, int fused_pool, int latency_events,
-                                               int need_passes, Workspace ws) {
+                                               int mid_cluster_events, int need_passes, Workspace ws) {
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
-  __shared__ int n_fps;
+  __shared__ int n_fps, n_mid;
   __shared__ int s_n[kBinCache];  // event sizes (cls in the sign: -1 - cls for non-FPS events)
   for (int i = threadIdx.x; i < kNumSchedules * kBins; i += blockDim.x) (&hist[0][0])[i] = 0;
   if (threadIdx.x < kNumLists) cnt[threadIdx.x] = 0;
@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     ws.hdr->status = 0;
     ws.hdr->detail = 0;
     n_fps = 0;
+    n_mid = 0;
   }
   __syncthreads();
   // pass 1: classify and count FPS events (four events per thread in flight)
@@ -135,6 +136,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
             cls = kClsSkip;
           } else {
             atomicAdd(&n_fps, 1);
+            if (n > kCtaCap && n <= kCtaSmemCap) atomicAdd(&n_mid, 1);
           }
         }
       }
@@ -144,9 +146,14 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
   }
   __syncthreads();
   const bool few = n_fps <= latency_events;
+  // few mid-size events: an 8-CTA cluster each (one pair per thread, the
+  // step bound by the cluster exchange) instead of one CTA reading 10+
+  // pairs per thread from shared memory; only under automatic scheduling
+  const bool few_mid = force < 0 && n_mid <= mid_cluster_events;
   auto schedule_of = [&](int n) {
     int q = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : (n <= kCluster8Cap ? 3 : 4)));
     if (q == 0 && few) q = 1;  // few events: lower latency per step on a whole CTA
+    if (q == 2 && few_mid) q = 3;
     if (force > q) q = force > 4 ? 4 : force;
     return q;
   };
@@ -247,7 +254,7 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
   count_launch();
   const int need_passes = chunk_all || pb.lloyd_iters > 0;
   k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
-                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, need_passes, ws);
+                           pb.fused_pool, kLatencyEventsPerSm * di.sm_count, di.sm_count / 8, need_passes, ws);
   return cudaGetLastError();
 }
 

@@ -822,7 +822,9 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
   const int hint = pb.max_event_hint;
   const int f = pb.force_schedule;
   const bool maybe_few = pb.B <= kLatencyEventsPerSm * di.sm_count;  // small events may move to the CTA
-  const int lower[kNumSchedules] = {pb.K, maybe_few ? pb.K : kWarpCap, kCtaCap, kCtaSmemCap, kCluster8Cap};
+  // (the 8-CTA cluster also takes mid-size events when there are few of them)
+  const int lower[kNumSchedules] = {pb.K, maybe_few ? pb.K : kWarpCap, kCtaCap, f < 0 ? kCtaCap : kCtaSmemCap,
+                                    kCluster8Cap};
   bool run[kNumSchedules];
   for (int q = 0; q < kNumSchedules; ++q) {
     const int lo = f >= q ? pb.K : lower[q];

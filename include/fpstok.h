@@ -243,8 +243,10 @@ void fps_set_stage_events(void *const *events, int n_events);
 
 /* Schedule fps_tokenize gives an event of n points: -1 none (n <= K, or n = 0),
  * 0 warp, 1 CTA, 2 CTA shared-memory, 3 8-CTA cluster, 4 16-CTA cluster; -2
- * if n exceeds fps_max_event_points().  When a batch has at most one FPS event
- * per SM, events of class 0 run on schedule 1 instead. */
+ * if n exceeds fps_max_event_points().  Two batch-level rules apply on top
+ * (automatic scheduling only): when a batch has at most one FPS event per SM,
+ * events of class 0 run on schedule 1; when it has at most one class-2 event
+ * per 8 SMs, those run on schedule 3. */
 int fps_schedule_for(int64_t n, int K, int force_schedule);
 
 #ifdef __cplusplus
