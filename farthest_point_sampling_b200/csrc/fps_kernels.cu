@@ -314,7 +314,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       if (i < n) tok[i] = lab[j];
     }
   }
-  if (po.feats) {  // token means: sort by token, balanced float64 sums over the event copy's space
+  if (po.feats) {  // token means: sort by token, then one thread per (token, feature) over its run
     constexpr int NMAX = 2 * NT * kMaxPairsCta;
     const int F = po.F;
     __syncthreads();
@@ -322,8 +322,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     int* perm = s_lab + NMAX;
     int* slab = perm + NMAX;
     int* cnt = slab + NMAX;  // cnt, start, cur: 3 x 256
-    float* s_feat = reinterpret_cast<float*>(cnt + 768);        // [n * F]
-    double* acc = reinterpret_cast<double*>(s_feat + NMAX * F);  // [K * F]
+    float* s_feat = reinterpret_cast<float*>(cnt + 768);  // [n * F]
 #pragma unroll
     for (int j = 0; j < 2 * NP; ++j) {
       const int i = j * NT + tid;
@@ -332,17 +331,25 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     const float* fe = po.feats + off * F;
 #pragma unroll 16
     for (int e = tid; e < n * F; e += NT) s_feat[e] = __ldg(fe + e);
-    for (int e = tid; e < K * F; e += NT) acc[e] = 0.0;
     label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, slab, tid, NT, [] { __syncthreads(); });
-    for (int v0 = 0; v0 < F; v0 += 8)
-      segment_sums(perm, slab, n, min(8, F - v0), v0, F, acc, tid, NT,
-                   [&](int i, int f) { return (double)s_feat[i * F + f]; });
-    __syncthreads();
-    for (int j = tid; j < K; j += NT) {
+    // the token's points are perm[start .. start + c): four independent float64
+    // partial sums per value, then the mean; no atomics, no accumulator array
+    const int* start = cnt + 256;
+    for (int q = tid; q < K * F; q += NT) {
+      const int j = q / F, f = q - j * F;
       const int c = cnt[j];
-      float* prow = po.pooled + (b * K + j) * F;
-      for (int f = 0; f < F; ++f) prow[f] = c ? (float)(acc[j * F + f] / (double)c) : 0.f;
-      po.counts[b * K + j] = c;
+      const int* pj = perm + start[j];
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      int t = 0;
+      for (; t + 4 <= c; t += 4) {
+        s0 += (double)s_feat[pj[t] * F + f];
+        s1 += (double)s_feat[pj[t + 1] * F + f];
+        s2 += (double)s_feat[pj[t + 2] * F + f];
+        s3 += (double)s_feat[pj[t + 3] * F + f];
+      }
+      for (; t < c; ++t) s0 += (double)s_feat[pj[t] * F + f];
+      po.pooled[(b * K + j) * F + f] = c ? (float)(((s0 + s1) + (s2 + s3)) / (double)c) : 0.f;
+      if (f == 0) po.counts[b * K + j] = c;
     }
   }
 }

@@ -188,8 +188,7 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
   if (opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0) {
     const size_t K = (size_t)opts->K, Fz = (size_t)F;
     if (K * Fz * sizeof(double) + K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
-    if ((size_t)(3 * kCtaCap + 768) * sizeof(int) + (size_t)kCtaCap * Fz * sizeof(float) +
-            K * Fz * sizeof(double) <= cta_region_bytes())
+    if ((size_t)(3 * kCtaCap + 768) * sizeof(int) + (size_t)kCtaCap * Fz * sizeof(float) <= cta_region_bytes())
       pb.fused_pool |= 2;
   }
   return run_tokenize(pb, ws, reinterpret_cast<cudaStream_t>(stream));
