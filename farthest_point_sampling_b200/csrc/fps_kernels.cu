@@ -328,10 +328,18 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       const int i = j * NT + tid;
       if (i < n) s_lab[i] = lab[j];
     }
+    // feature rows into shared memory by asynchronous copies, in flight while
+    // the labels are sorted; each thread waits for its own before the barrier
     const float* fe = po.feats + off * F;
-#pragma unroll 16
-    for (int e = tid; e < n * F; e += NT) s_feat[e] = __ldg(fe + e);
+    const uint32_t s_feat0 = (uint32_t)__cvta_generic_to_shared(s_feat);
+#pragma unroll 8
+    for (int e = tid; e < n * F; e += NT)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s_feat0 + 4u * (uint32_t)e), "l"(fe + e)
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
     label_sort(s_lab, n, K, cnt, cnt + 256, cnt + 512, perm, slab, tid, NT, [] { __syncthreads(); });
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
     // the token's points are perm[start .. start + c): four independent float64
     // partial sums per value, then the mean; no atomics, no accumulator array
     const int* start = cnt + 256;
