@@ -350,6 +350,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     launches0 = fps.launch_count()
+    stage_mask = 0  # stages the library actually ran (host-side record of its stage marks)
     wall0 = time.perf_counter()
     with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as clocks:
         for i in range(K):
@@ -358,6 +359,7 @@ def main():
             starts[i].record(stream)
             step()
             ends[i].record(stream)
+            stage_mask |= lib.fps_stage_mask()
         lib.fps_set_stage_events(None, 0)
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - wall0
@@ -421,10 +423,7 @@ def main():
         sched = np.where(sched == 0, 1, sched)
     if (sched == 2).sum() <= SM_COUNT // 8:  # few mid-size events: 8-CTA clusters
         sched = np.where(sched == 2, 3, sched)
-    ran = {0, 9, 8 if batch.assign_mode == 0 else 7}
-    ran |= {1 + s for s in (0, 1, 2, 3, 4) if (sched == s).any()}
-    if batch.lloyd_iters:
-        ran.add(6)
+    ran = {s for s in range(len(STAGES)) if (stage_mask >> s) & 1}
     stage_ms = {s: v for s, v in stage_ms.items() if s in ran}
 
     result = {

@@ -47,6 +47,7 @@ SIGNATURES = [
     ("fps_status_string", ctypes.c_char_p, [I]),
     ("fps_launch_count", ctypes.c_uint64, []),
     ("fps_set_stage_events", None, [ctypes.POINTER(P), I]),
+    ("fps_stage_mask", ctypes.c_uint, []),
     ("fps_schedule_for", I, [I64, I, I]),
 ]
 

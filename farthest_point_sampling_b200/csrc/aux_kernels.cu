@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps, n_mid;
-  __shared__ int s_n[kBinCache];  // event sizes (cls in the sign: -1 - cls for non-FPS events)
+  __shared__ int s_n[kBinCache];              // event sizes (-1 for events that are neither FPS nor passthrough)
+  __shared__ signed char s_cls[kBinCache];    // event classes, so later passes need no global re-reads
   for (int i = threadIdx.x; i < kNumSchedules * kBins; i += blockDim.x) (&hist[0][0])[i] = 0;
   if (threadIdx.x < kNumLists) cnt[threadIdx.x] = 0;
   if (threadIdx.x < 8) ws.hdr->next_item[threadIdx.x] = 0;
@@ -141,7 +142,10 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
         }
       }
       ws.cls[b] = cls;
-      if (b < kBinCache) s_n[b] = cls == kClsFps || cls == kClsPass ? (int)n : -1;
+      if (b < kBinCache) {
+        s_n[b] = cls == kClsFps || cls == kClsPass ? (int)n : -1;
+        s_cls[b] = (signed char)cls;
+      }
     }
   }
   __syncthreads();
@@ -158,9 +162,10 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     return q;
   };
   auto size_of = [&](int b) { return b < kBinCache ? s_n[b] : (int)(offsets[b + 1] - offsets[b]); };
+  auto cls_of = [&](int b) { return b < kBinCache ? (int)s_cls[b] : ws.cls[b]; };
   // pass 2: size histogram per schedule
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    if (ws.cls[b] != kClsFps) continue;
+    if (cls_of(b) != kClsFps) continue;
     const int n = size_of(b);
     const int q = schedule_of(n);
     atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1);
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
   // once per warp (warp_reserve) rather than once per event.
   for (int b0 = 0; b0 < B; b0 += blockDim.x) {
     const int b = b0 + threadIdx.x;
-    const int cls = b < B ? ws.cls[b] : kClsSkip;
+    const int cls = b < B ? cls_of(b) : kClsSkip;
     int n = 0;
     if (cls == kClsFps || cls == kClsPass) n = size_of(b);
     const int q = cls == kClsFps ? schedule_of(n) : 0;
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     const int b = b0 + threadIdx.x;
     int n = 0;
     if (b < B) {
-      const int cls = ws.cls[b];
+      const int cls = cls_of(b);
       if (cls == kClsFps || (chunk_all && cls == kClsPass)) n = size_of(b);
     }
     const int np = (n + kPass - 1) / kPass;
@@ -663,6 +668,11 @@ static size_t lloyd_smem_bytes(int K) {
   return (size_t)(2 * kPass + 3 * 256) * sizeof(int) + (size_t)kPass * (sizeof(float4) + sizeof(float)) +
          (size_t)K * 5 * sizeof(double);
 }
+// The update kernel keeps its centroids after that region, 16-byte aligned.
+__host__ __device__ constexpr size_t lloyd_cent_offset(int K) {
+  return ((size_t)(2 * kPass + 3 * 256) * sizeof(int) + (size_t)kPass * (sizeof(float4) + sizeof(float)) +
+          (size_t)K * 5 * sizeof(double) + 15) & ~(size_t)15;
+}
 __device__ __forceinline__ LloydSmem lloyd_smem(char* base) {
   LloydSmem m;
   m.perm = reinterpret_cast<int*>(base);
@@ -764,10 +774,11 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_sums(const float4* _
   }
 }
 
-// One Lloyd update and re-assignment: the centroids from the cell sums `in`
-// (an empty cell or a zero weight keeps its centroid), then the nearest of
-// them for every point of the piece.  Also clears `clear`, the buffer that
-// the next k_lloyd_sums accumulates into.
+// One Lloyd iteration: the centroids from the cell sums `in` (an empty cell
+// or a zero weight keeps its centroid), the nearest of them for every point
+// of the pass and, unless this is the last iteration (next == nullptr), the
+// pass's cell sums of the new labels added into `next`.  Also clears `clear`,
+// the buffer the following iteration accumulates into.
 __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* __restrict__ coords,
                                                                  const float* __restrict__ feats, int F,
                                                                  int charge_col,
@@ -775,9 +786,12 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* _
                                                                  int32_t* __restrict__ labels,
                                                                  float4* __restrict__ centroids, Workspace ws,
                                                                  const double* __restrict__ in,
+                                                                 double* __restrict__ next,
                                                                  double* __restrict__ clear, int64_t clear_n) {
   constexpr int T = kLloydThreads;
-  extern __shared__ Cent2 s_cent[];  // [pad_pairs(K)]
+  extern __shared__ __align__(16) char smem_c[];
+  const LloydSmem sm = lloyd_smem(smem_c);
+  Cent2* s_cent = reinterpret_cast<Cent2*>(smem_c + lloyd_cent_offset(K));  // [pad_pairs(K)]
   const int tid = threadIdx.x;
   for (int64_t e = (int64_t)blockIdx.x * T + tid; e < clear_n; e += (int64_t)gridDim.x * T) clear[e] = 0.0;
   int q0, q1;
@@ -816,37 +830,39 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* _
     int32_t* lab_out = labels + off;
     chunk_nearest<kNearestPairs, 1, T>(coords + off, npts, s_cent, pad_pairs(K) / 2,
                                        [&](int li, int l) { lab_out[li] = l; });
+    if (next) {  // this thread's own labels, read back
+      lloyd_piece_sums(coords + off, feats ? feats + off * F : nullptr, F, charge_col, lab_out, npts, K, sm,
+                       next + (int64_t)fs * K * 5, ws.hdr);
+      __syncthreads();  // the next pass re-zeroes the sums
+    }
   }
 }
 
-// Lloyd refinement: cell sums of the incoming labels into buffer 0; then
-// iteration t updates and re-assigns from buffer t % 2 and, unless it is the
-// last one, k_lloyd_sums adds the new labels' cell sums into buffer
-// (t + 1) % 2, which iteration t clears first (from t = 1 on; buffers 0 and
-// 1 start zeroed).
+// Lloyd refinement: cell sums of the incoming labels into buffer 0, then
+// iteration t updates from buffer t % 3, accumulates the next sums into
+// (t + 1) % 3 unless it is the last one, and clears (t + 2) % 3 when
+// iteration t + 1 will accumulate into it (buffers 0 and 1 start zeroed).
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s) {
   const DeviceInfo& di = device_info();
   const int K = pb.K;
   const float* feats = pb.charge_col >= 0 ? pb.feats : nullptr;
   const int64_t per = (int64_t)K * 5;
   const int grid = di.sm_count * kPassCtasPerSm;
-  auto sums = [&](double* out) {
-    count_launch();
-    k_lloyd_sums<<<grid, kLloydThreads, lloyd_smem_bytes(K), s>>>(pb.coords, feats, pb.F, pb.charge_col,
-                                                                         pb.offsets, K, labels, ws, out);
-    return cudaGetLastError();
-  };
   cudaError_t e;
-  if ((e = sums(ws.lloyd[0]))) return e;
+  count_launch();
+  k_lloyd_sums<<<grid, kLloydThreads, lloyd_smem_bytes(K), s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets,
+                                                                 K, labels, ws, ws.lloyd[0]);
+  if ((e = cudaGetLastError())) return e;
+  const size_t sm_step = lloyd_cent_offset(K) + (size_t)pad_pairs(K) * sizeof(Cent2);
   for (int t = 0; t < pb.lloyd_iters; ++t) {
     const bool last = t == pb.lloyd_iters - 1;
-    double* clear = (t >= 1 && !last) ? ws.lloyd[(t + 1) % 2] : nullptr;
+    double* clear = (t + 1 < pb.lloyd_iters - 1) ? ws.lloyd[(t + 2) % 3] : nullptr;
     count_launch();
-    k_lloyd_step<<<grid, kLloydThreads, (size_t)pad_pairs(K) * sizeof(Cent2), s>>>(
-        pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels, pb.centroids, ws, ws.lloyd[t % 2], clear,
-        clear ? (int64_t)ws.fps_slots * per : 0);
+    k_lloyd_step<<<grid, kLloydThreads, sm_step, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels,
+                                                      pb.centroids, ws, ws.lloyd[t % 3],
+                                                      last ? nullptr : ws.lloyd[(t + 1) % 3], clear,
+                                                      clear ? (int64_t)ws.fps_slots * per : 0);
     if ((e = cudaGetLastError())) return e;
-    if (!last && (e = sums(ws.lloyd[(t + 1) % 2]))) return e;
   }
   return cudaSuccess;
 }
@@ -857,6 +873,9 @@ cudaError_t prepare_aux_kernels() {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(k_lloyd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)lloyd_smem_bytes(256))))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_lloyd_step, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(lloyd_cent_offset(256) + (size_t)pad_pairs(256) * sizeof(Cent2)))))
     return e;
 
   const size_t pool_max = pool_smem_bytes(256, 64) > pool_smem_bytes(256, kStageMaxF)

@@ -16,8 +16,11 @@ void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_r
 static void* g_stage_events[32];
 static int g_n_stage_events = 0;
 
+static unsigned g_stage_mask;  // stages marked since the last fps_set_stage_events
+
 void stage_mark(int stage, int end, cudaStream_t s) {
   const int e = 2 * stage + end;
+  if (!end) g_stage_mask |= 1u << stage;
   if (e < g_n_stage_events && g_stage_events[e])
     cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_stage_events[e]), s);
 }
@@ -61,7 +64,7 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
   w.pool_event = c.take<int>(nb);
   w.pool_acc = c.take<double>(pool_slots * K * (F > 0 ? F : 1));
   w.pool_cnt = c.take<int>(pool_slots * K);
-  for (int i = 0; i < 2; ++i) w.lloyd[i] = lloyd ? c.take<double>(fps_slots * K * 5) : nullptr;
+  for (int i = 0; i < 3; ++i) w.lloyd[i] = lloyd ? c.take<double>(fps_slots * K * 5) : nullptr;
   w.labels = labels ? c.take<int>(P > 0 ? P : 1) : nullptr;
   w.fps_slots = (int)fps_slots;
   w.pool_slots = (int)pool_slots;
@@ -453,6 +456,7 @@ const char* fps_status_string(int status) {
 uint64_t fps_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 void fps_set_stage_events(void* const* events, int n_events) {
+  g_stage_mask = 0;
   if (!events || n_events <= 0) {
     g_n_stage_events = 0;
     return;
@@ -461,5 +465,7 @@ void fps_set_stage_events(void* const* events, int n_events) {
   for (int i = 0; i < n_events; ++i) g_stage_events[i] = events[i];
   g_n_stage_events = n_events;
 }
+
+unsigned fps_stage_mask(void) { return g_stage_mask; }
 
 }  // extern "C"

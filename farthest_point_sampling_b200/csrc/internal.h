@@ -62,7 +62,7 @@ struct Workspace {
   int* pool_event;  // [events] the events pooled in several chunks
   double* pool_acc; // [pool slots][K][F]
   int* pool_cnt;    // [pool slots][K]
-  double* lloyd[2]; // 2 x [fps slots][K][5] cell sums (W, S_x, S_y, S_z, S_t)
+  double* lloyd[3]; // 3 x [fps slots][K][5] cell sums (W, S_x, S_y, S_z, S_t)
   int* labels;      // [P] internal Voronoi labels (kNN mode with Lloyd)
   int fps_slots;    // capacity of the Lloyd slot range
   int pool_slots;   // capacity of the pooling slot range

@@ -241,6 +241,10 @@ uint64_t fps_launch_count(void);
  */
 void fps_set_stage_events(void *const *events, int n_events);
 
+/* Bit s set: stage s was started (its first event recorded) by a call since
+ * the last fps_set_stage_events.  Host-side bookkeeping for benchmarks. */
+unsigned fps_stage_mask(void);
+
 /* Schedule fps_tokenize gives an event of n points: -1 none (n <= K, or n = 0),
  * 0 warp, 1 CTA, 2 CTA shared-memory, 3 8-CTA cluster, 4 16-CTA cluster; -2
  * if n exceeds fps_max_event_points().  Two batch-level rules apply on top
