@@ -99,8 +99,10 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     n_mid = 0;
   }
   __syncthreads();
-  // pass 1: classify and count FPS events (four events per thread in flight)
+  // pass 1: classify and count FPS events (four events per thread in flight;
+  // counts kept per thread and added once per warp after the loop)
   constexpr int U = 4;
+  int my_fps = 0, my_mid = 0;
   for (int b0 = threadIdx.x; b0 < B; b0 += U * blockDim.x) {
     int64_t o0[U], o1[U];
     int st[U];
@@ -136,8 +138,8 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
             record_error(ws.hdr, kDevTooLarge);
             cls = kClsSkip;
           } else {
-            atomicAdd(&n_fps, 1);
-            if (n > kCtaCap && n <= kCtaSmemCap) atomicAdd(&n_mid, 1);
+            ++my_fps;
+            if (n > kCtaCap && n <= kCtaSmemCap) ++my_mid;
           }
         }
       }
@@ -147,6 +149,12 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
         s_cls[b] = (signed char)cls;
       }
     }
+  }
+  my_fps = __reduce_add_sync(kFull, my_fps);
+  my_mid = __reduce_add_sync(kFull, my_mid);
+  if ((threadIdx.x & 31) == 0) {
+    if (my_fps) atomicAdd(&n_fps, my_fps);
+    if (my_mid) atomicAdd(&n_mid, my_mid);
   }
   __syncthreads();
   const bool few = n_fps <= latency_events;

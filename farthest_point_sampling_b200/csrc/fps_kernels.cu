@@ -846,6 +846,8 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     const bool allowed = f < 0 || q == kNumSchedules - 1 || f <= q;
     run[q] = allowed && (hint == 0 || hint > lo);
   }
+  // at most one event per SM: every warp-class event runs on the CTA schedule
+  if (f < 0 && maybe_few) run[0] = false;
 
 
   const PoolOut none = {nullptr, 0, nullptr, nullptr};
