@@ -31,24 +31,6 @@ __device__ __forceinline__ int sched_shift(int q) {
   return q == 0 ? 1 : (q == 1 ? 4 : (q == 2 ? 6 : (q == 3 ? 9 : 10)));
 }
 
-// Reserves v consecutive entries of the shared counter *ctr for every lane
-// of the warp (all lanes call it; v may be 0) with one atomic per warp;
-// returns the lane's first entry.
-__device__ __forceinline__ int warp_reserve(int* ctr, int v) {
-  const int lane = threadIdx.x & 31;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
-  }
-  const int total = __shfl_sync(kFull, x, 31);
-  int base = 0;
-  if (lane == 31 && total > 0) base = atomicAdd(ctr, total);
-  base = __shfl_sync(kFull, base, 31);
-  return base + x - v;
-}
-
 // Exclusive prefix sum of v over the CTA and (in `total`) the CTA's sum;
 // tmp: 32 ints of shared memory.  Every thread of the CTA must call it.
 __device__ __forceinline__ int cta_exclusive_scan(int v, int* tmp, int& total) {
@@ -75,6 +57,49 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* tmp, int& total) {
   total = tmp[nw - 1];
   __syncthreads();  // tmp may be reused
   return before + x - v;
+}
+
+// 64-bit form of cta_exclusive_scan (tmp: 32 x 64 bits of shared memory).
+__device__ __forceinline__ unsigned long long cta_exclusive_scan64(unsigned long long v, unsigned long long* tmp,
+                                                                   unsigned long long& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  unsigned long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = lane < nw ? tmp[lane] : 0ull;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(kFull, w, o);
+      if (lane >= o) w += y;
+    }
+    tmp[lane] = w;
+  }
+  __syncthreads();
+  const unsigned long long before = warp > 0 ? tmp[warp - 1] : 0ull;
+  total = tmp[nw - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// Writes the work items (b, c * step), c < count, of every lane's event with
+// the whole warp: the events that have items are taken in turn and every
+// lane writes a share of each (all lanes call it).
+__device__ __forceinline__ void warp_fill_items(int2* dst, int base, int count, int b, int step) {
+  const int lane = threadIdx.x & 31;
+  unsigned m = __ballot_sync(kFull, count > 0);
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    const int sb = __shfl_sync(kFull, base, src), sc = __shfl_sync(kFull, count, src);
+    const int se = __shfl_sync(kFull, b, src);
+    for (int c = lane; c < sc; c += 32) dst[sb + c] = make_int2(se, c * step);
+  }
 }
 
 // One CTA: classifies every event, builds the per-schedule work lists sorted
@@ -205,9 +230,13 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     if (lane == 31) cnt[q] = run;
   }
   __syncthreads();
-  // pass 3: scatter into the sorted lists; pooling items and accumulator
-  // slots.  The loop is warp-uniform so that the shared counters are bumped
-  // once per warp (warp_reserve) rather than once per event.
+  // pass 3: scatter into the sorted lists; FPS slots, pooling items and
+  // accumulator slots.  Each 1024-event round reserves its slots with one
+  // CTA scan of the four counts packed into 64 bits (FPS slot 12 bits, pooled
+  // event 12, replica slots 16, pool chunks 20: a round's totals fit), and
+  // the warps write the pooling items cooperatively.
+  __shared__ unsigned long long s_tmp64[32];
+  int c_fps = 0, c_events = 0, c_slots = 0, c_chunks = 0;
   for (int b0 = 0; b0 < B; b0 += blockDim.x) {
     const int b = b0 + threadIdx.x;
     const int cls = b < B ? cls_of(b) : kClsSkip;
@@ -220,20 +249,36 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
                                    : (q == 2 ? ws.list_cta_smem : (q == 3 ? ws.list_cluster8 : ws.list_cluster16)));
       list[atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1)] = b;
     }
-    const int fslot = warp_reserve(&cnt[kListFps], cls == kClsFps ? 1 : 0);
     // pooling items (passthrough events of fps_tokenize are written directly;
     // events of schedules that pool in place are left out)
     const bool pooled_here = (cls == kClsFps && !((fused_pool >> q) & 1)) || (chunk_all && cls == kClsPass);
     const int npc = pooled_here ? (n + kPoolChunk - 1) / kPoolChunk : 0;
-    const int pbase = warp_reserve(&cnt[kListPoolChunks], npc);
-    for (int c = 0; c < npc; ++c) ws.pool_chunks[pbase + c] = make_int2(b, c);
-    const int pslot = warp_reserve(&cnt[kListPoolSlots], npc > 1 ? min(kPoolReplicas, npc) : 0);
-    const int pev = warp_reserve(&cnt[kListPoolEvents], npc > 1 ? 1 : 0);
+    const int nrep = npc > 1 ? min(kPoolReplicas, npc) : 0;
+    const unsigned long long v = (unsigned long long)npc | ((unsigned long long)nrep << 20) |
+                                 ((unsigned long long)(npc > 1 ? 1 : 0) << 36) |
+                                 ((unsigned long long)(cls == kClsFps ? 1 : 0) << 48);
+    unsigned long long tot;
+    const unsigned long long pre = cta_exclusive_scan64(v, s_tmp64, tot);
+    const int pbase = c_chunks + (int)(pre & 0xFFFFFull);
+    const int pslot = c_slots + (int)((pre >> 20) & 0xFFFFull);
+    const int pev = c_events + (int)((pre >> 36) & 0xFFFull);
+    const int fslot = c_fps + (int)((pre >> 48) & 0xFFFull);
+    warp_fill_items(ws.pool_chunks, pbase, npc, b, 1);
     if (npc > 1) ws.pool_event[pev] = b;
     if (b < B) {
       ws.fps_slot[b] = cls == kClsFps ? fslot : -1;
       ws.pool_slot[b] = npc > 1 ? pslot : -1;
     }
+    c_chunks += (int)(tot & 0xFFFFFull);
+    c_slots += (int)((tot >> 20) & 0xFFFFull);
+    c_events += (int)((tot >> 36) & 0xFFFull);
+    c_fps += (int)((tot >> 48) & 0xFFFull);
+  }
+  if (threadIdx.x == 0) {
+    cnt[kListFps] = c_fps;
+    cnt[kListPoolChunks] = c_chunks;
+    cnt[kListPoolSlots] = c_slots;
+    cnt[kListPoolEvents] = c_events;
   }
 
   __syncthreads();
@@ -254,7 +299,7 @@ __global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offset
     const int np = (n + kPass - 1) / kPass;
     int tot;
     const int base = carry + cta_exclusive_scan(np, s_tmp, tot);
-    for (int j = 0; j < np; ++j) ws.passes[base + j] = make_int2(b, j * kPass);
+    warp_fill_items(ws.passes, base, np, b, kPass);
     carry += tot;
   }
   if (threadIdx.x == 0) cnt[kListChunks] = carry;
