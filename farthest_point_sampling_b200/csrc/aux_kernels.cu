@@ -994,9 +994,6 @@ __device__ __forceinline__ uint64_t warp_merge64(uint64_t a, uint64_t b, int lan
   return v;
 }
 
-// A 32-point chunk with more passing keys than this is sorted and merged
-// into the list at once; fewer are inserted one by one.
-constexpr int kKnnInsertMax = 4;
 
 // Row order of the kNN kernel inside fps_tokenize: the FPS events of the
 // binning kernel's schedule lists, largest schedule first (each list is
@@ -1030,6 +1027,8 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
+  __shared__ uint64_t s_stage[256 / 32][32];  // per-warp staging slots (k <= 32)
+  uint64_t* stage = s_stage[threadIdx.x >> 5];
   int n_ev = B;
   if (ord.on) {
     n_ev = 0;
@@ -1061,6 +1060,7 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
       const float4 c = centroids[orow];
       const float4* pts = coords + o0;
       uint64_t thr = ~0ull;
+      int ns = 0;  // staged candidates (k <= 32)
       constexpr int U = 4;  // 32-point chunks loaded per iteration
       for (int base = 0; base < n; base += 32 * U) {
         float4 pt[U];
@@ -1074,14 +1074,28 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
           const int i = base + u * 32 + lane;
           const uint64_t key =
               i < n ? (((uint64_t)__float_as_uint(dist1(pt[u], c)) << 32) | (uint32_t)i) : ~0ull;
-          unsigned mask = __ballot_sync(kFull, key < thr);
           if constexpr (KPL == 1) {
-            if (__popc(mask) > kKnnInsertMax) {  // many candidates: sort them and merge
-              L[0] = warp_merge64(L[0], warp_sort64(key < thr ? key : ~0ull, lane), lane);
+            // candidates below the threshold go to the warp's staging slots; a
+            // chunk that would overflow them first sorts the staged keys and
+            // merges them into the list (refreshing the threshold)
+            bool pass = key < thr;
+            unsigned mask = __ballot_sync(kFull, pass);
+            int cnt = __popc(mask);
+            if (ns + cnt > 32) {
+              __syncwarp();
+              const uint64_t sv = lane < ns ? stage[lane] : ~0ull;
+              L[0] = warp_merge64(L[0], warp_sort64(sv, lane), lane);
               thr = __shfl_sync(kFull, L[0], kl);
-              mask = 0;
+              ns = 0;
+              pass = key < thr;
+              mask = __ballot_sync(kFull, pass);
+              cnt = __popc(mask);
+              __syncwarp();
             }
-          }
+            if (pass) stage[ns + __popc(mask & ((1u << lane) - 1u))] = key;
+            ns += cnt;
+          } else {
+          unsigned mask = __ballot_sync(kFull, key < thr);
           while (mask) {
             const int src = __ffs(mask) - 1;
             mask &= mask - 1;
@@ -1107,6 +1121,15 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
               if (q == kq) t = L[q];
             thr = __shfl_sync(kFull, t, kl);
           }
+          }
+        }
+      }
+      if constexpr (KPL == 1) {
+        if (ns > 0) {  // the last staged candidates
+          __syncwarp();
+          const uint64_t sv = lane < ns ? stage[lane] : ~0ull;
+          L[0] = warp_merge64(L[0], warp_sort64(sv, lane), lane);
+          __syncwarp();
         }
       }
     }
