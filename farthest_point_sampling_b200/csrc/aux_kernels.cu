@@ -999,14 +999,16 @@ __device__ __forceinline__ uint64_t warp_merge64(uint64_t a, uint64_t b, int lan
 // binning kernel's schedule lists, largest schedule first (each list is
 // sorted by decreasing size), so that the longest rows start first.
 struct KnnOrder {
-  const int* list[kNumSchedules];  // list[q] = the list of schedule kNumSchedules - 1 - q
-  int on;
+  const int* list[kNumSchedules];  // the lists, largest schedule first
+  int count_id[kNumSchedules];     // their n_items entries
+  int nlists;                      // 0: every event of the batch, in batch order
 };
 
 __device__ __forceinline__ int ordered_event(const WsHeader* hdr, const KnnOrder& o, int e) {
 #pragma unroll
   for (int q = 0; q < kNumSchedules; ++q) {
-    const int nq = hdr->n_items[kNumSchedules - 1 - q];
+    if (q >= o.nlists) break;
+    const int nq = hdr->n_items[o.count_id[q]];
     if (e < nq) return o.list[q][e];
     e -= nq;
   }
@@ -1030,16 +1032,15 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
   __shared__ uint64_t s_stage[256 / 32][32];  // per-warp staging slots (k <= 32)
   uint64_t* stage = s_stage[threadIdx.x >> 5];
   int n_ev = B;
-  if (ord.on) {
+  if (ord.nlists) {
     n_ev = 0;
-#pragma unroll
-    for (int q = 0; q < kNumSchedules; ++q) n_ev += hdr->n_items[q];
+    for (int q = 0; q < ord.nlists; ++q) n_ev += hdr->n_items[ord.count_id[q]];
   }
   const int64_t rows = (int64_t)n_ev * K;
   const int kq = (k - 1) >> 5, kl = (k - 1) & 31;
   for (int64_t r = gw; r < rows; r += nw) {
     const int e = (int)(r / K), j = (int)(r - (int64_t)e * K);
-    const int b = ord.on ? ordered_event(hdr, ord, e) : e;
+    const int b = ord.nlists ? ordered_event(hdr, ord, e) : e;
     const int64_t orow = (int64_t)b * K + j;  // output row
     const int64_t o0 = offsets[b], o1 = offsets[b + 1];
     int n = 0, nv = 0;
@@ -1147,7 +1148,7 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
                        const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, const float* feats,
                        int F, float* pooled, int32_t* counts, const Workspace* ws, WsHeader* hdr,
-                       cudaStream_t s) {
+                       cudaStream_t s, int only_schedule) {
   const DeviceInfo& di = device_info();
   const int64_t rows = (int64_t)B * K;
   int64_t blocks = (rows + 7) / 8;
@@ -1156,12 +1157,14 @@ cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, cons
   if (blocks < 1) blocks = 1;
   KnnOrder ord{};
   if (ws) {
-    ord.on = 1;
-    ord.list[0] = ws->list_cluster16;
-    ord.list[1] = ws->list_cluster8;
-    ord.list[2] = ws->list_cta_smem;
-    ord.list[3] = ws->list_cta;
-    ord.list[4] = ws->list_warp;
+    const int* lists[kNumSchedules] = {ws->list_warp, ws->list_cta, ws->list_cta_smem, ws->list_cluster8,
+                                       ws->list_cluster16};
+    for (int q = kNumSchedules - 1; q >= 0; --q) {
+      if (only_schedule >= 0 && q != only_schedule) continue;
+      ord.list[ord.nlists] = lists[q];
+      ord.count_id[ord.nlists] = q;  // the schedule lists are n_items[0 .. kNumSchedules)
+      ++ord.nlists;
+    }
   }
   count_launch();
   if (k <= 32)

@@ -855,6 +855,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
   const PoolOut po_warp = (pb.fused_pool & 1) ? pool : none;
   const PoolOut po_cta = (pb.fused_pool & 2) ? pool : none;
 
+  const bool knn_per_schedule = knn_with_fps(pb);
   std::lock_guard<std::mutex> lock(ctx.launch_mu);  // the fork/join events are shared per device
   if ((e = cudaEventRecord(ctx.fork, s))) return e;
   for (int q = 0; q < kNumSchedules; ++q) {
@@ -890,6 +891,12 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
         break;
     }
     if (e != cudaSuccess) return e;
+    // kNN mode without Lloyd: this schedule's kNN rows follow on its own
+    // stream, overlapping the other schedules' FPS (its stage includes them)
+    if (knn_per_schedule &&
+        (e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx, pb.feats, pb.F,
+                        pb.pooled, pb.counts, &ws, ws.hdr, hs, q)))
+      return e;
     mark(1 + q, 1, hs);
     if ((e = cudaEventRecord(ctx.join[q], hs))) return e;
   }

@@ -123,7 +123,9 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
     if ((e = launch_lloyd(pb, ws, labels, s))) return from_cuda(e);
     stage_mark(6, 1, s);
   }
-  if (pb.assign_mode == FPS_ASSIGN_KNN) {
+  if (pb.assign_mode == FPS_ASSIGN_KNN && knn_with_fps(pb)) {
+    // done by launch_fps, schedule by schedule
+  } else if (pb.assign_mode == FPS_ASSIGN_KNN) {
     stage_mark(7, 0, s);
     if ((e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx,
                         pb.feats, pb.F, pb.pooled, pb.counts, &ws, ws.hdr, s)))

@@ -96,6 +96,9 @@ void stage_mark(int stage, int end, cudaStream_t s);
 // FPS schedules plus the passthrough kernel (`pt`), all concurrent after the
 // binning kernel; returns once the work is enqueued and joined into `s`.
 cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws, cudaStream_t s, StageMark mark);
+// kNN mode without Lloyd: launch_fps runs each schedule's kNN rows on that
+// schedule's stream right after its FPS kernel.
+inline bool knn_with_fps(const Problem& pb) { return pb.assign_mode == 1 && pb.lloyd_iters == 0; }
 // Bytes of shared memory of the warp-schedule event copy (per warp) and of
 // the register-CTA schedule (per CTA): fused pooling must fit into them.
 size_t warp_region_bytes();
@@ -107,7 +110,7 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
                        const int32_t* valid_tokens, int K, int k, int32_t* knn_idx,
                        const float* feats, int F, float* pooled, int32_t* counts, const Workspace* ws,
-                       struct WsHeader* hdr, cudaStream_t s);
+                       struct WsHeader* hdr, cudaStream_t s, int only_schedule = -1);
 cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const float4* centroids,
                           const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,
                           cudaStream_t s);

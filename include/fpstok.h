@@ -235,7 +235,9 @@ uint64_t fps_launch_count(void);
  * from it; their events are recorded there).  Stages: 0 binning, 1 FPS warp
  * schedule, 2 FPS CTA schedule, 3 FPS CTA shared-memory schedule, 4 FPS 8-CTA
  * cluster, 5 FPS 16-CTA cluster, 6 Lloyd, 7 kNN gather + pool, 8 Voronoi pool
- * (events not pooled by their FPS kernel), 9 passthrough.  A stage that does
+ * (events not pooled by their FPS kernel), 9 passthrough.  In kNN mode
+ * without Lloyd each FPS stage also covers the kNN rows of its events (they
+ * run on that schedule's stream) and stage 7 is not used.  A stage that does
  * not run records nothing.  The events are cudaEvent_t handles the caller created; at most 32
  * are used.  Pass NULL to turn it off.  Not thread-safe: meant for benchmarks.
  */
