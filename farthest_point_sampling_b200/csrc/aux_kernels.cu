@@ -1150,9 +1150,12 @@ cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, cons
                        int F, float* pooled, int32_t* counts, const Workspace* ws, WsHeader* hdr,
                        cudaStream_t s, int only_schedule) {
   const DeviceInfo& di = device_info();
+  // one block per 8 rows (one row per warp), not a persistent grid: short
+  // blocks let the schedulers interleave the per-schedule kNN launches by
+  // stream priority (rows past the device's count exit at once)
   const int64_t rows = (int64_t)B * K;
   int64_t blocks = (rows + 7) / 8;
-  const int64_t cap = (int64_t)di.sm_count * 16;
+  const int64_t cap = (int64_t)1 << 24;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   KnnOrder ord{};

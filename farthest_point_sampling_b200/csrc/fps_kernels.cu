@@ -800,12 +800,16 @@ static cudaError_t prepare(int dev) {
   if ((e = prepare_block_kernel<8>(&info.cluster8_max_active)) != cudaSuccess) return e;
   if ((e = prepare_block_kernel<16>(&info.cluster16_max_active)) != cudaSuccess) return e;
   if ((e = prepare_aux_kernels()) != cudaSuccess) return e;
-  // FPS schedules (the critical path) on the highest priority, the passthrough
-  // kernel (which only has to finish before pooling) on the lowest
+  // FPS schedules (the critical path) on high priorities -- the larger the
+  // schedule's events, the higher, so that its work (and in kNN mode its
+  // rows) is scheduled first -- and the passthrough kernel, which only has
+  // to finish before pooling, on the lowest
   int least = 0, greatest = 0;
   if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest))) return e;
   for (int i = 0; i < kHelpers; ++i) {
-    const int prio = i == kHelpers - 1 ? least : greatest;
+    int prio = greatest + (kNumSchedules - 1 - i);  // numerically smaller = higher
+    if (prio > least) prio = least;
+    if (i == kHelpers - 1) prio = least;
     if ((e = cudaStreamCreateWithPriority(&ctx.helper[i], cudaStreamNonBlocking, prio))) return e;
     if ((e = cudaEventCreateWithFlags(&ctx.join[i], cudaEventDisableTiming))) return e;
   }
