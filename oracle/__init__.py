@@ -44,8 +44,11 @@ def bind(path: str):
     lib.fpso_pool_voronoi.argtypes = [P, I, P, I, I, P, P, P]
     lib.fpso_pool_knn.argtypes = [P, I, I, I, I, P, P, P]
     lib.fpso_tokenize.argtypes = [P, P, I, P, I, P, I, I, I, I, I, P, P, P, P, P, P]
+    lib.fpso_pool_voronoi_backward.argtypes = [P, I, P, I, I, P, P, P]
+    lib.fpso_pool_knn_backward.argtypes = [P, I, I, I, I, P, P, ctypes.c_int64, P]
     for f in (lib.fpso_fps, lib.fpso_assign, lib.fpso_knn, lib.fpso_lloyd,
-              lib.fpso_pool_voronoi, lib.fpso_pool_knn, lib.fpso_tokenize):
+              lib.fpso_pool_voronoi, lib.fpso_pool_knn, lib.fpso_tokenize,
+              lib.fpso_pool_voronoi_backward, lib.fpso_pool_knn_backward):
         f.restype = I
     return lib
 
@@ -170,6 +173,29 @@ def pool_knn(feats, knn_idx):
     counts = np.empty((B, K), np.int32)
     _check(_load().fpso_pool_knn(_p(feats), F, B, K, k, _p(knn_idx), _p(pooled), _p(counts)), "pool_knn")
     return pooled, counts
+
+
+def pool_voronoi_backward(grad_pooled, offsets, token_id, counts):
+    """Gradient of ``pool_voronoi`` with respect to the features, given the
+    gradient of the pooled rows [B, K, F] and the forward's counts [B, K]."""
+    grad_pooled, offsets = _f32(grad_pooled), _i64(offsets)
+    B, K, F = grad_pooled.shape
+    token_id = _i32(token_id)
+    out = np.empty((token_id.shape[0], F), np.float32)
+    _check(_load().fpso_pool_voronoi_backward(_p(grad_pooled), F, _p(offsets), B, K, _p(token_id),
+                                              _p(_i32(counts)), _p(out)), "pool_voronoi_backward")
+    return out
+
+
+def pool_knn_backward(grad_pooled, knn_idx, counts, P: int):
+    """Gradient of ``pool_knn`` with respect to the [P, F] features."""
+    grad_pooled, knn_idx = _f32(grad_pooled), _i32(knn_idx)
+    B, K, F = grad_pooled.shape
+    k = knn_idx.shape[2]
+    out = np.empty((P, F), np.float32)
+    _check(_load().fpso_pool_knn_backward(_p(grad_pooled), F, B, K, k, _p(knn_idx), _p(_i32(counts)), P,
+                                          _p(out)), "pool_knn_backward")
+    return out
 
 
 def tokenize(coords, feats, offsets, K: int, assign_mode: int = 0, k: int = 0, lloyd_iters: int = 0,

@@ -312,6 +312,65 @@ int fpso_pool_knn(const float *feats, int F, int B, int K, int k, const int32_t 
 }
 
 /*
+ * Backward of the Voronoi mean-pool: the vector-Jacobian product of
+ * fpso_pool_voronoi with respect to the features (graphnet PR #923, "What is
+ * added": the tests check gradients through the model, and the tokenizer sits
+ * inside the training step).  The pool is linear: point i of cell j enters
+ * pooled[b,j,:] with weight 1/counts[b,j], so
+ *   grad_feats[i,f] = grad_pooled[b, token_id[i], f] / counts[b, token_id[i]],
+ * the quotient taken in float64 and rounded once, and 0 for an unassigned
+ * point (token_id -1) or a cell whose count is 0.  counts are the forward's.
+ */
+int fpso_pool_voronoi_backward(const float *grad_pooled, int F, const int64_t *offsets, int B, int K,
+                               const int32_t *token_id, const int32_t *counts, float *grad_feats)
+{
+    if (K < 1 || F < 1 || bad_offsets(offsets, B)) return -1;
+    for (int b = 0; b < B; ++b) {
+        for (int64_t i = offsets[b]; i < offsets[b + 1]; ++i) {
+            int32_t j = token_id[i];
+            if (j >= K) return -1;
+            int32_t c = j >= 0 ? counts[(int64_t)b * K + j] : 0;
+            for (int f = 0; f < F; ++f) {
+                float g = 0.0f;
+                if (c > 0) g = (float)((double)grad_pooled[((int64_t)b * K + j) * F + f] / (double)c);
+                grad_feats[i * F + f] = g;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Backward of the kNN mean-pool: every valid entry i of row r = (b, j) took
+ * feats[i,:] with weight 1/counts[r], so grad_feats[i,:] is the sum over all
+ * rows that gathered i of grad_pooled[r,:] / counts[r].  The quotients and the
+ * sum are float64 (rows in order), rounded once to float32; points no row
+ * gathered get 0.  P is the number of feature rows.
+ */
+int fpso_pool_knn_backward(const float *grad_pooled, int F, int B, int K, int k, const int32_t *knn_idx,
+                           const int32_t *counts, int64_t P, float *grad_feats)
+{
+    if (K < 1 || F < 1 || k < 1 || B < 0 || P < 0) return -1;
+    double *acc = (double *)calloc((size_t)(P > 0 ? P : 1) * F, sizeof(double));
+    for (int64_t r = 0; r < (int64_t)B * K; ++r) {
+        if (counts[r] <= 0) continue;
+        for (int e = 0; e < k; ++e) {
+            int32_t i = knn_idx[r * k + e];
+            if (i < 0) continue;
+            if (i >= P) {
+                free(acc);
+                return -1;
+            }
+            for (int f = 0; f < F; ++f)
+                acc[(int64_t)i * F + f] += (double)grad_pooled[r * F + f] / (double)counts[r];
+        }
+    }
+    for (int64_t e = 0; e < P * F; ++e) grad_feats[e] = (float)acc[e];
+    free(acc);
+    return 0;
+}
+
+/*
  * The whole tokenizer: FPS (or passthrough) -> centroids -> Voronoi labels ->
  * Lloyd (events with N > K) -> Voronoi mean-pool, or kNN gather around the
  * final centroids and kNN mean-pool.  token_id may be NULL in kNN mode;

@@ -30,12 +30,18 @@ MUTATIONS = {
                           "S[4 * j + a] += q * (double)coords[4 * (off + i)];"),
     "pool_wrong_column": ("sum[(int64_t)j * F + f] += (double)feats[(off + i) * F + f];",
                           "sum[(int64_t)j * F + f] += (double)feats[(off + i) * F];"),
+    "pool_bwd_no_count": ("g = (float)((double)grad_pooled[((int64_t)b * K + j) * F + f] / (double)c);",
+                          "g = grad_pooled[((int64_t)b * K + j) * F + f];"),
+    "pool_bwd_wrong_event": ("g = (float)((double)grad_pooled[((int64_t)b * K + j) * F + f] / (double)c);",
+                             "g = (float)((double)grad_pooled[(int64_t)j * F + f] / (double)c);"),
+    "knn_bwd_first_feature": ("acc[(int64_t)i * F + f] += (double)grad_pooled[r * F + f] / (double)counts[r];",
+                              "acc[(int64_t)i * F + f] += (double)grad_pooled[r * F] / (double)counts[r];"),
 }
 
 PINS = [
     pins.pin_dist_golden, pins.pin_dist_error_bound, pins.pin_fps_fixtures, pins.pin_fps_bruteforce,
     pins.pin_fps_invariants, pins.pin_assign_bruteforce, pins.pin_knn_bruteforce,
-    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form,
+    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint,
 ]
 
 

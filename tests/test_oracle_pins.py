@@ -273,6 +273,110 @@ def test_pool_closed_forms():
 
 # ---------------------------------------------------------------- Lloyd
 
+# ---------------------------------------------------------------- pool backward
+#
+# The pool is linear in the features, so its vector-Jacobian product G -> dX is
+# its transpose: <G, pool(X)> = <dX, X> for every X and G (the adjoint
+# identity).  The forward side uses the numpy brute force, not the oracle.
+
+def _knn_pool_np(feats, knn_idx):
+    B, K, k = knn_idx.shape
+    out = np.zeros((B, K, feats.shape[1]))
+    for b in range(B):
+        for j in range(K):
+            rows = [i for i in knn_idx[b, j] if i >= 0]
+            if rows:
+                out[b, j] = feats[rows].astype(np.float64).mean(0)
+    return out
+
+
+def _backward_cases():
+    for b, K, starts in list(_tiny_batches())[:24]:
+        idx = bf.fps(b.coords, b.offsets, K, start_local=starts)
+        cents = _centroids(b, idx)
+        valid = np.minimum(b.sizes(), K).astype(np.int32)
+        tok = bf.assign(b.coords, b.offsets, cents, valid)
+        yield b, K, valid, cents, tok
+
+
+def pin_pool_backward_adjoint():
+    rng = np.random.default_rng(77)
+    for b, K, valid, cents, tok in _backward_cases():
+        B, F = len(b.offsets) - 1, b.feats.shape[1]
+        G = rng.normal(0, 1, (B, K, F)).astype(np.float32)
+        X = rng.normal(0, 1, b.feats.shape).astype(np.float32)
+        # Voronoi
+        wp, wc = bf.pool_voronoi(X, b.offsets, K, tok)
+        dX = oracle.pool_voronoi_backward(G, b.offsets, tok, wc)
+        lhs = float((G.astype(np.float64) * wp).sum())
+        rhs = float((dX.astype(np.float64) * X).sum())
+        scale = float(np.abs(G).sum() * np.abs(X).max()) + 1e-30
+        assert abs(lhs - rhs) <= 1e-6 * scale, (lhs, rhs)
+        # a point outside every cell gets no gradient
+        assert np.all(dX[tok < 0] == 0)
+        # kNN
+        k = 3
+        knn_idx = bf.knn(b.coords, b.offsets, cents, valid, k)
+        kp = _knn_pool_np(X, knn_idx)
+        kc = (knn_idx >= 0).sum(2).astype(np.int32)
+        dX = oracle.pool_knn_backward(G, knn_idx, kc, X.shape[0])
+        lhs = float((G.astype(np.float64) * kp).sum())
+        rhs = float((dX.astype(np.float64) * X).sum())
+        assert abs(lhs - rhs) <= 1e-6 * scale, (lhs, rhs)
+
+
+def test_pool_backward_adjoint():
+    pin_pool_backward_adjoint()
+
+
+def test_pool_backward_autograd():
+    """Reverse-mode autograd of a float64 torch scatter-mean, elementwise."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(78)
+    for b, K, valid, cents, tok in list(_backward_cases())[:10]:
+        B, F = len(b.offsets) - 1, b.feats.shape[1]
+        G = rng.normal(0, 1, (B, K, F)).astype(np.float32)
+        ev = np.repeat(np.arange(B), np.diff(b.offsets))
+        X = torch.tensor(b.feats, dtype=torch.float64, requires_grad=True)
+        keep = torch.from_numpy(tok >= 0)
+        cell = torch.from_numpy(ev * K + np.maximum(tok, 0)).long()
+        sums = torch.zeros(B * K, F, dtype=torch.float64).index_add(0, cell[keep], X[keep])
+        cnt = torch.zeros(B * K, dtype=torch.float64).index_add(0, cell[keep], torch.ones(int(keep.sum()),
+                                                                                            dtype=torch.float64))
+        pooled = sums / cnt.clamp(min=1).unsqueeze(1)
+        (pooled * torch.from_numpy(G.reshape(B * K, F)).double()).sum().backward()
+        want = X.grad.numpy().astype(np.float32)
+        got = oracle.pool_voronoi_backward(G, b.offsets, tok, cnt.numpy().astype(np.int32).reshape(B, K))
+        np.testing.assert_array_equal(got, want)
+
+        knn_idx = bf.knn(b.coords, b.offsets, cents, valid, 4)
+        X.grad = None
+        flat = torch.from_numpy(knn_idx.reshape(B * K, 4)).long()
+        m = (flat >= 0).double()
+        rows = X[flat.clamp(min=0)] * m.unsqueeze(2)
+        kc = m.sum(1)
+        pooled = rows.sum(1) / kc.clamp(min=1).unsqueeze(1)
+        (pooled * torch.from_numpy(G.reshape(B * K, F)).double()).sum().backward()
+        want = X.grad.numpy()
+        got = oracle.pool_knn_backward(G, knn_idx, kc.numpy().astype(np.int32).reshape(B, K), X.shape[0])
+        np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-7)
+
+
+def test_pool_backward_closed_forms():
+    # G = 1 on every row: each assigned point gets 1 / (size of its cell), and
+    # the gradients of one cell sum to 1 per feature
+    offsets = np.array([0, 5, 5, 9])
+    tok = np.array([0, 0, 1, 0, -1, 2, 2, 2, 0], np.int32)
+    counts = np.array([[3, 1, 0], [0, 0, 0], [1, 0, 3]], np.int32)
+    G = np.ones((3, 3, 2), np.float32)
+    dX = oracle.pool_voronoi_backward(G, offsets, tok, counts)
+    np.testing.assert_array_equal(dX[:, 0], np.float32([1 / 3, 1 / 3, 1, 1 / 3, 0, 1 / 3, 1 / 3, 1 / 3, 1]))
+    # kNN: a point gathered by two rows sums both rows' shares
+    knn_idx = np.array([[[0, 1], [1, -1]]], np.int32)
+    dX = oracle.pool_knn_backward(np.float32([[[2, 0], [3, 1]]]), knn_idx, np.int32([[2, 1]]), 3)
+    assert dX.tolist() == [[1, 0], [4, 1], [0, 0]]
+
+
 def pin_lloyd_closed_form():
     rng = np.random.default_rng(7)
     n, K = 40, 3
