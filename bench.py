@@ -63,6 +63,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-microbench", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls only")
+    ap.add_argument("--no-backward", action="store_true", help="skip the mean-pool backward measurement")
     return ap.parse_args()
 
 
@@ -476,6 +477,8 @@ def main():
         result["clocks"] = clocks.summary()
         if not args.no_e2e:
             result["e2e"] = e2e(fps, batch, kw, dev, args.e2e_steps)
+        if not args.no_backward:
+            result["pool_backward"] = pool_backward_roofline(fps, dev)
         if world == 1 and not args.no_cpu_baseline:
             rate, reps, el = cpu_oracle_rate(batch, args.cpu_seconds)
             result["cpu_baseline"] = {"value": rate, "unit": "events/s", "cores": 1, "kind": "oracle",
@@ -529,6 +532,105 @@ def microbench_fp32(dev):
     vals = [best[k] for k in ("scalar_fmul_fadd", "f32x2_add", "f32x2_mul") if best.get(k)]
     best["non_fma_peak"] = max(vals) if vals else None
     return best
+
+
+def pool_backward_roofline(fps, dev, reps=50):
+    """HBM roofline of the mean-pool backward (C ``segment_pool_backward``),
+    called through the C ABI on preallocated buffers.
+
+    Voronoi: the large-event shapes (8 events of 50k-200k points, K = 128,
+    F = 6) with seeded random labels; kNN: the 256-event kNN workload's
+    shapes (k = 32) with seeded random rows inside each event.  One call is
+    captured in a CUDA graph; each replay is timed with CUDA events on the
+    current stream, after a 256 MiB write that evicts the inputs from L2
+    (outside the events)."""
+    import ctypes
+    import json as _j
+
+    import torch
+    from farthest_point_sampling_b200 import _lib
+
+    lib = fps.load_library()
+    peaks = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    vp = ctypes.c_void_p
+    out = {}
+    for mode, wl in ((_lib.FPS_ASSIGN_VORONOI, "c3"), (_lib.FPS_ASSIGN_KNN, "c2")):
+        b = workloads.make_workload(wl)
+        sizes = b.sizes()
+        B, K, F, P = b.B, b.K, b.feats.shape[1], int(b.offsets[-1])
+        rng = np.random.default_rng(90 + mode)
+        G = torch.from_numpy(rng.normal(0, 1, (B, K, F)).astype(np.float32)).to(dev)
+        offsets = torch.from_numpy(b.offsets).to(dev)
+        counts_np = np.zeros((B, K), np.int32)
+        if mode == _lib.FPS_ASSIGN_VORONOI:
+            tok_np = np.concatenate([rng.integers(0, min(int(n), K), int(n)) for n in sizes]).astype(np.int32)
+            np.add.at(counts_np, (np.repeat(np.arange(B), sizes), tok_np), 1)
+            tok, knn, k = torch.from_numpy(tok_np).to(dev), None, 0
+            byts = 4 * P + 4 * F * P + B * K * (4 * F + 4) + 8 * (B + 1)
+            what = "4P token ids + 4FP gradient written + B*K*(4F+4) rows and counts + 8(B+1) offsets"
+        else:
+            k = b.k
+            rows = np.full((B, K, k), -1, np.int32)
+            for e, n in enumerate(sizes):
+                if n > 0:
+                    m = min(int(n), k)
+                    rows[e, :min(int(n), K), :m] = b.offsets[e] + np.stack(
+                        [rng.choice(int(n), m, replace=False) for _ in range(min(int(n), K))])
+            counts_np = (rows >= 0).sum(2).astype(np.int32)
+            tok, knn = None, torch.from_numpy(rows).to(dev)
+            byts = 4 * B * K * k + B * K * (4 * F + 4) + 4 * F * P
+            what = "4*B*K*k rows + B*K*(4F+4) gradient rows and counts + 4FP gradient written"
+        counts = torch.from_numpy(counts_np).to(dev)
+        grad = torch.empty((P, F), dtype=torch.float32, device=dev)
+        nb = lib.segment_pool_backward_workspace_bytes(P, B, K, F, mode)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+        n_before = lib.fps_launch_count()
+
+        def call(strm):
+            st = lib.segment_pool_backward(vp(G.data_ptr()), F, vp(offsets.data_ptr()), B, P, K, mode,
+                                           vp(tok.data_ptr()) if tok is not None else None,
+                                           vp(knn.data_ptr()) if knn is not None else None, k,
+                                           vp(counts.data_ptr()), vp(grad.data_ptr()), vp(ws.data_ptr()),
+                                           ws.numel(), vp(strm.cuda_stream))
+            if st != 0:
+                raise RuntimeError(f"segment_pool_backward failed: {st}")
+
+        for _ in range(3):
+            call(stream)
+        torch.cuda.synchronize(dev)
+        n_warm = lib.fps_launch_count() - n_before
+        # one call captured in a CUDA graph, replayed after an L2-evicting write
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap):
+            call(cap)
+        torch.cuda.synchronize(dev)
+        for _ in range(3):
+            flush.zero_()
+            g.replay()
+        st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        for i in range(reps):
+            flush.zero_()
+            st_ev[i].record(stream)
+            g.replay()
+            en_ev[i].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = float(np.mean([a.elapsed_time(c) for a, c in zip(st_ev, en_ev)]))
+        del g
+        achieved = byts / (ms / 1e3) / 1e9
+        out["voronoi" if mode == _lib.FPS_ASSIGN_VORONOI else "knn"] = {
+            "workload": f"{wl} shapes: B={B}, P={P}, K={K}, F={F}" + (f", k={k}" if k else ""),
+            "us_per_call": ms * 1e3, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "algorithmic_bytes": byts, "algorithmic": what,
+            "kernels_per_call": n_warm / 3,
+            "note": "memset + per-event scatter + rounding, timed together" if k else "quotient table + gather"}
+    return out
 
 
 def e2e(fps, batch, kw, dev, steps):

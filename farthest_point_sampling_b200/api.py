@@ -299,6 +299,74 @@ def segment_pool(feats: torch.Tensor, offsets: Optional[torch.Tensor], K: int,
     return pooled, counts
 
 
+def segment_pool_backward(grad_pooled: torch.Tensor, counts: torch.Tensor, P: int,
+                          offsets: Optional[torch.Tensor] = None, token_id: Optional[torch.Tensor] = None,
+                          knn_idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """C ``segment_pool_backward``: the gradient [P, F] of the pooled rows
+    ``grad_pooled [B,K,F]`` with respect to the features, given the forward's
+    ``counts [B,K]`` and its Voronoi labels (``offsets`` + ``token_id``) or
+    kNN rows (``knn_idx [B,K,k]``)."""
+    dev = _cuda_device(grad_pooled)
+    _need(grad_pooled, "grad_pooled", torch.float32, 3, dev)
+    _need(counts, "counts", torch.int32, 2, dev)
+    B, K, F = grad_pooled.shape
+    if tuple(counts.shape) != (B, K):
+        raise ValueError("counts must be [B, K] like grad_pooled")
+    lib = _lib.load()
+    if knn_idx is not None:
+        _need(knn_idx, "knn_idx", torch.int32, 3, dev)
+        if tuple(knn_idx.shape[:2]) != (B, K):
+            raise ValueError("knn_idx must be [B, K, k]")
+        mode, k, offp = _lib.FPS_ASSIGN_KNN, knn_idx.shape[2], None
+        if offsets is not None:  # lets each event's rows be summed in shared memory first
+            _need(offsets, "offsets", torch.int64, 1, dev)
+            if offsets.numel() != B + 1:
+                raise ValueError("offsets must be [B + 1]")
+            offp = offsets
+    else:
+        if token_id is None or offsets is None:
+            raise ValueError("the Voronoi backward needs offsets and token_id")
+        _need(offsets, "offsets", torch.int64, 1, dev)
+        _need(token_id, "token_id", torch.int32, 1, dev)
+        if offsets.numel() != B + 1 or token_id.numel() != P:
+            raise ValueError("offsets must be [B + 1] and token_id [P]")
+        mode, k, offp = _lib.FPS_ASSIGN_VORONOI, 0, offsets
+    ws = _workspace(lib.segment_pool_backward_workspace_bytes(P, B, K, F, mode), dev, workspace)
+    grad_feats = torch.empty((P, F), dtype=torch.float32, device=dev)
+    st = lib.segment_pool_backward(_ptr(grad_pooled), F, _ptr(offp), B, P, K, mode, _ptr(token_id),
+                                   _ptr(knn_idx), k, _ptr(counts), _ptr(grad_feats), _ptr(ws), ws.numel(),
+                                   _stream(dev))
+    _lib.check(st, "segment_pool_backward")
+    return grad_feats
+
+
+class _SegmentMean(torch.autograd.Function):
+    """Mean-pool with its gradient to the features; both directions are the
+    C ``segment_pool`` / ``segment_pool_backward`` calls."""
+
+    @staticmethod
+    def forward(ctx, feats, offsets, K, token_id, knn_idx):
+        pooled, counts = segment_pool(feats, offsets, K, token_id=token_id, knn_idx=knn_idx)
+        ctx.save_for_backward(offsets, token_id, knn_idx, counts)
+        ctx.P = feats.shape[0]
+        ctx.mark_non_differentiable(counts)
+        return pooled, counts
+
+    @staticmethod
+    def backward(ctx, grad_pooled, _grad_counts):
+        offsets, token_id, knn_idx, counts = ctx.saved_tensors
+        g = segment_pool_backward(grad_pooled.contiguous(), counts, ctx.P, offsets=offsets, token_id=token_id,
+                                  knn_idx=knn_idx)
+        return g, None, None, None, None
+
+
+def segment_mean(feats: torch.Tensor, offsets: Optional[torch.Tensor], K: int,
+                 token_id: Optional[torch.Tensor] = None, knn_idx: Optional[torch.Tensor] = None):
+    """``segment_pool`` that autograd differentiates with respect to
+    ``feats``.  Returns ``(pooled [B,K,F], counts [B,K])``."""
+    return _SegmentMean.apply(feats, offsets, K, token_id, knn_idx)
+
+
 def device_status(workspace: torch.Tensor) -> None:
     """Reads the device-side status word of a workspace (synchronises the
     current stream) and raises ``FpsError`` if a check failed."""

@@ -7,6 +7,7 @@
 #include "../../include/fpstok.h"
 #include "common.cuh"
 #include "internal.h"
+#include "pool_backward.h"
 
 namespace fpstok {
 
@@ -426,6 +427,46 @@ int segment_pool(const float* feats, int F, const int64_t* offsets, int B, int64
       (e = cudaMemsetAsync(ws.pool_cnt, 0, (size_t)ws.pool_slots * K * sizeof(int), s)))
     return from_cuda(e);
   return from_cuda(launch_pool_voronoi(feats, F, offsets, B, K, token_id, pooled, counts, ws, s));
+}
+
+size_t segment_pool_backward_workspace_bytes(int64_t P, int B, int K, int F, int mode) {
+  if (P < 0 || B < 0 || K < 1 || F < 1) return 0;
+  size_t n = align256(sizeof(WsHeader));
+  if (mode == FPS_ASSIGN_KNN) n += align256((size_t)P * F * sizeof(double));
+  return n;
+}
+
+int segment_pool_backward(const float* grad_pooled, int F, const int64_t* offsets, int B, int64_t P, int K,
+                          int mode, const int32_t* token_id, const int32_t* knn_idx, int k, const int32_t* counts,
+                          float* grad_feats, void* workspace, size_t workspace_bytes, fps_stream_t stream) {
+  if (B < 0 || P < 0) return FPS_ERR_ARG;
+  if (P >= ((int64_t)1 << 31)) return FPS_ERR_TOO_LARGE;
+  if (K < 1 || F < 1) return FPS_ERR_ARG;
+  if (K > FPS_MAX_K || F > FPS_MAX_F || (int64_t)B * K >= ((int64_t)1 << 31)) return FPS_ERR_TOO_LARGE;
+  if (mode != FPS_ASSIGN_VORONOI && mode != FPS_ASSIGN_KNN) return FPS_ERR_ARG;
+  if (P == 0) return FPS_OK;
+  if (!grad_feats || (B > 0 && (!grad_pooled || !counts))) return FPS_ERR_ARG;
+  if (mode == FPS_ASSIGN_KNN) {
+    if (k < 1) return FPS_ERR_ARG;
+    if (k > FPS_MAX_KNN) return FPS_ERR_TOO_LARGE;
+    if (B > 0 && !knn_idx) return FPS_ERR_ARG;
+  } else if (B == 0 || !offsets || !token_id) {
+    return FPS_ERR_ARG;  // every point belongs to an event
+  }
+  const size_t need = segment_pool_backward_workspace_bytes(P, B, K, F, mode);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+  char* scratch = static_cast<char*>(workspace) + align256(sizeof(WsHeader));
+  if (mode == FPS_ASSIGN_KNN) {
+    double* acc = reinterpret_cast<double*>(scratch);
+    return from_cuda(
+        launch_pool_bwd_knn(grad_pooled, F, offsets, B, K, k, knn_idx, counts, P, acc, grad_feats, hdr, s));
+  }
+  return from_cuda(
+      launch_pool_bwd_voronoi(grad_pooled, F, offsets, B, P, K, token_id, counts, grad_feats, hdr, s));
 }
 
 int fps_device_status(void* workspace, fps_stream_t stream, int* detail) {

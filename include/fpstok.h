@@ -208,6 +208,34 @@ int segment_pool(const float *feats, int F, const int64_t *offsets, int B, int64
                  float *pooled, int32_t *counts, void *workspace, size_t workspace_bytes,
                  fps_stream_t stream);
 
+/*
+ * Backward of segment_pool: the gradient of the pooled rows with respect to
+ * the features (graphnet PR #923, "What is added": the tokenizer sits inside
+ * the training step, and the tests check gradients).  The pool is linear, so
+ * with the forward's counts [B, K]:
+ *   mode FPS_ASSIGN_VORONOI: grad_feats[i,:] = grad_pooled[b, t, :] / counts[b, t]
+ *     for t = token_id[i] of point i of event b; 0 when t = -1 or the count
+ *     is 0.  offsets and token_id are required.  The result is exact: the
+ *     float32 division correctly rounded.
+ *   mode FPS_ASSIGN_KNN: grad_feats[i,:] = sum over the rows (b, j) whose
+ *     knn_idx entries hold i of grad_pooled[b, j, :] / counts[b, j]; 0 for a
+ *     point no row gathered.  offsets may be NULL; when given, the rows of
+ *     each event are summed in shared memory first (entries may still point
+ *     anywhere in 0..P-1).  The sum accumulates in float64 (in no fixed
+ *     order) and rounds once to float32.
+ * grad_pooled float32 [B, K, F]; grad_feats float32 [P, F] (every row is
+ * written).  Device-side problems (a token outside -1..K-1, a kNN index >= P,
+ * offsets that do not cover the points) leave that point's gradient 0 and
+ * are reported by fps_device_status().  Workspace: the size below (device,
+ * 256-byte aligned): a status word in Voronoi mode, plus P * F * 8 bytes in
+ * kNN mode.
+ */
+size_t segment_pool_backward_workspace_bytes(int64_t P, int B, int K, int F, int mode);
+int segment_pool_backward(const float *grad_pooled, int F, const int64_t *offsets, int B, int64_t P,
+                          int K, int mode, const int32_t *token_id, const int32_t *knn_idx, int k,
+                          const int32_t *counts, float *grad_feats, void *workspace,
+                          size_t workspace_bytes, fps_stream_t stream);
+
 /* Reads (and clears) the device-side status word in `workspace`; synchronises
  * `stream`.  Returns FPS_OK or FPS_ERR_DEVICE; *detail (optional) receives the
  * recorded reason (see FPS_DEV_* below). */

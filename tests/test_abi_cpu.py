@@ -92,6 +92,21 @@ def test_standalone_argument_errors():
     assert lib.segment_pool(x, 6, x, 2, 100, 8, 2, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
     assert lib.segment_pool(x, 0, x, 2, 100, 8, 0, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
     assert lib.segment_pool(x, 6, x, 2, 100, 8, 1, None, x, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    # segment_pool_backward(grad, F, offsets, B, P, K, mode, token_id, knn_idx, k, counts, grad_feats, ws, n, s)
+    bw = lib.segment_pool_backward
+    assert bw(x, 6, x, 2, 100, 8, 2, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG  # bad mode
+    assert bw(x, 0, x, 2, 100, 8, 0, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG  # F = 0
+    assert bw(x, 65, x, 2, 100, 8, 0, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
+    assert bw(x, 6, x, 2, 100, 300, 0, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
+    assert bw(x, 6, None, 2, 100, 8, 0, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG  # no offsets
+    assert bw(x, 6, x, 2, 100, 8, 0, None, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG  # no labels
+    assert bw(x, 6, x, 2, 100, 8, 0, x, None, 0, None, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG  # no counts
+    assert bw(x, 6, None, 2, 100, 8, 1, None, None, 4, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG  # no rows
+    assert bw(x, 6, None, 2, 100, 8, 1, None, x, 129, x, x, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
+    need = lib.segment_pool_backward_workspace_bytes(100, 2, 8, 6, 1)
+    assert need >= 100 * 6 * 8
+    assert bw(x, 6, None, 2, 100, 8, 1, None, x, 4, x, x, x, need - 1, None) == _lib.FPS_ERR_WORKSPACE
+    assert bw(x, 6, x, 2, 0, 8, 0, x, None, 0, x, x, None, 0, None) == _lib.FPS_OK  # nothing to do
 
 
 def test_workspace_sizes_grow_with_problem():
