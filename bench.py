@@ -629,7 +629,7 @@ def pool_backward_roofline(fps, dev, reps=50):
             "us_per_call": ms * 1e3, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "algorithmic_bytes": byts, "algorithmic": what,
             "kernels_per_call": n_warm / 3,
-            "note": "memset + per-event scatter + rounding, timed together" if k else "quotient table + gather"}
+            "note": "memset + per-event row masks and row-order sums + rounding, timed together" if k else "quotient table + gather"}
     return out
 
 

@@ -432,7 +432,8 @@ int segment_pool(const float* feats, int F, const int64_t* offsets, int B, int64
 size_t segment_pool_backward_workspace_bytes(int64_t P, int B, int K, int F, int mode) {
   if (P < 0 || B < 0 || K < 1 || F < 1) return 0;
   size_t n = align256(sizeof(WsHeader));
-  if (mode == FPS_ASSIGN_KNN) n += align256((size_t)P * F * sizeof(double));
+  if (mode == FPS_ASSIGN_KNN) n += align256((size_t)P * F * sizeof(double) * 2);
+  else n += align256((size_t)B * K * F * sizeof(float));
   return n;
 }
 
@@ -465,8 +466,8 @@ int segment_pool_backward(const float* grad_pooled, int F, const int64_t* offset
     return from_cuda(
         launch_pool_bwd_knn(grad_pooled, F, offsets, B, K, k, knn_idx, counts, P, acc, grad_feats, hdr, s));
   }
-  return from_cuda(
-      launch_pool_bwd_voronoi(grad_pooled, F, offsets, B, P, K, token_id, counts, grad_feats, hdr, s));
+  return from_cuda(launch_pool_bwd_voronoi(grad_pooled, F, offsets, B, P, K, token_id, counts,
+                                           reinterpret_cast<float*>(scratch), grad_feats, hdr, s));
 }
 
 int fps_device_status(void* workspace, fps_stream_t stream, int* detail) {

@@ -9,9 +9,9 @@
 //   kNN:     grad_feats[i,:] = sum over the rows (b, j) that gathered i of
 //            grad_pooled[b,j,:] / counts[b,j] -- a scatter, accumulated in
 //            float64 with red.global.add.f64 and rounded once.
-// Quotients are taken in float64 and rounded once to float32 (for the
-// Voronoi gather that equals a correctly rounded float32 division, which is
-// what it computes).
+// Quotients are taken in float64 and rounded once to float32; the Voronoi
+// path divides once per (token, feature) into a small table and then only
+// gathers.
 #include "common.cuh"
 #include "internal.h"
 #include "pool_backward.h"
@@ -24,7 +24,8 @@ constexpr int kBwdThreads = 256;
 constexpr int kBwdPts = 4;                      // points per thread of the Voronoi gather
 constexpr int kBwdTile = kBwdThreads * kBwdPts;  // points per block
 constexpr int kKnnBwdThreads = 512;
-constexpr int64_t kKnnBwdSmemBytes = 104 * 1024;  // shares + per-event float64 sums of the kNN scatter
+constexpr int kFeatGroup = 8;  // features summed together per thread in the kNN scatter
+constexpr int64_t kKnnBwdSmemBytes = 104 * 1024;  // shares and per-point row masks of the kNN scatter
 
 // Largest b in [lo, hi] with offsets[b] <= i (offsets non-decreasing), i.e.
 // the event holding point i when i < offsets[hi + 1].
@@ -37,26 +38,30 @@ __device__ __forceinline__ int event_of(const int64_t* __restrict__ offsets, int
   return lo;
 }
 
-// g / c as the float64 quotient rounded once to float32.  For c < 2^24 (exact
-// in float32) that is the correctly rounded float32 division: rounding the
-// 53-bit quotient to 24 bits cannot differ from rounding the exact quotient
-// (double rounding is harmless for division when 53 >= 2 * 24 + 2).
-__device__ __forceinline__ float share_f32(float g, int c) {
-  return c < (1 << 24) ? __fdiv_rn(g, (float)c) : (float)((double)g / (double)c);
+// quot[r, f] = grad_pooled[r, f] / counts[r] as the float64 quotient rounded
+// once to float32, 0 for an empty row: the division happens once per
+// (token, feature), and the per-point pass only gathers.
+__global__ void __launch_bounds__(256) k_pool_bwd_quot(const float* __restrict__ grad_pooled, int F, int64_t rows,
+                                                       const int32_t* __restrict__ counts,
+                                                       float* __restrict__ quot) {
+  const int64_t n = rows * F;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
+    const int c = counts[e / F];
+    quot[e] = c > 0 ? (float)((double)grad_pooled[e] / (double)c) : 0.f;
+  }
 }
 
 // The gather: one block per tile of kBwdTile points, kBwdPts per thread with
-// their loads issued together.  Per point its gradient row (b*K + token) and
-// count go to shared memory, then one thread per output element writes the
-// flat [P, F] gradient with coalesced stores.  e / F is taken as
-// __umulhi(e, fdiv) with fdiv = ceil(2^32 / F) (F >= 2), exact for
-// e < kBwdTile * F <= 2^16: the error e * (fdiv * F - 2^32) / 2^32 stays below 1/F.
+// their loads issued together.  Per point its quotient row (b*K + token) goes
+// to shared memory, then one thread per output element writes the flat
+// [P, F] gradient with coalesced stores.  e / F is taken as __umulhi(e, fdiv)
+// with fdiv = ceil(2^32 / F) (F >= 2): exact while e * (fdiv * F - 2^32) <
+// 2^32, which holds for every e < kBwdTile * F <= 2^16.
 __global__ void __launch_bounds__(kBwdThreads) k_pool_bwd_voronoi(
-    const float* __restrict__ grad_pooled, int F, uint32_t fdiv, const int64_t* __restrict__ offsets, int B,
-    int64_t P, int K, const int32_t* __restrict__ token_id, const int32_t* __restrict__ counts,
-    float* __restrict__ grad_feats, WsHeader* hdr) {
+    const float* __restrict__ quot, int F, uint32_t fdiv, const int64_t* __restrict__ offsets, int B, int64_t P,
+    int K, const int32_t* __restrict__ token_id, float* __restrict__ grad_feats, WsHeader* hdr) {
   __shared__ int s_row[kBwdTile];  // b*K + token, -1 when the point gets no gradient
-  __shared__ int s_cnt[kBwdTile];
   __shared__ int s_ev[2];
   const int64_t t0 = (int64_t)blockIdx.x * kBwdTile;
   const int n = (int)min((int64_t)kBwdTile, P - t0);
@@ -69,26 +74,17 @@ __global__ void __launch_bounds__(kBwdThreads) k_pool_bwd_voronoi(
   if (threadIdx.x < 2) s_ev[threadIdx.x] = event_of(offsets, 0, B - 1, threadIdx.x ? t0 + n - 1 : t0);
   __syncthreads();
   const int lo = s_ev[0], hi = max(s_ev[0], s_ev[1]);
-  int row[kBwdPts], b[kBwdPts];
 #pragma unroll
   for (int r = 0; r < kBwdPts; ++r) {
     const int p = threadIdx.x + r * kBwdThreads;
-    const int64_t i = t0 + p;
-    b[r] = p < n ? event_of(offsets, lo, hi, i) : lo;
-    row[r] = -1;
     if (p < n) {
-      if (__ldg(offsets + b[r]) > i || __ldg(offsets + b[r] + 1) <= i) record_error(hdr, kDevBadOffsets);
+      const int64_t i = t0 + p;
+      const int b = event_of(offsets, lo, hi, i);
+      int row = -1;
+      if (__ldg(offsets + b) > i || __ldg(offsets + b + 1) <= i) record_error(hdr, kDevBadOffsets);
       else if (t[r] >= K || t[r] < -1) record_error(hdr, kDevBadToken);
-      else if (t[r] >= 0) row[r] = b[r] * K + t[r];
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < kBwdPts; ++r) {
-    const int p = threadIdx.x + r * kBwdThreads;
-    const int c = row[r] >= 0 ? counts[row[r]] : 0;
-    if (p < n) {
-      s_row[p] = c > 0 ? row[r] : -1;
-      s_cnt[p] = c;
+      else if (t[r] >= 0) row = b * K + t[r];
+      s_row[p] = row;
     }
   }
   __syncthreads();
@@ -98,7 +94,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_pool_bwd_voronoi(
   for (uint32_t e = threadIdx.x; e < ne; e += kBwdThreads) {
     const uint32_t q = F == 1 ? e : __umulhi(e, fdiv);
     const int rw = s_row[q];
-    out[e] = rw >= 0 ? share_f32(__ldg(grad_pooled + (int64_t)rw * F + (e - q * F)), s_cnt[q]) : 0.f;
+    out[e] = rw >= 0 ? __ldg(quot + (int64_t)rw * F + (e - q * F)) : 0.f;
   }
 }
 
@@ -135,35 +131,51 @@ __global__ void __launch_bounds__(256) k_pool_bwd_knn(const float* __restrict__ 
   }
 }
 
-// kNN scatter with the rows grouped by event: one CTA takes all K rows of
-// event b.  It first stages the K x F float64 shares grad_pooled / counts in
-// shared memory (all loads issued together), then runs one thread per row
-// entry.  Shares for points inside the event (when its n x F float64 sums fit
-// in shared memory) are summed there and added to the global accumulators
-// with one reduction per (point, feature) touched, instead of one per (row
-// entry, feature); entries outside the event, and events too large for the
-// shared buffer, go straight to the global accumulators.  Entry e of the
-// event's K*k entries is row e / k, taken as __umulhi(e, kdiv) with
-// kdiv = ceil(2^32 / k) (k >= 2; exact for e < 2^15, k <= 128).
+// Whether event b (n points from off) gets the per-event path: its row masks
+// fit in shared memory and its points lie inside 0..P-1.
+__device__ __forceinline__ bool knn_event_local(int64_t off, int64_t n, int cap_n, int64_t P) {
+  return n > 0 && n <= cap_n && off >= 0 && off + n <= P;
+}
+
+// kNN scatter with the rows grouped by event.  Phase 1, one CTA per event:
+// stage the K x F float64 shares grad_pooled / counts in shared memory, mark
+// for each point of the event the rows that name it in a K-bit mask (shared
+// atomicOr, independent of order), then let each point sum the shares of its
+// marked rows in increasing row order -- the order a sequential loop over the
+// rows takes -- and store the sums (plain stores: only this CTA writes these
+// points of sums[]).  Entries that name a point outside their event, or a
+// point already marked in the same row, are added to extra[] with float64
+// atomics.  Phase 2, a warp per row over the whole grid: the rows of events
+// whose masks do not fit in shared memory add all their entries to extra[].
+// The gradient is (float)(sums + extra); extra is 0 when every row names
+// only its own event's points, once each, and the events fit, and then the
+// result is exactly the sequential row-order sum.  Entry e of the event's
+// K*k entries is row e / k = __umulhi(e, kdiv) with kdiv = ceil(2^32 / k)
+// (k >= 2; exact for e < 2^15, k <= 128).  The sums run one thread per
+// (point, group of up to kFeatGroup features) t: one scan of the mask feeds
+// the group's independent sums; the point is t / G = __umulhi(t, gdiv),
+// exact while t * (gdiv * G - 2^32) < 2^32, i.e. for every t < 2^26 (the
+// shared buffer caps t near 2^21).
 __global__ void __launch_bounds__(kKnnBwdThreads, 2) k_pool_bwd_knn_event(
     const float* __restrict__ grad_pooled, int F, const int64_t* __restrict__ offsets, int B, int K, int k,
-    uint32_t kdiv, const int32_t* __restrict__ knn_idx, const int32_t* __restrict__ counts, int64_t P,
-    int smem_points, double* __restrict__ acc, WsHeader* hdr) {
+    uint32_t kdiv, uint32_t gdiv, const int32_t* __restrict__ knn_idx, const int32_t* __restrict__ counts,
+    int64_t P, int cap_n, double* __restrict__ sums, double* __restrict__ extra, WsHeader* hdr) {
   extern __shared__ double s_mem[];
-  double* s_share = s_mem;                    // [K, F]; 0 rows for empty tokens
-  double* s_acc = s_mem + (size_t)K * F;      // [smem_points, F]
+  double* s_share = s_mem;                                                  // [K, F]; 0 rows for empty tokens
+  uint32_t* s_bits = reinterpret_cast<uint32_t*>(s_share + (size_t)K * F);  // [cap_n, W] row masks
+  const int W = (K + 31) >> 5;
   const int ke = K * k;
+  const int G = (F + kFeatGroup - 1) / kFeatGroup;
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     const int64_t off = offsets[b];
     const int64_t n = offsets[b + 1] - off;
-    const bool local = n > 0 && n <= smem_points && off >= 0 && off + n <= P;  // block-uniform
+    if (!knn_event_local(off, n, cap_n, P)) continue;  // block-uniform; phase 2 takes it
     const float* g = grad_pooled + (int64_t)b * K * F;
     for (int e = threadIdx.x; e < K * F; e += blockDim.x) {
       const int c = counts[(int64_t)b * K + e / F];
       s_share[e] = c > 0 ? (double)__ldg(g + e) / (double)c : 0.0;
     }
-    if (local)
-      for (int e = threadIdx.x; e < (int)n * F; e += blockDim.x) s_acc[e] = 0.0;
+    for (int i = threadIdx.x; i < (int)n * W; i += blockDim.x) s_bits[i] = 0u;
     __syncthreads();
     const int32_t* rows = knn_idx + (int64_t)b * ke;
 #pragma unroll 4
@@ -175,35 +187,74 @@ __global__ void __launch_bounds__(kKnnBwdThreads, 2) k_pool_bwd_knn_event(
       }
       if (v < 0) continue;
       const int j = k == 1 ? e : (int)__umulhi((uint32_t)e, kdiv);
-      const double* sh = s_share + j * F;
       const int64_t li = v - off;
-      if (local && li >= 0 && li < n) {
-        double* dst = s_acc + li * F;
-        for (int f = 0; f < F; ++f)
-          if (sh[f] != 0.0) atomicAdd(dst + f, sh[f]);
-      } else {
-        double* dst = acc + (int64_t)v * F;
-        for (int f = 0; f < F; ++f)
-          if (sh[f] != 0.0) atomicAdd(dst + f, sh[f]);
+      if (li >= 0 && li < n) {
+        const uint32_t bit = 1u << (j & 31);
+        if (!(atomicOr(s_bits + li * W + (j >> 5), bit) & bit)) continue;  // marked: summed below
       }
+      const double* sh = s_share + j * F;  // outside the event, or a repeat within the row
+      double* dst = extra + (int64_t)v * F;
+      for (int f = 0; f < F; ++f)
+        if (sh[f] != 0.0) atomicAdd(dst + f, sh[f]);
     }
     __syncthreads();
-    if (local) {
-      double* dst = acc + off * F;
-      for (int e = threadIdx.x; e < (int)n * F; e += blockDim.x) {
-        const double v = s_acc[e];
-        if (v != 0.0) atomicAdd(dst + e, v);  // +0 needs no add: the accumulators start at +0
+    for (int t = threadIdx.x; t < (int)n * G; t += blockDim.x) {
+      const int i = G == 1 ? t : (int)__umulhi((uint32_t)t, gdiv);
+      const int f0 = (t - i * G) * kFeatGroup;
+      const int nf = min(kFeatGroup, F - f0);
+      const uint32_t* bits = s_bits + (int64_t)i * W;
+      double sum[kFeatGroup];
+#pragma unroll
+      for (int q = 0; q < kFeatGroup; ++q) sum[q] = 0.0;
+      for (int w = 0; w < W; ++w) {
+        uint32_t m = bits[w];
+        while (m) {
+          const int j = (w << 5) + __ffs(m) - 1;
+          m &= m - 1;
+          const double* sh = s_share + j * F + f0;
+#pragma unroll
+          for (int q = 0; q < kFeatGroup; ++q)
+            if (q < nf) sum[q] += sh[q];
+        }
       }
+      double* dst = sums + (off + i) * F + f0;
+#pragma unroll
+      for (int q = 0; q < kFeatGroup; ++q)
+        if (q < nf) dst[q] = sum[q];
     }
     __syncthreads();
   }
+  // phase 2: rows of the events phase 1 skipped, a warp per row
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = gw; r < (int64_t)B * K; r += nw) {
+    const int b = (int)(r / K);
+    const int64_t off = offsets[b];
+    if (knn_event_local(off, offsets[b + 1] - off, cap_n, P)) continue;  // warp-uniform
+    const int c = counts[r];
+    if (c <= 0) continue;
+    const float* g = grad_pooled + r * F;
+    for (int e = lane; e < k; e += 32) {
+      const int v = knn_idx[r * k + e];
+      if (v >= P) record_error(hdr, kDevBadToken);
+      if (v < 0 || v >= P) continue;
+      double* dst = extra + (int64_t)v * F;
+      for (int f = 0; f < F; ++f) {
+        const double sh = (double)__ldg(g + f) / (double)c;
+        if (sh != 0.0) atomicAdd(dst + f, sh);
+      }
+    }
+  }
 }
 
-// Rounds the float64 accumulators to the float32 gradient.
-__global__ void __launch_bounds__(256) k_pool_bwd_round(const double* __restrict__ acc, int64_t n,
-                                                        float* __restrict__ out) {
+// Rounds the float64 accumulators to the float32 gradient: out = (float)(a + b),
+// b optional.
+__global__ void __launch_bounds__(256) k_pool_bwd_round(const double* __restrict__ a, const double* __restrict__ b,
+                                                        int64_t n, float* __restrict__ out) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) out[e] = (float)acc[e];
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride)
+    out[e] = (float)(b ? a[e] + b[e] : a[e]);
 }
 
 int grid_for(int64_t work_items, int per_block, int blocks_per_sm) {
@@ -217,14 +268,19 @@ int grid_for(int64_t work_items, int per_block, int blocks_per_sm) {
 }  // namespace
 
 cudaError_t launch_pool_bwd_voronoi(const float* grad_pooled, int F, const int64_t* offsets, int B, int64_t P,
-                                    int K, const int32_t* token_id, const int32_t* counts, float* grad_feats,
-                                    WsHeader* hdr, cudaStream_t s) {
+                                    int K, const int32_t* token_id, const int32_t* counts, float* quot,
+                                    float* grad_feats, WsHeader* hdr, cudaStream_t s) {
   if (P == 0) return cudaSuccess;
+  const int64_t rows = (int64_t)B * K;
+  count_launch();
+  k_pool_bwd_quot<<<grid_for(rows * F, 256, 8), 256, 0, s>>>(grad_pooled, F, rows, counts, quot);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const uint32_t fdiv = F > 1 ? (uint32_t)((((uint64_t)1 << 32) + F - 1) / F) : 0u;
   const int64_t blocks = (P + kBwdTile - 1) / kBwdTile;
   count_launch();
-  k_pool_bwd_voronoi<<<(unsigned)blocks, kBwdThreads, 0, s>>>(grad_pooled, F, fdiv, offsets, B, P, K, token_id,
-                                                              counts, grad_feats, hdr);
+  k_pool_bwd_voronoi<<<(unsigned)blocks, kBwdThreads, 0, s>>>(quot, F, fdiv, offsets, B, P, K, token_id,
+                                                              grad_feats, hdr);
   return cudaGetLastError();
 }
 
@@ -232,14 +288,18 @@ cudaError_t launch_pool_bwd_knn(const float* grad_pooled, int F, const int64_t* 
                                 const int32_t* knn_idx, const int32_t* counts, int64_t P, double* acc,
                                 float* grad_feats, WsHeader* hdr, cudaStream_t s) {
   if (P == 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)P * F * sizeof(double), s);
-  if (e != cudaSuccess) return e;
   const int64_t rows = (int64_t)B * K;
   const int64_t share_bytes = (int64_t)K * F * sizeof(double);
-  if (rows > 0 && offsets && share_bytes <= kKnnBwdSmemBytes) {
-    int64_t pts = (kKnnBwdSmemBytes - share_bytes) / ((int64_t)F * sizeof(double));
-    if (pts > P) pts = P;
-    const size_t smem = (size_t)(share_bytes + pts * F * (int64_t)sizeof(double));
+  const bool per_event = rows > 0 && offsets && share_bytes <= kKnnBwdSmemBytes / 2;
+  double* extra = per_event ? acc + (size_t)P * F : nullptr;
+  cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)P * F * sizeof(double) * (per_event ? 2 : 1), s);
+  if (e != cudaSuccess) return e;
+  if (per_event) {
+    // shared memory: the shares, then a K-bit row mask per point of the event
+    const int64_t mask_bytes = (int64_t)((K + 31) / 32) * sizeof(uint32_t);
+    int64_t cap = (kKnnBwdSmemBytes - share_bytes) / mask_bytes;
+    if (cap > P) cap = P;
+    const size_t smem = (size_t)(share_bytes + cap * mask_bytes);
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -250,9 +310,11 @@ cudaError_t launch_pool_bwd_knn(const float* grad_pooled, int F, const int64_t* 
       attr_set[dev] = true;
     }
     const uint32_t kdiv = k > 1 ? (uint32_t)((((uint64_t)1 << 32) + k - 1) / k) : 0u;
+    const int G = (F + kFeatGroup - 1) / kFeatGroup;
+    const uint32_t gdiv = G > 1 ? (uint32_t)((((uint64_t)1 << 32) + G - 1) / G) : 0u;
     count_launch();
-    k_pool_bwd_knn_event<<<grid_for(B, 1, 2), kKnnBwdThreads, smem, s>>>(grad_pooled, F, offsets, B, K, k, kdiv,
-                                                                         knn_idx, counts, P, (int)pts, acc, hdr);
+    k_pool_bwd_knn_event<<<grid_for(B, 1, 2), kKnnBwdThreads, smem, s>>>(
+        grad_pooled, F, offsets, B, K, k, kdiv, gdiv, knn_idx, counts, P, (int)cap, acc, extra, hdr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else if (rows > 0) {
     const int g = grid_for(rows, 8, 16);
@@ -266,7 +328,7 @@ cudaError_t launch_pool_bwd_knn(const float* grad_pooled, int F, const int64_t* 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   count_launch();
-  k_pool_bwd_round<<<grid_for((int64_t)P * F, 256, 8), 256, 0, s>>>(acc, (int64_t)P * F, grad_feats);
+  k_pool_bwd_round<<<grid_for((int64_t)P * F, 256, 8), 256, 0, s>>>(acc, extra, (int64_t)P * F, grad_feats);
   return cudaGetLastError();
 }
 

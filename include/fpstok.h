@@ -219,16 +219,18 @@ int segment_pool(const float *feats, int F, const int64_t *offsets, int B, int64
  *     float32 division correctly rounded.
  *   mode FPS_ASSIGN_KNN: grad_feats[i,:] = sum over the rows (b, j) whose
  *     knn_idx entries hold i of grad_pooled[b, j, :] / counts[b, j]; 0 for a
- *     point no row gathered.  offsets may be NULL; when given, the rows of
- *     each event are summed in shared memory first (entries may still point
- *     anywhere in 0..P-1).  The sum accumulates in float64 (in no fixed
- *     order) and rounds once to float32.
+ *     point no row gathered.  The shares are float64 and the sum rounds once
+ *     to float32.  With offsets (else NULL), an event whose rows name only
+ *     its own points and that fits the kernel's shared buffer (about 10^4
+ *     points at K = 128, k = 32, F = 6) is summed in row order, exactly as a
+ *     sequential loop over the rows would; other entries (they may name any
+ *     point in 0..P-1) meet in float64 in no fixed order.
  * grad_pooled float32 [B, K, F]; grad_feats float32 [P, F] (every row is
  * written).  Device-side problems (a token outside -1..K-1, a kNN index >= P,
  * offsets that do not cover the points) leave that point's gradient 0 and
  * are reported by fps_device_status().  Workspace: the size below (device,
- * 256-byte aligned): a status word in Voronoi mode, plus P * F * 8 bytes in
- * kNN mode.
+ * 256-byte aligned): about B * K * F * 4 bytes in Voronoi mode, P * F * 16
+ * in kNN mode.
  */
 size_t segment_pool_backward_workspace_bytes(int64_t P, int B, int K, int F, int mode);
 int segment_pool_backward(const float *grad_pooled, int F, const int64_t *offsets, int B, int64_t P,

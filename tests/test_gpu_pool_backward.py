@@ -1,9 +1,11 @@
 """Parity of the mean-pool backward (C ``segment_pool_backward``) with the oracle.
 
 The Voronoi gradient is a float64 quotient rounded once, so it is compared
-bit for bit; the kNN gradient sums float64 shares in an order the atomics
-choose and is compared within the float tolerance (1e-5 relative, 1e-6
-absolute floor).  Labels, kNN rows and counts come from the oracle or from
+bit for bit.  The kNN gradient of an event whose rows name only its own
+points, and whose points fit the kernel's shared buffer, is summed in row
+order like the oracle's and compared bit for bit too; otherwise float64
+shares meet in an order the atomics choose and the comparison uses the float
+tolerance (1e-5 relative, 1e-6 absolute floor).  Labels, kNN rows and counts come from the oracle or from
 seeded numpy draws, never from the CUDA path.
 """
 import numpy as np
@@ -102,10 +104,11 @@ def test_knn_backward(k):
     want = oracle.pool_knn_backward(G, knn, counts, b.coords.shape[0])
     got = fps.segment_pool_backward(_dev(G), _dev(counts), b.coords.shape[0], knn_idx=_dev(knn))
     assert_float_close(got.cpu().numpy(), want, f"segment_pool_backward knn k={k}")
-    # with offsets: each event's rows are summed in shared memory first
+    # with offsets every event here fits in shared memory: its entries are
+    # grouped by point and summed in row order, exactly as the oracle sums
     got = fps.segment_pool_backward(_dev(G), _dev(counts), b.coords.shape[0], knn_idx=_dev(knn),
                                     offsets=_dev(b.offsets))
-    assert_float_close(got.cpu().numpy(), want, f"segment_pool_backward knn k={k} (per event)")
+    np.testing.assert_array_equal(got.cpu().numpy(), want)
 
 
 def test_knn_backward_rows_outside_their_event():
