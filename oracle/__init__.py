@@ -46,9 +46,12 @@ def bind(path: str):
     lib.fpso_tokenize.argtypes = [P, P, I, P, I, P, I, I, I, I, I, P, P, P, P, P, P]
     lib.fpso_pool_voronoi_backward.argtypes = [P, I, P, I, I, P, P, P]
     lib.fpso_pool_knn_backward.argtypes = [P, I, I, I, I, P, P, ctypes.c_int64, P]
+    lib.fpso_pack_tokens.argtypes = [P, I, P, P, I, I, P, P, P]
+    lib.fpso_unpack_tokens.argtypes = [P, I, P, I, I, P]
     for f in (lib.fpso_fps, lib.fpso_assign, lib.fpso_knn, lib.fpso_lloyd,
               lib.fpso_pool_voronoi, lib.fpso_pool_knn, lib.fpso_tokenize,
-              lib.fpso_pool_voronoi_backward, lib.fpso_pool_knn_backward):
+              lib.fpso_pool_voronoi_backward, lib.fpso_pool_knn_backward, lib.fpso_pack_tokens,
+              lib.fpso_unpack_tokens):
         f.restype = I
     return lib
 
@@ -196,6 +199,35 @@ def pool_knn_backward(grad_pooled, knn_idx, counts, P: int):
     _check(_load().fpso_pool_knn_backward(_p(grad_pooled), F, B, K, k, _p(knn_idx), _p(_i32(counts)), P,
                                           _p(out)), "pool_knn_backward")
     return out
+
+
+def pack_tokens(src, offsets=None, valid=None):
+    """Packed layout of padded tokens ``src [B, K, D]``: returns
+    ``(dst [N_tok, D], doc_id [N_tok], tok_offsets [B + 1])``."""
+    src = _f32(src)
+    B, K, D = src.shape
+    if valid is None:
+        offsets = _i64(offsets)
+        n_tok = int(np.minimum(np.diff(offsets), K).sum()) if B else 0
+    else:
+        valid = _i32(valid)
+        n_tok = int(valid.astype(np.int64).sum())
+    dst = np.empty((max(n_tok, 1), D), np.float32)
+    doc = np.empty(max(n_tok, 1), np.int32)
+    tok = np.empty(B + 1, np.int64)
+    _check(_load().fpso_pack_tokens(_p(src), D, _p(offsets) if valid is None else None, _p(valid), B, K,
+                                    _p(dst), _p(doc), _p(tok)), "pack_tokens")
+    return dst[:n_tok], doc[:n_tok], tok
+
+
+def unpack_tokens(src, tok_offsets, K: int):
+    """Padded layout [B, K, D] of packed tokens ``src [N_tok, D]``."""
+    src, tok_offsets = _f32(src), _i64(tok_offsets)
+    B = tok_offsets.shape[0] - 1
+    D = src.shape[1]
+    dst = np.empty((B, K, D), np.float32)
+    _check(_load().fpso_unpack_tokens(_p(src), D, _p(tok_offsets), B, K, _p(dst)), "unpack_tokens")
+    return dst
 
 
 def tokenize(coords, feats, offsets, K: int, assign_mode: int = 0, k: int = 0, lloyd_iters: int = 0,

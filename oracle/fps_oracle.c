@@ -371,6 +371,55 @@ int fpso_pool_knn_backward(const float *grad_pooled, int F, int B, int K, int k,
 }
 
 /*
+ * Packed token layout for block-diagonal attention (graphnet PR #923, "What
+ * is added": models/utils.py pack / unpack / build_block_mask; the review
+ * thread on the block mask: doc_id holds the event index of every packed
+ * token and two tokens attend to each other when their doc_ids match).
+ * Event b has v_b tokens: valid[b] when given, else min(N_b, K) from the
+ * point offsets (the tokens the tokenizer fills).  pack lists the first v_b
+ * rows of src [B, K, D] of every event in event order:
+ *   tok_offsets[0] = 0, tok_offsets[b+1] = tok_offsets[b] + v_b,
+ *   dst[tok_offsets[b] + j, :] = src[b, j, :], doc_id[tok_offsets[b] + j] = b.
+ */
+int fpso_pack_tokens(const float *src, int D, const int64_t *offsets, const int32_t *valid, int B, int K,
+                     float *dst, int32_t *doc_id, int64_t *tok_offsets)
+{
+    if (D < 1 || K < 1 || B < 0 || (!valid && bad_offsets(offsets, B))) return -1;
+    tok_offsets[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t v;
+        if (valid) {
+            v = valid[b];
+            if (v < 0 || v > K) return -1;
+        } else {
+            int64_t n = offsets[b + 1] - offsets[b];
+            v = n < K ? n : K;
+        }
+        for (int64_t j = 0; j < v; ++j) {
+            int64_t t = tok_offsets[b] + j;
+            doc_id[t] = b;
+            for (int d = 0; d < D; ++d) dst[t * D + d] = src[((int64_t)b * K + j) * D + d];
+        }
+        tok_offsets[b + 1] = tok_offsets[b] + v;
+    }
+    return 0;
+}
+
+/* The inverse: dst[b, j, :] = src[tok_offsets[b] + j, :] for j < v_b, 0 after. */
+int fpso_unpack_tokens(const float *src, int D, const int64_t *tok_offsets, int B, int K, float *dst)
+{
+    if (D < 1 || K < 1 || B < 0 || tok_offsets[0] != 0) return -1;
+    for (int b = 0; b < B; ++b) {
+        int64_t v = tok_offsets[b + 1] - tok_offsets[b];
+        if (v < 0 || v > K) return -1;
+        for (int64_t j = 0; j < K; ++j)
+            for (int d = 0; d < D; ++d)
+                dst[((int64_t)b * K + j) * D + d] = j < v ? src[(tok_offsets[b] + j) * D + d] : 0.0f;
+    }
+    return 0;
+}
+
+/*
  * The whole tokenizer: FPS (or passthrough) -> centroids -> Voronoi labels ->
  * Lloyd (events with N > K) -> Voronoi mean-pool, or kNN gather around the
  * final centroids and kNN mean-pool.  token_id may be NULL in kNN mode;

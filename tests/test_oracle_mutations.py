@@ -34,6 +34,10 @@ MUTATIONS = {
                           "g = grad_pooled[((int64_t)b * K + j) * F + f];"),
     "pool_bwd_wrong_event": ("g = (float)((double)grad_pooled[((int64_t)b * K + j) * F + f] / (double)c);",
                              "g = (float)((double)grad_pooled[(int64_t)j * F + f] / (double)c);"),
+    "pack_drops_last_token": ("        for (int64_t j = 0; j < v; ++j) {\n            int64_t t = tok_offsets[b] + j;",
+                              "        for (int64_t j = 0; j + 1 < v; ++j) {\n            int64_t t = tok_offsets[b] + j;"),
+    "unpack_no_zero_pad": ("j < v ? src[(tok_offsets[b] + j) * D + d] : 0.0f;",
+                           "j < v ? src[(tok_offsets[b] + j) * D + d] : src[0];"),
     "knn_bwd_first_feature": ("acc[(int64_t)i * F + f] += (double)grad_pooled[r * F + f] / (double)counts[r];",
                               "acc[(int64_t)i * F + f] += (double)grad_pooled[r * F] / (double)counts[r];"),
 }
@@ -41,7 +45,7 @@ MUTATIONS = {
 PINS = [
     pins.pin_dist_golden, pins.pin_dist_error_bound, pins.pin_fps_fixtures, pins.pin_fps_bruteforce,
     pins.pin_fps_invariants, pins.pin_assign_bruteforce, pins.pin_knn_bruteforce,
-    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint,
+    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint, pins.pin_pack_tokens,
 ]
 
 

@@ -377,6 +377,38 @@ def test_pool_backward_closed_forms():
     assert dX.tolist() == [[1, 0], [4, 1], [0, 0]]
 
 
+# ---------------------------------------------------------------- packed tokens
+
+def pin_pack_tokens():
+    rng = np.random.default_rng(90)
+    for b, K, starts in list(_tiny_batches())[:30]:
+        B = len(b.offsets) - 1
+        D = int(rng.integers(1, 6))
+        src = rng.normal(0, 1, (B, K, D)).astype(np.float32)
+        n = np.diff(b.offsets)
+        v = np.minimum(n, K)
+        dst, doc, tok = oracle.pack_tokens(src, offsets=b.offsets)
+        # closed forms: the packed length, the scan, the event ids
+        assert dst.shape == (v.sum(), D)
+        assert np.array_equal(tok, np.concatenate([[0], np.cumsum(v)]))
+        assert np.array_equal(doc, np.repeat(np.arange(B), v))
+        # numpy's boolean-mask gather of the same rows, in row-major order
+        mask = np.arange(K)[None, :] < v[:, None]
+        assert np.array_equal(dst, src[mask])
+        # unpack inverts it and zeroes the padding
+        back = oracle.unpack_tokens(dst, tok, K)
+        assert np.array_equal(back, np.where(mask[:, :, None], src, 0))
+        # caller-given counts
+        vv = rng.integers(0, K + 1, B).astype(np.int32)
+        dst, doc, tok = oracle.pack_tokens(src, valid=vv)
+        mask = np.arange(K)[None, :] < vv[:, None]
+        assert np.array_equal(dst, src[mask]) and np.array_equal(doc, np.repeat(np.arange(B), vv))
+
+
+def test_pack_tokens():
+    pin_pack_tokens()
+
+
 def pin_lloyd_closed_form():
     rng = np.random.default_rng(7)
     n, K = 40, 3
