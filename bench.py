@@ -479,6 +479,7 @@ def main():
             result["e2e"] = e2e(fps, batch, kw, dev, args.e2e_steps)
         if not args.no_backward:
             result["pool_backward"] = pool_backward_roofline(fps, dev)
+            result["token_pack"] = token_pack_roofline(fps, dev)
         if world == 1 and not args.no_cpu_baseline:
             rate, reps, el = cpu_oracle_rate(batch, args.cpu_seconds)
             result["cpu_baseline"] = {"value": rate, "unit": "events/s", "cores": 1, "kind": "oracle",
@@ -631,6 +632,72 @@ def pool_backward_roofline(fps, dev, reps=50):
             "kernels_per_call": n_warm / 3,
             "note": "memset + per-event row masks and row-order sums + rounding, timed together" if k else "quotient table + gather"}
     return out
+
+
+def token_pack_roofline(fps, dev, reps=50):
+    """HBM roofline of the packed token layout (C ``fps_pack_tokens``) on the
+    small-event workload's shapes: 4096 events, K = 128 slots of F = 6 pooled
+    features, v_b = min(N_b, K) tokens each.  Graph-replayed and timed like
+    ``pool_backward_roofline``."""
+    import ctypes
+    import json as _j
+
+    import torch
+
+    lib = fps.load_library()
+    peaks = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    b = workloads.make_workload("c4")
+    B, K, D = b.B, b.K, b.feats.shape[1]
+    v = np.minimum(b.sizes(), K)
+    n_tok = int(v.sum())
+    src = torch.from_numpy(np.random.default_rng(95).normal(0, 1, (B, K, D)).astype(np.float32)).to(dev)
+    offsets = torch.from_numpy(b.offsets).to(dev)
+    dst = torch.empty((B * K, D), dtype=torch.float32, device=dev)
+    doc = torch.empty(B * K, dtype=torch.int32, device=dev)
+    tok = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    ws = torch.empty(max(lib.fps_pack_workspace_bytes(), 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    vp = ctypes.c_void_p
+
+    def call(strm):
+        st = lib.fps_pack_tokens(vp(src.data_ptr()), D, vp(offsets.data_ptr()), None, B, K, vp(dst.data_ptr()),
+                                 vp(doc.data_ptr()), vp(tok.data_ptr()), vp(ws.data_ptr()), ws.numel(),
+                                 vp(strm.cuda_stream))
+        if st != 0:
+            raise RuntimeError(f"fps_pack_tokens failed: {st}")
+
+    n_before = lib.fps_launch_count()
+    for _ in range(3):
+        call(stream)
+    torch.cuda.synchronize(dev)
+    per_call = (lib.fps_launch_count() - n_before) / 3
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(g, stream=cap):
+        call(cap)
+    torch.cuda.synchronize(dev)
+    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        st_ev[i].record(stream)
+        g.replay()
+        en_ev[i].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = float(np.mean([a.elapsed_time(c) for a, c in zip(st_ev, en_ev)]))
+    del g
+    byts = 8 * (B + 1) + 2 * 4 * D * n_tok + 4 * n_tok + 8 * (B + 1)
+    achieved = byts / (ms / 1e3) / 1e9
+    return {"workload": f"c4 shapes: B={B}, K={K}, D={D}, {n_tok} tokens", "us_per_call": ms * 1e3,
+            "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "algorithmic_bytes": byts,
+            "algorithmic": "8(B+1) offsets read + 4*D*N_tok rows read and written + 4*N_tok doc ids "
+                           "+ 8(B+1) token offsets",
+            "kernels_per_call": per_call, "note": "scan (one CTA) + per-event copy"}
 
 
 def e2e(fps, batch, kw, dev, steps):

@@ -340,6 +340,56 @@ def segment_pool_backward(grad_pooled: torch.Tensor, counts: torch.Tensor, P: in
     return grad_feats
 
 
+def pack_tokens(src: torch.Tensor, offsets: Optional[torch.Tensor] = None,
+                valid_tokens: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """C ``fps_pack_tokens``: the packed layout of padded tokens ``src [B, K, D]``
+    (event b keeps ``valid_tokens[b]`` rows, else ``min(N_b, K)`` from the
+    point ``offsets``).  Returns ``(dst [N_tok, D], doc_id [N_tok],
+    tok_offsets [B + 1])``; reading the packed length synchronises the
+    current stream once."""
+    dev = _cuda_device(src)
+    _need(src, "src", torch.float32, 3, dev)
+    B, K, D = src.shape
+    if valid_tokens is not None:
+        _need(valid_tokens, "valid_tokens", torch.int32, 1, dev)
+        if valid_tokens.numel() != B:
+            raise ValueError("valid_tokens must be [B]")
+    elif offsets is not None:
+        _need(offsets, "offsets", torch.int64, 1, dev)
+        if offsets.numel() != B + 1:
+            raise ValueError("offsets must be [B + 1]")
+    else:
+        raise ValueError("pack_tokens needs offsets or valid_tokens")
+    lib = _lib.load()
+    ws = _workspace(lib.fps_pack_workspace_bytes(), dev, workspace)
+    dst = torch.empty((max(B * K, 1), D), dtype=torch.float32, device=dev)
+    doc_id = torch.empty(max(B * K, 1), dtype=torch.int32, device=dev)
+    tok_offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    st = lib.fps_pack_tokens(_ptr(src), D, _ptr(offsets), _ptr(valid_tokens), B, K, _ptr(dst), _ptr(doc_id),
+                             _ptr(tok_offsets), _ptr(ws), ws.numel(), _stream(dev))
+    _lib.check(st, "fps_pack_tokens")
+    n_tok = int(tok_offsets[-1].item())
+    return dst[:n_tok], doc_id[:n_tok], tok_offsets
+
+
+def unpack_tokens(src: torch.Tensor, tok_offsets: torch.Tensor, K: int,
+                  workspace: Optional[torch.Tensor] = None):
+    """C ``fps_unpack_tokens``: packed rows ``src [N_tok, D]`` back to the
+    padded layout ``[B, K, D]`` with zero padding."""
+    dev = _cuda_device(src)
+    _need(src, "src", torch.float32, 2, dev)
+    _need(tok_offsets, "tok_offsets", torch.int64, 1, dev)
+    B = tok_offsets.numel() - 1
+    n_tok, D = src.shape
+    lib = _lib.load()
+    ws = _workspace(lib.fps_pack_workspace_bytes(), dev, workspace)
+    dst = torch.empty((B, K, D), dtype=torch.float32, device=dev)
+    st = lib.fps_unpack_tokens(_ptr(src), D, n_tok, _ptr(tok_offsets), B, K, _ptr(dst), _ptr(ws), ws.numel(),
+                               _stream(dev))
+    _lib.check(st, "fps_unpack_tokens")
+    return dst
+
+
 class _SegmentMean(torch.autograd.Function):
     """Mean-pool with its gradient to the features; both directions are the
     C ``segment_pool`` / ``segment_pool_backward`` calls."""

@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "pool_backward.h"
+#include "token_pack.h"
 
 namespace fpstok {
 
@@ -468,6 +469,38 @@ int segment_pool_backward(const float* grad_pooled, int F, const int64_t* offset
   }
   return from_cuda(launch_pool_bwd_voronoi(grad_pooled, F, offsets, B, P, K, token_id, counts,
                                            reinterpret_cast<float*>(scratch), grad_feats, hdr, s));
+}
+
+size_t fps_pack_workspace_bytes(void) { return align256(sizeof(WsHeader)); }
+
+int fps_pack_tokens(const float* src, int D, const int64_t* offsets, const int32_t* valid_tokens, int B, int K,
+                    float* dst, int32_t* doc_id, int64_t* tok_offsets, void* workspace, size_t workspace_bytes,
+                    fps_stream_t stream) {
+  if (B < 0 || K < 1 || D < 1) return FPS_ERR_ARG;
+  if ((int64_t)K * D >= ((int64_t)1 << 31)) return FPS_ERR_TOO_LARGE;
+  if (!tok_offsets || (B > 0 && (!src || !dst || !doc_id || (!offsets && !valid_tokens)))) return FPS_ERR_ARG;
+  if (!workspace || workspace_bytes < fps_pack_workspace_bytes() || !aligned(workspace, 256))
+    return FPS_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+  return from_cuda(launch_pack_tokens(src, D, offsets, valid_tokens, B, K, dst, doc_id, tok_offsets, hdr, s));
+}
+
+int fps_unpack_tokens(const float* src, int D, int64_t n_tok, const int64_t* tok_offsets, int B, int K, float* dst,
+                      void* workspace, size_t workspace_bytes, fps_stream_t stream) {
+  if (B < 0 || K < 1 || D < 1 || n_tok < 0) return FPS_ERR_ARG;
+  if ((int64_t)K * D >= ((int64_t)1 << 31)) return FPS_ERR_TOO_LARGE;
+  if (B == 0) return FPS_OK;
+  if (!tok_offsets || !dst || (n_tok > 0 && !src)) return FPS_ERR_ARG;
+  if (!workspace || workspace_bytes < fps_pack_workspace_bytes() || !aligned(workspace, 256))
+    return FPS_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+  return from_cuda(launch_unpack_tokens(src, D, n_tok, tok_offsets, B, K, dst, hdr, s));
 }
 
 int fps_device_status(void* workspace, fps_stream_t stream, int* detail) {

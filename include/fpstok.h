@@ -238,6 +238,33 @@ int segment_pool_backward(const float *grad_pooled, int F, const int64_t *offset
                           const int32_t *counts, float *grad_feats, void *workspace,
                           size_t workspace_bytes, fps_stream_t stream);
 
+/*
+ * Packed token layout for block-diagonal attention (graphnet PR #923, "What
+ * is added": models/utils.py pack / unpack / build_block_mask; review thread
+ * on the block mask: doc_id is the event index of every packed token, and
+ * tokens attend to each other when their doc_ids match).  Event b has v_b
+ * tokens: valid_tokens[b] when given (0..K), else min(N_b, K) from the point
+ * offsets (the slots the tokenizer fills).
+ *   fps_pack_tokens: tok_offsets [B+1] = 0, v_0, v_0 + v_1, ... (int64);
+ *     dst [tok_offsets[B], D] row tok_offsets[b] + j = src [B, K, D] row
+ *     (b, j) for j < v_b; doc_id [tok_offsets[B]] int32 = b on those rows.
+ *     dst and doc_id must hold B * K rows (the packed length is only known on
+ *     the device: read tok_offsets[B]).  offsets may be NULL when
+ *     valid_tokens is given.
+ *   fps_unpack_tokens: dst [B, K, D] row (b, j) = src row tok_offsets[b] + j
+ *     for j < v_b = tok_offsets[b+1] - tok_offsets[b], 0 for j >= v_b; src
+ *     holds n_tok rows.  An event whose span is not inside 0..n_tok or whose
+ *     v_b is outside 0..K is written as padding and reported by
+ *     fps_device_status().
+ * Workspace: fps_pack_workspace_bytes() (a status word), 256-byte aligned.
+ */
+size_t fps_pack_workspace_bytes(void);
+int fps_pack_tokens(const float *src, int D, const int64_t *offsets, const int32_t *valid_tokens, int B,
+                    int K, float *dst, int32_t *doc_id, int64_t *tok_offsets, void *workspace,
+                    size_t workspace_bytes, fps_stream_t stream);
+int fps_unpack_tokens(const float *src, int D, int64_t n_tok, const int64_t *tok_offsets, int B, int K,
+                      float *dst, void *workspace, size_t workspace_bytes, fps_stream_t stream);
+
 /* Reads (and clears) the device-side status word in `workspace`; synchronises
  * `stream`.  Returns FPS_OK or FPS_ERR_DEVICE; *detail (optional) receives the
  * recorded reason (see FPS_DEV_* below). */

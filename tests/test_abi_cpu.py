@@ -107,6 +107,17 @@ def test_standalone_argument_errors():
     assert need >= 2 * 100 * 6 * 8
     assert bw(x, 6, None, 2, 100, 8, 1, None, x, 4, x, x, x, need - 1, None) == _lib.FPS_ERR_WORKSPACE
     assert bw(x, 6, x, 2, 0, 8, 0, x, None, 0, x, x, None, 0, None) == _lib.FPS_OK  # nothing to do
+    # fps_pack_tokens(src, D, offsets, valid, B, K, dst, doc_id, tok_offsets, ws, n, s)
+    pk, upk = lib.fps_pack_tokens, lib.fps_unpack_tokens
+    wsb = lib.fps_pack_workspace_bytes()
+    assert pk(x, 0, x, None, 2, 8, x, x, x, x, wsb, None) == _lib.FPS_ERR_ARG  # D = 0
+    assert pk(x, 4, None, None, 2, 8, x, x, x, x, wsb, None) == _lib.FPS_ERR_ARG  # no offsets, no counts
+    assert pk(x, 4, x, None, 2, 0, x, x, x, x, wsb, None) == _lib.FPS_ERR_ARG  # K = 0
+    assert pk(x, 1 << 24, x, None, 2, 256, x, x, x, x, wsb, None) == _lib.FPS_ERR_TOO_LARGE
+    assert pk(x, 4, x, None, 2, 8, x, x, x, None, wsb, None) == _lib.FPS_ERR_WORKSPACE
+    assert upk(x, 4, -1, x, 2, 8, x, x, wsb, None) == _lib.FPS_ERR_ARG  # n_tok < 0
+    assert upk(x, 4, 10, None, 2, 8, x, x, wsb, None) == _lib.FPS_ERR_ARG  # no tok_offsets
+    assert upk(x, 4, 10, x, 0, 8, x, x, wsb, None) == _lib.FPS_OK  # B = 0
 
 
 def test_workspace_sizes_grow_with_problem():
