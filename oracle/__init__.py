@@ -47,11 +47,12 @@ def bind(path: str):
     lib.fpso_pool_voronoi_backward.argtypes = [P, I, P, I, I, P, P, P]
     lib.fpso_pool_knn_backward.argtypes = [P, I, I, I, I, P, P, ctypes.c_int64, P]
     lib.fpso_pack_tokens.argtypes = [P, I, P, P, I, I, P, P, P]
+    lib.fpso_token_summaries.argtypes = [P, P, I, I, P, I, I, P, P, P, P]
     lib.fpso_unpack_tokens.argtypes = [P, I, P, I, I, P]
     for f in (lib.fpso_fps, lib.fpso_assign, lib.fpso_knn, lib.fpso_lloyd,
               lib.fpso_pool_voronoi, lib.fpso_pool_knn, lib.fpso_tokenize,
               lib.fpso_pool_voronoi_backward, lib.fpso_pool_knn_backward, lib.fpso_pack_tokens,
-              lib.fpso_unpack_tokens):
+              lib.fpso_unpack_tokens, lib.fpso_token_summaries):
         f.restype = I
     return lib
 
@@ -199,6 +200,19 @@ def pool_knn_backward(grad_pooled, knn_idx, counts, P: int):
     _check(_load().fpso_pool_knn_backward(_p(grad_pooled), F, B, K, k, _p(knn_idx), _p(_i32(counts)), P,
                                           _p(out)), "pool_knn_backward")
     return out
+
+
+def token_summaries(coords, feats, offsets, K: int, token_id, charge_col: int = -1):
+    """Charge-weighted summaries per Voronoi token: ``(wsum [B,K], wcoords
+    [B,K,4], wfeats [B,K,F])``."""
+    coords, feats, offsets = _f32(coords, (4,)), _f32(feats), _i64(offsets)
+    B, F = offsets.shape[0] - 1, feats.shape[1]
+    wsum = np.empty((B, K), np.float32)
+    wc = np.empty((B, K, 4), np.float32)
+    wf = np.empty((B, K, F), np.float32)
+    _check(_load().fpso_token_summaries(_p(coords), _p(feats), F, charge_col, _p(offsets), B, K,
+                                        _p(_i32(token_id)), _p(wsum), _p(wc), _p(wf)), "token_summaries")
+    return wsum, wc, wf
 
 
 def pack_tokens(src, offsets=None, valid=None):

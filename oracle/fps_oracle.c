@@ -371,6 +371,53 @@ int fpso_pool_knn_backward(const float *grad_pooled, int F, int B, int K, int k,
 }
 
 /*
+ * Charge-weighted token summaries (graphnet PR #923, review thread on the
+ * no-charge case: the tokenizer uses the charge for weighting and for token
+ * summaries, with unit charge when there is no charge column; review thread
+ * on time encoding: a charge-weighted mean time).  The pages do not list the
+ * summaries; the reading taken here, per Voronoi token j of event b with
+ * cell C = {i in b : token_id[i] = j} and q_i = feats[i, charge_col] (1 when
+ * charge_col = -1):
+ *   wsum[b,j]      = sum_{i in C} q_i
+ *   wcoords[b,j,:] = sum q_i * coords[i,:] / wsum   (position and time)
+ *   wfeats[b,j,:]  = sum q_i * feats[i,:] / wsum
+ * sums in float64 in point order, each output rounded once to float32; the
+ * means are 0 when the cell is empty or wsum <= 0.
+ */
+int fpso_token_summaries(const float *coords, const float *feats, int F, int charge_col, const int64_t *offsets,
+                         int B, int K, const int32_t *token_id, float *wsum, float *wcoords, float *wfeats)
+{
+    if (K < 1 || F < 1 || charge_col < -1 || charge_col >= F || bad_offsets(offsets, B)) return -1;
+    const int V = 1 + 4 + F;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)K * V);
+    for (int b = 0; b < B; ++b) {
+        for (int64_t e = 0; e < (int64_t)K * V; ++e) acc[e] = 0.0;
+        for (int64_t i = offsets[b]; i < offsets[b + 1]; ++i) {
+            int32_t j = token_id[i];
+            if (j < 0) continue;
+            if (j >= K) {
+                free(acc);
+                return -1;
+            }
+            double q = charge_col >= 0 ? (double)feats[i * F + charge_col] : 1.0;
+            double *a = acc + (int64_t)j * V;
+            a[0] += q;
+            for (int c = 0; c < 4; ++c) a[1 + c] += q * (double)coords[4 * i + c];
+            for (int f = 0; f < F; ++f) a[5 + f] += q * (double)feats[i * F + f];
+        }
+        for (int j = 0; j < K; ++j) {
+            const double *a = acc + (int64_t)j * V;
+            int64_t r = (int64_t)b * K + j;
+            wsum[r] = (float)a[0];
+            for (int c = 0; c < 4; ++c) wcoords[r * 4 + c] = a[0] > 0.0 ? (float)(a[1 + c] / a[0]) : 0.0f;
+            for (int f = 0; f < F; ++f) wfeats[r * F + f] = a[0] > 0.0 ? (float)(a[5 + f] / a[0]) : 0.0f;
+        }
+    }
+    free(acc);
+    return 0;
+}
+
+/*
  * Packed token layout for block-diagonal attention (graphnet PR #923, "What
  * is added": models/utils.py pack / unpack / build_block_mask; the review
  * thread on the block mask: doc_id holds the event index of every packed

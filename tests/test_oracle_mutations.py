@@ -34,6 +34,10 @@ MUTATIONS = {
                           "g = grad_pooled[((int64_t)b * K + j) * F + f];"),
     "pool_bwd_wrong_event": ("g = (float)((double)grad_pooled[((int64_t)b * K + j) * F + f] / (double)c);",
                              "g = (float)((double)grad_pooled[(int64_t)j * F + f] / (double)c);"),
+    "summary_unweighted_coords": ("for (int c = 0; c < 4; ++c) a[1 + c] += q * (double)coords[4 * i + c];",
+                                  "for (int c = 0; c < 4; ++c) a[1 + c] += (double)coords[4 * i + c];"),
+    "summary_charge_from_col1": ("double q = charge_col >= 0 ? (double)feats[i * F + charge_col] : 1.0;",
+                                 "double q = charge_col >= 0 ? (double)feats[i * F + 1] : 1.0;"),
     "pack_drops_last_token": ("        for (int64_t j = 0; j < v; ++j) {\n            int64_t t = tok_offsets[b] + j;",
                               "        for (int64_t j = 0; j + 1 < v; ++j) {\n            int64_t t = tok_offsets[b] + j;"),
     "unpack_no_zero_pad": ("j < v ? src[(tok_offsets[b] + j) * D + d] : 0.0f;",
@@ -45,7 +49,7 @@ MUTATIONS = {
 PINS = [
     pins.pin_dist_golden, pins.pin_dist_error_bound, pins.pin_fps_fixtures, pins.pin_fps_bruteforce,
     pins.pin_fps_invariants, pins.pin_assign_bruteforce, pins.pin_knn_bruteforce,
-    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint, pins.pin_pack_tokens,
+    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint, pins.pin_pack_tokens, pins.pin_token_summaries,
 ]
 
 

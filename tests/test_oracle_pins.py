@@ -377,6 +377,40 @@ def test_pool_backward_closed_forms():
     assert dX.tolist() == [[1, 0], [4, 1], [0, 0]]
 
 
+# ---------------------------------------------------------------- token summaries
+
+def pin_token_summaries():
+    for b, K, valid, cents, tok in list(_backward_cases())[:16]:
+        B = len(b.offsets) - 1
+        ev = np.repeat(np.arange(B), np.diff(b.offsets))
+        # unit charge: the total is the count, the means the plain means
+        wsum, wc, wf = oracle.token_summaries(b.coords, b.feats, b.offsets, K, tok, charge_col=-1)
+        pooled, counts = bf.pool_voronoi(b.feats, b.offsets, K, tok)
+        assert np.array_equal(wsum, counts.astype(np.float32))
+        np.testing.assert_allclose(wf, pooled, rtol=1e-6, atol=1e-7)
+        cm, _ = bf.pool_voronoi(b.coords, b.offsets, K, tok)
+        np.testing.assert_allclose(wc, cm, rtol=1e-6, atol=1e-5)
+        # charge column 0: numpy's weighted average per cell
+        wsum, wc, wf = oracle.token_summaries(b.coords, b.feats, b.offsets, K, tok, charge_col=0)
+        q = b.feats[:, 0].astype(np.float64)
+        for e in range(B):
+            for j in range(K):
+                m = (ev == e) & (tok == j)
+                W = q[m].sum()
+                assert np.isclose(wsum[e, j], W, rtol=1e-6, atol=1e-7)
+                if m.any() and W > 0:
+                    np.testing.assert_allclose(wc[e, j], np.average(b.coords[m].astype(np.float64), 0, q[m]),
+                                               rtol=1e-6, atol=1e-5)
+                    np.testing.assert_allclose(wf[e, j], np.average(b.feats[m].astype(np.float64), 0, q[m]),
+                                               rtol=1e-5, atol=1e-6)
+                else:
+                    assert not wc[e, j].any() and not wf[e, j].any()
+
+
+def test_token_summaries():
+    pin_token_summaries()
+
+
 # ---------------------------------------------------------------- packed tokens
 
 def pin_pack_tokens():
