@@ -48,11 +48,14 @@ def bind(path: str):
     lib.fpso_pool_knn_backward.argtypes = [P, I, I, I, I, P, P, ctypes.c_int64, P]
     lib.fpso_pack_tokens.argtypes = [P, I, P, P, I, I, P, P, P]
     lib.fpso_token_summaries.argtypes = [P, P, I, I, P, I, I, P, P, P, P]
+    lib.fpso_philox4x32_10.argtypes = [P, P, P]
+    lib.fpso_philox4x32_10.restype = None
+    lib.fpso_random_starts.argtypes = [P, I, ctypes.c_uint64, ctypes.c_uint32, P]
     lib.fpso_unpack_tokens.argtypes = [P, I, P, I, I, P]
     for f in (lib.fpso_fps, lib.fpso_assign, lib.fpso_knn, lib.fpso_lloyd,
               lib.fpso_pool_voronoi, lib.fpso_pool_knn, lib.fpso_tokenize,
               lib.fpso_pool_voronoi_backward, lib.fpso_pool_knn_backward, lib.fpso_pack_tokens,
-              lib.fpso_unpack_tokens, lib.fpso_token_summaries):
+              lib.fpso_unpack_tokens, lib.fpso_token_summaries, lib.fpso_random_starts):
         f.restype = I
     return lib
 
@@ -199,6 +202,25 @@ def pool_knn_backward(grad_pooled, knn_idx, counts, P: int):
     out = np.empty((P, F), np.float32)
     _check(_load().fpso_pool_knn_backward(_p(grad_pooled), F, B, K, k, _p(knn_idx), _p(_i32(counts)), P,
                                           _p(out)), "pool_knn_backward")
+    return out
+
+
+def philox4x32_10(counter, key):
+    """One Philox4x32-10 block: four 32-bit words for a 4-word counter and a
+    2-word key."""
+    c = np.ascontiguousarray(counter, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.empty(4, np.uint32)
+    _load().fpso_philox4x32_10(_p(c), _p(k), _p(out))
+    return out
+
+
+def random_starts(offsets, seed: int, stream: int = 0):
+    """Random local FPS start index per event from Philox4x32-10."""
+    offsets = _i64(offsets)
+    B = offsets.shape[0] - 1
+    out = np.empty(B, np.int32)
+    _check(_load().fpso_random_starts(_p(offsets), B, seed, stream, _p(out)), "random_starts")
     return out
 
 

@@ -371,6 +371,60 @@ int fpso_pool_knn_backward(const float *grad_pooled, int F, int B, int K, int k,
 }
 
 /*
+ * Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+ * easy as 1, 2, 3", SC 2011), written from its definition: ten rounds of
+ *   (hi0, lo0) = M0 * c0,  (hi1, lo1) = M1 * c2   (32 x 32 -> 64-bit products)
+ *   c <- (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0)
+ * with M0 = 0xD2511F53, M1 = 0xCD9E8D57, and the key raised by the Weyl
+ * constants (0x9E3779B9, 0xBB67AE85) between rounds.
+ */
+void fpso_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+        c0 = n0;
+        c1 = n1;
+        c2 = n2;
+        c3 = n3;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+/*
+ * Random FPS start points (graphnet PR #923, review thread on the FPS
+ * arguments: start_idx, random_start and a generator).  Reading: event b
+ * starts at start_local[b] = floor(u * N_b / 2^32), u the first word of
+ * Philox4x32-10 at counter (b, stream, 0, 0) under key (seed low word, seed
+ * high word); 0 for an empty event.
+ */
+int fpso_random_starts(const int64_t *offsets, int B, uint64_t seed, uint32_t stream, int32_t *start_local)
+{
+    if (B < 0 || bad_offsets(offsets, B)) return -1;
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (int b = 0; b < B; ++b) {
+        const uint32_t ctr[4] = {(uint32_t)b, stream, 0u, 0u};
+        uint32_t x[4];
+        fpso_philox4x32_10(ctr, key, x);
+        uint64_t n = (uint64_t)(offsets[b + 1] - offsets[b]);
+        start_local[b] = (int32_t)(((uint64_t)x[0] * n) >> 32);
+    }
+    return 0;
+}
+
+/*
  * Charge-weighted token summaries (graphnet PR #923, review thread on the
  * no-charge case: the tokenizer uses the charge for weighting and for token
  * summaries, with unit charge when there is no charge column; review thread

@@ -34,6 +34,9 @@ MUTATIONS = {
                           "g = grad_pooled[((int64_t)b * K + j) * F + f];"),
     "pool_bwd_wrong_event": ("g = (float)((double)grad_pooled[((int64_t)b * K + j) * F + f] / (double)c);",
                              "g = (float)((double)grad_pooled[(int64_t)j * F + f] / (double)c);"),
+    "philox_no_key_bump": ("            k0 += 0x9E3779B9u;\n", ""),
+    "philox_swapped_words": ("uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;",
+                             "uint32_t n0 = hi0 ^ c1 ^ k0, n1 = lo0, n2 = hi1 ^ c3 ^ k1, n3 = lo1;"),
     "summary_unweighted_coords": ("for (int c = 0; c < 4; ++c) a[1 + c] += q * (double)coords[4 * i + c];",
                                   "for (int c = 0; c < 4; ++c) a[1 + c] += (double)coords[4 * i + c];"),
     "summary_charge_from_col1": ("double q = charge_col >= 0 ? (double)feats[i * F + charge_col] : 1.0;",
@@ -49,7 +52,7 @@ MUTATIONS = {
 PINS = [
     pins.pin_dist_golden, pins.pin_dist_error_bound, pins.pin_fps_fixtures, pins.pin_fps_bruteforce,
     pins.pin_fps_invariants, pins.pin_assign_bruteforce, pins.pin_knn_bruteforce,
-    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint, pins.pin_pack_tokens, pins.pin_token_summaries,
+    pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint, pins.pin_pack_tokens, pins.pin_token_summaries, pins.pin_random_starts,
 ]
 
 

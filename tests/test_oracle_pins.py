@@ -377,6 +377,44 @@ def test_pool_backward_closed_forms():
     assert dX.tolist() == [[1, 0], [4, 1], [0, 0]]
 
 
+# ---------------------------------------------------------------- random starts
+#
+# Known-answer vectors of Philox4x32-10 as published with the generator
+# (Salmon et al., SC 2011, and its reference distribution): counter, key,
+# expected output.
+PHILOX_KAT = [
+    ([0, 0, 0, 0], [0, 0], [0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8]),
+    ([0xffffffff] * 4, [0xffffffff] * 2, [0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd]),
+    ([0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344], [0xa4093822, 0x299f31d0],
+     [0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1]),
+]
+
+
+def pin_random_starts():
+    for ctr, key, want in PHILOX_KAT:
+        assert oracle.philox4x32_10(ctr, key).tolist() == want
+    rng = np.random.default_rng(120)
+    sizes = np.concatenate([[0, 1, 2, 3], rng.integers(1, 5000, 4000)])
+    offsets = np.concatenate([[0], np.cumsum(sizes)])
+    st = oracle.random_starts(offsets, seed=0x123456789ABCDEF, stream=7)
+    # the multiply-shift of the first Philox word, recomputed in Python integers
+    for b in range(6):
+        u = int(oracle.philox4x32_10([b, 7, 0, 0], [0x89ABCDEF, 0x1234567])[0])
+        assert st[b] == (u * int(sizes[b])) >> 32
+    assert np.all((st >= 0) & ((st < sizes) | (sizes == 0)))
+    # roughly uniform: the start's position within its event
+    frac = st[sizes > 100] / sizes[sizes > 100]
+    hist = np.histogram(frac, bins=10, range=(0, 1))[0]
+    assert hist.min() > 0.7 * hist.mean()
+    # another seed or stream gives other starts
+    assert not np.array_equal(st, oracle.random_starts(offsets, seed=1, stream=7))
+    assert not np.array_equal(st, oracle.random_starts(offsets, seed=0x123456789ABCDEF, stream=8))
+
+
+def test_random_starts():
+    pin_random_starts()
+
+
 # ---------------------------------------------------------------- token summaries
 
 def pin_token_summaries():
