@@ -480,6 +480,7 @@ def main():
         if not args.no_backward:
             result["pool_backward"] = pool_backward_roofline(fps, dev)
             result["token_pack"] = token_pack_roofline(fps, dev)
+            result["token_summaries"] = token_summaries_roofline(fps, dev)
         if world == 1 and not args.no_cpu_baseline:
             rate, reps, el = cpu_oracle_rate(batch, args.cpu_seconds)
             result["cpu_baseline"] = {"value": rate, "unit": "events/s", "cores": 1, "kind": "oracle",
@@ -632,6 +633,72 @@ def pool_backward_roofline(fps, dev, reps=50):
             "kernels_per_call": n_warm / 3,
             "note": "memset + per-event row masks and row-order sums + rounding, timed together" if k else "quotient table + gather"}
     return out
+
+
+def token_summaries_roofline(fps, dev, reps=30):
+    """HBM roofline of the charge-weighted token summaries (C
+    ``fps_token_summaries``) on the large-event workload's shapes (8 events,
+    about 0.9 M points, K = 128, F = 6, charge column 0) with seeded random
+    labels.  Graph-replayed and timed like ``pool_backward_roofline``."""
+    import ctypes
+    import json as _j
+
+    import torch
+
+    lib = fps.load_library()
+    peaks = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    b = workloads.make_workload("c3")
+    B, K, F, P = b.B, b.K, b.feats.shape[1], int(b.offsets[-1])
+    rng = np.random.default_rng(96)
+    coords = torch.from_numpy(b.coords).to(dev)
+    feats = torch.from_numpy(b.feats).to(dev)
+    offsets = torch.from_numpy(b.offsets).to(dev)
+    tok = torch.from_numpy(rng.integers(0, K, P).astype(np.int32)).to(dev)
+    wsum = torch.empty((B, K), dtype=torch.float32, device=dev)
+    wc = torch.empty((B, K, 4), dtype=torch.float32, device=dev)
+    wf = torch.empty((B, K, F), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(lib.fps_token_summaries_workspace_bytes(B, K, F), 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    vp = ctypes.c_void_p
+
+    def call(strm):
+        st = lib.fps_token_summaries(vp(coords.data_ptr()), vp(feats.data_ptr()), F, 0, vp(offsets.data_ptr()), B,
+                                     P, K, vp(tok.data_ptr()), vp(wsum.data_ptr()), vp(wc.data_ptr()),
+                                     vp(wf.data_ptr()), vp(ws.data_ptr()), ws.numel(), vp(strm.cuda_stream))
+        if st != 0:
+            raise RuntimeError(f"fps_token_summaries failed: {st}")
+
+    n_before = lib.fps_launch_count()
+    for _ in range(3):
+        call(stream)
+    torch.cuda.synchronize(dev)
+    per_call = (lib.fps_launch_count() - n_before) / 3
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(g, stream=cap):
+        call(cap)
+    torch.cuda.synchronize(dev)
+    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        st_ev[i].record(stream)
+        g.replay()
+        en_ev[i].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = float(np.mean([a.elapsed_time(c) for a, c in zip(st_ev, en_ev)]))
+    del g
+    byts = 16 * P + 4 * F * P + 4 * P + 8 * (B + 1) + B * K * (4 + 16 + 4 * F)
+    achieved = byts / (ms / 1e3) / 1e9
+    return {"workload": f"c3 shapes: B={B}, P={P}, K={K}, F={F}, charge column 0", "us_per_call": ms * 1e3,
+            "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "algorithmic_bytes": byts,
+            "algorithmic": "16P coords + 4FP feats + 4P token ids + 8(B+1) offsets read, B*K*(4+16+4F) written",
+            "kernels_per_call": per_call, "note": "memset + tile sums + finalize"}
 
 
 def token_pack_roofline(fps, dev, reps=50):

@@ -45,6 +45,9 @@ SIGNATURES = [
     ("segment_pool", I, [P, I, P, I, I64, I, I, P, P, I, P, P, P, SZ, P]),
     ("segment_pool_backward_workspace_bytes", SZ, [I64, I, I, I, I]),
     ("segment_pool_backward", I, [P, I, P, I, I64, I, I, P, P, I, P, P, P, SZ, P]),
+    ("fps_random_starts", I, [P, I, ctypes.c_uint64, ctypes.c_uint32, P, P]),
+    ("fps_token_summaries_workspace_bytes", SZ, [I, I, I]),
+    ("fps_token_summaries", I, [P, P, I, I, P, I, I64, I, P, P, P, P, P, SZ, P]),
     ("fps_pack_workspace_bytes", SZ, []),
     ("fps_pack_tokens", I, [P, I, P, P, I, I, P, P, P, P, SZ, P]),
     ("fps_unpack_tokens", I, [P, I, I64, P, I, I, P, P, SZ, P]),

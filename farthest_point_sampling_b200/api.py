@@ -110,7 +110,8 @@ def fps_tokenize(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tenso
                  charge_col: int = -1, start_local: Optional[torch.Tensor] = None,
                  force_schedule: int = -1, max_event_hint: int = 0,
                  workspace: Optional[torch.Tensor] = None, out: Optional[Dict[str, torch.Tensor]] = None,
-                 check_device: bool = False) -> Dict[str, torch.Tensor]:
+                 check_device: bool = False, random_start: bool = False, seed: int = 0,
+                 stream_id: int = 0) -> Dict[str, torch.Tensor]:
     """The whole tokenizer (C ``fps_tokenize``): FPS fused with Voronoi labels,
     optional charge-weighted Lloyd, then Voronoi mean-pool or kNN gather + pool.
 
@@ -119,7 +120,9 @@ def fps_tokenize(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tenso
     ``pooled [B,K,F]`` and ``counts [B,K]``.  ``offsets`` may live on the host,
     in which case the largest event size is passed to the library as a
     scheduling hint.  ``check_device=True`` synchronises and raises on a
-    device-side check failure (bad offsets or start index).
+    device-side check failure (bad offsets or start index).  With
+    ``random_start`` each event starts at a Philox4x32-10 draw for ``seed``
+    and ``stream_id`` (see :func:`random_starts`) instead of ``start_local``.
     """
     dev = _cuda_device(coords)
     _need(coords, "coords", torch.float32, 2, dev)
@@ -129,6 +132,10 @@ def fps_tokenize(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tenso
     if feats.shape[0] != coords.shape[0]:
         raise ValueError("feats and coords must have the same number of rows")
     offsets, hint = _prep_offsets(offsets, dev, max_event_hint)
+    if random_start:
+        if start_local is not None:
+            raise ValueError("give start_local or random_start, not both")
+        start_local = random_starts(offsets, seed, stream_id)
     if start_local is not None:
         _need(start_local, "start_local", torch.int32, 1, dev)
     opts = Options(K, assign_mode, k, lloyd_iters, charge_col, force_schedule, hint)
@@ -338,6 +345,46 @@ def segment_pool_backward(grad_pooled: torch.Tensor, counts: torch.Tensor, P: in
                                    _stream(dev))
     _lib.check(st, "segment_pool_backward")
     return grad_feats
+
+
+def random_starts(offsets: torch.Tensor, seed: int, stream_id: int = 0) -> torch.Tensor:
+    """C ``fps_random_starts``: a Philox4x32-10 draw of one local FPS start
+    index per event, int32 [B] on the device (for ``start_local``)."""
+    dev = _cuda_device(offsets)
+    _need(offsets, "offsets", torch.int64, 1, dev)
+    B = offsets.numel() - 1
+    out = torch.empty(max(B, 0), dtype=torch.int32, device=dev)
+    st = _lib.load().fps_random_starts(_ptr(offsets), B, int(seed) & 0xFFFFFFFFFFFFFFFF,
+                                       int(stream_id) & 0xFFFFFFFF, _ptr(out), _stream(dev))
+    _lib.check(st, "fps_random_starts")
+    return out
+
+
+def token_summaries(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tensor, K: int,
+                    token_id: torch.Tensor, charge_col: int = -1, workspace: Optional[torch.Tensor] = None):
+    """C ``fps_token_summaries``: per Voronoi token the total charge and the
+    charge-weighted means of the coordinates and features (unit charge when
+    ``charge_col`` is -1).  Returns ``(wsum [B,K], wcoords [B,K,4],
+    wfeats [B,K,F])``."""
+    dev = _cuda_device(coords)
+    _need(coords, "coords", torch.float32, 2, dev)
+    _need(feats, "feats", torch.float32, 2, dev)
+    _need(offsets, "offsets", torch.int64, 1, dev)
+    _need(token_id, "token_id", torch.int32, 1, dev)
+    P, F = feats.shape
+    if coords.shape != (P, 4) or token_id.numel() != P:
+        raise ValueError("coords must be [P, 4] and token_id [P] for feats [P, F]")
+    B = offsets.numel() - 1
+    lib = _lib.load()
+    ws = _workspace(lib.fps_token_summaries_workspace_bytes(B, K, F), dev, workspace)
+    wsum = torch.empty((B, K), dtype=torch.float32, device=dev)
+    wcoords = torch.empty((B, K, 4), dtype=torch.float32, device=dev)
+    wfeats = torch.empty((B, K, F), dtype=torch.float32, device=dev)
+    st = lib.fps_token_summaries(_ptr(coords), _ptr(feats), F, charge_col, _ptr(offsets), B, P, K,
+                                 _ptr(token_id), _ptr(wsum), _ptr(wcoords), _ptr(wfeats), _ptr(ws), ws.numel(),
+                                 _stream(dev))
+    _lib.check(st, "fps_token_summaries")
+    return wsum, wcoords, wfeats
 
 
 def pack_tokens(src: torch.Tensor, offsets: Optional[torch.Tensor] = None,

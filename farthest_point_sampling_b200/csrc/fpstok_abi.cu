@@ -9,6 +9,8 @@
 #include "internal.h"
 #include "pool_backward.h"
 #include "token_pack.h"
+#include "token_summary.h"
+#include "random_start.h"
 
 namespace fpstok {
 
@@ -469,6 +471,40 @@ int segment_pool_backward(const float* grad_pooled, int F, const int64_t* offset
   }
   return from_cuda(launch_pool_bwd_voronoi(grad_pooled, F, offsets, B, P, K, token_id, counts,
                                            reinterpret_cast<float*>(scratch), grad_feats, hdr, s));
+}
+
+int fps_random_starts(const int64_t* offsets, int B, uint64_t seed, uint32_t stream_id, int32_t* start_local,
+                      fps_stream_t stream) {
+  if (B < 0) return FPS_ERR_ARG;
+  if (B == 0) return FPS_OK;
+  if (!offsets || !start_local) return FPS_ERR_ARG;
+  return from_cuda(launch_random_starts(offsets, B, seed, stream_id, start_local, nullptr,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t fps_token_summaries_workspace_bytes(int B, int K, int F) {
+  if (B < 0 || K < 1 || F < 1) return 0;
+  return align256(sizeof(WsHeader)) + align256((size_t)B * K * (5 + F) * sizeof(double));
+}
+
+int fps_token_summaries(const float* coords, const float* feats, int F, int charge_col, const int64_t* offsets,
+                        int B, int64_t P, int K, const int32_t* token_id, float* wsum, float* wcoords,
+                        float* wfeats, void* workspace, size_t workspace_bytes, fps_stream_t stream) {
+  int rc = check_common(P, B, offsets);
+  if (rc) return rc;
+  if (K < 1 || F < 1 || charge_col < -1 || charge_col >= F) return FPS_ERR_ARG;
+  if (K > FPS_MAX_K || F > FPS_MAX_F) return FPS_ERR_TOO_LARGE;
+  if (B == 0) return FPS_OK;
+  if (!wsum || !wcoords || !wfeats || (P > 0 && (!coords || !feats || !token_id))) return FPS_ERR_ARG;
+  const size_t need = fps_token_summaries_workspace_bytes(B, K, F);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + align256(sizeof(WsHeader)));
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+  return from_cuda(launch_token_summaries(coords, feats, F, charge_col, offsets, B, P, K, token_id, acc, wsum,
+                                          wcoords, wfeats, hdr, s));
 }
 
 size_t fps_pack_workspace_bytes(void) { return align256(sizeof(WsHeader)); }

@@ -239,6 +239,42 @@ int segment_pool_backward(const float *grad_pooled, int F, const int64_t *offset
                           size_t workspace_bytes, fps_stream_t stream);
 
 /*
+ * Random FPS start points (graphnet PR #923, review thread on the FPS
+ * arguments: start_idx, random_start and a generator), for fps_tokenize's
+ * start_local.  start_local[b] = floor(u * N_b / 2^32) with u the first word
+ * of Philox4x32-10 (Salmon et al., SC 2011) at counter (b, stream_id, 0, 0)
+ * under the key (seed & 0xffffffff, seed >> 32); 0 for an empty event (or
+ * for an event whose offsets are inconsistent).  Deterministic for a given
+ * seed and stream_id; change stream_id to draw new starts from the same
+ * seed.  No workspace.
+ */
+int fps_random_starts(const int64_t *offsets, int B, uint64_t seed, uint32_t stream_id,
+                      int32_t *start_local, fps_stream_t stream);
+
+/*
+ * Charge-weighted token summaries (graphnet PR #923, review thread on the
+ * no-charge case: the tokenizer uses the charge for weighting and for token
+ * summaries, unit charge when there is no charge column; review thread on
+ * time encoding: the charge-weighted mean time).  The pages do not list the
+ * summaries; this library's reading, per Voronoi token j of event b over the
+ * points with token_id == j and q = feats[:, charge_col] (1 when
+ * charge_col = -1):
+ *   wsum    float32 [B, K]    = sum q
+ *   wcoords float32 [B, K, 4] = sum q * coords / wsum   (x, y, z, t)
+ *   wfeats  float32 [B, K, F] = sum q * feats / wsum
+ * Sums in float64 (in no fixed order), each output rounded once to float32;
+ * the means are 0 for an empty cell or wsum <= 0.  Token ids outside -1..K-1
+ * and offsets that do not cover the points are skipped and reported by
+ * fps_device_status().  Workspace: the size below (B * K * (5 + F) * 8 bytes
+ * and a status word), 256-byte aligned.
+ */
+size_t fps_token_summaries_workspace_bytes(int B, int K, int F);
+int fps_token_summaries(const float *coords, const float *feats, int F, int charge_col,
+                        const int64_t *offsets, int B, int64_t P, int K, const int32_t *token_id,
+                        float *wsum, float *wcoords, float *wfeats, void *workspace,
+                        size_t workspace_bytes, fps_stream_t stream);
+
+/*
  * Packed token layout for block-diagonal attention (graphnet PR #923, "What
  * is added": models/utils.py pack / unpack / build_block_mask; review thread
  * on the block mask: doc_id is the event index of every packed token, and

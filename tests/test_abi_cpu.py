@@ -118,6 +118,15 @@ def test_standalone_argument_errors():
     assert upk(x, 4, -1, x, 2, 8, x, x, wsb, None) == _lib.FPS_ERR_ARG  # n_tok < 0
     assert upk(x, 4, 10, None, 2, 8, x, x, wsb, None) == _lib.FPS_ERR_ARG  # no tok_offsets
     assert upk(x, 4, 10, x, 0, 8, x, x, wsb, None) == _lib.FPS_OK  # B = 0
+    # fps_token_summaries(coords, feats, F, charge_col, offsets, B, P, K, token_id, wsum, wc, wf, ws, n, s)
+    ts = lib.fps_token_summaries
+    nts = lib.fps_token_summaries_workspace_bytes(2, 8, 6)
+    assert nts >= 2 * 8 * 11 * 8
+    assert ts(x, x, 6, 6, x, 2, 100, 8, x, x, x, x, x, nts, None) == _lib.FPS_ERR_ARG  # charge_col >= F
+    assert ts(x, x, 6, -2, x, 2, 100, 8, x, x, x, x, x, nts, None) == _lib.FPS_ERR_ARG
+    assert ts(x, x, 6, 0, x, 2, 100, 300, x, x, x, x, x, nts, None) == _lib.FPS_ERR_TOO_LARGE
+    assert ts(x, x, 6, 0, x, 2, 100, 8, None, x, x, x, x, nts, None) == _lib.FPS_ERR_ARG  # no token ids
+    assert ts(x, x, 6, 0, x, 2, 100, 8, x, x, x, x, x, nts - 1, None) == _lib.FPS_ERR_WORKSPACE
 
 
 def test_workspace_sizes_grow_with_problem():
