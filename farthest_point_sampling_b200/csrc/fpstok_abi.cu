@@ -484,7 +484,8 @@ int fps_random_starts(const int64_t* offsets, int B, uint64_t seed, uint32_t str
 
 size_t fps_token_summaries_workspace_bytes(int B, int K, int F) {
   if (B < 0 || K < 1 || F < 1) return 0;
-  return align256(sizeof(WsHeader)) + align256((size_t)B * K * (5 + F) * sizeof(double));
+  return align256(sizeof(WsHeader)) +
+         align256((size_t)token_summary_replicas(B, K, F) * B * K * (5 + F) * sizeof(double));
 }
 
 int fps_token_summaries(const float* coords, const float* feats, int F, int charge_col, const int64_t* offsets,
@@ -496,6 +497,7 @@ int fps_token_summaries(const float* coords, const float* feats, int F, int char
   if (K > FPS_MAX_K || F > FPS_MAX_F) return FPS_ERR_TOO_LARGE;
   if (B == 0) return FPS_OK;
   if (!wsum || !wcoords || !wfeats || (P > 0 && (!coords || !feats || !token_id))) return FPS_ERR_ARG;
+  if (P > 0 && !aligned(coords, 16)) return FPS_ERR_ARG;
   const size_t need = fps_token_summaries_workspace_bytes(B, K, F);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

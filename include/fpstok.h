@@ -265,8 +265,9 @@ int fps_random_starts(const int64_t *offsets, int B, uint64_t seed, uint32_t str
  * Sums in float64 (in no fixed order), each output rounded once to float32;
  * the means are 0 for an empty cell or wsum <= 0.  Token ids outside -1..K-1
  * and offsets that do not cover the points are skipped and reported by
- * fps_device_status().  Workspace: the size below (B * K * (5 + F) * 8 bytes
- * and a status word), 256-byte aligned.
+ * fps_device_status().  Workspace: the size below, 256-byte aligned: up to
+ * 16 copies of a B * K * (5 + F) float64 accumulator (as many as fit in
+ * 32 MiB, at least one) and a status word.
  */
 size_t fps_token_summaries_workspace_bytes(int B, int K, int F);
 int fps_token_summaries(const float *coords, const float *feats, int F, int charge_col,
