@@ -115,7 +115,7 @@ def shard(batch, events):
 
 
 def algorithmic(batch):
-    """Distance evaluations and bytes of one step (the design doc accounting)."""
+    """Distance evaluations and algorithmic bytes of one step."""
     sizes = batch.sizes()
     K, F = batch.K, batch.F
     fpsev = sizes[sizes > K]

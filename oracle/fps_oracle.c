@@ -19,7 +19,7 @@
  *   backends always compute in float32.  Review thread on the no-charge case:
  *   unit charge when there is no charge column.
  *
- * Readings where the pages are silent (each one also listed in the design doc):
+ * Readings where the pages are silent:
  *   - distance d(i,c) = ((dx*dx + dy*dy) + dz*dz) + dt*dt in float32, each
  *     operation rounded to nearest, no fused multiply-add (build with
  *     -ffp-contract=off), raw (x,y,z,t), t unscaled;
