@@ -147,6 +147,22 @@ def test_binding_rejects_cpu_tensors_and_dtypes():
         fps.fps_tokenize(c, torch.zeros((10, 6)), torch.tensor([0, 10]), K=4)
     with pytest.raises(TypeError):
         fps.offsets_from_batch_ids(torch.zeros(5, dtype=torch.int32))
+    # every other entry point refuses host tensors too: there is no CPU path
+    off = torch.tensor([0, 10])
+    tok = torch.zeros(10, dtype=torch.int32)
+    calls = [
+        lambda: fps.segment_pool_backward(torch.zeros((1, 4, 6)), torch.zeros((1, 4), dtype=torch.int32), 10,
+                                          offsets=off, token_id=tok),
+        lambda: fps.segment_mean(torch.zeros((10, 6)), off, 4, token_id=tok),
+        lambda: fps.token_summaries(c, torch.zeros((10, 6)), off, 4, tok),
+        lambda: fps.random_starts(off, 1),
+        lambda: fps.pack_tokens(torch.zeros((1, 4, 6)), offsets=off),
+        lambda: fps.unpack_tokens(torch.zeros((4, 6)), torch.tensor([0, 4]), 4),
+        lambda: fps.segment_pool(torch.zeros((10, 6)), off, 4, token_id=tok),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
 
 
 def test_offsets_from_batch_ids():
