@@ -257,8 +257,14 @@ def cpu_oracle_rate_parallel(batch, seconds, rate1, max_workers=64):
     except AttributeError:
         cores = os.cpu_count() or 1
     w = max(1, min(cores, max_workers, batch.B))
-    parts = [shard(batch, p) for p in partition_events(batch.sizes(), batch.K, w)]
-    reps = max(1, int(round(seconds * rate1 * w / max(batch.B, 1))))
+    idx = partition_events(batch.sizes(), batch.K, w)
+    parts = [shard(batch, p) for p in idx]
+    # passes sized so that the largest slice (the map waits for it) runs about `seconds`
+    cost = event_cost(batch.sizes(), batch.K).astype(np.float64)
+    total = float(cost.sum())
+    share = max(float(cost[p].sum()) for p in idx) / total if total > 0 else 1.0 / w
+    t_pass = batch.B / max(rate1, 1e-9)  # one single-core pass over the whole batch
+    reps = max(1, int(round(seconds / max(t_pass * share, 1e-9))))
     with mp.get_context("spawn").Pool(w, initializer=_oracle_worker_init) as pool:
         pool.map(_oracle_slice, [(p, 1) for p in parts], chunksize=1)  # warm every worker
         t0 = time.perf_counter()
