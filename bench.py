@@ -3,13 +3,17 @@
 
 One step = one ``fps_tokenize`` call over one batch (binning, passthrough, FPS
 fused with the Voronoi labels, Lloyd if configured, kNN or Voronoi pooling),
-inputs resident in HBM.  The default workload is the 64-event track batch
-(N ~ lognormal(median 300, sigma 1), K = 128, Voronoi assign + mean-pool).
+inputs resident in HBM.  The headline workload is the batched K = 128 case:
+4096 small events (N ~ U{5..400}, about 31% passthrough), Voronoi assign +
+mean-pool.  The same JSON line carries a block for the large-event workload
+(8 showers of 50k-200k points, 3 charge-weighted Lloyd iterations), one for
+the 64-event track batch, and the K sweep (32, 64, 256) of the headline
+events, each timed the same way.
 
 Prints one JSON line (rank 0).  ``value`` is events/s over all GPUs; the
 per-kernel roofline uses CUDA events recorded by the library around each
-internal stage in the timed region.  ``--impl reference`` times the CPU
-oracle instead, on the host cores.
+internal stage in the timed region, against the measured float32 non-FMA op
+rate.  ``--impl reference`` times the CPU oracle instead, on the host cores.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        (N > 1: launch under torch.distributed.run, one process per GPU).
@@ -37,8 +41,10 @@ import workloads  # noqa: E402
 FP32_OPS_PER_EVAL = 11  # 4 sub + 4 mul + 3 add
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
-FP32_OPS_PER_LANE_CLK = 2  # nominal fallback only: the packed add/FMA mix issues ~2 float32 ops per lane per clock
+FP32_OPS_PER_LANE_CLK = 1  # non-FMA float32: one operation per lane per clock (packed or not)
 SM_MAX_MHZ_NOMINAL = 1965.0
+SIDE_WORKLOADS = ("c3", "c1")  # extra blocks on the headline line
+K_SWEEP = (32, 64, 256)  # the headline events at other K
 STAGES = ["bin", "fps_warp", "fps_cta", "fps_cta_smem", "fps_cluster8", "fps_cluster16", "lloyd",
           "knn+pool", "voronoi_pool", "passthrough"]
 STAGE_KERNELS = {0: "k_bin", 1: "k_fps_warp", 2: "k_fps_cta", 3: "k_fps_block<1>",
@@ -46,15 +52,18 @@ STAGE_KERNELS = {0: "k_bin", 1: "k_fps_warp", 2: "k_fps_cta", 3: "k_fps_block<1>
                  8: "k_pool_voronoi", 9: "k_passthrough"}
 FPS_STAGES = (1, 2, 3, 4, 5)
 METRIC = "FPS+assign events/s (K=128)"
+DEFAULT_WORKLOAD = "c4"
 
 
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c1", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--side-steps", type=int, default=300, help="timed steps of each extra block")
+    ap.add_argument("--no-side", action="store_true", help="headline workload only (no extra blocks, no K sweep)")
     ap.add_argument("--K", type=int, default=None, help="override K (c4 sweep)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle sample budget")
@@ -84,34 +93,23 @@ def global_batch(name, n_gpus, K=None):
 
 
 def event_cost(sizes, K):
-    return np.where(sizes > K, sizes.astype(np.float64) * K, sizes.astype(np.float64) * 0.01 + 1.0)
+    from farthest_point_sampling_b200 import sharding
+
+    return sharding.event_cost(sizes, K)
 
 
 def partition_events(sizes, K, world):
-    """Longest-processing-time split of events over ranks by N*K cost."""
-    cost = event_cost(np.asarray(sizes), K)
-    order = np.argsort(-cost, kind="stable")
-    load = np.zeros(world)
-    parts = [[] for _ in range(world)]
-    for e in order:
-        r = int(np.argmin(load))
-        parts[r].append(int(e))
-        load[r] += cost[e]
-    return [np.array(sorted(p), dtype=np.int64) for p in parts]
+    from farthest_point_sampling_b200 import sharding
+
+    return sharding.partition_events(sizes, K, world)
 
 
 def shard(batch, events):
-    sizes = batch.sizes()
-    cs, fs = [], []
-    for e in events:
-        o0, o1 = batch.offsets[e], batch.offsets[e + 1]
-        cs.append(batch.coords[o0:o1])
-        fs.append(batch.feats[o0:o1])
-    off = np.zeros(len(events) + 1, np.int64)
-    np.cumsum(sizes[events], out=off[1:])
-    return workloads.Batch(np.ascontiguousarray(np.concatenate(cs)) if cs else batch.coords[:0],
-                           np.ascontiguousarray(np.concatenate(fs)) if fs else batch.feats[:0], off, batch.K,
-                           batch.assign_mode, batch.k, batch.lloyd_iters, batch.charge_col, None, batch.name)
+    from farthest_point_sampling_b200 import sharding
+
+    c, f, off = sharding.shard_events(batch.coords, batch.feats, batch.offsets, events)
+    return workloads.Batch(c, f, off, batch.K, batch.assign_mode, batch.k, batch.lloyd_iters, batch.charge_col,
+                           None, batch.name)
 
 
 def algorithmic(batch):
@@ -322,6 +320,197 @@ def config_of(batch, args, l2):
 
 # ------------------------------------------------------------------ main
 
+def roofline_peak(mb, sm_count):
+    """The FP32 roofline denominator: the measured non-FMA float32 op rate
+    (the distance is made of separately rounded subtracts, multiplies and
+    adds), refused if it exceeds the issue ceiling of one operation per lane
+    per clock at the maximum SM clock.  Returns (peak TFLOP/s, source)."""
+    ceiling = sm_count * FP32_LANES_PER_SM * FP32_OPS_PER_LANE_CLK * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
+    nominal_src = (f"derived: {sm_count} SMs x {FP32_LANES_PER_SM} FP32 lanes x 1 non-FMA op per lane per clock "
+                   f"x {SM_MAX_MHZ_NOMINAL:.0f} MHz")
+    meas = (mb or {}).get("non_fma_peak")
+    if meas and meas <= 1.02 * ceiling:
+        return meas, ("measured in this run: best of the scalar FMUL+FADD and packed add / multiply chains "
+                      f"(microbench non_fma_peak); issue ceiling {ceiling:.1f}")
+    if meas:
+        return ceiling, f"{nominal_src} (the measured {meas:.1f} exceeded that ceiling and was refused)"
+    return ceiling, nominal_src
+
+
+def measure(fps, lib, batch, full, args, dev, world, rank, steps, flush, want_stages=True):
+    """Times ``steps`` fps_tokenize calls on ``batch`` (this rank's shard of
+    ``full``): eager calls with the library's stage events, then the same call
+    replayed from a CUDA graph.  L2 is flushed (256 MiB write) before every
+    step, outside the timed events.  Returns a dict; times are the max over
+    ranks."""
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    vp = ctypes.c_void_p
+    coords = torch.from_numpy(batch.coords).to(dev)
+    feats = torch.from_numpy(batch.feats).to(dev)
+    offsets = torch.from_numpy(batch.offsets).to(dev)
+    hint = int(batch.sizes().max()) if batch.B else 0
+    kw = dict(K=batch.K, assign_mode=batch.assign_mode, k=max(batch.k, 1), lloyd_iters=batch.lloyd_iters,
+              charge_col=batch.charge_col, max_event_hint=hint)
+    out = fps.fps_tokenize(coords, feats, offsets, check_device=True, **kw)
+    opts = fps.Options(**kw)
+    ws = torch.empty(max(lib.fps_workspace_bytes(batch.P, batch.B, batch.F, ctypes.byref(opts.c)), 256),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def make_call(strm):
+        """One fps_tokenize call with every argument prebuilt (no Python checks)."""
+        a = (vp(coords.data_ptr()), vp(feats.data_ptr()), batch.F, vp(offsets.data_ptr()), batch.B, batch.P,
+             None, ctypes.byref(opts.c), vp(out["centroid_idx"].data_ptr()), vp(out["token_id"].data_ptr()),
+             vp(out["knn_idx"].data_ptr()) if "knn_idx" in out else None, vp(out["centroids"].data_ptr()),
+             vp(out["pooled"].data_ptr()), vp(out["counts"].data_ptr()), vp(ws.data_ptr()), ws.numel(),
+             vp(strm.cuda_stream))
+        fn = lib.fps_tokenize
+
+        def call():
+            rc = fn(*a)
+            if rc:
+                raise fps.FpsError(rc, "fps_tokenize")
+        return call
+
+    step = make_call(stream)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    nst = 2 * len(STAGES)
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(steps)] \
+        if want_stages else []
+    for evs in stage_ev:  # materialise the handles the library records into
+        for e in evs:
+            e.record(stream)
+    stage_arr = [(vp * nst)(*[vp(e.cuda_event) for e in evs]) for evs in stage_ev]
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = fps.launch_count()
+    stage_mask = 0  # stages the library actually ran (host-side record of its stage marks)
+    for i in range(steps):
+        flush.zero_()
+        if want_stages:
+            lib.fps_set_stage_events(stage_arr[i], nst)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+        stage_mask |= lib.fps_stage_mask()
+    lib.fps_set_stage_events(None, 0)
+    torch.cuda.synchronize(dev)
+    launches_per_step = (fps.launch_count() - launches0) / steps
+    eager_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+
+    # the same step replayed from a CUDA graph (launch overhead removed)
+    graph_ms = None
+    if not args.no_graph:
+        g = torch.cuda.CUDAGraph()
+        cap_stream = torch.cuda.Stream(dev)
+        cap_stream.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap_stream):
+            make_call(cap_stream)()
+        torch.cuda.synchronize(dev)
+        for _ in range(args.warmup):
+            flush.zero_()
+            g.replay()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        gs = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            gs[i].record(stream)
+            g.replay()
+            ge[i].record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = sum(a.elapsed_time(b) for a, b in zip(gs, ge)) / steps
+        del g
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+
+    best_ms = graph_ms if graph_ms is not None else eager_ms
+    t = torch.tensor([best_ms, eager_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_per_step, eager_ms = float(t[0].item()), float(t[1].item())
+
+    # per-stage device time (recorded by the library inside the eager steps)
+    stage_ms = {}
+    for s_ in range(len(STAGES)):
+        ts = []
+        for evs in stage_ev:
+            try:
+                ts.append(evs[2 * s_].elapsed_time(evs[2 * s_ + 1]))
+            except RuntimeError:
+                break
+        if stage_ev and len(ts) == steps:
+            stage_ms[s_] = float(np.mean(ts))
+    ran = {s_ for s_ in range(len(STAGES)) if (stage_mask >> s_) & 1}
+    stage_ms = {s_: v for s_, v in stage_ms.items() if s_ in ran}
+    # which schedule every event of this shard ran on (the library's own rule)
+    sizes = batch.sizes()
+    sched = np.array([lib.fps_schedule_for(int(n), batch.K, -1) for n in sizes])
+    if (sched >= 0).sum() <= SM_COUNT:  # few events: the warp class runs on the CTA schedule
+        sched = np.where(sched == 0, 1, sched)
+    if (sched == 2).sum() <= SM_COUNT // 8:  # few mid-size events: 8-CTA clusters
+        sched = np.where(sched == 2, 3, sched)
+    evals_full, bytes_full = algorithmic(full)
+    return {"ms_per_step": ms_per_step, "eager_ms": eager_ms, "graph_ms": graph_ms, "stage_ms": stage_ms,
+            "launches_per_step": launches_per_step, "sched": sched, "kw": kw, "value": full.B / (ms_per_step / 1e3),
+            "evals": evals_full, "bytes": bytes_full}
+
+
+def roofline_block(m, batch, peak, peak_source, hbm, workload):
+    """Roofline of the dominant stage's kernel, plus the whole step against
+    the same bounds (the slower of the bytes at HBM peak and the
+    evaluations at the FP32 peak)."""
+    stage_ms = m["stage_ms"]
+    t_step = m["ms_per_step"] / 1e3
+    evals, byts = m["evals"], m["bytes"]
+    t_roof = max(byts / (hbm * 1e9), evals * FP32_OPS_PER_EVAL / (peak * 1e12))
+    step = {"evals": evals, "bytes": byts, "achieved_tflops": evals * FP32_OPS_PER_EVAL / t_step / 1e12,
+            "roofline_ms": t_roof * 1e3, "frac": t_roof / t_step,
+            "bound": "alu" if evals * FP32_OPS_PER_EVAL / (peak * 1e12) >= byts / (hbm * 1e9) else "hbm"}
+    if not stage_ms:
+        return {"step": step}
+    dom = max(stage_ms, key=stage_ms.get)
+    t_dom = stage_ms[dom] / 1e3
+    if dom in FPS_STAGES:
+        ev = int(sum(int(n) * batch.K for n, s_ in zip(batch.sizes(), m["sched"]) if s_ == dom - 1))
+        achieved = ev * FP32_OPS_PER_EVAL / t_dom / 1e12
+        roof = {"bound": "alu", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_source,
+                "algorithmic": f"{ev} point-centroid evals x {FP32_OPS_PER_EVAL} FP32 ops per launch",
+                "stage_us": stage_ms[dom] * 1e3,
+                "traffic": recorded_traffic(dom, workload)}
+    elif dom == 6:  # Lloyd: N*K re-assign evaluations per iteration
+        ev = int(sum(int(n) * batch.K for n in batch.sizes() if n > batch.K)) * batch.lloyd_iters
+        achieved = ev * FP32_OPS_PER_EVAL / t_dom / 1e12
+        roof = {"bound": "alu", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_source,
+                "algorithmic": f"{ev} point-centroid evals x {FP32_OPS_PER_EVAL} FP32 ops ({batch.lloyd_iters} "
+                               "re-assign passes)",
+                "stage_us": stage_ms[dom] * 1e3, "traffic": recorded_traffic(dom, workload)}
+    else:
+        achieved = byts / t_dom / 1e9
+        roof = {"bound": "hbm", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": hbm,
+                "unit": "GB/s", "frac": achieved / hbm, "stage_us": stage_ms[dom] * 1e3,
+                "traffic": recorded_traffic(dom, workload)}
+    roof["step"] = step
+    return roof
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -344,193 +533,93 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    full = global_batch(args.workload, world, args.K)
-    if world > 1:
-        parts = partition_events(full.sizes(), full.K, world)
-        batch = shard(full, parts[rank])
-    else:
-        batch = full
+    def shard_of(name, K=None):
+        full_ = global_batch(name, world, K)
+        if world > 1:
+            parts = partition_events(full_.sizes(), full_.K, world)
+            return full_, shard(full_, parts[rank])
+        return full_, full_
+
+    full, batch = shard_of(args.workload, args.K)
     fps.build()
-    fps.load_library()
-
-    coords = torch.from_numpy(batch.coords).to(dev)
-    feats = torch.from_numpy(batch.feats).to(dev)
-    offsets = torch.from_numpy(batch.offsets).to(dev)
-    hint = int(batch.sizes().max()) if batch.B else 0
-    kw = dict(K=batch.K, assign_mode=batch.assign_mode, k=max(batch.k, 1), lloyd_iters=batch.lloyd_iters,
-              charge_col=batch.charge_col, max_event_hint=hint)
-    out = fps.fps_tokenize(coords, feats, offsets, check_device=True, **kw)
     lib = fps.load_library()
-    import ctypes
-
-    opts = fps.Options(**kw)
-    ws = torch.empty(lib.fps_workspace_bytes(batch.P, batch.B, batch.F, ctypes.byref(opts.c)), dtype=torch.uint8,
-                     device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    vp = ctypes.c_void_p
 
-    def make_call(strm):
-        """One fps_tokenize call with every argument prebuilt (no Python checks)."""
-        args = (vp(coords.data_ptr()), vp(feats.data_ptr()), batch.F, vp(offsets.data_ptr()), batch.B, batch.P,
-                None, ctypes.byref(opts.c), vp(out["centroid_idx"].data_ptr()), vp(out["token_id"].data_ptr()),
-                vp(out["knn_idx"].data_ptr()) if "knn_idx" in out else None, vp(out["centroids"].data_ptr()),
-                vp(out["pooled"].data_ptr()), vp(out["counts"].data_ptr()), vp(ws.data_ptr()), ws.numel(),
-                vp(strm.cuda_stream))
-        fn = lib.fps_tokenize
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    mb = None
+    if rank == 0 and not args.no_microbench:
+        try:
+            mb = microbench_fp32(dev)
+        except Exception as exc:  # noqa: BLE001
+            mb = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    peak, peak_source = roofline_peak(mb if mb and "error" not in mb else None,
+                                      torch.cuda.get_device_properties(dev).multi_processor_count)
 
-        def call():
-            rc = fn(*args)
-            if rc:
-                raise fps.FpsError(rc, "fps_tokenize")
-        return call
-
-    step = make_call(stream)
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize(dev)
-
-    K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))] for _ in range(K)]
-    for evs in stage_ev:  # materialise the handles the library records into
-        for e in evs:
-            e.record(stream)
-    stage_arr = [(vp * len(evs))(*[vp(e.cuda_event) for e in evs]) for evs in stage_ev]
-    torch.cuda.synchronize(dev)
-
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = fps.launch_count()
-    stage_mask = 0  # stages the library actually ran (host-side record of its stage marks)
     wall0 = time.perf_counter()
     with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as clocks:
-        for i in range(K):
-            flush.zero_()
-            lib.fps_set_stage_events(stage_arr[i], len(STAGES) * 2)
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-            stage_mask |= lib.fps_stage_mask()
-        lib.fps_set_stage_events(None, 0)
-        torch.cuda.synchronize(dev)
-        wall = time.perf_counter() - wall0
-        launches = fps.launch_count() - launches0
-        launches_per_step = launches / K
-        eager_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / K
-
-        # the same step replayed from a CUDA graph (launch overhead removed)
-        graph_ms = None
-        if not args.no_graph:
-            g = torch.cuda.CUDAGraph()
-            cap_stream = torch.cuda.Stream(dev)
-            cap_stream.wait_stream(stream)
-            with torch.cuda.graph(g, stream=cap_stream):
-                make_call(cap_stream)()
-            torch.cuda.synchronize(dev)
-            for _ in range(args.warmup):
-                flush.zero_()
-                g.replay()
-            torch.cuda.synchronize(dev)
-            if world > 1:
-                dist.barrier()
-            gs = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-            ge = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-            for i in range(K):
-                flush.zero_()
-                gs[i].record(stream)
-                g.replay()
-                ge[i].record(stream)
-            torch.cuda.synchronize(dev)
-            graph_ms = sum(a.elapsed_time(b) for a, b in zip(gs, ge)) / K
-            del g
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-
-    best_ms = graph_ms if graph_ms is not None else eager_ms
-    t = torch.tensor([best_ms, eager_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_per_step, eager_ms = float(t[0].item()), float(t[1].item())
-    events_all = full.B
-    value = events_all / (ms_per_step / 1e3)
-    evals, _ = algorithmic(full)
-
-    # per-stage device time (recorded by the library inside the timed steps)
-    stage_ms = {}
-    for s in range(len(STAGES)):
-        ts = []
-        for evs in stage_ev:
-            try:
-                ts.append(evs[2 * s].elapsed_time(evs[2 * s + 1]))
-            except RuntimeError:
-                break
-        if len(ts) == K:
-            stage_ms[s] = float(np.mean(ts))
-    # stages that did not run in this workload keep their warm-up recordings: drop them
-    sizes = batch.sizes()
-    sched = np.array([lib.fps_schedule_for(int(n), batch.K, -1) for n in sizes])
-    if (sched >= 0).sum() <= SM_COUNT:  # few events: the warp class runs on the CTA schedule
-        sched = np.where(sched == 0, 1, sched)
-    if (sched == 2).sum() <= SM_COUNT // 8:  # few mid-size events: 8-CTA clusters
-        sched = np.where(sched == 2, 3, sched)
-    ran = {s for s in range(len(STAGES)) if (stage_mask >> s) & 1}
-    stage_ms = {s: v for s, v in stage_ms.items() if s in ran}
+        m = measure(fps, lib, batch, full, args, dev, world, rank, args.steps, flush)
+    wall = time.perf_counter() - wall0
 
     result = {
-        "metric": METRIC, "value": value, "unit": "events/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": m["value"], "unit": "events/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded generator shaped like the pages' events)",
         "config": config_of(batch, args, l2="flushed between steps (256 MiB write outside the timed events)"),
-        "gevals_per_s": evals / (ms_per_step / 1e3) / 1e9,
-        "gpu_launches": int(round(launches_per_step * K)),
-        "timing": {"graph_replay_ms_per_step": graph_ms, "eager_ms_per_step": eager_ms,
-                   "value_from": "graph replay" if graph_ms is not None else "eager calls",
-                   "kernels_per_step": launches_per_step},
-        "stage_ms": {STAGES[s]: round(v, 5) for s, v in sorted(stage_ms.items())},
+        "gevals_per_s": m["evals"] / (m["ms_per_step"] / 1e3) / 1e9,
+        "gpu_launches": int(round(m["launches_per_step"] * args.steps)),
+        "timing": {"graph_replay_ms_per_step": m["graph_ms"], "eager_ms_per_step": m["eager_ms"],
+                   "value_from": "graph replay" if m["graph_ms"] is not None else "eager calls",
+                   "kernels_per_step": m["launches_per_step"]},
+        "stage_ms": {STAGES[s_]: round(v, 5) for s_, v in sorted(m["stage_ms"].items())},
         "wall_s_timed_region": wall,
     }
-
     if rank == 0:
-        # roofline of the dominant kernel (FP32 issue bound for the FPS kernels)
-        dom = max(stage_ms, key=stage_ms.get)
-        t_dom = stage_ms[dom] / 1e3
-        mb = None if args.no_microbench else microbench_fp32(dev)
-        if mb and mb.get("f32x2_distance"):
-            peak = mb["f32x2_distance"]
-            peak_source = ("measured in this run: rate of the exact 11-op distance as the kernels compile it "
-                           "(microbench mode f32x2_distance); the plain non-FMA chain rate is non_fma_peak")
-        else:
-            peak = SM_COUNT * FP32_LANES_PER_SM * FP32_OPS_PER_LANE_CLK * SM_MAX_MHZ_NOMINAL * 1e6 / 1e12
-            peak_source = "derived: 148 SMs x 128 FP32 lanes x 2 (packed mix) x 1965 MHz"
-        if dom in FPS_STAGES:
-            ev = int(sum(int(n) * batch.K for n, s in zip(sizes, sched) if s == dom - 1))
-            achieved = ev * FP32_OPS_PER_EVAL / t_dom / 1e12
-            roof = {"bound": "alu", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": peak_source,
-                    "algorithmic": f"{ev} point-centroid evals x {FP32_OPS_PER_EVAL} FP32 ops per launch",
-                    "traffic": recorded_traffic(dom, args.workload)}
-        else:
-            _, byts = algorithmic(batch)
-            import json as _j
-
-            peaks = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
-                os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
-            hbm = float(peaks.get("hbm_gbs", 6650.0))
-            achieved = byts / t_dom / 1e9
-            roof = {"bound": "hbm", "kernel": STAGE_KERNELS[dom], "achieved": achieved, "peak": hbm,
-                    "unit": "GB/s", "frac": achieved / hbm, "traffic": recorded_traffic(dom, args.workload)}
+        roof = roofline_block(m, batch, peak, peak_source, hbm, args.workload)
         if mb:
             roof["microbench_fp32_tflops"] = mb
         result["roofline"] = roof
         result["clocks"] = clocks.summary()
         if not args.no_e2e:
-            result["e2e"] = e2e(fps, batch, kw, dev, args.e2e_steps)
+            result["e2e"] = e2e(fps, batch, m["kw"], dev, args.e2e_steps)
+
+    # extra blocks: other workloads and the K sweep, timed the same way (every rank takes part)
+    if not args.no_side:
+        side = {}
+        for name in SIDE_WORKLOADS:
+            if name == args.workload:
+                continue
+            f_, b_ = shard_of(name)
+            with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as ck:
+                ms_ = measure(fps, lib, b_, f_, args, dev, world, rank, args.side_steps, flush)
+            if rank == 0:
+                blk = {"workload": name, "value": ms_["value"], "unit": "events/s", "ms_per_step": ms_["ms_per_step"],
+                       "steps": args.side_steps, "gevals_per_s": ms_["evals"] / (ms_["ms_per_step"] / 1e3) / 1e9,
+                       "config": config_of(b_, args, l2="flushed between steps"),
+                       "stage_ms": {STAGES[s_]: round(v, 5) for s_, v in sorted(ms_["stage_ms"].items())},
+                       "roofline": roofline_block(ms_, b_, peak, peak_source, hbm, name),
+                       "kernels_per_step": ms_["launches_per_step"], "clocks": ck.summary()}
+                if not args.no_e2e:
+                    blk["e2e"] = e2e(fps, b_, ms_["kw"], dev, max(20, args.e2e_steps // 4))
+                side[name] = blk
+        if args.workload == DEFAULT_WORKLOAD and args.K is None:
+            sweep = {}
+            for Kx in K_SWEEP:
+                f_, b_ = shard_of(args.workload, Kx)
+                ms_ = measure(fps, lib, b_, f_, args, dev, world, rank, args.side_steps, flush)
+                if rank == 0:
+                    rb = roofline_block(ms_, b_, peak, peak_source, hbm, f"{args.workload}_K{Kx}")
+                    sweep[str(Kx)] = {"value": ms_["value"], "unit": "events/s", "ms_per_step": ms_["ms_per_step"],
+                                      "gevals_per_s": ms_["evals"] / (ms_["ms_per_step"] / 1e3) / 1e9,
+                                      "stage_ms": {STAGES[s_]: round(v, 5) for s_, v in sorted(ms_["stage_ms"].items())},
+                                      "dominant_frac": rb.get("frac"), "step_frac": rb["step"]["frac"]}
+            if rank == 0:
+                side["k_sweep"] = sweep
+        if rank == 0:
+            result["workloads"] = side
+
+    if rank == 0:
         if not args.no_backward:  # side measurements: a failure is recorded, the line still prints
             for key, fn in (("pool_backward", pool_backward_roofline), ("token_pack", token_pack_roofline),
                             ("token_summaries", token_summaries_roofline)):
@@ -563,8 +652,10 @@ def microbench_fp32(dev):
     """Measured FP32 rates (TFLOP/s, an FMA counted as two) of the microbenchmark modes.
 
     The non-FMA peak is the best of the scalar and the separate packed add and
-    multiply chains; "f32x2_distance" is the rate of the distance exactly as
-    the FPS kernels compute it.
+    multiply chains: the roofline denominator.  "f32x2_distance" is the rate of
+    the distance exactly as the FPS kernels compute it, every input
+    loop-carried; it is reported to show that the packed mix runs at that
+    same non-FMA rate (11 ops per evaluation, one per lane per clock).
     """
     import ctypes
 

@@ -15,9 +15,10 @@ from .api import (Options, device_status, fps_assign, fps_knn, fps_tokenize, fps
                   segment_pool_backward, set_stage_events, token_summaries, unpack_tokens)
 from ._lib import load as load_library, library_path
 from ._build import build, build_microbench
+from . import sharding
 
 __all__ = [
     "FpsError", "Options", "build", "build_microbench", "device_status", "fps_assign", "fps_knn", "fps_tokenize",
     "fps_tokenize_host", "launch_count", "library_path", "load_library", "lloyd_refine",
-    "offsets_from_batch_ids", "pack_tokens", "random_starts", "segment_mean", "segment_pool", "segment_pool_backward", "set_stage_events", "token_summaries", "unpack_tokens",
+    "offsets_from_batch_ids", "pack_tokens", "random_starts", "segment_mean", "segment_pool", "segment_pool_backward", "set_stage_events", "sharding", "token_summaries", "unpack_tokens",
 ]

@@ -35,6 +35,7 @@ SIGNATURES = [
     ("fps_host_workspace_bytes", SZ, [I64, I, I, P]),
     ("fps_tokenize_host", I, [P, P, I, P, I, I64, P, P, P, P, P, P, P, P, P, SZ, P]),
     ("fps_tokenize_static", I, [P, P, I, P, I, I64, P, P, P, P, P, P, P, P, P]),
+    ("fps_static_device_status", I, [P, ctypes.POINTER(I)]),
     ("fps_assign_workspace_bytes", SZ, [I64, I]),
     ("fps_assign", I, [P, P, I, I64, P, P, I, P, P, SZ, P]),
     ("fps_knn_workspace_bytes", SZ, [I64, I]),

@@ -110,6 +110,11 @@ static bool needs_labels(const fps_opts* o, const int32_t* token_id) {
   return o->assign_mode == FPS_ASSIGN_KNN && o->lloyd_iters > 0 && token_id == nullptr;
 }
 
+size_t tokenize_workspace_need(int64_t P, int B, int F, const fps_opts* o, const int32_t* token_id) {
+  if (!o || P < 0 || B < 0 || o->K < 1) return 0;
+  return carve(nullptr, P, B, o->K, F, o->lloyd_iters > 0, needs_labels(o, token_id)).bytes;
+}
+
 static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s) {
   Problem pb = pb0;
   int32_t* labels = pb.token_id ? pb.token_id : ws.labels;

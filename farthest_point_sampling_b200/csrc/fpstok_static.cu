@@ -17,13 +17,22 @@
 // that name is only a host-side stand-in, not a device address.  The device
 // address is looked up once per device with cudaGetSymbolAddress, on the
 // first call made while that device is current; make that first call before
-// any stream capture.  All calls share the one array and it keeps the last
-// call's contents; the tokenizer's kernels clear every scratch word that must
-// start at zero.  Calls whose work overlaps on the GPU (for example on two
-// streams) race on the array.
+// any stream capture.  The looked-up address is kept for the life of the
+// process: after cudaDeviceReset (or anything else that destroys the primary
+// context and unloads the module) it is stale, and calls to this entry point
+// on that device are not supported.  All calls share the one array and it
+// keeps the last call's contents; the tokenizer's kernels clear every scratch
+// word that must start at zero.  Calls whose work overlaps on the GPU (for
+// example on two streams) race on the array.
+//
+// fps_static_device_status reads back the device-side status word of the
+// last call on the current device (bad offsets, a start index outside its
+// event, an exchange that ran out of time), which fps_tokenize keeps at the
+// start of its workspace -- here, of the static array.
 #include <mutex>
 
 #include "../../include/fpstok.h"
+#include "internal.h"
 
 static __device__ __align__(256) unsigned char g_static_scratch[FPS_STATIC_SCRATCH_BYTES];
 
@@ -54,7 +63,7 @@ extern "C" int fps_tokenize_static(const float* coords, const float* feats, int 
                                    int32_t* centroid_idx, int32_t* token_id, int32_t* knn_idx,
                                    float* centroids, float* pooled, int32_t* counts, fps_stream_t stream) {
   if (opts != nullptr && P >= 0 && B >= 0 &&
-      fps_workspace_bytes(P, B, F, opts) > (size_t)FPS_STATIC_SCRATCH_BYTES)
+      fpstok::tokenize_workspace_need(P, B, F, opts, token_id) > (size_t)FPS_STATIC_SCRATCH_BYTES)
     return FPS_ERR_TOO_LARGE;  // the batch needs more scratch than the static array holds
   void* scratch = nullptr;
   if (B > 0) {
@@ -63,4 +72,11 @@ extern "C" int fps_tokenize_static(const float* coords, const float* feats, int 
   }
   return fps_tokenize(coords, feats, F, offsets, B, P, start_local, opts, centroid_idx, token_id, knn_idx,
                       centroids, pooled, counts, scratch, scratch ? (size_t)FPS_STATIC_SCRATCH_BYTES : 0, stream);
+}
+
+extern "C" int fps_static_device_status(fps_stream_t stream, int* detail) {
+  void* scratch = nullptr;
+  const int rc = static_scratch_address(&scratch);
+  if (rc != FPS_OK) return rc;
+  return fps_device_status(scratch, stream, detail);
 }

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+struct fps_opts;  // include/fpstok.h
+
 namespace fpstok {
 
 // Event classes written by the binning kernel.
@@ -130,5 +132,9 @@ const DeviceInfo& device_info();  // prepares the current device on first use
 cudaError_t prepare_aux_kernels();   // shared-memory attributes of the auxiliary kernels
 
 void count_launch(int n = 1);
+
+// Workspace bytes fps_tokenize needs for this exact call (the labels area is
+// reserved only when kNN mode runs Lloyd without a caller token_id buffer).
+size_t tokenize_workspace_need(int64_t P, int B, int F, const ::fps_opts* o, const int32_t* token_id);
 
 }  // namespace fpstok

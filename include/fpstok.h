@@ -148,17 +148,27 @@ int fps_tokenize_host(const float *coords, const float *feats, int F, const int6
  * cause.  Same arguments and results as fps_tokenize, without the workspace:
  * the scratch is a file-scope device array of FPS_STATIC_SCRATCH_BYTES
  * (8 MiB) that every GPU loading the library holds until the process exits.
- * Returns FPS_ERR_TOO_LARGE when the batch needs more scratch than that
- * (fps_workspace_bytes() tells how much it needs).  The first call on each
- * device looks up the array's device address (cudaGetSymbolAddress); make it
- * before any stream capture.  All calls share the array: calls whose work
- * overlaps on the GPU race.  It allocates and frees nothing.
+ * Returns FPS_ERR_TOO_LARGE when the batch needs more scratch than that:
+ * as much as fps_tokenize would take for the same arguments, which is
+ * fps_workspace_bytes() except that kNN mode with Lloyd and a non-NULL
+ * token_id needs no internal labels area.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress); make it before
+ * any stream capture.  That address is kept for the life of the process:
+ * after cudaDeviceReset on a device, calling this entry point there is not
+ * supported.  All calls share the array: calls whose work overlaps on the
+ * GPU race.  It allocates and frees nothing.
  */
 #define FPS_STATIC_SCRATCH_BYTES (8u << 20)
 int fps_tokenize_static(const float *coords, const float *feats, int F, const int64_t *offsets,
                         int B, int64_t P, const int32_t *start_local, const fps_opts *opts,
                         int32_t *centroid_idx, int32_t *token_id, int32_t *knn_idx,
                         float *centroids, float *pooled, int32_t *counts, fps_stream_t stream);
+
+/* fps_device_status for fps_tokenize_static: reads (and clears) the status
+ * word that the last fps_tokenize_static call on the current device left in
+ * the static array; synchronises `stream`.  Same results as
+ * fps_device_status. */
+int fps_static_device_status(fps_stream_t stream, int *detail);
 
 /*
  * Nearest-centroid assignment (components/fps.py nearest_assign):
@@ -172,9 +182,14 @@ int fps_assign(const float *coords, const int64_t *offsets, int B, int64_t P,
                void *workspace, size_t workspace_bytes, fps_stream_t stream);
 
 /*
- * kNN gather: for every valid centroid row j of event b, the k points of the
- * event with the smallest (d(p_i, c_j), i), ascending, as global indices,
- * -1 padded when the event has fewer than k points; invalid rows are all -1.
+ * kNN gather (graphnet PR #923, "What is added": farthest_point_sampling_with_knn
+ * in components/fps.py; Neptune README, "How it works", step 1 and
+ * "Parameters": assign_mode="knn" with k_neighbors): for every valid centroid
+ * row j of event b, the k points of the event with the smallest
+ * (d(p_i, c_j), i), ascending, as global indices, -1 padded when the event has
+ * fewer than k points; invalid rows are all -1.  centroids float32 [B, K, 4];
+ * valid_tokens int32 [B] or NULL for min(N, K); knn_idx int32 [B, K, k].
+ * Workspace: fps_knn_workspace_bytes() (a status word), 256-byte aligned.
  */
 size_t fps_knn_workspace_bytes(int64_t P, int B);
 int fps_knn(const float *coords, const int64_t *offsets, int B, int64_t P,

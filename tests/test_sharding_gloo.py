@@ -1,8 +1,9 @@
-"""Multi-process (gloo, world size 2) test of the event sharding used when the
-tokenizer runs on several GPUs: events are split over ranks with no data-path
-exchange; each rank tokenizes its shard; gathering the shards must reproduce
-the single-process result event by event.  The per-rank compute here is the
-CPU oracle, so the test needs no GPU."""
+"""Multi-process (gloo, world size 2) test of the library's event sharding
+(``farthest_point_sampling_b200.sharding``), used when the tokenizer runs on
+several GPUs: events are split over ranks with no data-path exchange; each
+rank tokenizes its shard; gathering the shards must reproduce the
+single-process result event by event.  The per-rank compute here is the CPU
+oracle, so the test needs no GPU."""
 import os
 import socket
 
@@ -15,6 +16,7 @@ import torch.multiprocessing as mp
 import bench
 import oracle
 import workloads
+from farthest_point_sampling_b200 import sharding
 
 
 def _free_port():
@@ -28,8 +30,9 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         full = bench.global_batch("c1", world)
-        parts = bench.partition_events(full.sizes(), full.K, world)
-        mine = bench.shard(full, parts[rank])
+        parts = sharding.partition_events(full.sizes(), full.K, world)
+        c, f, off = sharding.shard_events(full.coords, full.feats, full.offsets, parts[rank])
+        mine = workloads.Batch(c, f, off, full.K, full.assign_mode, full.k, full.lloyd_iters, full.charge_col)
         out = oracle.tokenize_batch(mine)
         # timing reduction as in bench.py: max over ranks
         t = torch.tensor([float(rank + 1)], dtype=torch.float64)
@@ -80,10 +83,24 @@ def test_two_rank_sharding_matches_single_process():
 def test_partition_is_balanced_and_complete():
     b = workloads.make_workload("c1", B=512)
     for world in (2, 4, 8):
-        parts = bench.partition_events(b.sizes(), b.K, world)
+        parts = sharding.partition_events(b.sizes(), b.K, world)
         allev = np.sort(np.concatenate(parts))
         assert np.array_equal(allev, np.arange(b.B))
-        cost = bench.event_cost(b.sizes(), b.K)
+        cost = sharding.event_cost(b.sizes(), b.K)
         loads = np.array([cost[p].sum() for p in parts])
         # LPT bound: no rank exceeds the mean by more than the largest event
         assert loads.max() <= loads.mean() + cost.max() + 1e-9
+
+
+def test_shard_events_torch_matches_numpy():
+    b = workloads.make_workload("c1")
+    parts = sharding.partition_events(b.sizes(), b.K, 3)
+    for p in parts:
+        c, f, off = sharding.shard_events(b.coords, b.feats, b.offsets, p)
+        tc, tf, toff = sharding.shard_events(torch.from_numpy(b.coords), torch.from_numpy(b.feats),
+                                             torch.from_numpy(b.offsets), p)
+        np.testing.assert_array_equal(tc.numpy(), c)
+        np.testing.assert_array_equal(tf.numpy(), f)
+        np.testing.assert_array_equal(toff.numpy(), off)
+        assert off[-1] == b.sizes()[p].sum()
+    assert bench.partition_events is not None  # bench.py delegates to the library helper
