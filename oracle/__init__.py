@@ -37,13 +37,15 @@ def bind(path: str):
     I = ctypes.c_int
     lib.fpso_dist.restype = ctypes.c_float
     lib.fpso_dist.argtypes = [P, P]
-    lib.fpso_fps.argtypes = [P, P, I, I, P, P, P]
-    lib.fpso_assign.argtypes = [P, P, I, P, P, I, P]
-    lib.fpso_knn.argtypes = [P, P, I, P, P, I, I, P]
-    lib.fpso_lloyd.argtypes = [P, P, I, I, P, I, I, I, P, P]
+    lib.fpso_dist_w.restype = ctypes.c_float
+    lib.fpso_dist_w.argtypes = [P, P, P]
+    lib.fpso_fps.argtypes = [P, P, I, I, P, P, P, P]
+    lib.fpso_assign.argtypes = [P, P, I, P, P, I, P, P]
+    lib.fpso_knn.argtypes = [P, P, I, P, P, I, I, P, P]
+    lib.fpso_lloyd.argtypes = [P, P, I, I, P, I, I, I, P, P, P]
     lib.fpso_pool_voronoi.argtypes = [P, I, P, I, I, P, P, P]
     lib.fpso_pool_knn.argtypes = [P, I, I, I, I, P, P, P]
-    lib.fpso_tokenize.argtypes = [P, P, I, P, I, P, I, I, I, I, I, P, P, P, P, P, P]
+    lib.fpso_tokenize.argtypes = [P, P, I, P, I, P, I, I, I, I, I, P, P, P, P, P, P, P]
     lib.fpso_pool_voronoi_backward.argtypes = [P, I, P, I, I, P, P, P]
     lib.fpso_pool_knn_backward.argtypes = [P, I, I, I, I, P, P, ctypes.c_int64, P]
     lib.fpso_pack_tokens.argtypes = [P, I, P, P, I, I, P, P, P]
@@ -118,45 +120,63 @@ def dist(p, c) -> np.float32:
     return np.float32(_load().fpso_dist(_p(p), _p(c)))
 
 
-def fps(coords, offsets, K: int, start_local=None, with_sel_dist: bool = False):
+def _w(axis_scale):
+    """Per-axis scale as a float32 [4] array, or None (no scaling)."""
+    return None if axis_scale is None else _f32(axis_scale).reshape(4)
+
+
+def dist_w(p, c, axis_scale) -> np.float32:
+    """The distance under a per-axis scale (both points scaled in float32 first)."""
+    p = _f32(p).reshape(4)
+    c = _f32(c).reshape(4)
+    w = _w(axis_scale)
+    return np.float32(_load().fpso_dist_w(_p(p), _p(c), _p(w)))
+
+
+def fps(coords, offsets, K: int, start_local=None, with_sel_dist: bool = False, axis_scale=None):
     coords, offsets = _f32(coords, (4,)), _i64(offsets)
     B = offsets.shape[0] - 1
     start_local = _i32(start_local)
+    w = _w(axis_scale)
     idx = np.empty((B, K), np.int32)
     sd = np.empty((B, K), np.float32) if with_sel_dist else None
-    _check(_load().fpso_fps(_p(coords), _p(offsets), B, K, _p(start_local), _p(idx), _p(sd)), "fps")
+    _check(_load().fpso_fps(_p(coords), _p(offsets), B, K, _p(start_local), _p(w), _p(idx), _p(sd)), "fps")
     return (idx, sd) if with_sel_dist else idx
 
 
-def assign(coords, offsets, centroids, K: int, valid=None):
+def assign(coords, offsets, centroids, K: int, valid=None, axis_scale=None):
     coords, offsets = _f32(coords, (4,)), _i64(offsets)
     B = offsets.shape[0] - 1
     centroids = _f32(centroids).reshape(B, K, 4)
+    w = _w(axis_scale)
     tok = np.empty(coords.shape[0], np.int32)
-    _check(_load().fpso_assign(_p(coords), _p(offsets), B, _p(centroids), _p(_i32(valid)), K, _p(tok)),
+    _check(_load().fpso_assign(_p(coords), _p(offsets), B, _p(centroids), _p(_i32(valid)), K, _p(w), _p(tok)),
            "assign")
     return tok
 
 
-def knn(coords, offsets, centroids, K: int, k: int, valid=None):
+def knn(coords, offsets, centroids, K: int, k: int, valid=None, axis_scale=None):
     coords, offsets = _f32(coords, (4,)), _i64(offsets)
     B = offsets.shape[0] - 1
     centroids = _f32(centroids).reshape(B, K, 4)
+    w = _w(axis_scale)
     out = np.empty((B, K, k), np.int32)
-    _check(_load().fpso_knn(_p(coords), _p(offsets), B, _p(centroids), _p(_i32(valid)), K, k, _p(out)),
+    _check(_load().fpso_knn(_p(coords), _p(offsets), B, _p(centroids), _p(_i32(valid)), K, k, _p(w), _p(out)),
            "knn")
     return out
 
 
-def lloyd(coords, feats, offsets, K: int, iters: int, centroids, token_id, charge_col: int = -1):
+def lloyd(coords, feats, offsets, K: int, iters: int, centroids, token_id, charge_col: int = -1,
+          axis_scale=None):
     coords, offsets = _f32(coords, (4,)), _i64(offsets)
     B = offsets.shape[0] - 1
     feats = _f32(feats)
     F = feats.shape[1] if feats.ndim == 2 else 0
     c = _f32(centroids).reshape(B, K, 4).copy()
     t = _i32(token_id).copy()
-    _check(_load().fpso_lloyd(_p(coords), _p(feats), F, charge_col, _p(offsets), B, K, iters, _p(c), _p(t)),
-           "lloyd")
+    w = _w(axis_scale)
+    _check(_load().fpso_lloyd(_p(coords), _p(feats), F, charge_col, _p(offsets), B, K, iters, _p(w), _p(c),
+                              _p(t)), "lloyd")
     return c, t
 
 
@@ -267,8 +287,9 @@ def unpack_tokens(src, tok_offsets, K: int):
 
 
 def tokenize(coords, feats, offsets, K: int, assign_mode: int = 0, k: int = 0, lloyd_iters: int = 0,
-             charge_col: int = -1, start_local=None) -> dict:
-    """The whole tokenizer on one packed batch; returns a dict of numpy outputs."""
+             charge_col: int = -1, start_local=None, axis_scale=None) -> dict:
+    """The whole tokenizer on one packed batch; returns a dict of numpy outputs.
+    ``axis_scale``: optional per-axis scale (wx, wy, wz, wt) of the distance."""
     coords, feats, offsets = _f32(coords, (4,)), _f32(feats), _i64(offsets)
     B = offsets.shape[0] - 1
     P = coords.shape[0]
@@ -281,8 +302,9 @@ def tokenize(coords, feats, offsets, K: int, assign_mode: int = 0, k: int = 0, l
         "pooled": np.empty((B, K, F), np.float32),
         "counts": np.empty((B, K), np.int32),
     }
+    w = _w(axis_scale)
     rc = _load().fpso_tokenize(_p(coords), _p(feats), F, _p(offsets), B, _p(_i32(start_local)), K,
-                               assign_mode, k, lloyd_iters, charge_col, _p(out["centroid_idx"]),
+                               assign_mode, k, lloyd_iters, charge_col, _p(w), _p(out["centroid_idx"]),
                                _p(out["token_id"]), _p(out["knn_idx"]), _p(out["centroids"]),
                                _p(out["pooled"]), _p(out["counts"]))
     _check(rc, "tokenize")
@@ -292,4 +314,4 @@ def tokenize(coords, feats, offsets, K: int, assign_mode: int = 0, k: int = 0, l
 def tokenize_batch(batch) -> dict:
     """``tokenize`` on a ``workloads.Batch``."""
     return tokenize(batch.coords, batch.feats, batch.offsets, batch.K, batch.assign_mode, batch.k,
-                    batch.lloyd_iters, batch.charge_col, batch.start_local)
+                    batch.lloyd_iters, batch.charge_col, batch.start_local, getattr(batch, "axis_scale", None))

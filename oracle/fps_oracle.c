@@ -22,7 +22,13 @@
  * Readings where the pages are silent:
  *   - distance d(i,c) = ((dx*dx + dy*dy) + dz*dz) + dt*dt in float32, each
  *     operation rounded to nearest, no fused multiply-add (build with
- *     -ffp-contract=off), raw (x,y,z,t), t unscaled;
+ *     -ffp-contract=off), raw (x,y,z,t), t unscaled by default;
+ *   - optional per-axis scale w = (wx, wy, wz, wt) (the time scale of the
+ *     review thread on the FPS arguments): both points' coordinates are
+ *     first multiplied by their axis weight in float32, then the distance
+ *     above is taken; w = NULL means no scaling, and w = (1,1,1,1) gives the
+ *     same bits.  Only the metric changes: centroid positions, Lloyd means
+ *     and pooled values stay in the caller's units;
  *   - first centroid = start_local[b] (default 0, the event's first point);
  *   - next centroid = the unselected point with the largest running minimum
  *     distance, lowest index on ties (so with only duplicates left it is the
@@ -57,6 +63,21 @@ float fpso_dist(const float *p, const float *c)
     return s;
 }
 
+/*
+ * The same distance with a per-axis scale: p and c are scaled coordinate by
+ * coordinate, each product rounded to float32, before the distance above.
+ */
+float fpso_dist_w(const float *p, const float *c, const float *w)
+{
+    if (w == NULL) return fpso_dist(p, c);
+    float ps[4], cs[4];
+    for (int a = 0; a < 4; ++a) {
+        ps[a] = w[a] * p[a];
+        cs[a] = w[a] * c[a];
+    }
+    return fpso_dist(ps, cs);
+}
+
 static int bad_offsets(const int64_t *offsets, int B)
 {
     if (B < 0 || offsets == NULL) return 1;
@@ -73,7 +94,7 @@ static int bad_offsets(const int64_t *offsets, int B)
  * s-th centroid had when it was chosen; slot 0 and passthrough slots get -1.
  */
 int fpso_fps(const float *coords, const int64_t *offsets, int B, int K,
-             const int32_t *start_local, int32_t *centroid_idx, float *sel_dist)
+             const int32_t *start_local, const float *w, int32_t *centroid_idx, float *sel_dist)
 {
     if (K < 1 || bad_offsets(offsets, B)) return -1;
     for (int64_t e = 0; e < (int64_t)B * K; ++e) {
@@ -100,7 +121,7 @@ int fpso_fps(const float *coords, const int64_t *offsets, int B, int K,
             if (s == K - 1) break;
             const float *pc = coords + 4 * (off + c);
             for (int64_t i = 0; i < n; ++i) {
-                float d = fpso_dist(coords + 4 * (off + i), pc);
+                float d = fpso_dist_w(coords + 4 * (off + i), pc, w);
                 if (d < dist[i]) dist[i] = d;
             }
             int64_t best = -1;
@@ -130,7 +151,7 @@ static int64_t n_valid(const int32_t *valid, int b, int64_t n, int K)
  * event has no valid centroid.
  */
 int fpso_assign(const float *coords, const int64_t *offsets, int B,
-                const float *centroids, const int32_t *valid, int K, int32_t *token_id)
+                const float *centroids, const int32_t *valid, int K, const float *w, int32_t *token_id)
 {
     if (K < 1 || bad_offsets(offsets, B)) return -1;
     for (int b = 0; b < B; ++b) {
@@ -143,7 +164,7 @@ int fpso_assign(const float *coords, const int64_t *offsets, int B,
             int32_t lab = -1;
             float best = 0.0f;
             for (int64_t j = 0; j < nv; ++j) {
-                float d = fpso_dist(p, cb + 4 * j);
+                float d = fpso_dist_w(p, cb + 4 * j, w);
                 if (lab < 0 || d < best) {
                     best = d;
                     lab = (int32_t)j;
@@ -174,7 +195,7 @@ static int dkey_cmp(const void *a, const void *b)
  * -1 padded when the event has fewer than k points; invalid rows all -1.
  */
 int fpso_knn(const float *coords, const int64_t *offsets, int B, const float *centroids,
-             const int32_t *valid, int K, int k, int32_t *knn_idx)
+             const int32_t *valid, int K, int k, const float *w, int32_t *knn_idx)
 {
     if (K < 1 || k < 1 || bad_offsets(offsets, B)) return -1;
     for (int64_t e = 0; e < (int64_t)B * K * k; ++e) knn_idx[e] = -1;
@@ -187,7 +208,7 @@ int fpso_knn(const float *coords, const int64_t *offsets, int B, const float *ce
         for (int64_t j = 0; j < nv; ++j) {
             const float *c = centroids + ((int64_t)b * K + j) * 4;
             for (int64_t i = 0; i < n; ++i) {
-                keys[i].d = fpso_dist(coords + 4 * (off + i), c);
+                keys[i].d = fpso_dist_w(coords + 4 * (off + i), c, w);
                 keys[i].i = i;
             }
             qsort(keys, (size_t)n, sizeof(dkey), dkey_cmp);
@@ -206,7 +227,7 @@ int fpso_knn(const float *coords, const int64_t *offsets, int B, const float *ce
  * then every point is re-assigned to its nearest centroid.
  */
 int fpso_lloyd(const float *coords, const float *feats, int F, int charge_col,
-               const int64_t *offsets, int B, int K, int iters,
+               const int64_t *offsets, int B, int K, int iters, const float *w,
                float *centroids, int32_t *token_id)
 {
     if (K < 1 || iters < 0 || charge_col >= F || bad_offsets(offsets, B)) return -1;
@@ -238,9 +259,9 @@ int fpso_lloyd(const float *coords, const float *feats, int F, int charge_col,
             for (int64_t i = 0; i < n; ++i) {
                 const float *p = coords + 4 * (off + i);
                 int32_t lab = 0;
-                float best = fpso_dist(p, cb);
+                float best = fpso_dist_w(p, cb, w);
                 for (int j = 1; j < K; ++j) {
-                    float d = fpso_dist(p, cb + 4 * j);
+                    float d = fpso_dist_w(p, cb + 4 * j, w);
                     if (d < best) {
                         best = d;
                         lab = j;
@@ -524,12 +545,12 @@ int fpso_unpack_tokens(const float *src, int D, const int64_t *tok_offsets, int 
  * The whole tokenizer: FPS (or passthrough) -> centroids -> Voronoi labels ->
  * Lloyd (events with N > K) -> Voronoi mean-pool, or kNN gather around the
  * final centroids and kNN mean-pool.  token_id may be NULL in kNN mode;
- * knn_idx is ignored in Voronoi mode.
+ * knn_idx is ignored in Voronoi mode; w (per-axis scale) may be NULL.
  */
 int fpso_tokenize(const float *coords, const float *feats, int F, const int64_t *offsets, int B,
                   const int32_t *start_local, int K, int assign_mode, int k, int lloyd_iters,
-                  int charge_col, int32_t *centroid_idx, int32_t *token_id, int32_t *knn_idx,
-                  float *centroids, float *pooled, int32_t *counts)
+                  int charge_col, const float *w, int32_t *centroid_idx, int32_t *token_id,
+                  int32_t *knn_idx, float *centroids, float *pooled, int32_t *counts)
 {
     if (K < 1 || F < 1 || (assign_mode != 0 && assign_mode != 1) || lloyd_iters < 0 ||
         charge_col >= F || bad_offsets(offsets, B))
@@ -537,13 +558,13 @@ int fpso_tokenize(const float *coords, const float *feats, int F, const int64_t 
     if (assign_mode == 1 && (k < 1 || knn_idx == NULL)) return -1;
     if (assign_mode == 0 && token_id == NULL) return -1;
     int64_t P = B > 0 ? offsets[B] : 0;
-    int rc = fpso_fps(coords, offsets, B, K, start_local, centroid_idx, NULL);
+    int rc = fpso_fps(coords, offsets, B, K, start_local, w, centroid_idx, NULL);
     if (rc) return rc;
     for (int64_t r = 0; r < (int64_t)B * K; ++r)
         for (int a = 0; a < 4; ++a)
             centroids[4 * r + a] = centroid_idx[r] >= 0 ? coords[4 * (int64_t)centroid_idx[r] + a] : 0.0f;
     int32_t *lab = (int32_t *)malloc(sizeof(int32_t) * (P > 0 ? P : 1));
-    rc = fpso_assign(coords, offsets, B, centroids, NULL, K, lab);
+    rc = fpso_assign(coords, offsets, B, centroids, NULL, K, w, lab);
     /* passthrough events: token j is point j */
     for (int b = 0; b < B && rc == 0; ++b) {
         int64_t off = offsets[b], n = offsets[b + 1] - off;
@@ -551,13 +572,13 @@ int fpso_tokenize(const float *coords, const float *feats, int F, const int64_t 
             for (int64_t i = 0; i < n; ++i) lab[off + i] = (int32_t)i;
     }
     if (rc == 0 && lloyd_iters > 0)
-        rc = fpso_lloyd(coords, feats, F, charge_col, offsets, B, K, lloyd_iters, centroids, lab);
+        rc = fpso_lloyd(coords, feats, F, charge_col, offsets, B, K, lloyd_iters, w, centroids, lab);
     if (rc == 0 && token_id)
         memcpy(token_id, lab, sizeof(int32_t) * (size_t)P);
     if (rc == 0 && assign_mode == 0) {
         rc = fpso_pool_voronoi(feats, F, offsets, B, K, lab, pooled, counts);
     } else if (rc == 0) {
-        rc = fpso_knn(coords, offsets, B, centroids, NULL, K, k, knn_idx);
+        rc = fpso_knn(coords, offsets, B, centroids, NULL, K, k, w, knn_idx);
         for (int b = 0; b < B && rc == 0; ++b) {
             int64_t off = offsets[b], n = offsets[b + 1] - off;
             if (n > K) continue;

@@ -45,6 +45,9 @@ MUTATIONS = {
                               "        for (int64_t j = 0; j + 1 < v; ++j) {\n            int64_t t = tok_offsets[b] + j;"),
     "unpack_no_zero_pad": ("j < v ? src[(tok_offsets[b] + j) * D + d] : 0.0f;",
                            "j < v ? src[(tok_offsets[b] + j) * D + d] : src[0];"),
+    "scale_wrong_axis": ("        ps[a] = w[a] * p[a];\n        cs[a] = w[a] * c[a];\n",
+                         "        ps[a] = w[3 - a] * p[a];\n        cs[a] = w[3 - a] * c[a];\n"),
+    "scale_point_only": ("        cs[a] = w[a] * c[a];\n", "        cs[a] = c[a];\n"),
     "knn_bwd_first_feature": ("acc[(int64_t)i * F + f] += (double)grad_pooled[r * F + f] / (double)counts[r];",
                               "acc[(int64_t)i * F + f] += (double)grad_pooled[r * F] / (double)counts[r];"),
 }
@@ -53,6 +56,7 @@ PINS = [
     pins.pin_dist_golden, pins.pin_dist_error_bound, pins.pin_fps_fixtures, pins.pin_fps_bruteforce,
     pins.pin_fps_invariants, pins.pin_assign_bruteforce, pins.pin_knn_bruteforce,
     pins.pin_pool_bruteforce, pins.pin_lloyd_closed_form, pins.pin_pool_backward_adjoint, pins.pin_pack_tokens, pins.pin_token_summaries, pins.pin_random_starts,
+    pins.pin_axis_scale,
 ]
 
 

@@ -27,7 +27,7 @@ def read_fps_fixture(name):
             if key == "coords":
                 mode = "coords"
                 continue
-            if key in ("N", "K", "start", "expected", "sel_dist"):
+            if key in ("N", "K", "start", "expected", "sel_dist", "scale", "unscaled_expected"):
                 mode = None
                 meta[key] = rest
                 continue
@@ -584,3 +584,89 @@ def test_tokenize_composition():
             want = bf.knn(b.coords, b.offsets, out["centroids"], valid, k)
             assert np.array_equal(out["knn_idx"][big], want[big])
             assert np.all(out["counts"][big] == min(k, 17))
+
+
+# ------------------------------------------------------------------ per-axis scale
+
+def _prescaled(coords, w):
+    """coords with every coordinate multiplied by its axis weight in float32."""
+    return (np.asarray(coords, np.float32) * np.asarray(w, np.float32)[None, :]).astype(np.float32)
+
+
+def pin_axis_scale():
+    """The per-axis scale multiplies both points' coordinates, axis by axis, in
+    float32 before the distance; only the metric changes."""
+    # hand-worked fixture: the time scale reorders FPS
+    path = os.path.join(GOLDEN, "fps_time_scale.txt")
+    meta = {}
+    coords = []
+    with open(path) as fh:
+        mode = None
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, *rest = line.split()
+            if key == "coords":
+                mode = "coords"
+                continue
+            if mode == "coords" and key not in ("expected", "sel_dist", "unscaled_expected"):
+                coords.append([float(v) for v in line.split()])
+                continue
+            mode = None
+            meta[key] = rest
+    pts = np.array(coords, np.float32)
+    K = int(meta["K"][0])
+    w = np.array([float(v) for v in meta["scale"]], np.float32)
+    idx, sd = oracle.fps(pts, [0, len(pts)], K, start_local=[int(meta["start"][0])], with_sel_dist=True,
+                         axis_scale=w)
+    assert idx[0].tolist() == [int(v) for v in meta["expected"]]
+    assert sd[0].tolist() == [float(v) for v in meta["sel_dist"]]
+    assert oracle.fps(pts, [0, len(pts)], K).tolist()[0] == [int(v) for v in meta["unscaled_expected"]]
+
+    # unit scale gives the same bits as no scale, through the whole tokenizer
+    for mode, k, it in ((0, 0, 2), (1, 7, 1)):
+        b = workloads.random_batch(71 + mode, [3, 40, 200, 513], 32, assign_mode=mode, k=k, lloyd_iters=it,
+                                   charge_col=0)
+        a = oracle.tokenize_batch(b)
+        b.axis_scale = (1.0, 1.0, 1.0, 1.0)
+        u = oracle.tokenize_batch(b)
+        for key in a:
+            if a[key] is not None:
+                assert np.array_equal(a[key], u[key]), key
+
+    # any scale: FPS, assignment and kNN equal the unscaled functions on
+    # coordinates (and centroids) scaled beforehand in float32
+    b = workloads.random_batch(73, [150, 300, 77], 24)
+    w = np.array([1.0, 1.0, 1.0, 0.3], np.float32)
+    sc = _prescaled(b.coords, w)
+    idx = oracle.fps(b.coords, b.offsets, b.K, axis_scale=w)
+    assert np.array_equal(idx, oracle.fps(sc, b.offsets, b.K))
+    cents = np.where(idx[..., None] >= 0, b.coords[np.maximum(idx, 0)], 0).astype(np.float32)
+    tok = oracle.assign(b.coords, b.offsets, cents, b.K, axis_scale=w)
+    assert np.array_equal(tok, oracle.assign(sc, b.offsets, _prescaled(cents.reshape(-1, 4), w), b.K))
+    kn = oracle.knn(b.coords, b.offsets, cents, b.K, 6, axis_scale=w)
+    assert np.array_equal(kn, oracle.knn(sc, b.offsets, _prescaled(cents.reshape(-1, 4), w), b.K, 6))
+
+    # power-of-two scales are exact in float32 and float64: the whole tokenizer
+    # (Lloyd included) equals the unscaled one on pre-scaled coordinates, with
+    # the centroids in the caller's units (divided back exactly)
+    w2 = np.array([0.5, 2.0, 1.0, 0.125], np.float32)
+    b = workloads.random_batch(74, [5, 260, 1000], 32, lloyd_iters=2, charge_col=0)
+    b.axis_scale = tuple(float(v) for v in w2)
+    got = oracle.tokenize_batch(b)
+    want = oracle.tokenize(_prescaled(b.coords, w2), b.feats, b.offsets, b.K, lloyd_iters=2, charge_col=0)
+    for key in ("centroid_idx", "token_id", "counts", "pooled"):
+        assert np.array_equal(got[key], want[key]), key
+    assert np.array_equal(got["centroids"] * w2, want["centroids"])
+
+    # a zero time weight ignores time: FPS equals FPS with t zeroed
+    b = workloads.random_batch(75, [90, 500], 16)
+    z = b.coords.copy()
+    z[:, 3] = 0.0
+    assert np.array_equal(oracle.fps(b.coords, b.offsets, b.K, axis_scale=[1, 1, 1, 0]),
+                          oracle.fps(z, b.offsets, b.K))
+
+
+def test_axis_scale():
+    pin_axis_scale()

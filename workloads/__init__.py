@@ -64,6 +64,7 @@ class Batch:
     charge_col: int = -1
     start_local: Optional[np.ndarray] = None  # i32 [B] or None (= 0)
     name: str = ""
+    axis_scale: Optional[tuple] = None  # (wx, wy, wz, wt) of the distance, or None (unscaled)
 
     @property
     def B(self) -> int:
