@@ -37,11 +37,11 @@ SIGNATURES = [
     ("fps_tokenize_static", I, [P, P, I, P, I, I64, P, P, P, P, P, P, P, P, P]),
     ("fps_static_device_status", I, [P, ctypes.POINTER(I)]),
     ("fps_assign_workspace_bytes", SZ, [I64, I]),
-    ("fps_assign", I, [P, P, I, I64, P, P, I, P, P, SZ, P]),
+    ("fps_assign", I, [P, P, I, I64, P, P, I, P, P, P, SZ, P]),
     ("fps_knn_workspace_bytes", SZ, [I64, I]),
-    ("fps_knn", I, [P, P, I, I64, P, P, I, I, P, P, SZ, P]),
+    ("fps_knn", I, [P, P, I, I64, P, P, I, I, P, P, P, SZ, P]),
     ("lloyd_workspace_bytes", SZ, [I64, I, I]),
-    ("lloyd_refine", I, [P, P, I, I, P, I, I64, I, I, P, P, P, SZ, P]),
+    ("lloyd_refine", I, [P, P, I, I, P, I, I64, I, I, P, P, P, P, SZ, P]),
     ("segment_pool_workspace_bytes", SZ, [I64, I, I, I]),
     ("segment_pool", I, [P, I, P, I, I64, I, I, P, P, I, P, P, P, SZ, P]),
     ("segment_pool_backward_workspace_bytes", SZ, [I64, I, I, I, I]),
@@ -55,6 +55,7 @@ SIGNATURES = [
     ("fps_device_status", I, [P, P, ctypes.POINTER(I)]),
     ("fps_status_string", ctypes.c_char_p, [I]),
     ("fps_launch_count", ctypes.c_uint64, []),
+    ("fps_set_exchange_test", None, [I, I]),
     ("fps_set_stage_events", None, [ctypes.POINTER(P), I]),
     ("fps_stage_mask", ctypes.c_uint, []),
     ("fps_schedule_for", I, [I64, I, I]),
@@ -65,7 +66,7 @@ class FpsOpts(ctypes.Structure):
     """``fps_opts`` of fpstok.h."""
 
     _fields_ = [("K", I), ("assign_mode", I), ("k", I), ("lloyd_iters", I), ("charge_col", I),
-                ("force_schedule", I), ("max_event_hint", I)]
+                ("force_schedule", I), ("max_event_hint", I), ("axis_scale", ctypes.c_float * 4)]
 
 
 _lib = None

@@ -77,16 +77,29 @@ def offsets_from_batch_ids(batch_ids: torch.Tensor, num_events: Optional[int] = 
     return off
 
 
+def _axis_scale(axis_scale) -> Optional[ctypes.Array]:
+    """Host array of the 4 per-axis weights (x, y, z, t) of the distance, or None."""
+    if axis_scale is None:
+        return None
+    w = [float(v) for v in axis_scale]
+    if len(w) != 4:
+        raise ValueError("axis_scale must hold 4 weights (x, y, z, t)")
+    return (ctypes.c_float * 4)(*w)
+
+
 class Options:
-    """Python view of ``fps_opts``."""
+    """Python view of ``fps_opts``.  ``axis_scale``: optional per-axis weights
+    (wx, wy, wz, wt) of the FPS / assignment distance (both points' coordinates
+    are multiplied by them in float32 first); None means unscaled."""
 
     def __init__(self, K: int = 128, assign_mode: Union[str, int] = "voronoi", k: int = 32,
                  lloyd_iters: int = 0, charge_col: int = -1, force_schedule: int = -1,
-                 max_event_hint: int = 0):
+                 max_event_hint: int = 0, axis_scale=None):
         if assign_mode not in _MODES:
             raise ValueError(f"assign_mode must be 'voronoi' or 'knn', got {assign_mode!r}")
+        w = _axis_scale(axis_scale)
         self.c = _lib.FpsOpts(int(K), _MODES[assign_mode], int(k), int(lloyd_iters), int(charge_col),
-                              int(force_schedule), int(max_event_hint))
+                              int(force_schedule), int(max_event_hint), w if w is not None else (ctypes.c_float * 4)())
 
     @property
     def knn(self) -> bool:
@@ -111,7 +124,7 @@ def fps_tokenize(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tenso
                  force_schedule: int = -1, max_event_hint: int = 0,
                  workspace: Optional[torch.Tensor] = None, out: Optional[Dict[str, torch.Tensor]] = None,
                  check_device: bool = False, random_start: bool = False, seed: int = 0,
-                 stream_id: int = 0) -> Dict[str, torch.Tensor]:
+                 stream_id: int = 0, axis_scale=None) -> Dict[str, torch.Tensor]:
     """The whole tokenizer (C ``fps_tokenize``): FPS fused with Voronoi labels,
     optional charge-weighted Lloyd, then Voronoi mean-pool or kNN gather + pool.
 
@@ -123,6 +136,8 @@ def fps_tokenize(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tenso
     device-side check failure (bad offsets or start index).  With
     ``random_start`` each event starts at a Philox4x32-10 draw for ``seed``
     and ``stream_id`` (see :func:`random_starts`) instead of ``start_local``.
+    ``axis_scale`` = (wx, wy, wz, wt) weights the coordinates in the distance
+    (e.g. a time scale); positions and means are returned in input units.
     """
     dev = _cuda_device(coords)
     _need(coords, "coords", torch.float32, 2, dev)
@@ -138,7 +153,7 @@ def fps_tokenize(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.Tenso
         start_local = random_starts(offsets, seed, stream_id)
     if start_local is not None:
         _need(start_local, "start_local", torch.int32, 1, dev)
-    opts = Options(K, assign_mode, k, lloyd_iters, charge_col, force_schedule, hint)
+    opts = Options(K, assign_mode, k, lloyd_iters, charge_col, force_schedule, hint, axis_scale)
     P, F = coords.shape[0], feats.shape[1]
     B = offsets.numel() - 1
     lib = _lib.load()
@@ -167,8 +182,8 @@ def fps_tokenize_host(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.
                       charge_col: int = -1, start_local: Optional[torch.Tensor] = None,
                       force_schedule: int = -1, device: Union[str, torch.device] = "cuda",
                       workspace: Optional[torch.Tensor] = None,
-                      out: Optional[Dict[str, torch.Tensor]] = None, synchronize: bool = True
-                      ) -> Dict[str, torch.Tensor]:
+                      out: Optional[Dict[str, torch.Tensor]] = None, synchronize: bool = True,
+                      axis_scale=None) -> Dict[str, torch.Tensor]:
     """C ``fps_tokenize_host``: host (ideally pinned) inputs and outputs; the
     library stages them through the device workspace on the current stream.
     With ``synchronize`` the results are ready on return."""
@@ -181,7 +196,7 @@ def fps_tokenize_host(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.
     P, F = coords.shape[0], feats.shape[1]
     B = offsets.numel() - 1
     hint = int((offsets[1:] - offsets[:-1]).max()) if B > 0 else 0
-    opts = Options(K, assign_mode, k, lloyd_iters, charge_col, force_schedule, hint)
+    opts = Options(K, assign_mode, k, lloyd_iters, charge_col, force_schedule, hint, axis_scale)
     lib = _lib.load()
     ws = _workspace(lib.fps_host_workspace_bytes(P, B, F, ctypes.byref(opts.c)), dev, workspace)
     pin = coords.is_pinned()
@@ -206,7 +221,7 @@ def fps_tokenize_host(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.
 
 def fps_assign(coords: torch.Tensor, offsets: torch.Tensor, centroids: torch.Tensor,
                valid_tokens: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+               out: Optional[torch.Tensor] = None, axis_scale=None) -> torch.Tensor:
     """C ``fps_assign`` (components/fps.py nearest_assign): nearest centroid
     slot of every point, lowest slot on ties; centroids [B, K, 4]."""
     dev = _cuda_device(coords)
@@ -222,14 +237,14 @@ def fps_assign(coords: torch.Tensor, offsets: torch.Tensor, centroids: torch.Ten
     ws = _workspace(lib.fps_assign_workspace_bytes(P, B), dev, workspace)
     tok = out if out is not None else torch.empty(P, dtype=torch.int32, device=dev)
     st = lib.fps_assign(_ptr(coords), _ptr(offsets), B, P, _ptr(centroids), _ptr(valid_tokens), K, _ptr(tok),
-                        _ptr(ws), ws.numel(), _stream(dev))
+                        _axis_scale(axis_scale), _ptr(ws), ws.numel(), _stream(dev))
     _lib.check(st, "fps_assign")
     return tok
 
 
 def fps_knn(coords: torch.Tensor, offsets: torch.Tensor, centroids: torch.Tensor, k: int,
             valid_tokens: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+            out: Optional[torch.Tensor] = None, axis_scale=None) -> torch.Tensor:
     """C ``fps_knn``: the k nearest points (d, then index) of every valid
     centroid row, global indices, -1 padded; centroids [B, K, 4]."""
     dev = _cuda_device(coords)
@@ -243,14 +258,14 @@ def fps_knn(coords: torch.Tensor, offsets: torch.Tensor, centroids: torch.Tensor
     ws = _workspace(lib.fps_knn_workspace_bytes(P, B), dev, workspace)
     res = out if out is not None else torch.empty((B, K, k), dtype=torch.int32, device=dev)
     st = lib.fps_knn(_ptr(coords), _ptr(offsets), B, P, _ptr(centroids), _ptr(valid_tokens), K, k, _ptr(res),
-                     _ptr(ws), ws.numel(), _stream(dev))
+                     _axis_scale(axis_scale), _ptr(ws), ws.numel(), _stream(dev))
     _lib.check(st, "fps_knn")
     return res
 
 
 def lloyd_refine(coords: torch.Tensor, feats: Optional[torch.Tensor], offsets: torch.Tensor,
                  centroids: torch.Tensor, token_id: torch.Tensor, iters: int, charge_col: int = -1,
-                 workspace: Optional[torch.Tensor] = None):
+                 workspace: Optional[torch.Tensor] = None, axis_scale=None):
     """C ``lloyd_refine``: ``iters`` charge-weighted Lloyd iterations of every
     event with N > K, updating ``centroids`` [B,K,4] and ``token_id`` [P] in
     place.  Returns them."""
@@ -267,7 +282,8 @@ def lloyd_refine(coords: torch.Tensor, feats: Optional[torch.Tensor], offsets: t
     lib = _lib.load()
     ws = _workspace(lib.lloyd_workspace_bytes(P, B, K), dev, workspace)
     st = lib.lloyd_refine(_ptr(coords), _ptr(feats), F, charge_col, _ptr(offsets), B, P, K, iters,
-                          _ptr(centroids), _ptr(token_id), _ptr(ws), ws.numel(), _stream(dev))
+                          _ptr(centroids), _ptr(token_id), _axis_scale(axis_scale), _ptr(ws), ws.numel(),
+                          _stream(dev))
     _lib.check(st, "lloyd_refine")
     return centroids, token_id
 

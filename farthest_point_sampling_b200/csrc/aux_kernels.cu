@@ -563,10 +563,10 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
 // coordinates, whose distance to any finite point is +inf.
 __host__ __device__ constexpr int pad_pairs(int nv) { return (nv + 1) & ~1; }
 
-__device__ __forceinline__ void load_cents_padded(const float4* __restrict__ c, int nv, Cent2* s) {
+__device__ __forceinline__ void load_cents_padded(const float4* __restrict__ c, int nv, Cent2* s, float4 w) {
   const float inf = __int_as_float(0x7f800000);
   for (int j = threadIdx.x; j < pad_pairs(nv); j += blockDim.x)
-    s[j] = cent2(j < nv ? c[j] : make_float4(inf, inf, inf, inf));
+    s[j] = cent2(j < nv ? scale4(c[j], w) : make_float4(inf, inf, inf, inf));
 }
 
 // Nearest centroid of this thread's 2 PR points (PR packed pairs) among the
@@ -619,7 +619,7 @@ __device__ __forceinline__ void nearest_pairs(const uint64_t (&X)[PR], const uin
 // for every valid local point li at the end of its pass.
 template <int PR, int NPASS, int T, typename Emit>
 __device__ __forceinline__ void chunk_nearest(const float4* __restrict__ pts, int npts,
-                                              const Cent2* __restrict__ cs, int ng, Emit emit) {
+                                              const Cent2* __restrict__ cs, int ng, float4 w, Emit emit) {
   const int tid = threadIdx.x;
 #pragma unroll 1
   for (int q = 0; q < NPASS; ++q) {
@@ -628,8 +628,8 @@ __device__ __forceinline__ void chunk_nearest(const float4* __restrict__ pts, in
     for (int p = 0; p < PR; ++p) {
       const int ia = tid + (2 * PR * q + 2 * p) * T, ib = ia + T;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-      if (ia < npts) a = ldg4(pts + ia);
-      if (ib < npts) c = ldg4(pts + ib);
+      if (ia < npts) a = scale4(ldg4(pts + ia), w);
+      if (ib < npts) c = scale4(ldg4(pts + ib), w);
       X[p] = pack2(a.x, c.x);
       Y[p] = pack2(a.y, c.y);
       Z[p] = pack2(a.z, c.z);
@@ -662,11 +662,12 @@ __device__ __forceinline__ void pass_range(const Workspace& ws, int& q0, int& q1
 // Standalone nearest-centroid assignment.
 constexpr int kAssignThreads = 256;
 
-__global__ void __launch_bounds__(kAssignThreads, 3) k_assign(const float4* __restrict__ coords,
+__global__ void __launch_bounds__(kAssignThreads, kPassCtasPerSm) k_assign(const float4* __restrict__ coords,
                                                               const int64_t* __restrict__ offsets, int K,
                                                               const float4* __restrict__ centroids,
                                                               const int32_t* __restrict__ valid,
-                                                              int32_t* __restrict__ token_id, Workspace ws) {
+                                                              int32_t* __restrict__ token_id, Workspace ws,
+                                                              float4 w) {
   constexpr int T = kAssignThreads;
   extern __shared__ Cent2 s_cent[];  // [pad_pairs(K)]
   int q0, q1;
@@ -684,13 +685,13 @@ __global__ void __launch_bounds__(kAssignThreads, 3) k_assign(const float4* __re
         record_error(ws.hdr, kDevBadToken);
         nv = 0;
       }
-      load_cents_padded(centroids + (int64_t)b * K, nv, s_cent);
+      load_cents_padded(centroids + (int64_t)b * K, nv, s_cent, w);
       __syncthreads();
       cur = b;
     }
     int32_t* out = token_id + off + i0;
     const int v = nv;
-    chunk_nearest<kNearestPairs, 1, T>(coords + off + i0, min(n - i0, kPass), s_cent, pad_pairs(nv) / 2,
+    chunk_nearest<kNearestPairs, 1, T>(coords + off + i0, min(n - i0, kPass), s_cent, pad_pairs(nv) / 2, w,
                                        [&](int li, int l) { out[li] = v > 0 ? l : -1; });
   }
 }
@@ -804,7 +805,7 @@ __device__ __forceinline__ void lloyd_piece_sums(const float4* __restrict__ pts,
 }
 
 // Cell sums of the current labels.
-__global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_sums(const float4* __restrict__ coords,
+__global__ void __launch_bounds__(kLloydThreads, kPassCtasPerSm) k_lloyd_sums(const float4* __restrict__ coords,
                                                                  const float* __restrict__ feats, int F,
                                                                  int charge_col,
                                                                  const int64_t* __restrict__ offsets, int K,
@@ -832,7 +833,7 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_sums(const float4* _
 // of the pass and, unless this is the last iteration (next == nullptr), the
 // pass's cell sums of the new labels added into `next`.  Also clears `clear`,
 // the buffer the following iteration accumulates into.
-__global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* __restrict__ coords,
+__global__ void __launch_bounds__(kLloydThreads, kPassCtasPerSm) k_lloyd_step(const float4* __restrict__ coords,
                                                                  const float* __restrict__ feats, int F,
                                                                  int charge_col,
                                                                  const int64_t* __restrict__ offsets, int K,
@@ -840,7 +841,8 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* _
                                                                  float4* __restrict__ centroids, Workspace ws,
                                                                  const double* __restrict__ in,
                                                                  double* __restrict__ next,
-                                                                 double* __restrict__ clear, int64_t clear_n) {
+                                                                 double* __restrict__ clear, int64_t clear_n,
+                                                                 float4 w) {
   constexpr int T = kLloydThreads;
   extern __shared__ __align__(16) char smem_c[];
   const LloydSmem sm = lloyd_smem(smem_c);
@@ -868,7 +870,7 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* _
           c.z = (float)(__ldcg(&sb[j * 5 + 3]) / W);
           c.w = (float)(__ldcg(&sb[j * 5 + 4]) / W);
         }
-        s_cent[j] = cent2(c);
+        s_cent[j] = cent2(scale4(c, w));  // the means stay in the caller's units
         if (writer) centroids[(int64_t)b * K + j] = c;
       }
       if (tid == 0 && (K & 1)) {
@@ -881,7 +883,7 @@ __global__ void __launch_bounds__(kLloydThreads, 3) k_lloyd_step(const float4* _
     const int64_t off = offsets[b] + i0;
     const int npts = min((int)(offsets[b + 1] - offsets[b]) - i0, kPass);
     int32_t* lab_out = labels + off;
-    chunk_nearest<kNearestPairs, 1, T>(coords + off, npts, s_cent, pad_pairs(K) / 2,
+    chunk_nearest<kNearestPairs, 1, T>(coords + off, npts, s_cent, pad_pairs(K) / 2, w,
                                        [&](int li, int l) { lab_out[li] = l; });
     if (next) {  // this thread's own labels, read back
       lloyd_piece_sums(coords + off, feats ? feats + off * F : nullptr, F, charge_col, lab_out, npts, K, sm,
@@ -914,7 +916,7 @@ cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels
     k_lloyd_step<<<grid, kLloydThreads, sm_step, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels,
                                                       pb.centroids, ws, ws.lloyd[t % 3],
                                                       last ? nullptr : ws.lloyd[(t + 1) % 3], clear,
-                                                      clear ? (int64_t)ws.fps_slots * per : 0);
+                                                      clear ? (int64_t)ws.fps_slots * per : 0, pb.w);
     if ((e = cudaGetLastError())) return e;
   }
   return cudaSuccess;
@@ -1025,7 +1027,7 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
                                              int32_t* __restrict__ knn_idx,
                                              const float* __restrict__ feats, int F,
                                              float* __restrict__ pooled, int32_t* __restrict__ counts,
-                                             KnnOrder ord, WsHeader* hdr) {
+                                             KnnOrder ord, WsHeader* hdr, float4 w, int scaled) {
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -1058,7 +1060,7 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
 #pragma unroll
     for (int q = 0; q < KPL; ++q) L[q] = ~0ull;
     if (j < nv) {
-      const float4 c = centroids[orow];
+      const float4 c = scale4(centroids[orow], w);
       const float4* pts = coords + o0;
       uint64_t thr = ~0ull;
       int ns = 0;  // staged candidates (k <= 32)
@@ -1069,6 +1071,10 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
         for (int u = 0; u < U; ++u) {
           const int i = base + u * 32 + lane;
           pt[u] = i < n ? ldg4(pts + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (scaled) {  // uniform: unscaled calls skip the multiplies
+#pragma unroll
+          for (int u = 0; u < U; ++u) pt[u] = scale4(pt[u], w);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -1148,7 +1154,7 @@ __global__ void __launch_bounds__(256) k_knn(const float4* __restrict__ coords,
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
                        const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, const float* feats,
                        int F, float* pooled, int32_t* counts, const Workspace* ws, WsHeader* hdr,
-                       cudaStream_t s, int only_schedule) {
+                       cudaStream_t s, float4 w, int scaled, int only_schedule) {
   const DeviceInfo& di = device_info();
   // one block per 8 rows (one row per warp), not a persistent grid: short
   // blocks let the schedulers interleave the per-schedule kNN launches by
@@ -1172,13 +1178,13 @@ cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, cons
   count_launch();
   if (k <= 32)
     k_knn<1><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
-                                         feats, F, pooled, counts, ord, hdr);
+                                         feats, F, pooled, counts, ord, hdr, w, scaled);
   else if (k <= 64)
     k_knn<2><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
-                                         feats, F, pooled, counts, ord, hdr);
+                                         feats, F, pooled, counts, ord, hdr, w, scaled);
   else
     k_knn<4><<<(int)blocks, 256, 0, s>>>(coords, offsets, B, centroids, valid_tokens, K, k, knn_idx,
-                                         feats, F, pooled, counts, ord, hdr);
+                                         feats, F, pooled, counts, ord, hdr, w, scaled);
   return cudaGetLastError();
 }
 
@@ -1227,12 +1233,12 @@ cudaError_t launch_pool_knn(const float* feats, int F, int B, int K, int k, cons
 
 cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const float4* centroids,
                           const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,
-                          cudaStream_t s) {
+                          cudaStream_t s, float4 w) {
   const DeviceInfo& di = device_info();
   const size_t sm = (size_t)pad_pairs(K) * sizeof(Cent2);
   count_launch();
   k_assign<<<di.sm_count * kPassCtasPerSm, kAssignThreads, sm, s>>>(coords, offsets, K, centroids, valid_tokens,
-                                                                token_id, ws);
+                                                                token_id, ws, w);
   return cudaGetLastError();
 }
 

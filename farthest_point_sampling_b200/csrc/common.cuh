@@ -20,6 +20,7 @@
 namespace fpstok {
 
 constexpr int kWarp = 32;
+constexpr int FPS_MAX_K_DEV = 256;  // FPS_MAX_K of the C ABI
 constexpr unsigned kFull = 0xffffffffu;
 // Running-minimum value of a slot that holds no point: negative, so it never
 // wins the arg-max (whose keys are the bit patterns of non-negative floats).
@@ -122,6 +123,14 @@ __device__ __forceinline__ float dist1(float4 p, float4 c) {
   return s;
 }
 
+// A point under the per-axis scale of the distance: each coordinate times
+// its weight, rounded to nearest on its own (scalar multiplies, which ptxas
+// never fuses into the subtract that follows).  w = (1, 1, 1, 1) returns the
+// same bits.
+__device__ __forceinline__ float4 scale4(float4 p, float4 w) {
+  return make_float4(__fmul_rn(p.x, w.x), __fmul_rn(p.y, w.y), __fmul_rn(p.z, w.z), __fmul_rn(p.w, w.w));
+}
+
 // Running-min / label update of one slot: strict '<' so that, over slots
 // visited in increasing order, the lowest slot wins ties.
 __device__ __forceinline__ void relax(float d, float& dist, int& lab, int s) {
@@ -143,6 +152,38 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
   float d;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Largest of the per-pair maxima pm[0 .. NP) of one lane (two interleaved
+// three-input chains, so the depth is about NP / 4).
+template <int NP>
+__device__ __forceinline__ float lane_max(const float* pm) {
+  float a = pm[0], b = NP > 1 ? pm[1] : kEmptySlot;
+#pragma unroll
+  for (int p = 2; p < NP; p += 4) {
+    a = p + 1 < NP ? max3f(a, pm[p], pm[p + 1]) : fmaxf(a, pm[p]);
+    if (p + 2 < NP) b = p + 3 < NP ? max3f(b, pm[p + 2], pm[p + 3]) : fmaxf(b, pm[p + 2]);
+  }
+  return fmaxf(a, b);
+}
+
+// The lane's lowest slot holding the arg-max key M: slots 2p and 2p+1 are
+// the two halves of packed pair p (lower slot = lower point index), pm[p] the
+// larger of their running minima.  One pass over the pairs from the top (so
+// the lowest pair wins) selects the pair and the value of its low half with
+// one compare; the low half wins when it holds M.  Returns the slot, or -1
+// when no slot of this lane holds M.
+template <int NP>
+__device__ __forceinline__ int lane_first_slot(const float* pm, const float* dist, int M) {
+  int cp = -1;
+  float lo = 0.f;
+#pragma unroll
+  for (int p = NP - 1; p >= 0; --p) {
+    const bool h = fkey(pm[p]) == M;
+    cp = h ? p : cp;
+    lo = h ? dist[2 * p] : lo;
+  }
+  return cp < 0 ? -1 : 2 * cp + (fkey(lo) == M ? 0 : 1);
 }
 
 // Centroid position stored with every component duplicated, so that two

@@ -78,26 +78,87 @@ __device__ __forceinline__ void prefetch_rows_l2(const float* lo, size_t bytes, 
   }
 }
 
-// One FPS event on one warp, NP point pairs per lane.
+// Layout of the warp schedule's per-warp shared memory: the event's points
+// (DupPoint: every coordinate twice, so two 128-bit loads give the packed
+// centroid), then the list of chosen local indices (the step's centroid is
+// recorded by one lane; positions and global indices are written once at the
+// end).  The points region is reused by the fused pooling afterwards.
+#ifndef FPS_WARP_DUP
+#define FPS_WARP_DUP 0
+#endif
+#ifndef FPS_RELAX_SEL
+#define FPS_RELAX_SEL 0
+#endif
+#if FPS_WARP_DUP
+typedef DupPoint WarpPt;
+#else
+typedef float4 WarpPt;
+#endif
+constexpr int kWarpPtBytes = (int)sizeof(WarpPt);
+constexpr int kWarpListInts = FPS_MAX_K_DEV;  // chosen local indices, one per step
+
+__device__ __forceinline__ WarpPt warp_pt(float4 a) {
+#if FPS_WARP_DUP
+  return dup_point(a);
+#else
+  return a;
+#endif
+}
+__device__ __forceinline__ float4 warp_pt_pos(const WarpPt& p) {
+#if FPS_WARP_DUP
+  return dup_to_float4(p);
+#else
+  return p;
+#endif
+}
+__device__ __forceinline__ Cent2 warp_pt_cent(const WarpPt& p, float4 w, int scaled) {
+  if (scaled) return cent2(scale4(warp_pt_pos(p), w));
+#if FPS_WARP_DUP
+  return cent2_dup(p);
+#else
+  return cent2(p);
+#endif
+}
+
+// Running-min / label update of the two points of one packed pair.
+__device__ __forceinline__ void relax2(uint64_t d, float& d0, float& d1, int& l0, int& l1, int s) {
+#if FPS_RELAX_SEL
+  const bool a = lo2(d) < d0, b = hi2(d) < d1;
+  l0 = a ? s : l0;
+  d0 = a ? lo2(d) : d0;
+  l1 = b ? s : l1;
+  d1 = b ? hi2(d) : d1;
+#else
+  relax(lo2(d), d0, l0, s);
+  relax(hi2(d), d1, l1, s);
+#endif
+}
+
+// One FPS event on one warp, NP point pairs per lane (lane l owns points
+// l + 32 j, slot j = 2 p + h of pair p and half h).
 template <int NP>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
-                                           int lane, float4* s_pts, int32_t* __restrict__ cidx,
+                                           int lane, WarpPt* s_pts, int* s_c, int32_t* __restrict__ cidx,
                                            float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
-                                           const PoolOut& po) {
+                                           const PoolOut& po, float4 w, int scaled) {
   if (po.feats && lane < 4) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), lane, 4);
   const uint64_t z2 = opaque_zero2();
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
   float dist[2 * NP];
   int lab[2 * NP];
-  unsigned taken = 0;  // bit j: slot j (point 32 j + lane) is selected or empty
+  unsigned empty = 0;  // bit j: slot j holds no point
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int i0 = 64 * p + lane, i1 = i0 + 32;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (i0 < n) a = ldg4(pts + i0);
     if (i1 < n) b = ldg4(pts + i1);
-    if (i0 < n) s_pts[i0] = a;
-    if (i1 < n) s_pts[i1] = b;
+    if (i0 < n) s_pts[i0] = warp_pt(a);  // caller's units: centroid outputs (scaled per step when needed)
+    if (i1 < n) s_pts[i1] = warp_pt(b);
+    if (scaled) {
+      a = scale4(a, w);
+      b = scale4(b, w);
+    }
     X[p] = pack2(a.x, b.x);
     Y[p] = pack2(a.y, b.y);
     Z[p] = pack2(a.z, b.z);
@@ -106,41 +167,50 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
     dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
     lab[2 * p] = 0;
     lab[2 * p + 1] = 0;
-    if (i0 >= n) taken |= 1u << (2 * p);
-    if (i1 >= n) taken |= 1u << (2 * p + 1);
+    if (i0 >= n) empty |= 1u << (2 * p);
+    if (i1 >= n) empty |= 1u << (2 * p + 1);
   }
   __syncwarp();
-  for (int s = 0; s < K; ++s) {
-    const float4 cp = s_pts[c];
-    if (lane == 0) {
-      cidx[s] = (int32_t)(off + c);
-      cpos[s] = cp;
-    }
-    if ((c & 31) == lane) taken |= 1u << (c >> 5);
-    const Cent2 C = cent2(cp);
-    float m0 = kEmptySlot, m1 = kEmptySlot;
+  // steps 0 .. K-2: update with c_s, then the next centroid by arg-max
+  for (int s = 0; s < K - 1; ++s) {
+    if (lane == 0) s_c[s] = c;
+    const Cent2 C = warp_pt_cent(s_pts[c], w, scaled);
+    float pm[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
       const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
-      relax(lo2(d), dist[2 * p], lab[2 * p], s);
-      relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
-      if (p & 1)
-        m1 = max3f(m1, dist[2 * p], dist[2 * p + 1]);
-      else
-        m0 = max3f(m0, dist[2 * p], dist[2 * p + 1]);
+      relax2(d, dist[2 * p], dist[2 * p + 1], lab[2 * p], lab[2 * p + 1], s);
+      pm[p] = fmaxf(dist[2 * p], dist[2 * p + 1]);
     }
-    if (s == K - 1) break;
-    const int M = __reduce_max_sync(kFull, fkey(fmaxf(m0, m1)));
-    unsigned cand = 0xffffffffu;  // lowest slot of this lane holding the maximum
-#pragma unroll
-    for (int j = 2 * NP - 1; j >= 0; --j) cand = fkey(dist[j]) == M ? (unsigned)(j * 32 + lane) : cand;
-    unsigned idx = __reduce_min_sync(kFull, cand);
-    if (M == 0) {  // only duplicates of chosen points remain
+    const int M = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
+    const int slot = lane_first_slot<NP>(pm, dist, M);  // lowest slot of this lane holding the maximum
+    unsigned idx = __reduce_min_sync(kFull, slot < 0 ? 0xffffffffu : (unsigned)(slot * 32 + lane));
+    if (M == 0) {  // only duplicates of chosen points remain: the lowest-index unselected point
+      __syncwarp();
+      unsigned taken = empty;
+      for (int t = 0; t <= s; ++t) {
+        const int ct = s_c[t];
+        if ((ct & 31) == lane) taken |= 1u << (ct >> 5);
+      }
       const unsigned free_slots = ~taken & low_bits(2 * NP);
-      cand = free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu;
-      idx = __reduce_min_sync(kFull, cand);
+      idx = __reduce_min_sync(kFull, free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu);
     }
     c = (int)idx;
+  }
+  {  // step K-1: the last centroid only updates the labels
+    if (lane == 0) s_c[K - 1] = c;
+    const Cent2 C = warp_pt_cent(s_pts[c], w, scaled);
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
+      relax2(d, dist[2 * p], dist[2 * p + 1], lab[2 * p], lab[2 * p + 1], K - 1);
+    }
+  }
+  __syncwarp();
+  for (int j = lane; j < K; j += 32) {  // the event's centroids, once
+    const int cj = s_c[j];
+    cidx[j] = (int32_t)(off + cj);
+    cpos[j] = warp_pt_pos(s_pts[cj]);
   }
   if (tok) {
 #pragma unroll
@@ -176,42 +246,50 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
     }
     __syncwarp();
     for (int j = lane; j < K; j += 32) {
-      const int c = cnt[j];
+      const int c2 = cnt[j];
       float* prow = po.pooled + (b * K + j) * F;
-      for (int f = 0; f < F; ++f) prow[f] = c ? (float)(acc[j * F + f] / (double)c) : 0.f;
-      po.counts[b * K + j] = c;
+      for (int f = 0; f < F; ++f) prow[f] = c2 ? (float)(acc[j * F + f] / (double)c2) : 0.f;
+      po.counts[b * K + j] = c2;
     }
   }
   __syncwarp();  // the next event overwrites this warp's copy
 }
 
+// Resident 128-thread blocks per SM of the warp schedule (its register budget).
+#ifndef FPS_WARP_MIN_BLOCKS
+#define FPS_WARP_MIN_BLOCKS 3
+#endif
+
 template <int NPMAX>
-__global__ void __launch_bounds__(128, 4) k_fps_warp(const float4* __restrict__ coords,
+__global__ void __launch_bounds__(128, FPS_WARP_MIN_BLOCKS) k_fps_warp(const float4* __restrict__ coords,
                                                      const int64_t* __restrict__ offsets,
                                                      const int32_t* __restrict__ start_local,
                                                      const int* __restrict__ list, WsHeader* hdr, int K,
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
-                                                     float4* __restrict__ centroids, PoolOut po) {
+                                                     float4* __restrict__ centroids, PoolOut po, float4 w,
+                                                     int scaled) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
-  extern __shared__ float4 s_pts_all[];
+  extern __shared__ __align__(16) unsigned char s_warp_all[];
   const int lane = threadIdx.x & 31;
-  float4* s_pts = s_pts_all + (threadIdx.x >> 5) * (64 * NPMAX);  // this warp's event copy
+  unsigned char* mine = s_warp_all + (size_t)(threadIdx.x >> 5) * (64 * NPMAX * kWarpPtBytes + kWarpListInts * 4);
+  WarpPt* s_pts = reinterpret_cast<WarpPt*>(mine);                      // this warp's event copy
+  int* s_c = reinterpret_cast<int*>(mine + 64 * NPMAX * kWarpPtBytes);  // its chosen local indices
   const int count = hdr->n_items[kListWarp];
   for (;;) {
-    int w = 0;
-    if (lane == 0) w = atomicAdd(&hdr->next_item[kListWarp], 1);
-    w = __shfl_sync(kFull, w, 0);
-    if (w >= count) break;
-    const int b = list[w];
+    int item = 0;
+    if (lane == 0) item = atomicAdd(&hdr->next_item[kListWarp], 1);
+    item = __shfl_sync(kFull, item, 0);
+    if (item >= count) break;
+    const int b = list[item];
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
     const int c0 = start_local ? start_local[b] : 0;
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define WARP_CALL(N)                                                                                   \
-  warp_event<N>(coords + off, n, c0, K, off, lane, s_pts, centroid_idx + (int64_t)b * K,               \
-                centroids + (int64_t)b * K, tok, b, po)
+  warp_event<N>(coords + off, n, c0, K, off, lane, s_pts, s_c, centroid_idx + (int64_t)b * K,          \
+                centroids + (int64_t)b * K, tok, b, po, w, scaled)
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
   }
@@ -232,7 +310,7 @@ template <int NP, int NT, int kMaxPairsCta>
 __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                           DupPoint* s_dup, int2* xk, int& round, int32_t* __restrict__ cidx,
                                           float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
-                                          const PoolOut& po) {
+                                          const PoolOut& po, float4 w, int scaled) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (po.feats && tid < 32) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), tid, 32);
@@ -247,8 +325,12 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (i0 < n) a = ldg4(pts + i0);
     if (i1 < n) b = ldg4(pts + i1);
-    if (i0 < n) s_dup[i0] = dup_point(a);
+    if (i0 < n) s_dup[i0] = dup_point(a);  // caller's units (scaled per step when needed)
     if (i1 < n) s_dup[i1] = dup_point(b);
+    if (scaled) {
+      a = scale4(a, w);
+      b = scale4(b, w);
+    }
     X[p] = pack2(a.x, b.x);
     Y[p] = pack2(a.y, b.y);
     Z[p] = pack2(a.z, b.z);
@@ -278,23 +360,19 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
       cpos[s] = dup_to_float4(cp);
     }
     if (c % NT == tid) taken |= 1u << (c / NT);
-    const Cent2 C = cent2_dup(cp);
-    float m0 = kEmptySlot, m1 = kEmptySlot;
+    const Cent2 C = scaled ? cent2(scale4(dup_to_float4(cp), w)) : cent2_dup(cp);
+    float pm[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
       const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
       relax(lo2(d), dist[2 * p], lab[2 * p], s);
       relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
-      if (p & 1)
-        m1 = max3f(m1, dist[2 * p], dist[2 * p + 1]);
-      else
-        m0 = max3f(m0, dist[2 * p], dist[2 * p + 1]);
+      pm[p] = fmaxf(dist[2 * p], dist[2 * p + 1]);
     }
     if (s == K - 1) break;
-    const int wM = __reduce_max_sync(kFull, fkey(fmaxf(m0, m1)));
-    unsigned cand = 0xffffffffu;
-#pragma unroll
-    for (int j = 2 * NP - 1; j >= 0; --j) cand = fkey(dist[j]) == wM ? (unsigned)(j * NT + tid) : cand;
+    const int wM = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
+    const int slot = lane_first_slot<NP>(pm, dist, wM);
+    const unsigned cand = slot < 0 ? 0xffffffffu : (unsigned)(slot * NT + tid);
     const unsigned widx = __reduce_min_sync(kFull, cand);
     int M;
     unsigned idx;
@@ -369,7 +447,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
                                                             const int* __restrict__ list, WsHeader* hdr, int K,
                                                             int32_t* __restrict__ centroid_idx,
                                                             int32_t* __restrict__ token_id,
-                                                            float4* __restrict__ centroids, PoolOut po) {
+                                                            float4* __restrict__ centroids, PoolOut po,
+                                                            float4 w, int scaled) {
   constexpr int kMaxPairs = PR;
   constexpr int NT = kCtaThreads, NW = NT / 32;
   static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
@@ -388,7 +467,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define CTA_CALL(N)                                                                                     \
   cta_event<N, NT, PR>(coords + off, n, c0, K, off, s_dup, xk, round, centroid_idx + (int64_t)b * K,    \
-                       centroids + (int64_t)b * K, tok, b, po)
+                       centroids + (int64_t)b * K, tok, b, po, w, scaled)
     FPS_DISPATCH_7((n + 2 * NT - 1) / (2 * NT), CTA_CALL)
 #undef CTA_CALL
   }
@@ -434,8 +513,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // try_wait already suspends in hardware between polls; this many polls is
 // far beyond any real exchange (microseconds), and ends a wait that a fault
-// elsewhere would otherwise leave spinning.
+// elsewhere would otherwise leave spinning.  It is a launch argument, so that
+// a test can make it short (fps_set_exchange_test).
 constexpr int kExchangeSpinLimit = 1 << 20;
+
+// Launch arguments of the cluster exchange: the poll limit of each wait and,
+// for tests, a CTA rank that skips its post in the first exchange of every
+// event (-1: none), which makes every wait of that round run out.
+struct ExchangeCfg {
+  int spin_limit;
+  int skip_rank;
+};
 
 // Slot of one posted candidate: (key, index, x, y) and (z, t).
 struct __align__(16) ExSlot {
@@ -451,72 +539,93 @@ struct BlockShared {
   static constexpr int E = CL * NW;  // posted entries per exchange round
 };
 
+// Point pairs per thread the shared-memory schedules also keep in registers
+// for an event of NP pairs per thread: the running minima, labels and pair
+// maxima (5 registers per pair) come first, the cached coordinates (8 per
+// pair) take what is left of the 255-register budget of a 256-thread block
+// (the budget is set where ptxas reports no spills); the other pairs are read
+// from shared memory every step.
+__host__ __device__ constexpr int block_reg_pairs(int np) {
+  return np < (215 - 5 * np) / 8 ? np : ((215 - 5 * np) / 8 > 0 ? (215 - 5 * np) / 8 : 0);
+}
+
+// Returns true when an exchange wait ran out (the CTA left the step loop and
+// wrote nothing more for this event).
 template <int NP, int CL, int NT>
-__device__ __forceinline__ void block_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
+__device__ __forceinline__ bool block_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                             int rank, ulonglong2* sXY, ulonglong2* sZT, int2* xkey, float4* xpos,
-                                            ExSlot* xslot, uint64_t* xbar, WsHeader* hdr, int& round,
-                                            int32_t* __restrict__ cidx, float4* __restrict__ cpos,
-                                            int32_t* __restrict__ tok) {
+                                            ExSlot* xslot, uint64_t* xbar, ExSlot* xbc, WsHeader* hdr, int& round,
+                                            const ExchangeCfg& xcfg, int32_t* __restrict__ cidx,
+                                            float4* __restrict__ cpos, int32_t* __restrict__ tok, float4 w,
+                                            int scaled) {
   constexpr int NW = NT / 32;
   constexpr int E = CL * NW;
   constexpr int G = CL * NT;
   static_assert(CL > 1 || E <= 32, "one warp reads the CTA's warp winners");
-  static_assert(CL == 1 || (CL <= 32 && 2 * CL <= 2 * E - NW), "posts and warp winners do not overlap");
+  static_assert(CL == 1 || CL <= 32, "one lane posts to each CTA of the cluster");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = rank * NT + tid;
 
   // One exchange of (key, index, position) candidates: the event's winner --
   // largest key, then lowest index -- in M, idx, pos on every thread.
-  // Clusters: the CTA's warp winners meet in shared memory; warp 0 sends the
-  // CTA winner into slot `rank` of every CTA with st.async, which signals the
-  // receiving CTA's mbarrier with its bytes; every thread waits (bounded) on
-  // its own mbarrier for the CL posts and reads them.  No cluster barrier and
-  // no release fence.  Rounds alternate between two slot sets and mbarriers
-  // (round & 1; phase parity (round >> 1) & 1): a CTA cannot post round r + 2
-  // before every peer has posted round r + 1, which each does after reading
-  // round r.  Posts arriving before the local arm are counted in the same
-  // phase (it cannot complete before the local arrival).
-  auto exchange = [&](int key, unsigned idx_in, float4 pos_in, int& M, unsigned& idx, float4& pos) {
+  // Clusters: every warp sends its winner into its own slot (rank * NW +
+  // warp) of every CTA of the cluster with st.async, which signals the
+  // receiving CTA's mbarrier with its bytes; every warp arrives on its own
+  // CTA's mbarrier once per round (count NW, each arrival expecting CL posts:
+  // NW * CL in all), lane 0 waits for the phase (bounded), and the warp
+  // reduces the E = CL * NW posted candidates itself.  No barrier of any kind
+  // per round.  Rounds alternate between two slot sets and mbarriers (round &
+  // 1; phase parity (round >> 1) & 1): a warp cannot post round r + 2 before
+  // every warp of the cluster has posted round r + 1, which each does after
+  // reading round r; a phase cannot complete before every local warp has
+  // arrived for it.  Returns false when the wait ran out (the warp leaves the
+  // event; the others follow within a round, as its posts stop).
+  auto exchange = [&](int key, unsigned idx_in, float4 pos_in, bool first, int& M, unsigned& idx,
+                      float4& pos) -> bool {
+    bool ok = true;
     if constexpr (CL > 1) {
-      int2* lkey = xkey + 2 * E - NW;  // warp winners
-      float4* lpos = xpos + 2 * E - NW;
+      static_assert(E % 32 == 0 && E <= 256, "posted candidates per lane");
       const int p = round & 1;
       const uint32_t parity = (uint32_t)(round >> 1) & 1u;
-      ExSlot* slots = xslot + p * CL;
+      ExSlot* slots = xslot + p * E;
       const uint32_t bar = smem_addr(&xbar[p]);
-      if (tid == 0) mbar_arrive_expect(bar, CL * kExSlotBytes);  // this round: CL posts
-      if (lane == 0) {
-        lkey[warp] = make_int2(key, (int)idx_in);
-        lpos[warp] = pos_in;
+      ++round;
+      if (lane == 0) mbar_arrive_expect(bar, CL * kExSlotBytes);
+      const bool post = !(first && rank == xcfg.skip_rank);
+      if (lane < CL && post) {  // this warp's winner into slot rank * NW + warp of CTA `lane`
+        const uint32_t ra = peer_addr(smem_addr(&slots[rank * NW + warp]), lane);
+        const uint32_t rb = peer_addr(bar, lane);
+        st_async_v4(ra, key, (int)idx_in, __float_as_int(pos_in.x), __float_as_int(pos_in.y), rb);
+        st_async_v2(ra + 16, __float_as_int(pos_in.z), __float_as_int(pos_in.w), rb);
       }
-      __syncthreads();
-      if (warp == 0) {
-        const int2 v = lane < NW ? lkey[lane] : make_int2(-0x7fffffff - 1, -1);
-        int cM;
-        unsigned cI;
-        warp_argmax(v.x, (unsigned)v.y, cM, cI);
-        const unsigned who = __ballot_sync(kFull, lane < NW && v.x == cM && (unsigned)v.y == cI);
-        const float4 cp = lpos[__ffs(who) - 1];
-        if (lane < CL) {  // the CTA winner into slot `rank` of every CTA, signalling its barrier
-          const uint32_t ra = peer_addr(smem_addr(&slots[rank]), lane);
-          const uint32_t rb = peer_addr(bar, lane);
-          st_async_v4(ra, cM, (int)cI, __float_as_int(cp.x), __float_as_int(cp.y), rb);
-          st_async_v2(ra + 16, __float_as_int(cp.z), __float_as_int(cp.w), rb);
-        }
+      bool got = false;
+      if (lane == 0)
+        for (int it = 0; it < xcfg.spin_limit && !got; ++it) got = mbar_try_wait(bar, parity);
+      got = __shfl_sync(kFull, got ? 1 : 0, 0) != 0;
+      if (!got) {
+        if (lane == 0) record_error(hdr, kDevExchangeTimeout);
+        return false;
       }
-      bool ok = false;
-      for (int it = 0; it < kExchangeSpinLimit && !ok; ++it) ok = mbar_try_wait(bar, parity);
-      if (!ok && tid == 0) record_error(hdr, kDevExchangeTimeout);  // carry on: control flow stays uniform
-      int2 v = make_int2(-0x7fffffff - 1, -1);
-      if (lane < CL) {
-        const int4 a = slots[lane].a;
-        v = make_int2(a.x, a.y);
+      int bk = -0x7fffffff - 1;  // best (key, index) of this lane's E / 32 slots, and which slot
+      unsigned bi = 0xffffffffu;
+      int bs = 0;
+#pragma unroll
+      for (int q = 0; q < E / 32; ++q) {
+        const int e = lane + 32 * q;
+        const int4 a = slots[e].a;
+        const bool better = a.x > bk || (a.x == bk && (unsigned)a.y < bi);
+        bk = better ? a.x : bk;
+        bi = better ? (unsigned)a.y : bi;
+        bs = better ? e : bs;
       }
-      warp_argmax(v.x, (unsigned)v.y, M, idx);
-      const unsigned who = __ballot_sync(kFull, lane < CL && v.x == M && (unsigned)v.y == idx);
-      const ExSlot& w = slots[__ffs(who) - 1];
-      pos = make_float4(__int_as_float(w.a.z), __int_as_float(w.a.w), __int_as_float(w.b.x), __int_as_float(w.b.y));
+      warp_argmax(bk, bi, M, idx);
+      const unsigned who = __ballot_sync(kFull, bk == M && bi == idx);
+      const ExSlot& x = slots[__shfl_sync(kFull, bs, __ffs(who) - 1)];
+      pos = make_float4(__int_as_float(x.a.z), __int_as_float(x.a.w), __int_as_float(x.b.x),
+                        __int_as_float(x.b.y));
+      return ok;
     } else {
+      (void)first;
       const int base = (round & 1) * E;
       if (lane == 0) {
         xkey[base + warp] = make_int2(key, (int)idx_in);
@@ -529,6 +638,7 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
       pos = xpos[base + __ffs(who) - 1];
     }
     ++round;
+    return ok;
   };
   auto local_pos = [&](unsigned idx) {
     const int gi = (int)(idx % (unsigned)G);
@@ -540,9 +650,11 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
                    : make_float4(lo2(xy.x), lo2(xy.y), lo2(zt.x), lo2(zt.y));
   };
 
+  constexpr int RP = block_reg_pairs(NP);
   const uint64_t z2 = opaque_zero2();
   float dist[2 * NP];
   int lab[2 * NP];
+  uint64_t RX[RP], RY[RP], RZ[RP], RT[RP];  // register copies of the first RP pairs
   unsigned long long taken = 0;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
@@ -550,8 +662,18 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (i0 < n) a = ldg4(pts + i0);
     if (i1 < n) b = ldg4(pts + i1);
+    if (scaled) {  // the distance reads scaled copies; positions handed out are the caller's
+      a = scale4(a, w);
+      b = scale4(b, w);
+    }
     sXY[p * NT + tid] = make_ulonglong2(pack2(a.x, b.x), pack2(a.y, b.y));
     sZT[p * NT + tid] = make_ulonglong2(pack2(a.z, b.z), pack2(a.w, b.w));
+    if (p < RP) {
+      RX[p] = pack2(a.x, b.x);
+      RY[p] = pack2(a.y, b.y);
+      RZ[p] = pack2(a.z, b.z);
+      RT[p] = pack2(a.w, b.w);
+    }
     dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
     dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
     lab[2 * p] = 0;
@@ -560,38 +682,41 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
     if (i1 >= n) taken |= 1ull << (2 * p + 1);
   }
 
-  float4 cc = ldg4(pts + c);
+  __syncthreads();  // every thread's pairs are in shared memory before any warp reads a winner's position
+  float4 cc = ldg4(pts + c);  // the current centroid, scaled like the points
+  if (scaled) cc = scale4(cc, w);
   for (int s = 0; s < K; ++s) {
     if (rank == 0 && tid == 0) {
       cidx[s] = (int32_t)(off + c);
-      cpos[s] = cc;
+      cpos[s] = scaled ? ldg4(pts + c) : cc;
     }
     if (c % G == g) taken |= 1ull << (c / G);
     const Cent2 C = cent2(cc);
-    float m0 = kEmptySlot, m1 = kEmptySlot;
+    float pm[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      const ulonglong2 xy = sXY[p * NT + tid];
-      const ulonglong2 zt = sZT[p * NT + tid];
-      const uint64_t d = dist2(xy.x, xy.y, zt.x, zt.y, C, z2);
+      uint64_t d;
+      if (p < RP) {
+        d = dist2(RX[p], RY[p], RZ[p], RT[p], C, z2);
+      } else {
+        const ulonglong2 xy = sXY[p * NT + tid];
+        const ulonglong2 zt = sZT[p * NT + tid];
+        d = dist2(xy.x, xy.y, zt.x, zt.y, C, z2);
+      }
       relax(lo2(d), dist[2 * p], lab[2 * p], s);
       relax(hi2(d), dist[2 * p + 1], lab[2 * p + 1], s);
-      if (p & 1)
-        m1 = max3f(m1, dist[2 * p], dist[2 * p + 1]);
-      else
-        m0 = max3f(m0, dist[2 * p], dist[2 * p + 1]);
+      pm[p] = fmaxf(dist[2 * p], dist[2 * p + 1]);
     }
     if (s == K - 1) break;
-    const int wM = __reduce_max_sync(kFull, fkey(fmaxf(m0, m1)));
-    unsigned wcand = 0xffffffffu;
-#pragma unroll
-    for (int j = 2 * NP - 1; j >= 0; --j) wcand = fkey(dist[j]) == wM ? (unsigned)(g + G * j) : wcand;
+    const int wM = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
+    const int slot = lane_first_slot<NP>(pm, dist, wM);
+    const unsigned wcand = slot < 0 ? 0xffffffffu : (unsigned)(g + G * slot);
     const unsigned widx = __reduce_min_sync(kFull, wcand);
     float4 wpos = make_float4(0.f, 0.f, 0.f, 0.f);
     if (wM >= 0) wpos = local_pos(widx);
     int M;
     unsigned idx;
-    exchange(wM, widx, wpos, M, idx, cc);
+    if (!exchange(wM, widx, wpos, s == 0, M, idx, cc)) return true;
     if (M == 0) {  // only duplicates of chosen points remain
       const unsigned long long mask = 2 * NP >= 64 ? ~0ull : ((1ull << (2 * NP)) - 1ull);
       const unsigned long long free_slots = ~taken & mask;
@@ -601,7 +726,7 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
       float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
       if (wmin != 0xffffffffu) p = local_pos(wmin);
       // keys: 1 for a real candidate, 0 for none; ties resolve to the lowest index
-      exchange(wmin != 0xffffffffu ? 1 : 0, wmin, p, M, idx, cc);
+      if (!exchange(wmin != 0xffffffffu ? 1 : 0, wmin, p, false, M, idx, cc)) return true;
     }
     c = (int)idx;
   }
@@ -612,6 +737,7 @@ __device__ __forceinline__ void block_event(const float4* __restrict__ pts, int 
       if (i < n) tok[i] = lab[j];
     }
   }
+  return false;
 }
 
 // Pair counts compiled for the shared-memory schedules; an event uses the
@@ -630,8 +756,10 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
                                                      int list_id, int K,
                                                      int32_t* __restrict__ centroid_idx,
                                                      int32_t* __restrict__ token_id,
-                                                     float4* __restrict__ centroids) {
+                                                     float4* __restrict__ centroids, ExchangeCfg xcfg,
+                                                     float4 w, int scaled) {
   static_assert(2 * PS <= 64, "selected-slot mask is 64 bits");
+  static_assert(PS == 24, "pair buckets of FPS_BLOCK_BUCKETS");
   constexpr int E = BlockShared<CL, NT>::E;
   constexpr int G = CL * NT;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -639,16 +767,19 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
   ulonglong2* sZT = sXY + PS * NT;                            // [PS][NT] packed (z, t)
   int2* xkey = reinterpret_cast<int2*>(sZT + PS * NT);        // [2][E] (key, index)
   float4* xpos = reinterpret_cast<float4*>(xkey + 2 * E);     // [2][E] candidate position
-  ExSlot* xslot = reinterpret_cast<ExSlot*>(xpos + 2 * E);    // [2][CL] posted CTA winners
-  uint64_t* xbar = reinterpret_cast<uint64_t*>(xslot + 2 * CL);  // [2] exchange mbarriers
+  ExSlot* xslot = reinterpret_cast<ExSlot*>(xpos + 2 * E);    // [2][E] posted warp winners (clusters)
+  ExSlot* xbc = xslot + 2 * E;                                 // unused placeholder (layout continuity)
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(xbc + 2);       // [2] exchange mbarriers
   __shared__ int s_item;
+  __shared__ int s_abort;  // an exchange wait of this CTA ran out (sticky for the launch)
 
   int rank = 0;
   if constexpr (CL > 1) {
     rank = (int)cg::this_cluster().block_rank();
     if (threadIdx.x == 0) {
-      mbar_init(smem_addr(&xbar[0]), 1);
-      mbar_init(smem_addr(&xbar[1]), 1);
+      s_abort = 0;
+      mbar_init(smem_addr(&xbar[0]), NT / 32);  // one arrival per warp and round
+      mbar_init(smem_addr(&xbar[1]), NT / 32);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     cg::this_cluster().sync();  // every CTA is running, its barriers initialised, before DSMEM use
@@ -677,12 +808,23 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     const int c0 = start_local ? start_local[b] : 0;
     int32_t* tok = token_id ? token_id + off : nullptr;
     const int np = (n + 2 * G - 1) / (2 * G);
-#define BLOCK_CALL(N)                                                                                   \
-  block_event<N, CL, NT>(coords + off, n, c0, K, off, rank, sXY, sZT, xkey, xpos, xslot, xbar, hdr, round, \
-                         centroid_idx + (int64_t)b * K, centroids + (int64_t)b * K, tok)
+    bool aborted = false;
+#define BLOCK_CALL(N)                                                                                         \
+  aborted = block_event<N, CL, NT>(coords + off, n, c0, K, off, rank, sXY, sZT, xkey, xpos, xslot, xbar, xbc, \
+                                   hdr, round, xcfg, centroid_idx + (int64_t)b * K, centroids + (int64_t)b * K, \
+                                   tok, w, scaled)
     FPS_BLOCK_BUCKETS(np, BLOCK_CALL)
 #undef BLOCK_CALL
-    if constexpr (CL > 1) cg::this_cluster().sync();  // s_item is rewritten for the next claim
+    if constexpr (CL > 1) {
+      if (aborted && (threadIdx.x & 31) == 0) s_abort = 1;  // any warp that left the event
+      cg::this_cluster().sync();  // s_item is rewritten for the next claim; abort flags are final
+      // A wait that ran out leaves its mbarrier phase incomplete, so no CTA of
+      // the cluster may run another event: every CTA reads every peer's flag
+      // (the same values after the barrier) and the cluster stops together.
+      int any = 0;
+      if (threadIdx.x < CL) any = *cg::this_cluster().map_shared_rank(&s_abort, (unsigned)threadIdx.x);
+      if (__syncthreads_or(any)) break;
+    }
   }
   if constexpr (CL > 1) cg::this_cluster().sync();  // no CTA leaves while peers may post into it
 }
@@ -694,18 +836,18 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
 // ------------------------------------------------------------------ launch
 
 constexpr int kWarpBlock = 128;
-constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * 64 * kWarpPairs * sizeof(float4);
+constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * (64 * kWarpPairs * kWarpPtBytes + kWarpListInts * 4);
 constexpr size_t kCtaSmem = kCtaSmemBytes;
 static_assert((size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint) <= kCtaSmem, "event copy fits");
 
-size_t warp_region_bytes() { return (size_t)64 * kWarpPairs * sizeof(float4); }
+size_t warp_region_bytes() { return (size_t)64 * kWarpPairs * kWarpPtBytes; }
 size_t cta_region_bytes() { return kCtaSmem; }
 
 template <int CL>
 constexpr size_t block_smem_bytes() {
   return (size_t)2 * kBlockPairs * kBlockThreads * sizeof(ulonglong2) +
          (size_t)2 * BlockShared<CL, kBlockThreads>::E * (sizeof(int2) + sizeof(float4)) +
-         (size_t)2 * CL * sizeof(ExSlot) + 2 * sizeof(uint64_t);
+         (size_t)2 * BlockShared<CL, kBlockThreads>::E * sizeof(ExSlot) + 2 * sizeof(ExSlot) + 2 * sizeof(uint64_t);
 }
 
 template <int CL>
@@ -731,6 +873,21 @@ static cudaError_t prepare_block_kernel(int* max_active_clusters) {
   return cudaOccupancyMaxActiveClusters(max_active_clusters, kern, &cfg);
 }
 
+// Exchange settings of the next launches: the default poll limit and no
+// skipped post, unless a test set others (fps_set_exchange_test).
+static ExchangeCfg g_exchange_cfg = {kExchangeSpinLimit, -1};
+static std::mutex g_exchange_mu;
+static ExchangeCfg exchange_cfg() {
+  std::lock_guard<std::mutex> lock(g_exchange_mu);
+  return g_exchange_cfg;
+}
+
+void set_exchange_test(int spin_limit, int skip_rank) {
+  std::lock_guard<std::mutex> lock(g_exchange_mu);
+  g_exchange_cfg.spin_limit = spin_limit > 0 ? spin_limit : kExchangeSpinLimit;
+  g_exchange_cfg.skip_rank = skip_rank;
+}
+
 template <int CL>
 static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list_id, const int* list,
                                 int n_groups, cudaStream_t s) {
@@ -753,7 +910,7 @@ static cudaError_t launch_block(const Problem& pb, const Workspace& ws, int list
   count_launch();
   return cudaLaunchKernelEx(&cfg, k_fps_block<CL, kBlockThreads, kBlockPairs>, pb.coords, pb.offsets,
                             pb.start_local, list, ws.hdr, list_id, pb.K, pb.centroid_idx, pb.token_id,
-                            pb.centroids);
+                            pb.centroids, exchange_cfg(), pb.w, pb.scaled);
 }
 
 // Per-device state: occupancy figures and the helper streams / events that
@@ -873,7 +1030,8 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
         count_launch();
         k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, hs>>>(pb.coords, pb.offsets, pb.start_local,
                                                                       ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                      pb.token_id, pb.centroids, po_warp);
+                                                                      pb.token_id, pb.centroids, po_warp, pb.w,
+                                                                      pb.scaled);
         e = cudaGetLastError();
         break;
       }
@@ -881,7 +1039,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
         count_launch();
         k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
             pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-            pb.centroids, po_cta);
+            pb.centroids, po_cta, pb.w, pb.scaled);
         e = cudaGetLastError();
         break;
       case 2:
@@ -899,7 +1057,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     // stream, overlapping the other schedules' FPS (its stage includes them)
     if (knn_per_schedule &&
         (e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx, pb.feats, pb.F,
-                        pb.pooled, pb.counts, &ws, ws.hdr, hs, q)))
+                        pb.pooled, pb.counts, &ws, ws.hdr, hs, pb.w, pb.scaled, q)))
       return e;
     mark(1 + q, 1, hs);
     if ((e = cudaEventRecord(ctx.join[q], hs))) return e;

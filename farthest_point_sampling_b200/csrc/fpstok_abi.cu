@@ -2,6 +2,7 @@
 // checks, workspace carving and the launch sequence.  No allocation, no
 // synchronisation (except fps_device_status, which exists to read back).
 #include <atomic>
+#include <cmath>
 #include <cstring>
 
 #include "../../include/fpstok.h"
@@ -78,6 +79,21 @@ static Workspace carve(void* base, int64_t P, int B, int K, int F, bool lloyd, b
 
 static int from_cuda(cudaError_t e) { return e == cudaSuccess ? FPS_OK : FPS_ERR_CUDA; }
 
+bool axis_scale_of(const float* w, float4* out, int* scaled) {
+  *out = make_float4(1.f, 1.f, 1.f, 1.f);
+  *scaled = 0;
+  if (!w) return true;
+  bool zero = true;
+  for (int a = 0; a < 4; ++a) {
+    if (!std::isfinite(w[a])) return false;
+    if (w[a] != 0.f) zero = false;
+  }
+  if (zero) return true;  // the zero-initialised default: unscaled
+  *out = make_float4(w[0], w[1], w[2], w[3]);
+  *scaled = (w[0] != 1.f || w[1] != 1.f || w[2] != 1.f || w[3] != 1.f) ? 1 : 0;
+  return true;
+}
+
 static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 static int check_common(int64_t P, int B, const int64_t* offsets) {
@@ -103,6 +119,9 @@ static int check_opts(const fps_opts* o, int F) {
   if (o->force_schedule < -1 || o->force_schedule > 4) return FPS_ERR_ARG;
   if (o->max_event_hint < 0) return FPS_ERR_ARG;
   if (o->max_event_hint > kClusterCap) return FPS_ERR_TOO_LARGE;
+  float4 w;
+  int scaled;
+  if (!axis_scale_of(o->axis_scale, &w, &scaled)) return FPS_ERR_ARG;
   return FPS_OK;
 }
 
@@ -137,7 +156,7 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
   } else if (pb.assign_mode == FPS_ASSIGN_KNN) {
     stage_mark(7, 0, s);
     if ((e = launch_knn(pb.coords, pb.offsets, pb.B, pb.centroids, nullptr, pb.K, pb.k, pb.knn_idx,
-                        pb.feats, pb.F, pb.pooled, pb.counts, &ws, ws.hdr, s)))
+                        pb.feats, pb.F, pb.pooled, pb.counts, &ws, ws.hdr, s, pb.w, pb.scaled)))
       return from_cuda(e);
     stage_mark(7, 1, s);
   } else {
@@ -199,6 +218,7 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
                 opts->force_schedule, opts->max_event_hint, centroid_idx, token_id,
                 opts->assign_mode == FPS_ASSIGN_KNN ? knn_idx : nullptr,
                 reinterpret_cast<float4*>(centroids), pooled, counts, 0};
+  axis_scale_of(opts->axis_scale, &pb.w, &pb.scaled);
   if (opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0) {
     const size_t K = (size_t)opts->K, Fz = (size_t)F;
     if (K * Fz * sizeof(double) + K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
@@ -292,10 +312,13 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
 size_t fps_assign_workspace_bytes(int64_t P, int B) { return carve(nullptr, P, B, 1, 1, false, false).bytes; }
 
 int fps_assign(const float* coords, const int64_t* offsets, int B, int64_t P, const float* centroids,
-               const int32_t* valid_tokens, int K, int32_t* token_id, void* workspace, size_t workspace_bytes,
-               fps_stream_t stream) {
+               const int32_t* valid_tokens, int K, int32_t* token_id, const float* axis_scale, void* workspace,
+               size_t workspace_bytes, fps_stream_t stream) {
   int rc = check_common(P, B, offsets);
   if (rc) return rc;
+  float4 w;
+  int scaled;
+  if (!axis_scale_of(axis_scale, &w, &scaled)) return FPS_ERR_ARG;
   if (K < 1) return FPS_ERR_ARG;
   if (K > FPS_MAX_K) return FPS_ERR_TOO_LARGE;
   if (B == 0 || P == 0) return FPS_OK;
@@ -315,7 +338,7 @@ int fps_assign(const float* coords, const int64_t* offsets, int B, int64_t P, co
   cudaError_t e;
   if ((e = launch_bin(pb, ws, 1, s))) return from_cuda(e);
   return from_cuda(launch_assign(reinterpret_cast<const float4*>(coords), offsets,
-                                 reinterpret_cast<const float4*>(centroids), valid_tokens, K, token_id, ws, s));
+                                 reinterpret_cast<const float4*>(centroids), valid_tokens, K, token_id, ws, s, w));
 }
 
 size_t fps_knn_workspace_bytes(int64_t P, int B) {
@@ -325,10 +348,13 @@ size_t fps_knn_workspace_bytes(int64_t P, int B) {
 }
 
 int fps_knn(const float* coords, const int64_t* offsets, int B, int64_t P, const float* centroids,
-            const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, void* workspace, size_t workspace_bytes,
-            fps_stream_t stream) {
+            const int32_t* valid_tokens, int K, int k, int32_t* knn_idx, const float* axis_scale, void* workspace,
+            size_t workspace_bytes, fps_stream_t stream) {
   int rc = check_common(P, B, offsets);
   if (rc) return rc;
+  float4 w;
+  int scaled;
+  if (!axis_scale_of(axis_scale, &w, &scaled)) return FPS_ERR_ARG;
   if (K < 1 || k < 1) return FPS_ERR_ARG;
   if (K > FPS_MAX_K || k > FPS_MAX_KNN) return FPS_ERR_TOO_LARGE;
   if (B == 0) return FPS_OK;
@@ -342,7 +368,7 @@ int fps_knn(const float* coords, const int64_t* offsets, int B, int64_t P, const
   if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
   return from_cuda(launch_knn(reinterpret_cast<const float4*>(coords), offsets, B,
                               reinterpret_cast<const float4*>(centroids), valid_tokens, K, k, knn_idx, nullptr,
-                              0, nullptr, nullptr, nullptr, hdr, s));
+                              0, nullptr, nullptr, nullptr, hdr, s, w, scaled));
 }
 
 size_t lloyd_workspace_bytes(int64_t P, int B, int K) {
@@ -351,10 +377,13 @@ size_t lloyd_workspace_bytes(int64_t P, int B, int K) {
 }
 
 int lloyd_refine(const float* coords, const float* feats, int F, int charge_col, const int64_t* offsets, int B,
-                 int64_t P, int K, int iters, float* centroids, int32_t* token_id, void* workspace,
-                 size_t workspace_bytes, fps_stream_t stream) {
+                 int64_t P, int K, int iters, float* centroids, int32_t* token_id, const float* axis_scale,
+                 void* workspace, size_t workspace_bytes, fps_stream_t stream) {
   int rc = check_common(P, B, offsets);
   if (rc) return rc;
+  float4 w;
+  int scaled;
+  if (!axis_scale_of(axis_scale, &w, &scaled)) return FPS_ERR_ARG;
   if (K < 1 || iters < 0 || charge_col < -1) return FPS_ERR_ARG;
   if (K > FPS_MAX_K) return FPS_ERR_TOO_LARGE;
   if (charge_col >= 0 && (F < 1 || charge_col >= F || !feats)) return FPS_ERR_ARG;
@@ -377,6 +406,8 @@ int lloyd_refine(const float* coords, const float* feats, int F, int charge_col,
   pb.charge_col = charge_col;
   pb.force_schedule = -1;
   pb.centroids = reinterpret_cast<float4*>(centroids);
+  pb.w = w;
+  pb.scaled = scaled;
   cudaError_t e;
   stage_mark(6, 0, s);
   if ((e = launch_bin(pb, ws, 0, s))) return from_cuda(e);
@@ -574,6 +605,8 @@ const char* fps_status_string(int status) {
 }
 
 uint64_t fps_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void fps_set_exchange_test(int spin_limit, int skip_rank) { set_exchange_test(spin_limit, skip_rank); }
 
 void fps_set_stage_events(void* const* events, int n_events) {
   g_stage_mask = 0;

@@ -36,13 +36,17 @@ constexpr int kCtaPairs = 5;                           // pairs per thread
 constexpr int kCtaCap = 2 * kCtaThreads * kCtaPairs;   // 2560
 constexpr size_t kCtaSmemBytes = 104 * 1024;           // register-CTA shared memory (event copy / pooling)
 constexpr int kBlockThreads = 256;                     // shared-memory CTA / cluster schedules
-constexpr int kBlockPairs = 24;                        // pairs per thread in shared memory
+constexpr int kBlockPairs = 24;                        // pairs per thread (all in shared memory, the first
+                                                       // ones also cached in registers)
 constexpr int kCtaSmemCap = kBlockThreads * 2 * kBlockPairs;  // 12288
 constexpr int kCluster8Cap = 8 * kCtaSmemCap;                 // 98304
 constexpr int kMaxCluster = 16;
 constexpr int kClusterCap = kMaxCluster * kCtaSmemCap;        // 196608
 constexpr int kPass = 1024;                            // points per Lloyd / assignment pass (256 threads x 4)
-constexpr int kPassCtasPerSm = 3;                      // resident CTAs per SM of the pass kernels
+#ifndef FPS_PASS_CTAS_PER_SM
+#define FPS_PASS_CTAS_PER_SM 3
+#endif
+constexpr int kPassCtasPerSm = FPS_PASS_CTAS_PER_SM;   // resident CTAs per SM of the pass kernels
 constexpr int kPoolChunk = 512;                        // points per pooling work item
 constexpr int kPoolReplicas = 16;                      // accumulator copies per event pooled in several chunks
 // With at most this many FPS events per SM, events of the warp class run on
@@ -87,7 +91,13 @@ struct Problem {
   float* pooled;
   int32_t* counts;
   int fused_pool;  // bit 0 / bit 1: the warp / register-CTA FPS kernels pool their own events
+  float4 w;        // per-axis scale of the distance ((1, 1, 1, 1) when unscaled)
+  int scaled;      // w differs from (1, 1, 1, 1)
 };
+
+// The per-axis scale of a call: (1, 1, 1, 1) for NULL or all-zero weights.
+// Returns false when a weight is not finite.
+bool axis_scale_of(const float* w, float4* out, int* scaled);
 
 // Kernel launchers (return the cudaError_t of the launch).
 cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cudaStream_t s);
@@ -112,10 +122,10 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
 cudaError_t launch_knn(const float4* coords, const int64_t* offsets, int B, const float4* centroids,
                        const int32_t* valid_tokens, int K, int k, int32_t* knn_idx,
                        const float* feats, int F, float* pooled, int32_t* counts, const Workspace* ws,
-                       struct WsHeader* hdr, cudaStream_t s, int only_schedule = -1);
+                       struct WsHeader* hdr, cudaStream_t s, float4 w, int scaled, int only_schedule = -1);
 cudaError_t launch_assign(const float4* coords, const int64_t* offsets, const float4* centroids,
                           const int32_t* valid_tokens, int K, int32_t* token_id, const Workspace& ws,
-                          cudaStream_t s);
+                          cudaStream_t s, float4 w);
 cudaError_t launch_pool_knn(const float* feats, int F, int B, int K, int k, const int32_t* knn_idx,
                             int64_t P, float* pooled, int32_t* counts, struct WsHeader* hdr,
                             cudaStream_t s);
@@ -132,6 +142,11 @@ const DeviceInfo& device_info();  // prepares the current device on first use
 cudaError_t prepare_aux_kernels();   // shared-memory attributes of the auxiliary kernels
 
 void count_launch(int n = 1);
+
+// Test setting of the cluster exchange of the next launches: the poll limit
+// of each wait (<= 0: the default) and a CTA rank that skips its post in the
+// first exchange of every event (-1: none).
+void set_exchange_test(int spin_limit, int skip_rank);
 
 // Workspace bytes fps_tokenize needs for this exact call (the labels area is
 // reserved only when kNN mode runs Lloyd without a caller token_id buffer).

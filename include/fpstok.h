@@ -18,7 +18,11 @@
  *
  * Exact semantics (readings where the pages are silent):
  *   d(i, c) = ((dx*dx + dy*dy) + dz*dz) + dt*dt in float32, each operation
- *   rounded to nearest-even, never fused; first centroid = start_local[b]
+ *   rounded to nearest-even, never fused; with an optional per-axis scale w
+ *   (the time scale of graphnet PR #923's review thread on the FPS
+ *   arguments), both points' coordinates are first multiplied by w in float32
+ *   (only the metric changes: centroid positions, Lloyd means and pooled
+ *   values stay in the caller's units); first centroid = start_local[b]
  *   (default 0); each next centroid = the unselected point with the largest
  *   running minimum distance, lowest index on ties (when every unselected
  *   point is at distance 0, the lowest-index unselected point); Voronoi label
@@ -104,6 +108,9 @@ typedef struct fps_opts {
     int charge_col;    /* feature column used as Lloyd weight; -1 = unit weight */
     int force_schedule;
     int max_event_hint;/* upper bound on the largest event's N, 0 = unknown */
+    float axis_scale[4];/* per-axis weights (wx, wy, wz, wt) of the distance: both points'
+                           coordinates are multiplied by them (float32, rounded) before the
+                           distance; all zero (a zero-initialised struct) = unscaled.  Finite. */
 } fps_opts;
 
 /* Largest event (points) the FPS schedules accept. */
@@ -174,12 +181,14 @@ int fps_static_device_status(fps_stream_t stream, int *detail);
  * Nearest-centroid assignment (components/fps.py nearest_assign):
  * token_id[i] = argmin over the event's first valid_tokens[b] centroid rows of
  * d(p_i, c_j), lowest slot on ties; -1 when the event has no valid row.
- * centroids float32 [B, K, 4]; valid_tokens int32 [B] or NULL for min(N, K).
+ * centroids float32 [B, K, 4]; valid_tokens int32 [B] or NULL for min(N, K);
+ * axis_scale: HOST pointer to the 4 per-axis weights of the distance (see
+ * fps_opts), or NULL for unscaled.
  */
 size_t fps_assign_workspace_bytes(int64_t P, int B);
 int fps_assign(const float *coords, const int64_t *offsets, int B, int64_t P,
                const float *centroids, const int32_t *valid_tokens, int K, int32_t *token_id,
-               void *workspace, size_t workspace_bytes, fps_stream_t stream);
+               const float *axis_scale, void *workspace, size_t workspace_bytes, fps_stream_t stream);
 
 /*
  * kNN gather (graphnet PR #923, "What is added": farthest_point_sampling_with_knn
@@ -188,13 +197,15 @@ int fps_assign(const float *coords, const int64_t *offsets, int B, int64_t P,
  * row j of event b, the k points of the event with the smallest
  * (d(p_i, c_j), i), ascending, as global indices, -1 padded when the event has
  * fewer than k points; invalid rows are all -1.  centroids float32 [B, K, 4];
- * valid_tokens int32 [B] or NULL for min(N, K); knn_idx int32 [B, K, k].
+ * valid_tokens int32 [B] or NULL for min(N, K); knn_idx int32 [B, K, k];
+ * axis_scale: HOST pointer to the 4 per-axis weights (see fps_opts) or NULL.
  * Workspace: fps_knn_workspace_bytes() (a status word), 256-byte aligned.
  */
 size_t fps_knn_workspace_bytes(int64_t P, int B);
 int fps_knn(const float *coords, const int64_t *offsets, int B, int64_t P,
             const float *centroids, const int32_t *valid_tokens, int K, int k,
-            int32_t *knn_idx, void *workspace, size_t workspace_bytes, fps_stream_t stream);
+            int32_t *knn_idx, const float *axis_scale, void *workspace, size_t workspace_bytes,
+            fps_stream_t stream);
 
 /*
  * Charge-weighted Lloyd refinement (README "How it works", step 1) of the
@@ -203,11 +214,14 @@ int fps_knn(const float *coords, const int64_t *offsets, int B, int64_t P,
  * the cell is empty or its weight <= 0) and every point is re-assigned.
  * centroids [B,K,4] and token_id [P] are read and updated in place; events
  * with N <= K are left untouched.  feats may be NULL when charge_col = -1.
+ * axis_scale: HOST pointer to the 4 per-axis weights of the re-assignment's
+ * distance (see fps_opts) or NULL; the means stay in the caller's units.
  */
 size_t lloyd_workspace_bytes(int64_t P, int B, int K);
 int lloyd_refine(const float *coords, const float *feats, int F, int charge_col,
                  const int64_t *offsets, int B, int64_t P, int K, int iters, float *centroids,
-                 int32_t *token_id, void *workspace, size_t workspace_bytes, fps_stream_t stream);
+                 int32_t *token_id, const float *axis_scale, void *workspace, size_t workspace_bytes,
+                 fps_stream_t stream);
 
 /*
  * Per-token mean-pool ("pools the pulses of each token", graphnet PR #923,
@@ -329,6 +343,20 @@ int fps_device_status(void *workspace, fps_stream_t stream, int *detail);
 /* A cluster FPS kernel gave up waiting for its peers' candidates (a bounded
  * wait ran out); that launch's results are not valid. */
 #define FPS_DEV_EXCHANGE_TIMEOUT 5
+
+/*
+ * Test hook of the cluster schedules' bounded exchange wait (host side only;
+ * it faults nothing).  Each exchange round of an 8- or 16-CTA cluster waits
+ * at most spin_limit polls of its mbarrier (spin_limit <= 0: the default,
+ * 2^20 polls); with skip_rank >= 0, CTA skip_rank of every cluster skips its
+ * post in the first exchange of each event, so every wait of that round runs
+ * out.  A wait that runs out records FPS_DEV_EXCHANGE_TIMEOUT; that CTA leaves
+ * the event at once, its peers leave within one more round, and the whole
+ * cluster then stops taking events: the launch's results are not valid, the
+ * CUDA context stays usable.  Applies to the launches made after the call;
+ * fps_set_exchange_test(0, -1) restores the defaults.
+ */
+void fps_set_exchange_test(int spin_limit, int skip_rank);
 
 /* Human-readable name of a status code. */
 const char *fps_status_string(int status);

@@ -25,6 +25,7 @@ def run_gpu(batch, force_schedule=-1, host_offsets=False, **kw):
     c, f, o, s = to_dev(batch)
     if host_offsets:
         o = torch.from_numpy(batch.offsets)
+    kw.setdefault("axis_scale", getattr(batch, "axis_scale", None))
     out = fps.fps_tokenize(c, f, o, K=batch.K, assign_mode=batch.assign_mode, k=max(batch.k, 1),
                            lloyd_iters=batch.lloyd_iters, charge_col=batch.charge_col, start_local=s,
                            force_schedule=force_schedule, check_device=True, **kw)
@@ -45,6 +46,7 @@ def compare(batch, gpu, ora=None):
     if ora is None:
         ora = oracle.tokenize_batch(batch)
     K = batch.K
+    w = getattr(batch, "axis_scale", None)
     np.testing.assert_array_equal(gpu["centroid_idx"], ora["centroid_idx"], err_msg="centroid_idx")
     sizes = batch.sizes()
     valid = np.minimum(sizes, K).astype(np.int32)
@@ -54,7 +56,7 @@ def compare(batch, gpu, ora=None):
     else:
         assert_float_close(gpu["centroids"], ora["centroids"], "lloyd centroids")
         # the final labels are the exact nearest centroids of the GPU's centroids
-        want = oracle.assign(batch.coords, batch.offsets, gpu["centroids"], K, valid=valid)
+        want = oracle.assign(batch.coords, batch.offsets, gpu["centroids"], K, valid=valid, axis_scale=w)
         pt = np.repeat(sizes <= K, sizes)
         want[pt] = ora["token_id"][pt]
         np.testing.assert_array_equal(gpu["token_id"], want, err_msg="token_id after Lloyd")
@@ -62,7 +64,7 @@ def compare(batch, gpu, ora=None):
         if batch.lloyd_iters == 0:
             np.testing.assert_array_equal(gpu["knn_idx"], ora["knn_idx"], err_msg="knn_idx")
         else:
-            want = oracle.knn(batch.coords, batch.offsets, gpu["centroids"], K, batch.k, valid=valid)
+            want = oracle.knn(batch.coords, batch.offsets, gpu["centroids"], K, batch.k, valid=valid, axis_scale=w)
             big = sizes > K
             np.testing.assert_array_equal(gpu["knn_idx"][big], want[big], err_msg="knn_idx after Lloyd")
             np.testing.assert_array_equal(gpu["knn_idx"][~big], ora["knn_idx"][~big])

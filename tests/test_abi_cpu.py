@@ -82,13 +82,20 @@ def test_standalone_argument_errors():
     lib = fps.load_library()
     P_ = ctypes.c_void_p
     x = P_(256)
-    assert lib.fps_assign(x, x, 2, 100, x, None, 0, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
-    assert lib.fps_assign(x, x, 2, 100, x, None, 300, x, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
-    assert lib.fps_assign(x, x, 2, 100, x, None, 8, x, x, 8, None) == _lib.FPS_ERR_WORKSPACE
-    assert lib.fps_knn(x, x, 2, 100, x, None, 8, 0, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
-    assert lib.fps_knn(x, x, 2, 100, x, None, 8, 129, x, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
-    assert lib.lloyd_refine(x, None, 0, 0, x, 2, 100, 8, 1, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
-    assert lib.lloyd_refine(x, x, 6, 0, x, 2, 100, 8, -1, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    assert lib.fps_assign(x, x, 2, 100, x, None, 0, x, None, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    assert lib.fps_assign(x, x, 2, 100, x, None, 300, x, None, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
+    assert lib.fps_assign(x, x, 2, 100, x, None, 8, x, None, x, 8, None) == _lib.FPS_ERR_WORKSPACE
+    assert lib.fps_knn(x, x, 2, 100, x, None, 8, 0, x, None, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    assert lib.fps_knn(x, x, 2, 100, x, None, 8, 129, x, None, x, 1 << 20, None) == _lib.FPS_ERR_TOO_LARGE
+    assert lib.lloyd_refine(x, None, 0, 0, x, 2, 100, 8, 1, x, x, None, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    assert lib.lloyd_refine(x, x, 6, 0, x, 2, 100, 8, -1, x, x, None, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    # a non-finite axis weight is an argument error, found before anything is launched
+    bad = (ctypes.c_float * 4)(1.0, 1.0, 1.0, float("inf"))
+    assert lib.fps_assign(x, x, 2, 100, x, None, 8, x, bad, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    assert lib.fps_knn(x, x, 2, 100, x, None, 8, 4, x, bad, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    assert lib.lloyd_refine(x, None, 0, -1, x, 2, 100, 8, 1, x, x, bad, x, 1 << 20, None) == _lib.FPS_ERR_ARG
+    nan_opts = fps.Options(K=16, axis_scale=(1.0, float("nan"), 1.0, 1.0))
+    assert _tok(lib, nan_opts) == _lib.FPS_ERR_ARG
     assert lib.segment_pool(x, 6, x, 2, 100, 8, 2, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
     assert lib.segment_pool(x, 0, x, 2, 100, 8, 0, x, None, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
     assert lib.segment_pool(x, 6, x, 2, 100, 8, 1, None, x, 0, x, x, x, 1 << 20, None) == _lib.FPS_ERR_ARG
