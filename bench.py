@@ -928,7 +928,7 @@ def e2e(fps, batch, kw, dev, steps):
 
     c = torch.from_numpy(batch.coords).pin_memory()
     f = torch.from_numpy(batch.feats).pin_memory()
-    o = torch.from_numpy(batch.offsets)
+    o = torch.from_numpy(batch.offsets).pin_memory()
     kw2 = {k: v for k, v in kw.items() if k not in ("max_event_hint",)}
     out = fps.fps_tokenize_host(c, f, o, device=dev, **kw2)
     stream = torch.cuda.current_stream(dev)

@@ -196,6 +196,11 @@ def fps_tokenize_host(coords: torch.Tensor, feats: torch.Tensor, offsets: torch.
     P, F = coords.shape[0], feats.shape[1]
     B = offsets.numel() - 1
     hint = int((offsets[1:] - offsets[:-1]).max()) if B > 0 else 0
+    if coords.is_pinned():  # small inputs too: a pageable copy would hold up the overlap of the slices
+        if not offsets.is_pinned():
+            offsets = offsets.pin_memory()
+        if start_local is not None and not start_local.is_pinned():
+            start_local = start_local.pin_memory()
     opts = Options(K, assign_mode, k, lloyd_iters, charge_col, force_schedule, hint, axis_scale)
     lib = _lib.load()
     ws = _workspace(lib.fps_host_workspace_bytes(P, B, F, ctypes.byref(opts.c)), dev, workspace)

@@ -105,7 +105,14 @@ __device__ __forceinline__ void warp_fill_items(int2* dst, int base, int count, 
 // One CTA: classifies every event, builds the per-schedule work lists sorted
 // by decreasing size (longest chains first), the (event, chunk) items of FPS
 // events, and the accumulator slots; resets the status word and the cursors.
-__global__ void __launch_bounds__(1024) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
+// Threads of the one binning CTA: its passes are chains of CTA barriers, and
+// a barrier of fewer warps is cheaper.
+#ifndef FPS_BIN_THREADS
+#define FPS_BIN_THREADS 1024
+#endif
+constexpr int kBinThreads = FPS_BIN_THREADS;
+
+__global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__ offsets, int B, int64_t P,
                                                int K, const int32_t* __restrict__ start_local,
                                                int force, int chunk_all, int fused_pool, int latency_events,
                                                int mid_cluster_events, int need_passes, Workspace ws) {
@@ -311,7 +318,7 @@ cudaError_t launch_bin(const Problem& pb, const Workspace& ws, int chunk_all, cu
   const DeviceInfo& di = device_info();
   count_launch();
   const int need_passes = chunk_all || pb.lloyd_iters > 0;
-  k_bin<<<1, 1024, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
+  k_bin<<<1, kBinThreads, 0, s>>>(pb.offsets, pb.B, pb.P, pb.K, pb.start_local, pb.force_schedule, chunk_all,
                            pb.fused_pool, kLatencyEventsPerSm * di.sm_count, di.sm_count / 8, need_passes, ws);
   return cudaGetLastError();
 }

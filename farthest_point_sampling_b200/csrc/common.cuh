@@ -157,7 +157,7 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
 // Largest of the per-pair maxima pm[0 .. NP) of one lane (two interleaved
 // three-input chains, so the depth is about NP / 4).
 template <int NP>
-__device__ __forceinline__ float lane_max(const float* pm) {
+__device__ __forceinline__ float lane_max(const float (&pm)[NP]) {
   float a = pm[0], b = NP > 1 ? pm[1] : kEmptySlot;
 #pragma unroll
   for (int p = 2; p < NP; p += 4) {
@@ -174,7 +174,7 @@ __device__ __forceinline__ float lane_max(const float* pm) {
 // one compare; the low half wins when it holds M.  Returns the slot, or -1
 // when no slot of this lane holds M.
 template <int NP>
-__device__ __forceinline__ int lane_first_slot(const float* pm, const float* dist, int M) {
+__device__ __forceinline__ int lane_first_slot(const float (&pm)[NP], const float (&dist)[2 * NP], int M) {
   int cp = -1;
   float lo = 0.f;
 #pragma unroll

@@ -111,8 +111,9 @@ __device__ __forceinline__ float4 warp_pt_pos(const WarpPt& p) {
   return p;
 #endif
 }
-__device__ __forceinline__ Cent2 warp_pt_cent(const WarpPt& p, float4 w, int scaled) {
-  if (scaled) return cent2(scale4(warp_pt_pos(p), w));
+template <bool SCALED>
+__device__ __forceinline__ Cent2 warp_pt_cent(const WarpPt& p, float4 w) {
+  if (SCALED) return cent2(scale4(warp_pt_pos(p), w));
 #if FPS_WARP_DUP
   return cent2_dup(p);
 #else
@@ -135,12 +136,14 @@ __device__ __forceinline__ void relax2(uint64_t d, float& d0, float& d1, int& l0
 }
 
 // One FPS event on one warp, NP point pairs per lane (lane l owns points
-// l + 32 j, slot j = 2 p + h of pair p and half h).
-template <int NP>
+// l + 32 j, slot j = 2 p + h of pair p and half h); SCALED: the per-axis
+// scale is applied (a separate instantiation, so the common loop has no
+// branch for it).
+template <int NP, bool SCALED>
 __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                            int lane, WarpPt* s_pts, int* s_c, int32_t* __restrict__ cidx,
                                            float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
-                                           const PoolOut& po, float4 w, int scaled) {
+                                           const PoolOut& po, float4 w) {
   if (po.feats && lane < 4) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), lane, 4);
   const uint64_t z2 = opaque_zero2();
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
@@ -155,7 +158,7 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
     if (i1 < n) b = ldg4(pts + i1);
     if (i0 < n) s_pts[i0] = warp_pt(a);  // caller's units: centroid outputs (scaled per step when needed)
     if (i1 < n) s_pts[i1] = warp_pt(b);
-    if (scaled) {
+    if (SCALED) {
       a = scale4(a, w);
       b = scale4(b, w);
     }
@@ -171,10 +174,13 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
     if (i1 >= n) empty |= 1u << (2 * p + 1);
   }
   __syncwarp();
-  // steps 0 .. K-2: update with c_s, then the next centroid by arg-max
-  for (int s = 0; s < K - 1; ++s) {
+  // steps 0 .. K-2: update with c_s, then the next centroid by arg-max.  The
+  // loop leaves early only when the maximum is 0 (every unselected point
+  // duplicates a chosen one); the rest of the steps then run below.
+  int s = 0;
+  for (; s < K - 1; ++s) {
     if (lane == 0) s_c[s] = c;
-    const Cent2 C = warp_pt_cent(s_pts[c], w, scaled);
+    const Cent2 C = warp_pt_cent<SCALED>(s_pts[c], w);
     float pm[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
@@ -183,23 +189,36 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       pm[p] = fmaxf(dist[2 * p], dist[2 * p + 1]);
     }
     const int M = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
+    if (M == 0) break;
     const int slot = lane_first_slot<NP>(pm, dist, M);  // lowest slot of this lane holding the maximum
-    unsigned idx = __reduce_min_sync(kFull, slot < 0 ? 0xffffffffu : (unsigned)(slot * 32 + lane));
-    if (M == 0) {  // only duplicates of chosen points remain: the lowest-index unselected point
-      __syncwarp();
-      unsigned taken = empty;
-      for (int t = 0; t <= s; ++t) {
-        const int ct = s_c[t];
-        if ((ct & 31) == lane) taken |= 1u << (ct >> 5);
-      }
-      const unsigned free_slots = ~taken & low_bits(2 * NP);
-      idx = __reduce_min_sync(kFull, free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu);
+    c = (int)__reduce_min_sync(kFull, slot < 0 ? 0xffffffffu : (unsigned)(slot * 32 + lane));
+  }
+  // only duplicates of chosen points remain: each next centroid is the
+  // lowest-index unselected point (steps s + 1 .. K - 2; step s's update is done)
+  if (s < K - 1) {
+    __syncwarp();
+    unsigned taken = empty;
+    for (int t = 0; t <= s; ++t) {
+      const int ct = s_c[t];
+      if ((ct & 31) == lane) taken |= 1u << (ct >> 5);
     }
-    c = (int)idx;
+    for (;;) {
+      const unsigned free_slots = ~taken & low_bits(2 * NP);
+      c = (int)__reduce_min_sync(kFull, free_slots ? (unsigned)((__ffs(free_slots) - 1) * 32 + lane) : 0xffffffffu);
+      if ((c & 31) == lane) taken |= 1u << (c >> 5);
+      if (++s == K - 1) break;
+      if (lane == 0) s_c[s] = c;
+      const Cent2 C = warp_pt_cent<SCALED>(s_pts[c], w);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
+        relax2(d, dist[2 * p], dist[2 * p + 1], lab[2 * p], lab[2 * p + 1], s);
+      }
+    }
   }
   {  // step K-1: the last centroid only updates the labels
     if (lane == 0) s_c[K - 1] = c;
-    const Cent2 C = warp_pt_cent(s_pts[c], w, scaled);
+    const Cent2 C = warp_pt_cent<SCALED>(s_pts[c], w);
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
       const uint64_t d = dist2(X[p], Y[p], Z[p], T[p], C, z2);
@@ -219,37 +238,53 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       if (i < n) tok[i] = lab[j];
     }
   }
-  if (po.feats) {  // token means: float64 shared sums over the event copy's space
+  if (po.feats) {  // token means: counting sort of the labels, then each lane sums its tokens' rows
     const int F = po.F;
     __syncwarp();
-    double* acc = reinterpret_cast<double*>(s_pts);  // [K * F]
-    int* cnt = reinterpret_cast<int*>(acc + K * F);   // [K]
-    for (int e = lane; e < K * F; e += 32) acc[e] = 0.0;
+    int* s_lab = reinterpret_cast<int*>(s_pts);  // [64 NP] over the event copy's space
+    int* perm = s_lab + 64 * NP;                 // [64 NP]
+    int* cnt = perm + 64 * NP;                   // [K], then start [K] and cur [K]
+    int* start = cnt + K;
+    int* cur = start + K;
     for (int j = lane; j < K; j += 32) cnt[j] = 0;
     __syncwarp();
-    const float* fe = po.feats + off * F;
 #pragma unroll
-    for (int j = 0; j < 2 * NP; ++j) {  // slot j: 32 consecutive rows, one per lane
+    for (int j = 0; j < 2 * NP; ++j) {
       const int i = j * 32 + lane;
-      if (i >= n) continue;
-      const int l = lab[j];
-      atomicAdd(&cnt[l], 1);
-      const float* row = fe + (int64_t)i * F;
-      for (int f0 = 0; f0 < F; f0 += 8) {
-        float v[8];
-#pragma unroll
-        for (int f = 0; f < 8; ++f) v[f] = f0 + f < F ? __ldg(row + f0 + f) : 0.f;
-#pragma unroll
-        for (int f = 0; f < 8; ++f)
-          if (f0 + f < F) atomicAdd(&acc[l * F + f0 + f], (double)v[f]);
+      if (i < n) {
+        s_lab[i] = lab[j];
+        atomicAdd(&cnt[lab[j]], 1);
       }
     }
     __syncwarp();
-    for (int j = lane; j < K; j += 32) {
-      const int c2 = cnt[j];
-      float* prow = po.pooled + (b * K + j) * F;
-      for (int f = 0; f < F; ++f) prow[f] = c2 ? (float)(acc[j * F + f] / (double)c2) : 0.f;
-      po.counts[b * K + j] = c2;
+    count_scan(cnt, start, cur, K, lane);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < n) perm[atomicAdd(&cur[lab[j]], 1)] = i;
+    }
+    __syncwarp();
+    const float* fe = po.feats + off * F;
+    for (int t = lane; t < K; t += 32) {  // token t: points perm[start .. start + c), in float64
+      const int c2 = cnt[t];
+      const int* pt = perm + start[t];
+      float* prow = po.pooled + (b * K + t) * F;
+      for (int f0 = 0; f0 < F; f0 += 8) {
+        double acc8[8];
+#pragma unroll
+        for (int f = 0; f < 8; ++f) acc8[f] = 0.0;
+        for (int q = 0; q < c2; ++q) {
+          const float* row = fe + (int64_t)pt[q] * F + f0;
+#pragma unroll
+          for (int f = 0; f < 8; ++f)
+            if (f0 + f < F) acc8[f] += (double)__ldg(row + f);
+        }
+#pragma unroll
+        for (int f = 0; f < 8; ++f)
+          if (f0 + f < F) prow[f0 + f] = c2 ? (float)(acc8[f] / (double)c2) : 0.f;
+      }
+      po.counts[b * K + t] = c2;
     }
   }
   __syncwarp();  // the next event overwrites this warp's copy
@@ -288,8 +323,12 @@ __global__ void __launch_bounds__(128, FPS_WARP_MIN_BLOCKS) k_fps_warp(const flo
     const int c0 = start_local ? start_local[b] : 0;
     int32_t* tok = token_id ? token_id + off : nullptr;
 #define WARP_CALL(N)                                                                                   \
-  warp_event<N>(coords + off, n, c0, K, off, lane, s_pts, s_c, centroid_idx + (int64_t)b * K,          \
-                centroids + (int64_t)b * K, tok, b, po, w, scaled)
+  if (scaled)                                                                                          \
+    warp_event<N, true>(coords + off, n, c0, K, off, lane, s_pts, s_c, centroid_idx + (int64_t)b * K,  \
+                        centroids + (int64_t)b * K, tok, b, po, w);                                    \
+  else                                                                                                 \
+    warp_event<N, false>(coords + off, n, c0, K, off, lane, s_pts, s_c, centroid_idx + (int64_t)b * K, \
+                         centroids + (int64_t)b * K, tok, b, po, w)
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
   }
@@ -372,8 +411,7 @@ __device__ __forceinline__ void cta_event(const float4* __restrict__ pts, int n,
     if (s == K - 1) break;
     const int wM = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
     const int slot = lane_first_slot<NP>(pm, dist, wM);
-    const unsigned cand = slot < 0 ? 0xffffffffu : (unsigned)(slot * NT + tid);
-    const unsigned widx = __reduce_min_sync(kFull, cand);
+    const unsigned widx = __reduce_min_sync(kFull, slot < 0 ? 0xffffffffu : (unsigned)(slot * NT + tid));
     int M;
     unsigned idx;
     exchange(wM, widx, M, idx);
@@ -546,7 +584,7 @@ struct BlockShared {
 // (the budget is set where ptxas reports no spills); the other pairs are read
 // from shared memory every step.
 __host__ __device__ constexpr int block_reg_pairs(int np) {
-  return np < (215 - 5 * np) / 8 ? np : ((215 - 5 * np) / 8 > 0 ? (215 - 5 * np) / 8 : 0);
+  return np < (140 - 5 * np) / 8 ? np : ((140 - 5 * np) / 8 > 0 ? (140 - 5 * np) / 8 : 0);
 }
 
 // Returns true when an exchange wait ran out (the CTA left the step loop and
@@ -568,61 +606,88 @@ __device__ __forceinline__ bool block_event(const float4* __restrict__ pts, int 
 
   // One exchange of (key, index, position) candidates: the event's winner --
   // largest key, then lowest index -- in M, idx, pos on every thread.
-  // Clusters: every warp sends its winner into its own slot (rank * NW +
-  // warp) of every CTA of the cluster with st.async, which signals the
-  // receiving CTA's mbarrier with its bytes; every warp arrives on its own
-  // CTA's mbarrier once per round (count NW, each arrival expecting CL posts:
-  // NW * CL in all), lane 0 waits for the phase (bounded), and the warp
-  // reduces the E = CL * NW posted candidates itself.  No barrier of any kind
-  // per round.  Rounds alternate between two slot sets and mbarriers (round &
-  // 1; phase parity (round >> 1) & 1): a warp cannot post round r + 2 before
-  // every warp of the cluster has posted round r + 1, which each does after
-  // reading round r; a phase cannot complete before every local warp has
-  // arrived for it.  Returns false when the wait ran out (the warp leaves the
-  // event; the others follow within a round, as its posts stop).
+  // Clusters: the CTA's warp winners meet in shared memory (one barrier);
+  // warp 0 reduces them and sends the CTA winner into slot `rank` of every
+  // CTA of the cluster with st.async, which signals the receiving CTA's
+  // mbarrier with its bytes; lane 0 of warp 0 waits (bounded) for the CL
+  // posts, warp 0 reduces them and broadcasts the winner with the outcome of
+  // the wait through shared memory (a second barrier), so that every thread
+  // of the CTA takes the same path.  No cluster barrier and no release fence.
+  // Rounds alternate between two slot sets and mbarriers (round & 1; phase
+  // parity (round >> 1) & 1): a CTA cannot post round r + 2 before every peer
+  // has posted round r + 1, which each does after reading round r.  Posts
+  // arriving before the local arm are counted in the same phase (it cannot
+  // complete before the local arrival).  Returns false when the wait ran
+  // out: every thread of the CTA leaves the event.
   auto exchange = [&](int key, unsigned idx_in, float4 pos_in, bool first, int& M, unsigned& idx,
                       float4& pos) -> bool {
     bool ok = true;
     if constexpr (CL > 1) {
-      static_assert(E % 32 == 0 && E <= 256, "posted candidates per lane");
+      int2* lkey = xkey + (round & 1) * NW;
+      float4* lpos = xpos + (round & 1) * NW;
       const int p = round & 1;
       const uint32_t parity = (uint32_t)(round >> 1) & 1u;
-      ExSlot* slots = xslot + p * E;
+      ExSlot* slots = xslot + p * CL;
+      ExSlot* bcs = reinterpret_cast<ExSlot*>(xpos + 2 * NW) + p;
       const uint32_t bar = smem_addr(&xbar[p]);
       ++round;
-      if (lane == 0) mbar_arrive_expect(bar, CL * kExSlotBytes);
-      const bool post = !(first && rank == xcfg.skip_rank);
-      if (lane < CL && post) {  // this warp's winner into slot rank * NW + warp of CTA `lane`
-        const uint32_t ra = peer_addr(smem_addr(&slots[rank * NW + warp]), lane);
-        const uint32_t rb = peer_addr(bar, lane);
-        st_async_v4(ra, key, (int)idx_in, __float_as_int(pos_in.x), __float_as_int(pos_in.y), rb);
-        st_async_v2(ra + 16, __float_as_int(pos_in.z), __float_as_int(pos_in.w), rb);
+      if (lane == 0) {
+        lkey[warp] = make_int2(key, (int)idx_in);
+        lpos[warp] = pos_in;
       }
-      bool got = false;
-      if (lane == 0)
-        for (int it = 0; it < xcfg.spin_limit && !got; ++it) got = mbar_try_wait(bar, parity);
-      got = __shfl_sync(kFull, got ? 1 : 0, 0) != 0;
-      if (!got) {
-        if (lane == 0) record_error(hdr, kDevExchangeTimeout);
-        return false;
+      __syncthreads();
+      if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect(bar, CL * kExSlotBytes);
+        const int2 v = lane < NW ? lkey[lane] : make_int2(-0x7fffffff - 1, -1);
+        int cM;
+        unsigned cI;
+        warp_argmax(v.x, (unsigned)v.y, cM, cI);
+        const unsigned who = __ballot_sync(kFull, lane < NW && v.x == cM && (unsigned)v.y == cI);
+        const float4 cp = lpos[__ffs(who) - 1];
+        const bool post = !(first && rank == xcfg.skip_rank);
+        if (lane < CL && post) {
+          const uint32_t ra = peer_addr(smem_addr(&slots[rank]), lane);
+          const uint32_t rb = peer_addr(bar, lane);
+          st_async_v4(ra, cM, (int)cI, __float_as_int(cp.x), __float_as_int(cp.y), rb);
+          st_async_v2(ra + 16, __float_as_int(cp.z), __float_as_int(cp.w), rb);
+        }
+        bool got = false;
+        if (lane == 0)
+          for (int it = 0; it < xcfg.spin_limit && !got; ++it) got = mbar_try_wait(bar, parity);
+        got = __shfl_sync(kFull, got ? 1 : 0, 0) != 0;
+        int2 w2 = make_int2(-0x7fffffff - 1, -1);
+        if (got && lane < CL) {
+          const int4 a = slots[lane].a;
+          w2 = make_int2(a.x, a.y);
+        }
+        int wM;
+        unsigned wI;
+        warp_argmax(w2.x, (unsigned)w2.y, wM, wI);
+        const unsigned wwho = __ballot_sync(kFull, lane < CL && w2.x == wM && (unsigned)w2.y == wI);
+        if (lane == 0) {
+          ExSlot bc;
+          bc.a = make_int4(wM, (int)wI, 0, 0);
+          bc.b = make_int2(0, 0);
+          bc.pad = make_int2(got ? 1 : 0, 0);
+          if (got) {
+            const ExSlot& x = slots[__ffs(wwho) - 1];
+            bc.a.z = x.a.z;
+            bc.a.w = x.a.w;
+            bc.b = x.b;
+          } else {
+            bc.a = make_int4(-1, 0, 0, 0);
+            record_error(hdr, kDevExchangeTimeout);
+          }
+          *bcs = bc;
+        }
       }
-      int bk = -0x7fffffff - 1;  // best (key, index) of this lane's E / 32 slots, and which slot
-      unsigned bi = 0xffffffffu;
-      int bs = 0;
-#pragma unroll
-      for (int q = 0; q < E / 32; ++q) {
-        const int e = lane + 32 * q;
-        const int4 a = slots[e].a;
-        const bool better = a.x > bk || (a.x == bk && (unsigned)a.y < bi);
-        bk = better ? a.x : bk;
-        bi = better ? (unsigned)a.y : bi;
-        bs = better ? e : bs;
-      }
-      warp_argmax(bk, bi, M, idx);
-      const unsigned who = __ballot_sync(kFull, bk == M && bi == idx);
-      const ExSlot& x = slots[__shfl_sync(kFull, bs, __ffs(who) - 1)];
-      pos = make_float4(__int_as_float(x.a.z), __int_as_float(x.a.w), __int_as_float(x.b.x),
-                        __int_as_float(x.b.y));
+      __syncthreads();
+      const ExSlot bc = *bcs;
+      M = bc.a.x;
+      idx = (unsigned)bc.a.y;
+      pos = make_float4(__int_as_float(bc.a.z), __int_as_float(bc.a.w), __int_as_float(bc.b.x),
+                        __int_as_float(bc.b.y));
+      ok = bc.pad.x != 0;
       return ok;
     } else {
       (void)first;
@@ -710,8 +775,7 @@ __device__ __forceinline__ bool block_event(const float4* __restrict__ pts, int 
     if (s == K - 1) break;
     const int wM = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
     const int slot = lane_first_slot<NP>(pm, dist, wM);
-    const unsigned wcand = slot < 0 ? 0xffffffffu : (unsigned)(g + G * slot);
-    const unsigned widx = __reduce_min_sync(kFull, wcand);
+    const unsigned widx = __reduce_min_sync(kFull, slot < 0 ? 0xffffffffu : (unsigned)(g + G * slot));
     float4 wpos = make_float4(0.f, 0.f, 0.f, 0.f);
     if (wM >= 0) wpos = local_pos(widx);
     int M;
@@ -767,8 +831,8 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
   ulonglong2* sZT = sXY + PS * NT;                            // [PS][NT] packed (z, t)
   int2* xkey = reinterpret_cast<int2*>(sZT + PS * NT);        // [2][E] (key, index)
   float4* xpos = reinterpret_cast<float4*>(xkey + 2 * E);     // [2][E] candidate position
-  ExSlot* xslot = reinterpret_cast<ExSlot*>(xpos + 2 * E);    // [2][E] posted warp winners (clusters)
-  ExSlot* xbc = xslot + 2 * E;                                 // unused placeholder (layout continuity)
+  ExSlot* xslot = reinterpret_cast<ExSlot*>(xpos + 2 * E);    // [2][CL] posted CTA winners (clusters)
+  ExSlot* xbc = xslot + 2 * CL;                                // spare (the broadcast lives in xpos)
   uint64_t* xbar = reinterpret_cast<uint64_t*>(xbc + 2);       // [2] exchange mbarriers
   __shared__ int s_item;
   __shared__ int s_abort;  // an exchange wait of this CTA ran out (sticky for the launch)
@@ -778,8 +842,8 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     rank = (int)cg::this_cluster().block_rank();
     if (threadIdx.x == 0) {
       s_abort = 0;
-      mbar_init(smem_addr(&xbar[0]), NT / 32);  // one arrival per warp and round
-      mbar_init(smem_addr(&xbar[1]), NT / 32);
+      mbar_init(smem_addr(&xbar[0]), 1);  // armed once per round, by warp 0
+      mbar_init(smem_addr(&xbar[1]), 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     cg::this_cluster().sync();  // every CTA is running, its barriers initialised, before DSMEM use
@@ -816,7 +880,7 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
     FPS_BLOCK_BUCKETS(np, BLOCK_CALL)
 #undef BLOCK_CALL
     if constexpr (CL > 1) {
-      if (aborted && (threadIdx.x & 31) == 0) s_abort = 1;  // any warp that left the event
+      if (aborted && threadIdx.x == 0) s_abort = 1;  // the whole CTA left the event
       cg::this_cluster().sync();  // s_item is rewritten for the next claim; abort flags are final
       // A wait that ran out leaves its mbarrier phase incomplete, so no CTA of
       // the cluster may run another event: every CTA reads every peer's flag
@@ -847,7 +911,7 @@ template <int CL>
 constexpr size_t block_smem_bytes() {
   return (size_t)2 * kBlockPairs * kBlockThreads * sizeof(ulonglong2) +
          (size_t)2 * BlockShared<CL, kBlockThreads>::E * (sizeof(int2) + sizeof(float4)) +
-         (size_t)2 * BlockShared<CL, kBlockThreads>::E * sizeof(ExSlot) + 2 * sizeof(ExSlot) + 2 * sizeof(uint64_t);
+         (size_t)2 * CL * sizeof(ExSlot) + 2 * sizeof(ExSlot) + 2 * sizeof(uint64_t);
 }
 
 template <int CL>

@@ -2,6 +2,7 @@
 // checks, workspace carving and the launch sequence.  No allocation, no
 // synchronisation (except fps_device_status, which exists to read back).
 #include <atomic>
+#include <mutex>
 #include <cmath>
 #include <cstring>
 
@@ -221,14 +222,19 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
   axis_scale_of(opts->axis_scale, &pb.w, &pb.scaled);
   if (opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0) {
     const size_t K = (size_t)opts->K, Fz = (size_t)F;
-    if (K * Fz * sizeof(double) + K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
+    if ((size_t)2 * kWarpCap * sizeof(int) + 3 * K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
     if ((size_t)(3 * kCtaCap + 768) * sizeof(int) + (size_t)kCtaCap * Fz * sizeof(float) <= cta_region_bytes())
       pb.fused_pool |= 2;
   }
   return run_tokenize(pb, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Host-pointer variant: staging layout after the regular workspace.
+// Host-pointer variant: staging layout after the regular workspace.  The
+// batch goes through in up to kHostChunks slices of consecutive events, each
+// slice's offsets in its own staging rows (slice c: rows b0 + c .. b1 + c).
+constexpr int kHostChunks = 4;
+constexpr int64_t kHostChunkMinPoints = 65536;  // smaller batches go in one piece
+
 struct HostStage {
   size_t coords, feats, offsets, start, cidx, tok, knn, cents, pooled, counts, total;
 };
@@ -245,7 +251,7 @@ static HostStage host_stage(size_t base, int64_t P, int B, int F, const fps_opts
   const int k = o->assign_mode == FPS_ASSIGN_KNN ? o->k : 0;
   h.coords = take((size_t)P * 16);
   h.feats = take((size_t)P * F * 4);
-  h.offsets = take((size_t)(B + 1) * 8);
+  h.offsets = take((size_t)(B + 1 + kHostChunks) * 8);
   h.start = take(has_start ? (size_t)B * 4 : 0);
   h.cidx = take((size_t)B * K * 4);
   h.tok = take((size_t)P * 4);
@@ -255,6 +261,39 @@ static HostStage host_stage(size_t base, int64_t P, int B, int F, const fps_opts
   h.counts = take((size_t)B * K * 4);
   h.total = off;
   return h;
+}
+
+// Streams and events of the host-buffer pipeline, per device: copies in and
+// out run on their own streams beside the caller's (compute) stream.
+struct HostPipe {
+  cudaStream_t in, out;
+  cudaEvent_t fork, in_done[kHostChunks], comp_done[kHostChunks], out_done;
+  bool ready;
+};
+constexpr int kMaxHostDevices = 64;
+static HostPipe g_pipe[kMaxHostDevices];
+static std::mutex g_pipe_mu;
+
+static cudaError_t host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxHostDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    if ((e = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking))) return e;
+    if ((e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking))) return e;
+    if ((e = cudaEventCreateWithFlags(&hp.fork, cudaEventDisableTiming))) return e;
+    if ((e = cudaEventCreateWithFlags(&hp.out_done, cudaEventDisableTiming))) return e;
+    for (int c = 0; c < kHostChunks; ++c) {
+      if ((e = cudaEventCreateWithFlags(&hp.in_done[c], cudaEventDisableTiming))) return e;
+      if ((e = cudaEventCreateWithFlags(&hp.comp_done[c], cudaEventDisableTiming))) return e;
+    }
+    hp.ready = true;
+  }
+  *out = &hp;
+  return cudaSuccess;
 }
 
 size_t fps_host_workspace_bytes(int64_t P, int B, int F, const fps_opts* opts) {
@@ -275,6 +314,13 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
   if (opts->assign_mode == FPS_ASSIGN_VORONOI && !token_id && P > 0) return FPS_ERR_ARG;
   if (opts->assign_mode == FPS_ASSIGN_KNN && !knn_idx) return FPS_ERR_ARG;
   if (P > 0 && (!coords || !feats)) return FPS_ERR_ARG;
+  if (offsets[0] != 0 || offsets[B] != P) return FPS_ERR_ARG;  // host offsets: checked here
+  for (int b = 0; b < B; ++b) {
+    const int64_t n = offsets[b + 1] - offsets[b];
+    if (n < 0) return FPS_ERR_ARG;
+    if (n > kClusterCap) return FPS_ERR_TOO_LARGE;
+    if (start_local && n > opts->K && (start_local[b] < 0 || start_local[b] >= n)) return FPS_ERR_ARG;
+  }
   const size_t base = fps_workspace_bytes(P, B, F, opts);
   const HostStage h = host_stage(base, P, B, F, opts, start_local != nullptr);
   if (!workspace || workspace_bytes < h.total || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
@@ -282,29 +328,77 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int K = opts->K;
   const int k = opts->assign_mode == FPS_ASSIGN_KNN ? opts->k : 0;
+  HostPipe* hp = nullptr;
+  cudaError_t e;
+  if ((e = host_pipe(&hp))) return from_cuda(e);
+
+  // slices of consecutive events with about equal points (host offsets)
+  int nc = (P >= kHostChunkMinPoints && B >= 2) ? (B < kHostChunks ? B : kHostChunks) : 1;
+  int bnd[kHostChunks + 1];
+  bnd[0] = 0;
+  for (int c = 1; c < nc; ++c) {
+    const int64_t target = P * c / nc;
+    int lo = bnd[c - 1] + 1, hi = B - (nc - c);  // at least one event per slice
+    while (lo < hi) {  // first b with offsets[b] >= target
+      const int mid = lo + (hi - lo) / 2;
+      if (offsets[mid] < target) lo = mid + 1;
+      else hi = mid;
+    }
+    bnd[c] = lo;
+  }
+  bnd[nc] = B;
+
   auto h2d = [&](size_t at, const void* src, size_t n) {
-    return n ? cudaMemcpyAsync(w + at, src, n, cudaMemcpyHostToDevice, s) : cudaSuccess;
+    return n ? cudaMemcpyAsync(w + at, src, n, cudaMemcpyHostToDevice, hp->in) : cudaSuccess;
   };
   auto d2h = [&](void* dst, size_t at, size_t n) {
-    return (n && dst) ? cudaMemcpyAsync(dst, w + at, n, cudaMemcpyDeviceToHost, s) : cudaSuccess;
+    return (n && dst) ? cudaMemcpyAsync(dst, w + at, n, cudaMemcpyDeviceToHost, hp->out) : cudaSuccess;
   };
-  cudaError_t e;
-  if ((e = h2d(h.coords, coords, (size_t)P * 16)) || (e = h2d(h.feats, feats, (size_t)P * F * 4)) ||
-      (e = h2d(h.offsets, offsets, (size_t)(B + 1) * 8)) ||
-      (e = h2d(h.start, start_local, start_local ? (size_t)B * 4 : 0)))
+  // copies in wait for the caller's earlier work (staging rows are reused across calls)
+  if ((e = cudaEventRecord(hp->fork, s)) || (e = cudaStreamWaitEvent(hp->in, hp->fork, 0)) ||
+      (e = cudaStreamWaitEvent(hp->out, hp->fork, 0)))
     return from_cuda(e);
-  rc = fps_tokenize(reinterpret_cast<const float*>(w + h.coords), reinterpret_cast<const float*>(w + h.feats),
-                    F, reinterpret_cast<const int64_t*>(w + h.offsets), B, P,
-                    start_local ? reinterpret_cast<const int32_t*>(w + h.start) : nullptr, opts,
-                    reinterpret_cast<int32_t*>(w + h.cidx), token_id ? reinterpret_cast<int32_t*>(w + h.tok) : nullptr,
-                    k ? reinterpret_cast<int32_t*>(w + h.knn) : nullptr, reinterpret_cast<float*>(w + h.cents),
-                    reinterpret_cast<float*>(w + h.pooled), reinterpret_cast<int32_t*>(w + h.counts), workspace,
-                    base, stream);
-  if (rc) return rc;
-  if ((e = d2h(centroid_idx, h.cidx, (size_t)B * K * 4)) || (e = d2h(token_id, h.tok, (size_t)P * 4)) ||
-      (e = d2h(k ? knn_idx : nullptr, h.knn, (size_t)B * K * k * 4)) ||
-      (e = d2h(centroids, h.cents, (size_t)B * K * 16)) || (e = d2h(pooled, h.pooled, (size_t)B * K * F * 4)) ||
-      (e = d2h(counts, h.counts, (size_t)B * K * 4)))
+  for (int c = 0; c < nc; ++c) {  // every slice's inputs, back to back
+    const int b0 = bnd[c], b1 = bnd[c + 1];
+    const int64_t p0 = offsets[b0], p1 = offsets[b1];
+    if ((e = h2d(h.coords + (size_t)p0 * 16, coords + p0 * 4, (size_t)(p1 - p0) * 16)) ||
+        (e = h2d(h.feats + (size_t)p0 * F * 4, feats + p0 * F, (size_t)(p1 - p0) * F * 4)) ||
+        (e = h2d(h.offsets + (size_t)(b0 + c) * 8, offsets + b0, (size_t)(b1 - b0 + 1) * 8)) ||
+        (e = h2d(h.start + (size_t)b0 * 4, start_local ? start_local + b0 : nullptr,
+                 start_local ? (size_t)(b1 - b0) * 4 : 0)) ||
+        (e = cudaEventRecord(hp->in_done[c], hp->in)))
+      return from_cuda(e);
+  }
+  for (int c = 0; c < nc; ++c) {  // each slice: rebase, tokenize, renumber on the caller's stream; copy out
+    const int b0 = bnd[c], b1 = bnd[c + 1], bc = b1 - b0;
+    const int64_t p0 = offsets[b0], pc = offsets[b1] - p0;
+    if ((e = cudaStreamWaitEvent(s, hp->in_done[c], 0))) return from_cuda(e);
+    int64_t* off_c = reinterpret_cast<int64_t*>(w + h.offsets) + b0 + c;
+    if ((e = launch_rebase_offsets(off_c, bc + 1, p0, s))) return from_cuda(e);
+    int32_t* cidx_c = reinterpret_cast<int32_t*>(w + h.cidx) + (int64_t)b0 * K;
+    int32_t* knn_c = k ? reinterpret_cast<int32_t*>(w + h.knn) + (int64_t)b0 * K * k : nullptr;
+    rc = fps_tokenize(reinterpret_cast<const float*>(w + h.coords) + p0 * 4,
+                      reinterpret_cast<const float*>(w + h.feats) + p0 * F, F, off_c, bc, pc,
+                      start_local ? reinterpret_cast<const int32_t*>(w + h.start) + b0 : nullptr, opts, cidx_c,
+                      token_id ? reinterpret_cast<int32_t*>(w + h.tok) + p0 : nullptr, knn_c,
+                      reinterpret_cast<float*>(w + h.cents) + (int64_t)b0 * K * 4,
+                      reinterpret_cast<float*>(w + h.pooled) + (int64_t)b0 * K * F,
+                      reinterpret_cast<int32_t*>(w + h.counts) + (int64_t)b0 * K, workspace, base, stream);
+    if (rc) return rc;
+    if ((e = launch_shift_indices(cidx_c, (int64_t)bc * K, (int32_t)p0, s))) return from_cuda(e);
+    if (knn_c && (e = launch_shift_indices(knn_c, (int64_t)bc * K * k, (int32_t)p0, s))) return from_cuda(e);
+    if ((e = cudaEventRecord(hp->comp_done[c], s)) || (e = cudaStreamWaitEvent(hp->out, hp->comp_done[c], 0)))
+      return from_cuda(e);
+    if ((e = d2h(centroid_idx + (int64_t)b0 * K, h.cidx + (size_t)b0 * K * 4, (size_t)bc * K * 4)) ||
+        (e = d2h(token_id ? token_id + p0 : nullptr, h.tok + (size_t)p0 * 4, (size_t)pc * 4)) ||
+        (e = d2h(k ? knn_idx + (int64_t)b0 * K * k : nullptr, h.knn + (size_t)b0 * K * k * 4,
+                 (size_t)bc * K * k * 4)) ||
+        (e = d2h(centroids + (int64_t)b0 * K * 4, h.cents + (size_t)b0 * K * 16, (size_t)bc * K * 16)) ||
+        (e = d2h(pooled + (int64_t)b0 * K * F, h.pooled + (size_t)b0 * K * F * 4, (size_t)bc * K * F * 4)) ||
+        (e = d2h(counts + (int64_t)b0 * K, h.counts + (size_t)b0 * K * 4, (size_t)bc * K * 4)))
+      return from_cuda(e);
+  }
+  if ((e = cudaEventRecord(hp->out_done, hp->out)) || (e = cudaStreamWaitEvent(s, hp->out_done, 0)))
     return from_cuda(e);
   return FPS_OK;
 }

@@ -143,6 +143,11 @@ cudaError_t prepare_aux_kernels();   // shared-memory attributes of the auxiliar
 
 void count_launch(int n = 1);
 
+// Chunk pipeline of the host-buffer entry point: offsets[i] -= base, and
+// non-negative indices += shift.
+cudaError_t launch_rebase_offsets(int64_t* off, int n, int64_t base, cudaStream_t s);
+cudaError_t launch_shift_indices(int32_t* idx, int64_t n, int32_t shift, cudaStream_t s);
+
 // Test setting of the cluster exchange of the next launches: the poll limit
 // of each wait (<= 0: the default) and a CTA rank that skips its post in the
 // first exchange of every event (-1: none).

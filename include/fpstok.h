@@ -137,8 +137,16 @@ int fps_tokenize(const float *coords, const float *feats, int F, const int64_t *
  * Same as fps_tokenize but every input and output pointer is a HOST pointer
  * (page-locked memory gives asynchronous copies).  The inputs are staged into
  * the device workspace, the tokenizer runs there and the outputs are copied
- * back, all on `stream`; the results are valid once the stream is
- * synchronised.  Workspace size: fps_host_workspace_bytes().
+ * back; the results are valid once `stream` is synchronised.  Batches of at
+ * least 65,536 points go through in up to 4 slices of consecutive events
+ * with about equal points: a slice's inputs are copied in on one internal
+ * stream, it is tokenized on `stream`, and its outputs are copied out on
+ * another internal stream, so that copies in, compute and copies out of
+ * different slices overlap; `stream` waits for everything before it is
+ * synchronised.  Because offsets and start_local are host data, they are
+ * checked here (non-decreasing, offsets[0] = 0, offsets[B] = P, each start
+ * inside its event) and a violation returns FPS_ERR_ARG before anything is
+ * copied.  Workspace size: fps_host_workspace_bytes().
  */
 size_t fps_host_workspace_bytes(int64_t P, int B, int F, const fps_opts *opts);
 int fps_tokenize_host(const float *coords, const float *feats, int F, const int64_t *offsets,

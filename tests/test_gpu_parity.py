@@ -178,11 +178,41 @@ def test_standalone_pool():
     assert_float_close(pooled.cpu().numpy(), wp, "segment_pool knn")
 
 
+def _host_run(b, **kw):
+    out = fps.fps_tokenize_host(torch.from_numpy(b.coords).pin_memory(), torch.from_numpy(b.feats).pin_memory(),
+                                torch.from_numpy(b.offsets), K=b.K, assign_mode=b.assign_mode, k=max(b.k, 1),
+                                lloyd_iters=b.lloyd_iters, charge_col=b.charge_col, **kw)
+    return {k: v.numpy() for k, v in out.items()}
+
+
 def test_host_entry_point():
     b = workloads.make_workload("c1")
-    out = fps.fps_tokenize_host(torch.from_numpy(b.coords).pin_memory(), torch.from_numpy(b.feats).pin_memory(),
-                                torch.from_numpy(b.offsets), K=b.K)
-    compare(b, {k: v.numpy() for k, v in out.items()})
+    compare(b, _host_run(b))
+
+
+@pytest.mark.parametrize("name", ["c4", "c2", "c3"])
+def test_host_entry_point_in_slices(name):
+    # batches of 65,536 points or more go through in slices of consecutive
+    # events (copies in, compute and copies out overlapping): the slices'
+    # global indices, kNN rows and Lloyd centroids must come back as one batch
+    b = workloads.make_workload(name)
+    assert b.P >= 65536
+    compare(b, _host_run(b))
+
+
+def test_host_entry_point_start_indices_and_host_checks():
+    b = workloads.random_batch(64, [40000, 30000, 20, 5000, 9000], 32, start_local=[7, 29999, 0, 4, 8])
+    st = torch.from_numpy(b.start_local)
+    compare(b, _host_run(b, start_local=st))
+    bad = st.clone()
+    bad[1] = 30000  # outside its event: refused on the host, nothing runs
+    with pytest.raises(fps.FpsError):
+        _host_run(b, start_local=bad)
+    off = torch.from_numpy(b.offsets).clone()
+    off[2] = off[1] - 1  # decreasing offsets
+    with pytest.raises(fps.FpsError):
+        fps.fps_tokenize_host(torch.from_numpy(b.coords).pin_memory(), torch.from_numpy(b.feats).pin_memory(), off,
+                              K=b.K)
 
 
 # ------------------------------------------------------------- degenerate inputs and errors
