@@ -96,6 +96,11 @@ typedef float4 WarpPt;
 #endif
 constexpr int kWarpPtBytes = (int)sizeof(WarpPt);
 constexpr int kWarpListInts = FPS_MAX_K_DEV;  // chosen local indices, one per step
+// Shared memory of one warp: the event copy and the list, then room for the
+// pooling's staged feature rows (the whole region is reused by it).
+constexpr int kWarpRegionBytes = 12288;
+static_assert(64 * kWarpPairs * kWarpPtBytes + kWarpListInts * 4 <= kWarpRegionBytes, "event copy and list fit");
+static_assert(8 * FPS_MAX_K_DEV + 4 * kWarpCap <= kWarpRegionBytes, "one staged feature per pass fits");
 
 __device__ __forceinline__ WarpPt warp_pt(float4 a) {
 #if FPS_WARP_DUP
@@ -140,10 +145,11 @@ __device__ __forceinline__ void relax2(uint64_t d, float& d0, float& d1, int& l0
 // scale is applied (a separate instantiation, so the common loop has no
 // branch for it).
 template <int NP, bool SCALED>
-__device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
+__device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, int c, int K, int64_t off,
                                            int lane, WarpPt* s_pts, int* s_c, int32_t* __restrict__ cidx,
                                            float4* __restrict__ cpos, int32_t* __restrict__ tok, int64_t b,
-                                           const PoolOut& po, float4 w) {
+                                           const PoolOut& po, float4 w, int* claim_ctr, int claim_base,
+                                           int& next) {
   if (po.feats && lane < 4) prefetch_rows_l2(po.feats + off * po.F, (size_t)n * po.F * sizeof(float), lane, 4);
   const uint64_t z2 = opaque_zero2();
   uint64_t X[NP], Y[NP], Z[NP], T[NP];
@@ -225,6 +231,8 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       relax2(d, dist[2 * p], dist[2 * p + 1], lab[2 * p], lab[2 * p + 1], K - 1);
     }
   }
+  // the next item is claimed here, so that the atomic's round trip overlaps the writes and the pooling below
+  if (lane == 0) next = claim_base + atomicAdd(claim_ctr, 1);
   __syncwarp();
   for (int j = lane; j < K; j += 32) {  // the event's centroids, once
     const int cj = s_c[j];
@@ -238,53 +246,63 @@ __device__ __forceinline__ void warp_event(const float4* __restrict__ pts, int n
       if (i < n) tok[i] = lab[j];
     }
   }
-  if (po.feats) {  // token means: counting sort of the labels, then each lane sums its tokens' rows
+  if (po.feats) {
+    // Token means.  Every point's rank inside its token (one shared atomic
+    // each), the token starts by a scan of the counts, then per pass of at
+    // most 8 features: the lanes copy their points' rows into shared memory
+    // in token order (independent loads, all in flight), and lane t sums
+    // token t's contiguous rows in float64.
     const int F = po.F;
     __syncwarp();
-    int* s_lab = reinterpret_cast<int*>(s_pts);  // [64 NP] over the event copy's space
-    int* perm = s_lab + 64 * NP;                 // [64 NP]
-    int* cnt = perm + 64 * NP;                   // [K], then start [K] and cur [K]
+    int* cnt = reinterpret_cast<int*>(s_pts);  // [K] counts, then [K] starts, then the staged rows
     int* start = cnt + K;
-    int* cur = start + K;
+    float* sf = reinterpret_cast<float*>(start + K);
     for (int j = lane; j < K; j += 32) cnt[j] = 0;
     __syncwarp();
+    int pos[2 * NP];
 #pragma unroll
-    for (int j = 0; j < 2 * NP; ++j) {
-      const int i = j * 32 + lane;
-      if (i < n) {
-        s_lab[i] = lab[j];
-        atomicAdd(&cnt[lab[j]], 1);
-      }
-    }
+    for (int j = 0; j < 2 * NP; ++j) pos[j] = j * 32 + lane < n ? atomicAdd(&cnt[lab[j]], 1) : 0;
     __syncwarp();
-    count_scan(cnt, start, cur, K, lane);
+    count_scan(cnt, start, start, K, lane);
     __syncwarp();
 #pragma unroll
-    for (int j = 0; j < 2 * NP; ++j) {
-      const int i = j * 32 + lane;
-      if (i < n) perm[atomicAdd(&cur[lab[j]], 1)] = i;
-    }
-    __syncwarp();
+    for (int j = 0; j < 2 * NP; ++j)
+      if (j * 32 + lane < n) pos[j] += start[lab[j]];
+    const int fcap = (kWarpRegionBytes - 8 * K) / (4 * n);  // features one pass can stage (>= 1)
+    const int FC = min(min(F, 8), fcap);
     const float* fe = po.feats + off * F;
-    for (int t = lane; t < K; t += 32) {  // token t: points perm[start .. start + c), in float64
-      const int c2 = cnt[t];
-      const int* pt = perm + start[t];
-      float* prow = po.pooled + (b * K + t) * F;
-      for (int f0 = 0; f0 < F; f0 += 8) {
-        double acc8[8];
+    for (int f0 = 0; f0 < F; f0 += FC) {
+      const int fc = min(FC, F - f0);
 #pragma unroll
-        for (int f = 0; f < 8; ++f) acc8[f] = 0.0;
-        for (int q = 0; q < c2; ++q) {
-          const float* row = fe + (int64_t)pt[q] * F + f0;
+      for (int j = 0; j < 2 * NP; ++j) {
+        const int i = j * 32 + lane;
+        if (i < n) {
+          const float* row = fe + (int64_t)i * F + f0;
+          float* dst = sf + pos[j] * fc;
 #pragma unroll
           for (int f = 0; f < 8; ++f)
-            if (f0 + f < F) acc8[f] += (double)__ldg(row + f);
+            if (f < fc) dst[f] = __ldg(row + f);
         }
+      }
+      __syncwarp();
+      for (int t = lane; t < K; t += 32) {
+        const int c2 = cnt[t];
+        const float* src = sf + start[t] * fc;
+        double a[8];
+#pragma unroll
+        for (int f = 0; f < 8; ++f) a[f] = 0.0;
+        for (int q = 0; q < c2; ++q, src += fc) {
+#pragma unroll
+          for (int f = 0; f < 8; ++f)
+            if (f < fc) a[f] += (double)src[f];
+        }
+        float* prow = po.pooled + (b * K + t) * F + f0;
 #pragma unroll
         for (int f = 0; f < 8; ++f)
-          if (f0 + f < F) prow[f0 + f] = c2 ? (float)(acc8[f] / (double)c2) : 0.f;
+          if (f < fc) prow[f] = c2 ? (float)(a[f] / (double)c2) : 0.f;
+        if (f0 == 0) po.counts[b * K + t] = c2;
       }
-      po.counts[b * K + t] = c2;
+      __syncwarp();
     }
   }
   __syncwarp();  // the next event overwrites this warp's copy
@@ -308,15 +326,16 @@ __global__ void __launch_bounds__(128, FPS_WARP_MIN_BLOCKS) k_fps_warp(const flo
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
   extern __shared__ __align__(16) unsigned char s_warp_all[];
   const int lane = threadIdx.x & 31;
-  unsigned char* mine = s_warp_all + (size_t)(threadIdx.x >> 5) * (64 * NPMAX * kWarpPtBytes + kWarpListInts * 4);
+  unsigned char* mine = s_warp_all + (size_t)(threadIdx.x >> 5) * kWarpRegionBytes;
   WarpPt* s_pts = reinterpret_cast<WarpPt*>(mine);                      // this warp's event copy
   int* s_c = reinterpret_cast<int*>(mine + 64 * NPMAX * kWarpPtBytes);  // its chosen local indices
   const int count = hdr->n_items[kListWarp];
-  for (;;) {
-    int item = 0;
-    if (lane == 0) item = atomicAdd(&hdr->next_item[kListWarp], 1);
-    item = __shfl_sync(kFull, item, 0);
-    if (item >= count) break;
+  // the first item of every warp is its global warp index; later ones come
+  // from the shared cursor, offset by the number of warps
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  int* ctr = &hdr->next_item[kListWarp];
+  int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  while (item < count) {
     const int b = list[item];
     const int64_t off = offsets[b];
     const int n = (int)(offsets[b + 1] - off);
@@ -325,12 +344,15 @@ __global__ void __launch_bounds__(128, FPS_WARP_MIN_BLOCKS) k_fps_warp(const flo
 #define WARP_CALL(N)                                                                                   \
   if (scaled)                                                                                          \
     warp_event<N, true>(coords + off, n, c0, K, off, lane, s_pts, s_c, centroid_idx + (int64_t)b * K,  \
-                        centroids + (int64_t)b * K, tok, b, po, w);                                    \
+                        centroids + (int64_t)b * K, tok, b, po, w, ctr, nwarps, next);                 \
   else                                                                                                 \
     warp_event<N, false>(coords + off, n, c0, K, off, lane, s_pts, s_c, centroid_idx + (int64_t)b * K, \
-                         centroids + (int64_t)b * K, tok, b, po, w)
+                         centroids + (int64_t)b * K, tok, b, po, w, ctr, nwarps, next)
+    int next = -1;
     FPS_DISPATCH_7((n + 63) >> 6, WARP_CALL)
 #undef WARP_CALL
+    if (lane == 0 && next < 0) next = nwarps + atomicAdd(ctr, 1);
+    item = __shfl_sync(kFull, next, 0);
   }
 }
 
@@ -900,11 +922,11 @@ __global__ void __launch_bounds__(NT, 1) k_fps_block(const float4* __restrict__ 
 // ------------------------------------------------------------------ launch
 
 constexpr int kWarpBlock = 128;
-constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * (64 * kWarpPairs * kWarpPtBytes + kWarpListInts * 4);
+constexpr size_t kWarpSmem = (size_t)(kWarpBlock / 32) * kWarpRegionBytes;
 constexpr size_t kCtaSmem = kCtaSmemBytes;
 static_assert((size_t)2 * kCtaThreads * kCtaPairs * sizeof(DupPoint) <= kCtaSmem, "event copy fits");
 
-size_t warp_region_bytes() { return (size_t)64 * kWarpPairs * kWarpPtBytes; }
+size_t warp_region_bytes() { return (size_t)kWarpRegionBytes; }
 size_t cta_region_bytes() { return kCtaSmem; }
 
 template <int CL>

@@ -222,7 +222,7 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
   axis_scale_of(opts->axis_scale, &pb.w, &pb.scaled);
   if (opts->assign_mode == FPS_ASSIGN_VORONOI && opts->lloyd_iters == 0) {
     const size_t K = (size_t)opts->K, Fz = (size_t)F;
-    if ((size_t)2 * kWarpCap * sizeof(int) + 3 * K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
+    if ((size_t)kWarpCap * sizeof(float) + 2 * K * sizeof(int) <= warp_region_bytes()) pb.fused_pool |= 1;
     if ((size_t)(3 * kCtaCap + 768) * sizeof(int) + (size_t)kCtaCap * Fz * sizeof(float) <= cta_region_bytes())
       pb.fused_pool |= 2;
   }
@@ -232,8 +232,10 @@ int fps_tokenize(const float* coords, const float* feats, int F, const int64_t* 
 // Host-pointer variant: staging layout after the regular workspace.  The
 // batch goes through in up to kHostChunks slices of consecutive events, each
 // slice's offsets in its own staging rows (slice c: rows b0 + c .. b1 + c).
-constexpr int kHostChunks = 4;
+constexpr int kHostChunks = 6;
 constexpr int64_t kHostChunkMinPoints = 65536;  // smaller batches go in one piece
+constexpr int kHostChunkMinEvents = 256;        // and so do batches of few (large) events: a slice of them
+                                                // would leave the GPU mostly idle
 
 struct HostStage {
   size_t coords, feats, offsets, start, cidx, tok, knn, cents, pooled, counts, total;
@@ -332,12 +334,14 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
   cudaError_t e;
   if ((e = host_pipe(&hp))) return from_cuda(e);
 
-  // slices of consecutive events with about equal points (host offsets)
-  int nc = (P >= kHostChunkMinPoints && B >= 2) ? (B < kHostChunks ? B : kHostChunks) : 1;
+  // slices of consecutive events by points: the first and the last half as
+  // large as the others, so that compute starts early and the tail (last
+  // compute and copy out) is short
+  const int nc = (P >= kHostChunkMinPoints && B >= kHostChunkMinEvents) ? kHostChunks : 1;
   int bnd[kHostChunks + 1];
   bnd[0] = 0;
   for (int c = 1; c < nc; ++c) {
-    const int64_t target = P * c / nc;
+    const int64_t target = P * (2 * c - 1) / (2 * (nc - 1));  // 1/(2(nc-1)) first, 1/(nc-1) each middle one
     int lo = bnd[c - 1] + 1, hi = B - (nc - c);  // at least one event per slice
     while (lo < hi) {  // first b with offsets[b] >= target
       const int mid = lo + (hi - lo) / 2;

@@ -111,7 +111,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
 // kNN mode without Lloyd: launch_fps runs each schedule's kNN rows on that
 // schedule's stream right after its FPS kernel.
 inline bool knn_with_fps(const Problem& pb) { return pb.assign_mode == 1 && pb.lloyd_iters == 0; }
-// Bytes of shared memory of the warp-schedule event copy (per warp) and of
+// Bytes of shared memory of one warp of the warp schedule and of
 // the register-CTA schedule (per CTA): fused pooling must fit into them.
 size_t warp_region_bytes();
 size_t cta_region_bytes();

@@ -138,8 +138,9 @@ int fps_tokenize(const float *coords, const float *feats, int F, const int64_t *
  * (page-locked memory gives asynchronous copies).  The inputs are staged into
  * the device workspace, the tokenizer runs there and the outputs are copied
  * back; the results are valid once `stream` is synchronised.  Batches of at
- * least 65,536 points go through in up to 4 slices of consecutive events
- * with about equal points: a slice's inputs are copied in on one internal
+ * least 65,536 points and 256 events go through in 6 slices of consecutive
+ * events (by points; the first and the last half as large as the others):
+ * a slice's inputs are copied in on one internal
  * stream, it is tokenized on `stream`, and its outputs are copied out on
  * another internal stream, so that copies in, compute and copies out of
  * different slices overlap; `stream` waits for everything before it is
