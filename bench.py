@@ -853,7 +853,7 @@ def token_summaries_roofline(fps, dev, reps=30):
             "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
             "algorithmic_bytes": byts,
             "algorithmic": "16P coords + 4FP feats + 4P token ids + 8(B+1) offsets read, B*K*(4+16+4F) written",
-            "kernels_per_call": per_call, "note": "memset + tile sums + finalize"}
+            "kernels_per_call": per_call, "note": "status-word memset + per-range sums + boundary finalize"}
 
 
 def token_pack_roofline(fps, dev, reps=50):

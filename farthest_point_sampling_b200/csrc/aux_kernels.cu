@@ -559,6 +559,12 @@ cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offset
                                                                      ws);
   cudaError_t e = cudaGetLastError();
   if (e) return e;
+  return launch_pool_finalize(offsets, K, F, pooled, counts, ws, s);
+}
+
+cudaError_t launch_pool_finalize(const int64_t* offsets, int K, int F, float* pooled, int32_t* counts,
+                                 const Workspace& ws, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
   count_launch();
   k_pool_finalize<<<di.sm_count * 2, 256, 0, s>>>(offsets, pooled, counts, K, F, ws);
   return cudaGetLastError();
@@ -811,6 +817,73 @@ __device__ __forceinline__ void lloyd_piece_sums(const float4* __restrict__ pts,
     if (sm.cnt[e / 5]) atomicAdd(&out[e], sm.acc[e]);
 }
 
+// Where the last Lloyd iteration writes the token means (Voronoi mode of
+// the tokenizer): feats == nullptr when it does not pool.
+struct LloydPool {
+  const float* feats;
+  float* pooled;
+  int32_t* counts;
+};
+
+// Token means of one pass in the last Lloyd iteration: the pass's points
+// sorted by their final label, float64 sums of their feature rows per token
+// in groups of up to 5 features (the accumulator of the cell sums), then the
+// means and counts of an event pooled in one piece written directly
+// (gacc == nullptr), or the sums and counts added into the event's
+// accumulator replica, whose means k_pool_finalize forms.  Each thread reads
+// back the labels it wrote for its own points.
+__device__ __forceinline__ void lloyd_piece_pool(const float* __restrict__ fe, int F, const int32_t* lab, int npts,
+                                                 int K, const LloydSmem& sm, float* __restrict__ prow,
+                                                 int32_t* __restrict__ crow, double* __restrict__ gacc,
+                                                 int* __restrict__ gcnt) {
+  constexpr int T = kLloydThreads;
+  const int tid = threadIdx.x;
+  for (int j = tid; j < K; j += T) sm.cnt[j] = 0;
+  __syncthreads();
+  int l[kLloydPts];
+#pragma unroll
+  for (int r = 0; r < kLloydPts; ++r) {
+    const int li = tid + r * T;
+    l[r] = li < npts ? lab[li] : -1;
+    if ((unsigned)l[r] >= (unsigned)K) l[r] = -1;  // never: the labels were just written
+    if (l[r] >= 0) atomicAdd(&sm.cnt[l[r]], 1);
+  }
+  __syncthreads();
+  if (tid < 32) count_scan(sm.cnt, sm.start, sm.cur, K, tid);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kLloydPts; ++r) {
+    if (l[r] >= 0) {
+      const int pos = atomicAdd(&sm.cur[l[r]], 1);
+      sm.perm[pos] = tid + r * T;
+      sm.slab[pos] = l[r];
+    }
+  }
+  __syncthreads();
+  const int nsorted = sm.start[K - 1] + sm.cnt[K - 1];
+  for (int g0 = 0; g0 < F; g0 += 5) {
+    const int V = min(5, F - g0);
+    for (int e = tid; e < K * 5; e += T) sm.acc[e] = 0.0;
+    __syncthreads();
+    segment_sums(sm.perm, sm.slab, nsorted, V, 0, 5, sm.acc, tid, T,
+                 [&](int i, int v) { return (double)__ldg(fe + (int64_t)i * F + g0 + v); });
+    __syncthreads();
+    for (int e = tid; e < K * 5; e += T) {
+      const int j = e / 5, v = e - 5 * j;
+      if (v >= V) continue;
+      const int c = sm.cnt[j];
+      if (!gacc) prow[j * F + g0 + v] = c ? (float)(sm.acc[e] / (double)c) : 0.f;
+      else if (c) atomicAdd(&gacc[j * F + g0 + v], sm.acc[e]);
+    }
+    if (g0 == 0)
+      for (int j = tid; j < K; j += T) {
+        if (!gacc) crow[j] = sm.cnt[j];
+        else if (sm.cnt[j]) atomicAdd(&gcnt[j], sm.cnt[j]);
+      }
+    __syncthreads();
+  }
+}
+
 // Cell sums of the current labels.
 __global__ void __launch_bounds__(kLloydThreads, kPassCtasPerSm) k_lloyd_sums(const float4* __restrict__ coords,
                                                                  const float* __restrict__ feats, int F,
@@ -849,7 +922,7 @@ __global__ void __launch_bounds__(kLloydThreads, kPassCtasPerSm) k_lloyd_step(co
                                                                  const double* __restrict__ in,
                                                                  double* __restrict__ next,
                                                                  double* __restrict__ clear, int64_t clear_n,
-                                                                 float4 w) {
+                                                                 float4 w, LloydPool pool) {
   constexpr int T = kLloydThreads;
   extern __shared__ __align__(16) char smem_c[];
   const LloydSmem sm = lloyd_smem(smem_c);
@@ -896,6 +969,20 @@ __global__ void __launch_bounds__(kLloydThreads, kPassCtasPerSm) k_lloyd_step(co
       lloyd_piece_sums(coords + off, feats ? feats + off * F : nullptr, F, charge_col, lab_out, npts, K, sm,
                        next + (int64_t)fs * K * 5, ws.hdr);
       __syncthreads();  // the next pass re-zeroes the sums
+    } else if (pool.feats) {  // the last iteration: the pass's token means (replica piece % nrep)
+      const int ps = ws.pool_slot[b];
+      double* gacc = nullptr;
+      int* gcnt = nullptr;
+      if (ps >= 0) {
+        const int n = (int)(offsets[b + 1] - offsets[b]);
+        const int nrep = min(kPoolReplicas, (n + kPoolChunk - 1) / kPoolChunk);
+        const int slot = ps + (i0 / kPass) % nrep;
+        gacc = ws.pool_acc + (int64_t)slot * K * F;
+        gcnt = ws.pool_cnt + (int64_t)slot * K;
+      }
+      lloyd_piece_pool(pool.feats + off * F, F, lab_out, npts, K, sm, pool.pooled + (int64_t)b * K * F,
+                       pool.counts + (int64_t)b * K, gacc, gcnt);
+      __syncthreads();
     }
   }
 }
@@ -920,10 +1007,11 @@ cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels
     const bool last = t == pb.lloyd_iters - 1;
     double* clear = (t + 1 < pb.lloyd_iters - 1) ? ws.lloyd[(t + 2) % 3] : nullptr;
     count_launch();
+    const LloydPool pool = {last && lloyd_pools(pb) ? pb.feats : nullptr, pb.pooled, pb.counts};
     k_lloyd_step<<<grid, kLloydThreads, sm_step, s>>>(pb.coords, feats, pb.F, pb.charge_col, pb.offsets, K, labels,
                                                       pb.centroids, ws, ws.lloyd[t % 3],
                                                       last ? nullptr : ws.lloyd[(t + 1) % 3], clear,
-                                                      clear ? (int64_t)ws.fps_slots * per : 0, pb.w);
+                                                      clear ? (int64_t)ws.fps_slots * per : 0, pb.w, pool);
     if ((e = cudaGetLastError())) return e;
   }
   return cudaSuccess;

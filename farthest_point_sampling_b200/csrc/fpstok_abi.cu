@@ -165,7 +165,11 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
     // in place needs no pool kernel
     const bool none_left = pb.max_event_hint > 0 && pb.max_event_hint <= kCtaCap && pb.force_schedule <= 1 &&
                            (pb.fused_pool & 3) == 3;
-    if (!none_left) {
+    if (pb.lloyd_iters > 0 && lloyd_pools(pb)) {  // the last Lloyd iteration pooled; the replicas' means
+      stage_mark(8, 0, s);
+      if ((e = launch_pool_finalize(pb.offsets, pb.K, pb.F, pb.pooled, pb.counts, ws, s))) return from_cuda(e);
+      stage_mark(8, 1, s);
+    } else if (!none_left) {
       stage_mark(8, 0, s);
       if ((e = launch_pool_voronoi(pb.feats, pb.F, pb.offsets, pb.B, pb.K, labels, pb.pooled, pb.counts, ws, s)))
         return from_cuda(e);
@@ -618,8 +622,7 @@ int fps_random_starts(const int64_t* offsets, int B, uint64_t seed, uint32_t str
 
 size_t fps_token_summaries_workspace_bytes(int B, int K, int F) {
   if (B < 0 || K < 1 || F < 1) return 0;
-  return align256(sizeof(WsHeader)) +
-         align256((size_t)token_summary_replicas(B, K, F) * B * K * (5 + F) * sizeof(double));
+  return align256(sizeof(WsHeader)) + align256(token_summary_partial_bytes(K, F));
 }
 
 int fps_token_summaries(const float* coords, const float* feats, int F, int charge_col, const int64_t* offsets,
@@ -636,10 +639,10 @@ int fps_token_summaries(const float* coords, const float* feats, int F, int char
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* hdr = static_cast<WsHeader*>(workspace);
-  double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + align256(sizeof(WsHeader)));
+  double* partial = reinterpret_cast<double*>(static_cast<char*>(workspace) + align256(sizeof(WsHeader)));
   cudaError_t e;
   if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
-  return from_cuda(launch_token_summaries(coords, feats, F, charge_col, offsets, B, P, K, token_id, acc, wsum,
+  return from_cuda(launch_token_summaries(coords, feats, F, charge_col, offsets, B, P, K, token_id, partial, wsum,
                                           wcoords, wfeats, hdr, s));
 }
 

@@ -115,7 +115,13 @@ inline bool knn_with_fps(const Problem& pb) { return pb.assign_mode == 1 && pb.l
 // the register-CTA schedule (per CTA): fused pooling must fit into them.
 size_t warp_region_bytes();
 size_t cta_region_bytes();
+// Lloyd refinement; in the tokenizer's Voronoi mode (lloyd_pools) the last
+// iteration also pools the token means (k_pool_finalize still follows for
+// the events pooled over several pieces).
+inline bool lloyd_pools(const Problem& pb) { return pb.assign_mode == 0 && pb.pooled && pb.feats; }
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s);
+cudaError_t launch_pool_finalize(const int64_t* offsets, int K, int F, float* pooled, int32_t* counts,
+                                 const Workspace& ws, cudaStream_t s);
 cudaError_t launch_pool_voronoi(const float* feats, int F, const int64_t* offsets, int B, int K,
                                 const int32_t* labels, float* pooled, int32_t* counts,
                                 const Workspace& ws, cudaStream_t s);

@@ -6,13 +6,16 @@
 // float64 sums, means 0 for an empty cell or wsum <= 0, each output rounded
 // once to float32.
 //
-// k_token_sums takes the point array in tiles of kSumTile points, staging the
-// tile's coordinate and feature rows in shared memory (coalesced) when they
-// fit.  A tile that spans few events sorts its points by (event, token) with
-// a counting sort in shared memory and adds each non-empty (token, value) sum
-// to the float64 accumulators once; a tile spanning more events than its bucket
-// table holds (events of a few points each) adds point by point.
-// k_token_finalize sums the replicas in order, divides and rounds.
+// k_token_sums gives every CTA one contiguous range of points (the whole
+// array split evenly over the grid), so that the inputs stream through once.
+// The CTA walks the events that meet its range; for each it takes the
+// event's points in tiles: rows staged in shared memory, a counting sort by
+// token, then one thread per (token, group of values) adds its points' q and
+// q-weighted values in float64 registers and once into the event's
+// accumulators [K, 5 + F] in shared memory (no atomics).  It then writes the
+// event's means directly when the event lies inside its range, or else its
+// partial sums into its own slot of the workspace.  k_token_finalize then adds, per event cut by a
+// range boundary, the partial sums of the CTAs it spans in CTA order.
 #include "../../include/fpstok.h"
 #include "common.cuh"
 #include "internal.h"
@@ -23,230 +26,280 @@ namespace fpstok {
 namespace {
 
 constexpr int kSumThreads = 256;
-constexpr int kSumPts = 4;
-constexpr int kSumTile = kSumThreads * kSumPts;
-constexpr int kMaxBuckets = 2048;  // (events in the tile) * K of the counting sort
-// Tiles add into up to kSumMaxReplicas copies of the accumulators (tile i into
-// copy i mod R), as many as fit in kSumReplicaBudget bytes: the tiles of a large
-// event would otherwise all serialise on the same few accumulator lines.
-constexpr int kSumMaxReplicas = 16;
-constexpr int64_t kSumReplicaBudget = 32ll << 20;
-constexpr int kSumStageBytes = 160 * 1024;  // dynamic shared memory for the staged tile rows
+constexpr int kSumTile = 1024;                   // points staged and sorted at a time
+constexpr int kSumGroup = 8;                     // features summed together by one thread
+constexpr int kSumMinPoints = 1024;              // points per CTA at least
+constexpr int kSumMaxCtas = 512;                 // CTAs (partial-sum slots) at most
+constexpr int kSumCtasPerSm = 3;                 // resident CTAs per SM (shared memory at K = 128, F <= 8)
+constexpr int64_t kSumPartialBudget = 32ll << 20;  // bytes of partial sums at most
 
-__device__ __forceinline__ int sum_event_of(const int64_t* __restrict__ offsets, int lo, int hi, int64_t i) {
+// First event b >= lo whose span ends after point p (offsets[b + 1] > p),
+// searching [lo, hi]; hi when none.
+__device__ __forceinline__ int sum_first_event_after(const int64_t* __restrict__ offsets, int lo, int hi,
+                                                     int64_t p) {
   while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(offsets + mid) <= i) lo = mid;
-    else hi = mid - 1;
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(offsets + mid + 1) > p) hi = mid;
+    else lo = mid + 1;
   }
   return lo;
 }
 
-// Value v of point i: q, q * coords[i, v-1] (v = 1..4), q * feats[i, v-5].
-__device__ __forceinline__ double summary_value(const float* __restrict__ coords, const float* __restrict__ feats,
-                                                int F, int charge_col, int64_t i, int v) {
-  const double q = charge_col >= 0 ? (double)__ldg(feats + i * F + charge_col) : 1.0;
-  if (v == 0) return q;
-  if (v < 5) return q * (double)__ldg(coords + 4 * i + (v - 1));
-  return q * (double)__ldg(feats + i * F + (v - 5));
-}
-
-// Value v of tile point p (point i): q, q * coords[i, v-1] (v = 1..4),
-// q * feats[i, v-5], read from the tile's rows staged in shared memory (sc:
-// [n, 4], sf: [n, F]) when staged, else from global memory.
-__device__ __forceinline__ double tile_value(const float* sc, const float* sf, bool staged,
-                                             const float* __restrict__ coords, const float* __restrict__ feats,
-                                             int F, int charge_col, int64_t t0, int p, int v) {
-  if (!staged) return summary_value(coords, feats, F, charge_col, t0 + p, v);
-  const double q = charge_col >= 0 ? (double)sf[p * F + charge_col] : 1.0;
-  if (v == 0) return q;
-  if (v < 5) return q * (double)sc[p * 4 + (v - 1)];
-  return q * (double)sf[p * F + (v - 5)];
-}
-
-__global__ void __launch_bounds__(kSumThreads) k_token_sums(const float* __restrict__ coords,
+__global__ void __launch_bounds__(kSumThreads) k_token_sums(const float4* __restrict__ coords,
                                                             const float* __restrict__ feats, int F, int charge_col,
                                                             const int64_t* __restrict__ offsets, int B, int64_t P,
-                                                            int K, const int32_t* __restrict__ token_id, int reps,
-                                                            int staged, double* __restrict__ acc, WsHeader* hdr) {
-  extern __shared__ float s_rows[];  // staged tile rows: coords [kSumTile, 4], then feats [kSumTile, F]
-  __shared__ int s_cnt[kMaxBuckets];        // counts, then fill cursors
-  __shared__ int s_start[kMaxBuckets + 1];  // exclusive scan of the counts
-  __shared__ int s_perm[kSumTile];          // tile points sorted by bucket
-  __shared__ int s_key[kSumTile];           // bucket of each tile point, -1 none
-  __shared__ int s_ev[2];
-  __shared__ int s_warp[kSumThreads / 32];
+                                                            int K, const int32_t* __restrict__ token_id,
+                                                            int64_t chunk, float* __restrict__ wsum,
+                                                            float* __restrict__ wcoords, float* __restrict__ wfeats,
+                                                            double* __restrict__ partial, WsHeader* hdr) {
+  extern __shared__ __align__(16) unsigned char s_raw[];
   const int V = 5 + F;
+  const int KV = K * V;
+  const bool staged = F <= kSumGroup;
+  float4* s_c = reinterpret_cast<float4*>(s_raw);                        // [tile] coordinates (16-byte copies)
+  double* s_acc = reinterpret_cast<double*>(s_c + kSumTile);              // [K, V]
+  float* s_q = reinterpret_cast<float*>(s_acc + KV);                      // [tile] charges
+  int* s_lab = reinterpret_cast<int*>(s_q + kSumTile);                    // [tile] tokens (-1: none)
+  int* s_perm = s_lab + kSumTile;                                         // [tile] points sorted by token
+  int* s_cnt = s_perm + kSumTile;                                         // [256] counts, [256] starts,
+  int* s_start = s_cnt + 256;                                             // [256] fill cursors
+  int* s_cur = s_start + 256;
+  float* s_f = reinterpret_cast<float*>(s_cur + 256);                     // [tile, F] when staged
+  const int NG = 1 + (F + kSumGroup - 1) / kSumGroup;  // value groups: (q, q*coords), then features
   const int tid = threadIdx.x;
-  const int rep = blockIdx.x % reps;  // accumulator replica of this tile
-  const int64_t t0 = (int64_t)blockIdx.x * kSumTile;
-  const int n = (int)min((int64_t)kSumTile, P - t0);
-  int t[kSumPts];
-#pragma unroll
-  for (int r = 0; r < kSumPts; ++r) {
-    const int p = tid + r * kSumThreads;
-    t[r] = p < n ? token_id[t0 + p] : -1;
-  }
-  float* sc = s_rows;
-  float* sf = s_rows + 4 * kSumTile;
-  if (staged) {  // coalesced copies of the tile's rows
-    const float4* c4 = reinterpret_cast<const float4*>(coords) + t0;
-    for (int p = tid; p < n; p += kSumThreads) reinterpret_cast<float4*>(sc)[p] = __ldg(c4 + p);
-    const float* fr = feats + t0 * F;
-    for (int e = tid; e < n * F; e += kSumThreads) sf[e] = __ldg(fr + e);
-  }
-  if (tid < 2) s_ev[tid] = sum_event_of(offsets, 0, B - 1, tid ? t0 + n - 1 : t0);
-  __syncthreads();
-  const int lo = s_ev[0], hi = max(s_ev[0], s_ev[1]);
-  const int64_t nb64 = (int64_t)(hi - lo + 1) * K;
-  const bool dense = nb64 <= kMaxBuckets;  // block-uniform
-  const int NB = dense ? (int)nb64 : 0;
-  for (int e = tid; e < NB; e += kSumThreads) s_cnt[e] = 0;
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kSumPts; ++r) {
-    const int p = tid + r * kSumThreads;
-    if (p >= n) continue;
-    const int64_t i = t0 + p;
-    const int b = sum_event_of(offsets, lo, hi, i);
-    int key = -1;
-    if (__ldg(offsets + b) > i || __ldg(offsets + b + 1) <= i) record_error(hdr, kDevBadOffsets);
-    else if (t[r] >= K || t[r] < -1) record_error(hdr, kDevBadToken);
-    else if (t[r] >= 0) key = (b - lo) * K + t[r];
-    if (key >= 0 && !dense) {  // point by point into the accumulators
-      double* a = acc + (((int64_t)rep * B + b) * K + t[r]) * V;
-      for (int v = 0; v < V; ++v) atomicAdd(a + v, summary_value(coords, feats, F, charge_col, i, v));
-      key = -1;
+  const bool last_cta = blockIdx.x == gridDim.x - 1;
+  const int64_t p0 = (int64_t)blockIdx.x * chunk;
+  const int64_t p1 = last_cta ? P : min(P, p0 + chunk);
+  if (blockIdx.x == 0 && tid == 0 && (offsets[0] != 0 || offsets[B] != P)) record_error(hdr, kDevBadOffsets);
+  // the event holding point p0, preceded by the empty events that start at p0
+  int b = sum_first_event_after(offsets, 0, B - 1, p0);
+  while (b > 0 && offsets[b - 1] >= p0 && offsets[b] == p0) --b;
+  for (; b < B; ++b) {
+    const int64_t e0 = offsets[b], e1 = offsets[b + 1];
+    if (e0 >= p1 && !(last_cta && e0 == P)) break;  // the next range's events
+    if (e1 < e0 || e0 < 0 || e1 > P) {
+      if (tid == 0) record_error(hdr, kDevBadOffsets);
+      continue;
     }
-    s_key[p] = key;
-    if (key >= 0) atomicAdd(s_cnt + key, 1);
-  }
-  __syncthreads();
-  if (!dense) return;
-  // exclusive scan of s_cnt[0..NB): contiguous chunks per thread, then warps
-  {
-    const int lane = tid & 31, warp = tid >> 5;
-    const int ch = (NB + kSumThreads - 1) / kSumThreads;
-    const int a = min(NB, tid * ch), z = min(NB, a + ch);
-    int sum = 0;
-    for (int e = a; e < z; ++e) sum += s_cnt[e];
-    int x = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = lane < kSumThreads / 32 ? s_warp[lane] : 0;
-      const int w0 = w;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
+    const int64_t s0 = max(e0, p0), s1 = min(e1, p1);
+    for (int e = tid; e < KV; e += kSumThreads) s_acc[e] = 0.0;
+    for (int64_t t0 = s0; t0 < s1; t0 += kSumTile) {
+      const int n = (int)min((int64_t)kSumTile, s1 - t0);
+      // the tile's rows into shared memory by asynchronous copies, in flight
+      // while the tokens are loaded and counted
+      for (int j = tid; j < K; j += kSumThreads) s_cnt[j] = 0;
+      const uint32_t sc0 = (uint32_t)__cvta_generic_to_shared(s_c);
+#pragma unroll 4
+      for (int li = tid; li < n; li += kSumThreads)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sc0 + 16u * (uint32_t)li), "l"(coords + t0 + li)
+                     : "memory");
+      if (staged) {
+        const float* fr = feats + t0 * F;
+        const uint32_t sf0 = (uint32_t)__cvta_generic_to_shared(s_f);
+#pragma unroll 8
+        for (int e = tid; e < n * F; e += kSumThreads)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sf0 + 4u * (uint32_t)e), "l"(fr + e)
+                       : "memory");
       }
-      if (lane < kSumThreads / 32) s_warp[lane] = w - w0;
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      __syncthreads();  // counts zeroed
+#pragma unroll 4
+      for (int li = tid; li < n; li += kSumThreads) {
+        const int64_t i = t0 + li;
+        int t = token_id[i];
+        if (t < -1 || t >= K) {
+          record_error(hdr, kDevBadToken);
+          t = -1;
+        }
+        s_lab[li] = t;
+        if (!staged) s_q[li] = charge_col >= 0 ? __ldg(feats + i * F + charge_col) : 1.f;
+        if (t >= 0) atomicAdd(&s_cnt[t], 1);
+      }
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+      if (staged)
+        for (int li = tid; li < n; li += kSumThreads) s_q[li] = charge_col >= 0 ? s_f[li * F + charge_col] : 1.f;
+      if (tid < 32) count_scan(s_cnt, s_start, s_cur, K, tid);
+      __syncthreads();
+      for (int li = tid; li < n; li += kSumThreads) {
+        const int t = s_lab[li];
+        if (t >= 0) s_perm[atomicAdd(&s_cur[t], 1)] = li;
+      }
+      __syncthreads();
+      // one thread per (token, value group): its points in sorted order,
+      // float64 sums in registers, added once into the token's accumulators
+      for (int it = tid; it < K * NG; it += kSumThreads) {
+        const int j = it / NG, g = it - j * NG;
+        const int c = s_cnt[j];
+        if (c == 0) continue;
+        const int* pj = s_perm + s_start[j];
+        double a[kSumGroup];
+#pragma unroll
+        for (int v = 0; v < kSumGroup; ++v) a[v] = 0.0;
+        double* dst = s_acc + j * V;
+        if (g == 0) {
+          for (int m = 0; m < c; ++m) {
+            const int li = pj[m];
+            const double q = (double)s_q[li];
+            const float4 p = s_c[li];
+            a[0] += q;
+            a[1] += q * (double)p.x;
+            a[2] += q * (double)p.y;
+            a[3] += q * (double)p.z;
+            a[4] += q * (double)p.w;
+          }
+#pragma unroll
+          for (int v = 0; v < 5; ++v) dst[v] += a[v];
+        } else {
+          const int f0 = (g - 1) * kSumGroup;
+          const int nf = min(kSumGroup, F - f0);
+          for (int m = 0; m < c; ++m) {
+            const int li = pj[m];
+            const double q = (double)s_q[li];
+            const float* row = staged ? s_f + li * F + f0 : feats + (t0 + li) * F + f0;
+#pragma unroll
+            for (int v = 0; v < kSumGroup; ++v)
+              if (v < nf) a[v] += q * (double)row[v];
+          }
+#pragma unroll
+          for (int v = 0; v < kSumGroup; ++v)
+            if (v < nf) dst[5 + f0 + v] += a[v];
+        }
+      }
+      __syncthreads();
+    }
+    if (s0 >= s1) __syncthreads();  // (no tile ran: the zeroing must still finish)
+    if (e0 >= p0 && e1 <= p1) {  // the whole event lies in this range: its means
+      for (int e = tid; e < KV; e += kSumThreads) {
+        const int j = e / V, v = e - j * V;
+        const double W = s_acc[j * V];
+        const int64_t r = (int64_t)b * K + j;
+        if (v == 0) wsum[r] = (float)W;
+        else if (v < 5) wcoords[r * 4 + (v - 1)] = W > 0.0 ? (float)(s_acc[e] / W) : 0.f;
+        else wfeats[r * F + (v - 5)] = W > 0.0 ? (float)(s_acc[e] / W) : 0.f;
+      }
+    } else {  // cut by a range boundary: slot 1 when it starts here, else slot 0
+      double* dst = partial + ((int64_t)blockIdx.x * 2 + (e0 >= p0 ? 1 : 0)) * KV;
+      for (int e = tid; e < KV; e += kSumThreads) dst[e] = s_acc[e];
     }
     __syncthreads();
-    int run = s_warp[warp] + x - sum;
-    for (int e = a; e < z; ++e) {
-      s_start[e] = run;
-      run += s_cnt[e];
-    }
-    if (tid == kSumThreads - 1) s_start[NB] = run;
-  }
-  __syncthreads();
-  for (int e = tid; e < NB; e += kSumThreads) s_cnt[e] = s_start[e];
-  __syncthreads();
-  for (int p = tid; p < n; p += kSumThreads) {
-    const int key = s_key[p];
-    if (key >= 0) s_perm[atomicAdd(s_cnt + key, 1)] = p;
-  }
-  __syncthreads();
-  // one item per (bucket, value): the bucket's points in sorted order
-  for (int it = tid; it < NB * V; it += kSumThreads) {
-    const int bk = it / V, v = it - bk * V;
-    const int a = s_start[bk], z = s_start[bk + 1];
-    if (a == z) continue;
-    double sum = 0.0;  // in sorted order, four values at a time
-    int m = a;
-    for (; m + 4 <= z; m += 4) {
-      double x[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        x[u] = tile_value(sc, sf, staged, coords, feats, F, charge_col, t0, s_perm[m + u], v);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) sum += x[u];
-    }
-    for (; m < z; ++m) sum += tile_value(sc, sf, staged, coords, feats, F, charge_col, t0, s_perm[m], v);
-    const int b = lo + bk / K, j = bk - (bk / K) * K;
-    atomicAdd(acc + (((int64_t)rep * B + b) * K + j) * V + v, sum);
   }
 }
 
-__global__ void __launch_bounds__(256) k_token_finalize(const double* __restrict__ acc, int reps, int F,
-                                                        int64_t rows, float* __restrict__ wsum,
-                                                        float* __restrict__ wcoords, float* __restrict__ wfeats) {
+// One CTA per range boundary c * chunk (c = 1 .. G-1).  An event cut by
+// nb boundaries gets nb CTAs, each taking a slice of its K (5 + F) values.
+// Per block of up to 256 values the CTA's threads split the ranges the
+// event spans into S consecutive groups, sum each group in range order, and
+// one thread per value adds the group sums in group order: a fixed order,
+// with the loads of all groups in flight together.
+__global__ void __launch_bounds__(256) k_token_finalize(const int64_t* __restrict__ offsets, int B, int64_t P,
+                                                        int K, int F, int64_t chunk, int G,
+                                                        const double* __restrict__ partial,
+                                                        float* __restrict__ wsum, float* __restrict__ wcoords,
+                                                        float* __restrict__ wfeats) {
+  __shared__ double s_w[256], s_x[256];
+  const int c = blockIdx.x + 1;
+  const int64_t p = (int64_t)c * chunk;
+  if (p >= P) return;
+  const int b = sum_first_event_after(offsets, 0, B - 1, p);
+  const int64_t e0 = offsets[b], e1 = offsets[b + 1];
+  if (!(e0 < p && p < e1) || e0 < 0 || e1 > P) return;  // no event is cut here (uniform)
+  const int cf = (int)(e0 / chunk);
+  const int cl = (int)min((int64_t)G - 1, (e1 - 1) / chunk);
+  const int nb = cl - cf;        // boundaries inside the event: one CTA each
+  const int slice = c - cf - 1;  // this CTA's share of the values
   const int V = 5 + F;
-  const int64_t n = rows * V;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
-    const int64_t r = e / V;
-    const int v = (int)(e - r * V);
-    double W = 0.0, x = 0.0;
-    for (int q = 0; q < reps; ++q) {  // replicas in order
-      W += acc[(int64_t)q * n + r * V];
-      x += acc[(int64_t)q * n + e];
+  const int KV = K * V;
+  const int R = cl - cf + 1;     // ranges the event spans
+  const int lo = (int)((int64_t)KV * slice / nb), hi = (int)((int64_t)KV * (slice + 1) / nb);
+  const int tid = threadIdx.x;
+  for (int v0 = lo; v0 < hi; v0 += 256) {
+    const int nv = min(256, hi - v0);
+    const int S = min(R, 256 / nv);      // range groups
+    const int per = (R + S - 1) / S;     // ranges per group
+    if (tid < nv * S) {
+      const int ev = tid % nv, grp = tid / nv;
+      const int e = v0 + ev, j = e / V;
+      const int r0 = cf + grp * per, r1 = min(cl + 1, r0 + per);
+      double W = 0.0, x = 0.0;
+#pragma unroll 4
+      for (int r = r0; r < r1; ++r) {
+        const double* src = partial + ((int64_t)r * 2 + (r == cf ? 1 : 0)) * KV;
+        W += src[j * V];
+        x += src[e];
+      }
+      s_w[tid] = W;
+      s_x[tid] = x;
     }
-    if (v == 0) wsum[r] = (float)W;
-    else if (v < 5) wcoords[r * 4 + (v - 1)] = W > 0.0 ? (float)(x / W) : 0.f;
-    else wfeats[r * F + (v - 5)] = W > 0.0 ? (float)(x / W) : 0.f;
+    __syncthreads();
+    if (tid < nv) {
+      const int e = v0 + tid, j = e / V, v = e - j * V;
+      double W = 0.0, x = 0.0;
+      for (int g = 0; g < S; ++g) {
+        W += s_w[g * nv + tid];
+        x += s_x[g * nv + tid];
+      }
+      const int64_t row = (int64_t)b * K + j;
+      if (v == 0) wsum[row] = (float)W;
+      else if (v < 5) wcoords[row * 4 + (v - 1)] = W > 0.0 ? (float)(x / W) : 0.f;
+      else wfeats[row * F + (v - 5)] = W > 0.0 ? (float)(x / W) : 0.f;
+    }
+    __syncthreads();
   }
+}
+
+// Shared memory of k_token_sums: the tile's coordinates, the accumulators,
+// the tile's charges, tokens and counting sort, and its feature rows.
+size_t token_sums_smem(int K, int F) {
+  return (size_t)K * (5 + F) * sizeof(double) + (size_t)kSumTile * (sizeof(float4) + sizeof(float) + 2 * sizeof(int)) +
+         3 * 256 * sizeof(int) + (F <= kSumGroup ? (size_t)kSumTile * F * sizeof(float) : 0);
 }
 
 }  // namespace
 
-int token_summary_replicas(int B, int K, int F) {
-  const int64_t one = (int64_t)B * K * (5 + F) * (int64_t)sizeof(double);
-  int64_t r = one > 0 ? kSumReplicaBudget / one : kSumMaxReplicas;
-  if (r > kSumMaxReplicas) r = kSumMaxReplicas;
-  return r < 1 ? 1 : (int)r;
+int token_summary_ctas(int K, int F) {
+  const int64_t per = 2ll * K * (5 + F) * (int64_t)sizeof(double);
+  int64_t g = per > 0 ? kSumPartialBudget / per : kSumMaxCtas;
+  if (g > kSumMaxCtas) g = kSumMaxCtas;
+  return g < 1 ? 1 : (int)g;
+}
+
+size_t token_summary_partial_bytes(int K, int F) {
+  return (size_t)token_summary_ctas(K, F) * 2 * K * (5 + F) * sizeof(double);
 }
 
 cudaError_t launch_token_summaries(const float* coords, const float* feats, int F, int charge_col,
                                    const int64_t* offsets, int B, int64_t P, int K, const int32_t* token_id,
-                                   double* acc, float* wsum, float* wcoords, float* wfeats, WsHeader* hdr,
+                                   double* partial, float* wsum, float* wcoords, float* wfeats, WsHeader* hdr,
                                    cudaStream_t s) {
-  const int64_t rows = (int64_t)B * K;
-  const int V = 5 + F;
-  const int reps = token_summary_replicas(B, K, F);
-  cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)reps * rows * V * sizeof(double), s);
+  int64_t G = (P + kSumMinPoints - 1) / kSumMinPoints;
+  if (G > token_summary_ctas(K, F)) G = token_summary_ctas(K, F);
+  const int64_t resident = (int64_t)device_info().sm_count * kSumCtasPerSm;  // one wave
+  if (G > resident) G = resident;
+  if (G < 1) G = 1;
+  const int64_t chunk = P > 0 ? (P + G - 1) / G : 1;
+  const size_t smem = token_sums_smem(K, F);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (P > 0) {
-    // stage the tile's rows in shared memory when they fit (F up to about 36)
-    const size_t rows_bytes = (size_t)kSumTile * (4 + F) * sizeof(float);
-    const int staged = rows_bytes <= (size_t)kSumStageBytes;
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-      if ((e = cudaFuncSetAttribute(k_token_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, kSumStageBytes)))
-        return e;
-      attr_set[dev] = true;
-    }
-    count_launch();
-    k_token_sums<<<(unsigned)((P + kSumTile - 1) / kSumTile), kSumThreads, staged ? rows_bytes : 0, s>>>(
-        coords, feats, F, charge_col, offsets, B, P, K, token_id, reps, staged, acc, hdr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const int most = (int)token_sums_smem(FPS_MAX_K, FPS_MAX_F);
+    if ((e = cudaFuncSetAttribute(k_token_sums, cudaFuncAttributeMaxDynamicSharedMemorySize, most))) return e;
+    attr_set[dev] = true;
   }
-  const DeviceInfo& di = device_info();
-  int64_t g = (rows * V + 255) / 256;
-  if (g > (int64_t)di.sm_count * 8) g = (int64_t)di.sm_count * 8;
-  if (g < 1) g = 1;
   count_launch();
-  k_token_finalize<<<(unsigned)g, 256, 0, s>>>(acc, reps, F, rows, wsum, wcoords, wfeats);
-  return cudaGetLastError();
+  k_token_sums<<<(unsigned)G, kSumThreads, smem, s>>>(reinterpret_cast<const float4*>(coords), feats, F, charge_col,
+                                                      offsets, B, P, K, token_id, chunk, wsum, wcoords, wfeats,
+                                                      partial, hdr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (G > 1) {
+    count_launch();
+    k_token_finalize<<<(unsigned)(G - 1), 256, 0, s>>>(offsets, B, P, K, F, chunk, (int)G, partial, wsum, wcoords,
+                                                      wfeats);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace fpstok

@@ -8,14 +8,16 @@ namespace fpstok {
 
 struct WsHeader;
 
-// Accumulator copies the summaries use for B events, K tokens, F features.
-int token_summary_replicas(int B, int K, int F);
+// CTAs (contiguous point ranges) the summaries use at most for K tokens and
+// F features, and the bytes of their float64 partial sums (2 K (5 + F) each).
+int token_summary_ctas(int K, int F);
+size_t token_summary_partial_bytes(int K, int F);
 
 // wsum [B,K], wcoords [B,K,4], wfeats [B,K,F] from the Voronoi labels;
-// acc: float64 [replicas, B, K, 5 + F] scratch (cleared here).
+// partial: token_summary_partial_bytes(K, F) of scratch (no clearing needed).
 cudaError_t launch_token_summaries(const float* coords, const float* feats, int F, int charge_col,
                                    const int64_t* offsets, int B, int64_t P, int K, const int32_t* token_id,
-                                   double* acc, float* wsum, float* wcoords, float* wfeats, WsHeader* hdr,
+                                   double* partial, float* wsum, float* wcoords, float* wfeats, WsHeader* hdr,
                                    cudaStream_t s);
 
 }  // namespace fpstok

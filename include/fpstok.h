@@ -303,9 +303,10 @@ int fps_random_starts(const int64_t *offsets, int B, uint64_t seed, uint32_t str
  * Sums in float64 (in no fixed order), each output rounded once to float32;
  * the means are 0 for an empty cell or wsum <= 0.  Token ids outside -1..K-1
  * and offsets that do not cover the points are skipped and reported by
- * fps_device_status().  Workspace: the size below, 256-byte aligned: up to
- * 16 copies of a B * K * (5 + F) float64 accumulator (as many as fit in
- * 32 MiB, at least one) and a status word.
+ * fps_device_status().  Workspace: the size below (it does not depend on B),
+ * 256-byte aligned: a status word and the float64 partial sums of the events
+ * cut by the boundaries of the per-CTA point ranges, 2 * K * (5 + F) values
+ * for each of up to 512 ranges (as many as fit in 32 MiB, at least one).
  */
 size_t fps_token_summaries_workspace_bytes(int B, int K, int F);
 int fps_token_summaries(const float *coords, const float *feats, int F, int charge_col,
