@@ -26,6 +26,7 @@ constexpr int kBwdTile = kBwdThreads * kBwdPts;  // points per block
 constexpr int kKnnBwdThreads = 512;
 constexpr int kFeatGroup = 8;  // features summed together per thread in the kNN scatter
 constexpr int64_t kKnnBwdSmemBytes = 104 * 1024;  // shares and per-point row masks of the kNN scatter
+constexpr int kBwdRowGroup = 16;  // rows of one event per warp in the kNN scatter's second phase
 
 // Largest b in [lo, hi] with offsets[b] <= i (offsets non-decreasing), i.e.
 // the event holding point i when i < offsets[hi + 1].
@@ -145,8 +146,9 @@ __device__ __forceinline__ bool knn_event_local(int64_t off, int64_t n, int cap_
 // rows takes -- and store the sums (plain stores: only this CTA writes these
 // points of sums[]).  Entries that name a point outside their event, or a
 // point already marked in the same row, are added to extra[] with float64
-// atomics.  Phase 2, a warp per row over the whole grid: the rows of events
-// whose masks do not fit in shared memory add all their entries to extra[].
+// atomics.  Phase 2, a warp per 16 rows of one event over the whole grid:
+// the rows of events whose masks do not fit in shared memory add all their
+// entries to extra[].
 // The gradient is (float)(sums + extra); extra is 0 when every row names
 // only its own event's points, once each, and the events fit, and then the
 // result is exactly the sequential row-order sum.  Entry e of the event's
@@ -224,25 +226,31 @@ __global__ void __launch_bounds__(kKnnBwdThreads, 2) k_pool_bwd_knn_event(
     }
     __syncthreads();
   }
-  // phase 2: rows of the events phase 1 skipped, a warp per row
+  // phase 2: rows of the events phase 1 skipped, a warp per group of
+  // kBwdRowGroup rows of one event (one locality check per group)
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t r = gw; r < (int64_t)B * K; r += nw) {
-    const int b = (int)(r / K);
+  const int groups = (K + kBwdRowGroup - 1) / kBwdRowGroup;
+  for (int64_t it = gw; it < (int64_t)B * groups; it += nw) {
+    const int b = (int)(it / groups);
+    const int j0 = (int)(it - (int64_t)b * groups) * kBwdRowGroup;
     const int64_t off = offsets[b];
     if (knn_event_local(off, offsets[b + 1] - off, cap_n, P)) continue;  // warp-uniform
-    const int c = counts[r];
-    if (c <= 0) continue;
-    const float* g = grad_pooled + r * F;
-    for (int e = lane; e < k; e += 32) {
-      const int v = knn_idx[r * k + e];
-      if (v >= P) record_error(hdr, kDevBadToken);
-      if (v < 0 || v >= P) continue;
-      double* dst = extra + (int64_t)v * F;
-      for (int f = 0; f < F; ++f) {
-        const double sh = (double)__ldg(g + f) / (double)c;
-        if (sh != 0.0) atomicAdd(dst + f, sh);
+    for (int j = j0; j < min(K, j0 + kBwdRowGroup); ++j) {
+      const int64_t r = (int64_t)b * K + j;
+      const int c = counts[r];
+      if (c <= 0) continue;
+      const float* g = grad_pooled + r * F;
+      for (int e = lane; e < k; e += 32) {
+        const int v = knn_idx[r * k + e];
+        if (v >= P) record_error(hdr, kDevBadToken);
+        if (v < 0 || v >= P) continue;
+        double* dst = extra + (int64_t)v * F;
+        for (int f = 0; f < F; ++f) {
+          const double sh = (double)__ldg(g + f) / (double)c;
+          if (sh != 0.0) atomicAdd(dst + f, sh);
+        }
       }
     }
   }
