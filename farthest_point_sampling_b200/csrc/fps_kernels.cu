@@ -98,7 +98,7 @@ constexpr int kWarpPtBytes = (int)sizeof(WarpPt);
 constexpr int kWarpListInts = FPS_MAX_K_DEV;  // chosen local indices, one per step
 // Shared memory of one warp: the event copy and the list, then room for the
 // pooling's staged feature rows (the whole region is reused by it).
-constexpr int kWarpRegionBytes = 12288;
+constexpr int kWarpRegionBytes = 15360;
 static_assert(64 * kWarpPairs * kWarpPtBytes + kWarpListInts * 4 <= kWarpRegionBytes, "event copy and list fit");
 static_assert(8 * FPS_MAX_K_DEV + 4 * kWarpCap <= kWarpRegionBytes, "one staged feature per pass fits");
 
@@ -248,15 +248,39 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
   }
   if (po.feats) {
     // Token means.  Every point's rank inside its token (one shared atomic
-    // each), the token starts by a scan of the counts, then per pass of at
-    // most 8 features: the lanes copy their points' rows into shared memory
-    // in token order (independent loads, all in flight), and lane t sums
-    // token t's contiguous rows in float64.
+    // each) and the token starts by a scan of the counts.  When the event's
+    // whole feature block fits beside them, it is copied into shared memory
+    // by asynchronous copies (16-byte pieces, in flight during the sort), and
+    // lane t sums token t's rows, found through the sorted point list, in
+    // float64.  Otherwise, per pass of at most 8 features, the lanes copy
+    // their points' rows into shared memory in token order and lane t sums
+    // token t's contiguous rows.
     const int F = po.F;
     __syncwarp();
-    int* cnt = reinterpret_cast<int*>(s_pts);  // [K] counts, then [K] starts, then the staged rows
+    int* cnt = reinterpret_cast<int*>(s_pts);  // [K] counts, then [K] starts, then the rest
     int* start = cnt + K;
-    float* sf = reinterpret_cast<float*>(start + K);
+    const float* fe = po.feats + off * F;
+    const int pad = (int)((reinterpret_cast<uintptr_t>(fe) >> 2) & 3);  // floats before a 16-byte boundary
+    const int head = (4 - pad) & 3;
+    const size_t list_bytes = ((size_t)(2 * K + n) * 4 + 15) & ~(size_t)15;
+    const bool whole = list_bytes + (size_t)(pad + n * F) * 4 <= (size_t)kWarpRegionBytes;
+    int* perm = start + K;                                                 // [n] points in token order
+    float* sfb = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(cnt) + list_bytes);
+    if (whole) {  // element e of the block lands at sfb[pad + e]: 16-byte pieces stay aligned on both sides
+      const int total = n * F;
+      const int h = min(head, total);
+      const uint32_t s0 = (uint32_t)__cvta_generic_to_shared(sfb) + 4u * (uint32_t)pad;
+      if (lane < h)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s0 + 4u * lane), "l"(fe + lane) : "memory");
+      const int nb = (total - h) >> 2;
+      for (int k = lane; k < nb; k += 32)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s0 + 4u * (uint32_t)(h + 4 * k)),
+                     "l"(fe + h + 4 * k)
+                     : "memory");
+      for (int e = h + 4 * nb + lane; e < total; e += 32)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s0 + 4u * (uint32_t)e), "l"(fe + e) : "memory");
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
     for (int j = lane; j < K; j += 32) cnt[j] = 0;
     __syncwarp();
     int pos[2 * NP];
@@ -268,41 +292,71 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
 #pragma unroll
     for (int j = 0; j < 2 * NP; ++j)
       if (j * 32 + lane < n) pos[j] += start[lab[j]];
-    const int fcap = (kWarpRegionBytes - 8 * K) / (4 * n);  // features one pass can stage (>= 1)
-    const int FC = min(min(F, 8), fcap);
-    const float* fe = po.feats + off * F;
-    for (int f0 = 0; f0 < F; f0 += FC) {
-      const int fc = min(FC, F - f0);
+    if (whole) {
 #pragma unroll
-      for (int j = 0; j < 2 * NP; ++j) {
-        const int i = j * 32 + lane;
-        if (i < n) {
-          const float* row = fe + (int64_t)i * F + f0;
-          float* dst = sf + pos[j] * fc;
-#pragma unroll
-          for (int f = 0; f < 8; ++f)
-            if (f < fc) dst[f] = __ldg(row + f);
-        }
-      }
+      for (int j = 0; j < 2 * NP; ++j)
+        if (j * 32 + lane < n) perm[pos[j]] = j * 32 + lane;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
       __syncwarp();
+      const float* rows = sfb + pad;
       for (int t = lane; t < K; t += 32) {
         const int c2 = cnt[t];
-        const float* src = sf + start[t] * fc;
-        double a[8];
+        const int* pj = perm + start[t];
+        float* prow = po.pooled + (b * K + t) * F;
+        for (int f0 = 0; f0 < F; f0 += 8) {
+          double a[8];
 #pragma unroll
-        for (int f = 0; f < 8; ++f) a[f] = 0.0;
-        for (int q = 0; q < c2; ++q, src += fc) {
+          for (int f = 0; f < 8; ++f) a[f] = 0.0;
+          for (int q = 0; q < c2; ++q) {
+            const float* src = rows + pj[q] * F + f0;
+#pragma unroll
+            for (int f = 0; f < 8; ++f)
+              if (f0 + f < F) a[f] += (double)src[f];
+          }
 #pragma unroll
           for (int f = 0; f < 8; ++f)
-            if (f < fc) a[f] += (double)src[f];
+            if (f0 + f < F) prow[f0 + f] = c2 ? (float)(a[f] / (double)c2) : 0.f;
         }
-        float* prow = po.pooled + (b * K + t) * F + f0;
-#pragma unroll
-        for (int f = 0; f < 8; ++f)
-          if (f < fc) prow[f] = c2 ? (float)(a[f] / (double)c2) : 0.f;
-        if (f0 == 0) po.counts[b * K + t] = c2;
+        po.counts[b * K + t] = c2;
       }
       __syncwarp();
+    } else {
+      float* sf = reinterpret_cast<float*>(start + K);
+      const int fcap = (kWarpRegionBytes - 8 * K) / (4 * n);  // features one pass can stage (>= 1)
+      const int FC = min(min(F, 8), fcap);
+      for (int f0 = 0; f0 < F; f0 += FC) {
+        const int fc = min(FC, F - f0);
+#pragma unroll
+        for (int j = 0; j < 2 * NP; ++j) {
+          const int i = j * 32 + lane;
+          if (i < n) {
+            const float* row = fe + (int64_t)i * F + f0;
+            float* dst = sf + pos[j] * fc;
+#pragma unroll
+            for (int f = 0; f < 8; ++f)
+              if (f < fc) dst[f] = __ldg(row + f);
+          }
+        }
+        __syncwarp();
+        for (int t = lane; t < K; t += 32) {
+          const int c2 = cnt[t];
+          const float* src = sf + start[t] * fc;
+          double a[8];
+#pragma unroll
+          for (int f = 0; f < 8; ++f) a[f] = 0.0;
+          for (int q = 0; q < c2; ++q, src += fc) {
+#pragma unroll
+            for (int f = 0; f < 8; ++f)
+              if (f < fc) a[f] += (double)src[f];
+          }
+          float* prow = po.pooled + (b * K + t) * F + f0;
+#pragma unroll
+          for (int f = 0; f < 8; ++f)
+            if (f < fc) prow[f] = c2 ? (float)(a[f] / (double)c2) : 0.f;
+          if (f0 == 0) po.counts[b * K + t] = c2;
+        }
+        __syncwarp();
+      }
     }
   }
   __syncwarp();  // the next event overwrites this warp's copy
