@@ -244,7 +244,24 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
   // the warps write the pooling items cooperatively.
   __shared__ unsigned long long s_tmp64[32];
   int c_fps = 0, c_events = 0, c_slots = 0, c_chunks = 0;
-  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+  // Without Lloyd, assignment passes or any event pooled outside its FPS
+  // kernel, nothing reads the slots and items: the lists alone are written.
+  bool need_items = need_passes != 0;
+  for (int q = 0; q < kNumSchedules; ++q)
+    if (cnt[q] > 0 && !((fused_pool >> q) & 1)) need_items = true;
+  if (!need_items) {
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+      if (cls_of(b) != kClsFps) continue;
+      const int n = size_of(b);
+      const int q = schedule_of(n);
+      int* list = q == 0 ? ws.list_warp
+                         : (q == 1 ? ws.list_cta
+                                   : (q == 2 ? ws.list_cta_smem : (q == 3 ? ws.list_cluster8 : ws.list_cluster16)));
+      list[atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1)] = b;
+    }
+    c_fps = n_fps;
+  }
+  for (int b0 = 0; need_items && b0 < B; b0 += blockDim.x) {
     const int b = b0 + threadIdx.x;
     const int cls = b < B ? cls_of(b) : kClsSkip;
     int n = 0;
