@@ -1,6 +1,7 @@
 // C ABI of the fpstok tokenizer (declared in include/fpstok.h): argument
 // checks, workspace carving and the launch sequence.  No allocation, no
 // synchronisation (except fps_device_status, which exists to read back).
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <cmath>
@@ -380,6 +381,12 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
   for (int c = 0; c < nc; ++c) {  // each slice: rebase, tokenize, renumber on the caller's stream; copy out
     const int b0 = bnd[c], b1 = bnd[c + 1], bc = b1 - b0;
     const int64_t p0 = offsets[b0], pc = offsets[b1] - p0;
+    // the sizes are on the host: the slice's largest event is an exact size
+    // hint, so schedules and the pool kernel with nothing to do are not launched
+    fps_opts oc = *opts;
+    int64_t nmax = 0;
+    for (int b = b0; b < b1; ++b) nmax = std::max(nmax, offsets[b + 1] - offsets[b]);
+    if (nmax > 0 && (oc.max_event_hint <= 0 || nmax < oc.max_event_hint)) oc.max_event_hint = (int)nmax;
     if ((e = cudaStreamWaitEvent(s, hp->in_done[c], 0))) return from_cuda(e);
     int64_t* off_c = reinterpret_cast<int64_t*>(w + h.offsets) + b0 + c;
     if ((e = launch_rebase_offsets(off_c, bc + 1, p0, s))) return from_cuda(e);
@@ -387,7 +394,7 @@ int fps_tokenize_host(const float* coords, const float* feats, int F, const int6
     int32_t* knn_c = k ? reinterpret_cast<int32_t*>(w + h.knn) + (int64_t)b0 * K * k : nullptr;
     rc = fps_tokenize(reinterpret_cast<const float*>(w + h.coords) + p0 * 4,
                       reinterpret_cast<const float*>(w + h.feats) + p0 * F, F, off_c, bc, pc,
-                      start_local ? reinterpret_cast<const int32_t*>(w + h.start) + b0 : nullptr, opts, cidx_c,
+                      start_local ? reinterpret_cast<const int32_t*>(w + h.start) + b0 : nullptr, &oc, cidx_c,
                       token_id ? reinterpret_cast<int32_t*>(w + h.tok) + p0 : nullptr, knn_c,
                       reinterpret_cast<float*>(w + h.cents) + (int64_t)b0 * K * 4,
                       reinterpret_cast<float*>(w + h.pooled) + (int64_t)b0 * K * F,
