@@ -55,6 +55,22 @@ def test_edge_sizes(K):
     compare(b, run_gpu(b))
 
 
+@pytest.mark.parametrize("F", [1, 7, 12, 40, 64])
+def test_fused_pooling_feature_counts(F):
+    """The pooling the warp and register-CTA schedules fuse into FPS, across
+    feature counts: with few features the warp copies the event's whole
+    feature block into shared memory (447 points x 7 features still fit, 448
+    do not), with more it stages a few features per pass; the register CTA
+    pools in place only while its feature rows fit, else the pool kernel
+    takes its events.  Event sizes around the warp and CTA capacities and
+    around 16-byte boundaries of the feature block."""
+    sizes = [129, 130, 131, 250, 383, 446, 447, 448, 449, 900, 2559, 2560, 5, 0, 300, 301]
+    b = workloads.random_batch(900 + F, sizes, 128, F=F)
+    compare(b, run_gpu(b))
+    b = workloads.random_batch(950 + F, [447, 448] * 40 + [200] * 40, 128, F=F)
+    compare(b, run_gpu(b))
+
+
 @pytest.mark.parametrize("kind", ["dup", "grid", "allsame"])
 def test_ties_and_duplicates(kind):
     sizes = [40, 200, 700, 3000, 15000]
