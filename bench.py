@@ -185,10 +185,16 @@ class ClockSampler:
 # ------------------------------------------------------------------ profiles (ncu traffic)
 
 def kernel_source_hash():
+    """Hash of the FPS kernel sources with comments and blank lines removed
+    (a comment edit leaves the compiled kernels, and their traffic, as they
+    were)."""
     h = hashlib.sha256()
     for name in ("fps_kernels.cu", "common.cuh", "internal.h"):
-        with open(os.path.join(ROOT, "farthest_point_sampling_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "farthest_point_sampling_b200", "csrc", name)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

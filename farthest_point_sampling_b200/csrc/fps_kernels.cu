@@ -27,12 +27,16 @@
 //                            warp-class events when there are few events.
 //   CTA-smem    N <= 12288   one 256-thread CTA per event, points in shared
 //                            memory as packed f32x2 pairs.
-//   cluster-8   N <= 98304   an 8-CTA cluster per event (same layout); every
-//   cluster-16  N <= 196608  warp posts its winner into every CTA's shared
-//                            memory over DSMEM; one barrier.cluster per step.
+//   cluster-8   N <= 98304   an 8-CTA cluster per event (same layout): warp 0
+//   cluster-16  N <= 196608  of every CTA posts the CTA's winner into a slot
+//                            of every CTA's shared memory with st.async, which
+//                            signals that CTA's mbarrier; a bounded wait on it,
+//                            no cluster barrier per step.
 // Each event runs a step loop compiled for its exact number of point pairs
-// (one dispatch per event), and work items are claimed from a counter in
-// decreasing size order so that the longest chains start first.
+// (one dispatch per event; in the warp schedule an out-of-line function per
+// pair count), and work items are claimed from a counter in decreasing size
+// order so that the longest chains start first.  The warp and register-CTA
+// schedules also pool their events' token means in place.
 #include <cooperative_groups.h>
 
 #include <mutex>
