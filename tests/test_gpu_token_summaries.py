@@ -51,13 +51,25 @@ def test_summaries_large_events():
 
 @pytest.mark.parametrize("F", [1, 6, 7])
 def test_summaries_many_tiny_events(F):
-    """Events of 0-6 points: most tiles span more events than the bucket
-    table holds and add point by point."""
+    """Events of 0-6 points: every CTA's range holds hundreds of whole events
+    (summed one event at a time and written directly), and the events cut by
+    a range boundary are finished from the partial sums."""
     rng = np.random.default_rng(111 + F)
     sizes = rng.integers(0, 7, 5000)
     b = workloads.random_batch(112 + F, sizes, 4, F=F)
     tok = np.concatenate([rng.integers(-1, 4, int(n)) for n in sizes]).astype(np.int32)
     _check(b, 4, tok, 0 if F > 1 else -1)
+
+
+@pytest.mark.parametrize("F", [9, 12, 64])
+def test_summaries_wide_rows(F):
+    """More than 8 features: the rows are read from global memory per value
+    group instead of being staged, in groups of 8 features per thread."""
+    rng = np.random.default_rng(120 + F)
+    b = workloads.random_batch(121 + F, [0, 3, 700, 1024, 1025, 5000, 20000, 1], 16, F=F)
+    tok = np.concatenate([rng.integers(-1, 16, int(n)) for n in b.sizes()]).astype(np.int32)
+    _check(b, 16, tok, 0)
+    _check(b, 16, tok, -1)
 
 
 def test_summaries_mixed_sizes():
