@@ -176,19 +176,19 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
     Y[p] = pack2(a.y, b.y);
     Z[p] = pack2(a.z, b.z);
     T[p] = pack2(a.w, b.w);
-    dist[2 * p] = i0 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-    dist[2 * p + 1] = i1 < n ? __int_as_float(0x7f800000) : kEmptySlot;
-    lab[2 * p] = 0;
-    lab[2 * p + 1] = 0;
     if (i0 >= n) empty |= 1u << (2 * p);
     if (i1 >= n) empty |= 1u << (2 * p + 1);
   }
-  __syncwarp();
-  // steps 0 .. K-2: update with c_s, then the next centroid by arg-max.  The
-  // loop leaves early only when the maximum is 0 (every unselected point
-  // duplicates a chosen one); the rest of the steps then run below.
-  int s = 0;
-  for (; s < K - 1; ++s) {
+  auto reset = [&]() {
+#pragma unroll
+    for (int j = 0; j < 2 * NP; ++j) {
+      dist[j] = (empty >> j) & 1u ? kEmptySlot : __int_as_float(0x7f800000);
+      lab[j] = 0;
+    }
+  };
+  // One step: update with c_s = c, then c = the arg-max (lowest index among
+  // equal maxima); returns the maximum's key.
+  auto step = [&](int s) -> int {
     if (lane == 0) s_c[s] = c;
     const Cent2 C = warp_pt_cent<SCALED>(s_pts[c], w);
     float pm[NP];
@@ -199,9 +199,26 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
       pm[p] = fmaxf(dist[2 * p], dist[2 * p + 1]);
     }
     const int M = __reduce_max_sync(kFull, fkey(lane_max<NP>(pm)));
-    if (M == 0) break;
     const int slot = lane_first_slot<NP>(pm, dist, M);  // lowest slot of this lane holding the maximum
     c = (int)__reduce_min_sync(kFull, slot < 0 ? 0xffffffffu : (unsigned)(slot * 32 + lane));
+    return M;
+  };
+  reset();
+  __syncwarp();
+  // steps 0 .. K-2 without an exit test: a zero maximum (every unselected
+  // point duplicates a chosen one, so the arg-max may return a chosen point)
+  // is only recorded, and such an event is run again from the start below,
+  // leaving at its first zero maximum.  The chosen index stays a point of the
+  // event either way (empty slots never hold the maximum).
+  const int c_first = c;
+  bool zero = false;
+  for (int s = 0; s < K - 1; ++s) zero |= step(s) == 0;
+  int s = K - 1;
+  if (zero) {
+    reset();
+    c = c_first;
+    for (s = 0; s < K - 1; ++s)
+      if (step(s) == 0) break;
   }
   // only duplicates of chosen points remain: each next centroid is the
   // lowest-index unselected point (steps s + 1 .. K - 2; step s's update is done)
@@ -317,9 +334,12 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
             for (int f = 0; f < 8; ++f)
               if (f0 + f < F) a[f] += (double)src[f];
           }
+          // the mean as the sum times the float64 reciprocal of the count
+          // (within an ulp of the float64 quotient)
+          const double inv = c2 ? 1.0 / (double)c2 : 0.0;
 #pragma unroll
           for (int f = 0; f < 8; ++f)
-            if (f0 + f < F) prow[f0 + f] = c2 ? (float)(a[f] / (double)c2) : 0.f;
+            if (f0 + f < F) prow[f0 + f] = (float)(a[f] * inv);
         }
         po.counts[b * K + t] = c2;
       }
@@ -354,9 +374,10 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
               if (f < fc) a[f] += (double)src[f];
           }
           float* prow = po.pooled + (b * K + t) * F + f0;
+          const double inv = c2 ? 1.0 / (double)c2 : 0.0;
 #pragma unroll
           for (int f = 0; f < 8; ++f)
-            if (f < fc) prow[f] = c2 ? (float)(a[f] / (double)c2) : 0.f;
+            if (f < fc) prow[f] = (float)(a[f] * inv);
           if (f0 == 0) po.counts[b * K + t] = c2;
         }
         __syncwarp();

@@ -86,6 +86,22 @@ def test_ties_and_duplicates(kind):
     compare(b, run_gpu(b))
 
 
+@pytest.mark.parametrize("force", [-1, 0])
+def test_warp_events_with_few_distinct_points(force):
+    """Warp-schedule events with fewer distinct points than K: the arg-max
+    reaches a zero maximum, after which the remaining centroids are the
+    lowest-index unselected points.  The warp loop runs without an exit test
+    and runs such an event again with one; every third event is one point
+    repeated.  300 events, so that the automatic schedule is the warp one."""
+    rng = np.random.default_rng(31)
+    sizes = [int(n) for n in rng.integers(129, 449, 300)]
+    b = workloads.random_batch(32, sizes, 128, dup_frac=0.7)
+    for e in range(0, b.B, 3):
+        o0, o1 = b.offsets[e], b.offsets[e + 1]
+        b.coords[o0:o1] = b.coords[o0]
+    compare(b, run_gpu(b, force_schedule=force))
+
+
 @pytest.mark.parametrize("force", [0, 1, 2, 3, 4])
 def test_forced_schedules_agree(force):
     sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000, 98304, 98305]
