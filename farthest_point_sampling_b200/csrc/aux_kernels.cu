@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
                                                int K, const int32_t* __restrict__ start_local,
                                                int force, int chunk_all, int fused_pool, int latency_events,
                                                int mid_cluster_events, int need_passes, Workspace ws) {
+  // a kernel launched after this one as a programmatic dependent may start
+  // now; it waits for this kernel's completion before it reads the lists
+  asm volatile("griddepcontrol.launch_dependents;");
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
   __shared__ int n_fps, n_mid;

@@ -403,6 +403,9 @@ __global__ void __launch_bounds__(128, FPS_WARP_MIN_BLOCKS) k_fps_warp(const flo
                                                      int scaled) {
   constexpr int kMaxPairs = NPMAX;
   static_assert(2 * NPMAX <= 32, "selected-slot mask is 32 bits");
+  // Launched as a programmatic dependent of the binning kernel: the CTAs
+  // start while it runs and wait here for its lists (a no-op otherwise).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) unsigned char s_warp_all[];
   const int lane = threadIdx.x & 31;
   unsigned char* mine = s_warp_all + (size_t)(threadIdx.x >> 5) * kWarpRegionBytes;
@@ -1174,6 +1177,8 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
   }
   // at most one event per SM: every warp-class event runs on the CTA schedule
   if (f < 0 && maybe_few) run[0] = false;
+  bool warp_only = run[0];
+  for (int q = 1; q < kNumSchedules; ++q) warp_only = warp_only && !run[q];
 
 
   const PoolOut none = {nullptr, 0, nullptr, nullptr};
@@ -1186,18 +1191,32 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
   if ((e = cudaEventRecord(ctx.fork, s))) return e;
   for (int q = 0; q < kNumSchedules; ++q) {
     if (!run[q]) continue;
-    cudaStream_t hs = ctx.helper[q];
-    if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
+    // When the warp schedule is the only FPS schedule, it follows the
+    // binning kernel on the caller's stream as a programmatic dependent
+    // launch (its CTAs are placed while the binning runs); otherwise every
+    // schedule runs on its own stream, so that no schedule's CTAs take the
+    // SMs ahead of another's longest events.
+    const bool chained = q == 0 && warp_only;
+    cudaStream_t hs = chained ? s : ctx.helper[q];
+    if (!chained && (e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
     mark(1 + q, 0, hs);
     switch (q) {
       case 0: {
         const int blocks = di.sm_count * (di.warp_blocks_per_sm > 0 ? di.warp_blocks_per_sm : 1);
         count_launch();
-        k_fps_warp<kWarpPairs><<<blocks, kWarpBlock, kWarpSmem, hs>>>(pb.coords, pb.offsets, pb.start_local,
-                                                                      ws.list_warp, ws.hdr, pb.K, pb.centroid_idx,
-                                                                      pb.token_id, pb.centroids, po_warp, pb.w,
-                                                                      pb.scaled);
-        e = cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(kWarpBlock);
+        cfg.dynamicSmemBytes = kWarpSmem;
+        cfg.stream = hs;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = chained ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, k_fps_warp<kWarpPairs>, pb.coords, pb.offsets, pb.start_local,
+                               (const int*)ws.list_warp, ws.hdr, pb.K, pb.centroid_idx, pb.token_id, pb.centroids,
+                               po_warp, pb.w, pb.scaled);
         break;
       }
       case 1:
@@ -1225,7 +1244,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
                         pb.pooled, pb.counts, &ws, ws.hdr, hs, pb.w, pb.scaled, q)))
       return e;
     mark(1 + q, 1, hs);
-    if ((e = cudaEventRecord(ctx.join[q], hs))) return e;
+    if (!chained && (e = cudaEventRecord(ctx.join[q], hs))) return e;
   }
   {  // passthrough rows and accumulator clearing overlap the FPS kernels (enqueued last, lowest priority)
     cudaStream_t hs = ctx.helper[kHelpers - 1];
@@ -1237,7 +1256,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;
   }
   for (int q = 0; q < kNumSchedules; ++q)
-    if (run[q] && (e = cudaStreamWaitEvent(s, ctx.join[q], 0))) return e;
+    if (run[q] && !(q == 0 && warp_only) && (e = cudaStreamWaitEvent(s, ctx.join[q], 0))) return e;
   return cudaStreamWaitEvent(s, ctx.join[kHelpers - 1], 0);
 }
 
