@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
   asm volatile("griddepcontrol.launch_dependents;");
   __shared__ int cnt[kNumLists];
   __shared__ int hist[kNumSchedules][kBins];
-  __shared__ int n_fps, n_mid;
+  __shared__ int n_fps, n_mid, n_warp;
   __shared__ int s_n[kBinCache];              // event sizes (-1 for events that are neither FPS nor passthrough)
   __shared__ signed char s_cls[kBinCache];    // event classes, so later passes need no global re-reads
   for (int i = threadIdx.x; i < kNumSchedules * kBins; i += blockDim.x) (&hist[0][0])[i] = 0;
@@ -132,12 +132,20 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
     ws.hdr->detail = 0;
     n_fps = 0;
     n_mid = 0;
+    n_warp = 0;
   }
   __syncthreads();
   // pass 1: classify and count FPS events (four events per thread in flight;
-  // counts kept per thread and added once per warp after the loop)
+  // counts kept per thread and added once per warp after the loop), and
+  // histogram their sizes under the schedule they get when neither the
+  // few-events nor the few-mid-size rule applies (pass 2 redoes it if one does)
   constexpr int U = 4;
-  int my_fps = 0, my_mid = 0;
+  int my_fps = 0, my_mid = 0, my_warp = 0;
+  auto plain_schedule_of = [&](int n) {
+    int q = n <= kWarpCap ? 0 : (n <= kCtaCap ? 1 : (n <= kCtaSmemCap ? 2 : (n <= kCluster8Cap ? 3 : 4)));
+    if (force > q) q = force > 4 ? 4 : force;
+    return q;
+  };
   for (int b0 = threadIdx.x; b0 < B; b0 += U * blockDim.x) {
     int64_t o0[U], o1[U];
     int st[U];
@@ -175,6 +183,9 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
           } else {
             ++my_fps;
             if (n > kCtaCap && n <= kCtaSmemCap) ++my_mid;
+            const int q = plain_schedule_of((int)n);
+            if (q == 0) ++my_warp;
+            atomicAdd(&hist[q][min((int)n >> sched_shift(q), kBins - 1)], 1);
           }
         }
       }
@@ -187,9 +198,11 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
   }
   my_fps = __reduce_add_sync(kFull, my_fps);
   my_mid = __reduce_add_sync(kFull, my_mid);
+  my_warp = __reduce_add_sync(kFull, my_warp);
   if ((threadIdx.x & 31) == 0) {
     if (my_fps) atomicAdd(&n_fps, my_fps);
     if (my_mid) atomicAdd(&n_mid, my_mid);
+    if (my_warp) atomicAdd(&n_warp, my_warp);
   }
   __syncthreads();
   const bool few = n_fps <= latency_events;
@@ -206,14 +219,18 @@ __global__ void __launch_bounds__(kBinThreads) k_bin(const int64_t* __restrict__
   };
   auto size_of = [&](int b) { return b < kBinCache ? s_n[b] : (int)(offsets[b + 1] - offsets[b]); };
   auto cls_of = [&](int b) { return b < kBinCache ? (int)s_cls[b] : ws.cls[b]; };
-  // pass 2: size histogram per schedule
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    if (cls_of(b) != kClsFps) continue;
-    const int n = size_of(b);
-    const int q = schedule_of(n);
-    atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1);
+  // pass 2 (only when a rule above moves events): size histogram per schedule
+  if ((few && n_warp > 0) || (few_mid && n_mid > 0)) {
+    for (int i = threadIdx.x; i < kNumSchedules * kBins; i += blockDim.x) (&hist[0][0])[i] = 0;
+    __syncthreads();
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+      if (cls_of(b) != kClsFps) continue;
+      const int n = size_of(b);
+      const int q = schedule_of(n);
+      atomicAdd(&hist[q][min(n >> sched_shift(q), kBins - 1)], 1);
+    }
+    __syncthreads();
   }
-  __syncthreads();
   // exclusive scan from the largest bucket down (one warp per schedule, 8
   // buckets per lane): list position of each bucket
   if (threadIdx.x < 32 * kNumSchedules) {
