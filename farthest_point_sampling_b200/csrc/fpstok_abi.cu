@@ -606,14 +606,15 @@ int segment_pool_backward(const float* grad_pooled, int F, const int64_t* offset
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FPS_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* hdr = static_cast<WsHeader*>(workspace);
-  cudaError_t e;
-  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
   char* scratch = static_cast<char*>(workspace) + align256(sizeof(WsHeader));
   if (mode == FPS_ASSIGN_KNN) {
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
     double* acc = reinterpret_cast<double*>(scratch);
     return from_cuda(
         launch_pool_bwd_knn(grad_pooled, F, offsets, B, K, k, knn_idx, counts, P, acc, grad_feats, hdr, s));
   }
+  // the quotient kernel resets the status word (Voronoi: B > 0, so it runs)
   return from_cuda(launch_pool_bwd_voronoi(grad_pooled, F, offsets, B, P, K, token_id, counts,
                                            reinterpret_cast<float*>(scratch), grad_feats, hdr, s));
 }
@@ -664,9 +665,7 @@ int fps_pack_tokens(const float* src, int D, const int64_t* offsets, const int32
   if (!workspace || workspace_bytes < fps_pack_workspace_bytes() || !aligned(workspace, 256))
     return FPS_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  WsHeader* hdr = static_cast<WsHeader*>(workspace);
-  cudaError_t e;
-  if ((e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s))) return from_cuda(e);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);  // its status word is reset by the scan kernel
   return from_cuda(launch_pack_tokens(src, D, offsets, valid_tokens, B, K, dst, doc_id, tok_offsets, hdr, s));
 }
 

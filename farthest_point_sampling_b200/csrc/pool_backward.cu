@@ -41,10 +41,17 @@ __device__ __forceinline__ int event_of(const int64_t* __restrict__ offsets, int
 
 // quot[r, f] = grad_pooled[r, f] / counts[r] as the float64 quotient rounded
 // once to float32, 0 for an empty row: the division happens once per
-// (token, feature), and the per-point pass only gathers.
+// (token, feature), and the per-point pass only gathers.  With hdr, thread 0
+// first resets the call's status word; the gather, its programmatic
+// dependent, may start at once and waits for this kernel before its checks.
 __global__ void __launch_bounds__(256) k_pool_bwd_quot(const float* __restrict__ grad_pooled, int F, int64_t rows,
                                                        const int32_t* __restrict__ counts,
-                                                       float* __restrict__ quot) {
+                                                       float* __restrict__ quot, WsHeader* hdr) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) {
+    hdr->status = 0;
+    hdr->detail = 0;
+  }
   const int64_t n = rows * F;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
@@ -72,6 +79,9 @@ __global__ void __launch_bounds__(kBwdThreads) k_pool_bwd_voronoi(
     const int p = threadIdx.x + r * kBwdThreads;
     t[r] = p < n ? token_id[t0 + p] : -1;
   }
+  // the quotient table and the reset status word (a no-op outside a
+  // programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (threadIdx.x < 2) s_ev[threadIdx.x] = event_of(offsets, 0, B - 1, threadIdx.x ? t0 + n - 1 : t0);
   __syncthreads();
   const int lo = s_ev[0], hi = max(s_ev[0], s_ev[1]);
@@ -281,15 +291,23 @@ cudaError_t launch_pool_bwd_voronoi(const float* grad_pooled, int F, const int64
   if (P == 0) return cudaSuccess;
   const int64_t rows = (int64_t)B * K;
   count_launch();
-  k_pool_bwd_quot<<<grid_for(rows * F, 256, 8), 256, 0, s>>>(grad_pooled, F, rows, counts, quot);
+  k_pool_bwd_quot<<<grid_for(rows * F, 256, 8), 256, 0, s>>>(grad_pooled, F, rows, counts, quot, hdr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const uint32_t fdiv = F > 1 ? (uint32_t)((((uint64_t)1 << 32) + F - 1) / F) : 0u;
   const int64_t blocks = (P + kBwdTile - 1) / kBwdTile;
   count_launch();
-  k_pool_bwd_voronoi<<<(unsigned)blocks, kBwdThreads, 0, s>>>(quot, F, fdiv, offsets, B, P, K, token_id,
-                                                              grad_feats, hdr);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_pool_bwd_voronoi, (const float*)quot, F, fdiv, offsets, B, P, K, token_id,
+                            grad_feats, hdr);
 }
 
 cudaError_t launch_pool_bwd_knn(const float* grad_pooled, int F, const int64_t* offsets, int B, int K, int k,

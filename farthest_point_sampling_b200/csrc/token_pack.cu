@@ -38,16 +38,22 @@ __device__ __forceinline__ int64_t tokens_of(const int64_t* __restrict__ offsets
 
 // tok_offsets[0] = 0, tok_offsets[b+1] = tok_offsets[b] + v_b, by one CTA in
 // tiles of kScanThreads * kScanPer events (kScanPer consecutive events per
-// thread, so the small-event batches take one tile).
+// thread, so the small-event batches take one tile).  Resets the call's
+// status word first (before the barrier that precedes every check).
 __global__ void __launch_bounds__(kScanThreads) k_pack_scan(const int64_t* __restrict__ offsets,
                                                             const int32_t* __restrict__ valid, int B, int K,
                                                             int64_t* __restrict__ tok_offsets, WsHeader* hdr) {
+  // the copy kernel, launched as a programmatic dependent, may start now: it
+  // reads its source rows and then waits for this kernel's offsets
+  asm volatile("griddepcontrol.launch_dependents;");
   __shared__ int64_t s_warp[kScanThreads / 32];
   __shared__ int64_t s_carry;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     s_carry = 0;
     tok_offsets[0] = 0;
+    hdr->status = 0;  // this call's status word (the copy kernel records nothing)
+    hdr->detail = 0;
   }
   __syncthreads();
   for (int64_t t0 = 0; t0 < B; t0 += (int64_t)kScanThreads * kScanPer) {
@@ -91,7 +97,10 @@ __global__ void __launch_bounds__(kScanThreads) k_pack_scan(const int64_t* __res
 
 // One block per event: dst rows tok_offsets[b] .. + v_b <- src[b, 0:v_b, :],
 // doc_id over the same rows <- b.  v_b comes from the inputs again, so only
-// the destination base waits on the scan's result.
+// the destination base waits on the scan's result: launched as the scan's
+// programmatic dependent, the block loads its first kPre elements per thread
+// before it waits for the scan (a no-op wait otherwise).
+constexpr int kPre = 8;
 __global__ void __launch_bounds__(kCopyThreads) k_pack_copy(const float* __restrict__ src, int D, int K,
                                                             const int64_t* __restrict__ offsets,
                                                             const int32_t* __restrict__ valid,
@@ -107,10 +116,22 @@ __global__ void __launch_bounds__(kCopyThreads) k_pack_copy(const float* __restr
     v = (int)(n < 0 ? 0 : (n < K ? n : K));
   }
   const float* s = src + (int64_t)b * K * D;
+  const int n = v * D;
+  float pre[kPre];
+#pragma unroll
+  for (int q = 0; q < kPre; ++q) {
+    const int e = threadIdx.x + q * kCopyThreads;
+    pre[q] = e < n ? s[e] : 0.f;
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t base = tok_offsets[b];
   float* d = dst + base * D;
-  const int n = v * D;
-  for (int e = threadIdx.x; e < n; e += kCopyThreads) d[e] = s[e];
+#pragma unroll
+  for (int q = 0; q < kPre; ++q) {
+    const int e = threadIdx.x + q * kCopyThreads;
+    if (e < n) d[e] = pre[q];
+  }
+  for (int e = threadIdx.x + kPre * kCopyThreads; e < n; e += kCopyThreads) d[e] = s[e];
   for (int j = threadIdx.x; j < v; j += kCopyThreads) doc_id[base + j] = b;
 }
 
@@ -140,8 +161,16 @@ cudaError_t launch_pack_tokens(const float* src, int D, const int64_t* offsets, 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || B == 0) return e;
   count_launch();
-  k_pack_copy<<<B, kCopyThreads, 0, s>>>(src, D, K, offsets, valid, tok_offsets, dst, doc_id);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)B);
+  cfg.blockDim = dim3(kCopyThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_pack_copy, src, D, K, offsets, valid, (const int64_t*)tok_offsets, dst, doc_id);
 }
 
 cudaError_t launch_unpack_tokens(const float* src, int D, int64_t n_tok, const int64_t* tok_offsets, int B, int K,

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kSumThreads) k_token_sums(const float4* __rest
                                                             int64_t chunk, float* __restrict__ wsum,
                                                             float* __restrict__ wcoords, float* __restrict__ wfeats,
                                                             double* __restrict__ partial, WsHeader* hdr) {
+  // the boundary kernel may be launched now; it waits for this one's sums
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ __align__(16) unsigned char s_raw[];
   const int V = 5 + F;
   const int KV = K * V;
@@ -212,6 +214,9 @@ __global__ void __launch_bounds__(256) k_token_finalize(const int64_t* __restric
   const int KV = K * V;
   const int R = cl - cf + 1;     // ranges the event spans
   const int lo = (int)((int64_t)KV * slice / nb), hi = (int)((int64_t)KV * (slice + 1) / nb);
+  // launched as the sums kernel's programmatic dependent: the search above
+  // ran while it finished; its partial sums are read from here on
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x;
   for (int v0 = lo; v0 < hi; v0 += 256) {
     const int nv = min(256, hi - v0);
@@ -295,9 +300,17 @@ cudaError_t launch_token_summaries(const float* coords, const float* feats, int 
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (G > 1) {
     count_launch();
-    k_token_finalize<<<(unsigned)(G - 1), 256, 0, s>>>(offsets, B, P, K, F, chunk, (int)G, partial, wsum, wcoords,
-                                                      wfeats);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(G - 1));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_token_finalize, offsets, B, P, K, F, chunk, (int)G, (const double*)partial, wsum,
+                           wcoords, wfeats);
   }
   return e;
 }
