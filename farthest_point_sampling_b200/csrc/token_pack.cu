@@ -17,7 +17,8 @@ namespace {
 
 constexpr int kScanThreads = 1024;
 constexpr int kScanPer = 4;  // consecutive events per scan thread
-constexpr int kCopyThreads = 128;
+constexpr int kCopyThreads = 128;   // unpack: one block per event
+constexpr int kPackThreads = 256;   // pack: one warp per event
 
 // Tokens of event b: valid[b] (clamped to 0..K, a value outside is recorded),
 // else min(N_b, K) from the point offsets.
@@ -95,44 +96,49 @@ __global__ void __launch_bounds__(kScanThreads) k_pack_scan(const int64_t* __res
   }
 }
 
-// One block per event: dst rows tok_offsets[b] .. + v_b <- src[b, 0:v_b, :],
-// doc_id over the same rows <- b.  v_b comes from the inputs again, so only
-// the destination base waits on the scan's result: launched as the scan's
-// programmatic dependent, the block loads its first kPre elements per thread
-// before it waits for the scan (a no-op wait otherwise).
-constexpr int kPre = 8;
-__global__ void __launch_bounds__(kCopyThreads) k_pack_copy(const float* __restrict__ src, int D, int K,
+// One warp per event (kPackThreads / 32 events per block): dst rows
+// tok_offsets[b] .. + v_b <- src[b, 0:v_b, :], doc_id over the same rows <-
+// b.  v_b comes from the inputs again, so only the destination base waits on
+// the scan's result: launched as the scan's programmatic dependent, each lane
+// loads its first kPre elements before it waits (a no-op wait otherwise),
+// and with a few blocks per SM every event's loads are in flight at once.
+constexpr int kPre = 24;
+__global__ void __launch_bounds__(kPackThreads) k_pack_copy(const float* __restrict__ src, int D, int K, int B,
                                                             const int64_t* __restrict__ offsets,
                                                             const int32_t* __restrict__ valid,
                                                             const int64_t* __restrict__ tok_offsets,
                                                             float* __restrict__ dst, int32_t* __restrict__ doc_id) {
-  const int b = blockIdx.x;
-  int v;
-  if (valid) {
-    const int32_t c = valid[b];
-    v = c < 0 ? 0 : (c > K ? K : c);
-  } else {
-    const int64_t n = offsets[b + 1] - offsets[b];
-    v = (int)(n < 0 ? 0 : (n < K ? n : K));
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (kPackThreads / 32) + (threadIdx.x >> 5);
+  int v = 0;
+  if (b < B) {
+    if (valid) {
+      const int32_t c = valid[b];
+      v = c < 0 ? 0 : (c > K ? K : c);
+    } else {
+      const int64_t n = offsets[b + 1] - offsets[b];
+      v = (int)(n < 0 ? 0 : (n < K ? n : K));
+    }
   }
   const float* s = src + (int64_t)b * K * D;
   const int n = v * D;
   float pre[kPre];
 #pragma unroll
   for (int q = 0; q < kPre; ++q) {
-    const int e = threadIdx.x + q * kCopyThreads;
+    const int e = lane + q * 32;
     pre[q] = e < n ? s[e] : 0.f;
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (b >= B) return;
   const int64_t base = tok_offsets[b];
   float* d = dst + base * D;
 #pragma unroll
   for (int q = 0; q < kPre; ++q) {
-    const int e = threadIdx.x + q * kCopyThreads;
+    const int e = lane + q * 32;
     if (e < n) d[e] = pre[q];
   }
-  for (int e = threadIdx.x + kPre * kCopyThreads; e < n; e += kCopyThreads) d[e] = s[e];
-  for (int j = threadIdx.x; j < v; j += kCopyThreads) doc_id[base + j] = b;
+  for (int e = lane + kPre * 32; e < n; e += 32) d[e] = s[e];
+  for (int j = lane; j < v; j += 32) doc_id[base + j] = b;
 }
 
 // One block per event: dst[b, 0:v_b, :] <- packed rows, dst[b, v_b:K, :] <- 0.
@@ -162,15 +168,16 @@ cudaError_t launch_pack_tokens(const float* src, int D, const int64_t* offsets, 
   if (e != cudaSuccess || B == 0) return e;
   count_launch();
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)B);
-  cfg.blockDim = dim3(kCopyThreads);
+  cfg.gridDim = dim3((unsigned)((B + kPackThreads / 32 - 1) / (kPackThreads / 32)));
+  cfg.blockDim = dim3(kPackThreads);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_pack_copy, src, D, K, offsets, valid, (const int64_t*)tok_offsets, dst, doc_id);
+  return cudaLaunchKernelEx(&cfg, k_pack_copy, src, D, K, B, offsets, valid, (const int64_t*)tok_offsets, dst,
+                            doc_id);
 }
 
 cudaError_t launch_unpack_tokens(const float* src, int D, int64_t n_tok, const int64_t* tok_offsets, int B, int K,
