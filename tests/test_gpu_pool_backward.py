@@ -56,6 +56,37 @@ def test_voronoi_backward_bitexact(F):
     np.testing.assert_array_equal(got.cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("F", [1, 6, 7])
+def test_voronoi_backward_unaligned_output(F):
+    """Through the C ABI into an output that starts 4 bytes past a 16-byte
+    boundary (the binding allocates aligned outputs): every element in place,
+    nothing written outside."""
+    import ctypes
+
+    from farthest_point_sampling_b200 import api
+    sizes = [300, 1025, 7, 0, 2048, 5]
+    K = 32
+    offsets, tok, counts = _random_labels(80 + F, sizes, K)
+    rng = np.random.default_rng(81 + F)
+    G = rng.normal(0, 3, (len(sizes), K, F)).astype(np.float32)
+    want = oracle.pool_voronoi_backward(G, offsets, tok, counts)
+    lib = fps.load_library()
+    P, B = len(tok), len(sizes)
+    buf = torch.full((P * F + 4,), 7.0, dtype=torch.float32, device="cuda")
+    out = buf[1:1 + P * F]
+    assert out.data_ptr() % 16 == 4
+    nb = lib.segment_pool_backward_workspace_bytes(P, B, K, F, 0)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+    g, c, o, t = _dev(G), _dev(counts), _dev(offsets), _dev(tok)
+    st = lib.segment_pool_backward(api._ptr(g), F, api._ptr(o), B, P, K, 0, api._ptr(t), None, 0, api._ptr(c),
+                                   ctypes.c_void_p(out.data_ptr()), api._ptr(ws), ws.numel(),
+                                   api._stream(torch.device("cuda")))
+    assert st == 0
+    fps.device_status(ws)
+    np.testing.assert_array_equal(out.cpu().numpy().reshape(P, F), want)
+    assert buf[0].item() == 7.0 and buf[-3:].cpu().tolist() == [7.0, 7.0, 7.0]
+
+
 def test_voronoi_backward_from_the_tokenizer_labels():
     b = workloads.make_workload("c1")
     ora = oracle.tokenize_batch(b)
