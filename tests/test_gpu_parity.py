@@ -102,6 +102,24 @@ def test_warp_events_with_few_distinct_points(force):
     compare(b, run_gpu(b, force_schedule=force))
 
 
+@pytest.mark.parametrize("name", ["c4", "mixed"])
+def test_warp_only_batches_with_a_size_hint(name):
+    """Host offsets give the library the largest event size; when every FPS
+    event fits the warp schedule, the warp kernel alone follows the binning,
+    as a programmatic dependent launch on the caller's stream.  The 4096-event
+    workload, and a batch with empty, tiny, N = K and N = K + 1 events between
+    the warp-size ones."""
+    if name == "c4":
+        b = workloads.make_workload("c4")
+    else:
+        rng = np.random.default_rng(41)
+        sizes = [int(n) for n in rng.integers(129, 449, 300)]
+        for i, n in enumerate([0, 1, 5, 127, 128, 129, 0, 448, 3]):
+            sizes.insert(i * 31, n)
+        b = workloads.random_batch(42, sizes, 128, dup_frac=0.02)
+    compare(b, run_gpu(b, host_offsets=True))
+
+
 @pytest.mark.parametrize("force", [0, 1, 2, 3, 4])
 def test_forced_schedules_agree(force):
     sizes = [129, 300, 448, 449, 2000, 2560, 2561, 12288, 12289, 40000, 98304, 98305]
