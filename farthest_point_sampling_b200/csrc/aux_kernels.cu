@@ -391,13 +391,28 @@ __global__ void __launch_bounds__(256) k_passthrough(Problem pb, Workspace ws, i
     const float* cf = reinterpret_cast<const float*>(pb.coords) + off * 4;
     float* outc = reinterpret_cast<float*>(pb.centroids) + (int64_t)b * K * 4;
     const int nc = n * 4;
-#pragma unroll 8
-    for (int e = lane; e < K * 4; e += 32) outc[e] = e < nc ? cf[e] : 0.f;
     const float* fe = pb.feats + off * F;
     float* outp = pb.pooled + (int64_t)b * K * F;
     const int nf = n * F;
-#pragma unroll 8
-    for (int e = lane; e < K * F; e += 32) outp[e] = e < nf ? fe[e] : 0.f;
+    // both rows' loads of a round are issued before its stores, so that an
+    // event costs about one memory round trip (K = 128, F <= 6: one round)
+    constexpr int R = 24;  // elements per lane and row per round
+    const int tc = K * 4, tp = K * F;
+    for (int r0 = 0; r0 < tc || r0 < tp; r0 += 32 * R) {
+      float vc[R], vp[R];
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        const int e = r0 + lane + 32 * u;
+        vc[u] = e < nc ? cf[e] : 0.f;
+        vp[u] = e < nf ? fe[e] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        const int e = r0 + lane + 32 * u;
+        if (e < tc) outc[e] = vc[u];
+        if (e < tp) outp[e] = vp[u];
+      }
+    }
     int32_t* ci = pb.centroid_idx + (int64_t)b * K;
     int32_t* co = pb.counts + (int64_t)b * K;
 #pragma unroll 4
