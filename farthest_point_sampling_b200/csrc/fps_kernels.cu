@@ -1250,7 +1250,12 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     cudaStream_t hs = ctx.helper[kHelpers - 1];
     if ((e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
     mark(kStagePassthrough, 0, hs);
-    if (pb.assign_mode == 0 && (e = launch_pool_clear(pb, ws, hs))) return e;  // Voronoi mode: the pool kernel may run
+    // Voronoi mode: the accumulators of a later pooling pass (the last Lloyd
+    // step, or the pool kernel) start cleared; none follows when every event
+    // is pooled in place
+    if (pb.assign_mode == 0 && (pb.lloyd_iters > 0 || pool_kernel_needed(pb)) &&
+        (e = launch_pool_clear(pb, ws, hs)))
+      return e;
     if ((e = launch_passthrough(pt, ws, hs))) return e;
     mark(kStagePassthrough, 1, hs);
     if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;

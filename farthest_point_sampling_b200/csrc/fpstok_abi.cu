@@ -164,8 +164,7 @@ static int run_tokenize(const Problem& pb0, const Workspace& ws, cudaStream_t s)
   } else {
     // with a size hint, a batch whose events all fit the schedules that pool
     // in place needs no pool kernel
-    const bool none_left = pb.max_event_hint > 0 && pb.max_event_hint <= kCtaCap && pb.force_schedule <= 1 &&
-                           (pb.fused_pool & 3) == 3;
+    const bool none_left = !pool_kernel_needed(pb);
     if (pb.lloyd_iters > 0 && lloyd_pools(pb)) {  // the last Lloyd iteration pooled; the replicas' means
       stage_mark(8, 0, s);
       if ((e = launch_pool_finalize(pb.offsets, pb.K, pb.F, pb.pooled, pb.counts, ws, s))) return from_cuda(e);

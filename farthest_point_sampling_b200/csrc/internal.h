@@ -119,6 +119,13 @@ size_t cta_region_bytes();
 // iteration also pools the token means (k_pool_finalize still follows for
 // the events pooled over several pieces).
 inline bool lloyd_pools(const Problem& pb) { return pb.assign_mode == 0 && pb.pooled && pb.feats; }
+// Voronoi mode without Lloyd: with a size hint that keeps every FPS event on
+// the warp and register-CTA schedules, which pool in place, no pool kernel
+// runs after the FPS kernels, and the pooling accumulators go unused.
+inline bool pool_kernel_needed(const Problem& pb) {
+  return !(pb.max_event_hint > 0 && pb.max_event_hint <= kCtaCap && pb.force_schedule <= 1 &&
+           (pb.fused_pool & 3) == 3);
+}
 cudaError_t launch_lloyd(const Problem& pb, const Workspace& ws, int32_t* labels, cudaStream_t s);
 cudaError_t launch_pool_finalize(const int64_t* offsets, int K, int F, float* pooled, int32_t* counts,
                                  const Workspace& ws, cudaStream_t s);
