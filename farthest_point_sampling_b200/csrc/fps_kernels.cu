@@ -594,6 +594,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) k_fps_cta(const float4* __rest
   constexpr int kMaxPairs = PR;
   constexpr int NT = kCtaThreads, NW = NT / 32;
   static_assert(2 * PR <= 32, "selected-slot mask is 32 bits");
+  // as the warp schedule: a programmatic dependent of the binning when it is
+  // the only FPS schedule (a no-op wait otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ DupPoint s_dup[];  // [2 * NT * PR] event copy for centroid look-up
   __shared__ int2 xk[2 * NW];           // (key, index) per warp, double-buffered
   __shared__ int s_item;
@@ -1177,8 +1180,8 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
   }
   // at most one event per SM: every warp-class event runs on the CTA schedule
   if (f < 0 && maybe_few) run[0] = false;
-  bool warp_only = run[0];
-  for (int q = 1; q < kNumSchedules; ++q) warp_only = warp_only && !run[q];
+  int n_run = 0;
+  for (int q = 0; q < kNumSchedules; ++q) n_run += run[q] ? 1 : 0;
 
 
   const PoolOut none = {nullptr, 0, nullptr, nullptr};
@@ -1191,12 +1194,12 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
   if ((e = cudaEventRecord(ctx.fork, s))) return e;
   for (int q = 0; q < kNumSchedules; ++q) {
     if (!run[q]) continue;
-    // When the warp schedule is the only FPS schedule, it follows the
-    // binning kernel on the caller's stream as a programmatic dependent
-    // launch (its CTAs are placed while the binning runs); otherwise every
-    // schedule runs on its own stream, so that no schedule's CTAs take the
-    // SMs ahead of another's longest events.
-    const bool chained = q == 0 && warp_only;
+    // When the warp or the register-CTA schedule is the only FPS schedule, it
+    // follows the binning kernel on the caller's stream as a programmatic
+    // dependent launch (its CTAs are placed while the binning runs);
+    // otherwise every schedule runs on its own stream, so that no schedule's
+    // CTAs take the SMs ahead of another's longest events.
+    const bool chained = n_run == 1 && q <= 1;
     cudaStream_t hs = chained ? s : ctx.helper[q];
     if (!chained && (e = cudaStreamWaitEvent(hs, ctx.fork, 0))) return e;
     mark(1 + q, 0, hs);
@@ -1219,13 +1222,23 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
                                po_warp, pb.w, pb.scaled);
         break;
       }
-      case 1:
+      case 1: {
         count_launch();
-        k_fps_cta<kCtaPairs><<<di.sm_count, kCtaThreads, kCtaSmem, hs>>>(
-            pb.coords, pb.offsets, pb.start_local, ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id,
-            pb.centroids, po_cta, pb.w, pb.scaled);
-        e = cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(di.sm_count);
+        cfg.blockDim = dim3(kCtaThreads);
+        cfg.dynamicSmemBytes = kCtaSmem;
+        cfg.stream = hs;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = chained ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, k_fps_cta<kCtaPairs>, pb.coords, pb.offsets, pb.start_local,
+                               (const int*)ws.list_cta, ws.hdr, pb.K, pb.centroid_idx, pb.token_id, pb.centroids,
+                               po_cta, pb.w, pb.scaled);
         break;
+      }
       case 2:
         e = launch_block<1>(pb, ws, kListCtaSmem, ws.list_cta_smem, di.sm_count, hs);
         break;
@@ -1261,7 +1274,7 @@ cudaError_t launch_fps(const Problem& pb, const Problem& pt, const Workspace& ws
     if ((e = cudaEventRecord(ctx.join[kHelpers - 1], hs))) return e;
   }
   for (int q = 0; q < kNumSchedules; ++q)
-    if (run[q] && !(q == 0 && warp_only) && (e = cudaStreamWaitEvent(s, ctx.join[q], 0))) return e;
+    if (run[q] && !(n_run == 1 && q <= 1) && (e = cudaStreamWaitEvent(s, ctx.join[q], 0))) return e;
   return cudaStreamWaitEvent(s, ctx.join[kHelpers - 1], 0);
 }
 
