@@ -83,21 +83,11 @@ __device__ __forceinline__ void prefetch_rows_l2(const float* lo, size_t bytes, 
 }
 
 // Layout of the warp schedule's per-warp shared memory: the event's points
-// (DupPoint: every coordinate twice, so two 128-bit loads give the packed
-// centroid), then the list of chosen local indices (the step's centroid is
-// recorded by one lane; positions and global indices are written once at the
-// end).  The points region is reused by the fused pooling afterwards.
-#ifndef FPS_WARP_DUP
-#define FPS_WARP_DUP 0
-#endif
-#ifndef FPS_RELAX_SEL
-#define FPS_RELAX_SEL 0
-#endif
-#if FPS_WARP_DUP
-typedef DupPoint WarpPt;
-#else
+// (float4, the caller's units), then the list of chosen local indices (the
+// step's centroid is recorded by one lane; positions and global indices are
+// written once at the end).  The points region is reused by the fused
+// pooling afterwards.
 typedef float4 WarpPt;
-#endif
 constexpr int kWarpPtBytes = (int)sizeof(WarpPt);
 constexpr int kWarpListInts = FPS_MAX_K_DEV;  // chosen local indices, one per step
 // Shared memory of one warp: the event copy and the list, then room for the
@@ -106,42 +96,16 @@ constexpr int kWarpRegionBytes = 15360;
 static_assert(64 * kWarpPairs * kWarpPtBytes + kWarpListInts * 4 <= kWarpRegionBytes, "event copy and list fit");
 static_assert(8 * FPS_MAX_K_DEV + 4 * kWarpCap <= kWarpRegionBytes, "one staged feature per pass fits");
 
-__device__ __forceinline__ WarpPt warp_pt(float4 a) {
-#if FPS_WARP_DUP
-  return dup_point(a);
-#else
-  return a;
-#endif
-}
-__device__ __forceinline__ float4 warp_pt_pos(const WarpPt& p) {
-#if FPS_WARP_DUP
-  return dup_to_float4(p);
-#else
-  return p;
-#endif
-}
+// The packed centroid of a stored point (scaled per step when SCALED).
 template <bool SCALED>
 __device__ __forceinline__ Cent2 warp_pt_cent(const WarpPt& p, float4 w) {
-  if (SCALED) return cent2(scale4(warp_pt_pos(p), w));
-#if FPS_WARP_DUP
-  return cent2_dup(p);
-#else
-  return cent2(p);
-#endif
+  return cent2(SCALED ? scale4(p, w) : p);
 }
 
 // Running-min / label update of the two points of one packed pair.
 __device__ __forceinline__ void relax2(uint64_t d, float& d0, float& d1, int& l0, int& l1, int s) {
-#if FPS_RELAX_SEL
-  const bool a = lo2(d) < d0, b = hi2(d) < d1;
-  l0 = a ? s : l0;
-  d0 = a ? lo2(d) : d0;
-  l1 = b ? s : l1;
-  d1 = b ? hi2(d) : d1;
-#else
   relax(lo2(d), d0, l0, s);
   relax(hi2(d), d1, l1, s);
-#endif
 }
 
 // One FPS event on one warp, NP point pairs per lane (lane l owns points
@@ -166,8 +130,8 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (i0 < n) a = ldg4(pts + i0);
     if (i1 < n) b = ldg4(pts + i1);
-    if (i0 < n) s_pts[i0] = warp_pt(a);  // caller's units: centroid outputs (scaled per step when needed)
-    if (i1 < n) s_pts[i1] = warp_pt(b);
+    if (i0 < n) s_pts[i0] = a;  // caller's units: centroid outputs (scaled per step when needed)
+    if (i1 < n) s_pts[i1] = b;
     if (SCALED) {
       a = scale4(a, w);
       b = scale4(b, w);
@@ -258,7 +222,7 @@ __device__ __noinline__ void warp_event(const float4* __restrict__ pts, int n, i
   for (int j = lane; j < K; j += 32) {  // the event's centroids, once
     const int cj = s_c[j];
     cidx[j] = (int32_t)(off + cj);
-    cpos[j] = warp_pt_pos(s_pts[cj]);
+    cpos[j] = s_pts[cj];
   }
   if (tok) {
 #pragma unroll
